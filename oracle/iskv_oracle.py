@@ -1,0 +1,348 @@
+"""Float64 restatement of iS-KV's per-head state machine.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).  Nothing here is blocked,
+fused or reordered beyond the method's own steps; numpy's LAPACK SVD and QR
+serve as library primitives for the two factorizations the method names.
+
+Notation follows the iS-KV explainer ("iS-KV -- Basis-synchronized online
+low-rank KV compression -- What does it mean?"):
+  d  head dimension, r rank, b = 64 block rows, W exact recent window,
+  B  d x r orthonormal basis, S r singular values, C n_c x r coefficients,
+  T  tokens appended, n_c tokens folded into (B, S, C).  The exact window is
+  rows [n_c, T).
+
+Readings of points the pages leave open (each one is stated where used):
+  * a block is folded once T - n_c >= W + b (Jargon: Block-incremental SVD;
+    body paragraph on folding 64 tokens as they leave the recent window);
+  * initial state B = I_d[:, :r], S = 0, n_c = 0;
+  * the residual is re-orthogonalized against B once more (twice is enough);
+  * the complement basis Q comes from a Householder QR of [B | E^T] with
+    k = min(b, d - r) columns ("rule Q"); it equals the QR of E^T when E has
+    full rank and k = b, and keeps [B, Q] orthonormal when r + b > d;
+  * truncation keeps the r largest singular values (fixed rank);
+  * RoPE is the rotate-half form on pairs (i, i + d/2) with
+    inv_freq_i = theta^(-2i/d) at absolute 0-based positions; keys are stored
+    pre-RoPE and rotated when attention reads them (Jargon: Pre-RoPE keys);
+  * bf16 coefficient storage is emulated by rounding to the nearest bf16
+    value (ties to even) wherever the stored coefficients are written.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+__all__ = [
+    "bf16_round",
+    "ready_blocks",
+    "rope_inv_freq",
+    "rope_rotate",
+    "fold_block",
+    "FoldResult",
+    "HeadFactor",
+    "dense_decode",
+    "full_kv_bytes",
+    "persistent_kv_bytes",
+]
+
+# ----------------------------------------------------------------------------
+# Storage rounding
+# ----------------------------------------------------------------------------
+
+_BF16_MAX = float.fromhex("0x1.fep127")
+
+
+def bf16_round(x):
+    """Round float64 values to the nearest bfloat16 value, ties to even.
+
+    bfloat16 keeps 8 significant bits and float32's exponent range.  For
+    |x| = m * 2^e with 0.5 <= m < 1 the quantum is 2^(e - 8) (bf16 subnormals:
+    2^-133).  Scaling by a power of two is exact, and ``np.round`` rounds half
+    to even, so the result is exact.  Pinned in the tests against torch's own
+    float32 -> bfloat16 conversion and against hand-built tie cases.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.array(x, copy=True)
+    fin = np.isfinite(x) & (x != 0)
+    if np.any(fin):
+        xv = x[fin]
+        _, e = np.frexp(xv)
+        e = np.maximum(e, -125)
+        q_exp = e - 8
+        scaled = np.ldexp(xv, -q_exp)
+        rv = np.ldexp(np.round(scaled), q_exp)
+        rv = np.where(np.abs(rv) > _BF16_MAX, np.copysign(np.inf, rv), rv)
+        out[fin] = rv
+    return out
+
+
+def _store(x, coef_round):
+    if coef_round is None:
+        return np.asarray(x, dtype=np.float64)
+    if coef_round == "bf16":
+        return bf16_round(x)
+    if coef_round == "f32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    raise ValueError(f"unknown coefficient storage {coef_round!r}")
+
+
+# ----------------------------------------------------------------------------
+# Window and block bookkeeping
+# ----------------------------------------------------------------------------
+
+
+def ready_blocks(T: int, n_c: int, W: int, b: int = 64) -> int:
+    """Number of whole b-row blocks that have left the exact window.
+
+    The newest W tokens stay exact; the rows [n_c, T - W) are old enough to be
+    folded, in whole blocks of b (the explainer's body: every time 64 tokens
+    leave the recent window they are folded in as one block).  Pinned by brute
+    force over all small (T, n_c, W) in the tests.
+    """
+    if T < 0 or n_c < 0 or W < 0 or b <= 0 or n_c > T:
+        raise ValueError("invalid counters")
+    excess = T - n_c - W
+    return excess // b if excess >= 0 else 0
+
+
+# ----------------------------------------------------------------------------
+# RoPE (Jargon: Pre-RoPE keys)
+# ----------------------------------------------------------------------------
+
+
+def rope_inv_freq(d: int, theta: float) -> np.ndarray:
+    """inv_freq_i = theta^(-2i/d) for the d/2 rotation pairs."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(theta), -2.0 * i / d)
+
+
+def rope_rotate(x, pos, theta: float) -> np.ndarray:
+    """Rotate rows of ``x`` (n x d) by RoPE at absolute positions ``pos``.
+
+    Pair i is (x[i], x[i + d/2]) and turns by the angle pos * inv_freq_i.
+    Pinned in the tests: norm preservation, R(a)^T R(b) = R(b - a) (scores
+    depend only on relative position), identity at position 0 and a
+    hand-computed d = 4 case.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    n, d = x.shape
+    h = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * rope_inv_freq(d, theta)[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[:, :h], x[:, h:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=1)
+
+
+# ----------------------------------------------------------------------------
+# One block fold: steps (a)-(d) of the block-incremental SVD
+# ----------------------------------------------------------------------------
+
+
+@dataclass
+class FoldResult:
+    B_new: np.ndarray   # d x r, new orthonormal basis  [B, Q] W_r
+    S_new: np.ndarray   # r, leading singular values of the core
+    W_top: np.ndarray   # r x r, W_r[0:r, :], the resync map for old rows
+    C_new: np.ndarray   # b x r, coefficients of the folded block
+    W_r: np.ndarray     # (r+k) x r
+    sigma: np.ndarray   # all r+k singular values of the core, descending
+    P: np.ndarray       # b x r projection of the block
+    E: np.ndarray       # b x d residual
+    Q: np.ndarray       # d x k complement basis
+    R_E: np.ndarray     # k x b, Q^T E^T
+    core: np.ndarray    # (r+b) x (r+k)
+
+
+def fold_block(B, S, X) -> FoldResult:
+    """Fold one block X (b x d) into the rank-r factorization (B, S).
+
+    Brand's block-incremental SVD as the iS-KV explainer applies it (Jargon:
+    Block-incremental SVD; body paragraph on the joint update of basis and
+    coefficients, solved on a small core whose size does not depend on the
+    history length):
+      (a) P = X B
+      (b) E = X - P B^T (re-orthogonalized once more), Q and R_E from rule Q
+      (c) core = [[diag S, 0], [P, R_E^T]], SVD core = U Sigma W^T, keep r
+      (d) B' = [B, Q] W_r, S' = sigma_1..r, new rows [P, R_E^T] W_r,
+          and W_top = W_r[0:r, :] for step (e), done by the caller.
+    Pinned in the tests: exactness when the history has rank <= r against the
+    covariance-route batch SVD, losslessness at r = d, orthonormality of B',
+    the reconstruction identity X = P B^T + R_E^T Q^T and the energy balance of
+    the truncation.
+    """
+    B = np.asarray(B, dtype=np.float64)
+    S = np.asarray(S, dtype=np.float64)
+    X = np.asarray(X, dtype=np.float64)
+    d, r = B.shape
+    b = X.shape[0]
+    k = min(b, d - r)
+
+    # (a) project the block onto the current basis
+    P = X @ B
+    # (b) residual, with one re-orthogonalization pass against B
+    E = X - P @ B.T
+    P2 = E @ B
+    E = E - P2 @ B.T
+    P = P + P2
+    # rule Q: Householder QR of [B | E^T]; columns r..r+k-1 of the full Q
+    M = np.concatenate([B, E.T], axis=1)
+    Qf, _ = np.linalg.qr(M, mode="complete")
+    Q = Qf[:, r:r + k]
+    R_E = Q.T @ E.T
+    # (c) the small core and its SVD, truncated to rank r
+    core = np.zeros((r + b, r + k))
+    core[:r, :r] = np.diag(S)
+    core[r:, :r] = P
+    core[r:, r:] = R_E.T
+    _, sigma, Wt = np.linalg.svd(core, full_matrices=True)
+    Wfull = Wt.T
+    W_r = Wfull[:, :r]
+    # (d) new basis, new singular values, coefficients of the new rows
+    B_new = np.concatenate([B, Q], axis=1) @ W_r
+    C_new = core[r:, :] @ W_r
+    return FoldResult(B_new=B_new, S_new=sigma[:r].copy(), W_top=W_r[:r, :].copy(),
+                      C_new=C_new, W_r=W_r, sigma=sigma, P=P, E=E, Q=Q, R_E=R_E,
+                      core=core)
+
+
+# ----------------------------------------------------------------------------
+# Per head-instance state: exact rows + (B, S, C)
+# ----------------------------------------------------------------------------
+
+
+class HeadFactor:
+    """One (sequence, layer, KV head, K-or-V) factor with its exact window.
+
+    ``coef_round`` selects the storage format of C: None (float64, exact
+    oracle), "f32" or "bf16" (emulated at every write: new rows at a fold and
+    every resync).  ``sync=False`` is the no-synchronization ablation: old
+    rows keep the coefficients of the basis they were written in.
+
+    ``fold(defer=True)`` postpones step (e) for the rows already stored; the
+    postponed rewrites are applied in order by ``sync()``, with one storage
+    rounding at the end.  With nothing read in between this equals the
+    per-fold rewrite in exact arithmetic (each rewrite is a right
+    multiplication of the rows that existed before that fold).
+    """
+
+    def __init__(self, d: int, r: int, W: int, b: int = 64, coef_round=None,
+                 sync: bool = True):
+        if not (0 < r <= d) or b <= 0 or W < 0:
+            raise ValueError("invalid factor shape")
+        self.d, self.r, self.W, self.b = d, r, W, b
+        self.coef_round = coef_round
+        self.sync_enabled = sync
+        self.B = np.eye(d)[:, :r].copy()
+        self.S = np.zeros(r)
+        self.C = np.zeros((0, r))
+        self.rows = np.zeros((0, d))
+        self.n_c = 0
+        self.pending = []           # [(rows_before_fold, W_top)]
+        self.history = []           # FoldResult per fold (for drift studies)
+
+    @property
+    def T(self) -> int:
+        return self.rows.shape[0]
+
+    def append(self, rows) -> int:
+        rows = np.asarray(rows, dtype=np.float64).reshape(-1, self.d)
+        self.rows = np.concatenate([self.rows, rows], axis=0)
+        return self.ready()
+
+    def ready(self) -> int:
+        return ready_blocks(self.T, self.n_c, self.W, self.b)
+
+    def fold(self, defer: bool = False, keep_history: bool = False) -> FoldResult:
+        if self.ready() < 1:
+            raise RuntimeError("no ready block")
+        X = self.rows[self.n_c:self.n_c + self.b]
+        res = fold_block(self.B, self.S, X)
+        # (e) basis synchronization of the rows stored so far
+        if self.sync_enabled and self.n_c > 0:
+            if defer:
+                self.pending.append((self.n_c, res.W_top))
+            else:
+                self.C[:self.n_c] = _store(self.C[:self.n_c] @ res.W_top, self.coef_round)
+        self.C = np.concatenate([self.C, _store(res.C_new, self.coef_round)], axis=0)
+        self.B, self.S = res.B_new, res.S_new
+        self.n_c += self.b
+        if keep_history:
+            self.history.append(res)
+        return res
+
+    def sync(self) -> None:
+        """Apply postponed rewrites in fold order, then round once."""
+        if not self.pending:
+            return
+        C = self.C.copy()
+        touched = 0
+        for n_rows, W_top in self.pending:
+            C[:n_rows] = C[:n_rows] @ W_top
+            touched = max(touched, n_rows)
+        C[:touched] = _store(C[:touched], self.coef_round)
+        self.C = C
+        self.pending = []
+
+    def reconstruct(self) -> np.ndarray:
+        """Pre-RoPE reconstruction C B^T of the folded rows (n_c x d)."""
+        if self.pending:
+            raise RuntimeError("postponed rewrites pending; call sync()")
+        return self.C @ self.B.T
+
+    def exact(self) -> np.ndarray:
+        return self.rows[self.n_c:]
+
+    def full(self) -> np.ndarray:
+        """All T rows as attention sees them: reconstructed, then exact."""
+        return np.concatenate([self.reconstruct(), self.exact()], axis=0)
+
+
+# ----------------------------------------------------------------------------
+# Decode attention over the mixed cache
+# ----------------------------------------------------------------------------
+
+
+def dense_decode(q, K_pre, V, theta: float, use_rope: bool = True) -> np.ndarray:
+    """Softmax attention of query heads ``q`` (g x d) over T rows.
+
+    ``K_pre`` holds the keys before RoPE (reconstructed rows, then the exact
+    window); they are rotated at absolute positions 0..T-1 here, the query is
+    taken as already rotated (it belongs to position T-1).  Scale 1/sqrt(d),
+    no mask.  This is the plain definition; the method's value-side shortcut
+    out = (p^T C_V) B_V^T + p_win^T V_win is the same sum regrouped.  Pinned by
+    brute-force loops in the tests.
+    """
+    q = np.atleast_2d(np.asarray(q, dtype=np.float64))
+    K_pre = np.asarray(K_pre, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    T, d = K_pre.shape
+    Kr = rope_rotate(K_pre, np.arange(T), theta) if use_rope else K_pre
+    s = (q @ Kr.T) / np.sqrt(d)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ V
+
+
+# ----------------------------------------------------------------------------
+# Memory accounting (Jargon: Persistent-KV compression)
+# ----------------------------------------------------------------------------
+
+
+def full_kv_bytes(tokens: int, layers: int, kv_heads: int, head_dim: int,
+                  elem_bytes: int) -> int:
+    """Bytes of an uncompressed K and V cache.  Pinned by the A40 memory test
+    figure of the explainer (full cache at a 32K input + 1,024 steps)."""
+    return tokens * layers * kv_heads * head_dim * 2 * elem_bytes
+
+
+def persistent_kv_bytes(n_c: int, n_w: int, d: int, r_k: int, r_v: int,
+                        coef_bytes: int, kv_bytes: int, basis_bytes: int = 4) -> int:
+    """Bytes kept between decode steps for one (sequence, layer, KV head):
+    both factors (C, B, S) plus both exact windows.  Excludes temporary
+    buffers, as the explainer's definition does.  Parity unpinned: the pages
+    print no kept-byte figure this formula can be checked against."""
+    factors = n_c * (r_k + r_v) * coef_bytes + (d + 1) * (r_k + r_v) * basis_bytes
+    window = 2 * n_w * d * kv_bytes
+    return factors + window

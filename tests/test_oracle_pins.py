@@ -1,0 +1,418 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test checks the oracle against what the pages or the mathematics fix:
+brute force on tiny inputs, closed forms, invariants, the covariance route to
+a batch SVD (KV-CoRE summary, section 2 Methodology), the exactness of Brand's
+update on histories of rank <= r, losslessness at r = d, and the one number
+the pages print that is pure arithmetic (the A40 full-cache size).  The
+mutation tests at the end plant mistakes in a copy of the oracle's fold and
+check that the pins catch them.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import iskv_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _low_rank_rows(n, d, rank, seed, noise=0.0):
+    g = _rng(seed)
+    G, _ = np.linalg.qr(g.standard_normal((d, rank)))
+    Z = g.standard_normal((n, rank)) * (2.0 ** -np.arange(rank) * 4 + 1)
+    return Z @ G.T + noise * g.standard_normal((n, d))
+
+
+def _cov_projector(H, m):
+    """Projector onto the top-m right singular subspace of H via the
+    eigenvectors of H^T H (the covariance route of the KV-CoRE summary)."""
+    w, V = np.linalg.eigh(H.T @ H)
+    idx = np.argsort(w)[::-1][:m]
+    Vm = V[:, idx]
+    return Vm @ Vm.T
+
+
+def _fold_all(f):
+    while f.ready() > 0:
+        f.fold()
+
+
+# ----------------------------------------------------------------------------
+# storage rounding
+# ----------------------------------------------------------------------------
+
+
+def test_bf16_round_matches_torch_on_float32_inputs():
+    x = _rng(0).standard_normal(200000).astype(np.float32) * 37.0
+    x = np.concatenate([x, np.float32([0.0, -0.0, 1e-30, -3e-39, 3.3e38])])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_round(x.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_bf16_round_ties_and_direct_rounding():
+    one = 1.0
+    # exact tie between 1 and 1 + 2^-7: to even (1)
+    assert O.bf16_round(one + 2.0 ** -8) == 1.0
+    # tie between 1 + 2^-7 (odd) and 1 + 2^-6 (even): to 1 + 2^-6
+    assert O.bf16_round(one + 3 * 2.0 ** -8) == one + 2.0 ** -6
+    # just above a tie: rounds up.  A detour through float32 would first make
+    # it an exact tie and then round down; the oracle rounds float64 directly.
+    assert O.bf16_round(one + 2.0 ** -8 + 2.0 ** -40) == one + 2.0 ** -7
+    assert O.bf16_round(-(one + 2.0 ** -8 + 2.0 ** -40)) == -(one + 2.0 ** -7)
+    # carry into the exponent
+    assert O.bf16_round(2.0 - 2.0 ** -9) == 2.0
+    assert np.isinf(O.bf16_round(3.5e38))
+
+
+# ----------------------------------------------------------------------------
+# bookkeeping
+# ----------------------------------------------------------------------------
+
+
+def test_ready_blocks_brute_force():
+    for W in (0, 64, 128, 192):
+        for T in range(0, 400):
+            for n_c in range(0, T + 1, 64):
+                # count by simulating the window: pop blocks while enough
+                # rows are older than the newest W
+                n, cnt = n_c, 0
+                while True:
+                    old = [j for j in range(n, T) if j < T - W]
+                    if len(old) >= 64:
+                        n += 64
+                        cnt += 1
+                    else:
+                        break
+                assert O.ready_blocks(T, n_c, W) == cnt, (T, n_c, W)
+
+
+def test_headfactor_counters_and_window_bounds():
+    f = O.HeadFactor(d=16, r=4, W=64)
+    g = _rng(1)
+    for step in range(700):
+        f.append(g.standard_normal((1, 16)))
+        _fold_all(f)
+        n_w = f.T - f.n_c
+        assert f.n_c % 64 == 0
+        assert (f.T < 64 + 64 and f.n_c == 0) or 64 <= n_w <= 127
+        assert 0 <= n_w < 64 + 64
+    assert f.T == 700 and f.n_c == 576
+
+
+# ----------------------------------------------------------------------------
+# RoPE
+# ----------------------------------------------------------------------------
+
+
+def test_rope_hand_computed_d4():
+    # d = 4, theta = 10000: inv_freq = [1, 0.01]; pairs (0, 2) and (1, 3)
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    got = O.rope_rotate(x, [1], 10000.0)[0]
+    c0, s0, c1, s1 = math.cos(1.0), math.sin(1.0), math.cos(0.01), math.sin(0.01)
+    want = [1 * c0 - 3 * s0, 2 * c1 - 4 * s1, 1 * s0 + 3 * c0, 2 * s1 + 4 * c1]
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-15)
+
+
+def test_rope_invariants():
+    g = _rng(2)
+    d, theta = 128, 1e6
+    x = g.standard_normal((5, d))
+    pos = np.array([0, 1, 1000, 65535, 262143])
+    y = O.rope_rotate(x, pos, theta)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    np.testing.assert_array_equal(O.rope_rotate(x[:1], [0], theta), x[:1])
+    q, k = g.standard_normal((1, d)), g.standard_normal((1, d))
+    for a, b in [(3, 10), (1000, 4000), (200000, 262000)]:
+        lhs = (O.rope_rotate(q, [a], theta) @ O.rope_rotate(k, [b], theta).T).item()
+        rhs = (q @ O.rope_rotate(k, [b - a], theta).T).item()
+        assert abs(lhs - rhs) < 1e-9 * (1 + abs(rhs))
+
+
+# ----------------------------------------------------------------------------
+# one fold
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("r", [16, 64, 96, 128])
+def test_fold_identities(r):
+    d = 128
+    g = _rng(3 + r)
+    B, _ = np.linalg.qr(g.standard_normal((d, r)))
+    S = np.sort(g.uniform(1, 10, r))[::-1]
+    X = g.standard_normal((64, d))
+    res = O.fold_block(B, S, X)
+    k = min(64, d - r)
+    assert res.Q.shape == (d, k) and res.R_E.shape == (k, 64)
+    # [B, Q] orthonormal
+    BQ = np.concatenate([B, res.Q], axis=1)
+    np.testing.assert_allclose(BQ.T @ BQ, np.eye(r + k), atol=1e-13)
+    # the block is represented exactly: X = P B^T + R_E^T Q^T
+    np.testing.assert_allclose(res.P @ B.T + res.R_E.T @ res.Q.T, X, atol=1e-12)
+    # new basis orthonormal, singular values sorted
+    np.testing.assert_allclose(res.B_new.T @ res.B_new, np.eye(r), atol=1e-12)
+    assert np.all(np.diff(res.sigma) <= 1e-12)
+    # energy balance: ||core||^2 = ||S||^2 + ||X||^2, discarded = tail sigma^2
+    e_core = np.sum(res.core ** 2)
+    np.testing.assert_allclose(e_core, np.sum(S ** 2) + np.sum(X ** 2), rtol=1e-12)
+    kept = np.sum(res.S_new ** 2)
+    np.testing.assert_allclose(e_core - kept, np.sum(res.sigma[r:] ** 2), rtol=1e-9, atol=1e-9)
+
+
+def test_one_fold_is_eckart_young_of_exact_history():
+    """History of rank <= r held exactly: one fold must give the best rank-r
+    approximation of [history; block] (batch SVD via the covariance route)."""
+    d, r = 128, 24
+    g = _rng(7)
+    H = _low_rank_rows(200, d, 10, 7)            # rank 10 <= r history
+    U, s, Vt = np.linalg.svd(H, full_matrices=False)
+    B = Vt[:r].T
+    S = s[:r]
+    C = U[:, :r] * S                              # C B^T = H exactly
+    X = g.standard_normal((64, d))
+    res = O.fold_block(B, S, X)
+    C_all = np.concatenate([C @ res.W_top, res.C_new], axis=0)
+    A = np.concatenate([H, X], axis=0)
+    P = _cov_projector(A, r)
+    np.testing.assert_allclose(res.B_new @ res.B_new.T, P, atol=1e-9)
+    np.testing.assert_allclose(C_all @ res.B_new.T, A @ P, atol=1e-9)
+
+
+def test_sync_closed_form():
+    """Old rows after (e): C' B'^T = (C B^T) B' B'^T, for any history."""
+    d, r = 128, 32
+    g = _rng(9)
+    f = O.HeadFactor(d, r, W=64)
+    f.append(_low_rank_rows(64 * 6, d, 48, 9, noise=0.05))
+    _fold_all(f)
+    before = f.reconstruct()
+    n_old = f.n_c
+    f.append(g.standard_normal((64, d)))
+    f.fold()
+    after = (f.C @ f.B.T)[:n_old]
+    np.testing.assert_allclose(after, before @ f.B @ f.B.T, atol=1e-11)
+
+
+# ----------------------------------------------------------------------------
+# whole-history pins
+# ----------------------------------------------------------------------------
+
+
+def test_exact_rank_history_is_reproduced():
+    """Rank 8 <= r = 16, no noise: zero residual and the batch projector."""
+    d, r = 128, 16
+    rows = _low_rank_rows(1024, d, 8, 11)
+    f = O.HeadFactor(d, r, W=128)
+    f.append(rows)
+    _fold_all(f)
+    assert f.n_c == 896
+    H = rows[:f.n_c]
+    err = np.abs(f.reconstruct() - H).max() / np.abs(H).max()
+    assert err < 1e-12
+    np.testing.assert_allclose(f.B[:, :8] @ f.B[:, :8].T, _cov_projector(H, 8), atol=1e-10)
+    np.testing.assert_allclose(f.B.T @ f.B, np.eye(r), atol=1e-10)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_full_rank_is_lossless(seed):
+    d = 128
+    rows = _rng(seed).standard_normal((64 * 7 + 30, d))
+    f = O.HeadFactor(d, d, W=64)
+    f.append(rows)
+    _fold_all(f)
+    np.testing.assert_allclose(f.reconstruct(), rows[:f.n_c], atol=1e-11)
+    q = _rng(seed + 100).standard_normal((4, d))
+    got = O.dense_decode(q, f.full(), rows, theta=1e6)
+    want = O.dense_decode(q, rows, rows, theta=1e6)
+    np.testing.assert_allclose(got, want, atol=1e-11)
+
+
+@pytest.mark.parametrize("r", [16, 96, 128])
+def test_orthonormal_after_many_folds_and_degenerate_blocks(r):
+    d = 128
+    g = _rng(r)
+    f = O.HeadFactor(d, r, W=0)
+    blocks = [np.zeros((64, d)), np.tile(g.standard_normal((1, d)), (64, 1)),
+              _low_rank_rows(64, d, 3, 1)]
+    blocks += [g.standard_normal((64, d)) * 10 ** g.uniform(-3, 3) for _ in range(20)]
+    blocks += [np.zeros((64, d))]
+    for Xb in blocks:
+        f.append(Xb)
+        f.fold()
+        assert np.linalg.norm(f.B.T @ f.B - np.eye(r)) < 1e-10
+
+
+def test_deferred_sync_equals_per_fold_sync():
+    d, r = 128, 32
+    rows = _low_rank_rows(64 * 12, d, 48, 13, noise=0.05)
+    a = O.HeadFactor(d, r, W=0)
+    b = O.HeadFactor(d, r, W=0)
+    a.append(rows)
+    b.append(rows)
+    while a.ready():
+        a.fold()
+        b.fold(defer=True)
+        if len(b.pending) == 5:
+            b.sync()
+    b.sync()
+    np.testing.assert_allclose(b.C, a.C, atol=1e-12)
+
+
+def test_no_sync_ablation_drifts():
+    """The explainer reports far larger drift when only the basis is updated;
+    the ablation must show it on a drifting low-rank stream."""
+    d, r = 128, 16
+    rows = _low_rank_rows(64 * 12, d, 12, 100, noise=0.01)
+    s = O.HeadFactor(d, r, W=0)
+    n = O.HeadFactor(d, r, W=0, sync=False)
+    s.append(rows)
+    n.append(rows)
+    _fold_all(s)
+    _fold_all(n)
+    H = rows[:s.n_c]
+    e_sync = np.linalg.norm(s.reconstruct() - H) / np.linalg.norm(H)
+    e_none = np.linalg.norm(n.C @ n.B.T - H) / np.linalg.norm(H)
+    assert e_sync < 0.05
+    assert e_none > 20 * e_sync
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+
+
+def _brute_decode(q, K, V, theta, use_rope):
+    """Pure-Python loops: rotate, score, softmax, weighted sum."""
+    T, d = len(K), len(K[0])
+    h = d // 2
+    out = []
+    for qh in q:
+        scores = []
+        for j in range(T):
+            kr = list(K[j])
+            if use_rope:
+                for i in range(h):
+                    a = j * theta ** (-2.0 * i / d)
+                    kr[i] = K[j][i] * math.cos(a) - K[j][i + h] * math.sin(a)
+                    kr[i + h] = K[j][i] * math.sin(a) + K[j][i + h] * math.cos(a)
+            scores.append(sum(qh[i] * kr[i] for i in range(d)) / math.sqrt(d))
+        m = max(scores)
+        w = [math.exp(s - m) for s in scores]
+        z = sum(w)
+        out.append([sum(w[j] * V[j][i] for j in range(T)) / z for i in range(d)])
+    return np.array(out)
+
+
+@pytest.mark.parametrize("use_rope", [False, True])
+def test_dense_decode_brute_force(use_rope):
+    g = _rng(21)
+    d, T = 8, 37
+    q = g.standard_normal((3, d)) * 2
+    K = g.standard_normal((T, d))
+    V = g.standard_normal((T, d))
+    got = O.dense_decode(q, K, V, theta=10000.0, use_rope=use_rope)
+    want = _brute_decode(q.tolist(), K.tolist(), V.tolist(), 10000.0, use_rope)
+    np.testing.assert_allclose(got, want, atol=1e-13)
+
+
+def test_dense_decode_special_cases():
+    g = _rng(22)
+    K = g.standard_normal((50, 16))
+    V = g.standard_normal((50, 16))
+    np.testing.assert_allclose(O.dense_decode(np.zeros((1, 16)), K, V, 1e6)[0], V.mean(0),
+                               atol=1e-14)
+    q = 1e4 * O.rope_rotate(K[17:18], [17], 1e6)
+    np.testing.assert_allclose(O.dense_decode(q, K, V, 1e6)[0], V[17], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# memory accounting
+# ----------------------------------------------------------------------------
+
+
+def test_full_kv_bytes_matches_a40_figure():
+    with open(os.path.join(GOLDEN, "a40_memory.json")) as fh:
+        gd = json.load(fh)
+    got = O.full_kv_bytes(gd["tokens"], gd["layers"], gd["kv_heads"], gd["head_dim"],
+                          gd["elem_bytes"]) / 2 ** 30
+    assert got == gd["full_gib"]
+
+
+# ----------------------------------------------------------------------------
+# mutation tests: plant mistakes in a copy of the fold, check the pins fail
+# ----------------------------------------------------------------------------
+
+
+def _mutated_fold(kind):
+    def fold(B, S, X):
+        B = np.asarray(B, float)
+        S = np.asarray(S, float)
+        X = np.asarray(X, float)
+        d, r = B.shape
+        b = X.shape[0]
+        k = min(b, d - r)
+        P = X @ B if kind != "negP" else -(X @ B)
+        E = X - (X @ B) @ B.T
+        M = np.concatenate([B, E.T], axis=1)
+        Qf, _ = np.linalg.qr(M, mode="complete")
+        Q = Qf[:, r:r + k] if kind != "index" else Qf[:, r - 1:r - 1 + k]
+        R_E = Q.T @ E.T
+        core = np.zeros((r + b, r + k))
+        core[:r, :r] = np.diag(S) if kind != "dropS" else 0.0
+        core[r:, :r] = P
+        core[r:, r:] = R_E.T
+        _, sigma, Wt = np.linalg.svd(core)
+        W = Wt.T if kind != "transpose" else Wt
+        W_r = W[:, :r] if kind != "smallest" else W[:, -r:]
+        return O.FoldResult(B_new=np.concatenate([B, Q], 1) @ W_r, S_new=sigma[:r],
+                            W_top=W_r[:r], C_new=core[r:] @ W_r, W_r=W_r, sigma=sigma,
+                            P=P, E=E, Q=Q, R_E=R_E, core=core)
+    return fold
+
+
+@pytest.mark.parametrize("kind", ["negP", "index", "dropS", "transpose", "smallest"])
+def test_pins_catch_planted_mistakes(kind, monkeypatch):
+    monkeypatch.setattr(O, "fold_block", _mutated_fold(kind))
+    caught = []
+    for check in (test_exact_rank_history_is_reproduced,
+                  lambda: test_fold_identities(64),
+                  test_sync_closed_form,
+                  lambda: test_full_rank_is_lossless(0)):
+        try:
+            check()
+        except (AssertionError, ValueError, np.linalg.LinAlgError):
+            caught.append(check)
+    assert caught, f"planted mistake {kind!r} went unnoticed"
+
+
+def test_residual_sign_is_absorbed_by_rule_q():
+    """Rule Q takes R_E = Q^T E^T with Q orthogonal to B, so any multiple of
+    the B-components in E cancels: a residual formed with the wrong sign
+    gives the same fold.  (Documents why that mutation is not a mistake.)"""
+    g = _rng(31)
+    B, _ = np.linalg.qr(g.standard_normal((128, 32)))
+    S = np.sort(g.uniform(1, 5, 32))[::-1]
+    X = g.standard_normal((64, 128))
+    good = O.fold_block(B, S, X)
+    Ebad = X + (X @ B) @ B.T
+    Qf, _ = np.linalg.qr(np.concatenate([B, Ebad.T], 1), mode="complete")
+    np.testing.assert_allclose(np.abs(Qf[:, 32:96].T @ Ebad.T), np.abs(good.R_E), atol=1e-11)
+
+
+def test_oracle_exports():
+    for name in ("bf16_round", "ready_blocks", "rope_rotate", "fold_block", "HeadFactor",
+                 "dense_decode", "full_kv_bytes"):
+        assert hasattr(oracle, name)
+    _ = itertools
