@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the iS-KV hot path on B200: compressed-KV decode over a
+32K-token, 36-layer, batch-8 Qwen3-8B-shaped cache (8 KV / 32 query heads,
+d 128, r_K 32, r_V 64, W 1024, bf16 K/V and coefficients, fp32 bases).
+
+One bench step = one fold period: 64 decode steps (per layer: append one
+token, decode attention for 32 query heads of 8 sequences), then one block
+fold of every layer (project, QR, core SVD, basis update, coefficient
+resync).  value = decode steps/s (each step = one token for all 8 sequences
+through all 36 layers); every timed step contains exactly one fold, so the
+block update is amortized honestly.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl iskv|reference]
+
+Multi-GPU: one process per GPU (torchrun), each an independent replica with
+its own batch (weak scaling, no data-path collective); rank 0 prints the
+max-over-ranks timing.  ``--impl reference`` times the float64 CPU oracle on
+the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode steps/s at 32K ctx; block-update µs; % of HBM roofline"
+UNIT = "decode steps/s"
+
+WORKLOADS = {
+    # name: batch, layers, kv_heads, q_heads, rank_k, rank_v, window, prefill, coef
+    "qwen3-36L-b8-32k": dict(batch=8, layers=36, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
+                             window=1024, prefill=32768, coef="bf16", gen="qwen3"),
+    "qwen3-1L-b1-16k": dict(batch=1, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
+                            window=1024, prefill=16384, coef="f32", gen="qwen3"),
+}
+DEFAULT_WORKLOAD = "qwen3-36L-b8-32k"
+D = 128
+BLOCK = 64
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            j = json.load(fh)
+        return float(j["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return 6650.0, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+
+def oracle_sample(wl, budget_s: float = 15.0, seed: int = 0):
+    """Time the float64 oracle, as it stands, on a bounded sample of the
+    workload: head decodes at the workload's context and block folds; scale
+    to decode steps/s of the full workload (all layers, sequences, heads,
+    one fold per 64 steps)."""
+    import numpy as np
+    from oracle import HeadFactor, dense_decode, fold_block
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    rng = np.random.default_rng(seed)
+    T = wl["prefill"]
+    n_c = ((T - wl["window"]) // BLOCK) * BLOCK
+    g = wl["q_heads"] // wl["kv_heads"]
+
+    def factor(r):
+        B, _ = np.linalg.qr(rng.standard_normal((D, r)))
+        f = HeadFactor(D, r, wl["window"])
+        f.B = B
+        f.S = np.sort(rng.uniform(1, 50, r))[::-1]
+        f.C = rng.standard_normal((n_c, r))
+        f.n_c = n_c
+        f.rows = rng.standard_normal((T, D))
+        return f
+
+    fk, fv = factor(wl["rank_k"]), factor(wl["rank_v"])
+    q = rng.standard_normal((g, D))
+    t_dec, n_dec = 0.0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s * 0.6 or n_dec < 2:
+        a = time.perf_counter()
+        dense_decode(q, fk.full(), fv.full(), 1e6)
+        t_dec += time.perf_counter() - a
+        n_dec += 1
+    t_fold, n_fold = 0.0, 0
+    t1 = time.perf_counter()
+    while time.perf_counter() - t1 < budget_s * 0.4 or n_fold < 2:
+        for f in (fk, fv):
+            X = rng.standard_normal((BLOCK, D))
+            a = time.perf_counter()
+            res = fold_block(f.B, f.S, X)
+            f.C @ res.W_top                    # step (e) over the history
+            t_fold += time.perf_counter() - a
+            n_fold += 1
+    heads = wl["layers"] * wl["batch"] * wl["kv_heads"]
+    per_dec = t_dec / n_dec
+    per_fold = t_fold / n_fold                   # one factor (K or V), averaged
+    step_s = heads * per_dec + 2 * heads * per_fold / BLOCK
+    sample = (f"{n_dec} head-decodes ({g} query heads over {T} tokens) and {n_fold} factor folds "
+              f"(with the rewrite of {n_c} rows) at the workload's shapes; scaled to {heads} "
+              f"(layer, sequence, KV head) decodes plus 1/64 fold of {2 * heads} factors per step")
+    return 1.0 / step_s, cores, sample, t_dec + t_fold
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+
+def run_iskv(args, rank, world, local_rank):
+    import torch
+
+    import online_rank_kv_b200 as ik
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    L, Bsz, H, Hq = wl["layers"], wl["batch"], wl["kv_heads"], wl["q_heads"]
+    g = Hq // H
+    coef = ik.BF16 if wl["coef"] == "bf16" else ik.F32
+    e2e_periods = max(1, args.steps // 2)
+    measure_periods = 1
+    periods = args.warmup + args.steps + e2e_periods + measure_periods
+    n_steps = periods * BLOCK
+    max_tokens = wl["prefill"] + n_steps + BLOCK
+    cfg = ik.Config(batch=Bsz, layers=L, kv_heads=H, q_heads=Hq, rank_k=wl["rank_k"],
+                    rank_v=wl["rank_v"], window=wl["window"], max_tokens=max_tokens,
+                    kv_dtype=ik.BF16, coef_dtype=coef, use_rope=1, rope_theta=1e6,
+                    max_deferred=64)
+    cache = ik.Cache(cfg)
+    kdt = torch.bfloat16
+    nh = L * Bsz * H
+    ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=1000 * rank + 1, device=dev,
+                        dtype=kdt)
+    vs = synth.KVStream(synth.spec_for(wl["gen"], "V"), nh, seed=1000 * rank + 2, device=dev,
+                        dtype=kdt)
+
+    # ---- prefill (untimed): fold with postponed rewrites, one rewrite per 64 folds
+    t_pre = time.time()
+    folds = 0
+    for _ in range(wl["prefill"] // BLOCK):
+        k = ks.next(BLOCK).view(L, Bsz, H, BLOCK, D)
+        v = vs.next(BLOCK).view(L, Bsz, H, BLOCK, D)
+        for l in range(L):
+            cache.append(l, k[l], v[l])
+        T, n_c = cache.counts(0)
+        while (T - n_c - wl["window"]) // BLOCK >= 1:
+            cache.compress_block(ik.ALL_LAYERS, defer=True)
+            folds += 1
+            if folds % 64 == 0:
+                cache.sync(ik.ALL_LAYERS)
+            T, n_c = cache.counts(0)
+    cache.sync(ik.ALL_LAYERS)
+    torch.cuda.synchronize()
+    prefill_s = time.time() - t_pre
+
+    # ---- decode inputs for every step, resident in HBM
+    kk = ks.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
+    vv = vs.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
+    qq = synth.query_batch(n_steps * L * Bsz * Hq, D, seed=1000 * rank + 3, device=dev,
+                           dtype=kdt).view(n_steps, L, Bsz, Hq, D)
+    outs = torch.empty(L, Bsz, Hq, D, dtype=torch.float32, device=dev)
+    kk = kk.view(n_steps, L, Bsz, H, 1, D)
+    vv = vv.view(n_steps, L, Bsz, H, 1, D)
+    stream = torch.cuda.current_stream()
+
+    step_ctr = [0]
+    dec_events = []
+
+    def period(host=None, time_decode=False):
+        for s in range(BLOCK):
+            i = step_ctr[0]
+            step_ctr[0] += 1
+            ev = time_decode and (s % 8 == 0)
+            for l in range(L):
+                if host is None:
+                    cache.append(l, kk[i, l], vv[i, l])
+                    if ev:
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record(stream)
+                    cache.decode_attention(l, qq[i, l], out=outs[l])
+                    if ev:
+                        e1.record(stream)
+                        T, n_c = cache.counts(l)
+                        dec_events.append((e0, e1, T, n_c))
+                else:
+                    hk, hv, hq, ho = host
+                    cache.append(l, hk[i, l], hv[i, l])
+                    cache.decode_attention(l, hq[i, l], out=ho[i % 2, l])
+        cache.compress_block(ik.ALL_LAYERS)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        period()
+    barrier()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        period(time_decode=True)
+    e_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(e_start.elapsed_time(e_end))
+    per_step_ms = ms / args.steps
+    decode_steps = args.steps * BLOCK * world
+    value = decode_steps / (ms / 1e3)
+
+    # decode-attention roofline from the events taken inside the timed region
+    peak, peak_src = _peaks()
+    dsum, bsum = 0.0, 0.0
+    kvb, cb = 2, (2 if coef == ik.BF16 else 4)
+    for e0, e1, T, n_c in dec_events:
+        t = e0.elapsed_time(e1) / 1e3
+        n_w = T - n_c
+        per_head = (n_c * (wl["rank_k"] + wl["rank_v"]) * cb + 2 * n_w * D * kvb
+                    + D * (wl["rank_k"] + wl["rank_v"]) * 4)
+        byts = Bsz * H * per_head + Bsz * Hq * D * (kvb + 4)
+        dsum += t
+        bsum += byts
+    dec_avg_us = dsum / max(1, len(dec_events)) * 1e6
+    achieved = bsum / dsum / 1e9 if dsum > 0 else 0.0
+
+    # ---- block update timing (fold and rewrite separately), untimed pass
+    fold_us = resync_us = None
+    for _ in range(BLOCK):
+        i = step_ctr[0]
+        step_ctr[0] += 1
+        for l in range(L):
+            cache.append(l, kk[i, l], vv[i, l])
+            cache.decode_attention(l, qq[i, l], out=outs[l])
+    f0, f1, f2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    cache_T, cache_nc = cache.counts(0)
+    f0.record(stream)
+    cache.compress_block(ik.ALL_LAYERS, defer=True)
+    f1.record(stream)
+    cache.sync(ik.ALL_LAYERS)
+    f2.record(stream)
+    torch.cuda.synchronize()
+    fold_us = f0.elapsed_time(f1) * 1e3
+    resync_us = f1.elapsed_time(f2) * 1e3
+    heads = L * Bsz * H
+    resync_bytes = 2 * cache_nc * (wl["rank_k"] + wl["rank_v"]) * cb * heads
+    resync_gbs = resync_bytes / (resync_us * 1e-6) / 1e9
+
+    # ---- end to end through the C ABI with pinned host buffers
+    hk = kk.cpu().pin_memory()
+    hv = vv.cpu().pin_memory()
+    hq = qq.cpu().pin_memory()
+    ho = torch.empty(2, L, Bsz, Hq, D, dtype=torch.float32).pin_memory()
+    barrier()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(e2e_periods):
+        period(host=(hk, hv, hq, ho))
+    x1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1))
+    e2e_value = e2e_periods * BLOCK * world / (e2e_ms / 1e3)
+    h2d = BLOCK * L * (2 * Bsz * H * D * kvb + Bsz * Hq * D * kvb)
+    d2h = BLOCK * L * Bsz * Hq * D * 4
+    status = cache.status()
+
+    launches_per_period = BLOCK * L * (2 + 2) + 6
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H, "q_heads": Hq,
+            "head_dim": D, "rank_k": wl["rank_k"], "rank_v": wl["rank_v"],
+            "window": wl["window"], "context_start": wl["prefill"],
+            "storage": f"K/V bf16, coefficients {wl['coef']}, bases fp32",
+            "step": "64 decode steps (append + decode attention, every layer) + 1 block fold "
+                    "of every layer (fold + coefficient rewrite)",
+            "l2": "inputs larger than L2 (each decode step streams ~15 GB)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "tokens_per_s": value * Bsz,
+        "block_update_us": fold_us + resync_us,
+        "fold_us": fold_us, "resync_us": resync_us, "resync_gbs": resync_gbs,
+        "decode_attention_us_avg": dec_avg_us,
+        "prefill_s": prefill_s,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "decode attention (split-K decode + combine), per layer call",
+                     "peak_source": peak_src},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_period * args.steps,
+        "clocks": clk,
+        "device_status": status,
+    }
+    cache.close()
+    return result
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="iskv", choices=["iskv", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        wl = WORKLOADS[args.workload]
+        vals = []
+        cores = sample = None
+        per = max(2.0, args.cpu_budget / max(1, args.steps + args.warmup))
+        for i in range(args.warmup + args.steps):
+            v, cores, sample, _ = oracle_sample(wl, budget_s=per, seed=i)
+            if i >= args.warmup:
+                vals.append(v)
+        value = statistics.mean(vals)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * BLOCK / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": wl["batch"], "layers": wl["layers"],
+                       "kv_heads": wl["kv_heads"], "q_heads": wl["q_heads"],
+                       "context_start": wl["prefill"]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
+    try:
+        res = run_iskv(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                v, cores, sample, used = oracle_sample(WORKLOADS[args.workload],
+                                                       budget_s=args.cpu_budget)
+                res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                       "sample": sample + f" ({used:.1f} s of CPU work)"}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+/*
+ * iskv.h -- C ABI of the B200 (sm_100a) iS-KV cache: basis-synchronized online
+ * low-rank KV compression.
+ *
+ * Method source: "iS-KV -- Basis-synchronized online low-rank KV compression
+ * -- What does it mean?" (learnaivisually.com explainer).  Per KV head the
+ * newest W tokens stay exact; every 64-row block that leaves that window is
+ * folded into a rank-r factorization (coefficients C, n x r; orthonormal basis
+ * B, d x r; singular values S) by Brand's block-incremental SVD, and every old
+ * coefficient row is rewritten in the new basis at the same update (Jargon:
+ * Block-incremental SVD; the body paragraph on basis synchronization and
+ * drift).  Keys are stored before RoPE and rotated when read (Jargon:
+ * Pre-RoPE keys).  Decode attention reads the mixed cache directly, without
+ * rebuilding values (ASKV design report, Design requirements: no
+ * reconstruction on the decode path).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Return value: ISKV_OK (0) or a negative ISKV_ERR_* code.  Nothing throws
+ *    across the ABI.  iskv_strerror() names a code.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Work is enqueued on it and the call returns without
+ *    waiting, except iskv_status, iskv_get_counts and iskv_destroy.  Calls on
+ *    one cache must be ordered on one stream (or ordered by the caller).
+ *  - Caller buffers (k, v, q, out, ...): contiguous, row-major, owned by the
+ *    caller and borrowed only for the stream-ordered duration of the call.
+ *    They may be device memory or host memory (pinned or pageable); host
+ *    buffers are detected with cudaPointerGetAttributes and staged through the
+ *    cache's own device buffers with cudaMemcpyAsync on `stream`.
+ *  - Counters: T (tokens appended) and n_c (tokens folded, a multiple of 64)
+ *    are kept per layer on the host and are shared by the whole batch; they
+ *    advance when a call is enqueued, so they are exact integers at all times.
+ *  - The cache owns all of its device memory, allocated once in iskv_create
+ *    for `max_tokens`; no entry point allocates after that.
+ */
+#ifndef ISKV_H
+#define ISKV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define ISKV_API __attribute__((visibility("default")))
+#else
+#define ISKV_API
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define ISKV_OK                 0
+#define ISKV_ERR_INVALID_ARG   -1  /* bad pointer, shape, layer or config   */
+#define ISKV_ERR_CAPACITY      -2  /* T would exceed max_tokens, or the exact
+                                      window would overflow its ring        */
+#define ISKV_ERR_STATE         -3  /* no ready block to fold, decode of an
+                                      empty cache, postponed rewrites pending,
+                                      or too many postponed folds           */
+#define ISKV_ERR_CUDA          -4  /* a CUDA runtime call failed            */
+#define ISKV_ERR_NOCONVERGE    -5  /* a core SVD hit its sweep limit (sticky;
+                                      results are finite but less accurate) */
+#define ISKV_ERR_NOMEM         -6  /* device allocation failed in create    */
+#define ISKV_ERR_UNSUPPORTED   -7  /* shape outside the compiled kernels    */
+
+/* ---- element types ----------------------------------------------------- */
+#define ISKV_F32   0
+#define ISKV_BF16  1
+
+/* ---- selectors and flags ----------------------------------------------- */
+#define ISKV_WHICH_K 0
+#define ISKV_WHICH_V 1
+#define ISKV_ALL_LAYERS (-1)
+/* iskv_compress_block flag: fold now, postpone the rewrite of the rows that
+ * are already stored (step (e)) until iskv_sync.  Meant for prefill, where
+ * nothing reads the cache between folds: the postponed rewrites are applied
+ * in fold order by one pass over the stored rows.                          */
+#define ISKV_FOLD_DEFER_SYNC 1
+
+typedef struct iskv_cache* iskv_t;
+
+/* Shape and format of one cache (a batch of equal-length sequences, every
+ * layer of a model).  head_dim must be 128 and block 64 in this build.      */
+typedef struct {
+    int32_t batch;          /* sequences                                    */
+    int32_t layers;         /* model layers held by this cache (<= 128)     */
+    int32_t kv_heads;       /* KV heads per layer                           */
+    int32_t q_heads;        /* query heads; a multiple of kv_heads (GQA)    */
+    int32_t head_dim;       /* d = 128                                      */
+    int32_t rank_k;         /* r_K: multiple of 16, 16 <= r_K <= d          */
+    int32_t rank_v;         /* r_V: multiple of 16, 16 <= r_V <= d          */
+    int32_t window;         /* W: exact recent tokens, multiple of 64       */
+    int32_t block;          /* rows folded at once: 64                      */
+    int32_t max_tokens;     /* capacity of T per layer                      */
+    int32_t kv_dtype;       /* ISKV_F32 or ISKV_BF16: k, v and q elements    */
+    int32_t coef_dtype;     /* ISKV_F32 or ISKV_BF16: stored coefficients C  */
+    int32_t use_rope;       /* 1: keys are rotated by RoPE when read         */
+    double  rope_theta;     /* RoPE base (1e6 for Qwen3-shaped caches)       */
+    int32_t sync;           /* 1: rewrite old rows at every fold (the method);
+                               0: no-synchronization ablation               */
+    int32_t max_deferred;   /* folds whose rewrite may be postponed before an
+                               iskv_sync is required (0: no postponing)     */
+    int32_t jacobi_max_sweeps; /* sweep limit of the core SVD (0: 40)        */
+    int32_t ring_extra;     /* exact-window ring rows beyond W + 64 (0: 64)  */
+} iskv_config;
+
+/* Fill `cfg` with the defaults of the one-layer Qwen3-8B-shaped cache
+ * (8 KV / 32 query heads, d 128, r_K 32, r_V 64, W 1024, bf16 K/V, fp32 C,
+ * RoPE theta 1e6).  Returns ISKV_OK, or ISKV_ERR_INVALID_ARG for NULL.     */
+ISKV_API int iskv_config_default(iskv_config* cfg);
+
+/* Create a cache: validates `cfg`, allocates every device buffer for
+ * max_tokens on `stream`, sets B = I_d[:, :r], S = 0, T = n_c = 0.  On
+ * success *out owns the cache; on failure *out is NULL and nothing leaks.   */
+ISKV_API int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out);
+
+/* Synchronize the cache's streams, free everything.  NULL is a no-op.      */
+ISKV_API int iskv_destroy(iskv_t h);
+
+/* Append t tokens to every sequence of `layer`: k, v are
+ * [batch, kv_heads, t, head_dim] in kv_dtype, PRE-RoPE.  T += t.  Never folds.
+ * *ready_blocks (may be NULL) receives floor((T - n_c - W) / 64), at least 0:
+ * the whole blocks that have left the exact window and may be folded.
+ * Errors: CAPACITY if T + t > max_tokens or the ring would hold more than
+ * W + 64 + ring_extra rows (fold first).                                   */
+ISKV_API int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t,
+                void* stream, int* ready_blocks);
+
+/* Fold the oldest ready block of `layer` (or of every layer that has one,
+ * for ISKV_ALL_LAYERS), K and V factors of every (sequence, KV head), in one
+ * launch: (a) P = X B; (b) residual and Householder QR of the complement;
+ * (c) one-sided Jacobi SVD of the (r+64) x (r+k) core, truncated to r;
+ * (d) B' = [B, Q] W_r, S' and the block's coefficient rows; (e) unless
+ * ISKV_FOLD_DEFER_SYNC is set, every old row is rewritten, C <- C W_r[0:r,:].
+ * n_c += 64.  Errors: STATE if the layer has no ready block (for
+ * ISKV_ALL_LAYERS: if no layer has one) or if a deferred fold would exceed
+ * max_deferred.                                                           */
+ISKV_API int iskv_compress_block(iskv_t h, int layer, int flags, void* stream);
+
+/* Apply the postponed rewrites of `layer` (or ISKV_ALL_LAYERS) in fold order:
+ * one pass over the stored rows, each row multiplied by the product of the
+ * W_r[0:r,:] of the folds that came after it was written.  No-op if nothing
+ * is pending.                                                              */
+ISKV_API int iskv_sync(iskv_t h, int layer, void* stream);
+
+/* Decode attention of `layer`: q is [batch, q_heads, head_dim] in kv_dtype,
+ * already rotated for position T - 1; out is [batch, q_heads, head_dim]
+ * fp32.  Query head j reads KV head j / (q_heads / kv_heads).  Scores over
+ * all T tokens (folded rows rebuilt as C_K B_K^T and rotated at their absolute
+ * positions, exact rows rotated likewise), scale 1/sqrt(d), one softmax; the
+ * value side is (p^T C_V) B_V^T + p_win^T V_win.  Errors: STATE if T = 0 or
+ * rewrites are pending.                                                    */
+ISKV_API int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out,
+                          void* stream);
+
+/* Rebuild the folded rows of one factor before RoPE: out is
+ * [batch, kv_heads, n_c, head_dim] fp32 = C B^T.  `which` is ISKV_WHICH_K or
+ * ISKV_WHICH_V.  Errors: STATE if rewrites are pending.                    */
+ISKV_API int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* stream);
+
+/* Copy out one factor: basis [batch, kv_heads, head_dim, r] fp32 (row i of a
+ * head is basis row i), sigma [batch, kv_heads, r] fp32, coef
+ * [batch, kv_heads, n_c, r] in coef_dtype.  Any pointer may be NULL.        */
+ISKV_API int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
+                     void* coef, void* stream);
+
+/* Host counters of `layer`: tokens appended and tokens folded.             */
+ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
+
+/* Synchronize the cache's work and return its sticky device status:
+ * ISKV_OK, ISKV_ERR_NOCONVERGE or ISKV_ERR_CUDA.  Clears nothing.          */
+ISKV_API int iskv_status(iskv_t h);
+
+/* Static string naming a status code.                                     */
+ISKV_API const char* iskv_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISKV_H */

@@ -1,0 +1,535 @@
+// C ABI of the iS-KV cache (declared in include/iskv.h): configuration checks,
+// device buffers, host counters and the order of kernel launches.
+//
+// Bookkeeping follows the iS-KV explainer ("iS-KV -- Basis-synchronized online
+// low-rank KV compression -- What does it mean?": the newest W tokens stay
+// exact; every 64 tokens that leave that window are folded as one block):
+// T and n_c are host integers per layer, advanced when a call is enqueued;
+// ready blocks = floor((T - n_c - W) / 64) when positive.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "iskv_internal.cuh"
+
+using namespace iskv;
+
+struct iskv_cache {
+    iskv_config cfg{};
+    int device = 0;
+    int64_t cap = 0;      // ring rows per head
+    int64_t n_max = 0;    // coefficient rows per head
+    int BH = 0;
+    int D = 1;            // postponed-fold slots per head
+    int kv_bytes = 4, coef_bytes = 4;
+    // device memory
+    void* ring_k = nullptr;
+    void* ring_v = nullptr;
+    void* coef_k = nullptr;
+    void* coef_v = nullptr;
+    float* basis_k = nullptr;
+    float* basis_v = nullptr;
+    __nv_bfloat16* bsplit_k = nullptr;
+    __nv_bfloat16* bsplit_v = nullptr;
+    float* sigma_k = nullptr;
+    float* sigma_v = nullptr;
+    float* pend_k = nullptr;
+    float* pend_v = nullptr;
+    int* seg_rows = nullptr;
+    float* partial = nullptr;
+    float2* rope = nullptr;
+    int* status = nullptr;
+    void* stage_in = nullptr;     // host-input staging
+    size_t stage_in_bytes = 0;
+    float* stage_out = nullptr;   // host-output staging
+    size_t stage_out_bytes = 0;
+    int max_splits = 256;
+    // host counters
+    std::vector<int64_t> T, n_c;
+    std::vector<int> n_pend;
+};
+
+namespace {
+
+constexpr size_t kStageBytes = 16u << 20;
+
+bool is_device_ptr(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+int validate(const iskv_config* c) {
+    if (!c) return ISKV_ERR_INVALID_ARG;
+    if (c->batch < 1 || c->layers < 1 || c->layers > kMaxLayers || c->kv_heads < 1 ||
+        c->q_heads < 1 || c->q_heads % c->kv_heads != 0)
+        return ISKV_ERR_INVALID_ARG;
+    if (c->q_heads / c->kv_heads > kMaxGroup) return ISKV_ERR_UNSUPPORTED;
+    if (c->head_dim != kHeadDim || c->block != kBlock) return ISKV_ERR_UNSUPPORTED;
+    for (int r : {c->rank_k, c->rank_v})
+        if (r < 16 || r > kHeadDim || r % 16 != 0) return ISKV_ERR_UNSUPPORTED;
+    if (c->window < 0 || c->window % kBlock != 0 || c->max_tokens < 1) return ISKV_ERR_INVALID_ARG;
+    if ((c->kv_dtype != ISKV_F32 && c->kv_dtype != ISKV_BF16) ||
+        (c->coef_dtype != ISKV_F32 && c->coef_dtype != ISKV_BF16))
+        return ISKV_ERR_INVALID_ARG;
+    if (c->use_rope != 0 && c->use_rope != 1) return ISKV_ERR_INVALID_ARG;
+    if (c->use_rope && !(c->rope_theta > 1.0)) return ISKV_ERR_INVALID_ARG;
+    if (c->sync != 0 && c->sync != 1) return ISKV_ERR_INVALID_ARG;
+    if (c->max_deferred < 0 || c->max_deferred > kMaxDeferred) return ISKV_ERR_INVALID_ARG;
+    if (c->jacobi_max_sweeps < 0 || c->jacobi_max_sweeps > 1000) return ISKV_ERR_INVALID_ARG;
+    if (c->ring_extra < 0 || c->ring_extra % kBlock != 0) return ISKV_ERR_INVALID_ARG;
+    return ISKV_OK;
+}
+
+FactorView view(const iskv_cache* h, int which) {
+    FactorView f{};
+    const bool K = which == ISKV_WHICH_K;
+    f.coef = K ? h->coef_k : h->coef_v;
+    f.basis = K ? h->basis_k : h->basis_v;
+    f.bsplit = K ? h->bsplit_k : h->bsplit_v;
+    f.sigma = K ? h->sigma_k : h->sigma_v;
+    f.pend = K ? h->pend_k : h->pend_v;
+    f.seg_rows = h->seg_rows;   // identical for K and V: both fold together
+    f.ring = K ? h->ring_k : h->ring_v;
+    f.r = K ? h->cfg.rank_k : h->cfg.rank_v;
+    f.coef_bf16 = h->cfg.coef_dtype == ISKV_BF16;
+    f.kv_bf16 = h->cfg.kv_dtype == ISKV_BF16;
+    f.n_max = h->n_max;
+    f.cap = h->cap;
+    f.D = h->D;
+    f.BH = h->BH;
+    return f;
+}
+
+int64_t ready_of(const iskv_cache* h, int layer) {
+    const int64_t excess = h->T[layer] - h->n_c[layer] - h->cfg.window;
+    return excess >= 0 ? excess / kBlock : 0;
+}
+
+#define CU(x)                                          \
+    do {                                               \
+        cudaError_t e_ = (x);                          \
+        if (e_ != cudaSuccess) return ISKV_ERR_CUDA;   \
+    } while (0)
+
+void free_all(iskv_cache* h) {
+    void* ptrs[] = {h->ring_k, h->ring_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
+                    h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
+                    h->seg_rows, h->partial, h->rope, h->status, h->stage_in, h->stage_out};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+}
+
+template <typename T>
+int dalloc(T** p, size_t bytes) {
+    void* q = nullptr;
+    if (bytes == 0) bytes = 16;
+    if (cudaMalloc(&q, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return ISKV_ERR_NOMEM;
+    }
+    *p = reinterpret_cast<T*>(q);
+    return ISKV_OK;
+}
+
+// Layers named by a call: one, or all of them.
+bool layers_of(const iskv_cache* h, int layer, std::vector<int>* out) {
+    out->clear();
+    if (layer == ISKV_ALL_LAYERS) {
+        for (int l = 0; l < h->cfg.layers; ++l) out->push_back(l);
+        return true;
+    }
+    if (layer < 0 || layer >= h->cfg.layers) return false;
+    out->push_back(layer);
+    return true;
+}
+
+// Rewrite the rows of the listed layers: compose postponed W_top, then the
+// per-segment rewrite.  `nseg`, `rows` per listed layer.
+int run_resync(iskv_cache* h, const std::vector<int>& layers, const std::vector<int>& nseg,
+               const std::vector<int>& rows, cudaStream_t s) {
+    ResyncLaunch rl{};
+    for (size_t i = 0; i < layers.size(); ++i) {
+        if (nseg[i] <= 0 || rows[i] <= 0) continue;
+        rl.layer[rl.n_tasks] = layers[i];
+        rl.n_seg[rl.n_tasks] = nseg[i];
+        rl.n_rows[rl.n_tasks] = rows[i];
+        ++rl.n_tasks;
+    }
+    if (rl.n_tasks == 0) return ISKV_OK;
+    bool chained = false;
+    for (int i = 0; i < rl.n_tasks; ++i) chained = chained || rl.n_seg[i] > 1;
+    for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) {
+        FactorView f = view(h, which);
+        if (chained) CU(launch_compose(f, rl, s));
+        CU(launch_resync(f, rl, s));
+    }
+    return ISKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int iskv_config_default(iskv_config* c) {
+    if (!c) return ISKV_ERR_INVALID_ARG;
+    std::memset(c, 0, sizeof(*c));
+    c->batch = 1;
+    c->layers = 1;
+    c->kv_heads = 8;
+    c->q_heads = 32;
+    c->head_dim = kHeadDim;
+    c->rank_k = 32;
+    c->rank_v = 64;
+    c->window = 1024;
+    c->block = kBlock;
+    c->max_tokens = 16384;
+    c->kv_dtype = ISKV_BF16;
+    c->coef_dtype = ISKV_F32;
+    c->use_rope = 1;
+    c->rope_theta = 1e6;
+    c->sync = 1;
+    c->max_deferred = 0;
+    c->jacobi_max_sweeps = 0;
+    c->ring_extra = 0;
+    return ISKV_OK;
+}
+
+int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
+    if (!out) return ISKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = validate(cfg);
+    if (rc != ISKV_OK) return rc;
+    iskv_cache* h = new (std::nothrow) iskv_cache();
+    if (!h) return ISKV_ERR_NOMEM;
+    h->cfg = *cfg;
+    if (h->cfg.jacobi_max_sweeps == 0) h->cfg.jacobi_max_sweeps = 40;
+    if (h->cfg.ring_extra == 0) h->cfg.ring_extra = kBlock;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaGetDevice(&h->device) != cudaSuccess) {
+        delete h;
+        return ISKV_ERR_CUDA;
+    }
+    const iskv_config& c = h->cfg;
+    h->BH = c.batch * c.kv_heads;
+    h->cap = (int64_t)c.window + kBlock + c.ring_extra;
+    int64_t nm = (int64_t)c.max_tokens - c.window;
+    if (nm < 0) nm = 0;
+    h->n_max = (nm / kBlock) * kBlock + 2 * kBlock;   // slack rows for whole tiles
+    h->D = c.max_deferred > 0 ? c.max_deferred : 1;
+    h->kv_bytes = c.kv_dtype == ISKV_BF16 ? 2 : 4;
+    h->coef_bytes = c.coef_dtype == ISKV_BF16 ? 2 : 4;
+    h->T.assign(c.layers, 0);
+    h->n_c.assign(c.layers, 0);
+    h->n_pend.assign(c.layers, 0);
+
+    const size_t heads = (size_t)c.layers * h->BH;
+    const size_t d = kHeadDim;
+    size_t ring_bytes = heads * h->cap * d * h->kv_bytes;
+    rc = ISKV_OK;
+    rc = rc ? rc : dalloc(&h->ring_k, ring_bytes);
+    rc = rc ? rc : dalloc(&h->ring_v, ring_bytes);
+    rc = rc ? rc : dalloc(&h->coef_k, heads * h->n_max * c.rank_k * h->coef_bytes);
+    rc = rc ? rc : dalloc(&h->coef_v, heads * h->n_max * c.rank_v * h->coef_bytes);
+    rc = rc ? rc : dalloc(&h->basis_k, heads * d * c.rank_k * 4);
+    rc = rc ? rc : dalloc(&h->basis_v, heads * d * c.rank_v * 4);
+    rc = rc ? rc : dalloc(&h->bsplit_k, heads * 2 * d * c.rank_k * 2);
+    rc = rc ? rc : dalloc(&h->bsplit_v, heads * 2 * d * c.rank_v * 2);
+    rc = rc ? rc : dalloc(&h->sigma_k, heads * c.rank_k * 4);
+    rc = rc ? rc : dalloc(&h->sigma_v, heads * c.rank_v * 4);
+    rc = rc ? rc : dalloc(&h->pend_k, heads * h->D * (size_t)c.rank_k * c.rank_k * 4);
+    rc = rc ? rc : dalloc(&h->pend_v, heads * h->D * (size_t)c.rank_v * c.rank_v * 4);
+    rc = rc ? rc : dalloc(&h->seg_rows, (size_t)c.layers * h->D * 4);
+    rc = rc ? rc : dalloc(&h->partial, (size_t)c.batch * c.q_heads * h->max_splits *
+                                           (2 + c.rank_v + d) * 4);
+    rc = rc ? rc : dalloc(&h->status, 16);
+    h->stage_in_bytes = kStageBytes;
+    h->stage_out_bytes = kStageBytes;
+    rc = rc ? rc : dalloc(&h->stage_in, h->stage_in_bytes);
+    rc = rc ? rc : dalloc(&h->stage_out, h->stage_out_bytes);
+    if (rc == ISKV_OK && c.use_rope) {
+        rc = dalloc(&h->rope, (size_t)c.max_tokens * (d / 2) * sizeof(float2));
+        if (rc == ISKV_OK) {
+            // cos/sin of pos * theta^(-2i/d), evaluated in double precision
+            std::vector<float2> tab((size_t)c.max_tokens * (d / 2));
+            std::vector<double> inv(d / 2);
+            for (size_t i = 0; i < d / 2; ++i) inv[i] = std::pow(c.rope_theta, -2.0 * (double)i / (double)d);
+            for (int64_t p = 0; p < c.max_tokens; ++p)
+                for (size_t i = 0; i < d / 2; ++i) {
+                    const double ang = (double)p * inv[i];
+                    tab[p * (d / 2) + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+                }
+            if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) !=
+                cudaSuccess)
+                rc = ISKV_ERR_CUDA;
+        }
+    }
+    if (rc == ISKV_OK) {
+        if (cudaMemsetAsync(h->ring_k, 0, ring_bytes, s) != cudaSuccess ||
+            cudaMemsetAsync(h->ring_v, 0, ring_bytes, s) != cudaSuccess ||
+            cudaMemsetAsync(h->coef_k, 0, heads * h->n_max * c.rank_k * h->coef_bytes, s) != cudaSuccess ||
+            cudaMemsetAsync(h->coef_v, 0, heads * h->n_max * c.rank_v * h->coef_bytes, s) != cudaSuccess ||
+            cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess ||
+            cudaMemsetAsync(h->seg_rows, 0, (size_t)c.layers * h->D * 4, s) != cudaSuccess ||
+            launch_init_factor(view(h, ISKV_WHICH_K), c.layers, s) != cudaSuccess ||
+            launch_init_factor(view(h, ISKV_WHICH_V), c.layers, s) != cudaSuccess)
+            rc = ISKV_ERR_CUDA;
+    }
+    if (rc != ISKV_OK) {
+        free_all(h);
+        delete h;
+        return rc;
+    }
+    *out = h;
+    return ISKV_OK;
+}
+
+int iskv_destroy(iskv_t h) {
+    if (!h) return ISKV_OK;
+    cudaDeviceSynchronize();
+    free_all(h);
+    delete h;
+    return ISKV_OK;
+}
+
+int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* stream,
+                int* ready_blocks) {
+    if (!h || !k || !v || t < 0 || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
+    const int64_t T1 = h->T[layer] + t;
+    if (T1 > h->cfg.max_tokens || T1 - h->n_c[layer] > h->cap) return ISKV_ERR_CAPACITY;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (t > 0) {
+        const size_t row_bytes = (size_t)kHeadDim * h->kv_bytes;
+        const size_t head_stride = (size_t)h->cap * row_bytes;
+        char* rk = reinterpret_cast<char*>(h->ring_k) + (size_t)layer * h->BH * head_stride;
+        char* rv = reinterpret_cast<char*>(h->ring_v) + (size_t)layer * h->BH * head_stride;
+        const void* srcs[2] = {k, v};
+        char* rings[2] = {rk, rv};
+        for (int w = 0; w < 2; ++w) {
+            if (is_device_ptr(srcs[w])) {
+                CU(launch_append(rings[w], srcs[w], h->BH, t, h->T[layer], h->cap, h->kv_bytes, s));
+            } else {
+                // stage token chunks of every (sequence, head) through device memory
+                const int chunk = (int)std::max<size_t>(1, h->stage_in_bytes / ((size_t)h->BH * row_bytes));
+                for (int t0 = 0; t0 < t; t0 += chunk) {
+                    const int n = std::min(chunk, t - t0);
+                    CU(cudaMemcpy2DAsync(h->stage_in, n * row_bytes,
+                                         reinterpret_cast<const char*>(srcs[w]) + t0 * row_bytes,
+                                         (size_t)t * row_bytes, n * row_bytes, h->BH,
+                                         cudaMemcpyDefault, s));
+                    CU(launch_append(rings[w], h->stage_in, h->BH, n, h->T[layer] + t0, h->cap,
+                                     h->kv_bytes, s));
+                }
+            }
+        }
+    }
+    h->T[layer] = T1;
+    if (ready_blocks) *ready_blocks = (int)ready_of(h, layer);
+    return ISKV_OK;
+}
+
+int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
+    if (!h || (flags & ~ISKV_FOLD_DEFER_SYNC)) return ISKV_ERR_INVALID_ARG;
+    std::vector<int> ls;
+    if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
+    const bool want_defer = (flags & ISKV_FOLD_DEFER_SYNC) != 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    FoldLaunch fl{};
+    fl.max_sweeps = h->cfg.jacobi_max_sweeps;
+    std::vector<int> fold_layers;
+    for (int l : ls) {
+        if (ready_of(h, l) < 1) continue;
+        fold_layers.push_back(l);
+    }
+    if (fold_layers.empty()) return ISKV_ERR_STATE;
+    // every layer of this call postpones if asked to, or if it already has
+    // postponed folds (their rewrites must come first, in order)
+    for (int l : fold_layers) {
+        const bool defer = h->cfg.sync && (want_defer || h->n_pend[l] > 0);
+        if (defer && h->n_pend[l] >= h->D) return ISKV_ERR_STATE;
+        if (defer && h->cfg.max_deferred == 0 && want_defer) return ISKV_ERR_STATE;
+    }
+    for (int l : fold_layers) {
+        const bool defer = h->cfg.sync && (want_defer || h->n_pend[l] > 0);
+        fl.layer[fl.n_tasks] = l;
+        fl.n_c[fl.n_tasks] = (int)h->n_c[l];
+        fl.slot[fl.n_tasks] = defer ? h->n_pend[l] : 0;
+        ++fl.n_tasks;
+    }
+    for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) CU(launch_fold(view(h, which), fl, h->status, s));
+    std::vector<int> rl_layers, rl_seg, rl_rows;
+    for (int l : fold_layers) {
+        const bool defer = h->cfg.sync && (want_defer || h->n_pend[l] > 0);
+        const int64_t old = h->n_c[l];
+        h->n_c[l] += kBlock;
+        if (!h->cfg.sync) continue;
+        if (defer) {
+            h->n_pend[l] += 1;
+            if (!want_defer) {   // finish the postponed chain now
+                rl_layers.push_back(l);
+                rl_seg.push_back(h->n_pend[l]);
+                rl_rows.push_back((int)old);
+                h->n_pend[l] = 0;
+            }
+        } else if (old > 0) {
+            rl_layers.push_back(l);
+            rl_seg.push_back(1);
+            rl_rows.push_back((int)old);
+        }
+    }
+    return run_resync(h, rl_layers, rl_seg, rl_rows, s);
+}
+
+int iskv_sync(iskv_t h, int layer, void* stream) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    std::vector<int> ls;
+    if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
+    std::vector<int> rl_layers, rl_seg, rl_rows;
+    for (int l : ls) {
+        if (h->n_pend[l] == 0) continue;
+        rl_layers.push_back(l);
+        rl_seg.push_back(h->n_pend[l]);
+        rl_rows.push_back((int)(h->n_c[l] - kBlock));
+        h->n_pend[l] = 0;
+    }
+    return run_resync(h, rl_layers, rl_seg, rl_rows, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* stream) {
+    if (!h || !q || !out || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
+    if (h->T[layer] == 0 || h->n_pend[layer] > 0) return ISKV_ERR_STATE;
+    const iskv_config& c = h->cfg;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t q_bytes = (size_t)c.batch * c.q_heads * kHeadDim * h->kv_bytes;
+    const size_t o_bytes = (size_t)c.batch * c.q_heads * kHeadDim * sizeof(float);
+    const void* qd = q;
+    if (!is_device_ptr(q)) {
+        if (q_bytes > h->stage_in_bytes) return ISKV_ERR_UNSUPPORTED;
+        CU(cudaMemcpyAsync(h->stage_in, q, q_bytes, cudaMemcpyDefault, s));
+        qd = h->stage_in;
+    }
+    const bool host_out = !is_device_ptr(out);
+    if (host_out && o_bytes > h->stage_out_bytes) return ISKV_ERR_UNSUPPORTED;
+    float* od = host_out ? h->stage_out : out;
+
+    DecodeArgs a{};
+    a.K = view(h, ISKV_WHICH_K);
+    a.V = view(h, ISKV_WHICH_V);
+    a.q = qd;
+    a.partial = h->partial;
+    a.rope = c.use_rope ? h->rope : nullptr;
+    a.layer = layer;
+    a.B = c.batch;
+    a.Hkv = c.kv_heads;
+    a.Hq = c.q_heads;
+    a.g = c.q_heads / c.kv_heads;
+    a.T = h->T[layer];
+    a.n_c = h->n_c[layer];
+    a.scale = 1.0f / std::sqrt((float)kHeadDim);
+    // split the token axis so that the grid covers the GPU several times
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
+    const int64_t want = (int64_t)4 * sms;
+    int64_t splits = (want + h->BH - 1) / h->BH;
+    const int64_t max_by_tokens = (a.T + 63) / 64;
+    if (splits > max_by_tokens) splits = max_by_tokens;
+    if (splits > h->max_splits) splits = h->max_splits;
+    if (splits < 1) splits = 1;
+    int64_t tps = (a.T + splits - 1) / splits;
+    tps = ((tps + 63) / 64) * 64;
+    splits = (a.T + tps - 1) / tps;
+    a.tokens_per_split = tps;
+    a.splits = (int)splits;
+    CU(launch_decode(a, s));
+    CU(launch_combine(a, od, s));
+    if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
+    return ISKV_OK;
+}
+
+int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* stream) {
+    if (!h || !out || layer < 0 || layer >= h->cfg.layers ||
+        (which != ISKV_WHICH_K && which != ISKV_WHICH_V))
+        return ISKV_ERR_INVALID_ARG;
+    if (h->n_pend[layer] > 0) return ISKV_ERR_STATE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const FactorView f = view(h, which);
+    const int64_t rows = h->n_c[layer];
+    if (rows == 0) return ISKV_OK;
+    if (is_device_ptr(out)) {
+        CU(launch_reconstruct(f, layer, 0, rows, out, s));
+        return ISKV_OK;
+    }
+    const size_t row_bytes = (size_t)kHeadDim * sizeof(float);
+    int64_t chunk = (int64_t)(h->stage_out_bytes / (row_bytes * h->BH));
+    chunk = (chunk / 64) * 64;
+    if (chunk < 64) return ISKV_ERR_UNSUPPORTED;
+    for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+        const int64_t n = std::min(chunk, rows - r0);
+        CU(launch_reconstruct(f, layer, r0, n, h->stage_out, s));
+        CU(cudaMemcpy2DAsync(reinterpret_cast<char*>(out) + r0 * row_bytes, rows * row_bytes,
+                             h->stage_out, n * row_bytes, n * row_bytes, h->BH, cudaMemcpyDefault, s));
+    }
+    return ISKV_OK;
+}
+
+int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma, void* coef,
+                     void* stream) {
+    if (!h || layer < 0 || layer >= h->cfg.layers || (which != ISKV_WHICH_K && which != ISKV_WHICH_V))
+        return ISKV_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const FactorView f = view(h, which);
+    const size_t heads = h->BH;
+    const int r = f.r;
+    if (basis)
+        CU(cudaMemcpyAsync(basis, f.basis + (size_t)layer * heads * kHeadDim * r,
+                           heads * kHeadDim * r * sizeof(float), cudaMemcpyDefault, s));
+    if (sigma)
+        CU(cudaMemcpyAsync(sigma, f.sigma + (size_t)layer * heads * r, heads * r * sizeof(float),
+                           cudaMemcpyDefault, s));
+    if (coef && h->n_c[layer] > 0) {
+        const size_t rb = (size_t)r * h->coef_bytes;
+        const char* src = reinterpret_cast<const char*>(f.coef) + (size_t)layer * heads * h->n_max * rb;
+        CU(cudaMemcpy2DAsync(coef, h->n_c[layer] * rb, src, h->n_max * rb, h->n_c[layer] * rb, heads,
+                             cudaMemcpyDefault, s));
+    }
+    return ISKV_OK;
+}
+
+int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c) {
+    if (!h || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
+    if (T) *T = h->T[layer];
+    if (n_c) *n_c = h->n_c[layer];
+    return ISKV_OK;
+}
+
+int iskv_status(iskv_t h) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return ISKV_ERR_CUDA;
+    int st = 0;
+    if (cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return ISKV_ERR_CUDA;
+    if (st & kStatusNoConverge) return ISKV_ERR_NOCONVERGE;
+    return ISKV_OK;
+}
+
+const char* iskv_strerror(int code) {
+    switch (code) {
+        case ISKV_OK: return "ok";
+        case ISKV_ERR_INVALID_ARG: return "invalid argument";
+        case ISKV_ERR_CAPACITY: return "capacity exceeded (max_tokens or exact-window ring)";
+        case ISKV_ERR_STATE: return "invalid state (no ready block, empty cache, or pending rewrites)";
+        case ISKV_ERR_CUDA: return "CUDA runtime error";
+        case ISKV_ERR_NOCONVERGE: return "core SVD reached its sweep limit";
+        case ISKV_ERR_NOMEM: return "device allocation failed";
+        case ISKV_ERR_UNSUPPORTED: return "shape not supported by the compiled kernels";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+// Internal declarations of the iS-KV CUDA library (sm_100a).  Not part of the
+// C ABI: only the .cu files of this library include it.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/iskv.h"
+
+namespace iskv {
+
+constexpr int kHeadDim = 128;     // d
+constexpr int kBlock = 64;        // rows folded at once (b)
+constexpr int kMaxLayers = 128;   // layers per cache (bounds kernel params)
+constexpr int kMaxDeferred = 64;  // postponed folds per layer
+constexpr int kMaxGroup = 8;      // query heads per KV head in the decode
+
+// Status bits of the sticky device word.
+constexpr int kStatusNoConverge = 1;
+
+// ---------------------------------------------------------------------------
+// Element conversions (explicit round-to-nearest-even for bf16 stores).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// Launch descriptors (passed by value; sized well under the 4 KB limit).
+// ---------------------------------------------------------------------------
+
+// One factor (K or V) of every layer: element pointers of layer 0 and the
+// per-layer strides, so kernels address any (layer, sequence*head) pair.
+struct FactorView {
+    void* coef;          // [L][BH][n_max][r], coef dtype
+    float* basis;        // [L][BH][d][r]
+    __nv_bfloat16* bsplit;  // [L][BH][2][d][r]: bf16 hi and lo parts of basis
+    float* sigma;        // [L][BH][r]
+    float* pend;         // [L][BH][D][r*r]: W_r[0:r,:] of postponed folds
+    int* seg_rows;       // [L][D]: n_c before each postponed fold
+    const void* ring;    // [L][BH][cap][d], kv dtype (exact rows)
+    int r;
+    int coef_bf16;       // 1: coef stored as bf16
+    int kv_bf16;         // 1: ring stored as bf16
+    int64_t n_max;       // coefficient rows per head
+    int64_t cap;         // ring rows per head
+    int D;               // postponed-fold slots per head
+    int BH;              // batch * kv_heads
+};
+
+struct FoldLaunch {
+    int n_tasks;                 // layers folded by this launch
+    int layer[kMaxLayers];
+    int n_c[kMaxLayers];         // n_c before the fold
+    int slot[kMaxLayers];        // postponed-fold slot receiving W_r[0:r,:]
+    int max_sweeps;
+};
+
+struct ResyncLaunch {
+    int n_tasks;
+    int layer[kMaxLayers];
+    int n_seg[kMaxLayers];       // postponed folds to apply (segments)
+    int n_rows[kMaxLayers];      // rows to visit (n_c before the last fold)
+};
+
+struct DecodeArgs {
+    FactorView K, V;
+    const void* q;               // [B][Hq][d], kv dtype
+    float* partial;              // [B][Hq][splits][2 + r_V + d]
+    const float2* rope;          // [max_tokens][d/2] (cos, sin), or null
+    int layer, B, Hkv, Hq, g;
+    int64_t T, n_c;
+    int splits;
+    int64_t tokens_per_split;
+    float scale;                 // 1/sqrt(d)
+};
+
+// ---------------------------------------------------------------------------
+// Host launchers (one per kernel file).
+// ---------------------------------------------------------------------------
+cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s);
+cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0,
+                          int64_t cap, int elem_bytes, cudaStream_t s);
+cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status,
+                        cudaStream_t s);
+cudaError_t launch_compose(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);
+cudaError_t launch_resync(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const DecodeArgs& a, float* out, cudaStream_t s);
+cudaError_t launch_reconstruct(const FactorView& f, int layer, int64_t row0, int64_t rows,
+                               float* out, cudaStream_t s);
+
+size_t fold_smem_bytes(int r);
+
+}  // namespace iskv

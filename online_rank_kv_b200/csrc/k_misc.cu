@@ -1,0 +1,109 @@
+// Small kernels of the cache: factor initialization, appending exact rows to
+// the window ring, and rebuilding folded rows (C B^T, before RoPE).
+#include "iskv_internal.cuh"
+
+namespace iskv {
+
+namespace {
+
+// B = I_d[:, :r] (fp32 and its bf16 hi/lo parts), S = 0.
+__global__ void init_factor_kernel(FactorView f, int layers) {
+    const int64_t heads = (int64_t)layers * f.BH;
+    const int r = f.r;
+    const int64_t per = (int64_t)kHeadDim * r;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < heads * per;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t h = e / per, w = e % per;
+        const int i = (int)(w / r), j = (int)(w % r);
+        const float v = (i == j) ? 1.f : 0.f;
+        f.basis[e] = v;
+        f.bsplit[h * 2 * per + w] = __float2bfloat16_rn(v);
+        f.bsplit[h * 2 * per + per + w] = __float2bfloat16_rn(0.f);
+        if (w < r) f.sigma[h * r + w] = 0.f;
+    }
+}
+
+// ring[bh][(T0 + t) mod cap][:] = src[bh][t][:], 16-byte vectors.
+__global__ void append_kernel(uint4* ring, const uint4* src, int BH, int t, int64_t T0,
+                              int64_t cap, int vec_per_row) {
+    const int64_t total = (int64_t)BH * t * vec_per_row;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t v = e % vec_per_row;
+        const int64_t row = e / vec_per_row;
+        const int64_t bh = row / t, tt = row % t;
+        const int64_t slot = (T0 + tt) % cap;
+        ring[(bh * cap + slot) * vec_per_row + v] = src[e];
+    }
+}
+
+constexpr int kRecRows = 64;
+
+// out[bh][row][i] = sum_j C[row0 + row][j] B[i][j] for rows of one chunk.
+template <typename CoefT>
+__global__ void __launch_bounds__(256) reconstruct_kernel(FactorView f, int layer, int64_t row0,
+                                                          int64_t rows, float* out) {
+    const int bh = blockIdx.y;
+    const int64_t t0 = (int64_t)blockIdx.x * kRecRows;
+    if (t0 >= rows) return;
+    const int r = f.r;
+    extern __shared__ float sm[];
+    float* sB = sm;                       // d x (r+1), padded rows
+    float* sC = sm + kHeadDim * (r + 1);  // kRecRows x r
+    const int64_t hidx = (int64_t)layer * f.BH + bh;
+    const float* B = f.basis + hidx * kHeadDim * r;
+    const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + (hidx * f.n_max + row0 + t0) * r;
+    const int nt = (int)((rows - t0) < kRecRows ? (rows - t0) : kRecRows);
+    for (int e = threadIdx.x; e < kHeadDim * r; e += blockDim.x) sB[(e / r) * (r + 1) + e % r] = B[e];
+    for (int e = threadIdx.x; e < kRecRows * r; e += blockDim.x)
+        sC[e] = (e / r < nt) ? to_f32(C[e]) : 0.f;
+    __syncthreads();
+    float* o = out + ((int64_t)bh * rows + t0) * kHeadDim;
+    for (int e = threadIdx.x; e < nt * kHeadDim; e += blockDim.x) {
+        const int t = e / kHeadDim, i = e % kHeadDim;
+        float acc = 0.f;
+        for (int j = 0; j < r; ++j) acc = fmaf(sC[t * r + j], sB[i * (r + 1) + j], acc);
+        o[e] = acc;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s) {
+    init_factor_kernel<<<1184, 256, 0, s>>>(f, layers);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0, int64_t cap,
+                          int elem_bytes, cudaStream_t s) {
+    const int vec_per_row = kHeadDim * elem_bytes / 16;
+    const int64_t total = (int64_t)BH * t * vec_per_row;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 4736) blocks = 4736;
+    if (blocks < 1) blocks = 1;
+    append_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(ring),
+                                                   reinterpret_cast<const uint4*>(src), BH, t, T0,
+                                                   cap, vec_per_row);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reconstruct(const FactorView& f, int layer, int64_t row0, int64_t rows,
+                               float* out, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    const size_t bytes = ((size_t)kHeadDim * (f.r + 1) + (size_t)kRecRows * f.r) * sizeof(float);
+    dim3 grid((unsigned)((rows + kRecRows - 1) / kRecRows), f.BH);
+    if (f.coef_bf16) {
+        auto k = reconstruct_kernel<__nv_bfloat16>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 256, bytes, s>>>(f, layer, row0, rows, out);
+    } else {
+        auto k = reconstruct_kernel<float>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 256, bytes, s>>>(f, layer, row0, rows, out);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace iskv

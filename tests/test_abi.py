@@ -1,0 +1,99 @@
+"""The C-ABI library loads and exports every entry point ``include/iskv.h``
+declares, and its host-side argument checks work without a GPU."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "iskv.h")
+
+
+def _lib():
+    so = os.path.join(ROOT, "online_rank_kv_b200", "libiskv.so")
+    if not os.path.exists(so):
+        from online_rank_kv_b200.build import build
+        build()
+    import online_rank_kv_b200 as ik
+    return ik
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ISKV_API\s+[\w\s\*]+?\b(iskv_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("iskv_create", "iskv_append", "iskv_compress_block", "iskv_decode_attention",
+              "iskv_reconstruct", "iskv_destroy", "iskv_status", "iskv_sync"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported():
+    ik = _lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", ik.lib_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (iskv_\w+)", out))
+    for n in _declared():
+        assert n in exported, n
+        assert hasattr(ik.LIB, n)
+    assert set(ik.EXPORTED) == set(_declared())
+
+
+def test_config_struct_layout_matches_header(tmp_path):
+    ik = _lib()
+    src = tmp_path / "sz.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "iskv.h"\n'
+                   'int main(){printf("%zu %zu %zu %zu",sizeof(iskv_config),'
+                   'offsetof(iskv_config,rope_theta),offsetof(iskv_config,sync),'
+                   'offsetof(iskv_config,ring_extra));return 0;}\n')
+    exe = tmp_path / "sz"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    C = ik._Cfg
+    assert got == [ctypes.sizeof(C), C.rope_theta.offset, C.sync.offset, C.ring_extra.offset]
+
+
+def test_defaults_and_strings():
+    ik = _lib()
+    c = ik._Cfg()
+    assert ik.LIB.iskv_config_default(ctypes.byref(c)) == 0
+    assert (c.kv_heads, c.q_heads, c.head_dim, c.rank_k, c.rank_v, c.window, c.block) == \
+        (8, 32, 128, 32, 64, 1024, 64)
+    assert ik.LIB.iskv_config_default(None) == -1
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        assert len(ik.LIB.iskv_strerror(code)) > 0
+    assert ik.LIB.iskv_strerror(42) == b"unknown status"
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 64, -7), ("block", 32, -7), ("rank_k", 24, -7), ("rank_v", 144, -7),
+    ("q_heads", 12, -1), ("window", 100, -1), ("layers", 0, -1), ("layers", 129, -1),
+    ("kv_dtype", 3, -1), ("coef_dtype", 7, -1), ("max_deferred", 65, -1),
+    ("ring_extra", 10, -1), ("max_tokens", 0, -1), ("q_heads", 8 * 9, -7),
+    ("rope_theta", 0.5, -1), ("sync", 2, -1),
+])
+def test_create_rejects_bad_configs_before_touching_the_gpu(field, value, code):
+    ik = _lib()
+    c = ik._Cfg()
+    ik.LIB.iskv_config_default(ctypes.byref(c))
+    setattr(c, field, value)
+    h = ctypes.c_void_p(123)
+    assert ik.LIB.iskv_create(ctypes.byref(c), None, ctypes.byref(h)) == code
+    assert h.value is None
+
+
+def test_null_handles():
+    ik = _lib()
+    assert ik.LIB.iskv_destroy(None) == 0
+    assert ik.LIB.iskv_create(None, None, None) == -1
+    T = ctypes.c_int64()
+    assert ik.LIB.iskv_get_counts(None, 0, ctypes.byref(T), None) == -1
+    assert ik.LIB.iskv_status(None) == -1
+    assert ik.LIB.iskv_compress_block(None, 0, 0, None) == -1
