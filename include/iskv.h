@@ -154,7 +154,8 @@ ISKV_API int iskv_decode_attention(iskv_t h, int layer, const void* q, float* ou
 
 /* Rebuild the folded rows of one factor before RoPE: out is
  * [batch, kv_heads, n_c, head_dim] fp32 = C B^T.  `which` is ISKV_WHICH_K or
- * ISKV_WHICH_V.  Errors: STATE if rewrites are pending.                    */
+ * ISKV_WHICH_V.  With n_c = 0 nothing is written and `out` may be NULL.
+ * Errors: STATE if rewrites are pending.                                   */
 ISKV_API int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* stream);
 
 /* Copy out one factor: basis [batch, kv_heads, head_dim, r] fp32 (row i of a

@@ -453,14 +453,15 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
 }
 
 int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* stream) {
-    if (!h || !out || layer < 0 || layer >= h->cfg.layers ||
+    if (!h || layer < 0 || layer >= h->cfg.layers ||
         (which != ISKV_WHICH_K && which != ISKV_WHICH_V))
         return ISKV_ERR_INVALID_ARG;
     if (h->n_pend[layer] > 0) return ISKV_ERR_STATE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const FactorView f = view(h, which);
     const int64_t rows = h->n_c[layer];
-    if (rows == 0) return ISKV_OK;
+    if (rows == 0) return ISKV_OK;   // nothing folded: an empty result
+    if (!out) return ISKV_ERR_INVALID_ARG;
     if (is_device_ptr(out)) {
         CU(launch_reconstruct(f, layer, 0, rows, out, s));
         return ISKV_OK;

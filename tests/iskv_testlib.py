@@ -93,10 +93,17 @@ class Pair:
             if defer_every > 0:
                 self.sync(l)
 
+    def ring_free(self) -> int:
+        """Rows the exact-window ring can still take before a fold."""
+        c = self.cfg
+        cap = c.window + 64 + (c.ring_extra or 64)
+        T, n_c = self.cache.counts(0)
+        return cap - (T - n_c)
+
     def prefill(self, tokens: int, chunk: int = 64, defer_every: int = 0):
         done = 0
         while done < tokens:
-            n = min(chunk, tokens - done)
+            n = min(chunk, tokens - done, self.ring_free())
             self.append(n)
             done += n
             self.fold_ready(defer_every)
@@ -123,7 +130,7 @@ class Pair:
         for which, of in ((ik.WHICH_K, self.ok), (ik.WHICH_V, self.ov)):
             got = self.cache.reconstruct(layer, which).cpu().numpy()
             for (l, b, h) in self.heads:
-                if l == layer and of[(l, b, h)].n_c > 0:
+                if l == layer and of[(l, b, h)].n_c > 0 and got.shape[2] > 0:
                     out[(which, b, h)] = rel_err(got[b, h], of[(l, b, h)].reconstruct())
         return out
 
