@@ -174,6 +174,53 @@ ISKV_API int iskv_status(iskv_t h);
 /* Static string naming a status code.                                     */
 ISKV_API const char* iskv_strerror(int code);
 
+/* ---- decode attention without any device allocation --------------------
+ * The method's pages have no counterpart to this entry point: it is a
+ * packaging of the decode above for callers that cannot call cudaMalloc,
+ * such as a serving engine that owns and plans all of its device memory
+ * (and forbids allocations after start-up), or a latency-critical path that
+ * must avoid cudaMalloc's device-wide synchronization.  Such a caller keeps
+ * the factors in its own buffers (laid out as the cache keeps them) and
+ * passes them here; nothing is allocated and nothing is staged.
+ *
+ * All pointers are device memory, owned by the caller, borrowed for the
+ * stream-ordered duration of the call:
+ *   coef_k, coef_v  [batch*kv_heads][coef_rows][r] in coef_dtype (rows 0..n_c-1
+ *                   are read);
+ *   basis_k, basis_v [batch*kv_heads][head_dim][r] fp32;
+ *   ring_k, ring_v  [batch*kv_heads][ring_rows][head_dim] in kv_dtype, pre-RoPE;
+ *                   exact row j (n_c <= j < T) sits at slot j % ring_rows;
+ *   rope            [T][head_dim/2] (cos, sin) float pairs of j * theta^(-2i/d),
+ *                   or NULL for no RoPE;
+ *   q [batch][q_heads][head_dim] kv_dtype, out [batch][q_heads][head_dim] fp32.
+ * The split-K partial results live in a library-owned device array of 4 MiB
+ * (2^20 floats), present on every GPU that loads the library until the
+ * process exits; a call needs batch * q_heads * (2 + rank_v + head_dim)
+ * floats per split and is rejected with ISKV_ERR_CAPACITY when even one split
+ * does not fit.  The first call on a device looks up that array's device
+ * address (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  Calls share the array: calls that overlap on the GPU race and
+ * must be serialized by the caller.  Errors: INVALID_ARG (null or host
+ * pointer, inconsistent sizes), UNSUPPORTED (shape), CAPACITY, CUDA.       */
+typedef struct {
+    int32_t batch, kv_heads, q_heads, head_dim, rank_k, rank_v;
+    int32_t kv_dtype, coef_dtype;
+    int64_t T;            /* tokens, >= 1                                   */
+    int64_t n_c;          /* folded rows, a multiple of 64, <= T            */
+    int64_t coef_rows;    /* row capacity per head of coef_k / coef_v       */
+    int64_t ring_rows;    /* row capacity per head of ring_k / ring_v       */
+    const void* coef_k;
+    const float* basis_k;
+    const void* coef_v;
+    const float* basis_v;
+    const void* ring_k;
+    const void* ring_v;
+    const float* rope;
+} iskv_decode_operands;
+
+ISKV_API int iskv_decode_attention_noalloc(const iskv_decode_operands* ops, const void* q,
+                                           float* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,7 +16,7 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["Config", "Cache", "IskvError", "lib_path", "LIB", "F32", "BF16",
+__all__ = ["Config", "Cache", "IskvError", "DecodeOperands", "lib_path", "LIB", "F32", "BF16",
            "WHICH_K", "WHICH_V", "ALL_LAYERS", "FOLD_DEFER_SYNC", "EXPORTED"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -59,6 +59,15 @@ class _Cfg(ctypes.Structure):
             "sync", "max_deferred", "jacobi_max_sweeps", "ring_extra")]
 
 
+class DecodeOperands(ctypes.Structure):
+    """Mirror of ``iskv_decode_operands`` (allocation-free decode)."""
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "kv_heads", "q_heads", "head_dim", "rank_k", "rank_v", "kv_dtype",
+        "coef_dtype")] + [(n, ctypes.c_int64) for n in ("T", "n_c", "coef_rows", "ring_rows")] + [
+        (n, ctypes.c_void_p) for n in ("coef_k", "basis_k", "coef_v", "basis_v", "ring_k",
+                                       "ring_v", "rope")]
+
+
 _vp, _i, _i64p = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)
 _SIGS = {
     "iskv_config_default": ([ctypes.POINTER(_Cfg)], _i),
@@ -73,6 +82,7 @@ _SIGS = {
     "iskv_get_counts": ([_vp, _i, _i64p, _i64p], _i),
     "iskv_status": ([_vp], _i),
     "iskv_strerror": ([_i], ctypes.c_char_p),
+    "iskv_decode_attention_noalloc": ([ctypes.POINTER(DecodeOperands), _vp, _vp, _vp], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(LIB, _name)
