@@ -152,29 +152,41 @@ def test_rank_edge_cases(rk, rv):
             assert rel_err(rec[b, h], X) < 1e-5
 
 
-def test_no_sync_ablation_drifts_more():
-    """The no-synchronization ablation must match the oracle's ablation and
-    show clearly larger reconstruction drift than the synchronized cache (on
-    this generator the keys' outlier channels keep their basis fairly stable,
-    so the contrast is ~2x for K and larger for V)."""
+def test_no_sync_ablation():
+    """The no-synchronization ablation keeps every old coefficient row in the
+    basis it was written in.  Reading such rows in a later basis is not
+    basis-invariant: it depends on the sign and rotation choices of each core
+    SVD, which differ between any two correct SVD codes.  So only what is
+    unique is compared with the oracle's ablation: the stored rows' norms (a
+    row is never rewritten, and its norm is that of the block's projection at
+    its fold), the singular values, and the newest block's reconstruction
+    (written in the current basis).  The basis itself must be identical to the
+    synchronized cache's (the fold does not read C), and the drift against the
+    appended rows must be clearly larger than with synchronization."""
+    ik = _ik()
     cfg_s = qwen_cfg(kv_heads=2, q_heads=8, window=128, max_tokens=2048)
     cfg_n = qwen_cfg(kv_heads=2, q_heads=8, window=128, max_tokens=2048, sync=0)
     ps = Pair(cfg_s, "qwen3", seed=6)
     pn = Pair(cfg_n, "qwen3", seed=6)
     ps.prefill(1536)
     pn.prefill(1536)
-    ik = _ik()
     for which, of_s, of_n in ((ik.WHICH_K, ps.ok, pn.ok), (ik.WHICH_V, ps.ov, pn.ov)):
+        bs, ss, _ = ps.cache.factors(0, which)
+        bn, sn, cn = pn.cache.factors(0, which)
+        assert torch.equal(bs, bn) and torch.equal(ss, sn)
         rs = ps.cache.reconstruct(0, which).cpu().double().numpy()
         rn = pn.cache.reconstruct(0, which).cpu().double().numpy()
+        cn = cn.cpu().double().numpy()
         for (l, b, h) in ps.heads:
             X = of_s[(l, b, h)].rows[:rs.shape[2]]
             ds = np.linalg.norm(rs[b, h] - X) / np.linalg.norm(X)
             dn = np.linalg.norm(rn[b, h] - X) / np.linalg.norm(X)
             assert dn > 1.5 * ds, (which, ds, dn)
-            # the ablation itself is compared with the oracle's ablation
             fn = of_n[(l, b, h)]
-            assert rel_err(rn[b, h], fn.C @ fn.B.T) < TOL_F32
+            assert rel_err(np.linalg.norm(cn[b, h], axis=1), np.linalg.norm(fn.C, axis=1)) < TOL_F32
+            assert rel_err(sn[b, h].cpu().numpy(), fn.S) < TOL_F32
+            last = slice(fn.n_c - 64, fn.n_c)
+            assert rel_err(rn[b, h][last], (fn.C @ fn.B.T)[last]) < TOL_F32
 
 
 def test_decode_before_any_fold_and_host_buffers():
