@@ -61,6 +61,8 @@ extern "C" {
                                       results are finite but less accurate) */
 #define ISKV_ERR_NOMEM         -6  /* device allocation failed in create    */
 #define ISKV_ERR_UNSUPPORTED   -7  /* shape outside the compiled kernels    */
+#define ISKV_ERR_DEVICE_TIMEOUT -8 /* a bounded device-side wait gave up (sticky;
+                                      the results of that call are incomplete) */
 
 /* ---- element types ----------------------------------------------------- */
 #define ISKV_F32   0
@@ -167,8 +169,9 @@ ISKV_API int iskv_get_factors(iskv_t h, int layer, int which, float* basis, floa
 /* Host counters of `layer`: tokens appended and tokens folded.             */
 ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
 
-/* Synchronize the cache's work and return its sticky device status:
- * ISKV_OK, ISKV_ERR_NOCONVERGE or ISKV_ERR_CUDA.  Clears nothing.          */
+/* Synchronize the device and return the cache's sticky device status:
+ * ISKV_OK, ISKV_ERR_DEVICE_TIMEOUT, ISKV_ERR_NOCONVERGE or ISKV_ERR_CUDA.
+ * Clears nothing.                                                          */
 ISKV_API int iskv_status(iskv_t h);
 
 /* Static string naming a status code.                                     */

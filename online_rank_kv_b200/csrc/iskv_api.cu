@@ -9,11 +9,13 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
 
 #include "iskv_internal.cuh"
+#include "tc_util.cuh"
 
 using namespace iskv;
 
@@ -47,6 +49,8 @@ struct iskv_cache {
     float* stage_out = nullptr;   // host-output staging
     size_t stage_out_bytes = 0;
     int max_splits = 256;
+    bool use_tc = true;           // tensor-core paths for bf16 coefficients
+    int sms = 148;
     // host counters
     std::vector<int64_t> T, n_c;
     std::vector<int> n_pend;
@@ -55,6 +59,7 @@ struct iskv_cache {
 namespace {
 
 constexpr size_t kStageBytes = 16u << 20;
+constexpr bool kDecodeTcDefault = false;
 
 bool is_device_ptr(const void* p) {
     cudaPointerAttributes at;
@@ -99,6 +104,7 @@ FactorView view(const iskv_cache* h, int which) {
     f.ring = K ? h->ring_k : h->ring_v;
     f.r = K ? h->cfg.rank_k : h->cfg.rank_v;
     f.coef_bf16 = h->cfg.coef_dtype == ISKV_BF16;
+    f.coef_blocked = f.coef_bf16;   // bf16 rows live in 8x8 core-matrix blocks
     f.kv_bf16 = h->cfg.kv_dtype == ISKV_BF16;
     f.n_max = h->n_max;
     f.cap = h->cap;
@@ -168,7 +174,10 @@ int run_resync(iskv_cache* h, const std::vector<int>& layers, const std::vector<
     for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) {
         FactorView f = view(h, which);
         if (chained) CU(launch_compose(f, rl, s));
-        CU(launch_resync(f, rl, s));
+        if (f.coef_blocked)
+            CU(launch_resync_tc(f, rl, h->status, s));
+        else
+            CU(launch_resync(f, rl, s));
     }
     return ISKV_OK;
 }
@@ -225,6 +234,12 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     h->D = c.max_deferred > 0 ? c.max_deferred : 1;
     h->kv_bytes = c.kv_dtype == ISKV_BF16 ? 2 : 4;
     h->coef_bytes = c.coef_dtype == ISKV_BF16 ? 2 : 4;
+    {
+        // tensor-core decode over folded rows: on unless ISKV_TENSOR_CORES=0
+        const char* env = std::getenv("ISKV_TENSOR_CORES");
+        h->use_tc = kDecodeTcDefault ? !(env && env[0] == '0') : (env && env[0] == '1');
+        cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+    }
     h->T.assign(c.layers, 0);
     h->n_c.assign(c.layers, 0);
     h->n_pend.assign(c.layers, 0);
@@ -254,13 +269,15 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     rc = rc ? rc : dalloc(&h->stage_in, h->stage_in_bytes);
     rc = rc ? rc : dalloc(&h->stage_out, h->stage_out_bytes);
     if (rc == ISKV_OK && c.use_rope) {
-        rc = dalloc(&h->rope, (size_t)c.max_tokens * (d / 2) * sizeof(float2));
+        // at least 128 positions: the tensor-core decode reads the in-tile offsets 0..127
+        const int64_t npos = c.max_tokens > 128 ? c.max_tokens : 128;
+        rc = dalloc(&h->rope, (size_t)npos * (d / 2) * sizeof(float2));
         if (rc == ISKV_OK) {
             // cos/sin of pos * theta^(-2i/d), evaluated in double precision
-            std::vector<float2> tab((size_t)c.max_tokens * (d / 2));
+            std::vector<float2> tab((size_t)npos * (d / 2));
             std::vector<double> inv(d / 2);
             for (size_t i = 0; i < d / 2; ++i) inv[i] = std::pow(c.rope_theta, -2.0 * (double)i / (double)d);
-            for (int64_t p = 0; p < c.max_tokens; ++p)
+            for (int64_t p = 0; p < npos; ++p)
                 for (size_t i = 0; i < d / 2; ++i) {
                     const double ang = (double)p * inv[i];
                     tab[p * (d / 2) + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
@@ -432,9 +449,61 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.T = h->T[layer];
     a.n_c = h->n_c[layer];
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
+    const int sms = h->sms;
+    if (h->use_tc && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 && a.n_c > 0) {
+        // folded rows: persistent tensor-core kernel, one CTA per SM over the
+        // flattened (head, 128-token tile) space; exact rows: extra splits
+        DecodeTcArgs t{};
+        t.K = a.K;
+        t.V = a.V;
+        t.q = qd;
+        t.partial = h->partial;
+        t.rope = a.rope;
+        t.status = h->status;
+        t.layer = layer;
+        t.B = c.batch;
+        t.Hkv = c.kv_heads;
+        t.Hq = c.q_heads;
+        t.g = a.g;
+        t.n_c = a.n_c;
+        t.scale = a.scale;
+        t.tiles_per_head = (int)((a.n_c + 127) / 128);
+        t.total_tiles = (int64_t)h->BH * t.tiles_per_head;
+        int64_t ncta = std::min<int64_t>(sms, t.total_tiles);
+        t.tiles_per_cta = (int)((t.total_tiles + ncta - 1) / ncta);
+        t.ncta = (int)((t.total_tiles + t.tiles_per_cta - 1) / t.tiles_per_cta);
+        int slots_c = 1;
+        for (int hh = 0; hh < h->BH; ++hh) {
+            const int64_t first = ((int64_t)hh * t.tiles_per_head) / t.tiles_per_cta;
+            const int64_t last = ((int64_t)(hh + 1) * t.tiles_per_head - 1) / t.tiles_per_cta;
+            slots_c = std::max<int>(slots_c, (int)(last - first + 1));
+        }
+        t.slots_c = slots_c;
+        t.stages = 4;
+        while (t.stages > 2 && decode_tc_smem_bytes(c.rank_k, c.rank_v, t.stages) > 227 * 1024) --t.stages;
+        const int64_t n_w = a.T - a.n_c;
+        int64_t sw = 0, tps_w = 64;
+        if (n_w > 0) {
+            sw = std::min<int64_t>((n_w + 63) / 64, std::max<int64_t>(1, (2 * sms + h->BH - 1) / h->BH));
+            tps_w = ((n_w + sw - 1) / sw + 63) / 64 * 64;
+            sw = (n_w + tps_w - 1) / tps_w;
+        }
+        if (slots_c + sw > h->max_splits) return ISKV_ERR_UNSUPPORTED;
+        t.splits_total = (int)(slots_c + sw);
+        CU(launch_decode_tc(t, s));
+        a.splits_total = t.splits_total;
+        if (sw > 0) {
+            a.j_begin = a.n_c;
+            a.split_base = slots_c;
+            a.splits = (int)sw;
+            a.tokens_per_split = tps_w;
+            CU(launch_decode(a, s));
+        }
+        CU(launch_combine(a, od, s));
+        if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
+        return ISKV_OK;
+    }
     // split the token axis so that the grid covers the GPU several times
-    int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
     const int64_t want = (int64_t)4 * sms;
     int64_t splits = (want + h->BH - 1) / h->BH;
     const int64_t max_by_tokens = (a.T + 63) / 64;
@@ -494,10 +563,20 @@ int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
         CU(cudaMemcpyAsync(sigma, f.sigma + (size_t)layer * heads * r, heads * r * sizeof(float),
                            cudaMemcpyDefault, s));
     if (coef && h->n_c[layer] > 0) {
+        const int64_t rows = h->n_c[layer];
         const size_t rb = (size_t)r * h->coef_bytes;
-        const char* src = reinterpret_cast<const char*>(f.coef) + (size_t)layer * heads * h->n_max * rb;
-        CU(cudaMemcpy2DAsync(coef, h->n_c[layer] * rb, src, h->n_max * rb, h->n_c[layer] * rb, heads,
-                             cudaMemcpyDefault, s));
+        if (is_device_ptr(coef)) {
+            CU(launch_copy_coef(f, layer, 0, rows, coef, s));
+        } else {
+            int64_t chunk = (int64_t)(h->stage_out_bytes / (rb * heads));
+            if (chunk < 1) return ISKV_ERR_UNSUPPORTED;
+            for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+                const int64_t n = std::min(chunk, rows - r0);
+                CU(launch_copy_coef(f, layer, r0, n, h->stage_out, s));
+                CU(cudaMemcpy2DAsync(reinterpret_cast<char*>(coef) + r0 * rb, rows * rb, h->stage_out,
+                                     n * rb, n * rb, heads, cudaMemcpyDefault, s));
+            }
+        }
     }
     return ISKV_OK;
 }
@@ -515,6 +594,7 @@ int iskv_status(iskv_t h) {
     int st = 0;
     if (cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return ISKV_ERR_CUDA;
+    if (st & tc::kStatusTimeout) return ISKV_ERR_DEVICE_TIMEOUT;
     if (st & kStatusNoConverge) return ISKV_ERR_NOCONVERGE;
     return ISKV_OK;
 }
@@ -529,6 +609,7 @@ const char* iskv_strerror(int code) {
         case ISKV_ERR_NOCONVERGE: return "core SVD reached its sweep limit";
         case ISKV_ERR_NOMEM: return "device allocation failed";
         case ISKV_ERR_UNSUPPORTED: return "shape not supported by the compiled kernels";
+        case ISKV_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up; that call's results are incomplete";
         default: return "unknown status";
     }
 }

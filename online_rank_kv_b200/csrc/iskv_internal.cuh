@@ -44,6 +44,16 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Element offset of coefficient (row, c) inside one head's coefficient
+// array.  Row-major, or (the cache's bf16 layout) 8-row x 8-column core
+// matrices of 16 bytes per row, 8-row groups outermost: a tile of whole
+// 8-row groups is contiguous and lands in shared memory, by one bulk copy,
+// in the layout the tensor cores read without swizzling.
+__host__ __device__ __forceinline__ int64_t coef_index(int blocked, int r, int64_t row, int c) {
+    return blocked ? ((row >> 3) * (r >> 3) + (c >> 3)) * 64 + (row & 7) * 8 + (c & 7)
+                   : row * r + c;
+}
+
 // ---------------------------------------------------------------------------
 // Launch descriptors (passed by value; sized well under the 4 KB limit).
 // ---------------------------------------------------------------------------
@@ -53,13 +63,14 @@ __device__ __forceinline__ float warp_max(float v) {
 struct FactorView {
     void* coef;          // [L][BH][n_max][r], coef dtype
     float* basis;        // [L][BH][d][r]
-    __nv_bfloat16* bsplit;  // [L][BH][2][d][r]: bf16 hi and lo parts of basis
+    __nv_bfloat16* bsplit;  // [L][BH][2][d x r blocked 8x8]: bf16 hi and lo parts of basis
     float* sigma;        // [L][BH][r]
     float* pend;         // [L][BH][D][r*r]: W_r[0:r,:] of postponed folds
     int* seg_rows;       // [L][D]: n_c before each postponed fold
     const void* ring;    // [L][BH][cap][d], kv dtype (exact rows)
     int r;
     int coef_bf16;       // 1: coef stored as bf16
+    int coef_blocked;    // 1: coef rows in 8x8 core-matrix blocks (see coef_index)
     int kv_bf16;         // 1: ring stored as bf16
     int64_t n_max;       // coefficient rows per head
     int64_t cap;         // ring rows per head
@@ -92,6 +103,29 @@ struct DecodeArgs {
     int splits;
     int64_t tokens_per_split;
     float scale;                 // 1/sqrt(d)
+    // token range and partial slots of this launch (0 = [0, T), slots 0..splits-1)
+    int64_t j_begin;             // first token of split 0
+    int split_base;              // partial slot of split 0
+    int splits_total;            // partial slots per query head (0: splits)
+};
+
+// Tensor-core decode over the folded rows (bf16 blocked coefficients).
+struct DecodeTcArgs {
+    FactorView K, V;
+    const void* q;               // [B][Hq][d] bf16
+    float* partial;              // [B][Hq][splits_total][2 + r_V + d]
+    const float2* rope;          // [>= 128 positions][d/2], or null
+    int* status;
+    int layer, B, Hkv, Hq, g;
+    int64_t n_c;
+    int tiles_per_head;          // ceil(n_c / 128)
+    int64_t total_tiles;         // BH * tiles_per_head
+    int tiles_per_cta;
+    int ncta;
+    int slots_c;                 // compressed partial slots per query head
+    int splits_total;
+    int stages;                  // shared-memory pipeline depth (2..4)
+    float scale;
 };
 
 // ---------------------------------------------------------------------------
@@ -108,6 +142,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_reconstruct(const FactorView& f, int layer, int64_t row0, int64_t rows,
                                float* out, cudaStream_t s);
+cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64_t rows, void* dst,
+                             cudaStream_t s);
+cudaError_t launch_resync_tc(const FactorView& f, const ResyncLaunch& rl, int* status,
+                             cudaStream_t s);
+cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
+size_t decode_tc_smem_bytes(int rK, int rV, int ns);
 
 size_t fold_smem_bytes(int r);
 

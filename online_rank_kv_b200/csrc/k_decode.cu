@@ -53,9 +53,11 @@ decode_kernel(DecodeArgs a) {
     const int BH = a.K.BH;
     const int bh = b * a.Hkv + kvh;
     const int64_t hidx = (int64_t)a.layer * BH + bh;
-    const int64_t j0 = (int64_t)split * a.tokens_per_split;
+    const int64_t j0 = a.j_begin + (int64_t)split * a.tokens_per_split;
     int64_t j1 = j0 + a.tokens_per_split;
     if (j1 > a.T) j1 = a.T;
+    const int slots = a.splits_total > 0 ? a.splits_total : a.splits;
+    const int slot = a.split_base + split;
 
     const Smem L = smem_layout(rK, rV, g);
     extern __shared__ float sm[];
@@ -99,9 +101,11 @@ decode_kernel(DecodeArgs a) {
 
         if (comp) {
             for (int e = tid; e < kTile * rK; e += kThreads)
-                sCk[e] = (e / rK < nt) ? to_f32(Ck[j * rK + e]) : 0.f;
+                sCk[e] = (e / rK < nt) ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, j + e / rK, e % rK)])
+                                       : 0.f;
             for (int e = tid; e < kTile * rV; e += kThreads)
-                sCv[e] = (e / rV < nt) ? to_f32(Cv[j * rV + e]) : 0.f;
+                sCv[e] = (e / rV < nt) ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, j + e / rV, e % rV)])
+                                       : 0.f;
             __syncthreads();
             for (int e = tid; e < kTile * d; e += kThreads) {
                 const int t = e / d, i = e % d;
@@ -191,12 +195,12 @@ decode_kernel(DecodeArgs a) {
         const int e = tid + u * kThreads;
         if (e < n_acc) {
             const int h = e / width, col = e % width;
-            float* P = a.partial + (((int64_t)b * a.Hq + kvh * g + h) * a.splits + split) * stride;
+            float* P = a.partial + (((int64_t)b * a.Hq + kvh * g + h) * slots + slot) * stride;
             P[2 + col] = acc[u];
         }
     }
     if (tid < g) {
-        float* P = a.partial + (((int64_t)b * a.Hq + kvh * g + tid) * a.splits + split) * stride;
+        float* P = a.partial + (((int64_t)b * a.Hq + kvh * g + tid) * slots + slot) * stride;
         P[0] = sMax[tid];
         P[1] = sSum[tid];
     }
@@ -209,26 +213,30 @@ combine_kernel(DecodeArgs a, float* out) {
     const int kvh = qh / a.g;
     const int64_t hidx = (int64_t)a.layer * a.V.BH + b * a.Hkv + kvh;
     const int stride = 2 + rV + d;
-    const float* P = a.partial + ((int64_t)b * a.Hq + qh) * a.splits * stride;
+    const int slots = a.splits_total > 0 ? a.splits_total : a.splits;
+    const float* P = a.partial + ((int64_t)b * a.Hq + qh) * slots * stride;
     __shared__ float sW[256];
     __shared__ float sAcc[kHeadDim];
     float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, P[s * stride]);
+    for (int s = 0; s < slots; ++s) M = fmaxf(M, P[s * stride]);
     float Ls = 0.f;
-    for (int s = tid; s < a.splits; s += blockDim.x) {
+    for (int s = tid; s < slots; s += blockDim.x) {
         const float ms = P[s * stride];
-        const float w = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-        sW[s] = w;
+        sW[s] = (ms == -INFINITY) ? 0.f : __expf(ms - M);
     }
     __syncthreads();
-    for (int s = 0; s < a.splits; ++s) Ls = fmaf(sW[s], P[s * stride + 1], Ls);
+    // empty slots (weight 0) are skipped: their other entries are not written
+    for (int s = 0; s < slots; ++s)
+        if (sW[s] != 0.f) Ls = fmaf(sW[s], P[s * stride + 1], Ls);
     if (tid < rV) {
         float v = 0.f;
-        for (int s = 0; s < a.splits; ++s) v = fmaf(sW[s], P[s * stride + 2 + tid], v);
+        for (int s = 0; s < slots; ++s)
+            if (sW[s] != 0.f) v = fmaf(sW[s], P[s * stride + 2 + tid], v);
         sAcc[tid] = v;
     }
     float vd = 0.f;
-    for (int s = 0; s < a.splits; ++s) vd = fmaf(sW[s], P[s * stride + 2 + rV + tid], vd);
+    for (int s = 0; s < slots; ++s)
+        if (sW[s] != 0.f) vd = fmaf(sW[s], P[s * stride + 2 + rV + tid], vd);
     __syncthreads();
     const float* Bv = a.V.basis + hidx * d * rV;
     float o = vd;

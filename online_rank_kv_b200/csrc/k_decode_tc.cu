@@ -1,0 +1,492 @@
+// Decode attention over the folded (compressed) rows on the 5th-generation
+// tensor cores, for bf16-stored coefficients.
+//
+// Method: "iS-KV -- Basis-synchronized online low-rank KV compression -- What
+// does it mean?" (Jargon: Pre-RoPE keys -- folded keys are rebuilt before
+// RoPE and rotated when read) and the ASKV design report (Design
+// requirements: values are never rebuilt on the decode path).  For query
+// head h of KV head h/g and folded token j < n_c:
+//   k_j = C_K[j] B_K^T,  s_j = q_h . RoPE(k_j, j) / sqrt(d),
+//   partial softmax (m, l) and acc_h = sum_j p_j C_V[j]   (r_V wide);
+// the exact window and the split merge are done by decode_kernel and
+// combine_kernel (k_decode.cu), which applies B_V^T once per query head.
+//
+// Persistent design, one CTA per SM, the flattened (head, 128-token tile)
+// space cut into equal contiguous ranges; per CTA 10 warps:
+//   warp 0  producer: 1-D bulk copies (TMA engine) of the C_K and C_V tiles
+//           (contiguous in the blocked layout) into an NS-stage ring, and of
+//           the bf16 hi/lo basis of each head it visits;
+//   warp 1  MMA issuer: K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens,
+//           N=128 dims, fp32 accumulator in TMEM (two buffers);
+//   warps 2-9 epilogue, one token row per pair of threads (warps w and w+4
+//           reach the same TMEM lanes); each thread of the pair owns half of
+//           the 64 rotation pairs and half of the query heads:
+//           * rotate its half row of K^ by R_t (t = row within the tile; the
+//             thread's cos/sin(t w_i) live in registers) and write it back to
+//             TMEM rounded to tf32; the query is pre-rotated per tile by
+//             R_{j0}^T (j0 = tile start), so q'.(R_t k) = q.(R_{j0+t} k);
+//           * scores S = K_rot q'^T on the tensor cores (kind::tf32, A from
+//             TMEM, q' as tf32 hi+lo parts in the N dimension);
+//           * online softmax per query head (tile max over the 128 rows);
+//           * p as bf16 hi+lo parts -> O = C_V^T P (kind::f16, C_V tile read
+//             MN-major in place), accumulated with the running rescale.
+// Every mbarrier wait is bounded; on timeout the CTA records
+// ISKV status bit 2, stops, drains its copies and frees its TMEM.
+#include "iskv_internal.cuh"
+#include "tc_util.cuh"
+
+namespace iskv {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kTile = 128;
+constexpr int kThreads = 320;
+constexpr int kEpi = 256;        // epilogue threads (warps 2-9)
+constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
+constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
+constexpr int kBufCols = 160;    // per TMEM buffer: K^ 128 | S 16 | O 16
+constexpr uint32_t kTmemCols = 512;
+
+struct __align__(8) Bars {
+    uint64_t full[4], empty[4];
+    uint64_t bk_full[2], bk_empty[2];
+    uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
+};
+
+struct SmemPlan {
+    uint32_t bk, stage, stage_k, qb, pb, total;
+};
+
+__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns) {
+    SmemPlan p;
+    uint32_t off = 1024;                                        // barriers, scratch
+    p.bk = off;                off += 2 * (2 * kTile * rK * 2);  // two heads x (hi, lo)
+    p.stage_k = (uint32_t)kTile * rK * 2;
+    p.stage = off;             off += ns * (p.stage_k + kTile * rV * 2 + 1024);
+    p.qb = off;                off += 2 * (kQN * kTile * 4);
+    p.pb = off;                off += 2 * (kPN * kTile * 2);
+    p.total = off;
+    return p;
+}
+
+// v[idx] for a runtime idx without forcing v into local memory
+__device__ __forceinline__ float pick16(const uint32_t (&v)[16], int idx) {
+    float r = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) r = (k == idx) ? __uint_as_float(v[k]) : r;
+    return r;
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// offsets of the tf32 (K-major, 8 x 4 core matrices) and bf16 (8 x 8) B operands
+__device__ __forceinline__ int qb_off(int n, int k) {
+    return ((n >> 3) * (kTile / 4) + (k >> 2)) * 32 + (n & 7) * 4 + (k & 3);
+}
+__device__ __forceinline__ int pb_off(int n, int k) {
+    return ((n >> 3) * (kTile / 8) + (k >> 3)) * 64 + (n & 7) * 8 + (k & 7);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+decode_tc_kernel(DecodeTcArgs a) {
+    const int cta = blockIdx.x;
+    const int64_t f0 = (int64_t)cta * a.tiles_per_cta;
+    int64_t f1 = f0 + a.tiles_per_cta;
+    if (f1 > a.total_tiles) f1 = a.total_tiles;
+    if (f0 >= f1) return;
+    const int ntiles = (int)(f1 - f0);
+    const int tph = a.tiles_per_head;
+    const int rK = a.K.r, rV = a.V.r, g = a.g, ns = a.stages;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int d = kHeadDim;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    Bars* bars = reinterpret_cast<Bars*>(smem);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + sizeof(Bars));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 4);
+    float* red = reinterpret_cast<float*>(smem + 512);          // [2][4][8]: tile max, l sums
+    const SmemPlan P = plan_smem(rK, rV, ns);
+    float* sq = reinterpret_cast<float*>(smem + P.total);       // queries of the head, g x d fp32
+    uint8_t* bk = smem + P.bk;
+    uint8_t* stage = smem + P.stage;
+    uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
+    __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
+    const uint32_t stage_bytes = P.stage_k + kTile * rV * 2 + 1024;
+    const uint32_t bk_bytes = 2 * kTile * rK * 2;
+
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&bars->full[i], 1);
+            mbar_init(&bars->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->bk_full[i], 1);
+            mbar_init(&bars->bk_empty[i], 1);
+            mbar_init(&bars->kh_full[i], 1);
+            mbar_init(&bars->kfree[i], 1);
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->o_full[i], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // zero the padding rows (n >= 2g) of the q' and p operands once
+    for (int e = tid; e < 2 * kQN * kTile; e += kThreads) {
+        const int buf = e / (kQN * kTile), w = e % (kQN * kTile);
+        const int n = w / kTile, k = w % kTile;
+        if (n >= 2 * g) qb[buf * kQN * kTile + qb_off(n, k)] = 0u;
+    }
+    for (int e = tid; e < 2 * kPN * kTile; e += kThreads) {
+        const int buf = e / (kPN * kTile), w = e % (kPN * kTile);
+        const int n = w / kTile, k = w % kTile;
+        if (n >= 2 * g) pb[buf * kPN * kTile + pb_off(n, k)] = __float2bfloat16_rn(0.f);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const long long deadline = clock64() + kWaitCycles;
+    const int BH = a.K.BH;
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusTimeout);
+    };
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            int hs = -1, prev = -1, issued = 0;
+            for (int n = 0; n < ntiles && !*abort_flag; ++n) {
+                const int64_t fi = f0 + n;
+                const int head = (int)(fi / tph), tile = (int)(fi % tph);
+                const int64_t hidx = (int64_t)a.layer * BH + head;
+                if (head != prev) {
+                    ++hs;
+                    const int hb = hs & 1;
+                    if (hs >= 2 && !mbar_wait(&bars->bk_empty[hb], ((hs - 2) >> 1) & 1, deadline)) {
+                        fail();
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars->bk_full[hb], bk_bytes);
+                    bulk_g2s(bk + hb * bk_bytes, a.K.bsplit + hidx * 2 * d * rK, bk_bytes, &bars->bk_full[hb]);
+                    prev = head;
+                }
+                const int st = n % ns;
+                if (n >= ns && !mbar_wait(&bars->empty[st], ((n / ns) - 1) & 1, deadline)) {
+                    fail();
+                    break;
+                }
+                uint8_t* sk = stage + st * stage_bytes;
+                const __nv_bfloat16* gk = reinterpret_cast<const __nv_bfloat16*>(a.K.coef) +
+                                          hidx * a.K.n_max * rK + (int64_t)tile * kTile * rK;
+                const __nv_bfloat16* gv = reinterpret_cast<const __nv_bfloat16*>(a.V.coef) +
+                                          hidx * a.V.n_max * rV + (int64_t)tile * kTile * rV;
+                mbar_arrive_expect_tx(&bars->full[st], P.stage_k + kTile * rV * 2);
+                bulk_g2s(sk, gk, P.stage_k, &bars->full[st]);
+                bulk_g2s(sk + P.stage_k, gv, kTile * rV * 2, &bars->full[st]);
+                issued = n + 1;
+            }
+            if (*abort_flag) {
+                // drain the copies this thread issued (bounded)
+                for (int n = issued - ns > 0 ? issued - ns : 0; n < issued; ++n)
+                    mbar_wait(&bars->full[n % ns], (n / ns) & 1, deadline + kWaitCycles);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- reconstruction MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f32acc(1, kTile, d, 0, 0);
+            const uint32_t sbo = (uint32_t)(rK / 8) * 128;
+            int hs = -1, prev = -1;
+            for (int n = 0; n < ntiles && !*abort_flag; ++n) {
+                const int64_t fi = f0 + n;
+                const int head = (int)(fi / tph);
+                if (head != prev) {
+                    ++hs;
+                    if (!mbar_wait(&bars->bk_full[hs & 1], (hs >> 1) & 1, deadline)) {
+                        fail();
+                        break;
+                    }
+                    prev = head;
+                }
+                const int st = n % ns, b = n & 1;
+                if (!mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) {
+                    fail();
+                    break;
+                }
+                if (n >= 2 && !mbar_wait(&bars->kfree[b], ((n >> 1) - 1) & 1, deadline)) {
+                    fail();
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(stage + st * stage_bytes);
+                const uint32_t b0 = smem_u32(bk + (hs & 1) * bk_bytes);
+                const uint32_t dk = tmem + b * kBufCols;
+                for (int ks = 0; ks < rK / 16; ++ks)
+                    for (int part = 0; part < 2; ++part) {
+                        const uint64_t ad = desc_noswizzle(a0 + ks * 256, 128, sbo);
+                        const uint64_t bd = desc_noswizzle(b0 + part * (kTile * rK * 2) + ks * 256, 128, sbo);
+                        mma_f16_ss(dk, ad, bd, idesc, (ks | part) != 0);
+                    }
+                mma_commit(&bars->kh_full[b]);
+                const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
+                if (seg_end) mma_commit(&bars->bk_empty[hs & 1]);
+            }
+        }
+    } else {
+        // ---------------- epilogue: 256 threads, two per token row ----------------
+        const int ept = tid - 64;                 // 0..255
+        const int sp = warp & 3;                  // TMEM sub-partition of this warp
+        const int half = ept >> 7;                // which half of the pairs / heads
+        const int row = sp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+        const int i0 = half * 32;                 // first rotation pair of this thread
+        const int gh = (g + 1) / 2;               // heads of half 0
+        const int h_lo = half ? gh : 0, h_hi = half ? g : gh;
+        float cs_c[32], cs_s[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            float2 v = make_float2(1.f, 0.f);
+            if (a.rope) v = a.rope[row * 64 + i0 + u];
+            cs_c[u] = v.x;
+            cs_s[u] = v.y;
+        }
+        const int MV = rV <= 64 ? 64 : 128;
+        const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
+        const bool acc_ok = c_acc >= 0 && c_acc < rV;
+        const uint32_t idesc_s = idesc_f32acc(2, kTile, kQN, 0, 0);
+        const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 0);
+        const uint32_t sbo_q = (kTile / 4) * 128;
+        const uint32_t sbo_p = (kTile / 8) * 128;
+        const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
+        constexpr int kH = kMaxGroup / 2;         // heads per thread at most
+
+        float m_run[kH], l_thr[kH], acc[kH], alpha[kH];
+        bool have_prev = false;
+        int cur_head = -1;
+        for (int n = 0; n < ntiles; ++n) {
+            if (*abort_flag) break;
+            const int64_t fi = f0 + n;
+            const int head = (int)(fi / tph), tile = (int)(fi % tph);
+            const int b = n & 1, st = n % ns;
+            const uint32_t kh = tmem + b * kBufCols;
+            if (head != cur_head) {
+                // new head segment: its queries, fresh softmax state
+                const int bq = head / a.Hkv, kvh = head % a.Hkv;
+                const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                          ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
+                epi_sync();
+                for (int e = ept; e < g * d; e += kEpi) sq[e] = __bfloat162float(qg[e]);
+#pragma unroll
+                for (int u = 0; u < kH; ++u) {
+                    m_run[u] = -INFINITY;
+                    l_thr[u] = 0.f;
+                    acc[u] = 0.f;
+                    alpha[u] = 0.f;
+                }
+                have_prev = false;
+                cur_head = head;
+                epi_sync();
+            }
+            const int64_t j0 = (int64_t)tile * kTile;
+            const int valid = (int)((a.n_c - j0) < kTile ? (a.n_c - j0) : kTile);
+            // q' = R_{j0}^T q for this tile, tf32 hi / lo parts as the B operand
+            uint32_t* qbb = qb + b * kQN * kTile;
+            for (int item = ept; item < g * 64; item += kEpi) {
+                const int h = item >> 6, i = item & 63;
+                float c0 = 1.f, s0 = 0.f;
+                if (a.rope) {
+                    const float2 v = a.rope[j0 * 64 + i];
+                    c0 = v.x;
+                    s0 = v.y;
+                }
+                const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
+                const float y1 = fmaf(c0, x1, s0 * x2);
+                const float y2 = fmaf(c0, x2, -s0 * x1);
+                const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
+                qbb[qb_off(h, i)] = t1;
+                qbb[qb_off(h, i + 64)] = t2;
+                qbb[qb_off(g + h, i)] = to_tf32(y1 - __uint_as_float(t1));
+                qbb[qb_off(g + h, i + 64)] = to_tf32(y2 - __uint_as_float(t2));
+            }
+            fence_async_smem();
+            // rotate this thread's half row of K^ and store it back as tf32
+            if (!mbar_wait(&bars->kh_full[b], (n >> 1) & 1, deadline)) fail();
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 32; c += 16) {
+                uint32_t x1[16], x2[16];
+                tmem_ld16(kh + lane_base + i0 + c, x1);
+                tmem_ld16(kh + lane_base + 64 + i0 + c, x2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const float k1 = __uint_as_float(x1[u]), k2 = __uint_as_float(x2[u]);
+                    const float co = cs_c[c + u], si = cs_s[c + u];
+                    x1[u] = to_tf32(fmaf(k1, co, -k2 * si));
+                    x2[u] = to_tf32(fmaf(k1, si, k2 * co));
+                }
+                tmem_st16(kh + lane_base + i0 + c, x1);
+                tmem_st16(kh + lane_base + 64 + i0 + c, x2);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            epi_sync();
+            if (ept == 0 && !*abort_flag) {
+                tc_fence_after();
+                const uint32_t q0 = smem_u32(qbb);
+                for (int ks = 0; ks < d / 8; ++ks)
+                    mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
+                                idesc_s, ks != 0);
+                mma_commit(&bars->s_full[b]);
+            }
+            // accumulate the previous tile's p^T C_V (its MMA ran meanwhile)
+            if (have_prev) {
+                const int pbuf = (n - 1) & 1;
+                if (!mbar_wait(&bars->o_full[pbuf], ((n - 1) >> 1) & 1, deadline)) fail();
+                tc_fence_after();
+                uint32_t o[16];
+                tmem_ld16(tmem + pbuf * kBufCols + 144 + lane_base, o);
+                tmem_wait_ld();
+                if (acc_ok) {
+#pragma unroll
+                    for (int u = 0; u < kH; ++u) {
+                        const int h = h_lo + u;
+                        if (h < h_hi)
+                            acc[u] = fmaf(acc[u], alpha[u], pick16(o, h) + pick16(o, g + h));
+                    }
+                }
+            }
+            // scores of this thread's heads, online softmax
+            if (!mbar_wait(&bars->s_full[b], (n >> 1) & 1, deadline)) fail();
+            tc_fence_after();
+            uint32_t sv[16];
+            tmem_ld16(kh + 128 + lane_base, sv);
+            tmem_wait_ld();
+            float sc[kH];
+#pragma unroll
+            for (int u = 0; u < kH; ++u) {
+                const int h = h_lo + u;
+                sc[u] = -INFINITY;
+                if (h < h_hi && row < valid)
+                    sc[u] = (pick16(sv, h) + pick16(sv, g + h)) * a.scale;
+                const float wm = warp_max(sc[u]);
+                if (lane == 0 && h < h_hi) red[sp * 8 + h] = wm;
+            }
+            epi_sync();
+            __nv_bfloat16* pbb = pb + b * kPN * kTile;
+#pragma unroll
+            for (int u = 0; u < kH; ++u) {
+                const int h = h_lo + u;
+                if (h >= h_hi) break;
+                const float tmax = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
+                const float m_new = fmaxf(m_run[u], tmax);
+                const float al = (m_run[u] == -INFINITY) ? 0.f : __expf(m_run[u] - m_new);
+                const float p = (sc[u] == -INFINITY) ? 0.f : __expf(sc[u] - m_new);
+                l_thr[u] = fmaf(l_thr[u], al, p);
+                m_run[u] = m_new;
+                alpha[u] = al;
+                const __nv_bfloat16 ph = __float2bfloat16_rn(p);
+                pbb[pb_off(h, row)] = ph;
+                pbb[pb_off(g + h, row)] = __float2bfloat16_rn(p - __bfloat162float(ph));
+            }
+            fence_async_smem();
+            tc_fence_before();
+            epi_sync();
+            if (ept == 0 && !*abort_flag) {
+                mbar_arrive(&bars->kfree[b]);   // K^/S buffer b may be overwritten
+                tc_fence_after();
+                const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
+                const uint32_t p0 = smem_u32(pbb);
+                for (int ks = 0; ks < kTile / 16; ++ks)
+                    mma_f16_ss(tmem + b * kBufCols + 144,
+                               desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
+                               desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_o, ks != 0);
+                mma_commit(&bars->o_full[b]);
+                mma_commit(&bars->empty[st]);
+            }
+            have_prev = true;
+            const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
+            if (seg_end) {
+                if (!mbar_wait(&bars->o_full[b], (n >> 1) & 1, deadline)) fail();
+                tc_fence_after();
+                uint32_t o[16];
+                tmem_ld16(tmem + b * kBufCols + 144 + lane_base, o);
+                tmem_wait_ld();
+                if (acc_ok) {
+#pragma unroll
+                    for (int u = 0; u < kH; ++u) {
+                        const int h = h_lo + u;
+                        if (h < h_hi)
+                            acc[u] = fmaf(acc[u], alpha[u], pick16(o, h) + pick16(o, g + h));
+                    }
+                }
+                have_prev = false;
+                // l over the 128 rows of each head
+#pragma unroll
+                for (int u = 0; u < kH; ++u) {
+                    const int h = h_lo + u;
+                    const float ws = warp_sum(l_thr[u]);
+                    if (lane == 0 && h < h_hi) red[32 + sp * 8 + h] = ws;
+                }
+                tc_fence_before();
+                epi_sync();
+                const int bq = head / a.Hkv, kvh = head % a.Hkv;
+                const int c_first = (int)(((int64_t)head * tph) / a.tiles_per_cta);
+                const int slot = cta - c_first;
+                const int stride = 2 + rV + d;
+                for (int u = 0; u < kH; ++u) {
+                    const int h = h_lo + u;
+                    if (h >= h_hi) break;
+                    float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
+                    if (acc_ok) Pp[2 + c_acc] = acc[u];
+                    for (int i = ept & 127; i < d; i += 128) Pp[2 + rV + i] = 0.f;
+                    if ((ept & 127) == 0) {
+                        Pp[0] = m_run[u];
+                        Pp[1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
+                    }
+                }
+                // this CTA ends the head: mark the head's unused compressed slots empty
+                if (ept == 0 && f1 >= (int64_t)(head + 1) * tph) {
+                    for (int h = 0; h < g; ++h)
+                        for (int sl = slot + 1; sl < a.slots_c; ++sl) {
+                            float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + sl) * stride;
+                            Pp[0] = -INFINITY;
+                            Pp[1] = 0.f;
+                        }
+                }
+                epi_sync();
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+size_t decode_tc_smem_bytes(int rK, int rV, int ns) {
+    return plan_smem(rK, rV, ns).total + (size_t)kMaxGroup * kHeadDim * 4;
+}
+
+cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s) {
+    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages);
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bytes);
+    if (e != cudaSuccess) return e;
+    decode_tc_kernel<<<a.ncta, kThreads, bytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace iskv

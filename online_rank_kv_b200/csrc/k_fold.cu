@@ -334,10 +334,10 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
     // ---- (d) outputs: S', new coefficient rows, W_top
     float* gSw = f.sigma + hidx * r;
     for (int t = tid; t < r; t += kThreads) gSw[t] = nrm[perm[t]];
-    CoefT* gC = reinterpret_cast<CoefT*>(f.coef) + (hidx * f.n_max + n_c) * r;
+    CoefT* gC = reinterpret_cast<CoefT*>(f.coef) + hidx * f.n_max * r;
     for (int e = tid; e < b * r; e += kThreads) {
         int t = e / r, cc = e % r;
-        gC[(int64_t)t * r + cc] = from_f32<CoefT>(sA[perm[cc] * m + r + t]);
+        gC[coef_index(f.coef_blocked, r, n_c + t, cc)] = from_f32<CoefT>(sA[perm[cc] * m + r + t]);
     }
     float* gW = f.pend + (hidx * f.D + slot) * (int64_t)r * r;
     for (int e = tid; e < r * r; e += kThreads) {
@@ -378,8 +378,9 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
         const float v = fmaf(-0.5f, corr, 1.5f * sBn[e]);
         gBw[e] = v;
         const __nv_bfloat16 h = __float2bfloat16_rn(v);
-        gHi[e] = h;
-        gLo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
+        const int64_t bo = coef_index(1, r, i, cc);
+        gHi[bo] = h;
+        gLo[bo] = __float2bfloat16_rn(v - __bfloat162float(h));
     }
 }
 

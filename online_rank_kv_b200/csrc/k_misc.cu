@@ -17,8 +17,9 @@ __global__ void init_factor_kernel(FactorView f, int layers) {
         const int i = (int)(w / r), j = (int)(w % r);
         const float v = (i == j) ? 1.f : 0.f;
         f.basis[e] = v;
-        f.bsplit[h * 2 * per + w] = __float2bfloat16_rn(v);
-        f.bsplit[h * 2 * per + per + w] = __float2bfloat16_rn(0.f);
+        const int64_t bo = coef_index(1, r, i, j);
+        f.bsplit[h * 2 * per + bo] = __float2bfloat16_rn(v);
+        f.bsplit[h * 2 * per + per + bo] = __float2bfloat16_rn(0.f);
         if (w < r) f.sigma[h * r + w] = 0.f;
     }
 }
@@ -52,11 +53,13 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(FactorView f, int laye
     float* sC = sm + kHeadDim * (r + 1);  // kRecRows x r
     const int64_t hidx = (int64_t)layer * f.BH + bh;
     const float* B = f.basis + hidx * kHeadDim * r;
-    const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + (hidx * f.n_max + row0 + t0) * r;
+    const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + hidx * f.n_max * r;
     const int nt = (int)((rows - t0) < kRecRows ? (rows - t0) : kRecRows);
     for (int e = threadIdx.x; e < kHeadDim * r; e += blockDim.x) sB[(e / r) * (r + 1) + e % r] = B[e];
-    for (int e = threadIdx.x; e < kRecRows * r; e += blockDim.x)
-        sC[e] = (e / r < nt) ? to_f32(C[e]) : 0.f;
+    for (int e = threadIdx.x; e < kRecRows * r; e += blockDim.x) {
+        const int t = e / r, c = e % r;
+        sC[e] = (t < nt) ? to_f32(C[coef_index(f.coef_blocked, r, row0 + t0 + t, c)]) : 0.f;
+    }
     __syncthreads();
     float* o = out + ((int64_t)bh * rows + t0) * kHeadDim;
     for (int e = threadIdx.x; e < nt * kHeadDim; e += blockDim.x) {
@@ -67,7 +70,38 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(FactorView f, int laye
     }
 }
 
+// dst[bh][row][c] (row-major, coefficient dtype) = C[row0 + row][c], any layout.
+template <typename CoefT>
+__global__ void copy_coef_kernel(FactorView f, int layer, int64_t row0, int64_t rows, CoefT* dst) {
+    const int r = f.r;
+    const int64_t total = (int64_t)f.BH * rows * r;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int c = (int)(e % r);
+        const int64_t row = (e / r) % rows;
+        const int64_t bh = e / ((int64_t)r * rows);
+        const int64_t hidx = (int64_t)layer * f.BH + bh;
+        const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + hidx * f.n_max * r;
+        dst[e] = C[coef_index(f.coef_blocked, r, row0 + row, c)];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64_t rows, void* dst,
+                             cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    const int64_t total = (int64_t)f.BH * rows * f.r;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 4736) blocks = 4736;
+    if (f.coef_bf16)
+        copy_coef_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            f, layer, row0, rows, reinterpret_cast<__nv_bfloat16*>(dst));
+    else
+        copy_coef_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(f, layer, row0, rows,
+                                                                 reinterpret_cast<float*>(dst));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s) {
     init_factor_kernel<<<1184, 256, 0, s>>>(f, layers);

@@ -70,15 +70,17 @@ resync_kernel(FactorView f, ResyncLaunch rl) {
     float* sC = sm + r * r;            // rows x r
     const int64_t hidx = (int64_t)layer * f.BH + bh;
     const float* W = f.pend + (hidx * f.D + seg) * (int64_t)r * r;
-    CoefT* C = reinterpret_cast<CoefT*>(f.coef) + (hidx * f.n_max + row0) * r;
+    CoefT* C = reinterpret_cast<CoefT*>(f.coef) + hidx * f.n_max * r;
+    const int bl = f.coef_blocked;
     for (int e = threadIdx.x; e < r * r; e += kResyncThreads) sW[e] = W[e];
-    for (int e = threadIdx.x; e < kResyncRows * r; e += kResyncThreads) sC[e] = to_f32(C[e]);
+    for (int e = threadIdx.x; e < kResyncRows * r; e += kResyncThreads)
+        sC[e] = to_f32(C[coef_index(bl, r, row0 + e / r, e % r)]);
     __syncthreads();
     for (int e = threadIdx.x; e < kResyncRows * r; e += kResyncThreads) {
         const int t = e / r, cc = e % r;
         float acc = 0.f;
         for (int j = 0; j < r; ++j) acc = fmaf(sC[t * r + j], sW[j * r + cc], acc);
-        C[e] = from_f32<CoefT>(acc);
+        C[coef_index(bl, r, row0 + t, cc)] = from_f32<CoefT>(acc);
     }
 }
 
