@@ -59,7 +59,7 @@ struct iskv_cache {
 namespace {
 
 constexpr size_t kStageBytes = 16u << 20;
-constexpr bool kDecodeTcDefault = false;
+constexpr bool kDecodeTcDefault = true;
 
 bool is_device_ptr(const void* p) {
     cudaPointerAttributes at;
@@ -479,8 +479,16 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
             slots_c = std::max<int>(slots_c, (int)(last - first + 1));
         }
         t.slots_c = slots_c;
-        t.stages = 4;
-        while (t.stages > 2 && decode_tc_smem_bytes(c.rank_k, c.rank_v, t.stages) > 227 * 1024) --t.stages;
+        // deepest pipeline that fits: two basis buffers if possible, else one
+        t.stages = 0;
+        for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
+            for (int ns = 4; ns >= 2; --ns)
+                if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk) <= 227 * 1024) {
+                    t.stages = ns;
+                    t.basis_bufs = nbk;
+                    break;
+                }
+        if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
         const int64_t n_w = a.T - a.n_c;
         int64_t sw = 0, tps_w = 64;
         if (n_w > 0) {

@@ -125,6 +125,7 @@ struct DecodeTcArgs {
     int slots_c;                 // compressed partial slots per query head
     int splits_total;
     int stages;                  // shared-memory pipeline depth (2..4)
+    int basis_bufs;              // bf16 basis buffers (1 or 2 heads in flight)
     float scale;
 };
 
@@ -147,7 +148,7 @@ cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64
 cudaError_t launch_resync_tc(const FactorView& f, const ResyncLaunch& rl, int* status,
                              cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
-size_t decode_tc_smem_bytes(int rK, int rV, int ns);
+size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk);
 
 size_t fold_smem_bytes(int r);
 

@@ -59,10 +59,10 @@ struct SmemPlan {
     uint32_t bk, stage, stage_k, qb, pb, total;
 };
 
-__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns) {
+__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk) {
     SmemPlan p;
     uint32_t off = 1024;                                        // barriers, scratch
-    p.bk = off;                off += 2 * (2 * kTile * rK * 2);  // two heads x (hi, lo)
+    p.bk = off;                off += nbk * (2 * kTile * rK * 2);  // nbk heads x (hi, lo)
     p.stage_k = (uint32_t)kTile * rK * 2;
     p.stage = off;             off += ns * (p.stage_k + kTile * rV * 2 + 1024);
     p.qb = off;                off += 2 * (kQN * kTile * 4);
@@ -98,7 +98,7 @@ decode_tc_kernel(DecodeTcArgs a) {
     if (f0 >= f1) return;
     const int ntiles = (int)(f1 - f0);
     const int tph = a.tiles_per_head;
-    const int rK = a.K.r, rV = a.V.r, g = a.g, ns = a.stages;
+    const int rK = a.K.r, rV = a.V.r, g = a.g, ns = a.stages, nbk = a.basis_bufs;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int d = kHeadDim;
 
@@ -106,8 +106,11 @@ decode_tc_kernel(DecodeTcArgs a) {
     Bars* bars = reinterpret_cast<Bars*>(smem);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + sizeof(Bars));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 4);
+    // the epilogue's copy of the flag, taken by one thread before a named
+    // barrier so that all 256 epilogue threads leave the loop together
+    volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);
     float* red = reinterpret_cast<float*>(smem + 512);          // [2][4][8]: tile max, l sums
-    const SmemPlan P = plan_smem(rK, rV, ns);
+    const SmemPlan P = plan_smem(rK, rV, ns, nbk);
     float* sq = reinterpret_cast<float*>(smem + P.total);       // queries of the head, g x d fp32
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
@@ -170,8 +173,8 @@ decode_tc_kernel(DecodeTcArgs a) {
                 const int64_t hidx = (int64_t)a.layer * BH + head;
                 if (head != prev) {
                     ++hs;
-                    const int hb = hs & 1;
-                    if (hs >= 2 && !mbar_wait(&bars->bk_empty[hb], ((hs - 2) >> 1) & 1, deadline)) {
+                    const int hb = hs % nbk;
+                    if (hs >= nbk && !mbar_wait(&bars->bk_empty[hb], ((hs / nbk) - 1) & 1, deadline)) {
                         fail();
                         break;
                     }
@@ -211,7 +214,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 const int head = (int)(fi / tph);
                 if (head != prev) {
                     ++hs;
-                    if (!mbar_wait(&bars->bk_full[hs & 1], (hs >> 1) & 1, deadline)) {
+                    if (!mbar_wait(&bars->bk_full[hs % nbk], (hs / nbk) & 1, deadline)) {
                         fail();
                         break;
                     }
@@ -228,7 +231,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 }
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(stage + st * stage_bytes);
-                const uint32_t b0 = smem_u32(bk + (hs & 1) * bk_bytes);
+                const uint32_t b0 = smem_u32(bk + (hs % nbk) * bk_bytes);
                 const uint32_t dk = tmem + b * kBufCols;
                 for (int ks = 0; ks < rK / 16; ++ks)
                     for (int part = 0; part < 2; ++part) {
@@ -238,7 +241,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                     }
                 mma_commit(&bars->kh_full[b]);
                 const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
-                if (seg_end) mma_commit(&bars->bk_empty[hs & 1]);
+                if (seg_end) mma_commit(&bars->bk_empty[hs % nbk]);
             }
         }
     } else {
@@ -273,7 +276,9 @@ decode_tc_kernel(DecodeTcArgs a) {
         bool have_prev = false;
         int cur_head = -1;
         for (int n = 0; n < ntiles; ++n) {
-            if (*abort_flag) break;
+            if (ept == 0) *epi_abort = *abort_flag;
+            epi_sync();
+            if (*epi_abort) break;                // uniform across the epilogue
             const int64_t fi = f0 + n;
             const int head = (int)(fi / tph), tile = (int)(fi % tph);
             const int b = n & 1, st = n % ns;
@@ -283,7 +288,6 @@ decode_tc_kernel(DecodeTcArgs a) {
                 const int bq = head / a.Hkv, kvh = head % a.Hkv;
                 const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.q) +
                                           ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
-                epi_sync();
                 for (int e = ept; e < g * d; e += kEpi) sq[e] = __bfloat162float(qg[e]);
 #pragma unroll
                 for (int u = 0; u < kH; ++u) {
@@ -476,12 +480,12 @@ decode_tc_kernel(DecodeTcArgs a) {
 
 }  // namespace
 
-size_t decode_tc_smem_bytes(int rK, int rV, int ns) {
-    return plan_smem(rK, rV, ns).total + (size_t)kMaxGroup * kHeadDim * 4;
+size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk) {
+    return plan_smem(rK, rV, ns, nbk).total + (size_t)kMaxGroup * kHeadDim * 4;
 }
 
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s) {
-    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages);
+    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages, a.basis_bufs);
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;

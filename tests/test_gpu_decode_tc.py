@@ -1,0 +1,99 @@
+"""Tensor-core decode over the folded rows (bf16 coefficients) against the
+float64 oracle (bf16 storage emulated) and against the CUDA-core decode on an
+identical cache.  Covers the shapes the kernel's layouts depend on: value MMA
+with M=64 and M=128 (r_V <= 64 and > 64), r = d, the smallest ranks, query
+groups 1..8, no exact rows at all, CTAs whose tile ranges span several heads,
+and sharply peaked ("recall") queries aimed at a folded token.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from iskv_testlib import Pair, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 2e-2
+
+
+def _cfg(**kw):
+    import online_rank_kv_b200 as ik
+    c = ik.Config(batch=2, layers=1, kv_heads=2, q_heads=8, rank_k=32, rank_v=64, window=256,
+                  max_tokens=4096, kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1,
+                  rope_theta=1e6, max_deferred=8)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _pair(tc: bool, cfg, seed):
+    old = os.environ.get("ISKV_TENSOR_CORES")
+    os.environ["ISKV_TENSOR_CORES"] = "1" if tc else "0"
+    try:
+        return Pair(cfg, "qwen3", seed=seed)
+    finally:
+        if old is None:
+            del os.environ["ISKV_TENSOR_CORES"]
+        else:
+            os.environ["ISKV_TENSOR_CORES"] = old
+
+
+@pytest.mark.parametrize("rk,rv,g,W,T", [
+    (32, 64, 4, 256, 2048 + 40),
+    (64, 96, 4, 256, 1500),
+    (128, 128, 2, 128, 900),
+    (16, 16, 1, 128, 700),
+    (32, 48, 8, 0, 1024),
+])
+def test_tc_decode_matches_oracle_and_cuda_core(rk, rv, g, W, T):
+    cfg = _cfg(rank_k=rk, rank_v=rv, q_heads=2 * g, window=W, max_tokens=T + 256)
+    pt = _pair(True, cfg, seed=31 + rk + rv)
+    pc = _pair(False, cfg, seed=31 + rk + rv)
+    pt.prefill(T, chunk=64, defer_every=8)
+    pc.prefill(T, chunk=64, defer_every=8)
+    T_, n_c = pt.cache.counts(0)
+    assert n_c > 0
+    for _ in range(2):
+        q = pt.query()
+        errs, out_t = pt.decode(0, q)
+        out_c = pc.cache.decode_attention(0, q.cuda()).cpu().numpy()
+        assert max(errs.values()) < TOL_BF16, errs
+        assert rel_err(out_t, out_c) < 5e-3
+    assert pt.cache.status() == 0
+
+
+def test_tc_decode_ctas_span_heads():
+    """64 (sequence, KV head) pairs with 3 tiles each: 192 tiles on 148 SMs,
+    so most CTAs cover parts of two heads."""
+    cfg = _cfg(batch=8, kv_heads=8, q_heads=32, window=128, max_tokens=1024)
+    p = _pair(True, cfg, seed=41)
+    p.prefill(128 + 3 * 128 - 64 + 17, chunk=64)
+    T, n_c = p.cache.counts(0)
+    assert n_c == 320                       # 2.5 tiles: last tile half full
+    errs, _ = p.decode(0, p.query())
+    assert max(errs.values()) < TOL_BF16, errs
+    assert p.cache.status() == 0
+
+
+def test_tc_decode_recall_query():
+    """A query aimed at one folded token (its score ~25 above the rest):
+    the sharpest attention the decode has to reproduce."""
+    cfg = _cfg(kv_heads=2, q_heads=8, window=256)
+    p = _pair(True, cfg, seed=43)
+    p.prefill(2048)
+    q = p.query().double()
+    pos = 333
+    for b in range(cfg.batch):
+        for h in range(cfg.kv_heads):
+            kp = torch.from_numpy(p.ok[(0, b, h)].reconstruct()[pos])
+            # score of token pos = beta |k| / sqrt(d) = 25
+            beta = 25.0 * np.sqrt(128) / float(torch.linalg.vector_norm(kp))
+            for j in range(4):
+                q[b, h * 4 + j] = synth.recall_query(kp, pos, cfg.rope_theta, beta)
+    q = q.to(torch.bfloat16)
+    errs, _ = p.decode(0, q)
+    assert max(errs.values()) < TOL_BF16, errs
