@@ -39,6 +39,8 @@ WORKLOADS = {
     # name: batch, layers, kv_heads, q_heads, rank_k, rank_v, window, prefill, coef
     "qwen3-36L-b8-32k": dict(batch=8, layers=36, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
                              window=1024, prefill=32768, coef="bf16", gen="qwen3"),
+    "qwen3-1L-b8-32k": dict(batch=8, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
+                            window=1024, prefill=32768, coef="bf16", gen="qwen3"),
     "qwen3-1L-b1-16k": dict(batch=1, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
                             window=1024, prefill=16384, coef="f32", gen="qwen3"),
 }

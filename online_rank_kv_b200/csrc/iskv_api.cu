@@ -450,7 +450,8 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.n_c = h->n_c[layer];
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
     const int sms = h->sms;
-    if (h->use_tc && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 && a.n_c > 0) {
+    if (h->use_tc && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 && a.n_c > 0 &&
+        decode_tc_supports_group(a.g)) {
         // folded rows: persistent tensor-core kernel, one CTA per SM over the
         // flattened (head, 128-token tile) space; exact rows: extra splits
         DecodeTcArgs t{};

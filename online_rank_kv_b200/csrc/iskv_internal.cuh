@@ -148,6 +148,7 @@ cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64
 cudaError_t launch_resync_tc(const FactorView& f, const ResyncLaunch& rl, int* status,
                              cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
+bool decode_tc_supports_group(int g);
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk);
 
 size_t fold_smem_bytes(int r);

@@ -18,22 +18,24 @@
 //           the bf16 hi/lo basis of each head it visits;
 //   warp 1  MMA issuer: K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens,
 //           N=128 dims, fp32 accumulator in TMEM (two buffers);
-//   warps 2-9 epilogue, one token row per pair of threads (warps w and w+4
-//           reach the same TMEM lanes); each thread of the pair owns half of
-//           the 64 rotation pairs and half of the query heads:
-//           * rotate its half row of K^ by R_t (t = row within the tile; the
-//             thread's cos/sin(t w_i) live in registers) and write it back to
-//             TMEM rounded to tf32; the query is pre-rotated per tile by
-//             R_{j0}^T (j0 = tile start), so q'.(R_t k) = q.(R_{j0+t} k);
+//   warps 2-9 epilogue, two ping-pong groups of 4 warps (group = tile
+//           parity), one token row per thread:
+//           * rotate its row of K^ by R_t (t = row within the tile; the
+//             row's cos/sin(t w_i) sit in spare TMEM columns) and write it
+//             back to TMEM rounded to tf32; the query is pre-rotated per tile
+//             by R_{j0}^T (j0 = tile start), so q'.(R_t k) = q.(R_{j0+t} k);
 //           * scores S = K_rot q'^T on the tensor cores (kind::tf32, A from
 //             TMEM, q' as tf32 hi+lo parts in the N dimension);
-//           * online softmax per query head (tile max over the 128 rows);
+//           * online softmax per query head and group; at the end of each
+//             head the two groups' states are merged by log-sum-exp;
 //           * p as bf16 hi+lo parts -> O = C_V^T P (kind::f16, C_V tile read
 //             MN-major in place), accumulated with the running rescale.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // ISKV status bit 2, stops, drains its copies and frees its TMEM.
 #include "iskv_internal.cuh"
 #include "tc_util.cuh"
+
+#include <type_traits>
 
 namespace iskv {
 
@@ -43,16 +45,18 @@ using namespace tc;
 
 constexpr int kTile = 128;
 constexpr int kThreads = 320;
-constexpr int kEpi = 256;        // epilogue threads (warps 2-9)
+constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
 constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
 constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
 constexpr int kBufCols = 160;    // per TMEM buffer: K^ 128 | S 16 | O 16
+constexpr int kCsCol = 2 * kBufCols;   // per-row RoPE table: cos 64 | sin 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Bars {
     uint64_t full[4], empty[4];
     uint64_t bk_full[2], bk_empty[2];
     uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
+    uint64_t drain[2];   // abort path: completion of each issuer's outstanding MMAs
 };
 
 struct SmemPlan {
@@ -71,15 +75,11 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk) {
     return p;
 }
 
-// v[idx] for a runtime idx without forcing v into local memory
-__device__ __forceinline__ float pick16(const uint32_t (&v)[16], int idx) {
-    float r = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) r = (k == idx) ? __uint_as_float(v[k]) : r;
-    return r;
-}
-
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// barrier of one ping-pong group (ids 2 and 3, 128 threads)
+__device__ __forceinline__ void group_sync(int grp) {
+    asm volatile("bar.sync %0, 128;" ::"r"(2 + grp) : "memory");
+}
 
 // offsets of the tf32 (K-major, 8 x 4 core matrices) and bf16 (8 x 8) B operands
 __device__ __forceinline__ int qb_off(int n, int k) {
@@ -89,6 +89,7 @@ __device__ __forceinline__ int pb_off(int n, int k) {
     return ((n >> 3) * (kTile / 8) + (k >> 3)) * 64 + (n & 7) * 8 + (k & 7);
 }
 
+template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(DecodeTcArgs a) {
     const int cta = blockIdx.x;
@@ -98,7 +99,8 @@ decode_tc_kernel(DecodeTcArgs a) {
     if (f0 >= f1) return;
     const int ntiles = (int)(f1 - f0);
     const int tph = a.tiles_per_head;
-    const int rK = a.K.r, rV = a.V.r, g = a.g, ns = a.stages, nbk = a.basis_bufs;
+    const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs;
+    constexpr int g = G;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int d = kHeadDim;
 
@@ -109,7 +111,8 @@ decode_tc_kernel(DecodeTcArgs a) {
     // the epilogue's copy of the flag, taken by one thread before a named
     // barrier so that all 256 epilogue threads leave the loop together
     volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);
-    float* red = reinterpret_cast<float*>(smem + 512);          // [2][4][8]: tile max, l sums
+    volatile int* flag_max = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2]
+    float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
     const SmemPlan P = plan_smem(rK, rV, ns, nbk);
     float* sq = reinterpret_cast<float*>(smem + P.total);       // queries of the head, g x d fp32
     uint8_t* bk = smem + P.bk;
@@ -135,8 +138,11 @@ decode_tc_kernel(DecodeTcArgs a) {
             mbar_init(&bars->kfree[i], 1);
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->o_full[i], 1);
+            mbar_init(&bars->drain[i], 1);
         }
         *abort_flag = 0;
+        flag_max[0] = 0;
+        flag_max[1] = 0;
         fence_mbar_init();
     }
     // zero the padding rows (n >= 2g) of the q' and p operands once
@@ -243,24 +249,36 @@ decode_tc_kernel(DecodeTcArgs a) {
                 const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
                 if (seg_end) mma_commit(&bars->bk_empty[hs % nbk]);
             }
+            if (*abort_flag) {                        // let issued MMAs finish (bounded)
+                mma_commit(&bars->drain[0]);
+                mbar_wait(&bars->drain[0], 0, deadline + kWaitCycles);
+            }
         }
     } else {
-        // ---------------- epilogue: 256 threads, two per token row ----------------
+        // ---------------- epilogue: two groups of 4 warps, alternate tiles ----------------
         const int ept = tid - 64;                 // 0..255
+        const int grp = ept >> 7;                 // tiles n with n % 2 == grp
+        const int gt = ept & 127;                 // thread within the group
         const int sp = warp & 3;                  // TMEM sub-partition of this warp
-        const int half = ept >> 7;                // which half of the pairs / heads
         const int row = sp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-        const int i0 = half * 32;                 // first rotation pair of this thread
-        const int gh = (g + 1) / 2;               // heads of half 0
-        const int h_lo = half ? gh : 0, h_hi = half ? g : gh;
-        float cs_c[32], cs_s[32];
+        const uint32_t tcs = tmem + kCsCol;
+        // this row's in-tile RoPE table (cos, sin of row * w_i) into TMEM
+        if (grp == 0) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            float2 v = make_float2(1.f, 0.f);
-            if (a.rope) v = a.rope[row * 64 + i0 + u];
-            cs_c[u] = v.x;
-            cs_s[u] = v.y;
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                uint32_t vc[16], vs[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    float2 v = make_float2(1.f, 0.f);
+                    if (a.rope) v = a.rope[row * 64 + c0 + u];
+                    vc[u] = __float_as_uint(v.x);
+                    vs[u] = __float_as_uint(v.y);
+                }
+                tmem_st16(tcs + lane_base + c0, vc);
+                tmem_st16(tcs + lane_base + 64 + c0, vs);
+            }
+            tmem_wait_st();
         }
         const int MV = rV <= 64 ? 64 : 128;
         const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
@@ -270,196 +288,216 @@ decode_tc_kernel(DecodeTcArgs a) {
         const uint32_t sbo_q = (kTile / 4) * 128;
         const uint32_t sbo_p = (kTile / 8) * 128;
         const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
-        constexpr int kH = kMaxGroup / 2;         // heads per thread at most
+        float* gred = red + grp * 64;             // [max 4 x 8 | l 4 x 8] of this group
+        const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
+        uint32_t* qbb = qb + grp * kQN * kTile;
+        __nv_bfloat16* pbb = pb + grp * kPN * kTile;
 
-        float m_run[kH], l_thr[kH], acc[kH], alpha[kH];
-        bool have_prev = false;
-        int cur_head = -1;
-        for (int n = 0; n < ntiles; ++n) {
-            if (ept == 0) *epi_abort = *abort_flag;
-            epi_sync();
-            if (*epi_abort) break;                // uniform across the epilogue
-            const int64_t fi = f0 + n;
-            const int head = (int)(fi / tph), tile = (int)(fi % tph);
-            const int b = n & 1, st = n % ns;
-            const uint32_t kh = tmem + b * kBufCols;
-            if (head != cur_head) {
-                // new head segment: its queries, fresh softmax state
+        float m_run[G], l_thr[G], acc[G], alpha[G];
+        bool stop = false;
+        int n0 = 0;
+        while (n0 < ntiles) {
+            const int head = (int)((f0 + n0) / tph);
+            int s1 = (int)(((int64_t)head + 1) * tph - f0);
+            if (s1 > ntiles) s1 = ntiles;
+            // queries of the head, fresh softmax state; uniform abort check
+            {
                 const int bq = head / a.Hkv, kvh = head % a.Hkv;
                 const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.q) +
                                           ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
                 for (int e = ept; e < g * d; e += kEpi) sq[e] = __bfloat162float(qg[e]);
-#pragma unroll
-                for (int u = 0; u < kH; ++u) {
-                    m_run[u] = -INFINITY;
-                    l_thr[u] = 0.f;
-                    acc[u] = 0.f;
-                    alpha[u] = 0.f;
-                }
-                have_prev = false;
-                cur_head = head;
-                epi_sync();
             }
-            const int64_t j0 = (int64_t)tile * kTile;
-            const int valid = (int)((a.n_c - j0) < kTile ? (a.n_c - j0) : kTile);
-            // q' = R_{j0}^T q for this tile, tf32 hi / lo parts as the B operand
-            uint32_t* qbb = qb + b * kQN * kTile;
-            for (int item = ept; item < g * 64; item += kEpi) {
-                const int h = item >> 6, i = item & 63;
-                float c0 = 1.f, s0 = 0.f;
-                if (a.rope) {
-                    const float2 v = a.rope[j0 * 64 + i];
-                    c0 = v.x;
-                    s0 = v.y;
-                }
-                const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
-                const float y1 = fmaf(c0, x1, s0 * x2);
-                const float y2 = fmaf(c0, x2, -s0 * x1);
-                const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
-                qbb[qb_off(h, i)] = t1;
-                qbb[qb_off(h, i + 64)] = t2;
-                qbb[qb_off(g + h, i)] = to_tf32(y1 - __uint_as_float(t1));
-                qbb[qb_off(g + h, i + 64)] = to_tf32(y2 - __uint_as_float(t2));
-            }
-            fence_async_smem();
-            // rotate this thread's half row of K^ and store it back as tf32
-            if (!mbar_wait(&bars->kh_full[b], (n >> 1) & 1, deadline)) fail();
-            tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 32; c += 16) {
-                uint32_t x1[16], x2[16];
-                tmem_ld16(kh + lane_base + i0 + c, x1);
-                tmem_ld16(kh + lane_base + 64 + i0 + c, x2);
-                tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float k1 = __uint_as_float(x1[u]), k2 = __uint_as_float(x2[u]);
-                    const float co = cs_c[c + u], si = cs_s[c + u];
-                    x1[u] = to_tf32(fmaf(k1, co, -k2 * si));
-                    x2[u] = to_tf32(fmaf(k1, si, k2 * co));
-                }
-                tmem_st16(kh + lane_base + i0 + c, x1);
-                tmem_st16(kh + lane_base + 64 + i0 + c, x2);
+            for (int h = 0; h < G; ++h) {
+                m_run[h] = -INFINITY;
+                l_thr[h] = 0.f;
+                acc[h] = 0.f;
+                alpha[h] = 0.f;
             }
-            tmem_wait_st();
+            if (ept == 0) *epi_abort = *abort_flag;
             tc_fence_before();
             epi_sync();
-            if (ept == 0 && !*abort_flag) {
-                tc_fence_after();
-                const uint32_t q0 = smem_u32(qbb);
-                for (int ks = 0; ks < d / 8; ++ks)
-                    mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
-                                idesc_s, ks != 0);
-                mma_commit(&bars->s_full[b]);
-            }
-            // accumulate the previous tile's p^T C_V (its MMA ran meanwhile)
-            if (have_prev) {
-                const int pbuf = (n - 1) & 1;
-                if (!mbar_wait(&bars->o_full[pbuf], ((n - 1) >> 1) & 1, deadline)) fail();
-                tc_fence_after();
-                uint32_t o[16];
-                tmem_ld16(tmem + pbuf * kBufCols + 144 + lane_base, o);
-                tmem_wait_ld();
-                if (acc_ok) {
-#pragma unroll
-                    for (int u = 0; u < kH; ++u) {
-                        const int h = h_lo + u;
-                        if (h < h_hi)
-                            acc[u] = fmaf(acc[u], alpha[u], pick16(o, h) + pick16(o, g + h));
-                    }
-                }
-            }
-            // scores of this thread's heads, online softmax
-            if (!mbar_wait(&bars->s_full[b], (n >> 1) & 1, deadline)) fail();
             tc_fence_after();
-            uint32_t sv[16];
-            tmem_ld16(kh + 128 + lane_base, sv);
-            tmem_wait_ld();
-            float sc[kH];
-#pragma unroll
-            for (int u = 0; u < kH; ++u) {
-                const int h = h_lo + u;
-                sc[u] = -INFINITY;
-                if (h < h_hi && row < valid)
-                    sc[u] = (pick16(sv, h) + pick16(sv, g + h)) * a.scale;
-                const float wm = warp_max(sc[u]);
-                if (lane == 0 && h < h_hi) red[sp * 8 + h] = wm;
-            }
-            epi_sync();
-            __nv_bfloat16* pbb = pb + b * kPN * kTile;
-#pragma unroll
-            for (int u = 0; u < kH; ++u) {
-                const int h = h_lo + u;
-                if (h >= h_hi) break;
-                const float tmax = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
-                const float m_new = fmaxf(m_run[u], tmax);
-                const float al = (m_run[u] == -INFINITY) ? 0.f : __expf(m_run[u] - m_new);
-                const float p = (sc[u] == -INFINITY) ? 0.f : __expf(sc[u] - m_new);
-                l_thr[u] = fmaf(l_thr[u], al, p);
-                m_run[u] = m_new;
-                alpha[u] = al;
-                const __nv_bfloat16 ph = __float2bfloat16_rn(p);
-                pbb[pb_off(h, row)] = ph;
-                pbb[pb_off(g + h, row)] = __float2bfloat16_rn(p - __bfloat162float(ph));
-            }
-            fence_async_smem();
-            tc_fence_before();
-            epi_sync();
-            if (ept == 0 && !*abort_flag) {
-                mbar_arrive(&bars->kfree[b]);   // K^/S buffer b may be overwritten
+            stop = *epi_abort;                    // latched after the barrier: uniform
+            if (stop) break;
+            bool have_prev = false;
+            int last = -1;
+            for (int n = n0 + ((n0 & 1) != grp ? 1 : 0); n < s1; n += 2) {
+                const int st = n % ns;
+                const int64_t j0 = (int64_t)((f0 + n) % tph) * kTile;
+                const int valid = (int)((a.n_c - j0) < kTile ? (a.n_c - j0) : kTile);
+                // q' = R_{j0}^T q, tf32 hi / lo parts as the score MMA's B operand
+                for (int item = gt; item < g * 64; item += 128) {
+                    const int h = item >> 6, i = item & 63;
+                    float c0 = 1.f, s0 = 0.f;
+                    if (a.rope) {
+                        const float2 v = a.rope[j0 * 64 + i];
+                        c0 = v.x;
+                        s0 = v.y;
+                    }
+                    const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
+                    const float y1 = fmaf(c0, x1, s0 * x2);
+                    const float y2 = fmaf(c0, x2, -s0 * x1);
+                    const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
+                    qbb[qb_off(h, i)] = t1;
+                    qbb[qb_off(h, i + 64)] = t2;
+                    qbb[qb_off(g + h, i)] = to_tf32(y1 - __uint_as_float(t1));
+                    qbb[qb_off(g + h, i + 64)] = to_tf32(y2 - __uint_as_float(t2));
+                }
+                fence_async_smem();
+                // rotate this row of K^ by R_t, store back as tf32
+                if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
-                const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
-                const uint32_t p0 = smem_u32(pbb);
-                for (int ks = 0; ks < kTile / 16; ++ks)
-                    mma_f16_ss(tmem + b * kBufCols + 144,
-                               desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
-                               desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_o, ks != 0);
-                mma_commit(&bars->o_full[b]);
-                mma_commit(&bars->empty[st]);
-            }
-            have_prev = true;
-            const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
-            if (seg_end) {
-                if (!mbar_wait(&bars->o_full[b], (n >> 1) & 1, deadline)) fail();
-                tc_fence_after();
-                uint32_t o[16];
-                tmem_ld16(tmem + b * kBufCols + 144 + lane_base, o);
-                tmem_wait_ld();
-                if (acc_ok) {
 #pragma unroll
-                    for (int u = 0; u < kH; ++u) {
-                        const int h = h_lo + u;
-                        if (h < h_hi)
-                            acc[u] = fmaf(acc[u], alpha[u], pick16(o, h) + pick16(o, g + h));
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    uint32_t x1[16], x2[16], cc[16], ss[16];
+                    tmem_ld16(kh + lane_base + c0, x1);
+                    tmem_ld16(kh + lane_base + 64 + c0, x2);
+                    tmem_ld16(tcs + lane_base + c0, cc);
+                    tmem_ld16(tcs + lane_base + 64 + c0, ss);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const float k1 = __uint_as_float(x1[u]), k2 = __uint_as_float(x2[u]);
+                        const float co = __uint_as_float(cc[u]), si = __uint_as_float(ss[u]);
+                        x1[u] = to_tf32(fmaf(k1, co, -k2 * si));
+                        x2[u] = to_tf32(fmaf(k1, si, k2 * co));
+                    }
+                    tmem_st16(kh + lane_base + c0, x1);
+                    tmem_st16(kh + lane_base + 64 + c0, x2);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                group_sync(grp);                      // k_rot and q' of tile n complete
+                if (gt == 0 && !*abort_flag) {
+                    tc_fence_after();
+                    const uint32_t q0 = smem_u32(qbb);
+                    for (int ks = 0; ks < d / 8; ++ks)
+                        mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
+                                    idesc_s, ks != 0);
+                    mma_commit(&bars->s_full[grp]);
+                }
+                // this group's previous tile: p^T C_V accumulated (before O is reused)
+                if (have_prev) {
+                    if (!mbar_wait(&bars->o_full[grp], ((n - 2) >> 1) & 1, deadline)) fail();
+                    tc_fence_after();
+                    uint32_t o[16];
+                    tmem_ld16(kh + 144 + lane_base, o);
+                    tmem_wait_ld();
+                    if (acc_ok) {
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+                            acc[h] = fmaf(acc[h], alpha[h], __uint_as_float(o[h]) + __uint_as_float(o[G + h]));
                     }
                 }
-                have_prev = false;
-                // l over the 128 rows of each head
+                // scores and the tile max of each head
+                if (!mbar_wait(&bars->s_full[grp], (n >> 1) & 1, deadline)) fail();
+                tc_fence_after();
+                uint32_t sv[16];
+                tmem_ld16(kh + 128 + lane_base, sv);
+                tmem_wait_ld();
+                float sc[G];
 #pragma unroll
-                for (int u = 0; u < kH; ++u) {
-                    const int h = h_lo + u;
-                    const float ws = warp_sum(l_thr[u]);
-                    if (lane == 0 && h < h_hi) red[32 + sp * 8 + h] = ws;
+                for (int h = 0; h < G; ++h) {
+                    sc[h] = (row < valid) ? (__uint_as_float(sv[h]) + __uint_as_float(sv[G + h])) * a.scale
+                                          : -INFINITY;
+                    const float wm = warp_max(sc[h]);
+                    if (lane == 0) gred[sp * 8 + h] = wm;
                 }
                 tc_fence_before();
-                epi_sync();
+                group_sync(grp);
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float tmax = fmaxf(fmaxf(gred[h], gred[8 + h]), fmaxf(gred[16 + h], gred[24 + h]));
+                    const float m_new = fmaxf(m_run[h], tmax);
+                    const float al = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
+                    const float p = (sc[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_new);
+                    l_thr[h] = fmaf(l_thr[h], al, p);
+                    m_run[h] = m_new;
+                    alpha[h] = al;
+                    const __nv_bfloat16 ph = __float2bfloat16_rn(p);
+                    pbb[pb_off(h, row)] = ph;
+                    pbb[pb_off(G + h, row)] = __float2bfloat16_rn(p - __bfloat162float(ph));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                group_sync(grp);                      // P of tile n complete, max read
+                if (gt == 0 && !*abort_flag) {
+                    mbar_arrive(&bars->kfree[grp]);   // K^/S of this buffer may be overwritten
+                    tc_fence_after();
+                    const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
+                    const uint32_t p0 = smem_u32(pbb);
+                    for (int ks = 0; ks < kTile / 16; ++ks)
+                        mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
+                                   desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_o, ks != 0);
+                    mma_commit(&bars->o_full[grp]);
+                    mma_commit(&bars->empty[st]);
+                }
+                have_prev = true;
+                last = n;
+            }
+            // close this group's share of the head
+            if (have_prev) {
+                if (!mbar_wait(&bars->o_full[grp], (last >> 1) & 1, deadline)) fail();
+                tc_fence_after();
+                uint32_t o[16];
+                tmem_ld16(kh + 144 + lane_base, o);
+                tmem_wait_ld();
+                if (acc_ok) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        acc[h] = fmaf(acc[h], alpha[h], __uint_as_float(o[h]) + __uint_as_float(o[G + h]));
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float ws = warp_sum(l_thr[h]);
+                if (lane == 0) gred[32 + sp * 8 + h] = ws;
+            }
+            tc_fence_before();
+            group_sync(grp);
+            // a group's softmax state goes to its own q' buffer, idle now that
+            // its last score MMA of the head has completed: [m 8 | l 8 | acc 8 x 128]
+            static_assert((2 * kMaxGroup + kMaxGroup * kHeadDim) <= kQN * kTile, "exchange fits");
+            float* xg = reinterpret_cast<float*>(qbb);
+            if (gt == 0) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    xg[h] = m_run[h];
+                    xg[kMaxGroup + h] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
+                }
+            }
+            if (acc_ok) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) xg[2 * kMaxGroup + h * kHeadDim + c_acc] = acc[h];
+            }
+            epi_sync();                               // both groups published
+            if (grp == 0) {
+                // log-sum-exp merge of the two groups, one partial slot per head
+                const float* x0 = reinterpret_cast<const float*>(qb);
+                const float* x1 = reinterpret_cast<const float*>(qb + kQN * kTile);
                 const int bq = head / a.Hkv, kvh = head % a.Hkv;
                 const int c_first = (int)(((int64_t)head * tph) / a.tiles_per_cta);
                 const int slot = cta - c_first;
                 const int stride = 2 + rV + d;
-                for (int u = 0; u < kH; ++u) {
-                    const int h = h_lo + u;
-                    if (h >= h_hi) break;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float m0 = x0[h], m1 = x1[h];
+                    const float M = fmaxf(m0, m1);
+                    const float w0 = (m0 == -INFINITY) ? 0.f : __expf(m0 - M);
+                    const float w1 = (m1 == -INFINITY) ? 0.f : __expf(m1 - M);
                     float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
-                    if (acc_ok) Pp[2 + c_acc] = acc[u];
-                    for (int i = ept & 127; i < d; i += 128) Pp[2 + rV + i] = 0.f;
-                    if ((ept & 127) == 0) {
-                        Pp[0] = m_run[u];
-                        Pp[1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
+                    if (acc_ok)
+                        Pp[2 + c_acc] = x0[2 * kMaxGroup + h * kHeadDim + c_acc] * w0 +
+                                        x1[2 * kMaxGroup + h * kHeadDim + c_acc] * w1;
+                    Pp[2 + rV + gt] = 0.f;            // d = 128 = group size
+                    if (gt == 0) {
+                        Pp[0] = M;
+                        Pp[1] = x0[kMaxGroup + h] * w0 + x1[kMaxGroup + h] * w1;
                     }
                 }
                 // this CTA ends the head: mark the head's unused compressed slots empty
-                if (ept == 0 && f1 >= (int64_t)(head + 1) * tph) {
+                if (gt == 0 && f1 >= (int64_t)(head + 1) * tph) {
                     for (int h = 0; h < g; ++h)
                         for (int sl = slot + 1; sl < a.slots_c; ++sl) {
                             float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + sl) * stride;
@@ -467,8 +505,13 @@ decode_tc_kernel(DecodeTcArgs a) {
                             Pp[1] = 0.f;
                         }
                 }
-                epi_sync();
             }
+            epi_sync();                               // exchange area free again
+            n0 = s1;
+        }
+        if (ept == 0 && *abort_flag) {                // let issued MMAs finish (bounded)
+            mma_commit(&bars->drain[1]);
+            mbar_wait(&bars->drain[1], 0, deadline + kWaitCycles);
         }
     }
 
@@ -481,16 +524,30 @@ decode_tc_kernel(DecodeTcArgs a) {
 }  // namespace
 
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk) {
+    // + queries of the head (g x d fp32)
     return plan_smem(rK, rV, ns, nbk).total + (size_t)kMaxGroup * kHeadDim * 4;
 }
 
-cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s) {
+template <int G>
+cudaError_t launch_g(const DecodeTcArgs& a, cudaStream_t s) {
     const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages, a.basis_bufs);
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<<<a.ncta, kThreads, bytes, s>>>(a);
+    decode_tc_kernel<G><<<a.ncta, kThreads, bytes, s>>>(a);
     return cudaGetLastError();
+}
+
+bool decode_tc_supports_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s) {
+    switch (a.g) {
+        case 1: return launch_g<1>(a, s);
+        case 2: return launch_g<2>(a, s);
+        case 4: return launch_g<4>(a, s);
+        case 8: return launch_g<8>(a, s);
+        default: return cudaErrorNotSupported;
+    }
 }
 
 }  // namespace iskv
