@@ -106,6 +106,7 @@ FactorView view(const iskv_cache* h, int which) {
     f.coef_bf16 = h->cfg.coef_dtype == ISKV_BF16;
     f.coef_blocked = f.coef_bf16;   // bf16 rows live in 8x8 core-matrix blocks
     f.kv_bf16 = h->cfg.kv_dtype == ISKV_BF16;
+    f.ring_blocked = f.kv_bf16;     // and so do bf16 exact rows
     f.n_max = h->n_max;
     f.cap = h->cap;
     f.D = h->D;
@@ -330,7 +331,8 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
         char* rings[2] = {rk, rv};
         for (int w = 0; w < 2; ++w) {
             if (is_device_ptr(srcs[w])) {
-                CU(launch_append(rings[w], srcs[w], h->BH, t, h->T[layer], h->cap, h->kv_bytes, s));
+                CU(launch_append(rings[w], srcs[w], h->BH, t, h->T[layer], h->cap, h->kv_bytes,
+                                 h->cfg.kv_dtype == ISKV_BF16, s));
             } else {
                 // stage token chunks of every (sequence, head) through device memory
                 const int chunk = (int)std::max<size_t>(1, h->stage_in_bytes / ((size_t)h->BH * row_bytes));
@@ -341,7 +343,7 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
                                          (size_t)t * row_bytes, n * row_bytes, h->BH,
                                          cudaMemcpyDefault, s));
                     CU(launch_append(rings[w], h->stage_in, h->BH, n, h->T[layer] + t0, h->cap,
-                                     h->kv_bytes, s));
+                                     h->kv_bytes, h->cfg.kv_dtype == ISKV_BF16, s));
                 }
             }
         }
@@ -450,10 +452,11 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.n_c = h->n_c[layer];
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
     const int sms = h->sms;
-    if (h->use_tc && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 && a.n_c > 0 &&
+    if (h->use_tc && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 &&
         decode_tc_supports_group(a.g)) {
-        // folded rows: persistent tensor-core kernel, one CTA per SM over the
-        // flattened (head, 128-token tile) space; exact rows: extra splits
+        // one persistent tensor-core kernel, one CTA per SM, over the flattened
+        // (head, tile) space: 128-token tiles of folded rows, then 64-token
+        // tiles of exact rows, all under one online softmax per head
         DecodeTcArgs t{};
         t.K = a.K;
         t.V = a.V;
@@ -467,8 +470,10 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.Hq = c.q_heads;
         t.g = a.g;
         t.n_c = a.n_c;
+        t.T = a.T;
         t.scale = a.scale;
-        t.tiles_per_head = (int)((a.n_c + 127) / 128);
+        t.tiles_c = (int)((a.n_c + 127) / 128);
+        t.tiles_per_head = t.tiles_c + (int)((a.T - a.n_c + 63) / 64);
         t.total_tiles = (int64_t)h->BH * t.tiles_per_head;
         int64_t ncta = std::min<int64_t>(sms, t.total_tiles);
         t.tiles_per_cta = (int)((t.total_tiles + ncta - 1) / ncta);
@@ -479,7 +484,9 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
             const int64_t last = ((int64_t)(hh + 1) * t.tiles_per_head - 1) / t.tiles_per_cta;
             slots_c = std::max<int>(slots_c, (int)(last - first + 1));
         }
+        if (slots_c > h->max_splits) return ISKV_ERR_UNSUPPORTED;
         t.slots_c = slots_c;
+        t.splits_total = slots_c;
         // deepest pipeline that fits: two basis buffers if possible, else one
         t.stages = 0;
         for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
@@ -490,24 +497,9 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
                     break;
                 }
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
-        const int64_t n_w = a.T - a.n_c;
-        int64_t sw = 0, tps_w = 64;
-        if (n_w > 0) {
-            sw = std::min<int64_t>((n_w + 63) / 64, std::max<int64_t>(1, (2 * sms + h->BH - 1) / h->BH));
-            tps_w = ((n_w + sw - 1) / sw + 63) / 64 * 64;
-            sw = (n_w + tps_w - 1) / tps_w;
-        }
-        if (slots_c + sw > h->max_splits) return ISKV_ERR_UNSUPPORTED;
-        t.splits_total = (int)(slots_c + sw);
         CU(launch_decode_tc(t, s));
-        a.splits_total = t.splits_total;
-        if (sw > 0) {
-            a.j_begin = a.n_c;
-            a.split_base = slots_c;
-            a.splits = (int)sw;
-            a.tokens_per_split = tps_w;
-            CU(launch_decode(a, s));
-        }
+        a.splits = slots_c;
+        a.splits_total = slots_c;
         CU(launch_combine(a, od, s));
         if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
         return ISKV_OK;

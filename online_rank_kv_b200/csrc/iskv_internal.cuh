@@ -71,6 +71,7 @@ struct FactorView {
     int r;
     int coef_bf16;       // 1: coef stored as bf16
     int coef_blocked;    // 1: coef rows in 8x8 core-matrix blocks (see coef_index)
+    int ring_blocked;    // 1: exact rows in the same blocked layout (128 columns)
     int kv_bf16;         // 1: ring stored as bf16
     int64_t n_max;       // coefficient rows per head
     int64_t cap;         // ring rows per head
@@ -117,8 +118,9 @@ struct DecodeTcArgs {
     const float2* rope;          // [>= 128 positions][d/2], or null
     int* status;
     int layer, B, Hkv, Hq, g;
-    int64_t n_c;
-    int tiles_per_head;          // ceil(n_c / 128)
+    int64_t n_c, T;
+    int tiles_c;                 // folded-row tiles per head: ceil(n_c / 128)
+    int tiles_per_head;          // tiles_c + exact-row tiles of 64: ceil((T - n_c) / 64)
     int64_t total_tiles;         // BH * tiles_per_head
     int tiles_per_cta;
     int ncta;
@@ -134,7 +136,7 @@ struct DecodeTcArgs {
 // ---------------------------------------------------------------------------
 cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s);
 cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0,
-                          int64_t cap, int elem_bytes, cudaStream_t s);
+                          int64_t cap, int elem_bytes, int blocked, cudaStream_t s);
 cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status,
                         cudaStream_t s);
 cudaError_t launch_compose(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);

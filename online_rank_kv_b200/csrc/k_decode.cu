@@ -119,8 +119,8 @@ decode_kernel(DecodeArgs a) {
                 float kv = 0.f, vv = 0.f;
                 if (t < nt) {
                     const int64_t slot = (j + t) % a.K.cap;
-                    kv = to_f32(Rk[slot * d + i]);
-                    vv = to_f32(Rv[slot * d + i]);
+                    kv = to_f32(Rk[coef_index(a.K.ring_blocked, d, slot, i)]);
+                    vv = to_f32(Rv[coef_index(a.V.ring_blocked, d, slot, i)]);
                 }
                 sK[e] = kv;
                 sCv[e] = vv;
@@ -206,42 +206,52 @@ decode_kernel(DecodeArgs a) {
     }
 }
 
+// One CTA per (sequence, KV head): B_V is staged once (coalesced) for the
+// query group; thread i owns output dim i.
 __global__ void __launch_bounds__(kHeadDim)
 combine_kernel(DecodeArgs a, float* out) {
-    const int qh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-    const int rV = a.V.r, d = kHeadDim;
-    const int kvh = qh / a.g;
+    const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int rV = a.V.r, d = kHeadDim, g = a.g;
     const int64_t hidx = (int64_t)a.layer * a.V.BH + b * a.Hkv + kvh;
     const int stride = 2 + rV + d;
     const int slots = a.splits_total > 0 ? a.splits_total : a.splits;
-    const float* P = a.partial + ((int64_t)b * a.Hq + qh) * slots * stride;
-    __shared__ float sW[256];
-    __shared__ float sAcc[kHeadDim];
-    float M = -INFINITY;
-    for (int s = 0; s < slots; ++s) M = fmaxf(M, P[s * stride]);
-    float Ls = 0.f;
-    for (int s = tid; s < slots; s += blockDim.x) {
-        const float ms = P[s * stride];
-        sW[s] = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-    }
-    __syncthreads();
-    // empty slots (weight 0) are skipped: their other entries are not written
-    for (int s = 0; s < slots; ++s)
-        if (sW[s] != 0.f) Ls = fmaf(sW[s], P[s * stride + 1], Ls);
-    if (tid < rV) {
-        float v = 0.f;
-        for (int s = 0; s < slots; ++s)
-            if (sW[s] != 0.f) v = fmaf(sW[s], P[s * stride + 2 + tid], v);
-        sAcc[tid] = v;
-    }
-    float vd = 0.f;
-    for (int s = 0; s < slots; ++s)
-        if (sW[s] != 0.f) vd = fmaf(sW[s], P[s * stride + 2 + rV + tid], vd);
-    __syncthreads();
+    extern __shared__ float cs[];
+    float* sBv = cs;                               // d x (rV + 1)
+    float* sAcc = sBv + d * (rV + 1);              // rV
+    float* sW = sAcc + kHeadDim;                   // slots (<= 256)
     const float* Bv = a.V.basis + hidx * d * rV;
-    float o = vd;
-    for (int c = 0; c < rV; ++c) o = fmaf(sAcc[c], Bv[tid * rV + c], o);
-    out[((int64_t)b * a.Hq + qh) * d + tid] = o / Ls;
+    for (int e = tid; e < d * rV; e += blockDim.x) sBv[(e / rV) * (rV + 1) + e % rV] = Bv[e];
+    for (int hq = 0; hq < g; ++hq) {
+        const int qh = kvh * g + hq;
+        const float* P = a.partial + ((int64_t)b * a.Hq + qh) * slots * stride;
+        float M = -INFINITY;
+        for (int s = 0; s < slots; ++s) M = fmaxf(M, P[s * stride]);
+        __syncthreads();                           // sW / sAcc of the previous head consumed
+        for (int s = tid; s < slots; s += blockDim.x) {
+            const float ms = P[s * stride];
+            sW[s] = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+        }
+        __syncthreads();
+        // empty slots (weight 0) are skipped: their other entries are not written
+        float Ls = 0.f, vd = 0.f;
+        for (int s = 0; s < slots; ++s) {
+            const float w = sW[s];
+            if (w != 0.f) {
+                Ls = fmaf(w, P[s * stride + 1], Ls);
+                vd = fmaf(w, P[s * stride + 2 + rV + tid], vd);
+            }
+        }
+        if (tid < rV) {
+            float v = 0.f;
+            for (int s = 0; s < slots; ++s)
+                if (sW[s] != 0.f) v = fmaf(sW[s], P[s * stride + 2 + tid], v);
+            sAcc[tid] = v;
+        }
+        __syncthreads();
+        float o = vd;
+        for (int c = 0; c < rV; ++c) o = fmaf(sAcc[c], sBv[tid * (rV + 1) + c], o);
+        out[((int64_t)b * a.Hq + qh) * d + tid] = o / Ls;
+    }
 }
 
 }  // namespace
@@ -279,7 +289,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, float* out, cudaStream_t s) {
-    combine_kernel<<<dim3(a.Hq, a.B), kHeadDim, 0, s>>>(a, out);
+    const size_t bytes = ((size_t)kHeadDim * (a.V.r + 1) + kHeadDim + 256) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bytes);
+    if (e != cudaSuccess) return e;
+    combine_kernel<<<dim3(a.Hkv, a.B), kHeadDim, bytes, s>>>(a, out);
     return cudaGetLastError();
 }
 

@@ -8,14 +8,17 @@
 // head h of KV head h/g and folded token j < n_c:
 //   k_j = C_K[j] B_K^T,  s_j = q_h . RoPE(k_j, j) / sqrt(d),
 //   partial softmax (m, l) and acc_h = sum_j p_j C_V[j]   (r_V wide);
-// the exact window and the split merge are done by decode_kernel and
-// combine_kernel (k_decode.cu), which applies B_V^T once per query head.
+// and, for the exact rows j >= n_c (64-token tiles of the window ring),
+//   s_j = q_h . RoPE(K_j, j) / sqrt(d) and acc_d = sum_j p_j V_j (d wide),
+// all under one online softmax per head; combine_kernel (k_decode.cu) merges
+// the per-CTA partials and applies B_V^T once per query head.
 //
 // Persistent design, one CTA per SM, the flattened (head, 128-token tile)
 // space cut into equal contiguous ranges; per CTA 10 warps:
 //   warp 0  producer: 1-D bulk copies (TMA engine) of the C_K and C_V tiles
-//           (contiguous in the blocked layout) into an NS-stage ring, and of
-//           the bf16 hi/lo basis of each head it visits;
+//           or of the exact K and V rows (all contiguous in the blocked
+//           layout) into an NS-stage ring, and of the bf16 hi/lo basis of
+//           each head it visits;
 //   warp 1  MMA issuer: K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens,
 //           N=128 dims, fp32 accumulator in TMEM (two buffers);
 //   warps 2-9 epilogue, two ping-pong groups of 4 warps (group = tile
@@ -29,7 +32,8 @@
 //           * online softmax per query head and group; at the end of each
 //             head the two groups' states are merged by log-sum-exp;
 //           * p as bf16 hi+lo parts -> O = C_V^T P (kind::f16, C_V tile read
-//             MN-major in place), accumulated with the running rescale.
+//             MN-major in place; for exact rows O = V^T P with M = d),
+//             accumulated with the running rescale.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // ISKV status bit 2, stops, drains its copies and frees its TMEM.
 #include "iskv_internal.cuh"
@@ -44,6 +48,7 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;
+constexpr int kWinTile = 64;     // exact-row tiles: 64 rows never wrap the ring
 constexpr int kThreads = 320;
 constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
 constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
@@ -60,7 +65,7 @@ struct __align__(8) Bars {
 };
 
 struct SmemPlan {
-    uint32_t bk, stage, stage_k, qb, pb, total;
+    uint32_t bk, stage, stage_k, stage_bytes, qb, pb, total;
 };
 
 __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk) {
@@ -68,7 +73,10 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk) {
     uint32_t off = 1024;                                        // barriers, scratch
     p.bk = off;                off += nbk * (2 * kTile * rK * 2);  // nbk heads x (hi, lo)
     p.stage_k = (uint32_t)kTile * rK * 2;
-    p.stage = off;             off += ns * (p.stage_k + kTile * rV * 2 + 1024);
+    uint32_t sb = p.stage_k + kTile * rV * 2;
+    if (sb < 2 * kWinTile * kHeadDim * 2) sb = 2 * kWinTile * kHeadDim * 2;   // exact K and V rows
+    p.stage_bytes = sb + 1024;
+    p.stage = off;             off += ns * p.stage_bytes;
     p.qb = off;                off += 2 * (kQN * kTile * 4);
     p.pb = off;                off += 2 * (kPN * kTile * 2);
     p.total = off;
@@ -113,13 +121,16 @@ decode_tc_kernel(DecodeTcArgs a) {
     volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);
     volatile int* flag_max = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2]
     float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
+    float* mlx = reinterpret_cast<float*>(smem + 256);          // [2 groups][m 8 | l 8]
     const SmemPlan P = plan_smem(rK, rV, ns, nbk);
     float* sq = reinterpret_cast<float*>(smem + P.total);       // queries of the head, g x d fp32
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
     uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
-    const uint32_t stage_bytes = P.stage_k + kTile * rV * 2 + 1024;
+    const uint32_t stage_bytes = P.stage_bytes;
+    const int tiles_c = a.tiles_c;
+    constexpr uint32_t kWinBytes = kWinTile * kHeadDim * 2;   // one of K, V
     const uint32_t bk_bytes = 2 * kTile * rK * 2;
 
     if (warp == 1) {
@@ -194,13 +205,26 @@ decode_tc_kernel(DecodeTcArgs a) {
                     break;
                 }
                 uint8_t* sk = stage + st * stage_bytes;
-                const __nv_bfloat16* gk = reinterpret_cast<const __nv_bfloat16*>(a.K.coef) +
-                                          hidx * a.K.n_max * rK + (int64_t)tile * kTile * rK;
-                const __nv_bfloat16* gv = reinterpret_cast<const __nv_bfloat16*>(a.V.coef) +
-                                          hidx * a.V.n_max * rV + (int64_t)tile * kTile * rV;
-                mbar_arrive_expect_tx(&bars->full[st], P.stage_k + kTile * rV * 2);
-                bulk_g2s(sk, gk, P.stage_k, &bars->full[st]);
-                bulk_g2s(sk + P.stage_k, gv, kTile * rV * 2, &bars->full[st]);
+                if (tile < tiles_c) {
+                    const __nv_bfloat16* gk = reinterpret_cast<const __nv_bfloat16*>(a.K.coef) +
+                                              hidx * a.K.n_max * rK + (int64_t)tile * kTile * rK;
+                    const __nv_bfloat16* gv = reinterpret_cast<const __nv_bfloat16*>(a.V.coef) +
+                                              hidx * a.V.n_max * rV + (int64_t)tile * kTile * rV;
+                    mbar_arrive_expect_tx(&bars->full[st], P.stage_k + kTile * rV * 2);
+                    bulk_g2s(sk, gk, P.stage_k, &bars->full[st]);
+                    bulk_g2s(sk + P.stage_k, gv, kTile * rV * 2, &bars->full[st]);
+                } else {
+                    // exact rows j0..j0+63 sit in ring slots j0 % cap.. (no wrap: cap % 64 == 0)
+                    const int64_t j0 = a.n_c + (int64_t)(tile - tiles_c) * kWinTile;
+                    const int64_t slot0 = j0 % a.K.cap;
+                    const __nv_bfloat16* rk = reinterpret_cast<const __nv_bfloat16*>(a.K.ring) +
+                                              (hidx * a.K.cap + slot0) * d;
+                    const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(a.V.ring) +
+                                              (hidx * a.V.cap + slot0) * d;
+                    mbar_arrive_expect_tx(&bars->full[st], 2 * kWinBytes);
+                    bulk_g2s(sk, rk, kWinBytes, &bars->full[st]);
+                    bulk_g2s(sk + kWinBytes, rv, kWinBytes, &bars->full[st]);
+                }
                 issued = n + 1;
             }
             if (*abort_flag) {
@@ -235,17 +259,22 @@ decode_tc_kernel(DecodeTcArgs a) {
                     fail();
                     break;
                 }
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(stage + st * stage_bytes);
-                const uint32_t b0 = smem_u32(bk + (hs % nbk) * bk_bytes);
-                const uint32_t dk = tmem + b * kBufCols;
-                for (int ks = 0; ks < rK / 16; ++ks)
-                    for (int part = 0; part < 2; ++part) {
-                        const uint64_t ad = desc_noswizzle(a0 + ks * 256, 128, sbo);
-                        const uint64_t bd = desc_noswizzle(b0 + part * (kTile * rK * 2) + ks * 256, 128, sbo);
-                        mma_f16_ss(dk, ad, bd, idesc, (ks | part) != 0);
-                    }
-                mma_commit(&bars->kh_full[b]);
+                if ((int)(fi % tph) >= tiles_c) {
+                    // exact rows: nothing to rebuild, the epilogue reads them directly
+                    mbar_arrive(&bars->kh_full[b]);
+                } else {
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(stage + st * stage_bytes);
+                    const uint32_t b0 = smem_u32(bk + (hs % nbk) * bk_bytes);
+                    const uint32_t dk = tmem + b * kBufCols;
+                    for (int ks = 0; ks < rK / 16; ++ks)
+                        for (int part = 0; part < 2; ++part) {
+                            const uint64_t ad = desc_noswizzle(a0 + ks * 256, 128, sbo);
+                            const uint64_t bd = desc_noswizzle(b0 + part * (kTile * rK * 2) + ks * 256, 128, sbo);
+                            mma_f16_ss(dk, ad, bd, idesc, (ks | part) != 0);
+                        }
+                    mma_commit(&bars->kh_full[b]);
+                }
                 const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
                 if (seg_end) mma_commit(&bars->bk_empty[hs % nbk]);
             }
@@ -285,6 +314,7 @@ decode_tc_kernel(DecodeTcArgs a) {
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
         const uint32_t idesc_s = idesc_f32acc(2, kTile, kQN, 0, 0);
         const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 0);
+        const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 0);   // exact rows: M = d
         const uint32_t sbo_q = (kTile / 4) * 128;
         const uint32_t sbo_p = (kTile / 8) * 128;
         const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
@@ -293,7 +323,17 @@ decode_tc_kernel(DecodeTcArgs a) {
         uint32_t* qbb = qb + grp * kQN * kTile;
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
 
-        float m_run[G], l_thr[G], acc[G], alpha[G];
+        float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
+        // acc <- acc * alpha + (p^T C_V of a folded tile); accd likewise for exact tiles
+        // (both rescaled every tile: they share the running max)
+        auto accumulate = [&](const uint32_t (&o)[16], bool was_win) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float add = __uint_as_float(o[h]) + __uint_as_float(o[G + h]);
+                acc[h] = (acc_ok && !was_win) ? fmaf(acc[h], alpha[h], add) : acc[h] * alpha[h];
+                accd[h] = was_win ? fmaf(accd[h], alpha[h], add) : accd[h] * alpha[h];
+            }
+        };
         bool stop = false;
         int n0 = 0;
         while (n0 < ntiles) {
@@ -312,6 +352,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 m_run[h] = -INFINITY;
                 l_thr[h] = 0.f;
                 acc[h] = 0.f;
+                accd[h] = 0.f;
                 alpha[h] = 0.f;
             }
             if (ept == 0) *epi_abort = *abort_flag;
@@ -320,12 +361,16 @@ decode_tc_kernel(DecodeTcArgs a) {
             tc_fence_after();
             stop = *epi_abort;                    // latched after the barrier: uniform
             if (stop) break;
-            bool have_prev = false;
+            bool have_prev = false, prev_win = false;
             int last = -1;
             for (int n = n0 + ((n0 & 1) != grp ? 1 : 0); n < s1; n += 2) {
                 const int st = n % ns;
-                const int64_t j0 = (int64_t)((f0 + n) % tph) * kTile;
-                const int valid = (int)((a.n_c - j0) < kTile ? (a.n_c - j0) : kTile);
+                const int local = (int)((f0 + n) % tph);
+                const bool win = local >= tiles_c;    // exact rows (64-token tile)
+                const int64_t j0 = win ? a.n_c + (int64_t)(local - tiles_c) * kWinTile : (int64_t)local * kTile;
+                const int64_t lim = win ? a.T : a.n_c;
+                const int span = win ? kWinTile : kTile;
+                const int valid = (int)((lim - j0) < span ? (lim - j0) : span);
                 // q' = R_{j0}^T q, tf32 hi / lo parts as the score MMA's B operand
                 for (int item = gt; item < g * 64; item += 128) {
                     const int h = item >> 6, i = item & 63;
@@ -348,11 +393,33 @@ decode_tc_kernel(DecodeTcArgs a) {
                 // rotate this row of K^ by R_t, store back as tf32
                 if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
+                if (win && !mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) fail();
+                const uint4* krow = reinterpret_cast<const uint4*>(stage + st * stage_bytes);
 #pragma unroll
                 for (int c0 = 0; c0 < 64; c0 += 16) {
                     uint32_t x1[16], x2[16], cc[16], ss[16];
-                    tmem_ld16(kh + lane_base + c0, x1);
-                    tmem_ld16(kh + lane_base + 64 + c0, x2);
+                    if (!win) {
+                        tmem_ld16(kh + lane_base + c0, x1);
+                        tmem_ld16(kh + lane_base + 64 + c0, x2);
+                    } else {
+                        // this row's exact key, dims c0.. and 64 + c0.. (blocked 8 x 8 layout)
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                            for (int v = 0; v < 2; ++v) {
+                                uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
+                                if (row < valid)
+                                    q4 = krow[((row >> 3) * 16 + ((half * 64 + c0) >> 3) + v) * 8 + (row & 7)];
+                                uint32_t* dst = half ? x2 : x1;
+                                const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    dst[v * 8 + 2 * e] = w4[e] << 16;            // low bf16 -> fp32
+                                    dst[v * 8 + 2 * e + 1] = w4[e] & 0xFFFF0000u; // high bf16 -> fp32
+                                }
+                            }
+                        }
+                    }
                     tmem_ld16(tcs + lane_base + c0, cc);
                     tmem_ld16(tcs + lane_base + 64 + c0, ss);
                     tmem_wait_ld();
@@ -384,11 +451,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                     uint32_t o[16];
                     tmem_ld16(kh + 144 + lane_base, o);
                     tmem_wait_ld();
-                    if (acc_ok) {
-#pragma unroll
-                        for (int h = 0; h < G; ++h)
-                            acc[h] = fmaf(acc[h], alpha[h], __uint_as_float(o[h]) + __uint_as_float(o[G + h]));
-                    }
+                    accumulate(o, prev_win);
                 }
                 // scores and the tile max of each head
                 if (!mbar_wait(&bars->s_full[grp], (n >> 1) & 1, deadline)) fail();
@@ -425,15 +488,24 @@ decode_tc_kernel(DecodeTcArgs a) {
                 if (gt == 0 && !*abort_flag) {
                     mbar_arrive(&bars->kfree[grp]);   // K^/S of this buffer may be overwritten
                     tc_fence_after();
-                    const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
                     const uint32_t p0 = smem_u32(pbb);
-                    for (int ks = 0; ks < kTile / 16; ++ks)
-                        mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
-                                   desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_o, ks != 0);
+                    if (!win) {
+                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
+                        for (int ks = 0; ks < kTile / 16; ++ks)
+                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
+                                       desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_o, ks != 0);
+                    } else {
+                        // O = V^T P over 64 exact rows: A = V tile, MN-major, M = d
+                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + kWinBytes);
+                        for (int ks = 0; ks < kWinTile / 16; ++ks)
+                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
+                                       desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_ow, ks != 0);
+                    }
                     mma_commit(&bars->o_full[grp]);
                     mma_commit(&bars->empty[st]);
                 }
                 have_prev = true;
+                prev_win = win;
                 last = n;
             }
             // close this group's share of the head
@@ -443,11 +515,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 uint32_t o[16];
                 tmem_ld16(kh + 144 + lane_base, o);
                 tmem_wait_ld();
-                if (acc_ok) {
-#pragma unroll
-                    for (int h = 0; h < G; ++h)
-                        acc[h] = fmaf(acc[h], alpha[h], __uint_as_float(o[h]) + __uint_as_float(o[G + h]));
-                }
+                accumulate(o, prev_win);
             }
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -458,42 +526,47 @@ decode_tc_kernel(DecodeTcArgs a) {
             group_sync(grp);
             // a group's softmax state goes to its own q' buffer, idle now that
             // its last score MMA of the head has completed: [m 8 | l 8 | acc 8 x 128]
-            static_assert((2 * kMaxGroup + kMaxGroup * kHeadDim) <= kQN * kTile, "exchange fits");
-            float* xg = reinterpret_cast<float*>(qbb);
+            static_assert(2 * kMaxGroup * kHeadDim <= kQN * kTile, "exchange fits");
+            float* xg = reinterpret_cast<float*>(qbb);       // [acc 8 x 128 | accd 8 x 128]
+            float* xml = mlx + grp * 2 * kMaxGroup;          // [m 8 | l 8]
             if (gt == 0) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    xg[h] = m_run[h];
-                    xg[kMaxGroup + h] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
+                    xml[h] = m_run[h];
+                    xml[kMaxGroup + h] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
                 }
             }
-            if (acc_ok) {
 #pragma unroll
-                for (int h = 0; h < G; ++h) xg[2 * kMaxGroup + h * kHeadDim + c_acc] = acc[h];
+            for (int h = 0; h < G; ++h) {
+                if (acc_ok) xg[h * kHeadDim + c_acc] = acc[h];
+                xg[(kMaxGroup + h) * kHeadDim + row] = accd[h];
             }
             epi_sync();                               // both groups published
             if (grp == 0) {
                 // log-sum-exp merge of the two groups, one partial slot per head
                 const float* x0 = reinterpret_cast<const float*>(qb);
                 const float* x1 = reinterpret_cast<const float*>(qb + kQN * kTile);
+                const float* ml0 = mlx;
+                const float* ml1 = mlx + 2 * kMaxGroup;
                 const int bq = head / a.Hkv, kvh = head % a.Hkv;
                 const int c_first = (int)(((int64_t)head * tph) / a.tiles_per_cta);
                 const int slot = cta - c_first;
                 const int stride = 2 + rV + d;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    const float m0 = x0[h], m1 = x1[h];
+                    const float m0 = ml0[h], m1 = ml1[h];
                     const float M = fmaxf(m0, m1);
                     const float w0 = (m0 == -INFINITY) ? 0.f : __expf(m0 - M);
                     const float w1 = (m1 == -INFINITY) ? 0.f : __expf(m1 - M);
                     float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
                     if (acc_ok)
-                        Pp[2 + c_acc] = x0[2 * kMaxGroup + h * kHeadDim + c_acc] * w0 +
-                                        x1[2 * kMaxGroup + h * kHeadDim + c_acc] * w1;
-                    Pp[2 + rV + gt] = 0.f;            // d = 128 = group size
+                        Pp[2 + c_acc] = x0[h * kHeadDim + c_acc] * w0 + x1[h * kHeadDim + c_acc] * w1;
+                    // d = 128 = group size: thread gt owns dim gt of the exact-row sum
+                    Pp[2 + rV + gt] = x0[(kMaxGroup + h) * kHeadDim + gt] * w0 +
+                                      x1[(kMaxGroup + h) * kHeadDim + gt] * w1;
                     if (gt == 0) {
                         Pp[0] = M;
-                        Pp[1] = x0[kMaxGroup + h] * w0 + x1[kMaxGroup + h] * w1;
+                        Pp[1] = ml0[kMaxGroup + h] * w0 + ml1[kMaxGroup + h] * w1;
                     }
                 }
                 // this CTA ends the head: mark the head's unused compressed slots empty

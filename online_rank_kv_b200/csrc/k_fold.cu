@@ -110,7 +110,7 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
     }
     for (int e = tid; e < b * d; e += kThreads) {
         int t = e / d, i = e % d;
-        sM[(r + t) * d + i] = to_f32(ring[(slot0 + t) * d + i]);
+        sM[(r + t) * d + i] = to_f32(ring[coef_index(f.ring_blocked, d, slot0 + t, i)]);
     }
     for (int e = tid; e < m * n; e += kThreads) sA[e] = 0.f;
     __syncthreads();

@@ -24,9 +24,11 @@ __global__ void init_factor_kernel(FactorView f, int layers) {
     }
 }
 
-// ring[bh][(T0 + t) mod cap][:] = src[bh][t][:], 16-byte vectors.
+// ring[bh][(T0 + t) mod cap][:] = src[bh][t][:], 16-byte vectors; with
+// `blocked` (bf16 rows of 128) the destination is the 8x8 core-matrix layout:
+// vector v of slot s lands at ((s / 8) * 16 + v) * 8 + s % 8.
 __global__ void append_kernel(uint4* ring, const uint4* src, int BH, int t, int64_t T0,
-                              int64_t cap, int vec_per_row) {
+                              int64_t cap, int vec_per_row, int blocked) {
     const int64_t total = (int64_t)BH * t * vec_per_row;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -34,7 +36,9 @@ __global__ void append_kernel(uint4* ring, const uint4* src, int BH, int t, int6
         const int64_t row = e / vec_per_row;
         const int64_t bh = row / t, tt = row % t;
         const int64_t slot = (T0 + tt) % cap;
-        ring[(bh * cap + slot) * vec_per_row + v] = src[e];
+        const int64_t dst = blocked ? bh * cap * vec_per_row + ((slot >> 3) * vec_per_row + v) * 8 + (slot & 7)
+                                    : (bh * cap + slot) * vec_per_row + v;
+        ring[dst] = src[e];
     }
 }
 
@@ -109,7 +113,7 @@ cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s) 
 }
 
 cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0, int64_t cap,
-                          int elem_bytes, cudaStream_t s) {
+                          int elem_bytes, int blocked, cudaStream_t s) {
     const int vec_per_row = kHeadDim * elem_bytes / 16;
     const int64_t total = (int64_t)BH * t * vec_per_row;
     int64_t blocks = (total + 255) / 256;
@@ -117,7 +121,7 @@ cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0
     if (blocks < 1) blocks = 1;
     append_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(ring),
                                                    reinterpret_cast<const uint4*>(src), BH, t, T0,
-                                                   cap, vec_per_row);
+                                                   cap, vec_per_row, blocked);
     return cudaGetLastError();
 }
 

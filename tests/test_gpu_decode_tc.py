@@ -97,3 +97,19 @@ def test_tc_decode_recall_query():
     q = q.to(torch.bfloat16)
     errs, _ = p.decode(0, q)
     assert max(errs.values()) < TOL_BF16, errs
+
+
+def test_tc_decode_without_folded_rows():
+    """Nothing folded yet (T < W + 64): only exact-row tiles, including a
+    ragged last tile, go through the tensor-core kernel."""
+    cfg = _cfg(window=512, max_tokens=1024)
+    pt = _pair(True, cfg, seed=47)
+    pc = _pair(False, cfg, seed=47)
+    pt.prefill(300, chunk=100)
+    pc.prefill(300, chunk=100)
+    assert pt.cache.counts(0) == (300, 0)
+    q = pt.query()
+    errs, out_t = pt.decode(0, q)
+    out_c = pc.cache.decode_attention(0, q.cuda()).cpu().numpy()
+    assert max(errs.values()) < 1e-3, errs
+    assert rel_err(out_t, out_c) < 5e-3
