@@ -5,7 +5,7 @@ Argument marshalling only: tensors become raw pointers, the current CUDA
 stream becomes the ``stream`` argument, status codes become exceptions.
 Every step of the method runs in the library's kernels; there is no CPU or
 PyTorch fallback, and importing this package fails loudly when the compiled
-library is missing (build it with ``python -m online_rank_kv_b200.build``).
+library is missing (build it with ``python online_rank_kv_b200/build.py``).
 """
 
 from __future__ import annotations
@@ -29,7 +29,7 @@ def lib_path() -> str:
 if not os.path.exists(lib_path()):
     raise ImportError(
         f"{lib_path()} is missing: build the CUDA library first "
-        "(python -m online_rank_kv_b200.build)")
+        "(python online_rank_kv_b200/build.py)")
 
 LIB = ctypes.CDLL(lib_path())
 

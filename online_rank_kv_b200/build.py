@@ -1,6 +1,7 @@
 """Build the in-tree CUDA library ``libiskv.so`` for sm_100a with nvcc.
 
-Usage: ``python -m online_rank_kv_b200.build`` (or ``build()`` from Python).
+Usage: ``python online_rank_kv_b200/build.py`` (or ``build()`` from Python, with
+this file loaded on its own: importing the package needs the built library).
 Sources are every ``csrc/*.cu``; the result lands next to this file so it
 travels with the repository snapshot.  Objects are cached under ``_build/``
 and rebuilt when a source or header is newer than its object.

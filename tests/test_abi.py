@@ -15,8 +15,12 @@ HEADER = os.path.join(ROOT, "include", "iskv.h")
 def _lib():
     so = os.path.join(ROOT, "online_rank_kv_b200", "libiskv.so")
     if not os.path.exists(so):
-        from online_rank_kv_b200.build import build
-        build()
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(
+            "_iskv_build", os.path.join(ROOT, "online_rank_kv_b200", "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
     import online_rank_kv_b200 as ik
     return ik
 
