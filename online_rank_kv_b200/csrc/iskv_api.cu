@@ -40,6 +40,8 @@ struct iskv_cache {
     float* sigma_v = nullptr;
     float* pend_k = nullptr;
     float* pend_v = nullptr;
+    float* qscr_k = nullptr;      // fold scratch: Q of every (layer, head)
+    float* qscr_v = nullptr;
     int* seg_rows = nullptr;
     float* partial = nullptr;
     float2* rope = nullptr;
@@ -128,7 +130,7 @@ int64_t ready_of(const iskv_cache* h, int layer) {
 void free_all(iskv_cache* h) {
     void* ptrs[] = {h->ring_k, h->ring_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
-                    h->seg_rows, h->partial, h->rope, h->status, h->stage_in, h->stage_out};
+                    h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->rope, h->status, h->stage_in, h->stage_out};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -261,6 +263,8 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     rc = rc ? rc : dalloc(&h->sigma_v, heads * c.rank_v * 4);
     rc = rc ? rc : dalloc(&h->pend_k, heads * h->D * (size_t)c.rank_k * c.rank_k * 4);
     rc = rc ? rc : dalloc(&h->pend_v, heads * h->D * (size_t)c.rank_v * c.rank_v * 4);
+    rc = rc ? rc : dalloc(&h->qscr_k, heads * d * fold_q_cols(c.rank_k) * 4);
+    rc = rc ? rc : dalloc(&h->qscr_v, heads * d * fold_q_cols(c.rank_v) * 4);
     rc = rc ? rc : dalloc(&h->seg_rows, (size_t)c.layers * h->D * 4);
     rc = rc ? rc : dalloc(&h->partial, (size_t)c.batch * c.q_heads * h->max_splits *
                                            (2 + c.rank_v + d) * 4);
@@ -381,7 +385,10 @@ int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
         fl.slot[fl.n_tasks] = defer ? h->n_pend[l] : 0;
         ++fl.n_tasks;
     }
-    for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) CU(launch_fold(view(h, which), fl, h->status, s));
+    for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) {
+        fl.qscratch = which == ISKV_WHICH_K ? h->qscr_k : h->qscr_v;
+        CU(launch_fold(view(h, which), fl, h->status, s));
+    }
     std::vector<int> rl_layers, rl_seg, rl_rows;
     for (int l : fold_layers) {
         const bool defer = h->cfg.sync && (want_defer || h->n_pend[l] > 0);

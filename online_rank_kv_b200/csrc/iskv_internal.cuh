@@ -85,6 +85,7 @@ struct FoldLaunch {
     int n_c[kMaxLayers];         // n_c before the fold
     int slot[kMaxLayers];        // postponed-fold slot receiving W_r[0:r,:]
     int max_sweeps;
+    float* qscratch;             // [L][BH][d][k] fp32: Q of the fold in flight
 };
 
 struct ResyncLaunch {
@@ -154,5 +155,6 @@ bool decode_tc_supports_group(int g);
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk);
 
 size_t fold_smem_bytes(int r);
+int fold_q_cols(int r);   // k = min(64, d - r): columns of Q
 
 }  // namespace iskv

@@ -5,417 +5,857 @@
 // ("iS-KV -- Basis-synchronized online low-rank KV compression -- What does it
 // mean?", Jargon: Block-incremental SVD; body paragraph on the joint update of
 // basis and coefficients on a small core whose size does not depend on the
-// history length).  Steps inside the CTA, all in shared memory, fp32:
-//   (a) P = X B                                   (warp dot products)
-//   (b) Householder QR of [B | X^T] (d x (r+64)); its first r reflections
+// history length).  Steps inside the CTA, fp32, every intermediate in shared
+// memory or registers:
+//   (a) P = X B.
+//   (b) Householder QR of [B | X^T] (d x (r+64)).  Its first r reflections
 //       remove the B-components, i.e. they form the residual E = X - P B^T
-//       implicitly.  Q = columns r..r+k-1 of the orthogonal factor
-//       (k = min(64, d - r)), R_E = rows r..r+k-1 of the triangular factor
-//       over the X^T columns; this keeps [B, Q] orthonormal even when
-//       r + 64 > d or the residual is rank deficient.
-//   (c) core A = [[diag S, 0], [P, R_E^T]] ((r+64) x (r+k)); one-sided
-//       (Hestenes) Jacobi with accumulated right vectors V: each warp rotates
-//       one column pair, n/2 disjoint pairs per round (circle ordering),
-//       sweeps until no pair needs a rotation.  Singular values are the final
-//       column norms, sorted descending.
-//       fp32 rotations [[c, s], [-s, c]] keep the two columns exactly
-//       orthogonal but scale them by c^2 + s^2 (a few ulp off 1); after the
-//       sweeps every column of V is renormalized (and its column of A = K V
-//       with it) so this scaling does not compound over hundreds of folds.
-//   (d) S' = sigma_1..r, new coefficient rows = rows r.. of A V (first r
-//       sorted columns), W_top = V[0:r, perm[0:r]] for step (e),
-//       B' = [B, Q] V[:, perm[0:r]], followed by one Bjorck step
-//       B' <- B' (3I - B'^T B') / 2 that restores orthonormality to fp32
-//       rounding (a no-op in exact arithmetic), written as fp32 plus bf16
-//       hi/lo parts.
+//       implicitly; Q = columns r..r+k-1 of the orthogonal factor
+//       (k = min(64, d - r)) and R_E = rows r..r+k-1 of the triangular
+//       factor over the X^T columns.  This keeps [B, Q] orthonormal even when
+//       r + 64 > d or the residual is rank deficient.  Q is formed in place
+//       (backward accumulation of the reflectors) and parked in a global
+//       scratch slot until step (d).
+//   (c) SVD of the core K = [[diag S, 0], [P, R_E^T]] ((r+64) x n, n = r+k):
+//         - Householder QR of K, exploiting that column j < r of K has
+//           nonzeros only in row j and rows r..r+63: K = Q_K R (R n x n);
+//         - one-sided (Hestenes) Jacobi on the columns of R^T.  With
+//           R^T J = U Sigma, R = J Sigma U^T, so U holds the right singular
+//           vectors of K: no rotation has to be accumulated, and the
+//           QR-preconditioned Jacobi needs about 7 sweeps where Jacobi on K
+//           itself needs 8 and Jacobi on K^T 11-12;
+//         - the columns live in registers, eight per block, two blocks per
+//           warp: each round rotates eight disjoint pairs of the warp's two
+//           blocks (all pairs inside each block once per sweep, then all
+//           cross pairs), and blocks travel between warps in the round-robin
+//           (circle) order, so every pair of columns meets once per sweep;
+//         - column norms are carried through the sweep by the exact update
+//           of the rotation and recomputed at its start; a pair is rotated
+//           while |a_p . a_q| > tol |a_p| |a_q|; columns whose energy is
+//           below 1e-14 ||K||_F^2 are numerically zero and never rotated.
+//       sigma = final column norms, sorted descending; W_r = the matching
+//       unit columns.  Directions of numerically zero singular values (rank
+//       of K below r) are completed by orthonormal vectors (any completion
+//       is a correct truncation: K maps all of them to zero).  One Bjorck
+//       step W_r <- W_r (3I - W_r^T W_r)/2 restores orthonormality to fp32
+//       rounding (a no-op in exact arithmetic).
+//   (d) S' = sigma_1..r; W_top = W_r[0:r, :] for step (e);
+//       B'' = [B, Q] W_r; new coefficient rows = X B'' (equal to
+//       [P, R_E^T] W_r in exact arithmetic: X [B, Q] = [P, R_E^T] because
+//       [B, Q] spans the rows of X); B' = B'' after one Bjorck step, written
+//       as fp32 plus bf16 hi/lo parts.
+// Step (e), the rewrite of the stored coefficients, runs in the resync
+// kernels.
+#include <utility>
+
 #include "iskv_internal.cuh"
 
 namespace iskv {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr unsigned kFull = 0xffffffffu;
 
-struct Dims {
-    int r, k, m, n, c, nrefl;
+// smallest stride >= cols that is 8 (mod 32): 4 row-parts x 8 consecutive
+// columns of one warp then hit 32 distinct banks
+__host__ __device__ constexpr int stride8(int cols) { return cols + ((8 - cols % 32) + 32) % 32; }
+
+template <int R>
+struct Geo {
+    static constexpr int d = kHeadDim;
+    static constexpr int b = kBlock;
+    static constexpr int k = (d - R) < b ? (d - R) : b;   // Q columns
+    static constexpr int m = R + b;                         // core rows
+    static constexpr int n = R + k;                         // core columns
+    static constexpr int c = R + b;                         // columns of [B | X^T]
+    static constexpr int ldm = stride8(c);
+    static constexpr int ldk = stride8(n);
+    static constexpr int NR = n <= 96 ? 3 : 4;              // Jacobi rows per lane
+    static constexpr int npad = 32 * NR;
+    static constexpr int nwj = n / 16;                      // Jacobi warps (two 8-column blocks each)
+    static constexpr int nb = n / 8;                        // Jacobi blocks
+    static constexpr int ldw = R + 4;                       // W_r / B' staging stride (16-byte rows)
+    static constexpr int ldp = R + 4;                       // P stride
+    // region A: [B | X^T], then the core, the Jacobi exchange buffer, two
+    // d x R staging slots
+    static constexpr int regA0 = d * ldm > m * ldk ? d * ldm : m * ldk;
+    static constexpr int regA1 = n * npad > 2 * d * ldw ? n * npad : 2 * d * ldw;
+    static constexpr int regA = regA0 > regA1 ? regA0 : regA1;
+    // aux: P and R_E, later the r x r Gram matrices of the Bjorck steps
+    static constexpr int aux0 = b * ldp + k * b;
+    static constexpr int aux = aux0 > R * ldw ? aux0 : R * ldw;
+    // small arrays (floats): tau/vd/al of both QRs, 2 norms, sigma^2, rank,
+    // per-warp norms and rotation parameters, exchanged norms, flags
+    static constexpr int small = 6 * 128 + 4 + 128 + 128 + kWarps * 16 + kWarps * 16 + 128 + 16 + 128;
+    static constexpr int floats = regA + aux + small;
+    static_assert(n % 16 == 0 && n <= 128 && npad >= n, "core shape");
+    static_assert(R % 16 == 0 && R >= 16 && R <= 128, "rank");
 };
-
-__host__ __device__ inline Dims dims_for(int r) {
-    Dims x;
-    x.r = r;
-    x.k = (kHeadDim - r) < kBlock ? (kHeadDim - r) : kBlock;
-    x.m = r + kBlock;      // core rows
-    x.n = r + x.k;         // core columns
-    x.c = r + kBlock;      // columns of [B | X^T]
-    x.nrefl = r + x.k;     // reflections needed (<= d)
-    return x;
-}
-
-struct Layout {
-    size_t R1, R2, Q, small;
-};
-
-__host__ __device__ inline Layout layout_for(const Dims& x) {
-    Layout L;
-    size_t qr = (size_t)kHeadDim * x.c;
-    size_t vv = (size_t)x.n * x.n;
-    L.R1 = qr > vv ? qr : vv;               // [B|X^T] during QR, V afterwards
-    L.R2 = (size_t)x.m * x.n;               // core A, then B' staging
-    L.Q = (size_t)kHeadDim * x.k;
-    L.small = 2 * (size_t)x.c + 2 * (size_t)x.n + 8;
-    return L;
-}
 
 // Off-diagonal threshold of the one-sided Jacobi: a pair (p, q) is rotated
 // while |a_p . a_q| > tol * |a_p| |a_q|.
-__device__ __forceinline__ float jacobi_tol(int m) { return 4.0e-7f * sqrtf((float)m); }
+__device__ __forceinline__ float jacobi_tol(int len) { return 4.0e-7f * sqrtf((float)len); }
 
-template <typename KvT, typename CoefT>
-__global__ void __launch_bounds__(kThreads, 1)
+// ---------------------------------------------------------------------------
+// Householder QR in place of the rows x cols row-major matrix A (stride lda,
+// 8 mod 32), reflections j = 0..nrefl-1.  Below its diagonal, column j is
+// nonzero only in rows [max(j + 1, lo), rows) (lo = 0: dense), and every
+// reflection touches only row j and those rows.  H_j = I - tau_j v v^T with
+// v = (vd_j at row j, A[i][j] below); al_j = R[j][j].  The diagonal element
+// A[j][j] keeps its value from before reflection j; the upper triangle of A
+// becomes R.  Thread (warp, lane) owns column 8*warp + (lane & 7) of each
+// 64-column pass and the rows i = i0 + (lane >> 3) (mod 4).
+// ---------------------------------------------------------------------------
+__device__ void house_qr(float* A, int lda, int rows, int cols, int nrefl, int lo, float* tau,
+                         float* vd, float* al, float* nrm2) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int col = lane & 7, part = lane >> 3;
+    if (warp == 0) {
+        float s = 0.f;
+        for (int i = (lo > 1 ? lo : 1) + lane; i < rows; i += 32) s = fmaf(A[i * lda], A[i * lda], s);
+        s = warp_sum(s);
+        if (lane == 0) nrm2[0] = s;
+    }
+    __syncthreads();
+    for (int j = 0; j < nrefl; ++j) {
+        const float s = nrm2[j & 1];
+        const float ajj = A[j * lda + j];
+        float tj = 0.f, vj = 1.f, aj = ajj;
+        if (s > 0.f) {
+            const float nr = sqrtf(fmaf(ajj, ajj, s));
+            aj = -copysignf(nr, ajj);
+            vj = ajj - aj;
+            tj = 2.f / fmaf(vj, vj, s);
+        }
+        if (tid == 0) {
+            tau[j] = tj;
+            vd[j] = vj;
+            al[j] = aj;
+        }
+        const int i0 = (j + 1 > lo) ? j + 1 : lo;
+        const int inext = (j + 2 > lo) ? j + 2 : lo;   // rows of column j+1's next norm
+        for (int cb = j + 1 + warp * 8; cb < cols; cb += kWarps * 8) {
+            const int cc = cb + col;
+            const bool act = cc < cols;
+            float w = 0.f;
+            if (act) {
+                if (part == 0) w = vj * A[j * lda + cc];
+                for (int i = i0 + part; i < rows; i += 4) w = fmaf(A[i * lda + j], A[i * lda + cc], w);
+            }
+            w += __shfl_xor_sync(kFull, w, 8);
+            w += __shfl_xor_sync(kFull, w, 16);
+            const float tw = tj * w;
+            float sq = 0.f;
+            if (act) {
+                if (part == 0) A[j * lda + cc] = fmaf(-tw, vj, A[j * lda + cc]);
+                for (int i = i0 + part; i < rows; i += 4) {
+                    const float x = fmaf(-tw, A[i * lda + j], A[i * lda + cc]);
+                    A[i * lda + cc] = x;
+                    if (i >= inext) sq = fmaf(x, x, sq);
+                }
+            }
+            sq += __shfl_xor_sync(kFull, sq, 8);
+            sq += __shfl_xor_sync(kFull, sq, 16);
+            if (act && part == 0 && cc == j + 1) nrm2[(j + 1) & 1] = sq;
+        }
+        __syncthreads();
+    }
+}
+
+// Columns r..r+k-1 of the QR'd [B | X^T] (d x (r+64), stride lda) become
+// Q = H_0 ... H_{n-1} [e_r .. e_{r+k-1}], n = r + k: backward accumulation.
+// A column c of the block is set to H_c e_c the first time a reflection
+// reaches it (reflection c - 1); its strictly upper part (R entries, saved
+// beforehand) is cleared first.
+__device__ void form_q(float* A, int lda, int r, int k, const float* tau, const float* vd) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int col = lane & 7, part = lane >> 3;
+    constexpr int d = kHeadDim;
+    const int n = r + k;
+    for (int e = tid; e < d * k; e += kThreads) {
+        const int i = e / k, q = e - (e / k) * k;
+        if (i < r + q) A[i * lda + r + q] = 0.f;
+    }
+    __syncthreads();
+    for (int j = n - 1; j >= 0; --j) {
+        const float tj = tau[j], vj = vd[j];
+        const int cc = (j >= r ? j + 1 : r) + warp * 8 + col;   // <= 64 target columns: one pass
+        const bool act = cc < n;
+        const bool init = act && cc == j + 1;
+        float ti = 0.f, vi = 0.f;
+        if (init) {
+            ti = tau[j + 1];
+            vi = vd[j + 1];
+        }
+        float w = 0.f;
+        if (act) {
+            if (part == 0) w = vj * A[j * lda + cc];
+            for (int i = j + 1 + part; i < d; i += 4) {
+                float y = A[i * lda + cc];
+                if (init) {
+                    y = (i == j + 1) ? fmaf(-ti * vi, vi, 1.f) : -ti * vi * y;
+                    A[i * lda + cc] = y;
+                }
+                w = fmaf(A[i * lda + j], y, w);
+            }
+        }
+        w += __shfl_xor_sync(kFull, w, 8);
+        w += __shfl_xor_sync(kFull, w, 16);
+        const float tw = tj * w;
+        if (act) {
+            if (part == 0) A[j * lda + cc] = fmaf(-tw, vj, A[j * lda + cc]);
+            for (int i = j + 1 + part; i < d; i += 4)
+                A[i * lda + cc] = fmaf(-tw, A[i * lda + j], A[i * lda + cc]);
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Register-resident block Jacobi.  Warp g holds blocks "top" (a[0..7]) and
+// "bot" (a[8..15]); lane l holds rows l + 32u of each column.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int circ8(int s, int pos) { return pos == 0 ? 0 : 1 + (pos - 1 + s) % 7; }
+// pair i (0..7) of round s: inside the blocks (pairs 0..3 in top, 4..7 in bot)
+// or across them
+__host__ __device__ constexpr int pair_p(bool within, int s, int i) {
+    return within ? (i < 4 ? circ8(s, i) : 8 + circ8(s, i - 4)) : i;
+}
+__host__ __device__ constexpr int pair_q(bool within, int s, int i) {
+    return within ? (i < 4 ? circ8(s, 7 - i) : 8 + circ8(s, 7 - (i - 4))) : 8 + (i + s) % 8;
+}
+
+struct JacobiCtx {
+    float* nrm;      // this warp's 16 column norms^2
+    float2* par;     // this warp's 8 rotation parameters
+    int* any;        // this warp's "rotated" flag
+    float tol, tiny;
+    int lane;
+};
+
+template <int NR, bool WITHIN, int S>
+__device__ __forceinline__ void jacobi_round(float (&a)[16][NR], const JacobiCtx& cx) {
+    float g[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int u = 0; u < NR; ++u) acc = fmaf(a[pair_p(WITHIN, S, i)][u], a[pair_q(WITHIN, S, i)][u], acc);
+        g[i] = acc;
+    }
+    // transpose-reduce: afterwards lane l holds the full dot product of pair (l >> 2) & 7
+    const int lane = cx.lane;
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = b4 ? g[i] : g[i + 4];
+        const float keep = b4 ? g[i + 4] : g[i];
+        h[i] = keep + __shfl_xor_sync(kFull, send, 16);
+    }
+    float h2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b3 ? h[i] : h[i + 2];
+        const float keep = b3 ? h[i + 2] : h[i];
+        h2[i] = keep + __shfl_xor_sync(kFull, send, 8);
+    }
+    float gm;
+    {
+        const float send = b2 ? h2[0] : h2[1];
+        const float keep = b2 ? h2[1] : h2[0];
+        gm = keep + __shfl_xor_sync(kFull, send, 4);
+    }
+    gm += __shfl_xor_sync(kFull, gm, 2);
+    gm += __shfl_xor_sync(kFull, gm, 1);
+
+    const int ip = (lane >> 2) & 7;
+    const int p = pair_p(WITHIN, S, ip), q = pair_q(WITHIN, S, ip);
+    const float al = cx.nrm[p], be = cx.nrm[q];
+    float cs = 1.f, sn = 0.f, nal = al, nbe = be;
+    if (fminf(al, be) > cx.tiny && fabsf(gm) > cx.tol * sqrtf(al * be)) {
+        const float zeta = (be - al) / (2.f * gm);
+        const float t = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
+        cs = 1.f / sqrtf(fmaf(t, t, 1.f));
+        sn = cs * t;
+        nal = fmaf(-t, gm, al);
+        nbe = fmaf(t, gm, be);
+    }
+    __syncwarp();
+    if ((lane & 3) == 0) {
+        cx.par[ip] = make_float2(cs, sn);
+        if (sn != 0.f) {
+            cx.nrm[p] = nal;
+            cx.nrm[q] = nbe;
+            *cx.any = 1;
+        }
+    }
+    __syncwarp();
+    const float4* pv = reinterpret_cast<const float4*>(cx.par);
+    float c8[8], s8[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 v = pv[i];
+        c8[2 * i] = v.x;
+        s8[2 * i] = v.y;
+        c8[2 * i + 1] = v.z;
+        s8[2 * i + 1] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (s8[i] != 0.f) {   // warp-uniform
+#pragma unroll
+            for (int u = 0; u < NR; ++u) {
+                const float x = a[pair_p(WITHIN, S, i)][u], y = a[pair_q(WITHIN, S, i)][u];
+                a[pair_p(WITHIN, S, i)][u] = fmaf(c8[i], x, -s8[i] * y);
+                a[pair_q(WITHIN, S, i)][u] = fmaf(s8[i], x, c8[i] * y);
+            }
+        }
+    }
+}
+
+template <int NR, bool WITHIN, int... Ss>
+__device__ __forceinline__ void jacobi_rounds(float (&a)[16][NR], const JacobiCtx& cx,
+                                              std::integer_sequence<int, Ss...>) {
+    (jacobi_round<NR, WITHIN, Ss>(a, cx), ...);
+}
+
+// Squared norms of the warp's 16 columns; lane l (even) gets column (l >> 1) & 15.
+template <int NR>
+__device__ __forceinline__ float col_norms16(const float (&a)[16][NR], int lane) {
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int u = 0; u < NR; ++u) s = fmaf(a[i][u], a[i][u], s);
+        x[i] = s;
+    }
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float send = b4 ? x[i] : x[i + 8];
+        y[i] = (b4 ? x[i + 8] : x[i]) + __shfl_xor_sync(kFull, send, 16);
+    }
+    float z[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = b3 ? y[i] : y[i + 4];
+        z[i] = (b3 ? y[i + 4] : y[i]) + __shfl_xor_sync(kFull, send, 8);
+    }
+    float w2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b2 ? z[i] : z[i + 2];
+        w2[i] = (b2 ? z[i + 2] : z[i]) + __shfl_xor_sync(kFull, send, 4);
+    }
+    float v;
+    {
+        const float send = b1 ? w2[0] : w2[1];
+        v = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(kFull, send, 2);
+    }
+    v += __shfl_xor_sync(kFull, v, 1);
+    return v;
+}
+
+__device__ __forceinline__ void jbar(int nthreads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Blocks move one position along the circle top_1 .. top_{G-1}, bot_{G-1} ..
+// bot_0 (top_0 stays): every pair of blocks shares a warp once in nb-1 moves,
+// after which every block is back at its start.
+template <int NR>
+__device__ __forceinline__ void block_move(float (&a)[16][NR], float* nrm, float* xbuf, float* xnrm,
+                                           int g, int G, int lane, int npad) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int u = 0; u < NR; ++u) xbuf[(16 * g + i) * npad + lane + 32 * u] = a[i][u];
+    if (lane < 16) xnrm[16 * g + lane] = nrm[lane];
+    jbar(G * 32);
+    const int st = g == 0 ? 0 : (g == 1 ? 1 : 2 * (g - 1));     // source position of the new top
+    const int sb = g == G - 1 ? 2 * (G - 1) : 2 * (g + 1) + 1;  // and of the new bottom
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int u = 0; u < NR; ++u) {
+            a[i][u] = xbuf[(8 * st + i) * npad + lane + 32 * u];
+            a[8 + i][u] = xbuf[(8 * sb + i) * npad + lane + 32 * u];
+        }
+    const float nv = lane < 8 ? xnrm[8 * st + lane] : (lane < 16 ? xnrm[8 * sb + lane - 8] : 0.f);
+    jbar(G * 32);
+    if (lane < 16) nrm[lane] = nv;
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// Small dense products on shared-memory operands.
+// ---------------------------------------------------------------------------
+
+// G = A^T A for the rows x R matrix A (stride ld); G: R x R, stride ld.
+template <int R>
+__device__ void gram(const float* A, int rows, int ld, float* G) {
+    constexpr int chunks = R / 4;
+    for (int e = threadIdx.x; e < R * chunks; e += kThreads) {
+        const int a = e / chunks, c4 = (e % chunks) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < rows; ++i) {
+            const float x = A[i * ld + a];
+            const float4 y = *reinterpret_cast<const float4*>(A + i * ld + c4);
+            acc.x = fmaf(x, y.x, acc.x);
+            acc.y = fmaf(x, y.y, acc.y);
+            acc.z = fmaf(x, y.z, acc.z);
+            acc.w = fmaf(x, y.w, acc.w);
+        }
+        *reinterpret_cast<float4*>(G + a * ld + c4) = acc;
+    }
+}
+
+// Row i of the Bjorck step: out[j] = 1.5 A[i][j] - 0.5 sum_a A[i][a] G[a][j],
+// for the half j in [h R/2, (h+1) R/2).
+template <int R>
+__device__ __forceinline__ void bjorck_row(const float* A, const float* G, int ld, int i, int h,
+                                           float (&out)[R / 2]) {
+    constexpr int H = R / 2;
+#pragma unroll
+    for (int v = 0; v < H; ++v) out[v] = 0.f;
+    for (int a = 0; a < R; ++a) {
+        const float x = A[i * ld + a];
+        const float4* gr = reinterpret_cast<const float4*>(G + a * ld + h * H);
+#pragma unroll
+        for (int v = 0; v < H / 4; ++v) {
+            const float4 y = gr[v];
+            out[4 * v] = fmaf(x, y.x, out[4 * v]);
+            out[4 * v + 1] = fmaf(x, y.y, out[4 * v + 1]);
+            out[4 * v + 2] = fmaf(x, y.z, out[4 * v + 2]);
+            out[4 * v + 3] = fmaf(x, y.w, out[4 * v + 3]);
+        }
+    }
+#pragma unroll
+    for (int v = 0; v < H; ++v) out[v] = fmaf(-0.5f, out[v], 1.5f * A[i * ld + h * H + v]);
+}
+
+template <typename KvT>
+__device__ __forceinline__ float ring_at(const void* ring, int blocked, int64_t slot, int i) {
+    return to_f32(reinterpret_cast<const KvT*>(ring)[coef_index(blocked, kHeadDim, slot, i)]);
+}
+
+__device__ __forceinline__ float x_at(const FactorView& f, const void* ring, int64_t slot, int i) {
+    return f.kv_bf16 ? ring_at<__nv_bfloat16>(ring, f.ring_blocked, slot, i)
+                     : ring_at<float>(ring, f.ring_blocked, slot, i);
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, (R <= 64 ? 2 : 1))
 fold_kernel(FactorView f, FoldLaunch fl, int* status) {
+    using Gm = Geo<R>;
+    constexpr int d = Gm::d, b = Gm::b, k = Gm::k, m = Gm::m, n = Gm::n, c = Gm::c;
+    constexpr int ldm = Gm::ldm, ldk = Gm::ldk, ldw = Gm::ldw, ldp = Gm::ldp;
+    constexpr int NR = Gm::NR, npad = Gm::npad, G = Gm::nwj, nb = Gm::nb;
     const int bh = blockIdx.x;
     const int task = blockIdx.y;
     const int layer = fl.layer[task];
     const int64_t n_c = fl.n_c[task];
     const int slot = fl.slot[task];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int d = kHeadDim;
-    constexpr int b = kBlock;
-    const Dims x = dims_for(f.r);
-    const int r = x.r, k = x.k, m = x.m, n = x.n, c = x.c, nrefl = x.nrefl;
-    const Layout L = layout_for(x);
 
-    extern __shared__ float smem[];
-    float* sM = smem;                 // d x c, column-major (stride d)
-    float* sV = smem;                 // n x n, column-major (stride n), after QR
-    float* sA = smem + L.R1;          // m x n, column-major (stride m)
-    float* sQ = sA + L.R2;            // d x k, column-major (stride d)
-    float* tau = sQ + L.Q;
-    float* vdiag = tau + c;
-    float* nrm = vdiag + c;
-    int* perm = reinterpret_cast<int*>(nrm + n);
-    int* flag = perm + n;
+    extern __shared__ __align__(16) float smem[];
+    float* A = smem;                           // region A
+    float* aux = A + Gm::regA;                 // P (b x ldp) and R_E (k x b); later Gram matrices
+    float* Pb = aux;
+    float* REb = aux + b * ldp;
+    float* sm = aux + Gm::aux;
+    float* tau1 = sm;
+    float* vd1 = sm + 128;
+    float* al1 = sm + 256;
+    float* tau2 = sm + 384;
+    float* vd2 = sm + 512;
+    float* al2 = sm + 640;
+    float* nrm2 = sm + 768;                    // 4
+    float* sig2 = sm + 772;                    // 128
+    int* rnk = reinterpret_cast<int*>(sm + 900);   // 128
+    float* wnrm = sm + 1028;                   // kWarps x 16
+    float2* wpar = reinterpret_cast<float2*>(sm + 1028 + kWarps * 16);   // kWarps x 8
+    float* xnrm = sm + 1028 + kWarps * 32;     // 128
+    int* flags = reinterpret_cast<int*>(sm + 1156 + kWarps * 32);       // 16
+    int* wany = flags;                         // kWarps
+    int* ncomp = flags + 8;
+    float* fro = reinterpret_cast<float*>(flags + 10);
+    int* cflag = flags + 16;                   // 128: rank slot awaiting completion
 
     const int64_t hidx = (int64_t)layer * f.BH + bh;
-    const float* gB = f.basis + hidx * d * r;
-    const float* gS = f.sigma + hidx * r;
-    const KvT* ring = reinterpret_cast<const KvT*>(f.ring) + hidx * f.cap * d;
+    const float* gB = f.basis + hidx * d * R;
+    const float* gS = f.sigma + hidx * R;
+    const void* ring = reinterpret_cast<const uint8_t*>(f.ring) + hidx * f.cap * d * (f.kv_bf16 ? 2 : 4);
     const int64_t slot0 = n_c % f.cap;
+    float* gQ = fl.qscratch + hidx * d * k;
 
-    // ---- load B (columns 0..r-1) and X^T (columns r..r+63); zero the core
-    for (int e = tid; e < d * r; e += kThreads) {
-        int i = e % d, j = e / d;
-        sM[j * d + i] = gB[(int64_t)i * r + j];
+    // ---- load [B | X^T]
+    for (int e = tid; e < d * R; e += kThreads) {
+        const int i = e / R, j = e - (e / R) * R;
+        A[i * ldm + j] = gB[e];
     }
     for (int e = tid; e < b * d; e += kThreads) {
-        int t = e / d, i = e % d;
-        sM[(r + t) * d + i] = to_f32(ring[coef_index(f.ring_blocked, d, slot0 + t, i)]);
+        const int t = e / d, i = e - (e / d) * d;
+        A[i * ldm + R + t] = x_at(f, ring, slot0 + t, i);
     }
-    for (int e = tid; e < m * n; e += kThreads) sA[e] = 0.f;
-    __syncthreads();
-    for (int j = tid; j < r; j += kThreads) sA[j * m + j] = gS[j];
-
-    // ---- (a) P = X B into core rows r..r+63, columns 0..r-1
-    for (int t = warp; t < b; t += kWarps) {
-        float xv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) xv[u] = sM[(r + t) * d + lane + 32 * u];
-        for (int j = 0; j < r; ++j) {
-            float p = 0.f;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) p = fmaf(xv[u], sM[j * d + lane + 32 * u], p);
-            p = warp_sum(p);
-            if (lane == 0) sA[j * m + r + t] = p;
-        }
-    }
+    if (tid < 16 + 128) flags[tid] = 0;
     __syncthreads();
 
-    // ---- (b) Householder QR of [B | X^T], reflections 0..nrefl-1
-    for (int j = 0; j < nrefl; ++j) {
-        if (warp == 0) {
-            float below = 0.f;
-            for (int i = j + 1 + lane; i < d; i += 32) {
-                float v = sM[j * d + i];
-                below = fmaf(v, v, below);
-            }
-            below = warp_sum(below);
-            if (lane == 0) {
-                float xj = sM[j * d + j];
-                if (below == 0.f) {
-                    tau[j] = 0.f;
-                    vdiag[j] = 1.f;
-                } else {
-                    float nr = sqrtf(fmaf(xj, xj, below));
-                    float alpha = -copysignf(nr, xj);
-                    float vj = xj - alpha;
-                    tau[j] = 2.f / fmaf(vj, vj, below);
-                    vdiag[j] = vj;
-                    sM[j * d + j] = alpha;
-                }
+    // ---- (a) P = X B: thread -> (row t, quarter of the columns)
+    {
+        constexpr int Q4 = R / 4;
+        const int t = tid >> 2, h = tid & 3;
+        float acc[Q4];
+#pragma unroll
+        for (int v = 0; v < Q4; ++v) acc[v] = 0.f;
+        for (int i = 0; i < d; ++i) {
+            const float x = A[i * ldm + R + t];
+            const float4* br = reinterpret_cast<const float4*>(A + i * ldm + h * Q4);
+#pragma unroll
+            for (int v = 0; v < Q4 / 4; ++v) {
+                const float4 y = br[v];
+                acc[4 * v] = fmaf(x, y.x, acc[4 * v]);
+                acc[4 * v + 1] = fmaf(x, y.y, acc[4 * v + 1]);
+                acc[4 * v + 2] = fmaf(x, y.z, acc[4 * v + 2]);
+                acc[4 * v + 3] = fmaf(x, y.w, acc[4 * v + 3]);
             }
         }
-        __syncthreads();
-        const float tj = tau[j];
-        if (tj != 0.f) {
-            const float vj = vdiag[j];
-            for (int col = j + 1 + warp; col < c; col += kWarps) {
-                float w = 0.f;
-                for (int i = j + lane; i < d; i += 32) {
-                    float vi = (i == j) ? vj : sM[j * d + i];
-                    w = fmaf(vi, sM[col * d + i], w);
-                }
-                w = warp_sum(w) * tj;
-                for (int i = j + lane; i < d; i += 32) {
-                    float vi = (i == j) ? vj : sM[j * d + i];
-                    sM[col * d + i] = fmaf(-w, vi, sM[col * d + i]);
-                }
-            }
-        }
-        __syncthreads();
+#pragma unroll
+        for (int v = 0; v < Q4; ++v) Pb[t * ldp + h * Q4 + v] = acc[v];
     }
+    __syncthreads();
 
-    // ---- R_E^T into the core, Q = H_0 ... H_{r+k-1} e_{r..r+k-1}
+    // ---- (b) Householder QR of [B | X^T]; R_E; Q in place, parked in global scratch
+    house_qr(A, ldm, d, c, n, 0, tau1, vd1, al1, nrm2);
     for (int e = tid; e < k * b; e += kThreads) {
-        int i = e / b, t = e % b;
-        sA[(r + i) * m + r + t] = (i <= t) ? sM[(r + t) * d + r + i] : 0.f;
+        const int i = e / b, t = e - (e / b) * b;
+        REb[e] = (i < t) ? A[(R + i) * ldm + R + t] : ((i == t) ? al1[R + t] : 0.f);
     }
-    for (int qi = warp; qi < k; qi += kWarps) {
-        float y[4];
+    __syncthreads();   // R_E read before form_q clears the upper triangle
+    if constexpr (k > 0) {
+        form_q(A, ldm, R, k, tau1, vd1);
+        for (int e = tid; e < d * k; e += kThreads) {
+            const int i = e / k, q = e - (e / k) * k;
+            gQ[e] = A[i * ldm + R + q];
+        }
+    }
+    __syncthreads();
+
+    // ---- (c) core K = [[diag S, 0], [P, R_E^T]] in region A, then its QR
+    for (int e = tid; e < m * n; e += kThreads) {
+        const int i = e / n, j = e - (e / n) * n;
+        float v;
+        if (i < R) {
+            v = (i == j) ? gS[i] : 0.f;
+        } else {
+            const int t = i - R;
+            v = (j < R) ? Pb[t * ldp + j] : REb[(j - R) * b + t];
+        }
+        A[i * ldk + j] = v;
+    }
+    __syncthreads();
+    house_qr(A, ldk, m, n, n, R, tau2, vd2, al2, nrm2);
+
+    // ---- one-sided Jacobi on the columns of R^T (warps 0..G-1)
+    float a[16][NR];
+    if (warp < G) {
+        const int g = warp;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) y[u] = (lane + 32 * u == r + qi) ? 1.f : 0.f;
-        for (int j = r + qi; j >= 0; --j) {
-            const float tj = tau[j];
-            if (tj == 0.f) continue;
-            float w = 0.f;
+        for (int i = 0; i < 16; ++i) {
+            const int cc = 16 * g + i;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                int i = lane + 32 * u;
-                float vi = (i < j) ? 0.f : ((i == j) ? vdiag[j] : sM[j * d + i]);
-                w = fmaf(vi, y[u], w);
-            }
-            w = warp_sum(w) * tj;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                int i = lane + 32 * u;
-                float vi = (i < j) ? 0.f : ((i == j) ? vdiag[j] : sM[j * d + i]);
-                y[u] = fmaf(-w, vi, y[u]);
+            for (int u = 0; u < NR; ++u) {
+                const int row = lane + 32 * u;
+                a[i][u] = (row == cc) ? al2[cc] : ((row > cc && row < n) ? A[cc * ldk + row] : 0.f);
             }
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) sQ[qi * d + lane + 32 * u] = y[u];
-    }
-    __syncthreads();
-
-    // ---- (c) one-sided Jacobi on the core; V = I
-    for (int e = tid; e < n * n; e += kThreads) sV[e] = (e / n == e % n) ? 1.f : 0.f;
-    __syncthreads();
-
-    const float tol = jacobi_tol(m);
-    const int ru = (m + 31) / 32;   // rows of A per lane (<= 6)
-    const int rv = (n + 31) / 32;   // rows of V per lane (<= 6)
-    float* fro = reinterpret_cast<float*>(flag + 1);   // Frobenius norm^2 of the core
-    bool converged = false;
-    for (int sweep = 0; sweep < fl.max_sweeps; ++sweep) {
-        for (int col = warp; col < n; col += kWarps) {
-            float s = 0.f;
-            for (int u = 0; u < ru; ++u) {
-                int i = lane + 32 * u;
-                float v = (i < m) ? sA[col * m + i] : 0.f;
-                s = fmaf(v, v, s);
-            }
+        float* nrm = wnrm + g * 16;
+        JacobiCtx cx{nrm, wpar + g * 8, wany + g, jacobi_tol(n), 0.f, lane};
+        {
+            const float v = col_norms16<NR>(a, lane);
+            float s = ((lane & 1) == 0) ? v : 0.f;
             s = warp_sum(s);
-            if (lane == 0) nrm[col] = s;
+            if (lane == 0) atomicAdd(fro, s);
         }
-        if (tid == 0) *flag = 0;
-        __syncthreads();
-        if (sweep == 0 && tid == 0) {
-            float t = 0.f;
-            for (int col = 0; col < n; ++col) t += nrm[col];
-            *fro = t;
+        jbar(G * 32);   // R fully read before the first block move; fro complete
+        cx.tiny = fmaf(1e-14f, *fro, 1e-35f);
+        bool converged = false;
+        for (int sweep = 0; sweep < fl.max_sweeps; ++sweep) {
+            {
+                const float v = col_norms16<NR>(a, lane);
+                if ((lane & 1) == 0) nrm[(lane >> 1) & 15] = v;
+                if (lane == 0) *cx.any = 0;
+                __syncwarp();
+            }
+            for (int br = 0; br < nb - 1; ++br) {
+                if (br == 0) jacobi_rounds<NR, true>(a, cx, std::make_integer_sequence<int, 7>{});
+                jacobi_rounds<NR, false>(a, cx, std::make_integer_sequence<int, 8>{});
+                block_move<NR>(a, nrm, A, xnrm, g, G, lane, npad);
+            }
+            jbar(G * 32);
+            int any = 0;
+            for (int w = 0; w < G; ++w) any |= wany[w];
+            jbar(G * 32);
+            if (!any) {
+                converged = true;
+                break;
+            }
         }
-        __syncthreads();
-        // columns below this energy are numerically zero and never rotated
-        const float tiny = fmaf(1e-14f, *fro, 1e-35f);
-        for (int round = 0; round < n - 1; ++round) {
-            for (int pi = warp; pi < n / 2; pi += kWarps) {
-                const int p = (pi == 0) ? 0 : 1 + (pi - 1 + round) % (n - 1);
-                const int qq = n - 1 - pi;
-                const int q = 1 + (qq - 1 + round) % (n - 1);
-                const float al = nrm[p], be = nrm[q];
-                float gm = 0.f;
-                for (int u = 0; u < ru; ++u) {
-                    int i = lane + 32 * u;
-                    if (i < m) gm = fmaf(sA[p * m + i], sA[q * m + i], gm);
+        if (!converged && g == 0 && lane == 0) atomicOr(status, kStatusNoConverge);
+        const float v = col_norms16<NR>(a, lane);
+        if ((lane & 1) == 0) sig2[16 * g + ((lane >> 1) & 15)] = v;
+    }
+    __syncthreads();
+    // ---- descending order of sigma (ties: lower column first)
+    const float tiny = fmaf(1e-14f, *fro, 1e-35f);
+    if (tid < n) {
+        const float v = sig2[tid];
+        int rk = 0;
+        for (int j = 0; j < n; ++j) {
+            const float u = sig2[j];
+            rk += (u > v) || (u == v && j < tid);
+        }
+        rnk[tid] = rk;
+    }
+    __syncthreads();
+    // ---- W (n x R, slot 0 of region A): unit columns at their rank
+    float* W = A;
+    float* W2 = A + d * ldw;
+    float* sigR = xnrm;   // sigma of rank slot j < R
+    if (warp < G) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int cc = 16 * warp + i;
+            const int rk = rnk[cc];
+            if (rk < R) {
+                const float s2 = sig2[cc];
+                const bool ok = s2 > tiny;
+                const float inv = ok ? 1.f / sqrtf(s2) : 0.f;
+#pragma unroll
+                for (int u = 0; u < NR; ++u) {
+                    const int row = lane + 32 * u;
+                    if (row < n) W[row * ldw + rk] = a[i][u] * inv;
                 }
-                gm = warp_sum(gm);
-                if (fminf(al, be) > tiny && fabsf(gm) > tol * sqrtf(fmaxf(al * be, 0.f))) {
-                    const float zeta = (be - al) / (2.f * gm);
-                    const float t = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
-                    const float cs = 1.f / sqrtf(fmaf(t, t, 1.f));
-                    const float sn = cs * t;
-                    for (int u = 0; u < ru; ++u) {
-                        int i = lane + 32 * u;
-                        if (i < m) {
-                            float ap = sA[p * m + i], aq = sA[q * m + i];
-                            sA[p * m + i] = fmaf(cs, ap, -sn * aq);
-                            sA[q * m + i] = fmaf(sn, ap, cs * aq);
-                        }
-                    }
-                    for (int u = 0; u < rv; ++u) {
-                        int i = lane + 32 * u;
-                        if (i < n) {
-                            float vp = sV[p * n + i], vq = sV[q * n + i];
-                            sV[p * n + i] = fmaf(cs, vp, -sn * vq);
-                            sV[q * n + i] = fmaf(sn, vp, cs * vq);
-                        }
-                    }
-                    if (lane == 0) {
-                        nrm[p] = fmaf(-t, gm, al);
-                        nrm[q] = fmaf(t, gm, be);
-                        *flag = 1;
+                if (lane == 0) {
+                    sigR[rk] = sqrtf(s2);
+                    if (!ok) {
+                        cflag[rk] = 1;
+                        atomicAdd(ncomp, 1);
                     }
                 }
             }
-            __syncthreads();
-        }
-        const int any = *flag;
-        __syncthreads();
-        if (!any) {
-            converged = true;
-            break;
         }
     }
-    if (!converged && tid == 0) atomicOr(status, kStatusNoConverge);
-
-    // ---- unit columns of V, with A = K V scaled alike
-    for (int col = warp; col < n; col += kWarps) {
-        float s = 0.f;
-        for (int u = 0; u < rv; ++u) {
-            int i = lane + 32 * u;
-            float v = (i < n) ? sV[col * n + i] : 0.f;
-            s = fmaf(v, v, s);
-        }
-        const float inv = 1.f / sqrtf(warp_sum(s));
-        for (int u = 0; u < rv; ++u) {
-            int i = lane + 32 * u;
-            if (i < n) sV[col * n + i] *= inv;
-        }
-        for (int u = 0; u < ru; ++u) {
-            int i = lane + 32 * u;
-            if (i < m) sA[col * m + i] *= inv;
+    __syncthreads();
+    // ---- completion of numerically zero directions (rank of K below R): one
+    // warp, slot by slot: e_i with the largest residual against the accepted
+    // columns, orthogonalized twice (classical Gram-Schmidt) and normalized
+    if (*ncomp > 0 && warp == 0) {
+        for (int sl = 0; sl < R; ++sl) {
+            if (!cflag[sl]) continue;
+            float best = -1.f;
+            int bi = 0;
+            for (int i = lane; i < n; i += 32) {
+                float acc = 0.f;
+                for (int j = 0; j < R; ++j)
+                    if (!cflag[j]) acc = fmaf(W[i * ldw + j], W[i * ldw + j], acc);
+                if (1.f - acc > best) {
+                    best = 1.f - acc;
+                    bi = i;
+                }
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ob = __shfl_xor_sync(kFull, best, o);
+                const int oi = __shfl_xor_sync(kFull, bi, o);
+                if (ob > best || (ob == best && oi < bi)) {
+                    best = ob;
+                    bi = oi;
+                }
+            }
+            float y[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) y[u] = (lane + 32 * u == bi) ? 1.f : 0.f;
+            for (int pass = 0; pass < 2; ++pass) {
+                for (int j = 0; j < R; ++j) {
+                    if (cflag[j]) continue;
+                    float dp = 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int row = lane + 32 * u;
+                        if (row < n) dp = fmaf(W[row * ldw + j], y[u], dp);
+                    }
+                    dp = warp_sum(dp);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int row = lane + 32 * u;
+                        if (row < n) y[u] = fmaf(-dp, W[row * ldw + j], y[u]);
+                    }
+                }
+            }
+            float nn = 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) nn = fmaf(y[u], y[u], nn);
+            const float inv = 1.f / sqrtf(warp_sum(nn));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int row = lane + 32 * u;
+                if (row < n) W[row * ldw + sl] = y[u] * inv;
+            }
+            __syncwarp();
+            if (lane == 0) cflag[sl] = 0;   // accepted from now on
+            __syncwarp();
         }
     }
     __syncthreads();
 
-    // ---- singular values (exact column norms) and descending order
-    for (int col = warp; col < n; col += kWarps) {
-        float s = 0.f;
-        for (int u = 0; u < ru; ++u) {
-            int i = lane + 32 * u;
-            float v = (i < m) ? sA[col * m + i] : 0.f;
-            s = fmaf(v, v, s);
-        }
-        s = warp_sum(s);
-        if (lane == 0) nrm[col] = sqrtf(s);
+    // ---- Bjorck step on W: W2 = 1.5 W - 0.5 W (W^T W)
+    float* Gm_ = aux;   // R x ldw (P and R_E are dead)
+    gram<R>(W, n, ldw, Gm_);
+    __syncthreads();
+    if (tid < 2 * n) {
+        float o[R / 2];
+        bjorck_row<R>(W, Gm_, ldw, tid >> 1, tid & 1, o);
+#pragma unroll
+        for (int v = 0; v < R / 2; ++v) W2[(tid >> 1) * ldw + (tid & 1) * (R / 2) + v] = o[v];
     }
     __syncthreads();
-    for (int col = tid; col < n; col += kThreads) {
-        const float v = nrm[col];
-        int rank = 0;
+
+    // ---- (d) outputs: S', W_top, B'' = [B, Q] W (slot 0), new rows X B''
+    float* gSw = f.sigma + hidx * R;
+    float* gW = f.pend + (hidx * f.D + slot) * (int64_t)R * R;
+    for (int e = tid; e < R * R; e += kThreads) {
+        const int i = e / R, j = e - (e / R) * R;
+        gW[e] = W2[i * ldw + j];
+    }
+    if (tid == 0 && bh == 0) f.seg_rows[layer * f.D + slot] = (int)n_c;
+    float* Bn = A;   // slot 0: B'' (d x R)
+    {
+        constexpr int H = R / 2;
+        const int i = tid >> 1, h = tid & 1;
+        float acc[H];
+#pragma unroll
+        for (int v = 0; v < H; ++v) acc[v] = 0.f;
+#pragma unroll 4
         for (int j = 0; j < n; ++j) {
-            const float u = nrm[j];
-            rank += (u > v) || (u == v && j < col);
+            const float x = (j < R) ? gB[i * R + j] : gQ[i * k + (j - R)];
+            const float4* wr = reinterpret_cast<const float4*>(W2 + j * ldw + h * H);
+#pragma unroll
+            for (int v = 0; v < H / 4; ++v) {
+                const float4 y = wr[v];
+                acc[4 * v] = fmaf(x, y.x, acc[4 * v]);
+                acc[4 * v + 1] = fmaf(x, y.y, acc[4 * v + 1]);
+                acc[4 * v + 2] = fmaf(x, y.z, acc[4 * v + 2]);
+                acc[4 * v + 3] = fmaf(x, y.w, acc[4 * v + 3]);
+            }
         }
-        perm[rank] = col;
+        __syncthreads();   // every thread is done with W (slot 0 is overwritten next)
+#pragma unroll
+        for (int v = 0; v < H; ++v) Bn[i * ldw + h * H + v] = acc[v];
     }
+    if (tid < R) gSw[tid] = sigR[tid];
     __syncthreads();
-
-    // ---- (d) outputs: S', new coefficient rows, W_top
-    float* gSw = f.sigma + hidx * r;
-    for (int t = tid; t < r; t += kThreads) gSw[t] = nrm[perm[t]];
-    CoefT* gC = reinterpret_cast<CoefT*>(f.coef) + hidx * f.n_max * r;
-    for (int e = tid; e < b * r; e += kThreads) {
-        int t = e / r, cc = e % r;
-        gC[coef_index(f.coef_blocked, r, n_c + t, cc)] = from_f32<CoefT>(sA[perm[cc] * m + r + t]);
+    {
+        // new coefficient rows n_c .. n_c+63 = X B''
+        constexpr int Q4 = R / 4;
+        const int t = tid >> 2, h = tid & 3;
+        float acc[Q4];
+#pragma unroll
+        for (int v = 0; v < Q4; ++v) acc[v] = 0.f;
+        for (int i = 0; i < d; ++i) {
+            const float x = x_at(f, ring, slot0 + t, i);
+            const float4* br = reinterpret_cast<const float4*>(Bn + i * ldw + h * Q4);
+#pragma unroll
+            for (int v = 0; v < Q4 / 4; ++v) {
+                const float4 y = br[v];
+                acc[4 * v] = fmaf(x, y.x, acc[4 * v]);
+                acc[4 * v + 1] = fmaf(x, y.y, acc[4 * v + 1]);
+                acc[4 * v + 2] = fmaf(x, y.z, acc[4 * v + 2]);
+                acc[4 * v + 3] = fmaf(x, y.w, acc[4 * v + 3]);
+            }
+        }
+        const int64_t row = n_c + t;
+        if (f.coef_bf16) {
+            __nv_bfloat16* gC = reinterpret_cast<__nv_bfloat16*>(f.coef) + hidx * f.n_max * R;
+#pragma unroll
+            for (int v = 0; v < Q4; ++v)
+                gC[coef_index(f.coef_blocked, R, row, h * Q4 + v)] = __float2bfloat16_rn(acc[v]);
+        } else {
+            float* gC = reinterpret_cast<float*>(f.coef) + hidx * f.n_max * R;
+#pragma unroll
+            for (int v = 0; v < Q4; ++v) gC[coef_index(f.coef_blocked, R, row, h * Q4 + v)] = acc[v];
+        }
     }
-    float* gW = f.pend + (hidx * f.D + slot) * (int64_t)r * r;
-    for (int e = tid; e < r * r; e += kThreads) {
-        int i = e / r, cc = e % r;
-        gW[e] = sV[perm[cc] * n + i];
-    }
-    if (bh == 0 && tid == 0) f.seg_rows[layer * f.D + slot] = (int)n_c;
+    // ---- Bjorck step on B'' and the stores of B' (fp32, bf16 hi/lo blocked)
+    gram<R>(Bn, d, ldw, Gm_);
     __syncthreads();
-
-    // ---- B' = [B, Q] V[:, perm[0:r]] staged in the core's space
-    float* sBn = sA;
-    for (int e = tid; e < d * r; e += kThreads) {
-        const int i = e % d, cc = e / d;
-        const float* vcol = sV + perm[cc] * n;
-        float acc = 0.f;
-        for (int j = 0; j < r; ++j) acc = fmaf(gB[(int64_t)i * r + j], vcol[j], acc);
-        for (int j = 0; j < k; ++j) acc = fmaf(sQ[j * d + i], vcol[r + j], acc);
-        sBn[i * r + cc] = acc;
-    }
-    __syncthreads();
-    // Bjorck step: G = B'^T B' (r x r, in V's space, no longer needed)
-    float* sG = sV;
-    for (int e = tid; e < r * r; e += kThreads) {
-        const int a = e / r, cc = e % r;
-        float acc = 0.f;
-        for (int i = 0; i < d; ++i) acc = fmaf(sBn[i * r + a], sBn[i * r + cc], acc);
-        sG[e] = acc;
-    }
-    __syncthreads();
-    float* gBw = f.basis + hidx * d * r;
-    __nv_bfloat16* gHi = f.bsplit + hidx * 2 * d * r;
-    __nv_bfloat16* gLo = gHi + d * r;
-    for (int e = tid; e < d * r; e += kThreads) {
-        const int i = e / r, cc = e % r;
-        // v = sum_j B'[i][j] (1.5 delta_jc - 0.5 G[j][c])
-        float corr = 0.f;
-        for (int j = 0; j < r; ++j) corr = fmaf(sBn[i * r + j], sG[j * r + cc], corr);
-        const float v = fmaf(-0.5f, corr, 1.5f * sBn[e]);
-        gBw[e] = v;
-        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-        const int64_t bo = coef_index(1, r, i, cc);
-        gHi[bo] = h;
-        gLo[bo] = __float2bfloat16_rn(v - __bfloat162float(h));
+    {
+        float o[R / 2];
+        const int i = tid >> 1, h = tid & 1;
+        bjorck_row<R>(Bn, Gm_, ldw, i, h, o);
+        float* gBw = f.basis + hidx * d * R;
+        __nv_bfloat16* gHi = f.bsplit + hidx * 2 * d * R;
+        __nv_bfloat16* gLo = gHi + d * R;
+        __syncthreads();   // gB (the old basis) was read by every thread above
+#pragma unroll
+        for (int v = 0; v < R / 2; ++v) {
+            const int j = h * (R / 2) + v;
+            const float x = o[v];
+            gBw[i * R + j] = x;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const int64_t bo = coef_index(1, R, i, j);
+            gHi[bo] = hi;
+            gLo[bo] = __float2bfloat16_rn(x - __bfloat162float(hi));
+        }
     }
 }
 
-template <typename KvT, typename CoefT>
-cudaError_t launch_fold_t(const FactorView& f, const FoldLaunch& fl, int* status,
-                          cudaStream_t s) {
-    const Dims x = dims_for(f.r);
-    const Layout L = layout_for(x);
-    const size_t bytes = (L.R1 + L.R2 + L.Q + L.small) * sizeof(float);
-    auto kern = fold_kernel<KvT, CoefT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int R>
+cudaError_t launch_fold_r(const FactorView& f, const FoldLaunch& fl, int* status, cudaStream_t s) {
+    const size_t bytes = (size_t)Geo<R>::floats * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(fold_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;
     dim3 grid(f.BH, fl.n_tasks);
-    kern<<<grid, kThreads, bytes, s>>>(f, fl, status);
+    fold_kernel<R><<<grid, kThreads, bytes, s>>>(f, fl, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t fold_smem_bytes(int r) {
-    const Dims x = dims_for(r);
-    const Layout L = layout_for(x);
-    return (L.R1 + L.R2 + L.Q + L.small) * sizeof(float);
+    switch (r) {
+        case 16: return Geo<16>::floats * sizeof(float);
+        case 32: return Geo<32>::floats * sizeof(float);
+        case 48: return Geo<48>::floats * sizeof(float);
+        case 64: return Geo<64>::floats * sizeof(float);
+        case 80: return Geo<80>::floats * sizeof(float);
+        case 96: return Geo<96>::floats * sizeof(float);
+        case 112: return Geo<112>::floats * sizeof(float);
+        case 128: return Geo<128>::floats * sizeof(float);
+        default: return 0;
+    }
 }
 
-cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status,
-                        cudaStream_t s) {
+int fold_q_cols(int r) { return (kHeadDim - r) < kBlock ? (kHeadDim - r) : kBlock; }
+
+cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status, cudaStream_t s) {
     if (fl.n_tasks <= 0) return cudaSuccess;
-    if (f.kv_bf16) {
-        return f.coef_bf16 ? launch_fold_t<__nv_bfloat16, __nv_bfloat16>(f, fl, status, s)
-                           : launch_fold_t<__nv_bfloat16, float>(f, fl, status, s);
+    switch (f.r) {
+        case 16: return launch_fold_r<16>(f, fl, status, s);
+        case 32: return launch_fold_r<32>(f, fl, status, s);
+        case 48: return launch_fold_r<48>(f, fl, status, s);
+        case 64: return launch_fold_r<64>(f, fl, status, s);
+        case 80: return launch_fold_r<80>(f, fl, status, s);
+        case 96: return launch_fold_r<96>(f, fl, status, s);
+        case 112: return launch_fold_r<112>(f, fl, status, s);
+        case 128: return launch_fold_r<128>(f, fl, status, s);
+        default: return cudaErrorInvalidValue;
     }
-    return f.coef_bf16 ? launch_fold_t<float, __nv_bfloat16>(f, fl, status, s)
-                       : launch_fold_t<float, float>(f, fl, status, s);
 }
 
 }  // namespace iskv

@@ -26,7 +26,7 @@ def rel_err(a, b) -> float:
 class Pair:
     """A CUDA cache and the oracle's per-head factors, fed identically."""
 
-    def __init__(self, cfg, workload: str, seed: int = 0, heads=None, device="cuda"):
+    def __init__(self, cfg, workload: str, seed: int = 0, heads=None, device="cuda", specs=None):
         import online_rank_kv_b200 as ik
         self.ik = ik
         self.cfg = cfg
@@ -36,8 +36,10 @@ class Pair:
         self.g = cfg.q_heads // cfg.kv_heads
         n = self.L * self.B * self.H
         kdt = cfg.kv_torch_dtype
-        self.ks = synth.KVStream(synth.spec_for(workload, "K"), n, seed=2 * seed + 1, dtype=kdt)
-        self.vs = synth.KVStream(synth.spec_for(workload, "V"), n, seed=2 * seed + 2, dtype=kdt)
+        sk, sv = specs if specs is not None else (synth.spec_for(workload, "K"),
+                                                  synth.spec_for(workload, "V"))
+        self.ks = synth.KVStream(sk, n, seed=2 * seed + 1, dtype=kdt)
+        self.vs = synth.KVStream(sv, n, seed=2 * seed + 2, dtype=kdt)
         self.heads = heads if heads is not None else [
             (l, b, h) for l in range(self.L) for b in range(self.B) for h in range(self.H)]
         rnd = "bf16" if cfg.coef_dtype == ik.BF16 else "f32"

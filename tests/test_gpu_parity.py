@@ -152,6 +152,59 @@ def test_rank_edge_cases(rk, rv):
             assert rel_err(rec[b, h], X) < 1e-5
 
 
+def test_rank_deficient_cores():
+    """Exactly rank-8 keys and rank-1 values without noise at r = 16: the core
+    has numerically zero singular values among the kept r, whose directions
+    an orthonormal completion represents.  Reconstructions stay exact
+    (rank <= r) and the bases orthonormal."""
+    import dataclasses
+
+    import synth
+    ik = _ik()
+    exact8 = dataclasses.replace(synth.spec_for("tiny", "K"), noise=0.0)
+    exact1 = dataclasses.replace(synth.spec_for("tiny", "V"), noise=0.0, decay=0.0)
+    p = Pair(tiny_cfg(), "tiny", seed=9, specs=(exact8, exact1))
+    p.prefill(1024, chunk=64)
+    p.check_counts()
+    for k, e in p.recon_errors(0).items():
+        assert e < TOL_F32, (k, e)
+    for which, of in ((ik.WHICH_K, p.ok), (ik.WHICH_V, p.ov)):
+        rec = p.cache.reconstruct(0, which).cpu().double().numpy()
+        X = of[(0, 0, 0)].rows[:rec.shape[2]]
+        assert rel_err(rec[0, 0], X) < 1e-5
+        basis, sigma, coef = p.cache.factors(0, which)
+        Bg = basis[0, 0].cpu().double().numpy()
+        assert np.isfinite(Bg).all() and np.isfinite(coef.cpu().numpy()).all()
+        assert np.abs(Bg.T @ Bg - np.eye(16)).max() < 1e-5
+    errs, _ = p.decode(0, p.query())
+    assert max(errs.values()) < TOL_F32, errs
+    assert p.cache.status() == 0
+
+
+def test_all_zero_stream():
+    """All-zero keys and values: every singular value of every core is zero,
+    the reconstruction is exactly zero and the bases stay orthonormal."""
+    ik = _ik()
+    cfg = tiny_cfg(rank_k=32, rank_v=64)
+    cache = ik.Cache(cfg)
+    z = torch.zeros(1, 1, 64, 128, device="cuda")
+    for _ in range(8):
+        for _ in range(cache.append(0, z, z)):
+            cache.compress_block(0)
+    assert cache.counts(0) == (512, 384)
+    for which, r in ((ik.WHICH_K, 32), (ik.WHICH_V, 64)):
+        rec = cache.reconstruct(0, which)
+        assert torch.isfinite(rec).all() and rec.abs().max().item() == 0.0
+        basis, sigma, coef = cache.factors(0, which)
+        Bg = basis[0, 0].cpu().double().numpy()
+        assert np.abs(Bg.T @ Bg - np.eye(r)).max() < 1e-5
+        assert sigma.abs().max().item() == 0.0
+    q = torch.randn(1, 1, 128, device="cuda")
+    out = cache.decode_attention(0, q)
+    assert torch.isfinite(out).all() and out.abs().max().item() == 0.0
+    assert cache.status() == 0
+
+
 def test_no_sync_ablation():
     """The no-synchronization ablation keeps every old coefficient row in the
     basis it was written in.  Reading such rows in a later basis is not
