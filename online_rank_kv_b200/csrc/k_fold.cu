@@ -80,7 +80,7 @@ struct Geo {
     static constexpr int ldp = R + 4;                       // P stride
     // region A: [B | X^T], then the core, the Jacobi exchange buffer, two
     // d x R staging slots
-    static constexpr int regA0 = d * ldm > m * ldk ? d * ldm : m * ldk;
+    static constexpr int regA0 = d * ldm > n * ldk ? d * ldm : n * ldk;   // >= n * d (reflectors)
     static constexpr int regA1 = n * npad > 2 * d * ldw ? n * npad : 2 * d * ldw;
     static constexpr int regA = regA0 > regA1 ? regA0 : regA1;
     // aux: P and R_E, later the r x r Gram matrices of the Bjorck steps
@@ -88,7 +88,7 @@ struct Geo {
     static constexpr int aux = aux0 > R * ldw ? aux0 : R * ldw;
     // small arrays (floats): tau/vd/al of both QRs, 2 norms, sigma^2, rank,
     // per-warp norms and rotation parameters, exchanged norms, flags
-    static constexpr int small = 6 * 128 + 4 + 128 + 128 + kWarps * 16 + kWarps * 16 + 128 + 16 + 128;
+    static constexpr int small = 6 * 128 + 4 + 128 + 128 + kWarps * 16 + kWarps * 16 + 128 + 16 + 128 + 384;
     static constexpr int floats = regA + aux + small;
     static_assert(n % 16 == 0 && n <= 128 && npad >= n, "core shape");
     static_assert(R % 16 == 0 && R >= 16 && R <= 128, "rank");
@@ -99,117 +99,192 @@ struct Geo {
 __device__ __forceinline__ float jacobi_tol(int len) { return 4.0e-7f * sqrtf((float)len); }
 
 // ---------------------------------------------------------------------------
-// Householder QR in place of the rows x cols row-major matrix A (stride lda,
-// 8 mod 32), reflections j = 0..nrefl-1.  Below its diagonal, column j is
-// nonzero only in rows [max(j + 1, lo), rows) (lo = 0: dense), and every
-// reflection touches only row j and those rows.  H_j = I - tau_j v v^T with
-// v = (vd_j at row j, A[i][j] below); al_j = R[j][j].  The diagonal element
-// A[j][j] keeps its value from before reflection j; the upper triangle of A
-// becomes R.  Thread (warp, lane) owns column 8*warp + (lane & 7) of each
-// 64-column pass and the rows i = i0 + (lane >> 3) (mod 4).
+// Register-resident Householder QR.  Thread (warp w, lane l) owns the matrix
+// columns cs + 64 t (cs = 8 w + (l & 7), t < CPT) over the rows
+// p RPP .. p RPP + RPP - 1 (p = l >> 3): the four row parts of a column share
+// a warp, so every column dot product is a register FMA chain plus two
+// shuffles.  Reflector j, H_j = I - tau_j v v^T, is published once as a full
+// column v (zeros above row j, vd_j at row j, the subdiagonal entries below)
+// in V + slot * ldv, slot = j (keep) or j & 1 (a two-slot ring); al_j = R[j][j].
+// Afterwards each thread's registers hold, per owned column c, R above row c,
+// the column's value at row c from before its own reflection, and the
+// reflector entries below.  Columns at or beyond `cols` must be zero.
 // ---------------------------------------------------------------------------
-__device__ void house_qr(float* A, int lda, int rows, int cols, int nrefl, int lo, float* tau,
-                         float* vd, float* al, float* nrm2) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int col = lane & 7, part = lane >> 3;
-    if (warp == 0) {
-        float s = 0.f;
-        for (int i = (lo > 1 ? lo : 1) + lane; i < rows; i += 32) s = fmaf(A[i * lda], A[i * lda], s);
-        s = warp_sum(s);
-        if (lane == 0) nrm2[0] = s;
+template <int RPP, int CPT, int T1>
+__device__ __forceinline__ void make_reflector(float (&x)[CPT][RPP], int jj, float* V, int ldv,
+                                               bool keep, float* tau, float* vd, float* al) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, p = lane >> 3;
+    const int cs1 = jj & 63;
+    if (warp != (cs1 >> 3)) return;   // warp-uniform: the owner warp
+    const bool own = (lane & 7) == (cs1 & 7);
+    float sp[4] = {0.f, 0.f, 0.f, 0.f}, dg = 0.f;
+#pragma unroll
+    for (int e = 0; e < RPP; ++e) {
+        const float v = x[T1][e];
+        const int row = p * RPP + e;
+        if (row > jj) sp[e & 3] = fmaf(v, v, sp[e & 3]);
+        if (row == jj) dg = v;
     }
-    __syncthreads();
-    for (int j = 0; j < nrefl; ++j) {
-        const float s = nrm2[j & 1];
-        const float ajj = A[j * lda + j];
-        float tj = 0.f, vj = 1.f, aj = ajj;
-        if (s > 0.f) {
-            const float nr = sqrtf(fmaf(ajj, ajj, s));
-            aj = -copysignf(nr, ajj);
-            vj = ajj - aj;
-            tj = 2.f / fmaf(vj, vj, s);
+    float s = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+    if (!own) {
+        s = 0.f;
+        dg = 0.f;
+    }
+    s += __shfl_xor_sync(kFull, s, 8);
+    s += __shfl_xor_sync(kFull, s, 16);
+    dg += __shfl_xor_sync(kFull, dg, 8);
+    dg += __shfl_xor_sync(kFull, dg, 16);
+    float tj = 0.f, vj = 1.f, aj = dg;
+    if (s > 0.f) {
+        const float nr = sqrtf(fmaf(dg, dg, s));
+        aj = -copysignf(nr, dg);
+        vj = dg - aj;
+        tj = 2.f / fmaf(vj, vj, s);
+    }
+    if (own) {
+        float* v = V + (keep ? jj : (jj & 1)) * ldv + p * RPP;
+#pragma unroll
+        for (int e = 0; e < RPP; e += 4) {
+            float4 o;
+            const int row = p * RPP + e;
+            o.x = row < jj ? 0.f : (row == jj ? vj : x[T1][e]);
+            o.y = row + 1 < jj ? 0.f : (row + 1 == jj ? vj : x[T1][e + 1]);
+            o.z = row + 2 < jj ? 0.f : (row + 2 == jj ? vj : x[T1][e + 2]);
+            o.w = row + 3 < jj ? 0.f : (row + 3 == jj ? vj : x[T1][e + 3]);
+            *reinterpret_cast<float4*>(v + e) = o;
         }
-        if (tid == 0) {
-            tau[j] = tj;
-            vd[j] = vj;
-            al[j] = aj;
+        if (p == 0) {
+            tau[jj] = tj;
+            vd[jj] = vj;
+            al[jj] = aj;
         }
-        const int i0 = (j + 1 > lo) ? j + 1 : lo;
-        const int inext = (j + 2 > lo) ? j + 2 : lo;   // rows of column j+1's next norm
-        for (int cb = j + 1 + warp * 8; cb < cols; cb += kWarps * 8) {
-            const int cc = cb + col;
-            const bool act = cc < cols;
-            float w = 0.f;
-            if (act) {
-                if (part == 0) w = vj * A[j * lda + cc];
-                for (int i = i0 + part; i < rows; i += 4) w = fmaf(A[i * lda + j], A[i * lda + cc], w);
-            }
-            w += __shfl_xor_sync(kFull, w, 8);
-            w += __shfl_xor_sync(kFull, w, 16);
-            const float tw = tj * w;
-            float sq = 0.f;
-            if (act) {
-                if (part == 0) A[j * lda + cc] = fmaf(-tw, vj, A[j * lda + cc]);
-                for (int i = i0 + part; i < rows; i += 4) {
-                    const float x = fmaf(-tw, A[i * lda + j], A[i * lda + cc]);
-                    A[i * lda + cc] = x;
-                    if (i >= inext) sq = fmaf(x, x, sq);
-                }
-            }
-            sq += __shfl_xor_sync(kFull, sq, 8);
-            sq += __shfl_xor_sync(kFull, sq, 16);
-            if (act && part == 0 && cc == j + 1) nrm2[(j + 1) & 1] = sq;
-        }
-        __syncthreads();
     }
 }
 
-// Columns r..r+k-1 of the QR'd [B | X^T] (d x (r+64), stride lda) become
-// Q = H_0 ... H_{n-1} [e_r .. e_{r+k-1}], n = r + k: backward accumulation.
-// A column c of the block is set to H_c e_c the first time a reflection
-// reaches it (reflection c - 1); its strictly upper part (R entries, saved
-// beforehand) is cleared first.
-__device__ void form_q(float* A, int lda, int r, int k, const float* tau, const float* vd) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int col = lane & 7, part = lane >> 3;
-    constexpr int d = kHeadDim;
-    const int n = r + k;
-    for (int e = tid; e < d * k; e += kThreads) {
-        const int i = e / k, q = e - (e / k) * k;
-        if (i < r + q) A[i * lda + r + q] = 0.f;
+template <int RPP>
+__device__ __forceinline__ float dot_split(const float (&a)[RPP], const float (&b)[RPP]) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+    for (int e = 0; e < RPP; e += 4) {
+        s0 = fmaf(a[e], b[e], s0);
+        s1 = fmaf(a[e + 1], b[e + 1], s1);
+        s2 = fmaf(a[e + 2], b[e + 2], s2);
+        s3 = fmaf(a[e + 3], b[e + 3], s3);
     }
+    return (s0 + s1) + (s2 + s3);
+}
+
+// Apply the current reflector (vr, tau tj, index j) to column slot t of the thread.
+template <int RPP, int CPT>
+__device__ __forceinline__ void reflect_slot(float (&x)[CPT][RPP], const float (&vr)[RPP], int t,
+                                             int col, int j, int cols, float tj) {
+    float w = dot_split<RPP>(vr, x[t]);
+    w += __shfl_xor_sync(kFull, w, 8);
+    w += __shfl_xor_sync(kFull, w, 16);
+    if (col > j && col < cols) {
+        const float tw = tj * w;
+#pragma unroll
+        for (int e = 0; e < RPP; ++e) x[t][e] = fmaf(-tw, vr[e], x[t][e]);
+    }
+}
+
+// One reflection step j (column j+1 lives in slot TN of its owner threads).
+template <int RPP, int CPT, int TN>
+__device__ __forceinline__ void qr_step(float (&x)[CPT][RPP], int j, int cols, int nrefl, float* V,
+                                        int ldv, bool keep, float* tau, float* vd, float* al) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, p = lane >> 3;
+    const int cs = warp * 8 + (lane & 7);
     __syncthreads();
+    const float* v = V + (keep ? j : (j & 1)) * ldv + p * RPP;
+    const float tj = tau[j];
+    auto load_v = [&](float (&vr)[RPP]) {
+#pragma unroll
+        for (int e = 0; e < RPP; e += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(v + e);
+            vr[e] = q.x;
+            vr[e + 1] = q.y;
+            vr[e + 2] = q.z;
+            vr[e + 3] = q.w;
+        }
+    };
+    // look-ahead: the warp owning column j+1 brings that column up to date and
+    // publishes the next reflector before its other columns (the reflector is
+    // reloaded afterwards rather than held across)
+    const int jn = j + 1;
+    const bool ahead = jn < nrefl && warp == ((jn & 63) >> 3);
+    if (ahead) {
+        float vr[RPP];
+        load_v(vr);
+        reflect_slot<RPP, CPT>(x, vr, TN, cs + 64 * TN, j, cols, tj);
+        make_reflector<RPP, CPT, TN>(x, jn, V, ldv, keep, tau, vd, al);
+    }
+    float vr[RPP];
+    load_v(vr);
+    // slots whose columns (8 per warp) are all finished (<= j) or absent are skipped
+    const int cw = warp * 8;
+#pragma unroll
+    for (int t = 0; t < CPT; ++t)
+        if ((t != TN || !ahead) && cw + 7 + 64 * t > j && cw + 64 * t < cols)
+            reflect_slot<RPP, CPT>(x, vr, t, cs + 64 * t, j, cols, tj);
+}
+
+template <int RPP, int CPT>
+__device__ void house_qr_reg(float (&x)[CPT][RPP], int cols, int nrefl, float* V, int ldv, bool keep,
+                             float* tau, float* vd, float* al) {
+    make_reflector<RPP, CPT, 0>(x, 0, V, ldv, keep, tau, vd, al);
+    // step j publishes reflector j+1, whose column sits in slot (j+1) / 64;
+    // steps whose j+1 lies beyond the last slot publish nothing (j+1 >= nrefl)
+    int j = 0;
+    for (; j < nrefl && j < 63; ++j) qr_step<RPP, CPT, 0>(x, j, cols, nrefl, V, ldv, keep, tau, vd, al);
+    if constexpr (CPT > 1)
+        for (; j < nrefl && j < 127; ++j) qr_step<RPP, CPT, 1>(x, j, cols, nrefl, V, ldv, keep, tau, vd, al);
+    if constexpr (CPT > 2)
+        for (; j < nrefl && j < 191; ++j) qr_step<RPP, CPT, 2>(x, j, cols, nrefl, V, ldv, keep, tau, vd, al);
+    for (; j < nrefl; ++j) qr_step<RPP, CPT, CPT - 1>(x, j, cols, nrefl, V, ldv, keep, tau, vd, al);
+    __syncthreads();
+}
+
+// Q = H_0 ... H_{n-1} [e_r .. e_{r+k-1}] from the kept reflectors (V, one
+// 128-row column per reflector): thread (warp w, lane l) accumulates column
+// q = 8 w + (l & 7) < k over rows 32 p .. 32 p + 31 backwards, starting with
+// H_{r+q} e_{r+q}; no barrier is needed.  Writes Q (d x k, row-major) to gQ.
+__device__ void form_q_reg(const float* V, int r, int k, int n, const float* tau, const float* vd,
+                           float* gQ) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, p = lane >> 3;
+    const int q = warp * 8 + (lane & 7);
+    const bool has = q < k;
+    float y[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) y[e] = 0.f;
     for (int j = n - 1; j >= 0; --j) {
-        const float tj = tau[j], vj = vd[j];
-        const int cc = (j >= r ? j + 1 : r) + warp * 8 + col;   // <= 64 target columns: one pass
-        const bool act = cc < n;
-        const bool init = act && cc == j + 1;
-        float ti = 0.f, vi = 0.f;
-        if (init) {
-            ti = tau[j + 1];
-            vi = vd[j + 1];
+        const float* v = V + j * kHeadDim + p * 32;
+        float vr[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+            const float4 t4 = *reinterpret_cast<const float4*>(v + e);
+            vr[e] = t4.x;
+            vr[e + 1] = t4.y;
+            vr[e + 2] = t4.z;
+            vr[e + 3] = t4.w;
         }
-        float w = 0.f;
-        if (act) {
-            if (part == 0) w = vj * A[j * lda + cc];
-            for (int i = j + 1 + part; i < d; i += 4) {
-                float y = A[i * lda + cc];
-                if (init) {
-                    y = (i == j + 1) ? fmaf(-ti * vi, vi, 1.f) : -ti * vi * y;
-                    A[i * lda + cc] = y;
-                }
-                w = fmaf(A[i * lda + j], y, w);
-            }
+        const float tj = tau[j];
+        if (has && j == r + q) {
+            const float f0 = -tj * vd[j];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) y[e] = fmaf(f0, vr[e], (p * 32 + e == j) ? 1.f : 0.f);
         }
+        float w = dot_split<32>(vr, y);
         w += __shfl_xor_sync(kFull, w, 8);
         w += __shfl_xor_sync(kFull, w, 16);
-        const float tw = tj * w;
-        if (act) {
-            if (part == 0) A[j * lda + cc] = fmaf(-tw, vj, A[j * lda + cc]);
-            for (int i = j + 1 + part; i < d; i += 4)
-                A[i * lda + cc] = fmaf(-tw, A[i * lda + j], A[i * lda + cc]);
+        if (has && j < r + q) {
+            const float tw = tj * w;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) y[e] = fmaf(-tw, vr[e], y[e]);
         }
-        __syncthreads();
+    }
+    if (has) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) gQ[(p * 32 + e) * k + q] = y[e];
     }
 }
 
@@ -231,7 +306,7 @@ struct JacobiCtx {
     float* nrm;      // this warp's 16 column norms^2
     float2* par;     // this warp's 8 rotation parameters
     int* any;        // this warp's "rotated" flag
-    float tol, tiny;
+    float tol2, tiny;
     int lane;
 };
 
@@ -274,10 +349,15 @@ __device__ __forceinline__ void jacobi_round(float (&a)[16][NR], const JacobiCtx
     const int ip = (lane >> 2) & 7;
     const int p = pair_p(WITHIN, S, ip), q = pair_q(WITHIN, S, ip);
     const float al = cx.nrm[p], be = cx.nrm[q];
+    // rotate while |g| > tol sqrt(al be), i.e. g^2 > tol^2 al be
+    const bool need = fminf(al, be) > cx.tiny && gm * gm > cx.tol2 * (al * be);
+    if (!__any_sync(kFull, need)) return;   // warp-uniform: nothing to rotate this round
     float cs = 1.f, sn = 0.f, nal = al, nbe = be;
-    if (fminf(al, be) > cx.tiny && fabsf(gm) > cx.tol * sqrtf(al * be)) {
-        const float zeta = (be - al) / (2.f * gm);
-        const float t = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
+    if (need) {
+        // zeta and t set the angle only; c and s are formed from t with
+        // correctly rounded operations, so c^2 + s^2 = 1 to rounding
+        const float zeta = __fdividef(be - al, 2.f * gm);
+        const float t = __fdividef(copysignf(1.f, zeta), fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
         cs = 1.f / sqrtf(fmaf(t, t, 1.f));
         sn = cs * t;
         nal = fmaf(-t, gm, al);
@@ -286,7 +366,7 @@ __device__ __forceinline__ void jacobi_round(float (&a)[16][NR], const JacobiCtx
     __syncwarp();
     if ((lane & 3) == 0) {
         cx.par[ip] = make_float2(cs, sn);
-        if (sn != 0.f) {
+        if (need) {
             cx.nrm[p] = nal;
             cx.nrm[q] = nbe;
             *cx.any = 1;
@@ -475,7 +555,6 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
     float* tau2 = sm + 384;
     float* vd2 = sm + 512;
     float* al2 = sm + 640;
-    float* nrm2 = sm + 768;                    // 4
     float* sig2 = sm + 772;                    // 128
     int* rnk = reinterpret_cast<int*>(sm + 900);   // 128
     float* wnrm = sm + 1028;                   // kWarps x 16
@@ -486,6 +565,7 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
     int* ncomp = flags + 8;
     float* fro = reinterpret_cast<float*>(flags + 10);
     int* cflag = flags + 16;                   // 128: rank slot awaiting completion
+    float* vring = reinterpret_cast<float*>(flags + 144);   // 2 x 192: reflectors of the core QR
 
     const int64_t hidx = (int64_t)layer * f.BH + bh;
     const float* gB = f.basis + hidx * d * R;
@@ -530,36 +610,67 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
     }
     __syncthreads();
 
-    // ---- (b) Householder QR of [B | X^T]; R_E; Q in place, parked in global scratch
-    house_qr(A, ldm, d, c, n, 0, tau1, vd1, al1, nrm2);
-    for (int e = tid; e < k * b; e += kThreads) {
-        const int i = e / b, t = e - (e / b) * b;
-        REb[e] = (i < t) ? A[(R + i) * ldm + R + t] : ((i == t) ? al1[R + t] : 0.f);
-    }
-    __syncthreads();   // R_E read before form_q clears the upper triangle
-    if constexpr (k > 0) {
-        form_q(A, ldm, R, k, tau1, vd1);
-        for (int e = tid; e < d * k; e += kThreads) {
-            const int i = e / k, q = e - (e / k) * k;
-            gQ[e] = A[i * ldm + R + q];
+    // ---- (b) Householder QR of [B | X^T] in registers; R_E; Q to global scratch
+    const int cs = warp * 8 + (lane & 7), prt = lane >> 3;
+    {
+        constexpr int CPT1 = (c + 63) / 64;
+        float x[CPT1][32];
+#pragma unroll
+        for (int t = 0; t < CPT1; ++t)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int col = cs + 64 * t;
+                x[t][e] = col < c ? A[(prt * 32 + e) * ldm + col] : 0.f;
+            }
+        __syncthreads();   // region A now holds the reflectors (n x d)
+        house_qr_reg<32, CPT1>(x, c, n, A, d, true, tau1, vd1, al1);
+#pragma unroll
+        for (int t = 0; t < CPT1; ++t) {
+            const int col = cs + 64 * t;
+            if (col >= R && col < R + b) {
+                const int tt = col - R;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = prt * 32 + e - R;
+                    if (i >= 0 && i < k) REb[i * b + tt] = (i < tt) ? x[t][e] : ((i == tt) ? al1[col] : 0.f);
+                }
+            }
         }
     }
-    __syncthreads();
+    if constexpr (k > 0) form_q_reg(A, R, k, n, tau1, vd1, gQ);
+    __syncthreads();   // R_E complete; reflectors no longer read
 
-    // ---- (c) core K = [[diag S, 0], [P, R_E^T]] in region A, then its QR
-    for (int e = tid; e < m * n; e += kThreads) {
-        const int i = e / n, j = e - (e / n) * n;
-        float v;
-        if (i < R) {
-            v = (i == j) ? gS[i] : 0.f;
-        } else {
-            const int t = i - R;
-            v = (j < R) ? Pb[t * ldp + j] : REb[(j - R) * b + t];
-        }
-        A[i * ldk + j] = v;
+    // ---- (c) QR of the core K = [[diag S, 0], [P, R_E^T]] in registers; R to region A
+    {
+        constexpr int RPP2 = ((m + 3) / 4 + 3) / 4 * 4;
+        constexpr int CPT2 = (n + 63) / 64;
+        float x[CPT2][RPP2];
+#pragma unroll
+        for (int t = 0; t < CPT2; ++t)
+#pragma unroll
+            for (int e = 0; e < RPP2; ++e) {
+                const int col = cs + 64 * t, row = prt * RPP2 + e;
+                float v = 0.f;
+                if (col < n && row < m) {
+                    if (row < R) {
+                        v = (row == col) ? gS[row] : 0.f;
+                    } else {
+                        const int tt = row - R;
+                        v = (col < R) ? Pb[tt * ldp + col] : REb[(col - R) * b + tt];
+                    }
+                }
+                x[t][e] = v;
+            }
+        house_qr_reg<RPP2, CPT2>(x, n, n, vring, 4 * RPP2, false, tau2, vd2, al2);
+#pragma unroll
+        for (int t = 0; t < CPT2; ++t)
+#pragma unroll
+            for (int e = 0; e < RPP2; ++e) {
+                const int col = cs + 64 * t, row = prt * RPP2 + e;
+                if (col < n && row <= col) A[row * ldk + col] = (row == col) ? al2[col] : x[t][e];
+            }
     }
     __syncthreads();
-    house_qr(A, ldk, m, n, n, R, tau2, vd2, al2, nrm2);
 
     // ---- one-sided Jacobi on the columns of R^T (warps 0..G-1)
     float a[16][NR];
@@ -575,7 +686,7 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
             }
         }
         float* nrm = wnrm + g * 16;
-        JacobiCtx cx{nrm, wpar + g * 8, wany + g, jacobi_tol(n), 0.f, lane};
+        JacobiCtx cx{nrm, wpar + g * 8, wany + g, jacobi_tol(n) * jacobi_tol(n), 0.f, lane};
         {
             const float v = col_norms16<NR>(a, lane);
             float s = ((lane & 1) == 0) ? v : 0.f;
