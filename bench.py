@@ -174,6 +174,28 @@ def oracle_sample(wl, budget_s: float = 15.0, seed: int = 0):
 # ---------------------------------------------------------------------------
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over all ranks (the slowest replica sets the time)."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(ms_max: float, steps: int, world: int) -> float:
+    """Whole-job decode steps/s: every rank runs its own replica (own batch),
+    so the job completes steps * 64 decode steps per rank in the slowest
+    rank's time."""
+    return steps * BLOCK * world / (ms_max / 1e3)
+
+
+def replica_seeds(rank: int):
+    """Seeds of the K, V and query streams of one replica (distinct per rank)."""
+    return 1000 * rank + 1, 1000 * rank + 2, 1000 * rank + 3
+
+
 def run_iskv(args, rank, world, local_rank):
     import torch
 
@@ -198,10 +220,9 @@ def run_iskv(args, rank, world, local_rank):
     cache = ik.Cache(cfg)
     kdt = torch.bfloat16
     nh = L * Bsz * H
-    ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=1000 * rank + 1, device=dev,
-                        dtype=kdt)
-    vs = synth.KVStream(synth.spec_for(wl["gen"], "V"), nh, seed=1000 * rank + 2, device=dev,
-                        dtype=kdt)
+    seed_k, seed_v, seed_q = replica_seeds(rank)
+    ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=seed_k, device=dev, dtype=kdt)
+    vs = synth.KVStream(synth.spec_for(wl["gen"], "V"), nh, seed=seed_v, device=dev, dtype=kdt)
 
     # ---- prefill (untimed): fold with postponed rewrites, one rewrite per 64 folds
     t_pre = time.time()
@@ -225,7 +246,7 @@ def run_iskv(args, rank, world, local_rank):
     # ---- decode inputs for every step, resident in HBM
     kk = ks.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
     vv = vs.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
-    qq = synth.query_batch(n_steps * L * Bsz * Hq, D, seed=1000 * rank + 3, device=dev,
+    qq = synth.query_batch(n_steps * L * Bsz * Hq, D, seed=seed_q, device=dev,
                            dtype=kdt).view(n_steps, L, Bsz, Hq, D)
     outs = torch.empty(L, Bsz, Hq, D, dtype=torch.float32, device=dev)
     kk = kk.view(n_steps, L, Bsz, H, 1, D)
@@ -263,13 +284,6 @@ def run_iskv(args, rank, world, local_rank):
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         period()
     barrier()
@@ -285,10 +299,9 @@ def run_iskv(args, rank, world, local_rank):
     e_end.record(stream)
     barrier()
     clk = clocks.stop()
-    ms = max_over_ranks(e_start.elapsed_time(e_end))
+    ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
     per_step_ms = ms / args.steps
-    decode_steps = args.steps * BLOCK * world
-    value = decode_steps / (ms / 1e3)
+    value = job_value(ms, args.steps, world)
 
     # decode-attention roofline from the events taken inside the timed region
     peak, peak_src = _peaks()
@@ -340,8 +353,8 @@ def run_iskv(args, rank, world, local_rank):
         period(host=(hk, hv, hq, ho))
     x1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(x0.elapsed_time(x1))
-    e2e_value = e2e_periods * BLOCK * world / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, dev)
+    e2e_value = job_value(e2e_ms, e2e_periods, world)
     h2d = BLOCK * L * (2 * Bsz * H * D * kvb + Bsz * Hq * D * kvb)
     d2h = BLOCK * L * Bsz * Hq * D * 4
     status = cache.status()
