@@ -44,6 +44,7 @@ struct iskv_cache {
     float* qscr_v = nullptr;
     int* seg_rows = nullptr;
     float* partial = nullptr;
+    int* done = nullptr;          // per-head arrival counters of the fused decode combine
     float2* rope = nullptr;
     int* status = nullptr;
     void* stage_in = nullptr;     // host-input staging
@@ -130,7 +131,7 @@ int64_t ready_of(const iskv_cache* h, int layer) {
 void free_all(iskv_cache* h) {
     void* ptrs[] = {h->ring_k, h->ring_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
-                    h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->rope, h->status, h->stage_in, h->stage_out};
+                    h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -269,6 +270,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     rc = rc ? rc : dalloc(&h->partial, (size_t)c.batch * c.q_heads * h->max_splits *
                                            (2 + c.rank_v + d) * 4);
     rc = rc ? rc : dalloc(&h->status, 16);
+    rc = rc ? rc : dalloc(&h->done, (size_t)h->BH * 4);
     h->stage_in_bytes = kStageBytes;
     h->stage_out_bytes = kStageBytes;
     rc = rc ? rc : dalloc(&h->stage_in, h->stage_in_bytes);
@@ -298,6 +300,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
             cudaMemsetAsync(h->coef_k, 0, heads * h->n_max * c.rank_k * h->coef_bytes, s) != cudaSuccess ||
             cudaMemsetAsync(h->coef_v, 0, heads * h->n_max * c.rank_v * h->coef_bytes, s) != cudaSuccess ||
             cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess ||
+            cudaMemsetAsync(h->done, 0, (size_t)h->BH * 4, s) != cudaSuccess ||
             cudaMemsetAsync(h->seg_rows, 0, (size_t)c.layers * h->D * 4, s) != cudaSuccess ||
             launch_init_factor(view(h, ISKV_WHICH_K), c.layers, s) != cudaSuccess ||
             launch_init_factor(view(h, ISKV_WHICH_V), c.layers, s) != cudaSuccess)
@@ -471,6 +474,8 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.partial = h->partial;
         t.rope = a.rope;
         t.status = h->status;
+        t.out = od;
+        t.done = h->done;
         t.layer = layer;
         t.B = c.batch;
         t.Hkv = c.kv_heads;
@@ -504,10 +509,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
                     break;
                 }
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
-        CU(launch_decode_tc(t, s));
-        a.splits = slots_c;
-        a.splits_total = slots_c;
-        CU(launch_combine(a, od, s));
+        CU(launch_decode_tc(t, s));   // merges the partials of each head itself
         if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
         return ISKV_OK;
     }

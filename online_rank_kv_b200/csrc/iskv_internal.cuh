@@ -118,6 +118,8 @@ struct DecodeTcArgs {
     float* partial;              // [B][Hq][splits_total][2 + r_V + d]
     const float2* rope;          // [>= 128 positions][d/2], or null
     int* status;
+    float* out;                  // [B][Hq][d] fp32: written by the last CTA of each head
+    int* done;                   // [BH] arrival counters, zero between calls
     int layer, B, Hkv, Hq, g;
     int64_t n_c, T;
     int tiles_c;                 // folded-row tiles per head: ceil(n_c / 128)

@@ -54,7 +54,7 @@ constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4
 constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
 constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
 constexpr int kBufCols = 160;    // per TMEM buffer: K^ 128 | S 16 | O 16
-constexpr int kCsCol = 2 * kBufCols;   // per-row RoPE table: cos 64 | sin 64 columns
+constexpr int kCsCol = 2 * kBufCols;   // per-row RoPE table: cos 64 | sin 64 | -sin 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Bars {
@@ -88,13 +88,31 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" :::
 __device__ __forceinline__ void group_sync(int grp) {
     asm volatile("bar.sync %0, 128;" ::"r"(2 + grp) : "memory");
 }
+// the same barrier, returning whether any of the group's threads passed true
+__device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(2 + grp)
+        : "memory");
+    return r != 0;
+}
+// a tile's probabilities use the running max while no score passes it by
+// more than this (p <= e^8); otherwise the tile takes the exact rescale
+constexpr float kLazyMax = 8.f;
 
 // offsets of the tf32 (K-major, 8 x 4 core matrices) and bf16 (8 x 8) B operands
 __device__ __forceinline__ int qb_off(int n, int k) {
     return ((n >> 3) * (kTile / 4) + (k >> 2)) * 32 + (n & 7) * 4 + (k & 3);
 }
+// p as the value MMA's B operand, MN-major: [token][16] in 8 x 8 blocks, so one
+// thread's (token's) 8 values of an n-block are one 16-byte row
 __device__ __forceinline__ int pb_off(int n, int k) {
-    return ((n >> 3) * (kTile / 8) + (k >> 3)) * 64 + (n & 7) * 8 + (k & 7);
+    return ((k >> 3) * (kPN / 8) + (n >> 3)) * 64 + (k & 7) * 8 + (n & 7);
 }
 
 template <int G>
@@ -120,6 +138,7 @@ decode_tc_kernel(DecodeTcArgs a) {
     // barrier so that all 256 epilogue threads leave the loop together
     volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);
     volatile int* flag_max = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2]
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 24);
     float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
     float* mlx = reinterpret_cast<float*>(smem + 256);          // [2 groups][m 8 | l 8]
     const SmemPlan P = plan_smem(rK, rV, ns, nbk);
@@ -296,16 +315,18 @@ decode_tc_kernel(DecodeTcArgs a) {
         if (grp == 0) {
 #pragma unroll
             for (int c0 = 0; c0 < 64; c0 += 16) {
-                uint32_t vc[16], vs[16];
+                uint32_t vc[16], vs[16], vn[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     float2 v = make_float2(1.f, 0.f);
                     if (a.rope) v = a.rope[row * 64 + c0 + u];
                     vc[u] = __float_as_uint(v.x);
                     vs[u] = __float_as_uint(v.y);
+                    vn[u] = __float_as_uint(-v.y);
                 }
                 tmem_st16(tcs + lane_base + c0, vc);
                 tmem_st16(tcs + lane_base + 64 + c0, vs);
+                tmem_st16(tcs + lane_base + 128 + c0, vn);
             }
             tmem_wait_st();
         }
@@ -313,10 +334,9 @@ decode_tc_kernel(DecodeTcArgs a) {
         const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
         const uint32_t idesc_s = idesc_f32acc(2, kTile, kQN, 0, 0);
-        const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 0);
-        const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 0);   // exact rows: M = d
+        const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 1);
+        const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 1);   // exact rows: M = d
         const uint32_t sbo_q = (kTile / 4) * 128;
-        const uint32_t sbo_p = (kTile / 8) * 128;
         const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
         float* gred = red + grp * 64;             // [max 4 x 8 | l 4 x 8] of this group
         const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
@@ -363,23 +383,30 @@ decode_tc_kernel(DecodeTcArgs a) {
             if (stop) break;
             bool have_prev = false, prev_win = false;
             int last = -1;
-            for (int n = n0 + ((n0 & 1) != grp ? 1 : 0); n < s1; n += 2) {
+            // first position of a tile (folded tiles of 128 rows, then exact tiles of 64)
+            auto tile_j0 = [&](int nn) {
+                const int lc = (int)((f0 + nn) % tph);
+                return lc >= tiles_c ? a.n_c + (int64_t)(lc - tiles_c) * kWinTile : (int64_t)lc * kTile;
+            };
+            // cos / sin(j0 w_i) for i = gt & 63 (the only frequency this thread
+            // rotates the query by), fetched one tile of the group ahead
+            const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
+            float2 rq = make_float2(1.f, 0.f);
+            if (a.rope && n_first < s1) rq = a.rope[tile_j0(n_first) * 64 + (gt & 63)];
+            for (int n = n_first; n < s1; n += 2) {
                 const int st = n % ns;
                 const int local = (int)((f0 + n) % tph);
                 const bool win = local >= tiles_c;    // exact rows (64-token tile)
-                const int64_t j0 = win ? a.n_c + (int64_t)(local - tiles_c) * kWinTile : (int64_t)local * kTile;
+                const int64_t j0 = tile_j0(n);
                 const int64_t lim = win ? a.T : a.n_c;
                 const int span = win ? kWinTile : kTile;
                 const int valid = (int)((lim - j0) < span ? (lim - j0) : span);
+                const float2 rq_cur = rq;
+                if (a.rope && n + 2 < s1) rq = a.rope[tile_j0(n + 2) * 64 + (gt & 63)];
                 // q' = R_{j0}^T q, tf32 hi / lo parts as the score MMA's B operand
                 for (int item = gt; item < g * 64; item += 128) {
                     const int h = item >> 6, i = item & 63;
-                    float c0 = 1.f, s0 = 0.f;
-                    if (a.rope) {
-                        const float2 v = a.rope[j0 * 64 + i];
-                        c0 = v.x;
-                        s0 = v.y;
-                    }
+                    const float c0 = rq_cur.x, s0 = rq_cur.y;
                     const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
                     const float y1 = fmaf(c0, x1, s0 * x2);
                     const float y2 = fmaf(c0, x2, -s0 * x1);
@@ -420,15 +447,26 @@ decode_tc_kernel(DecodeTcArgs a) {
                             }
                         }
                     }
+                    uint32_t nn[16];
                     tmem_ld16(tcs + lane_base + c0, cc);
                     tmem_ld16(tcs + lane_base + 64 + c0, ss);
+                    tmem_ld16(tcs + lane_base + 128 + c0, nn);
                     tmem_wait_ld();
+                    // (k1, k2) -> (k1 c - k2 s, k1 s + k2 c), two columns per packed
+                    // fp32 op; the tf32 score MMA reads the fp32 bits truncated
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const float k1 = __uint_as_float(x1[u]), k2 = __uint_as_float(x2[u]);
-                        const float co = __uint_as_float(cc[u]), si = __uint_as_float(ss[u]);
-                        x1[u] = to_tf32(fmaf(k1, co, -k2 * si));
-                        x2[u] = to_tf32(fmaf(k1, si, k2 * co));
+                    for (int u = 0; u < 16; u += 2) {
+                        const float2 k1 = make_float2(__uint_as_float(x1[u]), __uint_as_float(x1[u + 1]));
+                        const float2 k2 = make_float2(__uint_as_float(x2[u]), __uint_as_float(x2[u + 1]));
+                        const float2 co = make_float2(__uint_as_float(cc[u]), __uint_as_float(cc[u + 1]));
+                        const float2 si = make_float2(__uint_as_float(ss[u]), __uint_as_float(ss[u + 1]));
+                        const float2 ns = make_float2(__uint_as_float(nn[u]), __uint_as_float(nn[u + 1]));
+                        const float2 y1 = __ffma2_rn(k1, co, __fmul2_rn(k2, ns));
+                        const float2 y2 = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
+                        x1[u] = __float_as_uint(y1.x);
+                        x1[u + 1] = __float_as_uint(y1.y);
+                        x2[u] = __float_as_uint(y2.x);
+                        x2[u + 1] = __float_as_uint(y2.y);
                     }
                     tmem_st16(kh + lane_base + c0, x1);
                     tmem_st16(kh + lane_base + 64 + c0, x2);
@@ -460,31 +498,66 @@ decode_tc_kernel(DecodeTcArgs a) {
                 tmem_ld16(kh + 128 + lane_base, sv);
                 tmem_wait_ld();
                 float sc[G];
+                bool over = false;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     sc[h] = (row < valid) ? (__uint_as_float(sv[h]) + __uint_as_float(sv[G + h])) * a.scale
                                           : -INFINITY;
-                    const float wm = warp_max(sc[h]);
-                    if (lane == 0) gred[sp * 8 + h] = wm;
+                    over |= sc[h] > m_run[h] + kLazyMax;   // always true while m_run = -inf
                 }
-                tc_fence_before();
-                group_sync(grp);
+                // p of this row, bf16 hi parts then lo parts, one or two 16-byte rows
+                auto store_p = [&](const float (&pv)[G]) {
+                    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                    __nv_bfloat16 hv[2 * G];
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float tmax = fmaxf(fmaxf(gred[h], gred[8 + h]), fmaxf(gred[16 + h], gred[24 + h]));
-                    const float m_new = fmaxf(m_run[h], tmax);
-                    const float al = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
-                    const float p = (sc[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_new);
-                    l_thr[h] = fmaf(l_thr[h], al, p);
-                    m_run[h] = m_new;
-                    alpha[h] = al;
-                    const __nv_bfloat16 ph = __float2bfloat16_rn(p);
-                    pbb[pb_off(h, row)] = ph;
-                    pbb[pb_off(G + h, row)] = __float2bfloat16_rn(p - __bfloat162float(ph));
-                }
+                    for (int h = 0; h < G; ++h) {
+                        hv[h] = __float2bfloat16_rn(pv[h]);
+                        hv[G + h] = __float2bfloat16_rn(pv[h] - __bfloat162float(hv[h]));
+                    }
+#pragma unroll
+                    for (int e = 0; e < 2 * G; ++e) {
+                        const uint32_t bits = (uint32_t)__bfloat16_as_ushort(hv[e]);
+                        w[e >> 1] |= (e & 1) ? (bits << 16) : bits;
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(pbb + pb_off(0, row));
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (2 * G > 8) reinterpret_cast<uint4*>(pbb + pb_off(8, row))[0] = make_uint4(w[4], w[5], w[6], w[7]);
+                };
+                float pv[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    pv[h] = (sc[h] == -INFINITY || m_run[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_run[h]);
+                store_p(pv);
                 fence_async_smem();
                 tc_fence_before();
-                group_sync(grp);                      // P of tile n complete, max read
+                if (group_sync_or(grp, over)) {          // P complete; rare: exact rescale
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float wm = warp_max(sc[h]);
+                        if (lane == 0) gred[sp * 8 + h] = wm;
+                    }
+                    group_sync(grp);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float tmax = fmaxf(fmaxf(gred[h], gred[8 + h]), fmaxf(gred[16 + h], gred[24 + h]));
+                        const float m_new = fmaxf(m_run[h], tmax);
+                        const float al = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
+                        pv[h] = (sc[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_new);
+                        l_thr[h] = fmaf(l_thr[h], al, pv[h]);
+                        m_run[h] = m_new;
+                        alpha[h] = al;
+                    }
+                    store_p(pv);
+                    fence_async_smem();
+                    tc_fence_before();
+                    group_sync(grp);                  // rescaled P complete, maxima read
+                } else {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        l_thr[h] += pv[h];
+                        alpha[h] = 1.f;
+                    }
+                }
                 if (gt == 0 && !*abort_flag) {
                     mbar_arrive(&bars->kfree[grp]);   // K^/S of this buffer may be overwritten
                     tc_fence_after();
@@ -493,13 +566,13 @@ decode_tc_kernel(DecodeTcArgs a) {
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
                         for (int ks = 0; ks < kTile / 16; ++ks)
                             mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
-                                       desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_o, ks != 0);
+                                       desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
                     } else {
                         // O = V^T P over 64 exact rows: A = V tile, MN-major, M = d
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + kWinBytes);
                         for (int ks = 0; ks < kWinTile / 16; ++ks)
                             mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
-                                       desc_noswizzle(p0 + ks * 256, 128, sbo_p), idesc_ow, ks != 0);
+                                       desc_noswizzle(p0 + ks * 512, 256, 128), idesc_ow, ks != 0);
                     }
                     mma_commit(&bars->o_full[grp]);
                     mma_commit(&bars->empty[st]);
@@ -569,14 +642,73 @@ decode_tc_kernel(DecodeTcArgs a) {
                         Pp[1] = ml0[kMaxGroup + h] * w0 + ml1[kMaxGroup + h] * w1;
                     }
                 }
-                // this CTA ends the head: mark the head's unused compressed slots empty
-                if (gt == 0 && f1 >= (int64_t)(head + 1) * tph) {
-                    for (int h = 0; h < g; ++h)
-                        for (int sl = slot + 1; sl < a.slots_c; ++sl) {
-                            float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + sl) * stride;
-                            Pp[0] = -INFINITY;
-                            Pp[1] = 0.f;
+            }
+            // the last CTA to publish a partial of this head merges all of them
+            // (log-sum-exp), applies B_V^T once per query head and writes out;
+            // no CTA waits for another, so no ordering between CTAs is assumed
+            __threadfence();
+            epi_sync();
+            {
+                const int c_first = (int)(((int64_t)head * tph) / a.tiles_per_cta);
+                const int c_last = (int)((((int64_t)head + 1) * tph - 1) / a.tiles_per_cta);
+                if (ept == 0) {
+                    const int before = atomicAdd(a.done + head, 1);
+                    const int last = before == c_last - c_first;
+                    if (last) a.done[head] = 0;   // ready for the next call
+                    *last_flag = last;
+                }
+                epi_sync();
+                if (*last_flag) {
+                    __threadfence();
+                    const int bq = head / a.Hkv, kvh = head % a.Hkv;
+                    const int nsl = c_last - c_first + 1;
+                    const int stride = 2 + rV + d;
+                    // exchange area (q' buffers, 16 KB): merged acc [8][128], slot
+                    // weights [8][256], 1/L [8]
+                    static_assert((kMaxGroup * 128 + kMaxGroup * 256 + kMaxGroup) * 4 <= 2 * kQN * kTile * 4,
+                                  "combine scratch fits");
+                    float* sacc = reinterpret_cast<float*>(qb);
+                    float* sw = sacc + kMaxGroup * 128;
+                    float* sinv = sw + kMaxGroup * 256;
+                    const float* Pbase = a.partial + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * a.splits_total * stride;
+                    if (ept < g) {
+                        const float* Ph = Pbase + (int64_t)ept * a.splits_total * stride;
+                        float M = -INFINITY;
+                        for (int sl = 0; sl < nsl; ++sl) M = fmaxf(M, __ldcg(Ph + sl * stride));
+                        float L = 0.f;
+                        for (int sl = 0; sl < nsl; ++sl) {
+                            const float m = __ldcg(Ph + sl * stride);
+                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M);
+                            sw[ept * 256 + sl] = w;
+                            L = fmaf(w, __ldcg(Ph + sl * stride + 1), L);
                         }
+                        sinv[ept] = 1.f / L;
+                    }
+                    epi_sync();
+                    for (int e = ept; e < g * rV; e += kEpi) {
+                        const int h = e / rV, c = e - (e / rV) * rV;
+                        const float* Ph = Pbase + (int64_t)h * a.splits_total * stride;
+                        float v = 0.f;
+                        for (int sl = 0; sl < nsl; ++sl) v = fmaf(sw[h * 256 + sl], __ldcg(Ph + sl * stride + 2 + c), v);
+                        sacc[h * 128 + c] = v;
+                    }
+                    epi_sync();
+                    const float* Bv = a.V.basis + ((int64_t)a.layer * BH + head) * d * rV;
+                    for (int e = ept; e < g * d; e += kEpi) {
+                        const int h = e / d, i = e - (e / d) * d;
+                        const float* Ph = Pbase + (int64_t)h * a.splits_total * stride;
+                        float v = 0.f;
+                        for (int sl = 0; sl < nsl; ++sl) v = fmaf(sw[h * 256 + sl], __ldcg(Ph + sl * stride + 2 + rV + i), v);
+                        const float* br = Bv + (int64_t)i * rV;
+                        for (int c = 0; c < rV; c += 4) {
+                            const float4 b4 = *reinterpret_cast<const float4*>(br + c);
+                            v = fmaf(sacc[h * 128 + c], b4.x, v);
+                            v = fmaf(sacc[h * 128 + c + 1], b4.y, v);
+                            v = fmaf(sacc[h * 128 + c + 2], b4.z, v);
+                            v = fmaf(sacc[h * 128 + c + 3], b4.w, v);
+                        }
+                        a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + i] = v * sinv[h];
+                    }
                 }
             }
             epi_sync();                               // exchange area free again
