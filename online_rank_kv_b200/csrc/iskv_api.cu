@@ -499,15 +499,18 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         if (slots_c > h->max_splits) return ISKV_ERR_UNSUPPORTED;
         t.slots_c = slots_c;
         t.splits_total = slots_c;
-        // deepest pipeline that fits: two basis buffers if possible, else one
+        // deepest pipeline that fits: stages first, then two basis buffers, then
+        // double-buffered q'
         t.stages = 0;
-        for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
-            for (int ns = 4; ns >= 2; --ns)
-                if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk) <= 227 * 1024) {
-                    t.stages = ns;
-                    t.basis_bufs = nbk;
-                    break;
-                }
+        for (int ns = 4; ns >= 2 && t.stages == 0; --ns)
+            for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
+                for (int nqb = 2; nqb >= 1; --nqb)
+                    if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk, nqb) <= 227 * 1024) {
+                        t.stages = ns;
+                        t.basis_bufs = nbk;
+                        t.q_bufs = nqb;
+                        break;
+                    }
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
         CU(launch_decode_tc(t, s));   // merges the partials of each head itself
         if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));

@@ -49,7 +49,7 @@ using namespace tc;
 
 constexpr int kTile = 128;
 constexpr int kWinTile = 64;     // exact-row tiles: 64 rows never wrap the ring
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
 constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
 constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
@@ -59,16 +59,17 @@ constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Bars {
     uint64_t full[4], empty[4];
-    uint64_t bk_full[2], bk_empty[2];
+    uint64_t bk_full[2], bk_empty[4];      // bk_empty[buffer * 2 + group]
     uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
-    uint64_t drain[2];   // abort path: completion of each issuer's outstanding MMAs
+    uint64_t krot_ready[2], p_ready[2];   // epilogue -> group issuer: K_rot and q', P written
+    uint64_t drain[3];   // abort path: completion of each issuer's outstanding MMAs
 };
 
 struct SmemPlan {
     uint32_t bk, stage, stage_k, stage_bytes, qb, pb, total;
 };
 
-__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk) {
+__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, int nqb) {
     SmemPlan p;
     uint32_t off = 1024;                                        // barriers, scratch
     p.bk = off;                off += nbk * (2 * kTile * rK * 2);  // nbk heads x (hi, lo)
@@ -77,7 +78,7 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk) {
     if (sb < 2 * kWinTile * kHeadDim * 2) sb = 2 * kWinTile * kHeadDim * 2;   // exact K and V rows
     p.stage_bytes = sb + 1024;
     p.stage = off;             off += ns * p.stage_bytes;
-    p.qb = off;                off += 2 * (kQN * kTile * 4);
+    p.qb = off;                off += 2 * nqb * (kQN * kTile * 4);   // [group][nqb] q' buffers
     p.pb = off;                off += 2 * (kPN * kTile * 2);
     p.total = off;
     return p;
@@ -125,7 +126,7 @@ decode_tc_kernel(DecodeTcArgs a) {
     if (f0 >= f1) return;
     const int ntiles = (int)(f1 - f0);
     const int tph = a.tiles_per_head;
-    const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs;
+    const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs, nqb = a.q_bufs;
     constexpr int g = G;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int d = kHeadDim;
@@ -141,7 +142,7 @@ decode_tc_kernel(DecodeTcArgs a) {
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 24);
     float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
     float* mlx = reinterpret_cast<float*>(smem + 256);          // [2 groups][m 8 | l 8]
-    const SmemPlan P = plan_smem(rK, rV, ns, nbk);
+    const SmemPlan P = plan_smem(rK, rV, ns, nbk, nqb);
     float* sq = reinterpret_cast<float*>(smem + P.total);       // queries of the head, g x d fp32
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
@@ -161,22 +162,24 @@ decode_tc_kernel(DecodeTcArgs a) {
             mbar_init(&bars->full[i], 1);
             mbar_init(&bars->empty[i], 1);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(&bars->bk_empty[i], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->bk_full[i], 1);
-            mbar_init(&bars->bk_empty[i], 1);
             mbar_init(&bars->kh_full[i], 1);
             mbar_init(&bars->kfree[i], 1);
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->o_full[i], 1);
-            mbar_init(&bars->drain[i], 1);
+            mbar_init(&bars->krot_ready[i], kEpi / 2);
+            mbar_init(&bars->p_ready[i], 1);
         }
+        for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
         *abort_flag = 0;
         flag_max[0] = 0;
         flag_max[1] = 0;
         fence_mbar_init();
     }
     // zero the padding rows (n >= 2g) of the q' and p operands once
-    for (int e = tid; e < 2 * kQN * kTile; e += kThreads) {
+    for (int e = tid; e < 2 * nqb * kQN * kTile; e += kThreads) {
         const int buf = e / (kQN * kTile), w = e % (kQN * kTile);
         const int n = w / kTile, k = w % kTile;
         if (n >= 2 * g) qb[buf * kQN * kTile + qb_off(n, k)] = 0u;
@@ -210,7 +213,8 @@ decode_tc_kernel(DecodeTcArgs a) {
                 if (head != prev) {
                     ++hs;
                     const int hb = hs % nbk;
-                    if (hs >= nbk && !mbar_wait(&bars->bk_empty[hb], ((hs / nbk) - 1) & 1, deadline)) {
+                    if (hs >= nbk && (!mbar_wait(&bars->bk_empty[2 * hb], ((hs / nbk) - 1) & 1, deadline) ||
+                                      !mbar_wait(&bars->bk_empty[2 * hb + 1], ((hs / nbk) - 1) & 1, deadline))) {
                         fail();
                         break;
                     }
@@ -252,57 +256,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                     mbar_wait(&bars->full[n % ns], (n / ns) & 1, deadline + kWaitCycles);
             }
         }
-    } else if (warp == 1) {
-        // ---------------- reconstruction MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t idesc = idesc_f32acc(1, kTile, d, 0, 0);
-            const uint32_t sbo = (uint32_t)(rK / 8) * 128;
-            int hs = -1, prev = -1;
-            for (int n = 0; n < ntiles && !*abort_flag; ++n) {
-                const int64_t fi = f0 + n;
-                const int head = (int)(fi / tph);
-                if (head != prev) {
-                    ++hs;
-                    if (!mbar_wait(&bars->bk_full[hs % nbk], (hs / nbk) & 1, deadline)) {
-                        fail();
-                        break;
-                    }
-                    prev = head;
-                }
-                const int st = n % ns, b = n & 1;
-                if (!mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) {
-                    fail();
-                    break;
-                }
-                if (n >= 2 && !mbar_wait(&bars->kfree[b], ((n >> 1) - 1) & 1, deadline)) {
-                    fail();
-                    break;
-                }
-                if ((int)(fi % tph) >= tiles_c) {
-                    // exact rows: nothing to rebuild, the epilogue reads them directly
-                    mbar_arrive(&bars->kh_full[b]);
-                } else {
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(stage + st * stage_bytes);
-                    const uint32_t b0 = smem_u32(bk + (hs % nbk) * bk_bytes);
-                    const uint32_t dk = tmem + b * kBufCols;
-                    for (int ks = 0; ks < rK / 16; ++ks)
-                        for (int part = 0; part < 2; ++part) {
-                            const uint64_t ad = desc_noswizzle(a0 + ks * 256, 128, sbo);
-                            const uint64_t bd = desc_noswizzle(b0 + part * (kTile * rK * 2) + ks * 256, 128, sbo);
-                            mma_f16_ss(dk, ad, bd, idesc, (ks | part) != 0);
-                        }
-                    mma_commit(&bars->kh_full[b]);
-                }
-                const bool seg_end = (n + 1 == ntiles) || ((f0 + n + 1) / tph != head);
-                if (seg_end) mma_commit(&bars->bk_empty[hs % nbk]);
-            }
-            if (*abort_flag) {                        // let issued MMAs finish (bounded)
-                mma_commit(&bars->drain[0]);
-                mbar_wait(&bars->drain[0], 0, deadline + kWaitCycles);
-            }
-        }
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         // ---------------- epilogue: two groups of 4 warps, alternate tiles ----------------
         const int ept = tid - 64;                 // 0..255
         const int grp = ept >> 7;                 // tiles n with n % 2 == grp
@@ -333,14 +287,9 @@ decode_tc_kernel(DecodeTcArgs a) {
         const int MV = rV <= 64 ? 64 : 128;
         const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
-        const uint32_t idesc_s = idesc_f32acc(2, kTile, kQN, 0, 0);
-        const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 1);
-        const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 1);   // exact rows: M = d
-        const uint32_t sbo_q = (kTile / 4) * 128;
-        const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
         float* gred = red + grp * 64;             // [max 4 x 8 | l 4 x 8] of this group
         const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
-        uint32_t* qbb = qb + grp * kQN * kTile;
+        uint32_t* qbb = qb + nqb * grp * kQN * kTile;   // the group's first q' buffer (head-end exchange)
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
 
         float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
@@ -384,39 +333,47 @@ decode_tc_kernel(DecodeTcArgs a) {
             bool have_prev = false, prev_win = false;
             int last = -1;
             // first position of a tile (folded tiles of 128 rows, then exact tiles of 64)
+            const int64_t hbase = (int64_t)head * tph;   // flattened index of the head's tile 0
             auto tile_j0 = [&](int nn) {
-                const int lc = (int)((f0 + nn) % tph);
+                const int lc = (int)(f0 + nn - hbase);
                 return lc >= tiles_c ? a.n_c + (int64_t)(lc - tiles_c) * kWinTile : (int64_t)lc * kTile;
             };
-            // cos / sin(j0 w_i) for i = gt & 63 (the only frequency this thread
-            // rotates the query by), fetched one tile of the group ahead
+            // q' = R_{j0}^T q of tile nn as tf32 hi / lo parts (the score MMA's B
+            // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
+            // for i = gt & 63, the only frequency this thread rotates by
+            auto build_q = [&](int nn, float2 rv) {
+                uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQN * kTile;
+                for (int item = gt; item < g * 64; item += 128) {
+                    const int h = item >> 6, i = item & 63;
+                    const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
+                    const float y1 = fmaf(rv.x, x1, rv.y * x2);
+                    const float y2 = fmaf(rv.x, x2, -rv.y * x1);
+                    const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
+                    qd[qb_off(h, i)] = t1;
+                    qd[qb_off(h, i + 64)] = t2;
+                    qd[qb_off(g + h, i)] = to_tf32(y1 - __uint_as_float(t1));
+                    qd[qb_off(g + h, i + 64)] = to_tf32(y2 - __uint_as_float(t2));
+                }
+                fence_async_smem();
+            };
+            auto rope_of = [&](int nn) {
+                return a.rope ? a.rope[tile_j0(nn) * 64 + (gt & 63)] : make_float2(1.f, 0.f);
+            };
             const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
-            float2 rq = make_float2(1.f, 0.f);
-            if (a.rope && n_first < s1) rq = a.rope[tile_j0(n_first) * 64 + (gt & 63)];
+            // two q' buffers: tile n + 2's q' is built while tile n's scores run;
+            // one buffer: each tile builds its own before its RoPE
+            if (nqb == 2 && n_first < s1) build_q(n_first, rope_of(n_first));
             for (int n = n_first; n < s1; n += 2) {
                 const int st = n % ns;
-                const int local = (int)((f0 + n) % tph);
+                const int local = (int)(f0 + n - hbase);
                 const bool win = local >= tiles_c;    // exact rows (64-token tile)
                 const int64_t j0 = tile_j0(n);
                 const int64_t lim = win ? a.T : a.n_c;
                 const int span = win ? kWinTile : kTile;
                 const int valid = (int)((lim - j0) < span ? (lim - j0) : span);
-                const float2 rq_cur = rq;
-                if (a.rope && n + 2 < s1) rq = a.rope[tile_j0(n + 2) * 64 + (gt & 63)];
-                // q' = R_{j0}^T q, tf32 hi / lo parts as the score MMA's B operand
-                for (int item = gt; item < g * 64; item += 128) {
-                    const int h = item >> 6, i = item & 63;
-                    const float c0 = rq_cur.x, s0 = rq_cur.y;
-                    const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
-                    const float y1 = fmaf(c0, x1, s0 * x2);
-                    const float y2 = fmaf(c0, x2, -s0 * x1);
-                    const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
-                    qbb[qb_off(h, i)] = t1;
-                    qbb[qb_off(h, i + 64)] = t2;
-                    qbb[qb_off(g + h, i)] = to_tf32(y1 - __uint_as_float(t1));
-                    qbb[qb_off(g + h, i + 64)] = to_tf32(y2 - __uint_as_float(t2));
-                }
-                fence_async_smem();
+                // the next tile's query rotation, loaded now, used after this tile's RoPE
+                const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
+                if (nqb == 1) build_q(n, rope_of(n));
                 // rotate this row of K^ by R_t, store back as tf32
                 if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
@@ -473,15 +430,9 @@ decode_tc_kernel(DecodeTcArgs a) {
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                group_sync(grp);                      // k_rot and q' of tile n complete
-                if (gt == 0 && !*abort_flag) {
-                    tc_fence_after();
-                    const uint32_t q0 = smem_u32(qbb);
-                    for (int ks = 0; ks < d / 8; ++ks)
-                        mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
-                                    idesc_s, ks != 0);
-                    mma_commit(&bars->s_full[grp]);
-                }
+                mbar_arrive(&bars->krot_ready[grp]);  // this row of K_rot and its q' share are in place
+                // the next tile's q' goes to the other buffer while this tile's scores run
+                if (nqb == 2 && n + 2 < s1) build_q(n + 2, rq_next);
                 // this group's previous tile: p^T C_V accumulated (before O is reused)
                 if (have_prev) {
                     if (!mbar_wait(&bars->o_full[grp], ((n - 2) >> 1) & 1, deadline)) fail();
@@ -558,25 +509,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                         alpha[h] = 1.f;
                     }
                 }
-                if (gt == 0 && !*abort_flag) {
-                    mbar_arrive(&bars->kfree[grp]);   // K^/S of this buffer may be overwritten
-                    tc_fence_after();
-                    const uint32_t p0 = smem_u32(pbb);
-                    if (!win) {
-                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
-                        for (int ks = 0; ks < kTile / 16; ++ks)
-                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
-                                       desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
-                    } else {
-                        // O = V^T P over 64 exact rows: A = V tile, MN-major, M = d
-                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + kWinBytes);
-                        for (int ks = 0; ks < kWinTile / 16; ++ks)
-                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
-                                       desc_noswizzle(p0 + ks * 512, 256, 128), idesc_ow, ks != 0);
-                    }
-                    mma_commit(&bars->o_full[grp]);
-                    mma_commit(&bars->empty[st]);
-                }
+                if (gt == 0) mbar_arrive(&bars->p_ready[grp]);   // P of tile n complete
                 have_prev = true;
                 prev_win = win;
                 last = n;
@@ -618,7 +551,7 @@ decode_tc_kernel(DecodeTcArgs a) {
             if (grp == 0) {
                 // log-sum-exp merge of the two groups, one partial slot per head
                 const float* x0 = reinterpret_cast<const float*>(qb);
-                const float* x1 = reinterpret_cast<const float*>(qb + kQN * kTile);
+                const float* x1 = reinterpret_cast<const float*>(qb + nqb * kQN * kTile);
                 const float* ml0 = mlx;
                 const float* ml1 = mlx + 2 * kMaxGroup;
                 const int bq = head / a.Hkv, kvh = head % a.Hkv;
@@ -714,9 +647,116 @@ decode_tc_kernel(DecodeTcArgs a) {
             epi_sync();                               // exchange area free again
             n0 = s1;
         }
-        if (ept == 0 && *abort_flag) {                // let issued MMAs finish (bounded)
-            mma_commit(&bars->drain[1]);
-            mbar_wait(&bars->drain[1], 0, deadline + kWaitCycles);
+    } else if (warp >= 10) {
+        // ---------------- MMA issuer of group warp - 10 ----------------
+        // per tile n of the group: K^ = C_K (B_hi + B_lo)^T (issued as soon as the
+        // group's previous score MMA has released the K^ buffer), scores once the
+        // epilogue has rotated K^ and written q', values once P is written
+        const int grp = warp - 10;
+        if (lane == 0) {
+            const int MV = rV <= 64 ? 64 : 128;
+            const uint32_t idesc_k = idesc_f32acc(1, kTile, d, 0, 0);
+            const uint32_t idesc_s = idesc_f32acc(2, kTile, kQN, 0, 0);
+            const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 1);
+            const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 1);   // exact rows: M = d
+            const uint32_t sbo_k = (uint32_t)(rK / 8) * 128;
+            const uint32_t sbo_q = (kTile / 4) * 128;
+            const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
+            const uint32_t kh = tmem + grp * kBufCols;
+            const uint32_t qg = smem_u32(qb + nqb * grp * kQN * kTile);
+            const uint32_t p0 = smem_u32(pb + grp * kPN * kTile);
+            // K^ of tile n into this group's buffer; exact-row tiles need none
+            auto recon = [&](int n, int hb, bool win) -> bool {
+                const int st = n % ns;
+                if (!mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) return false;
+                if (win) {
+                    mbar_arrive(&bars->kh_full[grp]);
+                    return true;
+                }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(stage + st * stage_bytes);
+                const uint32_t b0 = smem_u32(bk + hb * bk_bytes);
+                for (int ks = 0; ks < rK / 16; ++ks)
+                    for (int part = 0; part < 2; ++part)
+                        mma_f16_ss(kh, desc_noswizzle(a0 + ks * 256, 128, sbo_k),
+                                   desc_noswizzle(b0 + part * (kTile * rK * 2) + ks * 256, 128, sbo_k),
+                                   idesc_k, (ks | part) != 0);
+                mma_commit(&bars->kh_full[grp]);
+                return true;
+            };
+            bool ok = true;
+            int hs = -1, n0 = 0;
+            while (ok && n0 < ntiles && !*abort_flag) {
+                const int head = (int)((f0 + n0) / tph);
+                const int64_t hbase = (int64_t)head * tph;
+                int s1 = (int)(hbase + tph - f0);
+                if (s1 > ntiles) s1 = ntiles;
+                ++hs;
+                const int hb = hs % nbk;
+                const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
+                if (n_first < s1) {
+                    ok = mbar_wait(&bars->bk_full[hb], (hs / nbk) & 1, deadline) &&
+                         (n_first < 2 || mbar_wait(&bars->kfree[grp], ((n_first >> 1) - 1) & 1, deadline)) &&
+                         recon(n_first, hb, (int)(f0 + n_first - hbase) >= tiles_c);
+                }
+                for (int n = n_first; ok && n < s1; n += 2) {
+                    const int st = n % ns;
+                    const bool win = (int)(f0 + n - hbase) >= tiles_c;
+                    if (!mbar_wait(&bars->krot_ready[grp], (n >> 1) & 1, deadline)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQN * kTile * 4);
+                    for (int ks = 0; ks < d / 8; ++ks)
+                        mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
+                                    idesc_s, ks != 0);
+                    mma_commit(&bars->s_full[grp]);
+                    mma_commit(&bars->kfree[grp]);
+                    // K_rot of tile n consumed: rebuild tile n + 2 while the epilogue runs
+                    // this tile's softmax.  Its data sits in stage (n + 2) % ns, which with
+                    // two stages is tile n's own: then it has to wait for value(n) below.
+                    auto next_recon = [&]() {
+                        return mbar_wait(&bars->kfree[grp], (n >> 1) & 1, deadline) &&
+                               recon(n + 2, hb, (int)(f0 + n + 2 - hbase) >= tiles_c);
+                    };
+                    if (ns >= 3 && n + 2 < s1 && !next_recon()) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(&bars->p_ready[grp], (n >> 1) & 1, deadline)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (!win) {
+                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
+                        for (int ks = 0; ks < kTile / 16; ++ks)
+                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
+                                       desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
+                    } else {
+                        // O = V^T P over 64 exact rows: A = V tile, MN-major, M = d
+                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + kWinBytes);
+                        for (int ks = 0; ks < kWinTile / 16; ++ks)
+                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
+                                       desc_noswizzle(p0 + ks * 512, 256, 128), idesc_ow, ks != 0);
+                    }
+                    mma_commit(&bars->o_full[grp]);
+                    mma_commit(&bars->empty[st]);
+                    if (ns < 3 && n + 2 < s1 && !next_recon()) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&bars->bk_empty[2 * hb + grp]);   // this group is done with the basis
+                n0 = s1;
+            }
+            if (!ok) fail();
+            if (*abort_flag) {                        // let issued MMAs finish (bounded)
+                mma_commit(&bars->drain[1 + grp]);
+                mbar_wait(&bars->drain[1 + grp], 0, deadline + kWaitCycles);
+            }
         }
     }
 
@@ -728,14 +768,14 @@ decode_tc_kernel(DecodeTcArgs a) {
 
 }  // namespace
 
-size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk) {
+size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb) {
     // + queries of the head (g x d fp32)
-    return plan_smem(rK, rV, ns, nbk).total + (size_t)kMaxGroup * kHeadDim * 4;
+    return plan_smem(rK, rV, ns, nbk, nqb).total + (size_t)kMaxGroup * kHeadDim * 4;
 }
 
 template <int G>
 cudaError_t launch_g(const DecodeTcArgs& a, cudaStream_t s) {
-    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages, a.basis_bufs);
+    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages, a.basis_bufs, a.q_bufs);
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;
