@@ -49,6 +49,14 @@ D = 128
 BLOCK = 64
 
 
+# DRAM bytes (read + write) of one decode-attention launch at the per-layer
+# shape of the 32K-context, batch-8 workloads (8 KV / 32 query heads, r_K 32,
+# r_V 64), from the ncu launch list in profiles/launches_qwen3-1L-b8-32k.md
+# (the 36-layer run issues the same launch once per layer).  None for
+# workloads without a capture.
+DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.7e6, "qwen3-1L-b8-32k": 433.7e6}
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -359,7 +367,9 @@ def run_iskv(args, rank, world, local_rank):
     d2h = BLOCK * L * Bsz * Hq * D * 4
     status = cache.status()
 
-    launches_per_period = BLOCK * L * (2 + 2) + 6
+    # per decode step and layer: append (K, V) + decode attention; per period:
+    # fold (K, V) + coefficient rewrite (K, V)
+    launches_per_period = BLOCK * L * 3 + 4
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
@@ -380,8 +390,11 @@ def run_iskv(args, rank, world, local_rank):
         "decode_attention_us_avg": dec_avg_us,
         "prefill_s": prefill_s,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "kernel": "decode attention (split-K decode + combine), per layer call",
+                     "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.workload)
+                     if coef == ik.BF16 else None,
+                     "kernel": "decode_tc_kernel (persistent split-K decode attention, "
+                               "per-head combine fused), one launch per layer call",
+                     "algorithmic_bytes_per_launch": bsum / max(1, len(dec_events)),
                      "peak_source": peak_src},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
