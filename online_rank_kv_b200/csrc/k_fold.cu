@@ -4,8 +4,8 @@
 // Method: Brand's block-incremental SVD as the iS-KV explainer applies it
 // ("iS-KV -- Basis-synchronized online low-rank KV compression -- What does it
 // mean?", Jargon: Block-incremental SVD; body paragraph on the joint update of
-// basis and coefficients on a small core whose size does not depend on the
-// history length).  Steps inside the CTA, fp32, every intermediate in shared
+// basis and coefficients, decomposed on a fixed-size core matrix independent
+// of the history's row count).  Steps inside the CTA, fp32, every intermediate in shared
 // memory or registers:
 //   (a) P = X B.
 //   (b) Householder QR of [B | X^T] (d x (r+64)).  Its first r reflections

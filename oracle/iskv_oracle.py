@@ -96,8 +96,8 @@ def ready_blocks(T: int, n_c: int, W: int, b: int = 64) -> int:
     """Number of whole b-row blocks that have left the exact window.
 
     The newest W tokens stay exact; the rows [n_c, T - W) are old enough to be
-    folded, in whole blocks of b (the explainer's body: every time 64 tokens
-    leave the recent window they are folded in as one block).  Pinned by brute
+    folded, in whole blocks of b (the explainer's body: the compressed history
+    grows by one 64-row block at a time, as blocks age out of the window).  Pinned by brute
     force over all small (T, n_c, W) in the tests.
     """
     if T < 0 or n_c < 0 or W < 0 or b <= 0 or n_c > T:
@@ -159,8 +159,8 @@ def fold_block(B, S, X) -> FoldResult:
 
     Brand's block-incremental SVD as the iS-KV explainer applies it (Jargon:
     Block-incremental SVD; body paragraph on the joint update of basis and
-    coefficients, solved on a small core whose size does not depend on the
-    history length):
+    coefficients, whose decomposition works on a fixed-size core matrix,
+    independent of how many rows the history holds):
       (a) P = X B
       (b) E = X - P B^T (re-orthogonalized once more), Q and R_E from rule Q
       (c) core = [[diag S, 0], [P, R_E^T]], SVD core = U Sigma W^T, keep r
