@@ -235,19 +235,42 @@ class HeadFactor:
         self.sync_enabled = sync
         self.B = np.eye(d)[:, :r].copy()
         self.S = np.zeros(r)
-        self.C = np.zeros((0, r))
-        self.rows = np.zeros((0, d))
+        # row storage grows by doubling (appending block by block to plain
+        # arrays would copy the whole history every time)
+        self._Cbuf = np.zeros((0, r))
+        self._rowbuf = np.zeros((0, d))
+        self._nrows = 0
         self.n_c = 0
         self.pending = []           # [(rows_before_fold, W_top)]
         self.history = []           # FoldResult per fold (for drift studies)
 
     @property
     def T(self) -> int:
-        return self.rows.shape[0]
+        return self._nrows
+
+    @property
+    def rows(self) -> np.ndarray:
+        """All appended rows (T x d), oldest first."""
+        return self._rowbuf[:self._nrows]
+
+    @property
+    def C(self) -> np.ndarray:
+        """Stored coefficient rows (n_c x r)."""
+        return self._Cbuf[:self.n_c]
+
+    @staticmethod
+    def _grown(buf: np.ndarray, need: int) -> np.ndarray:
+        if need <= buf.shape[0]:
+            return buf
+        out = np.zeros((max(need, 2 * buf.shape[0], 256), buf.shape[1]))
+        out[:buf.shape[0]] = buf
+        return out
 
     def append(self, rows) -> int:
         rows = np.asarray(rows, dtype=np.float64).reshape(-1, self.d)
-        self.rows = np.concatenate([self.rows, rows], axis=0)
+        self._rowbuf = self._grown(self._rowbuf, self._nrows + rows.shape[0])
+        self._rowbuf[self._nrows:self._nrows + rows.shape[0]] = rows
+        self._nrows += rows.shape[0]
         return self.ready()
 
     def ready(self) -> int:
@@ -264,7 +287,8 @@ class HeadFactor:
                 self.pending.append((self.n_c, res.W_top))
             else:
                 self.C[:self.n_c] = _store(self.C[:self.n_c] @ res.W_top, self.coef_round)
-        self.C = np.concatenate([self.C, _store(res.C_new, self.coef_round)], axis=0)
+        self._Cbuf = self._grown(self._Cbuf, self.n_c + self.b)
+        self._Cbuf[self.n_c:self.n_c + self.b] = _store(res.C_new, self.coef_round)
         self.B, self.S = res.B_new, res.S_new
         self.n_c += self.b
         if keep_history:
@@ -272,16 +296,29 @@ class HeadFactor:
         return res
 
     def sync(self) -> None:
-        """Apply postponed rewrites in fold order, then round once."""
+        """Apply postponed rewrites, then round once.
+
+        A row stored before postponed fold i (of k) is rewritten by
+        W_top(i) W_top(i+1) ... W_top(k), the folds that came after it, in
+        order; rows between the row counts of folds i-1 and i take the suffix
+        product starting at fold i.  The same matrices as rewriting after each
+        fold, grouped so that every row is multiplied once."""
         if not self.pending:
             return
-        C = self.C.copy()
-        touched = 0
-        for n_rows, W_top in self.pending:
-            C[:n_rows] = C[:n_rows] @ W_top
-            touched = max(touched, n_rows)
-        C[:touched] = _store(C[:touched], self.coef_round)
-        self.C = C
+        C = self.C                      # rewritten in place
+        k = len(self.pending)
+        suffix = [None] * k
+        acc = None
+        for i in range(k - 1, -1, -1):
+            W_top = self.pending[i][1]
+            acc = W_top if acc is None else W_top @ acc
+            suffix[i] = acc
+        lo = 0
+        for i, (n_rows, _) in enumerate(self.pending):
+            if n_rows > lo:
+                C[lo:n_rows] = C[lo:n_rows] @ suffix[i]
+                lo = n_rows
+        C[:lo] = _store(C[:lo], self.coef_round)
         self.pending = []
 
     def reconstruct(self) -> np.ndarray:

@@ -1,0 +1,242 @@
+"""The benchmark configurations at their full sizes, checked on sampled heads.
+
+All K/V are drawn on the GPU (the same seeded generator as the bench); the
+rows of the sampled (layer, sequence, KV head) instances are copied back and
+fed to the float64 oracle, which emulates the bf16 coefficient storage and the
+same postponed rewrites.  Tolerance 2e-2 (bf16-stored coefficients), counters
+exact.
+
+  * the 36-layer, batch-8, 32K-context Qwen3-8B-shaped cache (the bench
+    workload): sampled heads (seq 0, layers {0, 35}, KV heads {0, 7});
+  * the long chain-of-thought growth run: batch 1, 36 layers, r_K 64, r_V 96,
+    W 2048, subspace drift every 2K tokens, grown to 128K tokens, with
+    queries aimed at tokens older than 8K (recall of compressed history);
+  * the one-layer sweep: ranks {16, 32, 64, 128} at 4K and 16K contexts and
+    batch {1, 8}, its largest point (r 128, 256K context, batch 32), and the
+    no-synchronization ablation's reconstruction drift against the
+    synchronized path.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from iskv_testlib import rel_err
+from oracle import HeadFactor, dense_decode
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _one_blas_thread():
+    # the oracle's many small QR/SVD calls run faster on one BLAS thread
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        yield
+
+
+class SampledCache:
+    """A CUDA cache for every head plus oracle factors for a few of them."""
+
+    def __init__(self, cfg, workload, sample, seed, sync=True):
+        import online_rank_kv_b200 as ik
+        self.ik = ik
+        self.cfg = cfg
+        self.cache = ik.Cache(cfg)
+        self.L, self.B, self.H = cfg.layers, cfg.batch, cfg.kv_heads
+        self.g = cfg.q_heads // cfg.kv_heads
+        nh = self.L * self.B * self.H
+        self.ks = synth.KVStream(synth.spec_for(workload, "K"), nh, seed=2 * seed + 1, device="cuda",
+                                 dtype=torch.bfloat16)
+        self.vs = synth.KVStream(synth.spec_for(workload, "V"), nh, seed=2 * seed + 2, device="cuda",
+                                 dtype=torch.bfloat16)
+        self.sample = list(sample)
+        self.ok = {x: HeadFactor(128, cfg.rank_k, cfg.window, coef_round="bf16", sync=sync)
+                   for x in self.sample}
+        self.ov = {x: HeadFactor(128, cfg.rank_v, cfg.window, coef_round="bf16", sync=sync)
+                   for x in self.sample}
+        self.folds = 0
+        self.qseed = 5000 + seed
+
+    def append(self, t):
+        k = self.ks.next(t).view(self.L, self.B, self.H, t, 128)
+        v = self.vs.next(t).view(self.L, self.B, self.H, t, 128)
+        for l in range(self.L):
+            self.cache.append(l, k[l].contiguous(), v[l].contiguous())
+        for (l, b, h) in self.sample:
+            self.ok[(l, b, h)].append(k[l, b, h].double().cpu().numpy())
+            self.ov[(l, b, h)].append(v[l, b, h].double().cpu().numpy())
+
+    def fold_all(self, defer):
+        self.cache.compress_block(self.ik.ALL_LAYERS, defer=defer)
+        for x in self.sample:
+            self.ok[x].fold(defer=defer)
+            self.ov[x].fold(defer=defer)
+
+    def sync_all(self):
+        self.cache.sync(self.ik.ALL_LAYERS)
+        for x in self.sample:
+            self.ok[x].sync()
+            self.ov[x].sync()
+
+    def ready(self):
+        T, n_c = self.cache.counts(0)
+        return (T - n_c - self.cfg.window) // 64
+
+    def prefill(self, tokens, chunk=512, defer_every=64):
+        """Append in chunks; fold every ready block with postponed rewrites,
+        one rewrite per defer_every folds, as the bench prefills."""
+        done = 0
+        while done < tokens:
+            n = min(chunk, tokens - done)
+            self.append(n)
+            done += n
+            while self.ready() >= 1:
+                self.fold_all(defer=defer_every > 0)
+                self.folds += 1
+                if defer_every > 0 and self.folds % defer_every == 0:
+                    self.sync_all()
+        if defer_every > 0:
+            self.sync_all()
+
+    def check(self):
+        ik = self.ik
+        for l in sorted({x[0] for x in self.sample}):
+            T, n_c = self.cache.counts(l)
+            for x in self.sample:
+                if x[0] == l:
+                    assert (T, n_c) == (self.ok[x].T, self.ok[x].n_c)
+            for which, of in ((ik.WHICH_K, self.ok), (ik.WHICH_V, self.ov)):
+                got = self.cache.reconstruct(l, which)
+                for x in self.sample:
+                    if x[0] == l and of[x].n_c > 0:
+                        e = rel_err(got[x[1], x[2]].cpu().numpy(), of[x].reconstruct())
+                        assert e < TOL, (l, which, x, e)
+                del got
+
+    def decode_check(self, q=None):
+        """Decode every sampled layer with q (B x Hq x d); compare the sampled
+        heads' outputs with dense attention over the oracle's cache."""
+        c = self.cfg
+        if q is None:
+            q = synth.query_batch(c.batch * c.q_heads, 128, seed=self.qseed,
+                                  dtype=torch.bfloat16).view(c.batch, c.q_heads, 128)
+            self.qseed += 1
+        worst = 0.0
+        for l in sorted({x[0] for x in self.sample}):
+            out = self.cache.decode_attention(l, q.cuda()).cpu().numpy()
+            qn = q.double().numpy()
+            for x in self.sample:
+                if x[0] != l:
+                    continue
+                b, h = x[1], x[2]
+                want = dense_decode(qn[b, h * self.g:(h + 1) * self.g], self.ok[x].full(),
+                                    self.ov[x].full(), c.rope_theta, use_rope=True)
+                e = rel_err(out[b, h * self.g:(h + 1) * self.g], want)
+                worst = max(worst, e)
+        assert worst < TOL, worst
+        return worst
+
+
+def _cfg(**kw):
+    import online_rank_kv_b200 as ik
+    c = ik.Config(kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1, rope_theta=1e6,
+                  max_deferred=64, ring_extra=512)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_qwen3_36_layers_batch8_32k_sampled_heads():
+    cfg = _cfg(batch=8, layers=36, kv_heads=8, q_heads=32, rank_k=32, rank_v=64, window=1024,
+               max_tokens=32768 + 1024)
+    s = SampledCache(cfg, "qwen3", [(0, 0, 0), (0, 0, 7), (35, 0, 0), (35, 0, 7)], seed=70)
+    s.prefill(32768)
+    s.check()
+    s.decode_check()
+    # decode steps, then one block fold with an immediate rewrite (the bench's step)
+    for _ in range(3):
+        s.append(1)
+        s.decode_check()
+    while s.ready() < 1:
+        s.append(16)
+    s.fold_all(defer=False)
+    s.check()
+    s.decode_check()
+    assert s.cache.status() == 0
+
+
+def test_long_cot_growth_to_128k_with_recall():
+    cfg = _cfg(batch=1, layers=36, kv_heads=8, q_heads=32, rank_k=64, rank_v=96, window=2048,
+               max_tokens=131072 + 1024)
+    sample = [(0, 0, 0), (35, 0, 7)]
+    s = SampledCache(cfg, "cot", sample, seed=71)
+    s.prefill(8192)
+    s.check()
+    s.decode_check()
+    s.prefill(131072 - 8192)
+    T, n_c = s.cache.counts(0)
+    assert T == 131072 and n_c == ((T - 2048) // 64) * 64
+    s.check()
+    s.decode_check()
+    # queries whose top attention mass sits on a folded token older than 8K
+    g = cfg.q_heads // cfg.kv_heads
+    rng = np.random.default_rng(3)
+    q = synth.query_batch(cfg.q_heads, 128, seed=77, dtype=torch.float64).view(1, cfg.q_heads, 128)
+    for (l, b, h) in sample:
+        rec = s.ok[(l, b, h)].reconstruct()
+        for j in range(g):
+            pos = int(rng.integers(0, T - 8192 - 2048))
+            kp = torch.from_numpy(rec[pos])
+            beta = 25.0 * np.sqrt(128) / float(torch.linalg.vector_norm(kp))
+            q[b, h * g + j] = synth.recall_query(kp, pos, cfg.rope_theta, beta)
+    s.decode_check(q.to(torch.bfloat16))
+    assert s.cache.status() == 0
+
+
+@pytest.mark.parametrize("r", [16, 32, 64, 128])
+@pytest.mark.parametrize("T,B", [(4096, 1), (16384, 8)])
+def test_sweep_point(r, T, B):
+    cfg = _cfg(batch=B, layers=1, kv_heads=8, q_heads=32, rank_k=r, rank_v=r, window=1024,
+               max_tokens=T + 1024)
+    s = SampledCache(cfg, "qwen3", [(0, 0, 0), (0, B - 1, 7)], seed=80 + r)
+    s.prefill(T)
+    s.check()
+    s.decode_check()
+    assert s.cache.status() == 0
+
+
+def test_sweep_largest_point_r128_256k_batch32():
+    cfg = _cfg(batch=32, layers=1, kv_heads=8, q_heads=32, rank_k=128, rank_v=128, window=1024,
+               max_tokens=262144 + 1024)
+    s = SampledCache(cfg, "qwen3", [(0, 31, 5)], seed=90)
+    s.prefill(262144, chunk=512)
+    s.check()
+    s.decode_check()
+    assert s.cache.status() == 0
+
+
+def test_sweep_no_sync_drift():
+    """Reconstruction drift ||C B^T - K||_F / ||K||_F over the folded rows
+    (pre-RoPE keys), synchronized against the ablation that leaves old
+    coefficients in their old basis; the device caches and the oracle agree
+    on the synchronized value."""
+    import online_rank_kv_b200 as ik
+    drift = {}
+    for sync in (1, 0):
+        cfg = _cfg(batch=1, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64, window=1024,
+                   max_tokens=16384 + 1024, sync=sync)
+        s = SampledCache(cfg, "qwen3", [(0, 0, 3)], seed=95, sync=bool(sync))
+        s.prefill(16384)
+        T, n_c = s.cache.counts(0)
+        rec = s.cache.reconstruct(0, ik.WHICH_K)[0, 3].cpu().double().numpy()
+        K = s.ok[(0, 0, 3)].rows[:n_c]
+        drift[sync] = float(np.linalg.norm(rec - K) / np.linalg.norm(K))
+        if sync:
+            want = s.ok[(0, 0, 3)].reconstruct()
+            want_drift = float(np.linalg.norm(want - K) / np.linalg.norm(K))
+            assert abs(drift[1] - want_drift) < 0.1 * want_drift + 1e-4
+    assert drift[0] > 5 * drift[1], drift
