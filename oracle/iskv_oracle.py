@@ -258,6 +258,16 @@ class HeadFactor:
         """Stored coefficient rows (n_c x r)."""
         return self._Cbuf[:self.n_c]
 
+    @C.setter
+    def C(self, value) -> None:
+        # replaces the stored rows; n_c has to be set to match by the caller
+        self._Cbuf = np.array(value, dtype=np.float64).reshape(-1, self.r)
+
+    @rows.setter
+    def rows(self, value) -> None:
+        self._rowbuf = np.array(value, dtype=np.float64).reshape(-1, self.d)
+        self._nrows = self._rowbuf.shape[0]
+
     @staticmethod
     def _grown(buf: np.ndarray, need: int) -> np.ndarray:
         if need <= buf.shape[0]:
