@@ -128,6 +128,7 @@ decode_tc_kernel(DecodeTcArgs a) {
     const int tph = a.tiles_per_head;
     const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs, nqb = a.q_bufs;
     constexpr int g = G;
+    constexpr int kQItems = (G * 64 + 127) / 128;   // q' items per epilogue thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int d = kHeadDim;
 
@@ -259,6 +260,7 @@ decode_tc_kernel(DecodeTcArgs a) {
     } else if (warp >= 2 && warp < 10) {
         // ---------------- epilogue: two groups of 4 warps, alternate tiles ----------------
         const int ept = tid - 64;                 // 0..255
+        const int nc32 = (int)a.n_c, T32 = (int)a.T;
         const int grp = ept >> 7;                 // tiles n with n % 2 == grp
         const int gt = ept & 127;                 // thread within the group
         const int sp = warp & 3;                  // TMEM sub-partition of this warp
@@ -291,6 +293,17 @@ decode_tc_kernel(DecodeTcArgs a) {
         const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
         uint32_t* qbb = qb + nqb * grp * kQN * kTile;   // the group's first q' buffer (head-end exchange)
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
+        // q' operand offsets of this thread's items (hi of dims i, i + 64; lo likewise)
+        int qoff[kQItems][4];
+#pragma unroll
+        for (int k = 0; k < kQItems; ++k) {
+            const int item = gt + 128 * k;
+            const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
+            qoff[k][0] = qb_off(h, i);
+            qoff[k][1] = qb_off(h, i + 64);
+            qoff[k][2] = qb_off(G + h, i);
+            qoff[k][3] = qb_off(G + h, i + 64);
+        }
 
         float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
         // acc <- acc * alpha + (p^T C_V of a folded tile); accd likewise for exact tiles
@@ -334,30 +347,40 @@ decode_tc_kernel(DecodeTcArgs a) {
             int last = -1;
             // first position of a tile (folded tiles of 128 rows, then exact tiles of 64)
             const int64_t hbase = (int64_t)head * tph;   // flattened index of the head's tile 0
-            auto tile_j0 = [&](int nn) {
+            auto tile_j0 = [&](int nn) {   // positions fit in 32 bits (max_tokens is an int32)
                 const int lc = (int)(f0 + nn - hbase);
-                return lc >= tiles_c ? a.n_c + (int64_t)(lc - tiles_c) * kWinTile : (int64_t)lc * kTile;
+                return lc >= tiles_c ? nc32 + (lc - tiles_c) * kWinTile : lc * kTile;
             };
             // q' = R_{j0}^T q of tile nn as tf32 hi / lo parts (the score MMA's B
             // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
             // for i = gt & 63, the only frequency this thread rotates by
+            // this thread's items (head h, frequency i): item gt + 128 k; their
+            // query pair (q_i, q_{i+64}) stays in registers for the whole head
+            float qx1[kQItems], qx2[kQItems];
+#pragma unroll
+            for (int k = 0; k < kQItems; ++k) {
+                const int item = gt + 128 * k;
+                const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
+                qx1[k] = sq[h * d + i];
+                qx2[k] = sq[h * d + i + 64];
+            }
             auto build_q = [&](int nn, float2 rv) {
                 uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQN * kTile;
-                for (int item = gt; item < g * 64; item += 128) {
-                    const int h = item >> 6, i = item & 63;
-                    const float x1 = sq[h * d + i], x2 = sq[h * d + i + 64];
-                    const float y1 = fmaf(rv.x, x1, rv.y * x2);
-                    const float y2 = fmaf(rv.x, x2, -rv.y * x1);
+#pragma unroll
+                for (int k = 0; k < kQItems; ++k) {
+                    if (gt + 128 * k >= G * 64) break;
+                    const float y1 = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
+                    const float y2 = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
                     const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
-                    qd[qb_off(h, i)] = t1;
-                    qd[qb_off(h, i + 64)] = t2;
-                    qd[qb_off(g + h, i)] = to_tf32(y1 - __uint_as_float(t1));
-                    qd[qb_off(g + h, i + 64)] = to_tf32(y2 - __uint_as_float(t2));
+                    qd[qoff[k][0]] = t1;
+                    qd[qoff[k][1]] = t2;
+                    qd[qoff[k][2]] = to_tf32(y1 - __uint_as_float(t1));
+                    qd[qoff[k][3]] = to_tf32(y2 - __uint_as_float(t2));
                 }
                 fence_async_smem();
             };
             auto rope_of = [&](int nn) {
-                return a.rope ? a.rope[tile_j0(nn) * 64 + (gt & 63)] : make_float2(1.f, 0.f);
+                return a.rope ? a.rope[(int64_t)tile_j0(nn) * 64 + (gt & 63)] : make_float2(1.f, 0.f);
             };
             const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
             // two q' buffers: tile n + 2's q' is built while tile n's scores run;
@@ -367,10 +390,10 @@ decode_tc_kernel(DecodeTcArgs a) {
                 const int st = n % ns;
                 const int local = (int)(f0 + n - hbase);
                 const bool win = local >= tiles_c;    // exact rows (64-token tile)
-                const int64_t j0 = tile_j0(n);
-                const int64_t lim = win ? a.T : a.n_c;
+                const int j0 = tile_j0(n);
+                const int lim = win ? T32 : nc32;
                 const int span = win ? kWinTile : kTile;
-                const int valid = (int)((lim - j0) < span ? (lim - j0) : span);
+                const int valid = (lim - j0) < span ? (lim - j0) : span;
                 // the next tile's query rotation, loaded now, used after this tile's RoPE
                 const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
                 if (nqb == 1) build_q(n, rope_of(n));
