@@ -61,7 +61,7 @@ struct __align__(8) Bars {
     uint64_t full[4], empty[4];
     uint64_t bk_full[2], bk_empty[4];      // bk_empty[buffer * 2 + group]
     uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
-    uint64_t krot_ready[2], p_ready[2];   // epilogue -> group issuer: K_rot and q', P written
+    uint64_t krot_ready[2], krot_b[2], p_ready[2];   // epilogue -> group issuer: K_rot halves, P written
     uint64_t drain[3];   // abort path: completion of each issuer's outstanding MMAs
 };
 
@@ -171,6 +171,7 @@ decode_tc_kernel(DecodeTcArgs a) {
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->o_full[i], 1);
             mbar_init(&bars->krot_ready[i], kEpi / 2);
+            mbar_init(&bars->krot_b[i], kEpi / 2);
             mbar_init(&bars->p_ready[i], 1);
         }
         for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
@@ -450,10 +451,16 @@ decode_tc_kernel(DecodeTcArgs a) {
                     }
                     tmem_st16(kh + lane_base + c0, x1);
                     tmem_st16(kh + lane_base + 64 + c0, x2);
+                    if (c0 == 16 || c0 == 48) {
+                        // dims 0..31 and 64..95 of this row are rotated (first barrier),
+                        // then the rest (second): the score MMA starts on the first half
+                        // while the second is rotated.  One barrier per half, so every
+                        // phase counts each thread exactly once.
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(c0 == 16 ? &bars->krot_ready[grp] : &bars->krot_b[grp]);
+                    }
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bars->krot_ready[grp]);  // this row of K_rot and its q' share are in place
                 // the next tile's q' goes to the other buffer while this tile's scores run
                 if (nqb == 2 && n + 2 < s1) build_q(n + 2, rq_next);
                 // this group's previous tile: p^T C_V accumulated (before O is reused)
@@ -725,15 +732,28 @@ decode_tc_kernel(DecodeTcArgs a) {
                 for (int n = n_first; ok && n < s1; n += 2) {
                     const int st = n % ns;
                     const bool win = (int)(f0 + n - hbase) >= tiles_c;
-                    if (!mbar_wait(&bars->krot_ready[grp], (n >> 1) & 1, deadline)) {
+                    // scores in two halves of the head dimension, each once the epilogue
+                    // has rotated it: dims 0..31 and 64..95 (k-steps 0..3, 8..11), then
+                    // 32..63 and 96..127 (k-steps 4..7, 12..15)
+                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQN * kTile * 4);
+                    bool got = true;
+                    for (int half = 0; half < 2; ++half) {
+                        if (!mbar_wait(half ? &bars->krot_b[grp] : &bars->krot_ready[grp], (n >> 1) & 1,
+                                       deadline)) {
+                            got = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        for (int j = 0; j < 8; ++j) {
+                            const int ks = (j < 4 ? j : j + 4) + 4 * half;
+                            mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
+                                        idesc_s, (half | j) != 0);
+                        }
+                    }
+                    if (!got) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQN * kTile * 4);
-                    for (int ks = 0; ks < d / 8; ++ks)
-                        mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
-                                    idesc_s, ks != 0);
                     mma_commit(&bars->s_full[grp]);
                     mma_commit(&bars->kfree[grp]);
                     // K_rot of tile n consumed: rebuild tile n + 2 while the epilogue runs
