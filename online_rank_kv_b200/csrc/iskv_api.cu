@@ -430,6 +430,49 @@ int iskv_sync(iskv_t h, int layer, void* stream) {
     return run_resync(h, rl_layers, rl_seg, rl_rows, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Tile ranges of the persistent decode grid: contiguous runs of the flattened
+// (head, tile) space, at most nmax of them, of equal cost, where a run costs
+// its tiles plus kHeadSwitchTiles for every head it enters after its first
+// (publishing a partial, and restarting the pipeline on the next head's basis
+// and queries).  Smallest feasible cost by bisection, runs filled greedily.
+// Returns the number of runs; start[0..n] holds their bounds.
+static constexpr int64_t kHeadSwitchTiles = 4;
+
+static int fill_decode_runs(int64_t total, int64_t tph, int nmax, int64_t cost, int64_t* start) {
+    int k = 0;
+    int64_t p = 0;
+    while (p < total) {
+        if (k == nmax) return nmax + 1;
+        start[k++] = p;
+        int64_t budget = cost, q = p;
+        for (bool first = true; q < total; first = false) {
+            if (!first) {
+                budget -= kHeadSwitchTiles;
+                if (budget < 1) break;
+            }
+            const int64_t seg_end = std::min((q / tph + 1) * tph, total);
+            const int64_t take = std::min(seg_end - q, budget);
+            q += take;
+            budget -= take;
+            if (q < seg_end) break;
+        }
+        p = q > p ? q : p + 1;
+    }
+    start[k] = total;
+    return k;
+}
+
+static int partition_decode_tiles(int64_t total, int64_t tph, int nmax, int64_t* start) {
+    // hi: one run holds everything
+    int64_t lo = 1, hi = total + kHeadSwitchTiles * ((total + tph - 1) / tph);
+    while (lo < hi) {
+        const int64_t mid = lo + (hi - lo) / 2;
+        if (fill_decode_runs(total, tph, nmax, mid, start) <= nmax) hi = mid;
+        else lo = mid + 1;
+    }
+    return fill_decode_runs(total, tph, nmax, lo, start);
+}
+
 int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* stream) {
     if (!h || !q || !out || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
     if (h->T[layer] == 0 || h->n_pend[layer] > 0) return ISKV_ERR_STATE;
@@ -438,7 +481,9 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     const size_t q_bytes = (size_t)c.batch * c.q_heads * kHeadDim * h->kv_bytes;
     const size_t o_bytes = (size_t)c.batch * c.q_heads * kHeadDim * sizeof(float);
     const void* qd = q;
-    if (!is_device_ptr(q)) {
+    // host queries, or device queries off the 16-byte alignment of the bulk
+    // copies that fetch them, go through the staging buffer
+    if (!is_device_ptr(q) || (reinterpret_cast<uintptr_t>(q) & 15) != 0) {
         if (q_bytes > h->stage_in_bytes) return ISKV_ERR_UNSUPPORTED;
         CU(cudaMemcpyAsync(h->stage_in, q, q_bytes, cudaMemcpyDefault, s));
         qd = h->stage_in;
@@ -487,18 +532,31 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.tiles_c = (int)((a.n_c + 127) / 128);
         t.tiles_per_head = t.tiles_c + (int)((a.T - a.n_c + 63) / 64);
         t.total_tiles = (int64_t)h->BH * t.tiles_per_head;
-        int64_t ncta = std::min<int64_t>(sms, t.total_tiles);
-        t.tiles_per_cta = (int)((t.total_tiles + ncta - 1) / ncta);
-        t.ncta = (int)((t.total_tiles + t.tiles_per_cta - 1) / t.tiles_per_cta);
-        int slots_c = 1;
-        for (int hh = 0; hh < h->BH; ++hh) {
-            const int64_t first = ((int64_t)hh * t.tiles_per_head) / t.tiles_per_cta;
-            const int64_t last = ((int64_t)(hh + 1) * t.tiles_per_head - 1) / t.tiles_per_cta;
-            slots_c = std::max<int>(slots_c, (int)(last - first + 1));
+        // each CTA publishes two partials (one per epilogue group) for every head
+        // it visits; fewer CTAs when a head would span more slots than the
+        // partial buffer holds (few heads, long context)
+        int ncta = (int)std::min<int64_t>(std::min(sms, kDecodeMaxCtas), t.total_tiles);
+        // partial slots per query head: the buffer's, and the merge scratch's
+        // (slots x g <= 1024)
+        const int cap_slots = std::min(h->max_splits, 1024 / a.g);
+        int slots_c = 0;
+        for (;;) {
+            t.ncta = partition_decode_tiles(t.total_tiles, t.tiles_per_head, ncta, t.cta_start);
+            slots_c = 1;
+            int c0 = 0;
+            for (int hh = 0; hh < h->BH; ++hh) {
+                const int64_t f_first = (int64_t)hh * t.tiles_per_head, f_last = f_first + t.tiles_per_head - 1;
+                while (t.cta_start[c0 + 1] <= f_first) ++c0;
+                int c1 = c0;
+                while (t.cta_start[c1 + 1] <= f_last) ++c1;
+                slots_c = std::max(slots_c, c1 - c0 + 1);
+            }
+            if (2 * slots_c <= cap_slots || ncta == 1) break;
+            ncta = std::max(1, ncta * (cap_slots - 2) / (2 * slots_c));
         }
-        if (slots_c > h->max_splits) return ISKV_ERR_UNSUPPORTED;
+        if (2 * slots_c > cap_slots) return ISKV_ERR_UNSUPPORTED;
         t.slots_c = slots_c;
-        t.splits_total = slots_c;
+        t.splits_total = 2 * slots_c;
         // deepest pipeline that fits: stages first, then two basis buffers, then
         // double-buffered q'
         t.stages = 0;

@@ -112,6 +112,8 @@ struct DecodeArgs {
 };
 
 // Tensor-core decode over the folded rows (bf16 blocked coefficients).
+constexpr int kDecodeMaxCtas = 160;   // persistent decode grid: at most one CTA per SM
+
 struct DecodeTcArgs {
     FactorView K, V;
     const void* q;               // [B][Hq][d] bf16
@@ -125,8 +127,9 @@ struct DecodeTcArgs {
     int tiles_c;                 // folded-row tiles per head: ceil(n_c / 128)
     int tiles_per_head;          // tiles_c + exact-row tiles of 64: ceil((T - n_c) / 64)
     int64_t total_tiles;         // BH * tiles_per_head
-    int tiles_per_cta;
     int ncta;
+    // CTA i takes the flattened tiles [cta_start[i], cta_start[i + 1])
+    int64_t cta_start[kDecodeMaxCtas + 1];
     int slots_c;                 // compressed partial slots per query head
     int splits_total;
     int stages;                  // shared-memory pipeline depth (2..4)

@@ -10,30 +10,40 @@
 //   partial softmax (m, l) and acc_h = sum_j p_j C_V[j]   (r_V wide);
 // and, for the exact rows j >= n_c (64-token tiles of the window ring),
 //   s_j = q_h . RoPE(K_j, j) / sqrt(d) and acc_d = sum_j p_j V_j (d wide),
-// all under one online softmax per head; combine_kernel (k_decode.cu) merges
-// the per-CTA partials and applies B_V^T once per query head.
+// all under one online softmax per head.
 //
-// Persistent design, one CTA per SM, the flattened (head, 128-token tile)
-// space cut into equal contiguous ranges; per CTA 10 warps:
+// Persistent design, one CTA per SM; the flattened (head, tile) space is cut
+// into contiguous runs of equal cost (tiles, plus a fixed charge for every
+// head a run enters after its first), one run per CTA.  Per CTA 12 warps:
 //   warp 0  producer: 1-D bulk copies (TMA engine) of the C_K and C_V tiles
 //           or of the exact K and V rows (all contiguous in the blocked
-//           layout) into an NS-stage ring, and of the bf16 hi/lo basis of
-//           each head it visits;
-//   warp 1  MMA issuer: K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens,
-//           N=128 dims, fp32 accumulator in TMEM (two buffers);
+//           layout) into an NS-stage ring, and of the bf16 hi/lo basis and
+//           the bf16 queries of each head it visits;
+//   warp 1  TMEM allocation;
 //   warps 2-9 epilogue, two ping-pong groups of 4 warps (group = tile
 //           parity), one token row per thread:
 //           * rotate its row of K^ by R_t (t = row within the tile; the
 //             row's cos/sin(t w_i) sit in spare TMEM columns) and write it
-//             back to TMEM rounded to tf32; the query is pre-rotated per tile
-//             by R_{j0}^T (j0 = tile start), so q'.(R_t k) = q.(R_{j0+t} k);
-//           * scores S = K_rot q'^T on the tensor cores (kind::tf32, A from
-//             TMEM, q' as tf32 hi+lo parts in the N dimension);
-//           * online softmax per query head and group; at the end of each
-//             head the two groups' states are merged by log-sum-exp;
-//           * p as bf16 hi+lo parts -> O = C_V^T P (kind::f16, C_V tile read
-//             MN-major in place; for exact rows O = V^T P with M = d),
-//             accumulated with the running rescale.
+//             back to TMEM as fp16 pairs (dim i, dim 64 + i) per column; the
+//             query is pre-rotated per tile by R_{j0}^T (j0 = tile start), so
+//             q'.(R_t k) = q.(R_{j0+t} k);
+//           * online softmax per query head with a lazily updated maximum;
+//           * p as bf16 hi+lo parts for the value MMA;
+//           * at the end of a head the group publishes its own partial
+//             (m, l, r_V-wide and d-wide sums); the last group to publish
+//             a head's partial merges them all by log-sum-exp, applies
+//             B_V^T once per query head and writes the output.  The two
+//             groups never wait for each other.
+//   warps 10-11 MMA issuer of group 0 / 1:
+//           * K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens, N=128 dims,
+//             fp32 accumulator in TMEM, rebuilt two tiles ahead;
+//           * scores S = K_rot q'^T, kind::f16 with A from TMEM and q' as
+//             fp16 hi+lo parts in the N dimension, issued in two halves of
+//             the head dimension as the epilogue finishes rotating them;
+//           * O = C_V^T P (kind::f16, C_V tile read MN-major in place; for
+//             exact rows O = V^T P with M = d).
+// Rotated keys are held in fp16 (finite for |k| < 65504; the same 11-bit
+// significand as tf32); the query as fp16 hi + lo parts keeps ~22 bits.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // ISKV status bit 2, stops, drains its copies and frees its TMEM.
 #include "iskv_internal.cuh"
@@ -65,6 +75,12 @@ struct __align__(8) Bars {
     uint64_t drain[3];   // abort path: completion of each issuer's outstanding MMAs
 };
 
+// one basis buffer: B_hi, B_lo (bf16, 128 x r each), then the head's g <= 8
+// queries (bf16, g x d)
+__host__ __device__ inline uint32_t bk_stride(int rK) {
+    return (uint32_t)(2 * kTile * rK * 2 + kMaxGroup * kHeadDim * 2);
+}
+
 struct SmemPlan {
     uint32_t bk, stage, stage_k, stage_bytes, qb, pb, total;
 };
@@ -72,7 +88,7 @@ struct SmemPlan {
 __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, int nqb) {
     SmemPlan p;
     uint32_t off = 1024;                                        // barriers, scratch
-    p.bk = off;                off += nbk * (2 * kTile * rK * 2);  // nbk heads x (hi, lo)
+    p.bk = off;                off += nbk * bk_stride(rK);        // nbk heads x (hi, lo, queries)
     p.stage_k = (uint32_t)kTile * rK * 2;
     uint32_t sb = p.stage_k + kTile * rV * 2;
     if (sb < 2 * kWinTile * kHeadDim * 2) sb = 2 * kWinTile * kHeadDim * 2;   // exact K and V rows
@@ -106,9 +122,12 @@ __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
 // more than this (p <= e^8); otherwise the tile takes the exact rescale
 constexpr float kLazyMax = 8.f;
 
-// offsets of the tf32 (K-major, 8 x 4 core matrices) and bf16 (8 x 8) B operands
-__device__ __forceinline__ int qb_off(int n, int k) {
-    return ((n >> 3) * (kTile / 4) + (k >> 2)) * 32 + (n & 7) * 4 + (k & 3);
+// q' as the score MMA's B operand: fp16, K-major 8 x 8 core matrices over
+// K = 128 positions k, where k = 2u holds dim u and k = 2u + 1 dim 64 + u
+// (the order of the packed rotated keys in TMEM).  Word (32-bit) offset of
+// the pair (k = 2u, 2u + 1) of row n.
+__device__ __forceinline__ int qb_off(int n, int u) {
+    return ((n >> 3) * (kTile / 8) + (u >> 2)) * 32 + (n & 7) * 4 + (u & 3);
 }
 // p as the value MMA's B operand, MN-major: [token][16] in 8 x 8 blocks, so one
 // thread's (token's) 8 values of an n-block are one 16-byte row
@@ -116,13 +135,23 @@ __device__ __forceinline__ int pb_off(int n, int k) {
     return ((k >> 3) * (kPN / 8) + (n >> 3)) * 64 + (k & 7) * 8 + (n & 7);
 }
 
+// the CTA whose tile range holds flattened tile f
+__device__ __forceinline__ int cta_of(const DecodeTcArgs& a, int64_t f) {
+    int lo = 0, hi = a.ncta - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.cta_start[mid] <= f) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(DecodeTcArgs a) {
+decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     const int cta = blockIdx.x;
-    const int64_t f0 = (int64_t)cta * a.tiles_per_cta;
-    int64_t f1 = f0 + a.tiles_per_cta;
-    if (f1 > a.total_tiles) f1 = a.total_tiles;
+    const int64_t f0 = a.cta_start[cta];
+    const int64_t f1 = a.cta_start[cta + 1];
     if (f0 >= f1) return;
     const int ntiles = (int)(f1 - f0);
     const int tph = a.tiles_per_head;
@@ -138,13 +167,11 @@ decode_tc_kernel(DecodeTcArgs a) {
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 4);
     // the epilogue's copy of the flag, taken by one thread before a named
     // barrier so that all 256 epilogue threads leave the loop together
-    volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);
-    volatile int* flag_max = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2]
-    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 24);
+    volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);    // [2 groups]
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2 groups]
+    static_assert(sizeof(Bars) + 24 <= 512, "scratch words fit below the reduction area");
     float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
-    float* mlx = reinterpret_cast<float*>(smem + 256);          // [2 groups][m 8 | l 8]
     const SmemPlan P = plan_smem(rK, rV, ns, nbk, nqb);
-    float* sq = reinterpret_cast<float*>(smem + P.total);       // queries of the head, g x d fp32
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
     uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
@@ -152,7 +179,9 @@ decode_tc_kernel(DecodeTcArgs a) {
     const uint32_t stage_bytes = P.stage_bytes;
     const int tiles_c = a.tiles_c;
     constexpr uint32_t kWinBytes = kWinTile * kHeadDim * 2;   // one of K, V
-    const uint32_t bk_bytes = 2 * kTile * rK * 2;
+    const uint32_t bk_bytes = 2 * kTile * rK * 2;   // B_hi, B_lo of one head
+    const uint32_t bks = bk_stride(rK);
+    const uint32_t q_bytes = (uint32_t)g * d * 2;    // the head's queries, bf16
 
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -176,15 +205,13 @@ decode_tc_kernel(DecodeTcArgs a) {
         }
         for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
         *abort_flag = 0;
-        flag_max[0] = 0;
-        flag_max[1] = 0;
         fence_mbar_init();
     }
     // zero the padding rows (n >= 2g) of the q' and p operands once
-    for (int e = tid; e < 2 * nqb * kQN * kTile; e += kThreads) {
-        const int buf = e / (kQN * kTile), w = e % (kQN * kTile);
-        const int n = w / kTile, k = w % kTile;
-        if (n >= 2 * g) qb[buf * kQN * kTile + qb_off(n, k)] = 0u;
+    for (int e = tid; e < 2 * nqb * kQN * 64; e += kThreads) {
+        const int buf = e / (kQN * 64), w = e % (kQN * 64);
+        const int n = w / 64, u = w % 64;
+        if (n >= 2 * g) qb[buf * kQN * kTile + qb_off(n, u)] = 0u;
     }
     for (int e = tid; e < 2 * kPN * kTile; e += kThreads) {
         const int buf = e / (kPN * kTile), w = e % (kPN * kTile);
@@ -220,8 +247,12 @@ decode_tc_kernel(DecodeTcArgs a) {
                         fail();
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars->bk_full[hb], bk_bytes);
-                    bulk_g2s(bk + hb * bk_bytes, a.K.bsplit + hidx * 2 * d * rK, bk_bytes, &bars->bk_full[hb]);
+                    const int bq = head / a.Hkv, kvh = head % a.Hkv;
+                    const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.q) +
+                                              ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
+                    mbar_arrive_expect_tx(&bars->bk_full[hb], bk_bytes + q_bytes);
+                    bulk_g2s(bk + hb * bks, a.K.bsplit + hidx * 2 * d * rK, bk_bytes, &bars->bk_full[hb]);
+                    bulk_g2s(bk + hb * bks + bk_bytes, qg, q_bytes, &bars->bk_full[hb]);
                     prev = head;
                 }
                 const int st = n % ns;
@@ -268,25 +299,42 @@ decode_tc_kernel(DecodeTcArgs a) {
         const int row = sp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
         const uint32_t tcs = tmem + kCsCol;
-        // this row's in-tile RoPE table (cos, sin of row * w_i) into TMEM
-        if (grp == 0) {
+        // this row's in-tile RoPE table (cos, sin, -sin of row * w_i) into TMEM:
+        // group grp writes frequencies 32 grp .. 32 grp + 31, all loads issued first
+        {
+            float4 tv[16];
+            if (a.rope) {
+                const float4* src = reinterpret_cast<const float4*>(a.rope + row * 64 + grp * 32);
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
+                for (int u = 0; u < 16; ++u) tv[u] = src[u];
+            } else {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) tv[u] = make_float4(1.f, 0.f, 1.f, 0.f);
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
                 uint32_t vc[16], vs[16], vn[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    float2 v = make_float2(1.f, 0.f);
-                    if (a.rope) v = a.rope[row * 64 + c0 + u];
-                    vc[u] = __float_as_uint(v.x);
-                    vs[u] = __float_as_uint(v.y);
-                    vn[u] = __float_as_uint(-v.y);
+                for (int u = 0; u < 8; ++u) {
+                    const float4 v = tv[hh * 8 + u];
+                    vc[2 * u] = __float_as_uint(v.x);
+                    vs[2 * u] = __float_as_uint(v.y);
+                    vn[2 * u] = __float_as_uint(-v.y);
+                    vc[2 * u + 1] = __float_as_uint(v.z);
+                    vs[2 * u + 1] = __float_as_uint(v.w);
+                    vn[2 * u + 1] = __float_as_uint(-v.w);
                 }
+                const int c0 = grp * 32 + hh * 16;
                 tmem_st16(tcs + lane_base + c0, vc);
                 tmem_st16(tcs + lane_base + 64 + c0, vs);
                 tmem_st16(tcs + lane_base + 128 + c0, vn);
             }
             tmem_wait_st();
         }
+        // both halves of the table written before either group's first RoPE
+        tc_fence_before();
+        epi_sync();
+        tc_fence_after();
         const int MV = rV <= 64 ? 64 : 128;
         const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
@@ -295,15 +343,13 @@ decode_tc_kernel(DecodeTcArgs a) {
         uint32_t* qbb = qb + nqb * grp * kQN * kTile;   // the group's first q' buffer (head-end exchange)
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
         // q' operand offsets of this thread's items (hi of dims i, i + 64; lo likewise)
-        int qoff[kQItems][4];
+        int qoff[kQItems][2];
 #pragma unroll
         for (int k = 0; k < kQItems; ++k) {
             const int item = gt + 128 * k;
             const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
-            qoff[k][0] = qb_off(h, i);
-            qoff[k][1] = qb_off(h, i + 64);
-            qoff[k][2] = qb_off(G + h, i);
-            qoff[k][3] = qb_off(G + h, i + 64);
+            qoff[k][0] = qb_off(h, i);       // hi parts of dims i, 64 + i
+            qoff[k][1] = qb_off(G + h, i);   // lo parts
         }
 
         float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
@@ -318,18 +364,14 @@ decode_tc_kernel(DecodeTcArgs a) {
             }
         };
         bool stop = false;
-        int n0 = 0;
+        int n0 = 0, hs = -1;
+        // the two groups run through the heads independently: each keeps its own
+        // softmax state and publishes its own partial slot per head
         while (n0 < ntiles) {
             const int head = (int)((f0 + n0) / tph);
             int s1 = (int)(((int64_t)head + 1) * tph - f0);
             if (s1 > ntiles) s1 = ntiles;
-            // queries of the head, fresh softmax state; uniform abort check
-            {
-                const int bq = head / a.Hkv, kvh = head % a.Hkv;
-                const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                          ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
-                for (int e = ept; e < g * d; e += kEpi) sq[e] = __bfloat162float(qg[e]);
-            }
+            ++hs;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 m_run[h] = -INFINITY;
@@ -338,12 +380,17 @@ decode_tc_kernel(DecodeTcArgs a) {
                 accd[h] = 0.f;
                 alpha[h] = 0.f;
             }
-            if (ept == 0) *epi_abort = *abort_flag;
-            tc_fence_before();
-            epi_sync();
-            tc_fence_after();
-            stop = *epi_abort;                    // latched after the barrier: uniform
+            // group-uniform abort check
+            if (gt == 0) epi_abort[grp] = *abort_flag;
+            group_sync(grp);
+            stop = epi_abort[grp];                // latched after the barrier: uniform
             if (stop) break;
+            // this group's first tile of the head; none: only the empty partial
+            const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
+            // the head's queries arrived with its basis (the group's own tiles keep
+            // the buffer from being reused before this read)
+            const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(bk + (hs % nbk) * bks + bk_bytes);
+            if (n_first < s1 && !mbar_wait(&bars->bk_full[hs % nbk], (hs / nbk) & 1, deadline)) fail();
             bool have_prev = false, prev_win = false;
             int last = -1;
             // first position of a tile (folded tiles of 128 rows, then exact tiles of 64)
@@ -352,7 +399,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 const int lc = (int)(f0 + nn - hbase);
                 return lc >= tiles_c ? nc32 + (lc - tiles_c) * kWinTile : lc * kTile;
             };
-            // q' = R_{j0}^T q of tile nn as tf32 hi / lo parts (the score MMA's B
+            // q' = R_{j0}^T q of tile nn as fp16 hi / lo parts (the score MMA's B
             // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
             // for i = gt & 63, the only frequency this thread rotates by
             // this thread's items (head h, frequency i): item gt + 128 k; their
@@ -362,8 +409,8 @@ decode_tc_kernel(DecodeTcArgs a) {
             for (int k = 0; k < kQItems; ++k) {
                 const int item = gt + 128 * k;
                 const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
-                qx1[k] = sq[h * d + i];
-                qx2[k] = sq[h * d + i + 64];
+                qx1[k] = n_first < s1 ? __bfloat162float(sq[h * d + i]) : 0.f;
+                qx2[k] = n_first < s1 ? __bfloat162float(sq[h * d + i + 64]) : 0.f;
             }
             auto build_q = [&](int nn, float2 rv) {
                 uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQN * kTile;
@@ -372,18 +419,17 @@ decode_tc_kernel(DecodeTcArgs a) {
                     if (gt + 128 * k >= G * 64) break;
                     const float y1 = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
                     const float y2 = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
-                    const uint32_t t1 = to_tf32(y1), t2 = to_tf32(y2);
-                    qd[qoff[k][0]] = t1;
-                    qd[qoff[k][1]] = t2;
-                    qd[qoff[k][2]] = to_tf32(y1 - __uint_as_float(t1));
-                    qd[qoff[k][3]] = to_tf32(y2 - __uint_as_float(t2));
+                    const __half2 hi = __floats2half2_rn(y1, y2);
+                    const float2 hf = __half22float2(hi);
+                    const __half2 lo = __floats2half2_rn(y1 - hf.x, y2 - hf.y);
+                    qd[qoff[k][0]] = *reinterpret_cast<const uint32_t*>(&hi);
+                    qd[qoff[k][1]] = *reinterpret_cast<const uint32_t*>(&lo);
                 }
                 fence_async_smem();
             };
             auto rope_of = [&](int nn) {
                 return a.rope ? a.rope[(int64_t)tile_j0(nn) * 64 + (gt & 63)] : make_float2(1.f, 0.f);
             };
-            const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
             // two q' buffers: tile n + 2's q' is built while tile n's scores run;
             // one buffer: each tile builds its own before its RoPE
             if (nqb == 2 && n_first < s1) build_q(n_first, rope_of(n_first));
@@ -398,7 +444,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 // the next tile's query rotation, loaded now, used after this tile's RoPE
                 const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
                 if (nqb == 1) build_q(n, rope_of(n));
-                // rotate this row of K^ by R_t, store back as tf32
+                // rotate this row of K^ by R_t, store back as fp16 pairs
                 if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 if (win && !mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) fail();
@@ -434,7 +480,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                     tmem_ld16(tcs + lane_base + 128 + c0, nn);
                     tmem_wait_ld();
                     // (k1, k2) -> (k1 c - k2 s, k1 s + k2 c), two columns per packed
-                    // fp32 op; the tf32 score MMA reads the fp32 bits truncated
+                    // fp32 op, rounded to fp16 pairs for the score MMA
 #pragma unroll
                     for (int u = 0; u < 16; u += 2) {
                         const float2 k1 = make_float2(__uint_as_float(x1[u]), __uint_as_float(x1[u + 1]));
@@ -444,13 +490,14 @@ decode_tc_kernel(DecodeTcArgs a) {
                         const float2 ns = make_float2(__uint_as_float(nn[u]), __uint_as_float(nn[u + 1]));
                         const float2 y1 = __ffma2_rn(k1, co, __fmul2_rn(k2, ns));
                         const float2 y2 = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
-                        x1[u] = __float_as_uint(y1.x);
-                        x1[u + 1] = __float_as_uint(y1.y);
-                        x2[u] = __float_as_uint(y2.x);
-                        x2[u + 1] = __float_as_uint(y2.y);
+                        // column c0 + u <- fp16 (dim c0 + u, dim 64 + c0 + u): over
+                        // the fp32 columns this chunk has just read
+                        const __half2 p0 = __floats2half2_rn(y1.x, y2.x);
+                        const __half2 p1 = __floats2half2_rn(y1.y, y2.y);
+                        x1[u] = *reinterpret_cast<const uint32_t*>(&p0);
+                        x1[u + 1] = *reinterpret_cast<const uint32_t*>(&p1);
                     }
                     tmem_st16(kh + lane_base + c0, x1);
-                    tmem_st16(kh + lane_base + 64 + c0, x2);
                     if (c0 == 16 || c0 == 48) {
                         // dims 0..31 and 64..95 of this row are rotated (first barrier),
                         // then the rest (second): the score MMA starts on the first half
@@ -560,121 +607,123 @@ decode_tc_kernel(DecodeTcArgs a) {
             }
             tc_fence_before();
             group_sync(grp);
-            // a group's softmax state goes to its own q' buffer, idle now that
-            // its last score MMA of the head has completed: [m 8 | l 8 | acc 8 x 128]
-            static_assert(2 * kMaxGroup * kHeadDim <= kQN * kTile, "exchange fits");
-            float* xg = reinterpret_cast<float*>(qbb);       // [acc 8 x 128 | accd 8 x 128]
-            float* xml = mlx + grp * 2 * kMaxGroup;          // [m 8 | l 8]
-            if (gt == 0) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    xml[h] = m_run[h];
-                    xml[kMaxGroup + h] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
-                }
-            }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                if (acc_ok) xg[h * kHeadDim + c_acc] = acc[h];
-                xg[(kMaxGroup + h) * kHeadDim + row] = accd[h];
-            }
-            epi_sync();                               // both groups published
-            if (grp == 0) {
-                // log-sum-exp merge of the two groups, one partial slot per head
-                const float* x0 = reinterpret_cast<const float*>(qb);
-                const float* x1 = reinterpret_cast<const float*>(qb + nqb * kQN * kTile);
-                const float* ml0 = mlx;
-                const float* ml1 = mlx + 2 * kMaxGroup;
-                const int bq = head / a.Hkv, kvh = head % a.Hkv;
-                const int c_first = (int)(((int64_t)head * tph) / a.tiles_per_cta);
-                const int slot = cta - c_first;
-                const int stride = 2 + rV + d;
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float m0 = ml0[h], m1 = ml1[h];
-                    const float M = fmaxf(m0, m1);
-                    const float w0 = (m0 == -INFINITY) ? 0.f : __expf(m0 - M);
-                    const float w1 = (m1 == -INFINITY) ? 0.f : __expf(m1 - M);
-                    float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
-                    if (acc_ok)
-                        Pp[2 + c_acc] = x0[h * kHeadDim + c_acc] * w0 + x1[h * kHeadDim + c_acc] * w1;
-                    // d = 128 = group size: thread gt owns dim gt of the exact-row sum
-                    Pp[2 + rV + gt] = x0[(kMaxGroup + h) * kHeadDim + gt] * w0 +
-                                      x1[(kMaxGroup + h) * kHeadDim + gt] * w1;
-                    if (gt == 0) {
-                        Pp[0] = M;
-                        Pp[1] = ml0[kMaxGroup + h] * w0 + ml1[kMaxGroup + h] * w1;
-                    }
-                }
-            }
-            // the last CTA to publish a partial of this head merges all of them
-            // (log-sum-exp), applies B_V^T once per query head and writes out;
-            // no CTA waits for another, so no ordering between CTAs is assumed
-            __threadfence();
-            epi_sync();
+            // this group's partial of the head: slot 2 (cta - first cta of the head) + grp
+            const int bq = head / a.Hkv, kvh = head % a.Hkv;
+            const int c_first = cta_of(a, (int64_t)head * tph);
+            const int c_last = cta_of(a, ((int64_t)head + 1) * tph - 1);
+            const int stride = 2 + rV + d;
             {
-                const int c_first = (int)(((int64_t)head * tph) / a.tiles_per_cta);
-                const int c_last = (int)((((int64_t)head + 1) * tph - 1) / a.tiles_per_cta);
-                if (ept == 0) {
-                    const int before = atomicAdd(a.done + head, 1);
-                    const int last = before == c_last - c_first;
-                    if (last) a.done[head] = 0;   // ready for the next call
-                    *last_flag = last;
-                }
-                epi_sync();
-                if (*last_flag) {
-                    __threadfence();
-                    const int bq = head / a.Hkv, kvh = head % a.Hkv;
-                    const int nsl = c_last - c_first + 1;
-                    const int stride = 2 + rV + d;
-                    // exchange area (q' buffers, 16 KB): merged acc [8][128], slot
-                    // weights [8][256], 1/L [8]
-                    static_assert((kMaxGroup * 128 + kMaxGroup * 256 + kMaxGroup) * 4 <= 2 * kQN * kTile * 4,
-                                  "combine scratch fits");
-                    float* sacc = reinterpret_cast<float*>(qb);
-                    float* sw = sacc + kMaxGroup * 128;
-                    float* sinv = sw + kMaxGroup * 256;
-                    const float* Pbase = a.partial + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * a.splits_total * stride;
-                    if (ept < g) {
-                        const float* Ph = Pbase + (int64_t)ept * a.splits_total * stride;
-                        float M = -INFINITY;
-                        for (int sl = 0; sl < nsl; ++sl) M = fmaxf(M, __ldcg(Ph + sl * stride));
-                        float L = 0.f;
-                        for (int sl = 0; sl < nsl; ++sl) {
-                            const float m = __ldcg(Ph + sl * stride);
-                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M);
-                            sw[ept * 256 + sl] = w;
-                            L = fmaf(w, __ldcg(Ph + sl * stride + 1), L);
-                        }
-                        sinv[ept] = 1.f / L;
-                    }
-                    epi_sync();
-                    for (int e = ept; e < g * rV; e += kEpi) {
-                        const int h = e / rV, c = e - (e / rV) * rV;
-                        const float* Ph = Pbase + (int64_t)h * a.splits_total * stride;
-                        float v = 0.f;
-                        for (int sl = 0; sl < nsl; ++sl) v = fmaf(sw[h * 256 + sl], __ldcg(Ph + sl * stride + 2 + c), v);
-                        sacc[h * 128 + c] = v;
-                    }
-                    epi_sync();
-                    const float* Bv = a.V.basis + ((int64_t)a.layer * BH + head) * d * rV;
-                    for (int e = ept; e < g * d; e += kEpi) {
-                        const int h = e / d, i = e - (e / d) * d;
-                        const float* Ph = Pbase + (int64_t)h * a.splits_total * stride;
-                        float v = 0.f;
-                        for (int sl = 0; sl < nsl; ++sl) v = fmaf(sw[h * 256 + sl], __ldcg(Ph + sl * stride + 2 + rV + i), v);
-                        const float* br = Bv + (int64_t)i * rV;
-                        for (int c = 0; c < rV; c += 4) {
-                            const float4 b4 = *reinterpret_cast<const float4*>(br + c);
-                            v = fmaf(sacc[h * 128 + c], b4.x, v);
-                            v = fmaf(sacc[h * 128 + c + 1], b4.y, v);
-                            v = fmaf(sacc[h * 128 + c + 2], b4.z, v);
-                            v = fmaf(sacc[h * 128 + c + 3], b4.w, v);
-                        }
-                        a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + i] = v * sinv[h];
+                const int slot = 2 * (cta - c_first) + grp;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
+                    if (acc_ok) Pp[2 + c_acc] = acc[h];
+                    Pp[2 + rV + row] = accd[h];   // d = 128 = group size: row owns dim row
+                    if (gt == 0) {
+                        Pp[0] = m_run[h];
+                        Pp[1] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
                     }
                 }
             }
-            epi_sync();                               // exchange area free again
+            // the last group to publish a partial of this head merges all of them
+            // (log-sum-exp), applies B_V^T once per query head and writes out; no
+            // group waits for another, so no ordering between CTAs is assumed.
+            // Release: the group's writes, then one thread's fence and count.
+            group_sync(grp);
+            if (gt == 0) {
+                __threadfence();
+                const int before = atomicAdd(a.done + head, 1);
+                const int lst = before == 2 * (c_last - c_first) + 1;
+                if (lst) {
+                    a.done[head] = 0;   // ready for the next call
+                    __threadfence();    // acquire: every slot's writes are visible
+                }
+                last_flag[grp] = lst;
+            }
+            group_sync(grp);
+            if (last_flag[grp]) {
+                const int nsl = 2 * (c_last - c_first + 1);
+                const float* Pbase = a.partial + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * a.splits_total * stride;
+                const float* br = a.V.basis + (((int64_t)a.layer * BH + head) * d + gt) * rV;
+                for (int c = 0; c < rV; c += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(br + c));
+                // scratch: m, l of every (slot, head) in the group's first q' buffer
+                // (8 KB; the host keeps slots x g <= 1024), the [g][r_V] merged sums
+                // in its P buffer (4 KB); both idle once the head's last score and
+                // value MMAs have completed
+                static_assert(kMaxGroup * 128 * 4 <= kPN * kTile * 2, "merge sums fit the P buffer");
+                static_assert(2 * 1024 * 4 <= kQN * kTile * 4, "slot scratch fits one q' buffer");
+                float* sacc = reinterpret_cast<float*>(pbb);
+                float* sml = reinterpret_cast<float*>(qbb);   // [slot][G] m, then [slot][G] l
+                const int nml = nsl * G;
+                for (int e = gt; e < nml; e += 128) {
+                    const float* q = Pbase + ((int64_t)(e % G) * a.splits_total + e / G) * stride;
+                    sml[e] = __ldcg(q);
+                    sml[nml + e] = __ldcg(q + 1);
+                }
+                // this thread's columns (acc column gt, exact-row dim gt) of kC slots
+                // per batch; the first batch is in flight across the barrier
+                constexpr int kC = 32 / G;
+                float xa[kC][G], xd[kC][G];
+                auto load_batch = [&](int s0) {
+#pragma unroll
+                    for (int j = 0; j < kC; ++j)
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float* q = Pbase + ((int64_t)h * a.splits_total + s0 + j) * stride;
+                            const bool in = s0 + j < nsl;
+                            xa[j][h] = (in && gt < rV) ? __ldcg(q + 2 + gt) : 0.f;
+                            xd[j][h] = in ? __ldcg(q + 2 + rV + gt) : 0.f;
+                        }
+                };
+                load_batch(0);
+                group_sync(grp);
+                float M[G], L[G], va[G], vd[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    M[h] = -INFINITY;
+                    L[h] = 0.f;
+                    va[h] = 0.f;
+                    vd[h] = 0.f;
+                }
+                for (int sl = 0; sl < nsl; ++sl)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) M[h] = fmaxf(M[h], sml[sl * G + h]);
+                for (int s0 = 0; s0 < nsl; s0 += kC) {
+                    if (s0 > 0) load_batch(s0);
+#pragma unroll
+                    for (int j = 0; j < kC; ++j)
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            if (s0 + j >= nsl) continue;
+                            const float m = sml[(s0 + j) * G + h];
+                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M[h]);
+                            L[h] = fmaf(w, sml[nml + (s0 + j) * G + h], L[h]);
+                            va[h] = fmaf(w, xa[j][h], va[h]);
+                            vd[h] = fmaf(w, xd[j][h], vd[h]);   // exact-row sum, dim gt
+                        }
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    if (gt < rV) sacc[h * rV + gt] = va[h];
+                group_sync(grp);
+                // out[h][i] = (sum_c acc[h][c] B_V[i][c] + accd[h][i]) / L_h, i = gt
+#pragma unroll 4
+                for (int c = 0; c < rV; c += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(br + c);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float4 s4 = *reinterpret_cast<const float4*>(sacc + h * rV + c);
+                        vd[h] = fmaf(s4.x, b4.x, vd[h]);
+                        vd[h] = fmaf(s4.y, b4.y, vd[h]);
+                        vd[h] = fmaf(s4.z, b4.z, vd[h]);
+                        vd[h] = fmaf(s4.w, b4.w, vd[h]);
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + gt] = vd[h] / L[h];
+                group_sync(grp);                      // P buffer free again
+            }
             n0 = s1;
         }
     } else if (warp >= 10) {
@@ -686,11 +735,11 @@ decode_tc_kernel(DecodeTcArgs a) {
         if (lane == 0) {
             const int MV = rV <= 64 ? 64 : 128;
             const uint32_t idesc_k = idesc_f32acc(1, kTile, d, 0, 0);
-            const uint32_t idesc_s = idesc_f32acc(2, kTile, kQN, 0, 0);
+            const uint32_t idesc_s = idesc_f32acc(0, kTile, kQN, 0, 0);   // fp16 x fp16
             const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 1);
             const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 1);   // exact rows: M = d
             const uint32_t sbo_k = (uint32_t)(rK / 8) * 128;
-            const uint32_t sbo_q = (kTile / 4) * 128;
+            const uint32_t sbo_q = (kTile / 8) * 128;
             const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
             const uint32_t kh = tmem + grp * kBufCols;
             const uint32_t qg = smem_u32(qb + nqb * grp * kQN * kTile);
@@ -705,7 +754,7 @@ decode_tc_kernel(DecodeTcArgs a) {
                 }
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(stage + st * stage_bytes);
-                const uint32_t b0 = smem_u32(bk + hb * bk_bytes);
+                const uint32_t b0 = smem_u32(bk + hb * bks);
                 for (int ks = 0; ks < rK / 16; ++ks)
                     for (int part = 0; part < 2; ++part)
                         mma_f16_ss(kh, desc_noswizzle(a0 + ks * 256, 128, sbo_k),
@@ -744,10 +793,10 @@ decode_tc_kernel(DecodeTcArgs a) {
                             break;
                         }
                         tc_fence_after();
-                        for (int j = 0; j < 8; ++j) {
-                            const int ks = (j < 4 ? j : j + 4) + 4 * half;
-                            mma_tf32_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
-                                        idesc_s, (half | j) != 0);
+                        for (int j = 0; j < 4; ++j) {
+                            const int ks = 4 * half + j;   // K = 16: 8 TMEM columns per step
+                            mma_f16_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
+                                       idesc_s, (half | j) != 0);
                         }
                     }
                     if (!got) {
@@ -812,8 +861,7 @@ decode_tc_kernel(DecodeTcArgs a) {
 }  // namespace
 
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb) {
-    // + queries of the head (g x d fp32)
-    return plan_smem(rK, rV, ns, nbk, nqb).total + (size_t)kMaxGroup * kHeadDim * 4;
+    return plan_smem(rK, rV, ns, nbk, nqb).total;
 }
 
 template <int G>
