@@ -25,6 +25,7 @@ import json
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -54,7 +55,7 @@ BLOCK = 64
 # r_V 64), from the ncu launch list in profiles/launches_qwen3-1L-b8-32k.md
 # (the 36-layer run issues the same launch once per layer).  None for
 # workloads without a capture.
-DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.7e6, "qwen3-1L-b8-32k": 433.7e6}
+DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.9e6, "qwen3-1L-b8-32k": 433.9e6}
 
 
 def _peaks():
@@ -77,8 +78,16 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
+        self.lines = []
+        self.first = 0
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
 
     def start(self):
+        """Start sampling and return once the first sample has arrived (at most
+        a few seconds), so that even a short timed region is covered."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
@@ -86,16 +95,26 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+        t_end = time.time() + 5.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
+        self.first = len(self.lines)
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        # at least one sample taken after the timed region started
+        t_end = time.time() + 1.0
+        while len(self.lines) <= self.first and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out = ""
+        out = "".join(self.lines[self.first:])
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
