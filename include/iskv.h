@@ -20,7 +20,8 @@
  *    across the ABI.  iskv_strerror() names a code.
  *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *    default stream).  Work is enqueued on it and the call returns without
- *    waiting, except iskv_status, iskv_get_counts and iskv_destroy.  Calls on
+ *    waiting, except iskv_status, iskv_get_counts, iskv_kv_bytes and
+ *    iskv_destroy (host only or synchronizing).  Calls on
  *    one cache must be ordered on one stream (or ordered by the caller).
  *  - Caller buffers (k, v, q, out, ...): contiguous, row-major, owned by the
  *    caller and borrowed only for the stream-ordered duration of the call.
@@ -103,6 +104,14 @@ typedef struct {
                                iskv_sync is required (0: no postponing)     */
     int32_t jacobi_max_sweeps; /* sweep limit of the core SVD (0: 40)        */
     int32_t ring_extra;     /* exact-window ring rows beyond W + 64 (0: 64)  */
+    int32_t protect;        /* P: leading positions (the prompt's protected
+                               rows) kept exact and never folded (0: none).
+                               Positions 0..P-1 stay exact, P..P+n_c-1 are
+                               folded rows, P+n_c..T-1 the exact window.
+                               The iS-KV explainer ("What does it mean?",
+                               the paint-shop section) keeps a set of
+                               protected prompt positions exact beside the
+                               recent window.                               */
 } iskv_config;
 
 /* Fill `cfg` with the defaults of the one-layer Qwen3-8B-shaped cache
@@ -120,10 +129,11 @@ ISKV_API int iskv_destroy(iskv_t h);
 
 /* Append t tokens to every sequence of `layer`: k, v are
  * [batch, kv_heads, t, head_dim] in kv_dtype, PRE-RoPE.  T += t.  Never folds.
- * *ready_blocks (may be NULL) receives floor((T - n_c - W) / 64), at least 0:
- * the whole blocks that have left the exact window and may be folded.
- * Errors: CAPACITY if T + t > max_tokens or the ring would hold more than
- * W + 64 + ring_extra rows (fold first).                                   */
+ * *ready_blocks (may be NULL) receives floor((T - P - n_c - W) / 64), at
+ * least 0 (P = protected positions): the whole blocks that have left the
+ * exact window and may be folded.  Positions below P go to the protected
+ * rows.  Errors: CAPACITY if T + t > max_tokens or the ring would hold more
+ * than W + 64 + ring_extra rows (fold first).                              */
 ISKV_API int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t,
                 void* stream, int* ready_blocks);
 
@@ -168,6 +178,17 @@ ISKV_API int iskv_get_factors(iskv_t h, int layer, int which, float* basis, floa
 
 /* Host counters of `layer`: tokens appended and tokens folded.             */
 ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
+
+/* Persistent-KV bytes (the iS-KV explainer, Jargon: Persistent-KV
+ * compression): what the cache keeps between decode steps for every layer,
+ * sequence and KV head at the current T and n_c -- coefficient rows
+ * (n_c x (r_K + r_V) in coef_dtype), bases and singular values (fp32,
+ * (d + 1)(r_K + r_V)), exact window and protected rows (K and V in kv_dtype)
+ * -- and the bytes of the uncompressed K/V cache of the same T in kv_dtype.
+ * Neither counts preallocated capacity, the exact-window ring's spare rows
+ * or temporary buffers.  Either pointer may be NULL.  Host only, no GPU work.
+ * Errors: INVALID_ARG for a NULL cache.                                    */
+ISKV_API int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes);
 
 /* Synchronize the device and return the cache's sticky device status:
  * ISKV_OK, ISKV_ERR_DEVICE_TIMEOUT, ISKV_ERR_NOCONVERGE or ISKV_ERR_CUDA.

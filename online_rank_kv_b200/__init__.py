@@ -56,7 +56,7 @@ class _Cfg(ctypes.Structure):
         "batch", "layers", "kv_heads", "q_heads", "head_dim", "rank_k", "rank_v", "window",
         "block", "max_tokens", "kv_dtype", "coef_dtype", "use_rope")] + [
         ("rope_theta", ctypes.c_double)] + [(n, ctypes.c_int32) for n in (
-            "sync", "max_deferred", "jacobi_max_sweeps", "ring_extra")]
+            "sync", "max_deferred", "jacobi_max_sweeps", "ring_extra", "protect")]
 
 
 class DecodeOperands(ctypes.Structure):
@@ -80,6 +80,7 @@ _SIGS = {
     "iskv_reconstruct": ([_vp, _i, _i, _vp, _vp], _i),
     "iskv_get_factors": ([_vp, _i, _i, _vp, _vp, _vp, _vp], _i),
     "iskv_get_counts": ([_vp, _i, _i64p, _i64p], _i),
+    "iskv_kv_bytes": ([_vp, _i64p, _i64p], _i),
     "iskv_status": ([_vp], _i),
     "iskv_strerror": ([_i], ctypes.c_char_p),
     "iskv_decode_attention_noalloc": ([ctypes.POINTER(DecodeOperands), _vp, _vp, _vp], _i),
@@ -132,6 +133,7 @@ class Config:
     max_deferred: int = 0
     jacobi_max_sweeps: int = 0
     ring_extra: int = 0
+    protect: int = 0
 
     def _c(self) -> _Cfg:
         c = _Cfg()
@@ -234,6 +236,13 @@ class Cache:
         _check(LIB.iskv_get_counts(self._h, layer, ctypes.byref(T), ctypes.byref(n)),
                "iskv_get_counts")
         return T.value, n.value
+
+    def kv_bytes(self):
+        """(persistent bytes kept between decode steps, bytes of the uncompressed
+        K/V cache at the same T), summed over every layer, sequence and KV head."""
+        p, f = ctypes.c_int64(), ctypes.c_int64()
+        _check(LIB.iskv_kv_bytes(self._h, ctypes.byref(p), ctypes.byref(f)), "iskv_kv_bytes")
+        return p.value, f.value
 
     def status(self) -> int:
         return LIB.iskv_status(self._h)

@@ -30,6 +30,9 @@ struct iskv_cache {
     // device memory
     void* ring_k = nullptr;
     void* ring_v = nullptr;
+    void* prot_k = nullptr;       // protected rows 0..P-1, blocked like the ring
+    void* prot_v = nullptr;
+    int64_t pcap = 0;             // protected rows per head (P rounded up to 64)
     void* coef_k = nullptr;
     void* coef_v = nullptr;
     float* basis_k = nullptr;
@@ -92,6 +95,7 @@ int validate(const iskv_config* c) {
     if (c->max_deferred < 0 || c->max_deferred > kMaxDeferred) return ISKV_ERR_INVALID_ARG;
     if (c->jacobi_max_sweeps < 0 || c->jacobi_max_sweeps > 1000) return ISKV_ERR_INVALID_ARG;
     if (c->ring_extra < 0 || c->ring_extra % kBlock != 0) return ISKV_ERR_INVALID_ARG;
+    if (c->protect < 0 || c->protect > c->max_tokens) return ISKV_ERR_INVALID_ARG;
     return ISKV_OK;
 }
 
@@ -105,6 +109,9 @@ FactorView view(const iskv_cache* h, int which) {
     f.pend = K ? h->pend_k : h->pend_v;
     f.seg_rows = h->seg_rows;   // identical for K and V: both fold together
     f.ring = K ? h->ring_k : h->ring_v;
+    f.prot = K ? h->prot_k : h->prot_v;
+    f.P = h->cfg.protect;
+    f.pcap = h->pcap;
     f.r = K ? h->cfg.rank_k : h->cfg.rank_v;
     f.coef_bf16 = h->cfg.coef_dtype == ISKV_BF16;
     f.coef_blocked = f.coef_bf16;   // bf16 rows live in 8x8 core-matrix blocks
@@ -117,8 +124,14 @@ FactorView view(const iskv_cache* h, int which) {
     return f;
 }
 
+// rows of the layer's factor stream: the positions after the protected ones
+int64_t factor_rows(const iskv_cache* h, int layer) {
+    const int64_t tf = h->T[layer] - h->cfg.protect;
+    return tf > 0 ? tf : 0;
+}
+
 int64_t ready_of(const iskv_cache* h, int layer) {
-    const int64_t excess = h->T[layer] - h->n_c[layer] - h->cfg.window;
+    const int64_t excess = factor_rows(h, layer) - h->n_c[layer] - h->cfg.window;
     return excess >= 0 ? excess / kBlock : 0;
 }
 
@@ -129,7 +142,7 @@ int64_t ready_of(const iskv_cache* h, int layer) {
     } while (0)
 
 void free_all(iskv_cache* h) {
-    void* ptrs[] = {h->ring_k, h->ring_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
+    void* ptrs[] = {h->ring_k, h->ring_v, h->prot_k, h->prot_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
                     h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out};
     for (void* p : ptrs)
@@ -211,6 +224,7 @@ int iskv_config_default(iskv_config* c) {
     c->max_deferred = 0;
     c->jacobi_max_sweeps = 0;
     c->ring_extra = 0;
+    c->protect = 0;
     return ISKV_OK;
 }
 
@@ -232,6 +246,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     const iskv_config& c = h->cfg;
     h->BH = c.batch * c.kv_heads;
     h->cap = (int64_t)c.window + kBlock + c.ring_extra;
+    h->pcap = ((int64_t)c.protect + kBlock - 1) / kBlock * kBlock;
     int64_t nm = (int64_t)c.max_tokens - c.window;
     if (nm < 0) nm = 0;
     h->n_max = (nm / kBlock) * kBlock + 2 * kBlock;   // slack rows for whole tiles
@@ -254,6 +269,11 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     rc = ISKV_OK;
     rc = rc ? rc : dalloc(&h->ring_k, ring_bytes);
     rc = rc ? rc : dalloc(&h->ring_v, ring_bytes);
+    const size_t prot_bytes = heads * h->pcap * d * h->kv_bytes;
+    if (prot_bytes > 0) {
+        rc = rc ? rc : dalloc(&h->prot_k, prot_bytes);
+        rc = rc ? rc : dalloc(&h->prot_v, prot_bytes);
+    }
     rc = rc ? rc : dalloc(&h->coef_k, heads * h->n_max * c.rank_k * h->coef_bytes);
     rc = rc ? rc : dalloc(&h->coef_v, heads * h->n_max * c.rank_v * h->coef_bytes);
     rc = rc ? rc : dalloc(&h->basis_k, heads * d * c.rank_k * 4);
@@ -297,6 +317,8 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     if (rc == ISKV_OK) {
         if (cudaMemsetAsync(h->ring_k, 0, ring_bytes, s) != cudaSuccess ||
             cudaMemsetAsync(h->ring_v, 0, ring_bytes, s) != cudaSuccess ||
+            (prot_bytes > 0 && (cudaMemsetAsync(h->prot_k, 0, prot_bytes, s) != cudaSuccess ||
+                                cudaMemsetAsync(h->prot_v, 0, prot_bytes, s) != cudaSuccess)) ||
             cudaMemsetAsync(h->coef_k, 0, heads * h->n_max * c.rank_k * h->coef_bytes, s) != cudaSuccess ||
             cudaMemsetAsync(h->coef_v, 0, heads * h->n_max * c.rank_v * h->coef_bytes, s) != cudaSuccess ||
             cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess ||
@@ -327,19 +349,39 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
                 int* ready_blocks) {
     if (!h || !k || !v || t < 0 || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
     const int64_t T1 = h->T[layer] + t;
-    if (T1 > h->cfg.max_tokens || T1 - h->n_c[layer] > h->cap) return ISKV_ERR_CAPACITY;
+    const int64_t P = h->cfg.protect;
+    const int64_t tf1 = T1 > P ? T1 - P : 0;   // factor-stream rows after the call
+    if (T1 > h->cfg.max_tokens || tf1 - h->n_c[layer] > h->cap) return ISKV_ERR_CAPACITY;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (t > 0) {
         const size_t row_bytes = (size_t)kHeadDim * h->kv_bytes;
         const size_t head_stride = (size_t)h->cap * row_bytes;
+        const size_t prot_stride = (size_t)h->pcap * row_bytes;
         char* rk = reinterpret_cast<char*>(h->ring_k) + (size_t)layer * h->BH * head_stride;
         char* rv = reinterpret_cast<char*>(h->ring_v) + (size_t)layer * h->BH * head_stride;
+        char* pk = h->prot_k ? reinterpret_cast<char*>(h->prot_k) + (size_t)layer * h->BH * prot_stride : nullptr;
+        char* pv = h->prot_v ? reinterpret_cast<char*>(h->prot_v) + (size_t)layer * h->BH * prot_stride : nullptr;
         const void* srcs[2] = {k, v};
         char* rings[2] = {rk, rv};
+        char* prots[2] = {pk, pv};
+        const int blocked = h->cfg.kv_dtype == ISKV_BF16;
+        // n rows of src ([BH][src_t][d], from src_row0) at absolute positions
+        // pos0..: those below P to the protected rows, the rest to the ring at
+        // factor position (pos - P)
+        auto place = [&](int w, const void* src, int n, int src_t, int src_row0, int64_t pos0) -> int {
+            const int np = (int)std::max<int64_t>(0, std::min<int64_t>(pos0 + n, P) - pos0);
+            if (np > 0)
+                CU(launch_append(prots[w], src, h->BH, np, src_t, src_row0, pos0, h->pcap, h->kv_bytes,
+                                 blocked, s));
+            if (n > np)
+                CU(launch_append(rings[w], src, h->BH, n - np, src_t, src_row0 + np, pos0 + np - P, h->cap,
+                                 h->kv_bytes, blocked, s));
+            return ISKV_OK;
+        };
         for (int w = 0; w < 2; ++w) {
             if (is_device_ptr(srcs[w])) {
-                CU(launch_append(rings[w], srcs[w], h->BH, t, h->T[layer], h->cap, h->kv_bytes,
-                                 h->cfg.kv_dtype == ISKV_BF16, s));
+                const int rc = place(w, srcs[w], t, t, 0, h->T[layer]);
+                if (rc != ISKV_OK) return rc;
             } else {
                 // stage token chunks of every (sequence, head) through device memory
                 const int chunk = (int)std::max<size_t>(1, h->stage_in_bytes / ((size_t)h->BH * row_bytes));
@@ -349,8 +391,8 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
                                          reinterpret_cast<const char*>(srcs[w]) + t0 * row_bytes,
                                          (size_t)t * row_bytes, n * row_bytes, h->BH,
                                          cudaMemcpyDefault, s));
-                    CU(launch_append(rings[w], h->stage_in, h->BH, n, h->T[layer] + t0, h->cap,
-                                     h->kv_bytes, h->cfg.kv_dtype == ISKV_BF16, s));
+                    const int rc = place(w, h->stage_in, n, n, 0, h->T[layer] + t0);
+                    if (rc != ISKV_OK) return rc;
                 }
             }
         }
@@ -529,8 +571,10 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.n_c = a.n_c;
         t.T = a.T;
         t.scale = a.scale;
+        const int64_t P = c.protect, Pe = std::min<int64_t>(a.T, P);
         t.tiles_c = (int)((a.n_c + 127) / 128);
-        t.tiles_per_head = t.tiles_c + (int)((a.T - a.n_c + 63) / 64);
+        t.tiles_w = (int)((factor_rows(h, layer) - a.n_c + 63) / 64);
+        t.tiles_per_head = t.tiles_c + t.tiles_w + (int)((Pe + 63) / 64);
         t.total_tiles = (int64_t)h->BH * t.tiles_per_head;
         // each CTA publishes two partials (one per epilogue group) for every head
         // it visits; fewer CTAs when a head would span more slots than the
@@ -649,6 +693,24 @@ int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
             }
         }
     }
+    return ISKV_OK;
+}
+
+int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes) {
+    if (!h) return ISKV_ERR_INVALID_ARG;
+    const iskv_config& c = h->cfg;
+    const int64_t d = kHeadDim, rs = (int64_t)c.rank_k + c.rank_v;
+    int64_t kept = 0, full = 0;
+    for (int l = 0; l < c.layers; ++l) {
+        const int64_t T = h->T[l], n_c = h->n_c[l];
+        const int64_t exact = T - n_c;   // protected rows and the window
+        int64_t per_head = 2 * exact * d * h->kv_bytes;
+        if (n_c > 0) per_head += n_c * rs * h->coef_bytes + (d + 1) * rs * 4;   // C; B and S in fp32
+        kept += per_head * h->BH;
+        full += 2 * T * d * h->kv_bytes * h->BH;
+    }
+    if (persistent_bytes) *persistent_bytes = kept;
+    if (full_bytes) *full_bytes = full;
     return ISKV_OK;
 }
 

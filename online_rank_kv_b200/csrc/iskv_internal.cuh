@@ -67,7 +67,11 @@ struct FactorView {
     float* sigma;        // [L][BH][r]
     float* pend;         // [L][BH][D][r*r]: W_r[0:r,:] of postponed folds
     int* seg_rows;       // [L][D]: n_c before each postponed fold
-    const void* ring;    // [L][BH][cap][d], kv dtype (exact rows)
+    const void* ring;    // [L][BH][cap][d], kv dtype (exact window rows; factor
+                         // position j = absolute position - P sits at slot j % cap)
+    const void* prot;    // [L][BH][pcap][d], kv dtype (protected rows 0..P-1), or null
+    int64_t P;           // protected leading positions
+    int64_t pcap;        // protected rows per head (P rounded up to 64)
     int r;
     int coef_bf16;       // 1: coef stored as bf16
     int coef_blocked;    // 1: coef rows in 8x8 core-matrix blocks (see coef_index)
@@ -125,7 +129,8 @@ struct DecodeTcArgs {
     int layer, B, Hkv, Hq, g;
     int64_t n_c, T;
     int tiles_c;                 // folded-row tiles per head: ceil(n_c / 128)
-    int tiles_per_head;          // tiles_c + exact-row tiles of 64: ceil((T - n_c) / 64)
+    int tiles_w;                 // exact window tiles of 64: ceil((T - P - n_c) / 64)
+    int tiles_per_head;          // tiles_c + tiles_w + protected tiles of 64: ceil(min(T, P) / 64)
     int64_t total_tiles;         // BH * tiles_per_head
     int ncta;
     // CTA i takes the flattened tiles [cta_start[i], cta_start[i + 1])
@@ -142,8 +147,8 @@ struct DecodeTcArgs {
 // Host launchers (one per kernel file).
 // ---------------------------------------------------------------------------
 cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s);
-cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0,
-                          int64_t cap, int elem_bytes, int blocked, cudaStream_t s);
+cudaError_t launch_append(void* ring, const void* src, int BH, int t, int src_t, int src_row0,
+                          int64_t T0, int64_t cap, int elem_bytes, int blocked, cudaStream_t s);
 cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status,
                         cudaStream_t s);
 cudaError_t launch_compose(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);

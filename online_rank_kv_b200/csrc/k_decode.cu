@@ -5,11 +5,12 @@
 // and rotated when read) and the ASKV design report (Design requirements: no
 // reconstruction on the decode path, i.e. values stay in coefficient form).
 // For query head h of KV head h/g and token j:
-//   s_j = q_h . RoPE(k_j, j) / sqrt(d),  k_j = C_K[j] B_K^T (j < n_c) or the
-//   exact row (j >= n_c);  p = softmax(s) over all T tokens;
-//   out_h = (sum_{j<n_c} p_j C_V[j]) B_V^T + sum_{j>=n_c} p_j V_j.
+//   s_j = q_h . RoPE(k_j, j) / sqrt(d),  k_j = C_K[j - P] B_K^T for the folded
+//   positions P <= j < P + n_c, the exact row otherwise (the P protected
+//   positions and the window);  p = softmax(s) over all T tokens;
+//   out_h = (sum_folded p_j C_V[j - P]) B_V^T + sum_exact p_j V_j.
 // decode_kernel: one CTA per (split, KV head, sequence) streams 64-token
-// tiles of its split (never straddling n_c), keeps an online softmax (m, l)
+// tiles of its split (never straddling P or P + n_c), keeps an online softmax (m, l)
 // per query head and accumulates r_V-wide (folded) and d-wide (exact) sums.
 // combine_kernel merges the splits by log-sum-exp and applies B_V^T once.
 #include "iskv_internal.cuh"
@@ -90,21 +91,27 @@ decode_kernel(DecodeArgs a) {
     const CoefT* Cv = reinterpret_cast<const CoefT*>(a.V.coef) + hidx * a.V.n_max * rV;
     const KvT* Rk = reinterpret_cast<const KvT*>(a.K.ring) + hidx * a.K.cap * d;
     const KvT* Rv = reinterpret_cast<const KvT*>(a.V.ring) + hidx * a.V.cap * d;
+    const KvT* Pk = reinterpret_cast<const KvT*>(a.K.prot) + hidx * a.K.pcap * d;
+    const KvT* Pv = reinterpret_cast<const KvT*>(a.V.prot) + hidx * a.V.pcap * d;
+    const int64_t P = a.K.P, c_end = P + a.n_c;   // folded positions: [P, P + n_c)
     __syncthreads();
 
     for (int64_t j = j0; j < j1;) {
-        const bool comp = j < a.n_c;
+        const bool prot = j < P;
+        const bool comp = !prot && j < c_end;
         int64_t jend = j + kTile;
         if (jend > j1) jend = j1;
-        if (comp && jend > a.n_c) jend = a.n_c;
+        if (prot && jend > P) jend = P;
+        if (comp && jend > c_end) jend = c_end;
         const int nt = (int)(jend - j);
 
         if (comp) {
+            const int64_t jc = j - P;   // coefficient row
             for (int e = tid; e < kTile * rK; e += kThreads)
-                sCk[e] = (e / rK < nt) ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, j + e / rK, e % rK)])
+                sCk[e] = (e / rK < nt) ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, jc + e / rK, e % rK)])
                                        : 0.f;
             for (int e = tid; e < kTile * rV; e += kThreads)
-                sCv[e] = (e / rV < nt) ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, j + e / rV, e % rV)])
+                sCv[e] = (e / rV < nt) ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, jc + e / rV, e % rV)])
                                        : 0.f;
             __syncthreads();
             for (int e = tid; e < kTile * d; e += kThreads) {
@@ -117,8 +124,11 @@ decode_kernel(DecodeArgs a) {
             for (int e = tid; e < kTile * d; e += kThreads) {
                 const int t = e / d, i = e % d;
                 float kv = 0.f, vv = 0.f;
-                if (t < nt) {
-                    const int64_t slot = (j + t) % a.K.cap;
+                if (t < nt && prot) {
+                    kv = to_f32(Pk[coef_index(a.K.ring_blocked, d, j + t, i)]);
+                    vv = to_f32(Pv[coef_index(a.V.ring_blocked, d, j + t, i)]);
+                } else if (t < nt) {
+                    const int64_t slot = (j + t - P) % a.K.cap;   // factor position j - P
                     kv = to_f32(Rk[coef_index(a.K.ring_blocked, d, slot, i)]);
                     vv = to_f32(Rv[coef_index(a.V.ring_blocked, d, slot, i)]);
                 }

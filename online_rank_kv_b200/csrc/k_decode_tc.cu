@@ -177,7 +177,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
     const uint32_t stage_bytes = P.stage_bytes;
-    const int tiles_c = a.tiles_c;
+    const int tiles_c = a.tiles_c, tiles_cw = a.tiles_c + a.tiles_w;
     constexpr uint32_t kWinBytes = kWinTile * kHeadDim * 2;   // one of K, V
     const uint32_t bk_bytes = 2 * kTile * rK * 2;   // B_hi, B_lo of one head
     const uint32_t bks = bk_stride(rK);
@@ -270,13 +270,20 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     bulk_g2s(sk, gk, P.stage_k, &bars->full[st]);
                     bulk_g2s(sk + P.stage_k, gv, kTile * rV * 2, &bars->full[st]);
                 } else {
-                    // exact rows j0..j0+63 sit in ring slots j0 % cap.. (no wrap: cap % 64 == 0)
-                    const int64_t j0 = a.n_c + (int64_t)(tile - tiles_c) * kWinTile;
-                    const int64_t slot0 = j0 % a.K.cap;
-                    const __nv_bfloat16* rk = reinterpret_cast<const __nv_bfloat16*>(a.K.ring) +
-                                              (hidx * a.K.cap + slot0) * d;
-                    const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(a.V.ring) +
-                                              (hidx * a.V.cap + slot0) * d;
+                    const __nv_bfloat16 *rk, *rv;
+                    if (tile < tiles_cw) {
+                        // window rows at factor positions j0..j0+63 sit in ring slots
+                        // j0 % cap.. (no wrap: cap % 64 == 0)
+                        const int64_t j0 = a.n_c + (int64_t)(tile - tiles_c) * kWinTile;
+                        const int64_t slot0 = j0 % a.K.cap;
+                        rk = reinterpret_cast<const __nv_bfloat16*>(a.K.ring) + (hidx * a.K.cap + slot0) * d;
+                        rv = reinterpret_cast<const __nv_bfloat16*>(a.V.ring) + (hidx * a.V.cap + slot0) * d;
+                    } else {
+                        // protected rows j0..j0+63 (positions below P)
+                        const int64_t j0 = (int64_t)(tile - tiles_cw) * kWinTile;
+                        rk = reinterpret_cast<const __nv_bfloat16*>(a.K.prot) + (hidx * a.K.pcap + j0) * d;
+                        rv = reinterpret_cast<const __nv_bfloat16*>(a.V.prot) + (hidx * a.V.pcap + j0) * d;
+                    }
                     mbar_arrive_expect_tx(&bars->full[st], 2 * kWinBytes);
                     bulk_g2s(sk, rk, kWinBytes, &bars->full[st]);
                     bulk_g2s(sk + kWinBytes, rv, kWinBytes, &bars->full[st]);
@@ -292,7 +299,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     } else if (warp >= 2 && warp < 10) {
         // ---------------- epilogue: two groups of 4 warps, alternate tiles ----------------
         const int ept = tid - 64;                 // 0..255
-        const int nc32 = (int)a.n_c, T32 = (int)a.T;
+        // positions: protected [0, P), folded [P, P + n_c), window [P + n_c, T)
+        const int nc32 = (int)a.n_c, T32 = (int)a.T, P32 = (int)a.K.P;
+        const int Pe32 = T32 < P32 ? T32 : P32;
         const int grp = ept >> 7;                 // tiles n with n % 2 == grp
         const int gt = ept & 127;                 // thread within the group
         const int sp = warp & 3;                  // TMEM sub-partition of this warp
@@ -393,11 +402,14 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             if (n_first < s1 && !mbar_wait(&bars->bk_full[hs % nbk], (hs / nbk) & 1, deadline)) fail();
             bool have_prev = false, prev_win = false;
             int last = -1;
-            // first position of a tile (folded tiles of 128 rows, then exact tiles of 64)
+            // first position of a tile: folded tiles of 128 rows, then window tiles
+            // of 64, then protected tiles of 64
             const int64_t hbase = (int64_t)head * tph;   // flattened index of the head's tile 0
             auto tile_j0 = [&](int nn) {   // positions fit in 32 bits (max_tokens is an int32)
                 const int lc = (int)(f0 + nn - hbase);
-                return lc >= tiles_c ? nc32 + (lc - tiles_c) * kWinTile : lc * kTile;
+                return lc < tiles_c ? P32 + lc * kTile
+                                    : lc < tiles_cw ? P32 + nc32 + (lc - tiles_c) * kWinTile
+                                                    : (lc - tiles_cw) * kWinTile;
             };
             // q' = R_{j0}^T q of tile nn as fp16 hi / lo parts (the score MMA's B
             // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
@@ -438,7 +450,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 const int local = (int)(f0 + n - hbase);
                 const bool win = local >= tiles_c;    // exact rows (64-token tile)
                 const int j0 = tile_j0(n);
-                const int lim = win ? T32 : nc32;
+                const int lim = !win ? P32 + nc32 : local < tiles_cw ? T32 : Pe32;
                 const int span = win ? kWinTile : kTile;
                 const int valid = (lim - j0) < span ? (lim - j0) : span;
                 // the next tile's query rotation, loaded now, used after this tile's RoPE

@@ -27,8 +27,10 @@ __global__ void init_factor_kernel(FactorView f, int layers) {
 // ring[bh][(T0 + t) mod cap][:] = src[bh][t][:], 16-byte vectors; with
 // `blocked` (bf16 rows of 128) the destination is the 8x8 core-matrix layout:
 // vector v of slot s lands at ((s / 8) * 16 + v) * 8 + s % 8.
-__global__ void append_kernel(uint4* ring, const uint4* src, int BH, int t, int64_t T0,
-                              int64_t cap, int vec_per_row, int blocked) {
+// Rows src_row0 .. src_row0 + t - 1 of every head of src ([BH][src_t][d]) to
+// slots (T0 + i) % cap of the per-head ring ([BH][cap][d], blocked or not).
+__global__ void append_kernel(uint4* ring, const uint4* src, int BH, int t, int src_t, int src_row0,
+                              int64_t T0, int64_t cap, int vec_per_row, int blocked) {
     const int64_t total = (int64_t)BH * t * vec_per_row;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -38,7 +40,7 @@ __global__ void append_kernel(uint4* ring, const uint4* src, int BH, int t, int6
         const int64_t slot = (T0 + tt) % cap;
         const int64_t dst = blocked ? bh * cap * vec_per_row + ((slot >> 3) * vec_per_row + v) * 8 + (slot & 7)
                                     : (bh * cap + slot) * vec_per_row + v;
-        ring[dst] = src[e];
+        ring[dst] = src[(bh * src_t + src_row0 + tt) * vec_per_row + v];
     }
 }
 
@@ -112,16 +114,17 @@ cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s) 
     return cudaGetLastError();
 }
 
-cudaError_t launch_append(void* ring, const void* src, int BH, int t, int64_t T0, int64_t cap,
-                          int elem_bytes, int blocked, cudaStream_t s) {
+cudaError_t launch_append(void* ring, const void* src, int BH, int t, int src_t, int src_row0,
+                          int64_t T0, int64_t cap, int elem_bytes, int blocked, cudaStream_t s) {
+    if (t <= 0) return cudaSuccess;
     const int vec_per_row = kHeadDim * elem_bytes / 16;
     const int64_t total = (int64_t)BH * t * vec_per_row;
     int64_t blocks = (total + 255) / 256;
     if (blocks > 4736) blocks = 4736;
     if (blocks < 1) blocks = 1;
     append_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(ring),
-                                                   reinterpret_cast<const uint4*>(src), BH, t, T0,
-                                                   cap, vec_per_row, blocked);
+                                                   reinterpret_cast<const uint4*>(src), BH, t, src_t,
+                                                   src_row0, T0, cap, vec_per_row, blocked);
     return cudaGetLastError();
 }
 

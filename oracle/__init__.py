@@ -29,4 +29,5 @@ from .iskv_oracle import (  # noqa: F401
     HeadFactor,
     dense_decode,
     full_kv_bytes,
+    persistent_kv_bytes,
 )

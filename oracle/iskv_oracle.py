@@ -219,6 +219,13 @@ class HeadFactor:
     every resync).  ``sync=False`` is the no-synchronization ablation: old
     rows keep the coefficients of the basis they were written in.
 
+    ``protect`` = P leading positions (protected prompt rows, kept exact
+    beside the recent window: the explainer's paint-shop section and its
+    Persistent-KV compression entry) never enter the factor: the factor's
+    stream is rows P, P+1, ..., its blocks are counted and folded as if the
+    stream began there, and attention sees positions 0..P-1 exact, then the
+    n_c folded rows, then the window.
+
     ``fold(defer=True)`` postpones step (e) for the rows already stored; the
     postponed rewrites are applied in order by ``sync()``, with one storage
     rounding at the end.  With nothing read in between this equals the
@@ -227,10 +234,11 @@ class HeadFactor:
     """
 
     def __init__(self, d: int, r: int, W: int, b: int = 64, coef_round=None,
-                 sync: bool = True):
-        if not (0 < r <= d) or b <= 0 or W < 0:
+                 sync: bool = True, protect: int = 0):
+        if not (0 < r <= d) or b <= 0 or W < 0 or protect < 0:
             raise ValueError("invalid factor shape")
         self.d, self.r, self.W, self.b = d, r, W, b
+        self.P = protect
         self.coef_round = coef_round
         self.sync_enabled = sync
         self.B = np.eye(d)[:, :r].copy()
@@ -283,13 +291,18 @@ class HeadFactor:
         self._nrows += rows.shape[0]
         return self.ready()
 
+    @property
+    def T_factor(self) -> int:
+        """Rows of the factor's stream (those after the protected positions)."""
+        return max(0, self.T - self.P)
+
     def ready(self) -> int:
-        return ready_blocks(self.T, self.n_c, self.W, self.b)
+        return ready_blocks(self.T_factor, self.n_c, self.W, self.b)
 
     def fold(self, defer: bool = False, keep_history: bool = False) -> FoldResult:
         if self.ready() < 1:
             raise RuntimeError("no ready block")
-        X = self.rows[self.n_c:self.n_c + self.b]
+        X = self.rows[self.P + self.n_c:self.P + self.n_c + self.b]
         res = fold_block(self.B, self.S, X)
         # (e) basis synchronization of the rows stored so far
         if self.sync_enabled and self.n_c > 0:
@@ -337,12 +350,26 @@ class HeadFactor:
             raise RuntimeError("postponed rewrites pending; call sync()")
         return self.C @ self.B.T
 
+    def protected(self) -> np.ndarray:
+        """The protected rows (positions 0 .. min(T, P) - 1), as appended."""
+        return self.rows[:min(self.T, self.P)]
+
     def exact(self) -> np.ndarray:
-        return self.rows[self.n_c:]
+        """The exact window: positions P + n_c .. T - 1."""
+        return self.rows[self.P + self.n_c:]
 
     def full(self) -> np.ndarray:
-        """All T rows as attention sees them: reconstructed, then exact."""
-        return np.concatenate([self.reconstruct(), self.exact()], axis=0)
+        """All T rows in position order as attention sees them: protected,
+        reconstructed, then the exact window."""
+        return np.concatenate([self.protected(), self.reconstruct(), self.exact()], axis=0)
+
+    def kept_arrays(self) -> list:
+        """The arrays this factor keeps between decode steps: the protected and
+        window rows, and, once a block is folded, C, B and S."""
+        out = [self.protected(), self.exact()]
+        if self.n_c > 0:
+            out += [self.C, self.B, self.S]
+        return out
 
 
 # ----------------------------------------------------------------------------
@@ -385,11 +412,17 @@ def full_kv_bytes(tokens: int, layers: int, kv_heads: int, head_dim: int,
 
 
 def persistent_kv_bytes(n_c: int, n_w: int, d: int, r_k: int, r_v: int,
-                        coef_bytes: int, kv_bytes: int, basis_bytes: int = 4) -> int:
-    """Bytes kept between decode steps for one (sequence, layer, KV head):
-    both factors (C, B, S) plus both exact windows.  Excludes temporary
-    buffers, as the explainer's definition does.  Parity unpinned: the pages
-    print no kept-byte figure this formula can be checked against."""
-    factors = n_c * (r_k + r_v) * coef_bytes + (d + 1) * (r_k + r_v) * basis_bytes
-    window = 2 * n_w * d * kv_bytes
-    return factors + window
+                        coef_bytes: int, kv_bytes: int, basis_bytes: int = 4,
+                        n_p: int = 0) -> int:
+    """Bytes kept between decode steps for one (sequence, layer, KV head)
+    (Jargon: Persistent-KV compression): both factors (C, and B, S once a
+    block is folded), both exact windows (n_w rows) and both sets of
+    protected rows (n_p).  Excludes temporary buffers, as the explainer's
+    definition does.  Pinned against a count of the arrays the oracle keeps;
+    the explainer's kept-byte figure itself (1.808 GiB on the A40) cannot be
+    re-derived from what the pages state, so that number stays unpinned."""
+    factors = 0
+    if n_c > 0:
+        factors = n_c * (r_k + r_v) * coef_bytes + (d + 1) * (r_k + r_v) * basis_bytes
+    exact = 2 * (n_w + n_p) * d * kv_bytes
+    return factors + exact

@@ -43,10 +43,12 @@ class Pair:
         self.heads = heads if heads is not None else [
             (l, b, h) for l in range(self.L) for b in range(self.B) for h in range(self.H)]
         rnd = "bf16" if cfg.coef_dtype == ik.BF16 else "f32"
+        P = getattr(cfg, "protect", 0)
+        self.P = P
         self.ok = {x: HeadFactor(cfg.head_dim, cfg.rank_k, cfg.window, coef_round=rnd,
-                                 sync=bool(cfg.sync)) for x in self.heads}
+                                 sync=bool(cfg.sync), protect=P) for x in self.heads}
         self.ov = {x: HeadFactor(cfg.head_dim, cfg.rank_v, cfg.window, coef_round=rnd,
-                                 sync=bool(cfg.sync)) for x in self.heads}
+                                 sync=bool(cfg.sync), protect=P) for x in self.heads}
         self.qseed = 1000 + seed
 
     # -- inputs ------------------------------------------------------------
@@ -86,7 +88,7 @@ class Pair:
             cnt = 0
             while True:
                 T, n_c = self.cache.counts(l)
-                if (T - n_c - self.cfg.window) // 64 < 1:
+                if (max(0, T - self.P) - n_c - self.cfg.window) // 64 < 1:
                     break
                 self.fold(l, defer=defer_every > 0)
                 cnt += 1
@@ -100,7 +102,7 @@ class Pair:
         c = self.cfg
         cap = c.window + 64 + (c.ring_extra or 64)
         T, n_c = self.cache.counts(0)
-        return cap - (T - n_c)
+        return cap - (max(0, T - self.P) - n_c)
 
     def prefill(self, tokens: int, chunk: int = 64, defer_every: int = 0):
         done = 0

@@ -351,6 +351,103 @@ def test_full_kv_bytes_matches_a40_figure():
 
 
 # ----------------------------------------------------------------------------
+# protected rows (positions 0..P-1 kept exact, never folded)
+# ----------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("P", [1, 37, 64, 200])
+def test_protected_factor_is_the_unprotected_factor_of_the_shifted_stream(P):
+    """With P protected positions the factor sees the stream from row P on:
+    block counts, folds, coefficients and basis equal those of an
+    unprotected factor fed rows P, P+1, ...; attention sees the protected
+    rows first, unchanged."""
+    d, r, W = 128, 16, 128
+    rows = _low_rank_rows(P + 700, d, 12, seed=50 + P, noise=1e-3)
+    a = O.HeadFactor(d, r, W, protect=P)
+    b = O.HeadFactor(d, r, W)
+    for lo in range(0, rows.shape[0], 50):
+        chunk = rows[lo:lo + 50]
+        a.append(chunk)
+        tail = rows[max(lo, P):lo + 50]
+        if tail.shape[0]:
+            b.append(tail)
+        assert a.ready() == b.ready()
+        while a.ready() >= 1:
+            a.fold()
+            b.fold()
+    assert a.n_c == b.n_c > 0
+    np.testing.assert_array_equal(a.C, b.C)
+    np.testing.assert_array_equal(a.B, b.B)
+    np.testing.assert_array_equal(a.protected(), rows[:P])
+    np.testing.assert_array_equal(a.full()[:P], rows[:P])
+    np.testing.assert_array_equal(a.full()[P:], b.full())
+    assert a.full().shape[0] == rows.shape[0]
+
+
+def test_protected_ready_counts_brute_force():
+    """ready = floor((T - P - n_c - W) / b) when positive, by counting the
+    whole blocks that have left the window after the protected positions."""
+    W, bsz = 128, 64
+    for P in (0, 5, 64, 130):
+        for T in range(0, 900, 7):
+            for n_c in range(0, max(0, T - P) + 1, 64):
+                f = O.HeadFactor(128, 16, W, protect=P)
+                f.rows = np.zeros((T, 128))
+                f.n_c = n_c
+                free = [j for j in range(P + n_c, T) if j < T - W]   # folded-eligible rows
+                whole = 0
+                while (whole + 1) * bsz <= len(free):
+                    whole += 1
+                assert f.ready() == whole, (P, T, n_c)
+
+
+def test_protected_lossless_decode_equals_dense_attention():
+    """At r = d every row is reproduced, so decode over protected + folded +
+    window rows is dense attention over the raw rows, whatever P is."""
+    d, W, P = 128, 64, 70
+    g = _rng(61)
+    K = g.standard_normal((P + 400, d))
+    V = g.standard_normal((P + 400, d))
+    fk = O.HeadFactor(d, d, W, protect=P)
+    fv = O.HeadFactor(d, d, W, protect=P)
+    fk.append(K)
+    fv.append(V)
+    while fk.ready() >= 1:
+        fk.fold()
+        fv.fold()
+    assert fk.n_c >= 256
+    q = g.standard_normal((4, d))
+    np.testing.assert_allclose(O.dense_decode(q, fk.full(), fv.full(), 1e6),
+                               O.dense_decode(q, K, V, 1e6), atol=1e-10)
+
+
+def test_persistent_bytes_count_the_kept_arrays():
+    """The kept-byte formula equals a count of the arrays the oracle keeps
+    (elements times their stored width), for K and V factors with protected
+    rows, before and after the first fold."""
+    d, rk, rv, W, P = 128, 32, 64, 128, 40
+    g = _rng(62)
+    for n_rows in (100, P + W + 64 * 3 + 17):
+        fk = O.HeadFactor(d, rk, W, protect=P, coef_round="bf16")
+        fv = O.HeadFactor(d, rv, W, protect=P, coef_round="bf16")
+        X = g.standard_normal((n_rows, d))
+        fk.append(X)
+        fv.append(X)
+        while fk.ready() >= 1:
+            fk.fold()
+            fv.fold()
+        counted = 0
+        for f in (fk, fv):
+            prot, win = f.protected(), f.exact()
+            counted += (prot.size + win.size) * 2          # bf16 K/V rows
+            if f.n_c:
+                counted += f.C.size * 2 + (f.B.size + f.S.size) * 4   # bf16 C, fp32 B and S
+        n_w = fk.exact().shape[0]
+        n_p = fk.protected().shape[0]
+        assert O.persistent_kv_bytes(fk.n_c, n_w, d, rk, rv, 2, 2, 4, n_p=n_p) == counted
+
+
+# ----------------------------------------------------------------------------
 # mutation tests: plant mistakes in a copy of the fold, check the pins fail
 # ----------------------------------------------------------------------------
 
@@ -413,6 +510,6 @@ def test_residual_sign_is_absorbed_by_rule_q():
 
 def test_oracle_exports():
     for name in ("bf16_round", "ready_blocks", "rope_rotate", "fold_block", "HeadFactor",
-                 "dense_decode", "full_kv_bytes"):
+                 "dense_decode", "full_kv_bytes", "persistent_kv_bytes"):
         assert hasattr(oracle, name)
     _ = itertools
