@@ -243,8 +243,9 @@ def run_iskv(args, rank, world, local_rank):
     cfg = ik.Config(batch=Bsz, layers=L, kv_heads=H, q_heads=Hq, rank_k=wl["rank_k"],
                     rank_v=wl["rank_v"], window=wl["window"], max_tokens=max_tokens,
                     kv_dtype=ik.BF16, coef_dtype=coef, use_rope=1, rope_theta=1e6,
-                    max_deferred=64)
+                    max_deferred=64, protect=args.protect)
     cache = ik.Cache(cfg)
+    P = args.protect
     kdt = torch.bfloat16
     nh = L * Bsz * H
     seed_k, seed_v, seed_q = replica_seeds(rank)
@@ -260,7 +261,7 @@ def run_iskv(args, rank, world, local_rank):
         for l in range(L):
             cache.append(l, k[l], v[l])
         T, n_c = cache.counts(0)
-        while (T - n_c - wl["window"]) // BLOCK >= 1:
+        while (max(0, T - P) - n_c - wl["window"]) // BLOCK >= 1:
             cache.compress_block(ik.ALL_LAYERS, defer=True)
             folds += 1
             if folds % 64 == 0:
@@ -385,6 +386,7 @@ def run_iskv(args, rank, world, local_rank):
     h2d = BLOCK * L * (2 * Bsz * H * D * kvb + Bsz * Hq * D * kvb)
     d2h = BLOCK * L * Bsz * Hq * D * 4
     status = cache.status()
+    kept_bytes, full_bytes = cache.kv_bytes()
 
     # per decode step and layer: append (K, V) + decode attention; per period:
     # fold (K, V) + coefficient rewrite (K, V)
@@ -396,7 +398,7 @@ def run_iskv(args, rank, world, local_rank):
         "config": {
             "workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H, "q_heads": Hq,
             "head_dim": D, "rank_k": wl["rank_k"], "rank_v": wl["rank_v"],
-            "window": wl["window"], "context_start": wl["prefill"],
+            "window": wl["window"], "context_start": wl["prefill"], "protected_rows": P,
             "storage": f"K/V bf16, coefficients {wl['coef']}, bases fp32",
             "step": "64 decode steps (append + decode attention, every layer) + 1 block fold "
                     "of every layer (fold + coefficient rewrite)",
@@ -410,11 +412,15 @@ def run_iskv(args, rank, world, local_rank):
         "prefill_s": prefill_s,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.workload)
-                     if coef == ik.BF16 else None,
+                     if coef == ik.BF16 and P == 0 else None,
                      "kernel": "decode_tc_kernel (persistent split-K decode attention, "
                                "per-head combine fused), one launch per layer call",
                      "algorithmic_bytes_per_launch": bsum / max(1, len(dec_events)),
                      "peak_source": peak_src},
+        # bytes kept between decode steps at the end of the run against the
+        # uncompressed K/V cache of the same length (all layers and heads)
+        "persistent_kv": {"bytes": kept_bytes, "full_bytes": full_bytes,
+                          "compression": full_bytes / kept_bytes if kept_bytes else None},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_period * args.steps,
@@ -434,6 +440,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--protect", type=int, default=0,
+                    help="leading positions kept exact and never folded (protected prompt rows)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

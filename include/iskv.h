@@ -205,7 +205,9 @@ ISKV_API const char* iskv_strerror(int code);
  * (and forbids allocations after start-up), or a latency-critical path that
  * must avoid cudaMalloc's device-wide synchronization.  Such a caller keeps
  * the factors in its own buffers (laid out as the cache keeps them) and
- * passes them here; nothing is allocated and nothing is staged.
+ * passes them here; nothing is allocated and nothing is staged.  The
+ * operands describe a cache without protected rows (iskv_config.protect 0);
+ * caches with protected rows decode through iskv_decode_attention.
  *
  * All pointers are device memory, owned by the caller, borrowed for the
  * stream-ordered duration of the call:
