@@ -283,12 +283,22 @@ def run_iskv(args, rank, world, local_rank):
 
     step_ctr = [0]
     dec_events = []
+    step_events = []
+    side = torch.cuda.Stream(device=dev) if args.async_update else None
+    # asynchronous updates: layer l folds at step slot[l] of every 64-step
+    # period, on the side stream, right after its decode (its block is ready
+    # by then, or one period later; the ring holds up to 64 extra rows)
+    slot = [(l * BLOCK) // L for l in range(L)]
 
     def period(host=None, time_decode=False):
         for s in range(BLOCK):
             i = step_ctr[0]
             step_ctr[0] += 1
             ev = time_decode and (s % 8 == 0)
+            if time_decode:
+                se = torch.cuda.Event(enable_timing=True)
+                se.record(stream)
+                step_events.append(se)
             for l in range(L):
                 if host is None:
                     cache.append(l, kk[i, l], vv[i, l])
@@ -305,7 +315,12 @@ def run_iskv(args, rank, world, local_rank):
                     hk, hv, hq, ho = host
                     cache.append(l, hk[i, l], hv[i, l])
                     cache.decode_attention(l, hq[i, l], out=ho[i % 2, l])
-        cache.compress_block(ik.ALL_LAYERS)
+                if side is not None and slot[l] == s:
+                    T, n_c = cache.counts(l)
+                    if (max(0, T - P) - n_c - wl["window"]) // BLOCK >= 1:
+                        cache.compress_block_async(l, side, after=stream)
+        if side is None:
+            cache.compress_block(ik.ALL_LAYERS)
 
     def barrier():
         if world > 1:
@@ -325,11 +340,18 @@ def run_iskv(args, rank, world, local_rank):
     for _ in range(args.steps):
         period(time_decode=True)
     e_end.record(stream)
+    step_events.append(e_end)
     barrier()
     clk = clocks.stop()
     ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
     per_step_ms = ms / args.steps
     value = job_value(ms, args.steps, world)
+    # per-token latency: one decode step of every layer (and whatever block
+    # update work lands in it), between consecutive step events
+    tok_ms = sorted(step_events[j].elapsed_time(step_events[j + 1])
+                    for j in range(len(step_events) - 1))
+    token_latency = {"p50_ms": tok_ms[len(tok_ms) // 2], "p99_ms": tok_ms[int(0.99 * (len(tok_ms) - 1))],
+                     "max_ms": tok_ms[-1], "steps": len(tok_ms)}
 
     # decode-attention roofline from the events taken inside the timed region
     peak, peak_src = _peaks()
@@ -348,6 +370,14 @@ def run_iskv(args, rank, world, local_rank):
 
     # ---- block update timing (fold and rewrite separately), untimed pass
     fold_us = resync_us = None
+    if side is not None:
+        # bring every layer to the same phase (staggered folds leave up to 63
+        # more rows in some rings)
+        while True:
+            if all((max(0, cache.counts(l)[0] - P) - cache.counts(l)[1] - wl["window"]) // BLOCK < 1
+                   for l in range(L)):
+                break
+            cache.compress_block(ik.ALL_LAYERS)
     for _ in range(BLOCK):
         i = step_ctr[0]
         step_ctr[0] += 1
@@ -406,6 +436,9 @@ def run_iskv(args, rank, world, local_rank):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
         "tokens_per_s": value * Bsz,
+        "block_update_mode": "async per layer, staggered over the 64 steps (side stream)"
+                             if args.async_update else "sync, all layers at the end of the 64 steps",
+        "token_latency": token_latency,
         "block_update_us": fold_us + resync_us,
         "fold_us": fold_us, "resync_us": resync_us, "resync_gbs": resync_gbs,
         "decode_attention_us_avg": dec_avg_us,
@@ -440,6 +473,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--async-update", action="store_true",
+                    help="fold each layer on a second stream, one layer per decode step")
     ap.add_argument("--protect", type=int, default=0,
                     help="leading positions kept exact and never folded (protected prompt rows)")
     args = ap.parse_args()

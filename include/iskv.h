@@ -148,6 +148,21 @@ ISKV_API int iskv_append(iskv_t h, int layer, const void* k, const void* v, int 
  * max_deferred.                                                           */
 ISKV_API int iskv_compress_block(iskv_t h, int layer, int flags, void* stream);
 
+/* The same block update (fold and, unless postponed, rewrite) enqueued on a
+ * second stream, `stream`, so that it runs while the caller's stream `after`
+ * keeps decoding other layers.  It starts after everything enqueued so far on
+ * `after` (the appended rows); the next call that touches a folded layer, on
+ * whatever stream, is ordered after the update -- the swap to the updated
+ * factors happens at that call, and until the update completes nothing reads
+ * the layer.  Host counters (T, n_c) advance at once, as for
+ * iskv_compress_block.  All other calls on the cache stay on one stream.
+ * This serves the ASKV design report's requirement (Design requirements)
+ * that maintenance stay off the decode critical path: with one layer updated
+ * per call, its fold and rewrite overlap the other layers' decode.
+ * Errors: as iskv_compress_block, plus CUDA for event failures.            */
+ISKV_API int iskv_compress_block_async(iskv_t h, int layer, int flags, void* stream,
+                                       void* after);
+
 /* Apply the postponed rewrites of `layer` (or ISKV_ALL_LAYERS) in fold order:
  * one pass over the stored rows, each row multiplied by the product of the
  * W_r[0:r,:] of the folds that came after it was written.  No-op if nothing

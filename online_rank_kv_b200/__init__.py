@@ -81,6 +81,7 @@ _SIGS = {
     "iskv_get_factors": ([_vp, _i, _i, _vp, _vp, _vp, _vp], _i),
     "iskv_get_counts": ([_vp, _i, _i64p, _i64p], _i),
     "iskv_kv_bytes": ([_vp, _i64p, _i64p], _i),
+    "iskv_compress_block_async": ([_vp, _i, _i, _vp, _vp], _i),
     "iskv_status": ([_vp], _i),
     "iskv_strerror": ([_i], ctypes.c_char_p),
     "iskv_decode_attention_noalloc": ([ctypes.POINTER(DecodeOperands), _vp, _vp, _vp], _i),
@@ -191,6 +192,14 @@ class Cache:
     def compress_block(self, layer: int = ALL_LAYERS, defer: bool = False, stream=None) -> None:
         _check(LIB.iskv_compress_block(self._h, layer, FOLD_DEFER_SYNC if defer else 0,
                                        _stream(stream)), "iskv_compress_block")
+
+    def compress_block_async(self, layer: int, stream, after=None, defer: bool = False) -> None:
+        """The block update of `layer` on `stream` (a second stream), after the
+        work enqueued so far on `after` (default: the current stream); later
+        calls touching the layer are ordered after it by the library."""
+        _check(LIB.iskv_compress_block_async(self._h, layer, FOLD_DEFER_SYNC if defer else 0,
+                                             _stream(stream), _stream(after)),
+               "iskv_compress_block_async")
 
     def sync(self, layer: int = ALL_LAYERS, stream=None) -> None:
         _check(LIB.iskv_sync(self._h, layer, _stream(stream)), "iskv_sync")

@@ -60,6 +60,12 @@ struct iskv_cache {
     // host counters
     std::vector<int64_t> T, n_c;
     std::vector<int> n_pend;
+    // asynchronous block updates (iskv_compress_block_async): per layer, the
+    // event that completes the layer's last update and whether the next call
+    // touching the layer has yet to order its stream after it
+    std::vector<cudaEvent_t> upd_evt;
+    std::vector<char> upd_wait;
+    cudaEvent_t enq_evt = nullptr;   // orders an update's stream after the caller's
 };
 
 namespace {
@@ -141,7 +147,16 @@ int64_t ready_of(const iskv_cache* h, int layer) {
         if (e_ != cudaSuccess) return ISKV_ERR_CUDA;   \
     } while (0)
 
+void free_events(iskv_cache* h) {
+    for (cudaEvent_t e : h->upd_evt)
+        if (e) cudaEventDestroy(e);
+    h->upd_evt.clear();
+    if (h->enq_evt) cudaEventDestroy(h->enq_evt);
+    h->enq_evt = nullptr;
+}
+
 void free_all(iskv_cache* h) {
+    free_events(h);
     void* ptrs[] = {h->ring_k, h->ring_v, h->prot_k, h->prot_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
                     h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out};
@@ -162,6 +177,23 @@ int dalloc(T** p, size_t bytes) {
 }
 
 // Layers named by a call: one, or all of them.
+// A call on stream s that touches the listed layers runs after their last
+// asynchronous update (the swap to the updated factors happens here, at the
+// next call, not at the update's launch).  Callers keep every other call on
+// one stream, so one wait per update suffices.
+int order_after_updates(iskv_cache* h, const std::vector<int>& ls, cudaStream_t s) {
+    for (int l : ls)
+        if (h->upd_wait[l]) {
+            if (cudaStreamWaitEvent(s, h->upd_evt[l], 0) != cudaSuccess) return ISKV_ERR_CUDA;
+            h->upd_wait[l] = 0;
+        }
+    return ISKV_OK;
+}
+
+int order_after_update(iskv_cache* h, int layer, cudaStream_t s) {
+    return order_after_updates(h, std::vector<int>{layer}, s);
+}
+
 bool layers_of(const iskv_cache* h, int layer, std::vector<int>* out) {
     out->clear();
     if (layer == ISKV_ALL_LAYERS) {
@@ -262,11 +294,18 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     h->T.assign(c.layers, 0);
     h->n_c.assign(c.layers, 0);
     h->n_pend.assign(c.layers, 0);
+    h->upd_wait.assign(c.layers, 0);
+    h->upd_evt.assign(c.layers, nullptr);
 
     const size_t heads = (size_t)c.layers * h->BH;
     const size_t d = kHeadDim;
     size_t ring_bytes = heads * h->cap * d * h->kv_bytes;
     rc = ISKV_OK;
+    for (int l = 0; l < c.layers && rc == ISKV_OK; ++l)
+        if (cudaEventCreateWithFlags(&h->upd_evt[l], cudaEventDisableTiming) != cudaSuccess)
+            rc = ISKV_ERR_CUDA;
+    if (rc == ISKV_OK && cudaEventCreateWithFlags(&h->enq_evt, cudaEventDisableTiming) != cudaSuccess)
+        rc = ISKV_ERR_CUDA;
     rc = rc ? rc : dalloc(&h->ring_k, ring_bytes);
     rc = rc ? rc : dalloc(&h->ring_v, ring_bytes);
     const size_t prot_bytes = heads * h->pcap * d * h->kv_bytes;
@@ -350,6 +389,10 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
     if (!h || !k || !v || t < 0 || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
     const int64_t T1 = h->T[layer] + t;
     const int64_t P = h->cfg.protect;
+    {
+        const int rc = order_after_update(h, layer, reinterpret_cast<cudaStream_t>(stream));
+        if (rc != ISKV_OK) return rc;
+    }
     const int64_t tf1 = T1 > P ? T1 - P : 0;   // factor-stream rows after the call
     if (T1 > h->cfg.max_tokens || tf1 - h->n_c[layer] > h->cap) return ISKV_ERR_CAPACITY;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -402,12 +445,13 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
     return ISKV_OK;
 }
 
-int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
-    if (!h || (flags & ~ISKV_FOLD_DEFER_SYNC)) return ISKV_ERR_INVALID_ARG;
-    std::vector<int> ls;
-    if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
+namespace {
+
+// Fold (and rewrite) the ready blocks of the listed layers on stream s; the
+// layers that were folded go to *folded.
+int compress_on(iskv_cache* h, const std::vector<int>& ls, int flags, cudaStream_t s,
+                std::vector<int>* folded) {
     const bool want_defer = (flags & ISKV_FOLD_DEFER_SYNC) != 0;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     FoldLaunch fl{};
     fl.max_sweeps = h->cfg.jacobi_max_sweeps;
     std::vector<int> fold_layers;
@@ -454,13 +498,48 @@ int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
             rl_rows.push_back((int)old);
         }
     }
+    *folded = fold_layers;
     return run_resync(h, rl_layers, rl_seg, rl_rows, s);
+}
+
+}  // namespace
+
+int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
+    if (!h || (flags & ~ISKV_FOLD_DEFER_SYNC)) return ISKV_ERR_INVALID_ARG;
+    std::vector<int> ls, folded;
+    if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int rc = order_after_updates(h, ls, s);
+    return rc != ISKV_OK ? rc : compress_on(h, ls, flags, s, &folded);
+}
+
+int iskv_compress_block_async(iskv_t h, int layer, int flags, void* stream, void* after) {
+    if (!h || (flags & ~ISKV_FOLD_DEFER_SYNC)) return ISKV_ERR_INVALID_ARG;
+    std::vector<int> ls, folded;
+    if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the update sees everything enqueued so far on `after` (the appended rows)
+    // and runs after the layers' earlier updates
+    CU(cudaEventRecord(h->enq_evt, reinterpret_cast<cudaStream_t>(after)));
+    CU(cudaStreamWaitEvent(s, h->enq_evt, 0));
+    int rc = order_after_updates(h, ls, s);
+    if (rc == ISKV_OK) rc = compress_on(h, ls, flags, s, &folded);
+    if (rc != ISKV_OK) return rc;
+    for (int l : folded) {
+        CU(cudaEventRecord(h->upd_evt[l], s));
+        h->upd_wait[l] = 1;
+    }
+    return ISKV_OK;
 }
 
 int iskv_sync(iskv_t h, int layer, void* stream) {
     if (!h) return ISKV_ERR_INVALID_ARG;
     std::vector<int> ls;
     if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
+    {
+        const int rc = order_after_updates(h, ls, reinterpret_cast<cudaStream_t>(stream));
+        if (rc != ISKV_OK) return rc;
+    }
     std::vector<int> rl_layers, rl_seg, rl_rows;
     for (int l : ls) {
         if (h->n_pend[l] == 0) continue;
@@ -520,6 +599,10 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     if (h->T[layer] == 0 || h->n_pend[layer] > 0) return ISKV_ERR_STATE;
     const iskv_config& c = h->cfg;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    {
+        const int rc = order_after_update(h, layer, s);
+        if (rc != ISKV_OK) return rc;
+    }
     const size_t q_bytes = (size_t)c.batch * c.q_heads * kHeadDim * h->kv_bytes;
     const size_t o_bytes = (size_t)c.batch * c.q_heads * kHeadDim * sizeof(float);
     const void* qd = q;
@@ -642,6 +725,10 @@ int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* stream) {
         return ISKV_ERR_INVALID_ARG;
     if (h->n_pend[layer] > 0) return ISKV_ERR_STATE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    {
+        const int rc = order_after_update(h, layer, s);
+        if (rc != ISKV_OK) return rc;
+    }
     const FactorView f = view(h, which);
     const int64_t rows = h->n_c[layer];
     if (rows == 0) return ISKV_OK;   // nothing folded: an empty result
@@ -668,6 +755,10 @@ int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
     if (!h || layer < 0 || layer >= h->cfg.layers || (which != ISKV_WHICH_K && which != ISKV_WHICH_V))
         return ISKV_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    {
+        const int rc = order_after_update(h, layer, s);
+        if (rc != ISKV_OK) return rc;
+    }
     const FactorView f = view(h, which);
     const size_t heads = h->BH;
     const int r = f.r;
