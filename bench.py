@@ -231,6 +231,11 @@ def run_iskv(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if args.async_update:
+        # decode on a high-priority stream, block updates on a low-priority one:
+        # the block scheduler then places pending decode CTAs first
+        low, high = torch.cuda.Stream.priority_range()
+        torch.cuda.set_stream(torch.cuda.Stream(device=dev, priority=high))
     wl = WORKLOADS[args.workload]
     L, Bsz, H, Hq = wl["layers"], wl["batch"], wl["kv_heads"], wl["q_heads"]
     g = Hq // H
@@ -284,7 +289,8 @@ def run_iskv(args, rank, world, local_rank):
     step_ctr = [0]
     dec_events = []
     step_events = []
-    side = torch.cuda.Stream(device=dev) if args.async_update else None
+    side = (torch.cuda.Stream(device=dev, priority=torch.cuda.Stream.priority_range()[0])
+            if args.async_update else None)
     # asynchronous updates: layer l folds at step slot[l] of every 64-step
     # period, on the side stream, right after its decode (its block is ready
     # by then, or one period later; the ring holds up to 64 extra rows)
