@@ -654,18 +654,36 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.n_c = a.n_c;
         t.T = a.T;
         t.scale = a.scale;
+        // exact-row tiles of 64 rows, or of 32 when 64 rows of K and V would make
+        // a stage larger than a folded tile's C_K and C_V
+        const int64_t coef_tile = (int64_t)128 * (c.rank_k + c.rank_v) * 2;
+        t.win_rows = 2 * 64 * kHeadDim * 2 > coef_tile ? 32 : 64;
+        // deepest pipeline that fits: stages first, then two basis buffers, then
+        // double-buffered q'
+        t.stages = 0;
+        for (int ns = 6; ns >= 2 && t.stages == 0; --ns)
+            for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
+                for (int nqb = 2; nqb >= 1; --nqb)
+                    if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk, nqb, t.win_rows) <= 227 * 1024) {
+                        t.stages = ns;
+                        t.basis_bufs = nbk;
+                        t.q_bufs = nqb;
+                        break;
+                    }
+        if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
+        const int wt = t.win_rows;
         const int64_t P = c.protect, Pe = std::min<int64_t>(a.T, P);
         t.tiles_c = (int)((a.n_c + 127) / 128);
-        t.tiles_w = (int)((factor_rows(h, layer) - a.n_c + 63) / 64);
-        t.tiles_per_head = t.tiles_c + t.tiles_w + (int)((Pe + 63) / 64);
+        t.tiles_w = (int)((factor_rows(h, layer) - a.n_c + wt - 1) / wt);
+        t.tiles_per_head = t.tiles_c + t.tiles_w + (int)((Pe + wt - 1) / wt);
         t.total_tiles = (int64_t)h->BH * t.tiles_per_head;
         // each CTA publishes two partials (one per epilogue group) for every head
         // it visits; fewer CTAs when a head would span more slots than the
         // partial buffer holds (few heads, long context)
         int ncta = (int)std::min<int64_t>(std::min(sms, kDecodeMaxCtas), t.total_tiles);
         // partial slots per query head: the buffer's, and the merge scratch's
-        // (slots x g <= 1024)
-        const int cap_slots = std::min(h->max_splits, 1024 / a.g);
+        // (slots x g <= 512 per q' buffer of a group)
+        const int cap_slots = std::min(h->max_splits, 512 * t.q_bufs / a.g);
         int slots_c = 0;
         for (;;) {
             t.ncta = partition_decode_tiles(t.total_tiles, t.tiles_per_head, ncta, t.cta_start);
@@ -684,18 +702,6 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         if (2 * slots_c > cap_slots) return ISKV_ERR_UNSUPPORTED;
         t.slots_c = slots_c;
         t.splits_total = 2 * slots_c;
-        // deepest pipeline that fits: stages first, then two basis buffers, then
-        // double-buffered q'
-        t.stages = 0;
-        for (int ns = 4; ns >= 2 && t.stages == 0; --ns)
-            for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
-                for (int nqb = 2; nqb >= 1; --nqb)
-                    if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk, nqb) <= 227 * 1024) {
-                        t.stages = ns;
-                        t.basis_bufs = nbk;
-                        t.q_bufs = nqb;
-                        break;
-                    }
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
         CU(launch_decode_tc(t, s));   // merges the partials of each head itself
         if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));

@@ -137,7 +137,8 @@ struct DecodeTcArgs {
     int64_t cta_start[kDecodeMaxCtas + 1];
     int slots_c;                 // compressed partial slots per query head
     int splits_total;
-    int stages;                  // shared-memory pipeline depth (2..4)
+    int stages;                  // shared-memory pipeline depth (2..6)
+    int win_rows;                // rows of an exact-row tile: 64, or 32 when 64 would enlarge a stage
     int basis_bufs;              // bf16 basis buffers (1 or 2 heads in flight)
     int q_bufs;                  // q' buffers per epilogue group (1 or 2)
     float scale;
@@ -163,7 +164,7 @@ cudaError_t launch_resync_tc(const FactorView& f, const ResyncLaunch& rl, int* s
                              cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
 bool decode_tc_supports_group(int g);
-size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb);
+size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb, int wt);
 
 size_t fold_smem_bytes(int r);
 int fold_q_cols(int r);   // k = min(64, d - r): columns of Q

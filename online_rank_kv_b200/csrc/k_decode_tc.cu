@@ -58,7 +58,8 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;
-constexpr int kWinTile = 64;     // exact-row tiles: 64 rows never wrap the ring
+// exact-row tiles have 64 or 32 rows (the host's choice, win_rows): either
+// divides the ring and the protected-row capacity, so a tile never wraps
 constexpr int kThreads = 384;
 constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
 constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
@@ -68,7 +69,7 @@ constexpr int kCsCol = 2 * kBufCols;   // per-row RoPE table: cos 64 | sin 64 | 
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Bars {
-    uint64_t full[4], empty[4];
+    uint64_t full[6], empty[6];
     uint64_t bk_full[2], bk_empty[4];      // bk_empty[buffer * 2 + group]
     uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
     uint64_t krot_ready[2], krot_b[2], p_ready[2];   // epilogue -> group issuer: K_rot halves, P written
@@ -85,16 +86,18 @@ struct SmemPlan {
     uint32_t bk, stage, stage_k, stage_bytes, qb, pb, total;
 };
 
-__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, int nqb) {
+constexpr int kQWords = kQN * 64;   // one q' buffer: kQN rows of 128 fp16 (64 words)
+
+__host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, int nqb, int wt) {
     SmemPlan p;
     uint32_t off = 1024;                                        // barriers, scratch
     p.bk = off;                off += nbk * bk_stride(rK);        // nbk heads x (hi, lo, queries)
     p.stage_k = (uint32_t)kTile * rK * 2;
     uint32_t sb = p.stage_k + kTile * rV * 2;
-    if (sb < 2 * kWinTile * kHeadDim * 2) sb = 2 * kWinTile * kHeadDim * 2;   // exact K and V rows
+    if (sb < 2 * wt * kHeadDim * 2) sb = 2 * wt * kHeadDim * 2;   // exact K and V rows
     p.stage_bytes = sb + 1024;
     p.stage = off;             off += ns * p.stage_bytes;
-    p.qb = off;                off += 2 * nqb * (kQN * kTile * 4);   // [group][nqb] q' buffers
+    p.qb = off;                off += 2 * nqb * (kQWords * 4);   // [group][nqb] q' buffers
     p.pb = off;                off += 2 * (kPN * kTile * 2);
     p.total = off;
     return p;
@@ -156,6 +159,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     const int ntiles = (int)(f1 - f0);
     const int tph = a.tiles_per_head;
     const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs, nqb = a.q_bufs;
+    const int wt = a.win_rows;      // rows of an exact-row tile (64 or 32)
     constexpr int g = G;
     constexpr int kQItems = (G * 64 + 127) / 128;   // q' items per epilogue thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -171,14 +175,14 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2 groups]
     static_assert(sizeof(Bars) + 24 <= 512, "scratch words fit below the reduction area");
     float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
-    const SmemPlan P = plan_smem(rK, rV, ns, nbk, nqb);
+    const SmemPlan P = plan_smem(rK, rV, ns, nbk, nqb, wt);
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
     uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
     const uint32_t stage_bytes = P.stage_bytes;
     const int tiles_c = a.tiles_c, tiles_cw = a.tiles_c + a.tiles_w;
-    constexpr uint32_t kWinBytes = kWinTile * kHeadDim * 2;   // one of K, V
+    const uint32_t win_bytes = (uint32_t)wt * kHeadDim * 2;   // one of K, V
     const uint32_t bk_bytes = 2 * kTile * rK * 2;   // B_hi, B_lo of one head
     const uint32_t bks = bk_stride(rK);
     const uint32_t q_bytes = (uint32_t)g * d * 2;    // the head's queries, bf16
@@ -188,7 +192,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 6; ++i) {
             mbar_init(&bars->full[i], 1);
             mbar_init(&bars->empty[i], 1);
         }
@@ -211,7 +215,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     for (int e = tid; e < 2 * nqb * kQN * 64; e += kThreads) {
         const int buf = e / (kQN * 64), w = e % (kQN * 64);
         const int n = w / 64, u = w % 64;
-        if (n >= 2 * g) qb[buf * kQN * kTile + qb_off(n, u)] = 0u;
+        if (n >= 2 * g) qb[buf * kQWords + qb_off(n, u)] = 0u;
     }
     for (int e = tid; e < 2 * kPN * kTile; e += kThreads) {
         const int buf = e / (kPN * kTile), w = e % (kPN * kTile);
@@ -274,19 +278,19 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     if (tile < tiles_cw) {
                         // window rows at factor positions j0..j0+63 sit in ring slots
                         // j0 % cap.. (no wrap: cap % 64 == 0)
-                        const int64_t j0 = a.n_c + (int64_t)(tile - tiles_c) * kWinTile;
+                        const int64_t j0 = a.n_c + (int64_t)(tile - tiles_c) * wt;
                         const int64_t slot0 = j0 % a.K.cap;
                         rk = reinterpret_cast<const __nv_bfloat16*>(a.K.ring) + (hidx * a.K.cap + slot0) * d;
                         rv = reinterpret_cast<const __nv_bfloat16*>(a.V.ring) + (hidx * a.V.cap + slot0) * d;
                     } else {
                         // protected rows j0..j0+63 (positions below P)
-                        const int64_t j0 = (int64_t)(tile - tiles_cw) * kWinTile;
+                        const int64_t j0 = (int64_t)(tile - tiles_cw) * wt;
                         rk = reinterpret_cast<const __nv_bfloat16*>(a.K.prot) + (hidx * a.K.pcap + j0) * d;
                         rv = reinterpret_cast<const __nv_bfloat16*>(a.V.prot) + (hidx * a.V.pcap + j0) * d;
                     }
-                    mbar_arrive_expect_tx(&bars->full[st], 2 * kWinBytes);
-                    bulk_g2s(sk, rk, kWinBytes, &bars->full[st]);
-                    bulk_g2s(sk + kWinBytes, rv, kWinBytes, &bars->full[st]);
+                    mbar_arrive_expect_tx(&bars->full[st], 2 * win_bytes);
+                    bulk_g2s(sk, rk, win_bytes, &bars->full[st]);
+                    bulk_g2s(sk + win_bytes, rv, win_bytes, &bars->full[st]);
                 }
                 issued = n + 1;
             }
@@ -349,7 +353,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
         float* gred = red + grp * 64;             // [max 4 x 8 | l 4 x 8] of this group
         const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
-        uint32_t* qbb = qb + nqb * grp * kQN * kTile;   // the group's first q' buffer (head-end exchange)
+        uint32_t* qbb = qb + nqb * grp * kQWords;   // the group's first q' buffer (head-end exchange)
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
         // q' operand offsets of this thread's items (hi of dims i, i + 64; lo likewise)
         int qoff[kQItems][2];
@@ -408,8 +412,8 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             auto tile_j0 = [&](int nn) {   // positions fit in 32 bits (max_tokens is an int32)
                 const int lc = (int)(f0 + nn - hbase);
                 return lc < tiles_c ? P32 + lc * kTile
-                                    : lc < tiles_cw ? P32 + nc32 + (lc - tiles_c) * kWinTile
-                                                    : (lc - tiles_cw) * kWinTile;
+                                    : lc < tiles_cw ? P32 + nc32 + (lc - tiles_c) * wt
+                                                    : (lc - tiles_cw) * wt;
             };
             // q' = R_{j0}^T q of tile nn as fp16 hi / lo parts (the score MMA's B
             // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
@@ -425,7 +429,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 qx2[k] = n_first < s1 ? __bfloat162float(sq[h * d + i + 64]) : 0.f;
             }
             auto build_q = [&](int nn, float2 rv) {
-                uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQN * kTile;
+                uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQWords;
 #pragma unroll
                 for (int k = 0; k < kQItems; ++k) {
                     if (gt + 128 * k >= G * 64) break;
@@ -451,7 +455,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 const bool win = local >= tiles_c;    // exact rows (64-token tile)
                 const int j0 = tile_j0(n);
                 const int lim = !win ? P32 + nc32 : local < tiles_cw ? T32 : Pe32;
-                const int span = win ? kWinTile : kTile;
+                const int span = win ? wt : kTile;
                 const int valid = (lim - j0) < span ? (lim - j0) : span;
                 // the next tile's query rotation, loaded now, used after this tile's RoPE
                 const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
@@ -658,12 +662,11 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 const float* Pbase = a.partial + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * a.splits_total * stride;
                 const float* br = a.V.basis + (((int64_t)a.layer * BH + head) * d + gt) * rV;
                 for (int c = 0; c < rV; c += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(br + c));
-                // scratch: m, l of every (slot, head) in the group's first q' buffer
-                // (8 KB; the host keeps slots x g <= 1024), the [g][r_V] merged sums
-                // in its P buffer (4 KB); both idle once the head's last score and
-                // value MMAs have completed
+                // scratch: m, l of every (slot, head) in the group's q' buffers
+                // (nqb x 4 KB; the host keeps slots x g <= nqb x 512), the [g][r_V]
+                // merged sums in its P buffer (4 KB); both idle once the head's last
+                // score and value MMAs have completed
                 static_assert(kMaxGroup * 128 * 4 <= kPN * kTile * 2, "merge sums fit the P buffer");
-                static_assert(2 * 1024 * 4 <= kQN * kTile * 4, "slot scratch fits one q' buffer");
                 float* sacc = reinterpret_cast<float*>(pbb);
                 float* sml = reinterpret_cast<float*>(qbb);   // [slot][G] m, then [slot][G] l
                 const int nml = nsl * G;
@@ -754,7 +757,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             const uint32_t sbo_q = (kTile / 8) * 128;
             const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
             const uint32_t kh = tmem + grp * kBufCols;
-            const uint32_t qg = smem_u32(qb + nqb * grp * kQN * kTile);
+            const uint32_t qg = smem_u32(qb + nqb * grp * kQWords);
             const uint32_t p0 = smem_u32(pb + grp * kPN * kTile);
             // K^ of tile n into this group's buffer; exact-row tiles need none
             auto recon = [&](int n, int hb, bool win) -> bool {
@@ -796,7 +799,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     // scores in two halves of the head dimension, each once the epilogue
                     // has rotated it: dims 0..31 and 64..95 (k-steps 0..3, 8..11), then
                     // 32..63 and 96..127 (k-steps 4..7, 12..15)
-                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQN * kTile * 4);
+                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQWords * 4);
                     bool got = true;
                     for (int half = 0; half < 2; ++half) {
                         if (!mbar_wait(half ? &bars->krot_b[grp] : &bars->krot_ready[grp], (n >> 1) & 1,
@@ -840,8 +843,8 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
                     } else {
                         // O = V^T P over 64 exact rows: A = V tile, MN-major, M = d
-                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + kWinBytes);
-                        for (int ks = 0; ks < kWinTile / 16; ++ks)
+                        const uint32_t v0 = smem_u32(stage + st * stage_bytes + win_bytes);
+                        for (int ks = 0; ks < wt / 16; ++ks)
                             mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_ow, ks != 0);
                     }
@@ -872,13 +875,13 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
 
 }  // namespace
 
-size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb) {
-    return plan_smem(rK, rV, ns, nbk, nqb).total;
+size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb, int wt) {
+    return plan_smem(rK, rV, ns, nbk, nqb, wt).total;
 }
 
 template <int G>
 cudaError_t launch_g(const DecodeTcArgs& a, cudaStream_t s) {
-    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages, a.basis_bufs, a.q_bufs);
+    const size_t bytes = decode_tc_smem_bytes(a.K.r, a.V.r, a.stages, a.basis_bufs, a.q_bufs, a.win_rows);
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;
