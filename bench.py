@@ -55,7 +55,7 @@ BLOCK = 64
 # r_V 64), from the ncu launch list in profiles/launches_qwen3-1L-b8-32k.md
 # (the 36-layer run issues the same launch once per layer).  None for
 # workloads without a capture.
-DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.9e6, "qwen3-1L-b8-32k": 433.9e6}
+DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.3e6, "qwen3-1L-b8-32k": 433.3e6}
 
 
 def _peaks():
