@@ -14,6 +14,7 @@
 #include <new>
 #include <vector>
 
+#include "decode_plan.h"
 #include "iskv_internal.cuh"
 #include "tc_util.cuh"
 
@@ -551,49 +552,6 @@ int iskv_sync(iskv_t h, int layer, void* stream) {
     return run_resync(h, rl_layers, rl_seg, rl_rows, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Tile ranges of the persistent decode grid: contiguous runs of the flattened
-// (head, tile) space, at most nmax of them, of equal cost, where a run costs
-// its tiles plus kHeadSwitchTiles for every head it enters after its first
-// (publishing a partial, and restarting the pipeline on the next head's basis
-// and queries).  Smallest feasible cost by bisection, runs filled greedily.
-// Returns the number of runs; start[0..n] holds their bounds.
-static constexpr int64_t kHeadSwitchTiles = 4;
-
-static int fill_decode_runs(int64_t total, int64_t tph, int nmax, int64_t cost, int64_t* start) {
-    int k = 0;
-    int64_t p = 0;
-    while (p < total) {
-        if (k == nmax) return nmax + 1;
-        start[k++] = p;
-        int64_t budget = cost, q = p;
-        for (bool first = true; q < total; first = false) {
-            if (!first) {
-                budget -= kHeadSwitchTiles;
-                if (budget < 1) break;
-            }
-            const int64_t seg_end = std::min((q / tph + 1) * tph, total);
-            const int64_t take = std::min(seg_end - q, budget);
-            q += take;
-            budget -= take;
-            if (q < seg_end) break;
-        }
-        p = q > p ? q : p + 1;
-    }
-    start[k] = total;
-    return k;
-}
-
-static int partition_decode_tiles(int64_t total, int64_t tph, int nmax, int64_t* start) {
-    // hi: one run holds everything
-    int64_t lo = 1, hi = total + kHeadSwitchTiles * ((total + tph - 1) / tph);
-    while (lo < hi) {
-        const int64_t mid = lo + (hi - lo) / 2;
-        if (fill_decode_runs(total, tph, nmax, mid, start) <= nmax) hi = mid;
-        else lo = mid + 1;
-    }
-    return fill_decode_runs(total, tph, nmax, lo, start);
-}
-
 int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* stream) {
     if (!h || !q || !out || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
     if (h->T[layer] == 0 || h->n_pend[layer] > 0) return ISKV_ERR_STATE;
@@ -687,15 +645,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         int slots_c = 0;
         for (;;) {
             t.ncta = partition_decode_tiles(t.total_tiles, t.tiles_per_head, ncta, t.cta_start);
-            slots_c = 1;
-            int c0 = 0;
-            for (int hh = 0; hh < h->BH; ++hh) {
-                const int64_t f_first = (int64_t)hh * t.tiles_per_head, f_last = f_first + t.tiles_per_head - 1;
-                while (t.cta_start[c0 + 1] <= f_first) ++c0;
-                int c1 = c0;
-                while (t.cta_start[c1 + 1] <= f_last) ++c1;
-                slots_c = std::max(slots_c, c1 - c0 + 1);
-            }
+            slots_c = max_runs_per_head(t.cta_start, t.ncta, h->BH, t.tiles_per_head);
             if (2 * slots_c <= cap_slots || ncta == 1) break;
             ncta = std::max(1, ncta * (cap_slots - 2) / (2 * slots_c));
         }
