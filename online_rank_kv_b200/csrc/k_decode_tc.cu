@@ -5,10 +5,12 @@
 // does it mean?" (Jargon: Pre-RoPE keys -- folded keys are rebuilt before
 // RoPE and rotated when read) and the ASKV design report (Design
 // requirements: values are never rebuilt on the decode path).  For query
-// head h of KV head h/g and folded token j < n_c:
-//   k_j = C_K[j] B_K^T,  s_j = q_h . RoPE(k_j, j) / sqrt(d),
+// head h of KV head h/g and folded row j < n_c (position P + j after the P
+// protected positions):
+//   k_j = C_K[j] B_K^T,  s_j = q_h . RoPE(k_j, P + j) / sqrt(d),
 //   partial softmax (m, l) and acc_h = sum_j p_j C_V[j]   (r_V wide);
-// and, for the exact rows j >= n_c (64-token tiles of the window ring),
+// and, for the exact rows (tiles of 64 or 32 tokens: the window ring after
+// the folded rows, and the protected rows before them),
 //   s_j = q_h . RoPE(K_j, j) / sqrt(d) and acc_d = sum_j p_j V_j (d wide),
 // all under one online softmax per head.
 //
@@ -452,7 +454,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             for (int n = n_first; n < s1; n += 2) {
                 const int st = n % ns;
                 const int local = (int)(f0 + n - hbase);
-                const bool win = local >= tiles_c;    // exact rows (64-token tile)
+                const bool win = local >= tiles_c;    // exact rows (a tile of wt tokens)
                 const int j0 = tile_j0(n);
                 const int lim = !win ? P32 + nc32 : local < tiles_cw ? T32 : Pe32;
                 const int span = win ? wt : kTile;
@@ -842,7 +844,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                             mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
                     } else {
-                        // O = V^T P over 64 exact rows: A = V tile, MN-major, M = d
+                        // O = V^T P over wt exact rows: A = V tile, MN-major, M = d
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + win_bytes);
                         for (int ks = 0; ks < wt / 16; ++ks)
                             mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
