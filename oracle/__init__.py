@@ -30,4 +30,5 @@ from .iskv_oracle import (  # noqa: F401
     dense_decode,
     full_kv_bytes,
     persistent_kv_bytes,
+    LatentQuant,
 )

@@ -44,6 +44,7 @@ __all__ = [
     "dense_decode",
     "full_kv_bytes",
     "persistent_kv_bytes",
+    "LatentQuant",
 ]
 
 # ----------------------------------------------------------------------------
@@ -77,9 +78,75 @@ def bf16_round(x):
     return out
 
 
+class LatentQuant:
+    """Low-bit storage of coefficient rows, channel by channel (SVDq page,
+    Abstract: the key cache is moved into SVD latent channels, whose values
+    decay quickly, and the more significant channels get more precision).
+
+    Reading, for iS-KV's coefficients: column j of C is latent channel j, and
+    the factor keeps its columns in descending singular-value order, so
+    significance falls with j.  ``groups`` lists (channels, bits) from the
+    first channel on, bits 2..16; 0 bits drops the channels (stored as zero, the page's
+    compression of negligible channels).  Each row is quantized per group,
+    symmetrically and uniformly: scale = max |x| / (2^(b-1) - 1), code =
+    round-half-even(x / scale) in [-(2^(b-1) - 1), 2^(b-1) - 1]; a group of
+    zeros keeps scale 0.  The pages give no scale rule or bit schedule; this is
+    the plainest per-token choice.  Used as a coefficient storage format
+    (``coef_round``): applied at every write, new rows and every rewrite.
+    Oracle only: the CUDA path does not store this format yet.
+    """
+
+    def __init__(self, groups):
+        self.groups = [(int(n), int(b)) for n, b in groups]
+        if any(n <= 0 or not (b == 0 or 2 <= b <= 16) for n, b in self.groups):
+            raise ValueError("invalid channel groups")
+
+    def _spans(self, r):
+        if sum(n for n, _ in self.groups) != r:
+            raise ValueError("channel groups must cover the rank")
+        lo = 0
+        for n, b in self.groups:
+            yield lo, lo + n, b
+            lo += n
+
+    def quantize(self, C):
+        """Integer codes (same shape as C) and scales (rows x groups)."""
+        C = np.atleast_2d(np.asarray(C, dtype=np.float64))
+        codes = np.zeros(C.shape, dtype=np.int64)
+        scales = np.zeros((C.shape[0], len(self.groups)))
+        for g, (lo, hi, b) in enumerate(self._spans(C.shape[1])):
+            if b == 0:
+                continue
+            qmax = 2 ** (b - 1) - 1
+            amax = np.abs(C[:, lo:hi]).max(axis=1)
+            sc = amax / qmax
+            scales[:, g] = sc
+            safe = np.where(sc > 0, sc, 1.0)[:, None]
+            codes[:, lo:hi] = np.clip(np.round(C[:, lo:hi] / safe), -qmax, qmax).astype(np.int64)
+        return codes, scales
+
+    def dequantize(self, codes, scales):
+        codes = np.atleast_2d(codes)
+        out = np.zeros(codes.shape)
+        for g, (lo, hi, _) in enumerate(self._spans(codes.shape[1])):
+            out[:, lo:hi] = codes[:, lo:hi] * scales[:, g:g + 1]
+        return out
+
+    def __call__(self, C):
+        C = np.asarray(C, dtype=np.float64)
+        return self.dequantize(*self.quantize(C)).reshape(C.shape)
+
+    def bits_per_coefficient(self) -> float:
+        """Average code bits per stored coefficient (scales not counted)."""
+        n = sum(n for n, _ in self.groups)
+        return sum(n * b for n, b in self.groups) / n
+
+
 def _store(x, coef_round):
     if coef_round is None:
         return np.asarray(x, dtype=np.float64)
+    if isinstance(coef_round, LatentQuant):
+        return coef_round(x)
     if coef_round == "bf16":
         return bf16_round(x)
     if coef_round == "f32":

@@ -448,6 +448,90 @@ def test_persistent_bytes_count_the_kept_arrays():
 
 
 # ----------------------------------------------------------------------------
+# low-bit coefficients in latent channels (oracle only)
+# ----------------------------------------------------------------------------
+
+
+def test_latent_quant_is_the_nearest_grid_point():
+    """Per row and channel group the stored value is the nearest point of the
+    symmetric uniform grid {k * scale : |k| <= 2^(b-1) - 1}, found here by
+    brute force over every level; dropped groups are zero."""
+    g = _rng(70)
+    C = g.standard_normal((40, 32)) * (2.0 ** -np.arange(32) * 8 + 0.1)
+    C[3] = 0.0
+    q = O.LatentQuant([(4, 8), (12, 4), (8, 2), (8, 0)])
+    got = q(C)
+    codes, scales = q.quantize(C)
+    spans = [(0, 4, 8), (4, 16, 4), (16, 24, 2), (24, 32, 0)]
+    for gi, (lo, hi, b) in enumerate(spans):
+        for i in range(C.shape[0]):
+            if b == 0:
+                assert np.all(got[i, lo:hi] == 0)
+                continue
+            qmax = 2 ** (b - 1) - 1
+            sc = np.abs(C[i, lo:hi]).max() / qmax
+            assert scales[i, gi] == sc
+            if sc == 0:
+                assert np.all(got[i, lo:hi] == 0)
+                continue
+            levels = np.arange(-qmax, qmax + 1) * sc
+            for j in range(lo, hi):
+                d = np.abs(levels - C[i, j])
+                best = levels[np.argmin(d)]
+                assert abs(got[i, j] - C[i, j]) <= d.min() + 1e-15
+                assert abs(got[i, j] - best) <= 1e-15 or np.isclose(d[np.argsort(d)[:2]], d.min()).all()
+                assert abs(codes[i, j]) <= qmax
+    assert q.bits_per_coefficient() == (4 * 8 + 12 * 4 + 8 * 2) / 32
+
+
+def test_latent_quant_grid_values_round_trip_and_high_bits_converge():
+    q16 = O.LatentQuant([(16, 16)])
+    g = _rng(71)
+    C = g.standard_normal((20, 16))
+    codes, scales = q16.quantize(C)
+    np.testing.assert_array_equal(q16(q16(C)), q16(C))    # grid values are fixed points
+    assert np.max(np.abs(q16(C) - C)) <= np.max(scales) / 2 + 1e-15
+    assert np.max(np.abs(q16(C) - C)) / np.abs(C).max() < 2 ** -14
+
+
+def test_latent_channels_quantize_better_than_original_space():
+    """The premise the SVDq page states: when the latent channels' values decay
+    quickly, quantizing the coefficients with more bits for the leading
+    channels loses far less than quantizing the original 128 channels (per
+    token or per channel) with the same average bits."""
+    d, r, n = 128, 32, 512
+    g = _rng(72)
+    G, _ = np.linalg.qr(g.standard_normal((d, d)))
+    K = (g.standard_normal((n, d)) * (0.75 ** np.arange(d)) * 10) @ G.T
+    _, _, Vt = np.linalg.svd(K, full_matrices=False)
+    B = Vt[:r].T
+    C = K @ B
+    lat = O.LatentQuant([(8, 8), (8, 4), (16, 2)])        # 4 bits per coefficient
+    err_lat = np.linalg.norm(lat(C) @ B.T - C @ B.T)
+    per_token = O.LatentQuant([(d, 4)])(K)
+    per_channel = O.LatentQuant([(n, 4)])(K.T).T
+    err_orig = min(np.linalg.norm(per_token @ B @ B.T - C @ B.T),
+                   np.linalg.norm(per_channel @ B @ B.T - C @ B.T))
+    assert lat.bits_per_coefficient() == 4.0
+    assert err_lat < 0.3 * err_orig, (err_lat, err_orig)
+
+
+def test_factor_with_latent_quant_storage_tracks_the_exact_factor():
+    """Applied at every write (new rows and rewrites), a 12-bit-or-more schedule
+    keeps the reconstruction near the unquantized factor's."""
+    d, r, W = 128, 16, 128
+    rows = _low_rank_rows(900, d, 10, seed=73, noise=1e-3)
+    exact = O.HeadFactor(d, r, W)
+    quant = O.HeadFactor(d, r, W, coef_round=O.LatentQuant([(8, 16), (8, 12)]))
+    for f in (exact, quant):
+        f.append(rows)
+        while f.ready() >= 1:
+            f.fold()
+    ref = exact.reconstruct()
+    assert np.abs(quant.reconstruct() - ref).max() / np.abs(ref).max() < 1e-3
+
+
+# ----------------------------------------------------------------------------
 # mutation tests: plant mistakes in a copy of the fold, check the pins fail
 # ----------------------------------------------------------------------------
 
@@ -510,6 +594,6 @@ def test_residual_sign_is_absorbed_by_rule_q():
 
 def test_oracle_exports():
     for name in ("bf16_round", "ready_blocks", "rope_rotate", "fold_block", "HeadFactor",
-                 "dense_decode", "full_kv_bytes", "persistent_kv_bytes"):
+                 "dense_decode", "full_kv_bytes", "persistent_kv_bytes", "LatentQuant"):
         assert hasattr(oracle, name)
     _ = itertools
