@@ -67,6 +67,7 @@ struct iskv_cache {
     std::vector<cudaEvent_t> upd_evt;
     std::vector<char> upd_wait;
     cudaEvent_t enq_evt = nullptr;   // orders an update's stream after the caller's
+    DecodeGridPlan grid_plan;        // the last decode grid, reused while its shape holds
 };
 
 namespace {
@@ -638,18 +639,15 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         // each CTA publishes two partials (one per epilogue group) for every head
         // it visits; fewer CTAs when a head would span more slots than the
         // partial buffer holds (few heads, long context)
-        int ncta = (int)std::min<int64_t>(std::min(sms, kDecodeMaxCtas), t.total_tiles);
+        const int ncta = (int)std::min<int64_t>(std::min(sms, kDecodeMaxCtas), t.total_tiles);
         // partial slots per query head: the buffer's, and the merge scratch's
         // (slots x g <= 512 per q' buffer of a group)
         const int cap_slots = std::min(h->max_splits, 512 * t.q_bufs / a.g);
-        int slots_c = 0;
-        for (;;) {
-            t.ncta = partition_decode_tiles(t.total_tiles, t.tiles_per_head, ncta, t.cta_start);
-            slots_c = max_runs_per_head(t.cta_start, t.ncta, h->BH, t.tiles_per_head);
-            if (2 * slots_c <= cap_slots || ncta == 1) break;
-            ncta = std::max(1, ncta * (cap_slots - 2) / (2 * slots_c));
-        }
-        if (2 * slots_c > cap_slots) return ISKV_ERR_UNSUPPORTED;
+        if (!plan_decode_grid(t.total_tiles, t.tiles_per_head, h->BH, ncta, cap_slots, &h->grid_plan))
+            return ISKV_ERR_UNSUPPORTED;
+        t.ncta = h->grid_plan.nruns;
+        std::copy(h->grid_plan.start.begin(), h->grid_plan.start.begin() + t.ncta + 1, t.cta_start);
+        const int slots_c = h->grid_plan.slots;
         t.slots_c = slots_c;
         t.splits_total = 2 * slots_c;
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;

@@ -42,6 +42,15 @@ int main() {
         for (int i = 0; i <= n; ++i) std::printf(" %lld", (long long)st[i]);
         std::printf("\n");
     }
+    // the memoized grid plan: a head cap forces fewer runs; same inputs reuse
+    DecodeGridPlan p;
+    const bool ok1 = plan_decode_grid(4000, 4000, 1, 148, 20, &p);
+    const int n1 = p.nruns, s1 = p.slots;
+    const int64_t* before = p.start.data();
+    const bool ok2 = plan_decode_grid(4000, 4000, 1, 148, 20, &p);
+    const bool same = p.start.data() == before && p.nruns == n1;
+    const bool ok3 = plan_decode_grid(64 * 280, 280, 64, 148, 256, &p);
+    std::printf("memo %d %d %d %d %d %d %d\n", ok1, n1, s1, ok2, same, ok3, p.nruns);
 }
 """
 
@@ -76,7 +85,18 @@ def driver():
 def _run(exe, shapes):
     inp = "".join(f"{t} {h} {n}\n" for t, h, n in shapes)
     out = subprocess.run([exe], input=inp, capture_output=True, text=True, check=True).stdout
-    return [list(map(int, line.split())) for line in out.strip().splitlines()]
+    return [list(map(int, line.split())) for line in out.strip().splitlines()
+            if not line.startswith("memo")]
+
+
+def test_grid_plan_caps_slots_and_is_reused(driver):
+    out = subprocess.run([driver], input="", capture_output=True, text=True, check=True).stdout
+    memo = [line for line in out.splitlines() if line.startswith("memo")][0].split()[1:]
+    ok1, n1, s1, ok2, same, ok3, n3 = map(int, memo)
+    # one head of 4000 tiles, at most 20 slots: at most 10 runs share it
+    assert ok1 == 1 and 2 * s1 <= 20 and n1 == s1 <= 10
+    assert ok2 == 1 and same == 1          # same inputs: the stored plan, untouched
+    assert ok3 == 1 and n3 == 148          # new inputs: planned afresh
 
 
 def test_runs_cover_every_tile_within_the_bound(driver):
