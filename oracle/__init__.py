@@ -31,4 +31,5 @@ from .iskv_oracle import (  # noqa: F401
     full_kv_bytes,
     persistent_kv_bytes,
     LatentQuant,
+    joint_head_decode,
 )

@@ -45,6 +45,7 @@ __all__ = [
     "full_kv_bytes",
     "persistent_kv_bytes",
     "LatentQuant",
+    "joint_head_decode",
 ]
 
 # ----------------------------------------------------------------------------
@@ -464,6 +465,24 @@ def dense_decode(q, K_pre, V, theta: float, use_rope: bool = True) -> np.ndarray
     p = np.exp(s)
     p = p / p.sum(axis=1, keepdims=True)
     return p @ V
+
+
+def joint_head_decode(q, K_full, V_full, kv_heads: int, theta: float, use_rope: bool = True):
+    """Decode with one factor per layer over all KV heads (the joint-head
+    reading of the explainer's ranks 64/96/128, worked-example table): the
+    factor's rows are the KV heads' rows side by side (T x kv_heads*d), so a
+    HeadFactor of dimension kv_heads*d is the joint factor; query head h
+    attends over columns [k d, (k+1) d) of the joint rows, k = h // g.
+    ``q`` is (q_heads x d).  Oracle only: the CUDA path factors per head."""
+    q = np.atleast_2d(np.asarray(q, dtype=np.float64))
+    Hq, d = q.shape
+    g = Hq // kv_heads
+    out = np.zeros((Hq, d))
+    for h in range(Hq):
+        k = h // g
+        out[h] = dense_decode(q[h:h + 1], K_full[:, k * d:(k + 1) * d], V_full[:, k * d:(k + 1) * d],
+                              theta, use_rope)[0]
+    return out
 
 
 # ----------------------------------------------------------------------------

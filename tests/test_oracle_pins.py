@@ -532,6 +532,64 @@ def test_factor_with_latent_quant_storage_tracks_the_exact_factor():
 
 
 # ----------------------------------------------------------------------------
+# joint-head factor (one factor over all KV heads of a layer; oracle only)
+# ----------------------------------------------------------------------------
+
+
+def test_joint_head_factor_lossless_decode_equals_per_head_attention():
+    """At r = kv_heads*d the joint factor reproduces every row, so its decode
+    is dense attention of each query head over its own KV head's raw rows
+    (brute-force loops over heads and tokens)."""
+    H, d, g, W = 2, 16, 2, 64
+    gen = _rng(80)
+    T = 64 * 6 + 9
+    K = gen.standard_normal((T, H * d))
+    V = gen.standard_normal((T, H * d))
+    fk = O.HeadFactor(H * d, H * d, W)
+    fv = O.HeadFactor(H * d, H * d, W)
+    fk.append(K)
+    fv.append(V)
+    while fk.ready() >= 1:
+        fk.fold()
+        fv.fold()
+    assert fk.n_c > 0
+    q = gen.standard_normal((H * g, d))
+    got = O.joint_head_decode(q, fk.full(), fv.full(), H, 1e4)
+    for h in range(H * g):
+        k = h // g
+        Kr = O.rope_rotate(K[:, k * d:(k + 1) * d], np.arange(T), 1e4)
+        s = np.array([q[h] @ Kr[t] for t in range(T)]) / np.sqrt(d)
+        p = np.exp(s - s.max())
+        p /= p.sum()
+        want = sum(p[t] * V[t, k * d:(k + 1) * d] for t in range(T))
+        np.testing.assert_allclose(got[h], want, atol=1e-10)
+
+
+def test_joint_factor_uses_directions_shared_by_heads():
+    """Heads whose keys share a 12-dim subspace: one joint factor of rank 12
+    is exact (rank <= r), while per-head factors of rank 6 each (the same 12
+    coefficients per token) are not."""
+    H, d, W = 2, 32, 64
+    gen = _rng(81)
+    G, _ = np.linalg.qr(gen.standard_normal((H * d, 12)))
+    Z = gen.standard_normal((64 * 8, 12))
+    X = Z @ G.T
+    joint = O.HeadFactor(H * d, 12, W)
+    joint.append(X)
+    heads = [O.HeadFactor(d, 6, W) for _ in range(H)]
+    for k, f in enumerate(heads):
+        f.append(X[:, k * d:(k + 1) * d])
+    for f in [joint] + heads:
+        while f.ready() >= 1:
+            f.fold()
+    n = joint.n_c
+    err_joint = np.abs(joint.reconstruct() - X[:n]).max()
+    err_heads = max(np.abs(f.reconstruct() - X[:n, k * d:(k + 1) * d]).max() for k, f in enumerate(heads))
+    assert err_joint < 1e-10 * np.abs(X).max()
+    assert err_heads > 1e-3 * np.abs(X).max()
+
+
+# ----------------------------------------------------------------------------
 # mutation tests: plant mistakes in a copy of the fold, check the pins fail
 # ----------------------------------------------------------------------------
 
