@@ -87,3 +87,19 @@ def test_reference_arm_line():
     assert line["impl"] == "reference"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+
+
+def test_clock_samples_parse_reasons_and_median():
+    import bench
+    lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n",
+        "0, 1950, 1965, 980.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "0, 1965, 1965, 990.0, 0x0000000000000008, Active, Not Active, Not Active, Not Active\n",
+        "garbage line\n",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active\n",
+    ]
+    got = bench.parse_clock_samples(lines)
+    assert got == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
+                   "reasons": ["hw_slowdown", "sw_power_cap"], "samples": 3}
+    assert bench.parse_clock_samples([]) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                                             "samples": 0}
