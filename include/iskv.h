@@ -109,9 +109,9 @@ typedef struct {
                                Positions 0..P-1 stay exact, P..P+n_c-1 are
                                folded rows, P+n_c..T-1 the exact window.
                                The iS-KV explainer ("What does it mean?",
-                               the paint-shop section) keeps a set of
-                               protected prompt positions exact beside the
-                               recent window.                               */
+                               the paint-shop section) leaves some prompt
+                               positions uncompressed, besides the recent
+                               window.                                      */
 } iskv_config;
 
 /* Fill `cfg` with the defaults of the one-layer Qwen3-8B-shaped cache
