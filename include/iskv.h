@@ -156,9 +156,10 @@ ISKV_API int iskv_compress_block(iskv_t h, int layer, int flags, void* stream);
  * factors happens at that call, and until the update completes nothing reads
  * the layer.  Host counters (T, n_c) advance at once, as for
  * iskv_compress_block.  All other calls on the cache stay on one stream.
- * This serves the ASKV design report's requirement (Design requirements)
- * that maintenance stay off the decode critical path: with one layer updated
- * per call, its fold and rewrite overlap the other layers' decode.
+ * This answers the ASKV design report (Design requirements, the item on
+ * maintenance and the critical path): decoding should not have to wait for
+ * compression work.  With one layer updated per call, its fold and rewrite
+ * overlap the other layers' decode.
  * Errors: as iskv_compress_block, plus CUDA for event failures.            */
 ISKV_API int iskv_compress_block_async(iskv_t h, int layer, int flags, void* stream,
                                        void* after);
