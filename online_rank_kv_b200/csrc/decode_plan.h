@@ -67,37 +67,39 @@ inline int max_runs_per_head(const int64_t* start, int nruns, int heads, int64_t
 }
 
 // The grid plan of one decode call: at most nmax runs, fewer when a head
-// would span more than cap_slots partial slots (two per run).  Decode calls
+// would span more than cap_slots partial slots (per_run per run: one per
+// epilogue group).  Decode calls
 // repeat the same shape for 32 or more tokens in a row, so the last plan is
 // kept and reused while its inputs are unchanged.
 struct DecodeGridPlan {
     int64_t total = -1, tph = 0;
-    int heads = 0, nmax = 0, cap_slots = 0;
+    int heads = 0, nmax = 0, cap_slots = 0, per_run = 0;
     int nruns = 0, slots = 0;        // slots: the most runs sharing one head
     std::vector<int64_t> start;      // nruns + 1 bounds
 };
 
 // Fills *p (or keeps it when already planned for these inputs).  Returns
-// false when no plan keeps two slots per run within cap_slots.
+// false when no plan keeps per_run slots per run within cap_slots.
 inline bool plan_decode_grid(int64_t total, int64_t tph, int heads, int nmax, int cap_slots,
-                             DecodeGridPlan* p) {
+                             int per_run, DecodeGridPlan* p) {
     if (p->total == total && p->tph == tph && p->heads == heads && p->nmax == nmax &&
-        p->cap_slots == cap_slots)
-        return 2 * p->slots <= cap_slots;
+        p->cap_slots == cap_slots && p->per_run == per_run)
+        return per_run * p->slots <= cap_slots;
     p->total = total;
     p->tph = tph;
     p->heads = heads;
     p->nmax = nmax;
     p->cap_slots = cap_slots;
+    p->per_run = per_run;
     p->start.assign((size_t)nmax + 1, 0);
     int n = nmax;
     for (;;) {
         p->nruns = partition_decode_tiles(total, tph, n, p->start.data());
         p->slots = max_runs_per_head(p->start.data(), p->nruns, heads, tph);
-        if (2 * p->slots <= cap_slots || n == 1) break;
-        n = std::max(1, n * (cap_slots - 2) / (2 * p->slots));
+        if (per_run * p->slots <= cap_slots || n == 1) break;
+        n = std::max(1, n * (cap_slots - per_run) / (per_run * p->slots));
     }
-    return 2 * p->slots <= cap_slots;
+    return per_run * p->slots <= cap_slots;
 }
 
 }  // namespace iskv

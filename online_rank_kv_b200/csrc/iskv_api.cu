@@ -643,7 +643,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         // partial slots per query head: the buffer's, and the merge scratch's
         // (slots x g <= 512 per q' buffer of a group)
         const int cap_slots = std::min(h->max_splits, 512 * t.q_bufs / a.g);
-        if (!plan_decode_grid(t.total_tiles, t.tiles_per_head, h->BH, ncta, cap_slots, &h->grid_plan))
+        if (!plan_decode_grid(t.total_tiles, t.tiles_per_head, h->BH, ncta, cap_slots, 2, &h->grid_plan))
             return ISKV_ERR_UNSUPPORTED;
         t.ncta = h->grid_plan.nruns;
         std::copy(h->grid_plan.start.begin(), h->grid_plan.start.begin() + t.ncta + 1, t.cta_start);

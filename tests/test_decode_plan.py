@@ -44,12 +44,12 @@ int main() {
     }
     // the memoized grid plan: a head cap forces fewer runs; same inputs reuse
     DecodeGridPlan p;
-    const bool ok1 = plan_decode_grid(4000, 4000, 1, 148, 20, &p);
+    const bool ok1 = plan_decode_grid(4000, 4000, 1, 148, 20, 2, &p);
     const int n1 = p.nruns, s1 = p.slots;
     const int64_t* before = p.start.data();
-    const bool ok2 = plan_decode_grid(4000, 4000, 1, 148, 20, &p);
+    const bool ok2 = plan_decode_grid(4000, 4000, 1, 148, 20, 2, &p);
     const bool same = p.start.data() == before && p.nruns == n1;
-    const bool ok3 = plan_decode_grid(64 * 280, 280, 64, 148, 256, &p);
+    const bool ok3 = plan_decode_grid(64 * 280, 280, 64, 148, 256, 2, &p);
     std::printf("memo %d %d %d %d %d %d %d\n", ok1, n1, s1, ok2, same, ok3, p.nruns);
 }
 """
