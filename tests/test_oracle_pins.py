@@ -655,3 +655,67 @@ def test_oracle_exports():
                  "dense_decode", "full_kv_bytes", "persistent_kv_bytes", "LatentQuant"):
         assert hasattr(oracle, name)
     _ = itertools
+
+
+# mutations of the protected-row bookkeeping, the kept-byte formula and the
+# latent quantizer: each planted mistake must fail one of their pins
+
+
+class _FoldFromWrongRow(O.HeadFactor):
+    """Protected-row mistake: the block is taken at n_c instead of P + n_c."""
+
+    def fold(self, defer=False, keep_history=False):
+        res = O.fold_block(self.B, self.S, self.rows[self.n_c:self.n_c + self.b])
+        if self.sync_enabled and self.n_c > 0:
+            self.C[:self.n_c] = self.C[:self.n_c] @ res.W_top
+        self._Cbuf = self._grown(self._Cbuf, self.n_c + self.b)
+        self._Cbuf[self.n_c:self.n_c + self.b] = res.C_new
+        self.B, self.S = res.B_new, res.S_new
+        self.n_c += self.b
+        return res
+
+
+class _ReadyIgnoresProtect(O.HeadFactor):
+    """Protected-row mistake: blocks counted from position 0."""
+
+    def ready(self):
+        return O.ready_blocks(self.T, self.n_c, self.W, self.b)
+
+
+@pytest.mark.parametrize("cls", [_FoldFromWrongRow, _ReadyIgnoresProtect])
+def test_protected_row_pins_catch_planted_mistakes(cls, monkeypatch):
+    monkeypatch.setattr(O, "HeadFactor", cls)
+    with pytest.raises(AssertionError):
+        test_protected_factor_is_the_unprotected_factor_of_the_shifted_stream(37)
+
+
+def test_kept_bytes_pin_catches_a_dropped_term(monkeypatch):
+    real = O.persistent_kv_bytes
+
+    def no_protected(n_c, n_w, d, r_k, r_v, coef_bytes, kv_bytes, basis_bytes=4, n_p=0):
+        return real(n_c, n_w, d, r_k, r_v, coef_bytes, kv_bytes, basis_bytes, 0)
+
+    monkeypatch.setattr(O, "persistent_kv_bytes", no_protected)
+    with pytest.raises(AssertionError):
+        test_persistent_bytes_count_the_kept_arrays()
+
+
+def test_latent_quant_pin_catches_a_wrong_level_count(monkeypatch):
+    def wide(self, C):
+        # mistake: 2^b - 1 levels on each side instead of 2^(b-1) - 1
+        C = np.atleast_2d(np.asarray(C, dtype=np.float64))
+        codes = np.zeros(C.shape, dtype=np.int64)
+        scales = np.zeros((C.shape[0], len(self.groups)))
+        for g, (lo, hi, bits) in enumerate(self._spans(C.shape[1])):
+            if bits == 0:
+                continue
+            qmax = 2 ** bits - 1
+            sc = np.abs(C[:, lo:hi]).max(axis=1) / qmax
+            scales[:, g] = sc
+            safe = np.where(sc > 0, sc, 1.0)[:, None]
+            codes[:, lo:hi] = np.clip(np.round(C[:, lo:hi] / safe), -qmax, qmax)
+        return codes, scales
+
+    monkeypatch.setattr(O.LatentQuant, "quantize", wide)
+    with pytest.raises(AssertionError):
+        test_latent_quant_is_the_nearest_grid_point()
