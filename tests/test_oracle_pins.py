@@ -719,3 +719,17 @@ def test_latent_quant_pin_catches_a_wrong_level_count(monkeypatch):
     monkeypatch.setattr(O.LatentQuant, "quantize", wide)
     with pytest.raises(AssertionError):
         test_latent_quant_is_the_nearest_grid_point()
+
+
+def test_joint_head_pin_catches_a_wrong_head_slice(monkeypatch):
+    real = O.joint_head_decode
+
+    def shifted(q, K_full, V_full, kv_heads, theta, use_rope=True):
+        # mistake: query heads read the next KV head's columns
+        d = np.atleast_2d(q).shape[1]
+        return real(q, np.roll(K_full, -d, axis=1), np.roll(V_full, -d, axis=1), kv_heads, theta,
+                    use_rope)
+
+    monkeypatch.setattr(O, "joint_head_decode", shifted)
+    with pytest.raises(AssertionError):
+        test_joint_head_factor_lossless_decode_equals_per_head_attention()
