@@ -14,6 +14,8 @@
 #include <new>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "decode_plan.h"
 #include "iskv_internal.cuh"
 #include "tc_util.cuh"
@@ -71,6 +73,12 @@ struct iskv_cache {
 };
 
 namespace {
+
+// One NVTX range per API call (a no-op unless a profiler is attached).
+struct TraceRange {
+    explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+};
 
 constexpr size_t kStageBytes = 16u << 20;
 constexpr bool kDecodeTcDefault = true;
@@ -388,6 +396,7 @@ int iskv_destroy(iskv_t h) {
 
 int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* stream,
                 int* ready_blocks) {
+    TraceRange trace_("iskv_append");
     if (!h || !k || !v || t < 0 || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
     const int64_t T1 = h->T[layer] + t;
     const int64_t P = h->cfg.protect;
@@ -507,6 +516,7 @@ int compress_on(iskv_cache* h, const std::vector<int>& ls, int flags, cudaStream
 }  // namespace
 
 int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
+    TraceRange trace_("iskv_compress_block");
     if (!h || (flags & ~ISKV_FOLD_DEFER_SYNC)) return ISKV_ERR_INVALID_ARG;
     std::vector<int> ls, folded;
     if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
@@ -516,6 +526,7 @@ int iskv_compress_block(iskv_t h, int layer, int flags, void* stream) {
 }
 
 int iskv_compress_block_async(iskv_t h, int layer, int flags, void* stream, void* after) {
+    TraceRange trace_("iskv_compress_block_async");
     if (!h || (flags & ~ISKV_FOLD_DEFER_SYNC)) return ISKV_ERR_INVALID_ARG;
     std::vector<int> ls, folded;
     if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
@@ -535,6 +546,7 @@ int iskv_compress_block_async(iskv_t h, int layer, int flags, void* stream, void
 }
 
 int iskv_sync(iskv_t h, int layer, void* stream) {
+    TraceRange trace_("iskv_sync");
     if (!h) return ISKV_ERR_INVALID_ARG;
     std::vector<int> ls;
     if (!layers_of(h, layer, &ls)) return ISKV_ERR_INVALID_ARG;
@@ -554,6 +566,7 @@ int iskv_sync(iskv_t h, int layer, void* stream) {
 }
 
 int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* stream) {
+    TraceRange trace_("iskv_decode_attention");
     if (!h || !q || !out || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
     if (h->T[layer] == 0 || h->n_pend[layer] > 0) return ISKV_ERR_STATE;
     const iskv_config& c = h->cfg;
@@ -674,6 +687,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
 }
 
 int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* stream) {
+    TraceRange trace_("iskv_reconstruct");
     if (!h || layer < 0 || layer >= h->cfg.layers ||
         (which != ISKV_WHICH_K && which != ISKV_WHICH_V))
         return ISKV_ERR_INVALID_ARG;
