@@ -101,3 +101,33 @@ def test_null_handles():
     assert ik.LIB.iskv_get_counts(None, 0, ctypes.byref(T), None) == -1
     assert ik.LIB.iskv_status(None) == -1
     assert ik.LIB.iskv_compress_block(None, 0, 0, None) == -1
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    """The ctypes mirrors of iskv_config and iskv_decode_operands have the C
+    structs' size and field offsets (compiled here with the host compiler)."""
+    import shutil
+    cxx = shutil.which("g++") or shutil.which("c++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    ik = _lib()
+    structs = {"iskv_config": ik._Cfg, "iskv_decode_operands": ik.DecodeOperands}
+    lines = ['#include <cstddef>', '#include <cstdio>', '#include "iskv.h"', "int main() {"]
+    for cname, py in structs.items():
+        lines.append(f'    std::printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'    std::printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines.append("}")
+    src = tmp_path / "layout.cpp"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cxx, "-std=c++17", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
