@@ -220,13 +220,15 @@ ISKV_API const char* iskv_strerror(int code);
  * such as a serving engine that owns and plans all of its device memory
  * (and forbids allocations after start-up), or a latency-critical path that
  * must avoid cudaMalloc's device-wide synchronization.  Such a caller keeps
- * the factors in its own buffers (laid out as the cache keeps them) and
- * passes them here; nothing is allocated and nothing is staged.  The
+ * the factors in its own buffers, row-major as iskv_get_factors returns
+ * them (not the cache's internal 8 x 8 blocked bf16 layout), and passes them
+ * here; nothing is allocated and nothing is staged.  The
  * operands describe a cache without protected rows (iskv_config.protect 0);
  * caches with protected rows decode through iskv_decode_attention.
  *
- * All pointers are device memory, owned by the caller, borrowed for the
- * stream-ordered duration of the call:
+ * All pointers are device memory of the current device (or managed
+ * memory), owned by the caller, borrowed for the stream-ordered duration of
+ * the call:
  *   coef_k, coef_v  [batch*kv_heads][coef_rows][r] in coef_dtype (rows 0..n_c-1
  *                   are read);
  *   basis_k, basis_v [batch*kv_heads][head_dim][r] fp32;
@@ -240,10 +242,12 @@ ISKV_API const char* iskv_strerror(int code);
  * process exits; a call needs batch * q_heads * (2 + rank_v + head_dim)
  * floats per split and is rejected with ISKV_ERR_CAPACITY when even one split
  * does not fit.  The first call on a device looks up that array's device
- * address (cudaGetSymbolAddress); make that first call before any stream
- * capture.  Calls share the array: calls that overlap on the GPU race and
- * must be serialized by the caller.  Errors: INVALID_ARG (null or host
- * pointer, inconsistent sizes), UNSUPPORTED (shape), CAPACITY, CUDA.       */
+ * address (cudaGetSymbolAddress) and keeps it; make that first call before
+ * any stream capture, and do not use this entry point across a
+ * cudaDeviceReset (the array may move).  Calls share the array: calls that
+ * overlap on the GPU race and must be serialized by the caller.
+ * Errors: INVALID_ARG (null or host pointer, memory of another device,
+ * inconsistent sizes), UNSUPPORTED (shape), CAPACITY, CUDA.                */
 typedef struct {
     int32_t batch, kv_heads, q_heads, head_dim, rank_k, rank_v;
     int32_t kv_dtype, coef_dtype;

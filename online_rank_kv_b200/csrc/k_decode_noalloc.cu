@@ -13,7 +13,9 @@
 // library holds it until the process exits.  In host code its name is only a
 // host-side stand-in, so its device address is looked up once per device
 // with cudaGetSymbolAddress (on the first call on that device) and passed to
-// the kernels.  All calls share it: calls whose work overlaps on the GPU
+// the kernels.  That address is kept for the life of the process: after a
+// cudaDeviceReset the library image is loaded again and the array may move,
+// so this entry point must not be used across a cudaDeviceReset.  All calls share it: calls whose work overlaps on the GPU
 // (different streams, or several host threads) race on it and must be
 // serialized by the caller.  Nothing in it has to start at zero: every
 // partial a call reads was written earlier by the same call.
@@ -50,13 +52,17 @@ cudaError_t scratch_for_current_device(float** out) {
     return cudaSuccess;
 }
 
-bool on_device(const void* p) {
+// True for memory the kernels on device `dev` may read directly: device
+// memory of `dev` itself, or managed memory.  Device memory of another GPU is
+// refused (it would fault, or cross NVLink unplanned, if peer access is on).
+bool on_device(const void* p, int dev) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+    if (at.type == cudaMemoryTypeManaged) return true;
+    return at.type == cudaMemoryTypeDevice && at.device == dev;
 }
 
 }  // namespace
@@ -82,19 +88,21 @@ extern "C" int iskv_decode_attention_noalloc(const iskv_decode_operands* o, cons
         return ISKV_ERR_INVALID_ARG;
     if (o->coef_rows < o->n_c || o->ring_rows < 1 || o->ring_rows < o->T - o->n_c)
         return ISKV_ERR_INVALID_ARG;
-    // every operand must already be in device memory: nothing is staged
+    // every operand must already be in the current device's memory: nothing
+    // is staged, and nothing is read across GPUs
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ISKV_ERR_CUDA;
     const void* ptrs[] = {q, out, o->coef_k, o->coef_v, o->basis_k, o->basis_v, o->ring_k,
                           o->ring_v, o->rope};
     for (const void* p : ptrs)
-        if (p && !on_device(p)) return ISKV_ERR_INVALID_ARG;
+        if (p && !on_device(p, dev)) return ISKV_ERR_INVALID_ARG;
 
     // split the token axis as far as the scratch array allows
     const int64_t stride = 2 + o->rank_v + kHeadDim;
     const int64_t per_split = (int64_t)o->batch * o->q_heads * stride;
     const int64_t fit = kScratchFloats / per_split;
     if (fit < 1) return ISKV_ERR_CAPACITY;   // batch * q_heads too large for the scratch
-    int sms = 148, dev = 0;
-    cudaGetDevice(&dev);
+    int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t BH = (int64_t)o->batch * o->kv_heads;
     int64_t splits = (4 * (int64_t)sms + BH - 1) / BH;
