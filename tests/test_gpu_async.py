@@ -110,3 +110,54 @@ def test_async_update_with_postponed_rewrite_then_sync():
     q = synth.query_batch(cfg.batch * cfg.q_heads, D, seed=9, device="cuda",
                           dtype=torch.bfloat16).view(cfg.batch, cfg.q_heads, D)
     assert np.array_equal(a.decode_attention(0, q).cpu().numpy(), b.decode_attention(0, q).cpu().numpy())
+
+
+def test_async_updates_against_the_oracle():
+    """The asynchronous path against the float64 oracle, not only against the
+    synchronous cache: every layer folds on the side stream right after its
+    decode, and the decode outputs and reconstructions of sampled heads stay
+    within the bf16-coefficient tolerance of dense attention over the
+    oracle's factors (which fold at the same points)."""
+    import online_rank_kv_b200 as ik
+    from iskv_testlib import SampledCache, rel_err
+    from oracle import dense_decode
+
+    cfg = ik.Config(batch=2, layers=3, kv_heads=2, q_heads=8, rank_k=32, rank_v=64, window=256,
+                    max_tokens=4096, kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1,
+                    rope_theta=1e6, max_deferred=8, ring_extra=512)
+    sample = [(0, 0, 0), (1, 1, 1), (2, 0, 1), (2, 1, 0)]
+    s = SampledCache(cfg, "qwen3", sample, seed=33)
+    s.prefill(1024, chunk=256, defer_every=0)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    g = cfg.q_heads // cfg.kv_heads
+    worst, n_async, checks = 0.0, 0, 0
+    for step in range(160):
+        s.append(1)
+        q = synth.query_batch(cfg.layers * cfg.batch * cfg.q_heads, cfg.head_dim, seed=900 + step,
+                              dtype=torch.bfloat16).view(cfg.layers, cfg.batch, cfg.q_heads,
+                                                         cfg.head_dim)
+        for l in range(cfg.layers):
+            out = s.cache.decode_attention(l, q[l].contiguous().cuda())
+            if step % 8 == 0:
+                got = out.cpu().numpy()
+                qn = q[l].double().numpy()
+                for (ll, b, h) in sample:
+                    if ll != l:
+                        continue
+                    want = dense_decode(qn[b, h * g:(h + 1) * g], s.ok[(ll, b, h)].full(),
+                                        s.ov[(ll, b, h)].full(), cfg.rope_theta)
+                    worst = max(worst, rel_err(got[b, h * g:(h + 1) * g], want))
+                    checks += 1
+            T, n_c = s.cache.counts(l)
+            if (T - n_c - cfg.window) // 64 >= 1:
+                s.cache.compress_block_async(l, side, after=main)
+                for x in sample:
+                    if x[0] == l:
+                        s.ok[x].fold()
+                        s.ov[x].fold()
+                n_async += 1
+    assert n_async >= 2 * cfg.layers and checks > 0
+    assert worst < 2e-2, worst
+    s.check(tol=2e-2)
+    assert s.cache.status() == 0

@@ -22,7 +22,7 @@ import pytest
 import torch
 
 import synth
-from iskv_testlib import rel_err
+from iskv_testlib import SampledCache, rel_err
 from oracle import HeadFactor, dense_decode
 
 pytestmark = pytest.mark.gpu
@@ -36,109 +36,6 @@ def _one_blas_thread():
     from threadpoolctl import threadpool_limits
     with threadpool_limits(limits=1):
         yield
-
-
-class SampledCache:
-    """A CUDA cache for every head plus oracle factors for a few of them."""
-
-    def __init__(self, cfg, workload, sample, seed, sync=True):
-        import online_rank_kv_b200 as ik
-        self.ik = ik
-        self.cfg = cfg
-        self.cache = ik.Cache(cfg)
-        self.L, self.B, self.H = cfg.layers, cfg.batch, cfg.kv_heads
-        self.g = cfg.q_heads // cfg.kv_heads
-        nh = self.L * self.B * self.H
-        self.ks = synth.KVStream(synth.spec_for(workload, "K"), nh, seed=2 * seed + 1, device="cuda",
-                                 dtype=torch.bfloat16)
-        self.vs = synth.KVStream(synth.spec_for(workload, "V"), nh, seed=2 * seed + 2, device="cuda",
-                                 dtype=torch.bfloat16)
-        self.sample = list(sample)
-        self.ok = {x: HeadFactor(128, cfg.rank_k, cfg.window, coef_round="bf16", sync=sync)
-                   for x in self.sample}
-        self.ov = {x: HeadFactor(128, cfg.rank_v, cfg.window, coef_round="bf16", sync=sync)
-                   for x in self.sample}
-        self.folds = 0
-        self.qseed = 5000 + seed
-
-    def append(self, t):
-        k = self.ks.next(t).view(self.L, self.B, self.H, t, 128)
-        v = self.vs.next(t).view(self.L, self.B, self.H, t, 128)
-        for l in range(self.L):
-            self.cache.append(l, k[l].contiguous(), v[l].contiguous())
-        for (l, b, h) in self.sample:
-            self.ok[(l, b, h)].append(k[l, b, h].double().cpu().numpy())
-            self.ov[(l, b, h)].append(v[l, b, h].double().cpu().numpy())
-
-    def fold_all(self, defer):
-        self.cache.compress_block(self.ik.ALL_LAYERS, defer=defer)
-        for x in self.sample:
-            self.ok[x].fold(defer=defer)
-            self.ov[x].fold(defer=defer)
-
-    def sync_all(self):
-        self.cache.sync(self.ik.ALL_LAYERS)
-        for x in self.sample:
-            self.ok[x].sync()
-            self.ov[x].sync()
-
-    def ready(self):
-        T, n_c = self.cache.counts(0)
-        return (T - n_c - self.cfg.window) // 64
-
-    def prefill(self, tokens, chunk=512, defer_every=64):
-        """Append in chunks; fold every ready block with postponed rewrites,
-        one rewrite per defer_every folds, as the bench prefills."""
-        done = 0
-        while done < tokens:
-            n = min(chunk, tokens - done)
-            self.append(n)
-            done += n
-            while self.ready() >= 1:
-                self.fold_all(defer=defer_every > 0)
-                self.folds += 1
-                if defer_every > 0 and self.folds % defer_every == 0:
-                    self.sync_all()
-        if defer_every > 0:
-            self.sync_all()
-
-    def check(self):
-        ik = self.ik
-        for l in sorted({x[0] for x in self.sample}):
-            T, n_c = self.cache.counts(l)
-            for x in self.sample:
-                if x[0] == l:
-                    assert (T, n_c) == (self.ok[x].T, self.ok[x].n_c)
-            for which, of in ((ik.WHICH_K, self.ok), (ik.WHICH_V, self.ov)):
-                got = self.cache.reconstruct(l, which)
-                for x in self.sample:
-                    if x[0] == l and of[x].n_c > 0:
-                        e = rel_err(got[x[1], x[2]].cpu().numpy(), of[x].reconstruct())
-                        assert e < TOL, (l, which, x, e)
-                del got
-
-    def decode_check(self, q=None):
-        """Decode every sampled layer with q (B x Hq x d); compare the sampled
-        heads' outputs with dense attention over the oracle's cache."""
-        c = self.cfg
-        if q is None:
-            q = synth.query_batch(c.batch * c.q_heads, 128, seed=self.qseed,
-                                  dtype=torch.bfloat16).view(c.batch, c.q_heads, 128)
-            self.qseed += 1
-        worst = 0.0
-        for l in sorted({x[0] for x in self.sample}):
-            out = self.cache.decode_attention(l, q.cuda()).cpu().numpy()
-            qn = q.double().numpy()
-            for x in self.sample:
-                if x[0] != l:
-                    continue
-                b, h = x[1], x[2]
-                want = dense_decode(qn[b, h * self.g:(h + 1) * self.g], self.ok[x].full(),
-                                    self.ov[x].full(), c.rope_theta, use_rope=True)
-                e = rel_err(out[b, h * self.g:(h + 1) * self.g], want)
-                worst = max(worst, e)
-        assert worst < TOL, worst
-        return worst
 
 
 def _cfg(**kw):

@@ -1,0 +1,94 @@
+"""The decode-loop regime at length: hundreds of per-fold bf16 rewrites.
+
+In a decode loop every block fold rewrites every stored coefficient row in the
+new basis and stores it as bf16 again (the explainer's basis synchronization:
+the old coefficients are rewritten at every update, so their rounding happens
+once per fold).  The prefill tests postpone those rewrites; this file checks
+the per-fold regime itself, the one the bench times, against the float64
+oracle, which emulates the bf16 rounding at every rewrite:
+
+  * the 32K bench geometry (one layer, batch 8, 8 KV / 32 query heads, r_K 32,
+    r_V 64, W 1024, bf16 coefficients): 16K tokens prefilled with postponed
+    rewrites, then 256 folds with a rewrite after each, decode checks between;
+  * the chain-of-thought ranks (r_K 64, r_V 96 so k = 32, W 2048, batch 1,
+    drift every 2K tokens): 8K prefilled, then 256 per-fold rewrites.
+
+Beside the kernel error the test reports the format drift: the same oracle
+run with float64 coefficient storage against the bf16-emulating one (what
+bf16 storage itself costs, separate from kernel error).  Tolerance 2e-2 on
+reconstructions C B^T and decode outputs, counters exact.
+"""
+
+import pytest
+
+from iskv_testlib import SampledCache
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _one_blas_thread():
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        yield
+
+
+def _cfg(**kw):
+    import online_rank_kv_b200 as ik
+    c = ik.Config(kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1, rope_theta=1e6,
+                  max_deferred=64, ring_extra=512)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _chain(s, folds, check_every):
+    """`folds` decode periods: 64 tokens appended in four steps (a decode
+    check after the first every `check_every` periods), then one fold with
+    the rewrite of every stored row.  Returns the table of worst errors."""
+    rows = []
+    for i in range(1, folds + 1):
+        for part in range(4):
+            s.append(16)
+            if part == 0 and i % check_every == 0:
+                dec = s.decode_check(tol=TOL)
+        assert s.ready() == 1
+        s.fold_all(defer=False)
+        if i % check_every == 0 or i == folds:
+            rec = s.check(tol=TOL)
+            dec = s.decode_check(tol=TOL)
+            rows.append((i, rec, dec, s.format_drift()))
+    return rows
+
+
+def _report(name, rows):
+    print(f"\n{name}: per-fold rewrites against the oracle")
+    print(" folds  recon-err  decode-err  format-drift(bf16 vs fp64 storage)")
+    for i, rec, dec, drift in rows:
+        print(f" {i:5d}  {rec:9.2e}  {dec:10.2e}  {drift:9.2e}")
+
+
+def test_per_fold_rewrites_qwen3_geometry_256_folds():
+    cfg = _cfg(batch=8, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64, window=1024,
+               max_tokens=16384 + 256 * 64 + 1024)
+    s = SampledCache(cfg, "qwen3", [(0, 0, 0), (0, 3, 4), (0, 7, 7)], seed=110, shadow=True)
+    s.prefill(16384)
+    s.check(tol=TOL)
+    rows = _chain(s, 256, 32)
+    _report("qwen3 1 layer, batch 8, r_K 32, r_V 64", rows)
+    T, n_c = s.cache.counts(0)
+    assert n_c == 16384 - 1024 + 256 * 64
+    assert s.cache.status() == 0
+
+
+def test_per_fold_rewrites_cot_ranks_256_folds():
+    cfg = _cfg(batch=1, layers=1, kv_heads=8, q_heads=32, rank_k=64, rank_v=96, window=2048,
+               max_tokens=8192 + 256 * 64 + 1024)
+    s = SampledCache(cfg, "cot", [(0, 0, 1), (0, 0, 6)], seed=111, shadow=True)
+    s.prefill(8192)
+    s.check(tol=TOL)
+    rows = _chain(s, 256, 32)
+    _report("cot 1 layer, batch 1, r_K 64, r_V 96", rows)
+    assert s.cache.status() == 0

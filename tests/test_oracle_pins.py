@@ -733,3 +733,114 @@ def test_joint_head_pin_catches_a_wrong_head_slice(monkeypatch):
     monkeypatch.setattr(O, "joint_head_decode", shifted)
     with pytest.raises(AssertionError):
         test_joint_head_factor_lossless_decode_equals_per_head_attention()
+
+
+# ----------------------------------------------------------------------------
+# where bf16 coefficient storage rounds: new rows, each per-fold rewrite, and
+# once per postponed segment.  Pinned by two facts independent of the code:
+# a stored value is a bf16 number, and one round-to-nearest step moves a value
+# by at most the unit roundoff u = 2^-8 of bf16's 8-bit significand.
+# ----------------------------------------------------------------------------
+
+_U_BF16 = 2.0 ** -8
+
+
+def _is_bf16(x):
+    return np.array_equal(O.bf16_round(x), x)
+
+
+def _within_one_rounding(stored, exact):
+    return bool(np.all(np.abs(stored - exact) <= _U_BF16 * np.abs(exact)))
+
+
+def _storage_rows(seed):
+    return _low_rank_rows(64 * 14, 128, 24, seed=seed, noise=0.05)
+
+
+def test_bf16_storage_rounds_new_rows_and_every_rewrite_once():
+    """Per-fold rewrites: after every fold all stored coefficients are bf16
+    values, the block's rows are fold_block's C_new rounded once, and the old
+    rows are the previously stored rows times W_top rounded once."""
+    rows = _storage_rows(5)
+    f = O.HeadFactor(128, 16, 64, coef_round="bf16")
+    f.append(rows)
+    folds = 0
+    while f.ready() > 0:
+        prev = f.C.copy()
+        res = f.fold()
+        C = f.C
+        assert _is_bf16(C)
+        assert _within_one_rounding(C[prev.shape[0]:], res.C_new)
+        if prev.shape[0]:
+            assert _within_one_rounding(C[:prev.shape[0]], prev @ res.W_top)
+        folds += 1
+    assert folds >= 10
+
+
+def test_bf16_storage_rounds_a_postponed_segment_once():
+    """Postponed rewrites: new rows are rounded when written; iskv's postponed
+    segment is applied as one product per row and rounded once, so every row
+    stays within one rounding of (stored row) x W_top(i) ... W_top(k)."""
+    rows = _storage_rows(6)
+    f = O.HeadFactor(128, 16, 64, coef_round="bf16")
+    f.append(rows[:64 * 4])
+    _fold_all(f)
+    before = f.C.copy()
+    f.append(rows[64 * 4:])
+    tops, starts = [], []
+    while f.ready() > 0:
+        starts.append(f.n_c)
+        res = f.fold(defer=True)
+        tops.append(res.W_top)
+        assert _is_bf16(f.C)                      # new rows rounded at once
+    assert len(tops) >= 8
+    written = f.C.copy()                          # rows as stored before the rewrite
+    f.sync()
+    C = f.C
+    assert _is_bf16(C)
+    for i, n0 in enumerate(starts):
+        lo = starts[i - 1] if i > 0 else 0
+        if n0 <= lo:
+            continue
+        chain = np.eye(16)
+        for W_top in tops[i:]:
+            chain = chain @ W_top
+        src = before[lo:n0] if i == 0 else written[lo:n0]
+        assert _within_one_rounding(C[lo:n0], src @ chain), i
+
+
+def _skip_rounding(which):
+    real = O._store
+
+    def store(x, coef_round):
+        new_rows = np.shape(x)[0] == 64
+        if (which == "new" and new_rows) or (which == "rewrite" and not new_rows):
+            return np.asarray(x, dtype=np.float64)
+        return real(x, coef_round)
+    return store
+
+
+class _RoundsEveryPostponedStep(O.HeadFactor):
+    """Storage mistake: the postponed chain is rounded after every factor."""
+
+    def sync(self):
+        lo = 0
+        for i, (n_rows, _) in enumerate(self.pending):
+            if n_rows > lo:
+                for _, W_top in self.pending[i:]:
+                    self.C[lo:n_rows] = O.bf16_round(self.C[lo:n_rows] @ W_top)
+                lo = n_rows
+        self.pending = []
+
+
+@pytest.mark.parametrize("which", ["new", "rewrite"])
+def test_storage_pins_catch_a_dropped_rounding(which, monkeypatch):
+    monkeypatch.setattr(O, "_store", _skip_rounding(which))
+    with pytest.raises(AssertionError):
+        test_bf16_storage_rounds_new_rows_and_every_rewrite_once()
+
+
+def test_storage_pins_catch_a_rounding_per_postponed_step(monkeypatch):
+    monkeypatch.setattr(O, "HeadFactor", _RoundsEveryPostponedStep)
+    with pytest.raises(AssertionError):
+        test_bf16_storage_rounds_a_postponed_segment_once()
