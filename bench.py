@@ -45,6 +45,18 @@ WORKLOADS = {
     "qwen3-1L-b1-16k": dict(batch=1, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
                             window=1024, prefill=16384, coef="f32", gen="qwen3"),
 }
+# Long chain-of-thought growth: 36 layers, batch 1, grown from 8K to 128K
+# tokens; timed at each context bin, 30% of the decode steps carry queries
+# aimed at tokens older than 8K (recall of compressed history).
+GROWTH = {"cot-128k": dict(batch=1, layers=36, kv_heads=8, q_heads=32, rank_k=64, rank_v=96,
+                           window=2048, coef="bf16", gen="cot",
+                           bins=[8192, 16384, 32768, 65536, 131072], recall=0.3,
+                           recall_age=8192)}
+# One-layer sweep: ranks x contexts x batches, r_K = r_V = r, W 1024, plus the
+# no-synchronization ablation's reconstruction drift at one point.
+SWEEP = {"sweep": dict(layers=1, kv_heads=8, q_heads=32, window=1024, coef="bf16", gen="qwen3",
+                       ranks=[16, 32, 64, 128], contexts=[4096, 16384, 65536, 262144],
+                       batches=[1, 8, 32])}
 DEFAULT_WORKLOAD = "qwen3-36L-b8-32k"
 D = 128
 BLOCK = 64
@@ -52,10 +64,20 @@ BLOCK = 64
 
 # DRAM bytes (read + write) of one decode-attention launch at the per-layer
 # shape of the 32K-context, batch-8 workloads (8 KV / 32 query heads, r_K 32,
-# r_V 64), from the ncu launch list in profiles/launches_qwen3-1L-b8-32k.md
-# (the 36-layer run issues the same launch once per layer).  None for
-# workloads without a capture.
+# r_V 64), taken from an ncu launch list of the one-layer workload (the
+# 36-layer run issues the same launch once per layer).  Not measured by this
+# run: reported as copied, with its source, and only while the decode kernel
+# is the one that was captured (None otherwise, and for other workloads).
 DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.3e6, "qwen3-1L-b8-32k": 433.3e6}
+DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode launch "
+                         "at this per-layer shape (one-layer 32K workload, launch list of the "
+                         "timed steps); copied, not measured in this run")
+
+# What the path computes in: storage, tensor-core operand and accumulator types.
+PRECISION = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: bf16 MMA rebuilds keys "
+             "(basis as bf16 hi+lo) into fp32, rotated keys rounded to fp16, scores by fp16 "
+             "MMA with fp16 hi+lo queries, p as bf16 hi+lo, fp32 softmax and accumulators; "
+             "rewrite: bf16 MMA with an fp32-exact 3-part split of W_top; fold: fp32")
 
 
 def _peaks():
@@ -435,7 +457,12 @@ def run_iskv(args, rank, world, local_rank):
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate" if coef == ik.BF16
+                 else "fp32 math on bf16 K/V, fp32 coefficients",
+        "precision": PRECISION if coef == ik.BF16 else "bf16 K/V in HBM, fp32 coefficients "
+                     "and bases, fp32 CUDA-core math throughout",
+        "data": "synthetic",
         "config": {
             "workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H, "q_heads": Hq,
             "head_dim": D, "rank_k": wl["rank_k"], "rank_v": wl["rank_v"],
@@ -457,6 +484,7 @@ def run_iskv(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.workload)
                      if coef == ik.BF16 and P == 0 else None,
+                     "traffic_source": DECODE_TRAFFIC_SOURCE,
                      "kernel": "decode_tc_kernel (persistent split-K decode attention, "
                                "per-head combine fused), one launch per layer call",
                      "algorithmic_bytes_per_launch": bsum / max(1, len(dec_events)),
@@ -475,13 +503,340 @@ def run_iskv(args, rank, world, local_rank):
     return result
 
 
+def _decode_bytes(Bsz, H, Hq, rK, rV, T, n_c, cb, kvb=2):
+    """Algorithmic bytes of one decode call of one layer: coefficients, the
+    exact rows (K and V), the bases, queries and outputs."""
+    n_w = T - n_c
+    per_head = n_c * (rK + rV) * cb + 2 * n_w * D * kvb + D * (rK + rV) * 4
+    return Bsz * H * per_head + Bsz * Hq * D * (kvb + 4)
+
+
+def _time_periods(cache, ik, L, stream, n_periods, inputs, qfn, dec_events, step0):
+    """n_periods fold periods: 64 decode steps (append one token, decode, every
+    layer), then one fold of every layer with its rewrite.  Decode calls of
+    every 8th step are timed with events.  Returns the elapsed ms."""
+    import torch
+    kk, vv = inputs
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    i = step0
+    for _ in range(n_periods):
+        for s in range(BLOCK):
+            for l in range(L):
+                cache.append(l, kk[i, l], vv[i, l])
+                q = qfn(i, l)
+                if dec_events is not None and s % 8 == 0:
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    cache.decode_attention(l, q)
+                    b.record(stream)
+                    T, n_c = cache.counts(l)
+                    dec_events.append((a, b, T, n_c))
+                else:
+                    cache.decode_attention(l, q)
+            i += 1
+        cache.compress_block(ik.ALL_LAYERS)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def _fold_and_rewrite_us(cache, ik, stream):
+    """One fold of every layer with its rewrite postponed, then the rewrite:
+    (fold us, rewrite us).  Needs a ready block in every layer."""
+    import torch
+    f0, f1, f2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    f0.record(stream)
+    cache.compress_block(ik.ALL_LAYERS, defer=True)
+    f1.record(stream)
+    cache.sync(ik.ALL_LAYERS)
+    f2.record(stream)
+    torch.cuda.synchronize()
+    return f0.elapsed_time(f1) * 1e3, f1.elapsed_time(f2) * 1e3
+
+
+def _prefill_to(cache, ik, ks, vs, L, Bsz, H, W, target, archive=None):
+    """Append generated rows until T = target, folding every ready block with
+    postponed rewrites (one rewrite per 64 folds).  `archive` (optional)
+    receives the pre-RoPE keys at positions 17 mod 512 of every head."""
+    folds = 0
+    T, _ = cache.counts(0)
+    while T < target:
+        n = min(512, target - T)
+        k = ks.next(n)
+        v = vs.next(n)
+        if archive is not None:
+            for j in range(n):
+                if (T + j) % 512 == 17:
+                    archive["rows"].append(k[:, j].clone())
+                    archive["pos"].append(T + j)
+        k = k.view(L, Bsz, H, n, D)
+        v = v.view(L, Bsz, H, n, D)
+        for l in range(L):
+            cache.append(l, k[l], v[l])
+        T, n_c = cache.counts(0)
+        while (T - n_c - W) // BLOCK >= 1:
+            cache.compress_block(ik.ALL_LAYERS, defer=True)
+            folds += 1
+            if folds % 64 == 0:
+                cache.sync(ik.ALL_LAYERS)
+            T, n_c = cache.counts(0)
+    cache.sync(ik.ALL_LAYERS)
+
+
+def _bring_to_ready(cache, ik, ks, vs, L, Bsz, H, W):
+    """Append rows until every layer has one ready block (for the fold and
+    rewrite timing)."""
+    T, n_c = cache.counts(0)
+    need = W + BLOCK - (T - n_c)
+    if need > 0:
+        k = ks.next(need).view(L, Bsz, H, need, D)
+        v = vs.next(need).view(L, Bsz, H, need, D)
+        for l in range(L):
+            cache.append(l, k[l], v[l])
+
+
+def run_growth(args, rank, world, local_rank):
+    """Long chain-of-thought decode grown from 8K to 128K tokens: at each
+    context bin, `steps` timed fold periods (after one warm-up period), with
+    30% of the decode steps aiming every query at a token older than 8K."""
+    import torch
+
+    import online_rank_kv_b200 as ik
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = GROWTH[args.workload]
+    L, Bsz, H, Hq = wl["layers"], wl["batch"], wl["kv_heads"], wl["q_heads"]
+    rK, rV, W = wl["rank_k"], wl["rank_v"], wl["window"]
+    g = Hq // H
+    bins = wl["bins"]
+    per_bin = 1 + args.steps
+    n_steps = per_bin * BLOCK
+    max_tokens = bins[-1] + len(bins) * (n_steps + W + 2 * BLOCK) + 1024
+    cfg = ik.Config(batch=Bsz, layers=L, kv_heads=H, q_heads=Hq, rank_k=rK, rank_v=rV, window=W,
+                    max_tokens=max_tokens, kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1,
+                    rope_theta=1e6, max_deferred=64, ring_extra=512)
+    cache = ik.Cache(cfg)
+    nh = L * Bsz * H
+    seed_k, seed_v, seed_q = replica_seeds(rank)
+    ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=seed_k, device=dev, dtype=torch.bfloat16)
+    vs = synth.KVStream(synth.spec_for(wl["gen"], "V"), nh, seed=seed_v, device=dev, dtype=torch.bfloat16)
+    archive = {"rows": [], "pos": []}
+    stream = torch.cuda.current_stream()
+    gq = torch.Generator(device="cpu")
+    gq.manual_seed(seed_q)
+    peak, peak_src = _peaks()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    bins_out = []
+    tot_ms, tot_steps = 0.0, 0
+    t_pre = 0.0
+    for nb in bins:
+        a = time.time()
+        _prefill_to(cache, ik, ks, vs, L, Bsz, H, W, nb, archive)
+        torch.cuda.synchronize()
+        t_pre += time.time() - a
+        # inputs of this bin's periods, resident in HBM
+        kk = ks.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
+        vv = vs.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
+        kk = kk.view(n_steps, L, Bsz, H, 1, D)
+        vv = vv.view(n_steps, L, Bsz, H, 1, D)
+        qq = synth.query_batch(n_steps * L * Bsz * Hq, D, seed=seed_q + nb, device=dev,
+                               dtype=torch.bfloat16).view(n_steps, L, Bsz, Hq, D)
+        # recall steps: every query of the step aims at an archived key of its
+        # KV head older than recall_age tokens
+        T0, _ = cache.counts(0)
+        rows = torch.stack(archive["rows"], 1)          # [L*B*H, n_arch, D]
+        pos = torch.tensor(archive["pos"])
+        old = int((pos < T0 - wl["recall_age"]).sum())
+        recall = torch.rand(n_steps, generator=gq) < wl["recall"]
+        if old > 0:
+            for i in torch.nonzero(recall).flatten().tolist():
+                pick = torch.randint(0, old, (L, Bsz, Hq), generator=gq)
+                head = (torch.arange(L).view(L, 1, 1) * Bsz + torch.arange(Bsz).view(1, Bsz, 1)) * H \
+                    + torch.arange(Hq).view(1, 1, Hq) // g
+                kp = rows[head.flatten().to(dev), pick.flatten().to(dev)].double()
+                ps = pos[pick.flatten()].to(dev)
+                qr = synth.recall_queries(kp, ps, 1e6, 25.0 * D ** 0.5)
+                qr = qr / torch.linalg.vector_norm(kp, dim=-1, keepdim=True)
+                qq[i] = qr.view(L, Bsz, Hq, D).to(torch.bfloat16)
+        dec_events = []
+        qfn = lambda i, l: qq[i, l]
+        _time_periods(cache, ik, L, stream, 1, (kk, vv), qfn, None, 0)           # warm-up
+        ms = _time_periods(cache, ik, L, stream, args.steps, (kk, vv), qfn, dec_events, BLOCK)
+        ms = max_over_ranks(ms, world, dev)
+        dsum = sum(a.elapsed_time(b) for a, b, _, _ in dec_events) / 1e3
+        bsum = sum(_decode_bytes(Bsz, H, Hq, rK, rV, T, n_c, 2) for _, _, T, n_c in dec_events)
+        _bring_to_ready(cache, ik, ks, vs, L, Bsz, H, W)
+        T1, n_c1 = cache.counts(0)
+        fold_us, rw_us = _fold_and_rewrite_us(cache, ik, stream)
+        rw_bytes = 2 * n_c1 * (rK + rV) * 2 * L * Bsz * H
+        steps = args.steps * BLOCK
+        bins_out.append({"context": T0, "steps_per_s": steps / (ms / 1e3) * world,
+                         "ms_per_period": ms / args.steps,
+                         "decode_us": dsum / max(1, len(dec_events)) * 1e6,
+                         "decode_hbm_frac": (bsum / dsum / 1e9) / peak if dsum > 0 else None,
+                         "recall_steps": int(recall[BLOCK:].sum()),
+                         "fold_us": fold_us, "rewrite_us": rw_us,
+                         "rewrite_rows": n_c1, "rewrite_gbs": rw_bytes / (rw_us * 1e-6) / 1e9})
+        tot_ms += ms
+        tot_steps += steps
+        del kk, vv, qq
+    clk = clocks.stop()
+    status = cache.status()
+    kept, full = cache.kv_bytes()
+    cache.close()
+    value = tot_steps * world / (tot_ms / 1e3)
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": BLOCK, "ms_per_step": tot_ms / (args.steps * len(bins)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate", "precision": PRECISION,
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H,
+                   "q_heads": Hq, "head_dim": D, "rank_k": rK, "rank_v": rV, "window": W,
+                   "bins": bins, "recall_fraction": wl["recall"],
+                   "recall_age": wl["recall_age"],
+                   "step": f"per bin: 1 warm-up + {args.steps} timed fold periods (64 decode "
+                           "steps of every layer + 1 fold of every layer with its rewrite)",
+                   "l2": "inputs larger than L2 from the 16K bin on (coefficients of 36 layers)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "bins": bins_out,
+        "prefill_s": t_pre,
+        "persistent_kv": {"bytes": kept, "full_bytes": full,
+                          "compression": full / kept if kept else None},
+        "peak": {"hbm_gbs": peak, "source": peak_src},
+        "gpu_launches": (BLOCK * L * 3 + 4) * args.steps * len(bins),
+        "clocks": clk, "device_status": status,
+    }
+
+
+def run_sweep(args, rank, world, local_rank):
+    """One-layer sweep over ranks, contexts and batches: one JSON line per
+    point (decode steps/s, decode HBM fraction, fold and rewrite time), then
+    one line with the no-synchronization ablation's reconstruction drift."""
+    import torch
+
+    import online_rank_kv_b200 as ik
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = SWEEP[args.workload]
+    L, H, Hq, W = wl["layers"], wl["kv_heads"], wl["q_heads"], wl["window"]
+    peak, peak_src = _peaks()
+    stream = torch.cuda.current_stream()
+    seed_k, seed_v, seed_q = replica_seeds(rank)
+    periods = max(1, min(args.steps, 2))
+    lines = []
+    for r in wl["ranks"]:
+        for T in wl["contexts"]:
+            for Bsz in wl["batches"]:
+                n_steps = (1 + periods) * BLOCK
+                cfg = ik.Config(batch=Bsz, layers=L, kv_heads=H, q_heads=Hq, rank_k=r, rank_v=r,
+                                window=W, max_tokens=T + n_steps + W + 2 * BLOCK + 1024,
+                                kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1, rope_theta=1e6,
+                                max_deferred=64, ring_extra=512)
+                cache = ik.Cache(cfg)
+                nh = L * Bsz * H
+                ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=seed_k + r + T, device=dev,
+                                    dtype=torch.bfloat16)
+                vs = synth.KVStream(synth.spec_for(wl["gen"], "V"), nh, seed=seed_v + r + T, device=dev,
+                                    dtype=torch.bfloat16)
+                _prefill_to(cache, ik, ks, vs, L, Bsz, H, W, T)
+                kk = ks.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
+                vv = vs.next(n_steps).view(L, Bsz, H, n_steps, D).permute(3, 0, 1, 2, 4).contiguous()
+                kk = kk.view(n_steps, L, Bsz, H, 1, D)
+                vv = vv.view(n_steps, L, Bsz, H, 1, D)
+                qq = synth.query_batch(n_steps * L * Bsz * Hq, D, seed=seed_q + r + T + Bsz, device=dev,
+                                       dtype=torch.bfloat16).view(n_steps, L, Bsz, Hq, D)
+                qfn = lambda i, l: qq[i, l]
+                dec_events = []
+                clocks = ClockSampler(local_rank)
+                clocks.start()
+                _time_periods(cache, ik, L, stream, 1, (kk, vv), qfn, None, 0)
+                ms = _time_periods(cache, ik, L, stream, periods, (kk, vv), qfn, dec_events, BLOCK)
+                clk = clocks.stop()
+                ms = max_over_ranks(ms, world, dev)
+                dsum = sum(a.elapsed_time(b) for a, b, _, _ in dec_events) / 1e3
+                bsum = sum(_decode_bytes(Bsz, H, Hq, r, r, Tn, n_c, 2) for _, _, Tn, n_c in dec_events)
+                _bring_to_ready(cache, ik, ks, vs, L, Bsz, H, W)
+                _, n_c1 = cache.counts(0)
+                fold_us, rw_us = _fold_and_rewrite_us(cache, ik, stream)
+                status = cache.status()
+                cache.close()
+                del kk, vv, qq, cache, ks, vs
+                torch.cuda.empty_cache()
+                steps = periods * BLOCK
+                line = {
+                    "metric": METRIC, "value": steps * world / (ms / 1e3), "unit": UNIT,
+                    "n_gpus": world, "steps": periods, "warmup": BLOCK,
+                    "ms_per_step": ms / periods, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate",
+                    "data": "synthetic",
+                    "config": {"workload": f"sweep r{r} T{T} B{Bsz}", "batch": Bsz, "layers": L,
+                               "kv_heads": H, "q_heads": Hq, "rank_k": r, "rank_v": r, "window": W,
+                               "context_start": T,
+                               "step": "fold period: 64 decode steps + 1 fold with its rewrite"},
+                    "decode_us": dsum / max(1, len(dec_events)) * 1e6,
+                    "decode_hbm_frac": (bsum / dsum / 1e9) / peak if dsum > 0 else None,
+                    "peak": {"hbm_gbs": peak, "source": peak_src},
+                    "fold_us": fold_us, "rewrite_us": rw_us,
+                    "rewrite_gbs": 2 * n_c1 * 2 * r * 2 * L * Bsz * H / (rw_us * 1e-6) / 1e9,
+                    "clocks": clk, "device_status": status,
+                }
+                lines.append(line)
+                if rank == 0:
+                    print(json.dumps(line), flush=True)
+    # no-synchronization ablation: drift of the rebuilt pre-RoPE keys
+    drift = {}
+    for sync in (1, 0):
+        T = 16384
+        cfg = ik.Config(batch=1, layers=1, kv_heads=H, q_heads=Hq, rank_k=32, rank_v=64, window=W,
+                        max_tokens=T + 1024, kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1,
+                        rope_theta=1e6, max_deferred=64, ring_extra=512, sync=sync)
+        cache = ik.Cache(cfg)
+        ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), H, seed=seed_k + 7, device=dev,
+                            dtype=torch.bfloat16)
+        vs = synth.KVStream(synth.spec_for(wl["gen"], "V"), H, seed=seed_v + 7, device=dev,
+                            dtype=torch.bfloat16)
+        rows = []
+        Tn = 0
+        folds = 0
+        while Tn < T:
+            k = ks.next(512)
+            v = vs.next(512)
+            rows.append(k.float())
+            cache.append(0, k.view(1, H, 512, D), v.view(1, H, 512, D))
+            Tn, n_c = cache.counts(0)
+            while (Tn - n_c - W) // BLOCK >= 1:
+                cache.compress_block(0)
+                folds += 1
+                Tn, n_c = cache.counts(0)
+        Kx = torch.cat(rows, 1)[:, :n_c]
+        rec = cache.reconstruct(0, ik.WHICH_K)[0]
+        drift[sync] = float(torch.linalg.vector_norm(rec - Kx) / torch.linalg.vector_norm(Kx))
+        cache.close()
+    if rank == 0:
+        print(json.dumps({"metric": "reconstruction drift ||C B^T - K||_F / ||K||_F (pre-RoPE keys)",
+                          "workload": "sweep drift r_K 32, T 16384, batch 1, per-fold rewrites",
+                          "synchronized": drift[1], "no_sync_ablation": drift[0],
+                          "ratio": drift[0] / drift[1] if drift[1] > 0 else None}), flush=True)
+    return None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=6)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="iskv", choices=["iskv", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(WORKLOADS) + sorted(GROWTH) + sorted(SWEEP))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--async-update", action="store_true",
@@ -499,7 +854,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        wl = WORKLOADS[args.workload]
+        wl = WORKLOADS[args.workload if args.workload in WORKLOADS else DEFAULT_WORKLOAD]
         vals = []
         cores = sample = None
         per = max(2.0, args.cpu_budget / max(1, args.steps + args.warmup))
@@ -530,6 +885,14 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
     try:
+        if args.workload in SWEEP:
+            run_sweep(args, rank, world, local_rank)
+            return
+        if args.workload in GROWTH:
+            res = run_growth(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res = run_iskv(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:

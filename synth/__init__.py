@@ -25,7 +25,7 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["StreamSpec", "KVStream", "spec_for", "query_batch"]
+__all__ = ["StreamSpec", "KVStream", "spec_for", "query_batch", "recall_query", "recall_queries"]
 
 
 @dataclass(frozen=True)
@@ -160,3 +160,19 @@ def recall_query(k_pre: torch.Tensor, pos: int, theta: float, beta: float) -> to
     rot = torch.cat([x1 * c - x2 * s, x1 * s + x2 * c], dim=-1)
     return beta * rot / torch.linalg.vector_norm(k, dim=-1, keepdim=True).clamp_min(1e-30)
 
+
+def recall_queries(k_pre: torch.Tensor, pos: torch.Tensor, theta: float,
+                   beta: float) -> torch.Tensor:
+    """Many recall queries at once: row i is beta * RoPE(k_pre[i], pos[i]) /
+    |k_pre[i]| (the same construction as ``recall_query``), computed in
+    float64 on the rows' device."""
+    k = k_pre.to(torch.float64)
+    d = k.shape[-1]
+    h = d // 2
+    inv = torch.pow(torch.tensor(float(theta), dtype=torch.float64, device=k.device),
+                    -2.0 * torch.arange(h, dtype=torch.float64, device=k.device) / d)
+    ang = pos.to(torch.float64).reshape(-1, 1) * inv.reshape(1, -1)
+    c, s = torch.cos(ang), torch.sin(ang)
+    x1, x2 = k[..., :h], k[..., h:]
+    rot = torch.cat([x1 * c - x2 * s, x1 * s + x2 * c], dim=-1)
+    return beta * rot / torch.linalg.vector_norm(k, dim=-1, keepdim=True).clamp_min(1e-30)
