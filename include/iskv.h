@@ -63,7 +63,14 @@ extern "C" {
 #define ISKV_ERR_NOMEM         -6  /* device allocation failed in create    */
 #define ISKV_ERR_UNSUPPORTED   -7  /* shape outside the compiled kernels    */
 #define ISKV_ERR_DEVICE_TIMEOUT -8 /* a bounded device-side wait gave up (sticky;
-                                      the results of that call are incomplete) */
+                                      the results of that call are incomplete;
+                                      destroy the cache: its decode bookkeeping
+                                      may be left inconsistent)             */
+#define ISKV_ERR_RANGE         -9  /* a score of the tensor-core decode was not
+                                      finite: a rotated key or a query went
+                                      beyond fp16's range (|x| >= 65504), the
+                                      type its score MMA takes (sticky; that
+                                      call's outputs are not finite)        */
 
 /* ---- element types ----------------------------------------------------- */
 #define ISKV_F32   0
@@ -206,9 +213,9 @@ ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
  * Errors: INVALID_ARG for a NULL cache.                                    */
 ISKV_API int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes);
 
-/* Synchronize the device and return the cache's sticky device status:
- * ISKV_OK, ISKV_ERR_DEVICE_TIMEOUT, ISKV_ERR_NOCONVERGE or ISKV_ERR_CUDA.
- * Clears nothing.                                                          */
+/* Synchronize the device and return the cache's sticky device status, the
+ * most severe first: ISKV_ERR_CUDA, ISKV_ERR_DEVICE_TIMEOUT, ISKV_ERR_RANGE,
+ * ISKV_ERR_NOCONVERGE, else ISKV_OK.  Clears nothing.                      */
 ISKV_API int iskv_status(iskv_t h);
 
 /* Static string naming a status code.                                     */

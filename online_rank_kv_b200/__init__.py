@@ -40,7 +40,7 @@ ALL_LAYERS = -1
 FOLD_DEFER_SYNC = 1
 
 _ERRORS = {-1: "INVALID_ARG", -2: "CAPACITY", -3: "STATE", -4: "CUDA", -5: "NOCONVERGE",
-           -6: "NOMEM", -7: "UNSUPPORTED", -8: "DEVICE_TIMEOUT"}
+           -6: "NOMEM", -7: "UNSUPPORTED", -8: "DEVICE_TIMEOUT", -9: "RANGE"}
 
 
 class IskvError(RuntimeError):

@@ -60,6 +60,10 @@ struct iskv_cache {
     int max_splits = 256;
     bool use_tc = true;           // tensor-core paths for bf16 coefficients
     int sms = 148;
+    // clock cycles a tensor-core pipeline wait may take before the call gives
+    // up with DEVICE_TIMEOUT; tests shorten it through the environment to make
+    // the wait run out on purpose (ISKV_TEST_PIPELINE_WAIT_CYCLES)
+    long long pipe_wait = tc::kWaitCycles;
     // host counters
     std::vector<int64_t> T, n_c;
     std::vector<int> n_pend;
@@ -300,6 +304,8 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         const char* env = std::getenv("ISKV_TENSOR_CORES");
         h->use_tc = kDecodeTcDefault ? !(env && env[0] == '0') : (env && env[0] == '1');
         cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+        const char* w = std::getenv("ISKV_TEST_PIPELINE_WAIT_CYCLES");
+        if (w && std::atoll(w) > 0) h->pipe_wait = std::atoll(w);
     }
     h->T.assign(c.layers, 0);
     h->n_c.assign(c.layers, 0);
@@ -626,6 +632,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.n_c = a.n_c;
         t.T = a.T;
         t.scale = a.scale;
+        t.pipe_wait = h->pipe_wait;
         // exact-row tiles of 64 rows, or of 32 when 64 rows of K and V would make
         // a stage larger than a folded tile's C_K and C_V
         const int64_t coef_tile = (int64_t)128 * (c.rank_k + c.rank_v) * 2;
@@ -787,6 +794,7 @@ int iskv_status(iskv_t h) {
     if (cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return ISKV_ERR_CUDA;
     if (st & tc::kStatusTimeout) return ISKV_ERR_DEVICE_TIMEOUT;
+    if (st & kStatusRange) return ISKV_ERR_RANGE;
     if (st & kStatusNoConverge) return ISKV_ERR_NOCONVERGE;
     return ISKV_OK;
 }
@@ -802,6 +810,7 @@ const char* iskv_strerror(int code) {
         case ISKV_ERR_NOMEM: return "device allocation failed";
         case ISKV_ERR_UNSUPPORTED: return "shape not supported by the compiled kernels";
         case ISKV_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up; that call's results are incomplete";
+        case ISKV_ERR_RANGE: return "a rotated key or query left the fp16 range of the tensor-core decode";
         default: return "unknown status";
     }
 }

@@ -18,8 +18,10 @@ constexpr int kMaxLayers = 128;   // layers per cache (bounds kernel params)
 constexpr int kMaxDeferred = 64;  // postponed folds per layer
 constexpr int kMaxGroup = 8;      // query heads per KV head in the decode
 
-// Status bits of the sticky device word.
+// Status bits of the sticky device word (bit 2, a bounded wait that gave up,
+// is defined with the waits in tc_util.cuh).
 constexpr int kStatusNoConverge = 1;
+constexpr int kStatusRange = 4;   // a non-finite score in the tensor-core decode
 
 // ---------------------------------------------------------------------------
 // Element conversions (explicit round-to-nearest-even for bf16 stores).
@@ -142,6 +144,8 @@ struct DecodeTcArgs {
     int basis_bufs;              // bf16 basis buffers (1 or 2 heads in flight)
     int q_bufs;                  // q' buffers per epilogue group (1 or 2)
     float scale;
+    long long pipe_wait;         // clock cycles a pipeline wait may take before the
+                                 // call gives up (drain waits keep their own limit)
 };
 
 // ---------------------------------------------------------------------------

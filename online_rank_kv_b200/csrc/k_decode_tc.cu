@@ -47,7 +47,9 @@
 // Rotated keys are held in fp16 (finite for |k| < 65504; the same 11-bit
 // significand as tf32); the query as fp16 hi + lo parts keeps ~22 bits.
 // Every mbarrier wait is bounded; on timeout the CTA records
-// ISKV status bit 2, stops, drains its copies and frees its TMEM.
+// ISKV status bit 2, stops, drains its copies and frees its TMEM.  A score
+// that is not finite (a rotated key or query outside the fp16 range) sets
+// status bit 4.
 #include "iskv_internal.cuh"
 #include "tc_util.cuh"
 
@@ -229,7 +231,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const long long deadline = clock64() + kWaitCycles;
+    const long long deadline = clock64() + a.pipe_wait;
     const int BH = a.K.BH;
 
     auto fail = [&]() {
@@ -379,6 +381,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             }
         };
         bool stop = false;
+        bool range_bad = false;                   // a non-finite score seen by this thread
         int n0 = 0, hs = -1;
         // the two groups run through the heads independently: each keeps its own
         // softmax state and publishes its own partial slot per head
@@ -547,8 +550,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 bool over = false;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    sc[h] = (row < valid) ? (__uint_as_float(sv[h]) + __uint_as_float(sv[G + h])) * a.scale
-                                          : -INFINITY;
+                    const float raw = __uint_as_float(sv[h]) + __uint_as_float(sv[G + h]);
+                    sc[h] = (row < valid) ? raw * a.scale : -INFINITY;
+                    range_bad |= row < valid && !(fabsf(raw) <= 3.0e38f);   // inf or NaN
                     over |= sc[h] > m_run[h] + kLazyMax;   // always true while m_run = -inf
                 }
                 // p of this row, bf16 hi parts then lo parts, one or two 16-byte rows
@@ -743,6 +747,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             }
             n0 = s1;
         }
+        if (__any_sync(0xffffffffu, range_bad) && lane == 0) atomicOr(a.status, kStatusRange);
     } else if (warp >= 10) {
         // ---------------- MMA issuer of group warp - 10 ----------------
         // per tile n of the group: K^ = C_K (B_hi + B_lo)^T (issued as soon as the

@@ -71,8 +71,9 @@ def test_defaults_and_strings():
     assert (c.kv_heads, c.q_heads, c.head_dim, c.rank_k, c.rank_v, c.window, c.block) == \
         (8, 32, 128, 32, 64, 1024, 64)
     assert ik.LIB.iskv_config_default(None) == -1
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
-        assert len(ik.LIB.iskv_strerror(code)) > 0
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9):
+        assert ik.LIB.iskv_strerror(code) != b"unknown status"
+    assert set(ik._ERRORS) == {-1, -2, -3, -4, -5, -6, -7, -8, -9}
     assert ik.LIB.iskv_strerror(42) == b"unknown status"
 
 

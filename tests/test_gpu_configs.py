@@ -11,8 +11,9 @@ exact.
   * the long chain-of-thought growth run: batch 1, 36 layers, r_K 64, r_V 96,
     W 2048, subspace drift every 2K tokens, grown to 128K tokens, with
     queries aimed at tokens older than 8K (recall of compressed history);
-  * the one-layer sweep: ranks {16, 32, 64, 128} at 4K and 16K contexts and
-    batch {1, 8}, its largest point (r 128, 256K context, batch 32), and the
+  * the one-layer sweep, every point: ranks {16, 32, 64, 128} x contexts
+    {4K, 16K, 64K, 256K} x batches {1, 8, 32} (the three batch sizes of a
+    point run in lockstep and share one sampled head's rows), and the
     no-synchronization ablation's reconstruction drift against the
     synchronized path.
 """
@@ -94,26 +95,109 @@ def test_long_cot_growth_to_128k_with_recall():
     assert s.cache.status() == 0
 
 
+class LockstepSweep:
+    """Caches of batch 1, 8 and 32 at one (rank, context) point of the sweep,
+    fed in lockstep.  Each cache's own rows come from its seeded generator,
+    except that the last sequence's KV head 7 receives the same rows in all
+    three caches (a one-head stream), so one pair of oracle factors checks all
+    three batch sizes -- and a different sequence slot in each."""
+
+    BATCHES = (1, 8, 32)
+
+    def __init__(self, r, T, seed):
+        import online_rank_kv_b200 as ik
+        self.ik = ik
+        self.r, self.T = r, T
+        self.caches, self.ks, self.vs = {}, {}, {}
+        for B in self.BATCHES:
+            cfg = _cfg(batch=B, layers=1, kv_heads=8, q_heads=32, rank_k=r, rank_v=r,
+                       window=1024, max_tokens=T + 1024)
+            self.caches[B] = ik.Cache(cfg)
+            self.ks[B] = synth.KVStream(synth.spec_for("qwen3", "K"), B * 8, seed=seed + 2 * B,
+                                        device="cuda", dtype=torch.bfloat16)
+            self.vs[B] = synth.KVStream(synth.spec_for("qwen3", "V"), B * 8, seed=seed + 2 * B + 1,
+                                        device="cuda", dtype=torch.bfloat16)
+        self.cfg = cfg
+        self.sk = synth.KVStream(synth.spec_for("qwen3", "K"), 1, seed=seed + 100, device="cuda",
+                                 dtype=torch.bfloat16)
+        self.sv = synth.KVStream(synth.spec_for("qwen3", "V"), 1, seed=seed + 101, device="cuda",
+                                 dtype=torch.bfloat16)
+        self.ok = HeadFactor(128, r, 1024, coef_round="bf16")
+        self.ov = HeadFactor(128, r, 1024, coef_round="bf16")
+        self.folds = 0
+
+    def append(self, n):
+        rk, rv = self.sk.next(n)[0], self.sv.next(n)[0]
+        for B in self.BATCHES:
+            k = self.ks[B].next(n).view(B, 8, n, 128)
+            v = self.vs[B].next(n).view(B, 8, n, 128)
+            k[B - 1, 7] = rk
+            v[B - 1, 7] = rv
+            self.caches[B].append(0, k, v)
+        self.ok.append(rk.double().cpu().numpy())
+        self.ov.append(rv.double().cpu().numpy())
+
+    def prefill(self, chunk=512, defer_every=64):
+        done = 0
+        while done < self.T:
+            n = min(chunk, self.T - done)
+            self.append(n)
+            done += n
+            while self.ok.ready() >= 1:
+                for c in self.caches.values():
+                    c.compress_block(0, defer=True)
+                self.ok.fold(defer=True)
+                self.ov.fold(defer=True)
+                self.folds += 1
+                if self.folds % defer_every == 0:
+                    self.sync()
+        self.sync()
+
+    def sync(self):
+        for c in self.caches.values():
+            c.sync(0)
+        self.ok.sync()
+        self.ov.sync()
+
+    def check(self):
+        ik = self.ik
+        worst = 0.0
+        q = synth.query_batch(4, 128, seed=self.r + self.T, dtype=torch.bfloat16)
+        want = dense_decode(q.double().numpy(), self.ok.full(), self.ov.full(), 1e6)
+        for B, c in self.caches.items():
+            assert c.counts(0) == (self.ok.T, self.ok.n_c)
+            for which, of in ((ik.WHICH_K, self.ok), (ik.WHICH_V, self.ov)):
+                got = c.reconstruct(0, which)
+                e = rel_err(got[B - 1, 7].cpu().numpy(), of.reconstruct())
+                del got
+                assert e < TOL, (B, which, e)
+                worst = max(worst, e)
+            qb = synth.query_batch(B * 32, 128, seed=B, dtype=torch.bfloat16).view(B, 32, 128)
+            qb[B - 1, 28:32] = q
+            out = c.decode_attention(0, qb.cuda())[B - 1, 28:32].cpu().numpy()
+            e = rel_err(out, want)
+            assert e < TOL, (B, "decode", e)
+            worst = max(worst, e)
+            assert c.status() == 0
+        return worst
+
+    def close(self):
+        for c in self.caches.values():
+            c.close()
+        self.caches = {}
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("T", [4096, 16384, 65536, 262144])
 @pytest.mark.parametrize("r", [16, 32, 64, 128])
-@pytest.mark.parametrize("T,B", [(4096, 1), (16384, 8)])
-def test_sweep_point(r, T, B):
-    cfg = _cfg(batch=B, layers=1, kv_heads=8, q_heads=32, rank_k=r, rank_v=r, window=1024,
-               max_tokens=T + 1024)
-    s = SampledCache(cfg, "qwen3", [(0, 0, 0), (0, B - 1, 7)], seed=80 + r)
-    s.prefill(T)
+def test_sweep_grid(r, T):
+    """Every point of the one-layer sweep: ranks {16, 32, 64, 128} x contexts
+    {4K, 16K, 64K, 256K} x batches {1, 8, 32}, r_K = r_V = r, W 1024, bf16
+    coefficients; postponed rewrites while prefilling, as the bench does."""
+    s = LockstepSweep(r, T, seed=1000 + r + T // 1024)
+    s.prefill()
     s.check()
-    s.decode_check()
-    assert s.cache.status() == 0
-
-
-def test_sweep_largest_point_r128_256k_batch32():
-    cfg = _cfg(batch=32, layers=1, kv_heads=8, q_heads=32, rank_k=128, rank_v=128, window=1024,
-               max_tokens=262144 + 1024)
-    s = SampledCache(cfg, "qwen3", [(0, 31, 5)], seed=90)
-    s.prefill(262144, chunk=512)
-    s.check()
-    s.decode_check()
-    assert s.cache.status() == 0
+    s.close()
 
 
 def test_sweep_no_sync_drift():
