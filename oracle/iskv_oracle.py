@@ -94,11 +94,19 @@ class LatentQuant:
     zeros keeps scale 0.  The pages give no scale rule or bit schedule; this is
     the plainest per-token choice.  Used as a coefficient storage format
     (``coef_round``): applied at every write, new rows and every rewrite.
-    Oracle only: the CUDA path does not store this format yet.
+
+    ``fp32=True`` takes every rounding decision in IEEE float32, the precision
+    of the CUDA kernels that store this format: the values are first rounded
+    to float32, the group maximum and the scale amax / qmax are float32
+    (a correctly rounded division), each code is the float32 quotient x / scale
+    rounded half to even, and a stored value is the float32 product
+    code * scale.  Codes then agree bit for bit with a float32 quantizer fed
+    the same float32 values.
     """
 
-    def __init__(self, groups):
+    def __init__(self, groups, fp32: bool = False):
         self.groups = [(int(n), int(b)) for n, b in groups]
+        self.fp32 = bool(fp32)
         if any(n <= 0 or not (b == 0 or 2 <= b <= 16) for n, b in self.groups):
             raise ValueError("invalid channel groups")
 
@@ -113,24 +121,30 @@ class LatentQuant:
     def quantize(self, C):
         """Integer codes (same shape as C) and scales (rows x groups)."""
         C = np.atleast_2d(np.asarray(C, dtype=np.float64))
+        if self.fp32:
+            C = C.astype(np.float32)
         codes = np.zeros(C.shape, dtype=np.int64)
-        scales = np.zeros((C.shape[0], len(self.groups)))
+        scales = np.zeros((C.shape[0], len(self.groups)), dtype=C.dtype)
         for g, (lo, hi, b) in enumerate(self._spans(C.shape[1])):
             if b == 0:
                 continue
             qmax = 2 ** (b - 1) - 1
             amax = np.abs(C[:, lo:hi]).max(axis=1)
-            sc = amax / qmax
+            sc = amax / C.dtype.type(qmax)
             scales[:, g] = sc
-            safe = np.where(sc > 0, sc, 1.0)[:, None]
+            safe = np.where(sc > 0, sc, C.dtype.type(1.0))[:, None]
             codes[:, lo:hi] = np.clip(np.round(C[:, lo:hi] / safe), -qmax, qmax).astype(np.int64)
-        return codes, scales
+        return codes, scales.astype(np.float64)
 
     def dequantize(self, codes, scales):
         codes = np.atleast_2d(codes)
         out = np.zeros(codes.shape)
         for g, (lo, hi, _) in enumerate(self._spans(codes.shape[1])):
-            out[:, lo:hi] = codes[:, lo:hi] * scales[:, g:g + 1]
+            if self.fp32:
+                prod = codes[:, lo:hi].astype(np.float32) * scales[:, g:g + 1].astype(np.float32)
+                out[:, lo:hi] = prod.astype(np.float64)
+            else:
+                out[:, lo:hi] = codes[:, lo:hi] * scales[:, g:g + 1]
         return out
 
     def __call__(self, C):
@@ -141,6 +155,12 @@ class LatentQuant:
         """Average code bits per stored coefficient (scales not counted)."""
         n = sum(n for n, _ in self.groups)
         return sum(n * b for n, b in self.groups) / n
+
+    def row_bytes(self, scale_bytes: int = 4) -> int:
+        """Bytes one stored row keeps: its codes (bits per channel, whole
+        bytes per group) and one scale per group that has codes."""
+        return sum((n * b + 7) // 8 for n, b in self.groups) + scale_bytes * sum(
+            1 for _, b in self.groups if b > 0)
 
 
 def _store(x, coef_round):
@@ -499,7 +519,7 @@ def full_kv_bytes(tokens: int, layers: int, kv_heads: int, head_dim: int,
 
 def persistent_kv_bytes(n_c: int, n_w: int, d: int, r_k: int, r_v: int,
                         coef_bytes: int, kv_bytes: int, basis_bytes: int = 4,
-                        n_p: int = 0) -> int:
+                        n_p: int = 0, coef_row_bytes: int | None = None) -> int:
     """Bytes kept between decode steps for one (sequence, layer, KV head)
     (Jargon: Persistent-KV compression): both factors (C, and B, S once a
     block is folded), both exact windows (n_w rows) and both sets of
@@ -509,6 +529,9 @@ def persistent_kv_bytes(n_c: int, n_w: int, d: int, r_k: int, r_v: int,
     re-derived from what the pages state, so that number stays unpinned."""
     factors = 0
     if n_c > 0:
-        factors = n_c * (r_k + r_v) * coef_bytes + (d + 1) * (r_k + r_v) * basis_bytes
+        # coef_row_bytes: one row of K and V coefficients when they are not
+        # stored element by element (LatentQuant.row_bytes of both factors)
+        row = (r_k + r_v) * coef_bytes if coef_row_bytes is None else coef_row_bytes
+        factors = n_c * row + (d + 1) * (r_k + r_v) * basis_bytes
     exact = 2 * (n_w + n_p) * d * kv_bytes
     return factors + exact

@@ -844,3 +844,89 @@ def test_storage_pins_catch_a_rounding_per_postponed_step(monkeypatch):
     monkeypatch.setattr(O, "HeadFactor", _RoundsEveryPostponedStep)
     with pytest.raises(AssertionError):
         test_bf16_storage_rounds_a_postponed_segment_once()
+
+
+# ----------------------------------------------------------------------------
+# the float32-decision latent quantizer (the precision of the CUDA format)
+# ----------------------------------------------------------------------------
+
+
+def test_latent_quant_fp32_is_the_nearest_float32_grid_point():
+    """In float32 mode, per row and group: the scale is the float32 quotient
+    amax / qmax of the float32 values, and each stored value is the float32
+    product code * scale of the grid point nearest the float32 value (checked
+    by brute force over every level; a quotient within one float32 rounding
+    of a half-way point may go either way)."""
+    g = _rng(80)
+    C = g.standard_normal((64, 32)) * (2.0 ** -np.arange(32) * 8 + 0.1)
+    C[5] = 0.0
+    q = O.LatentQuant([(8, 8), (8, 4), (16, 2)], fp32=True)
+    codes, scales = q.quantize(C)
+    got = q.dequantize(codes, scales)
+    C32 = C.astype(np.float32)
+    for gi, (lo, hi, b) in enumerate([(0, 8, 8), (8, 16, 4), (16, 32, 2)]):
+        qmax = 2 ** (b - 1) - 1
+        for i in range(C.shape[0]):
+            amax = np.float32(np.abs(C32[i, lo:hi]).max())
+            sc = np.float32(amax / np.float32(qmax))
+            assert np.float32(scales[i, gi]) == sc and scales[i, gi] == float(sc)
+            if sc == 0:
+                assert np.all(got[i, lo:hi] == 0)
+                continue
+            for j in range(lo, hi):
+                x = float(C32[i, j])
+                k = codes[i, j]
+                assert abs(k) <= qmax
+                assert got[i, j] == float(np.float32(np.float32(k) * sc))
+                dist = np.abs(np.arange(-qmax, qmax + 1) * float(sc) - x)
+                near_half = abs(abs(x / float(sc)) % 1.0 - 0.5) < 1e-6
+                assert dist[k + qmax] <= dist.min() + 1e-12 or near_half
+
+
+def test_latent_quant_fp32_agrees_with_float64_away_from_half_way_points():
+    """float32 and float64 decisions differ only where the quotient x / scale
+    lies within float32 rounding of a half-way point, and then by one code."""
+    g = _rng(81)
+    C = g.standard_normal((400, 32)) * (2.0 ** -np.arange(32) * 8 + 0.1)
+    q64 = O.LatentQuant([(8, 8), (8, 4), (16, 2)])
+    q32 = O.LatentQuant([(8, 8), (8, 4), (16, 2)], fp32=True)
+    c64, s64 = q64.quantize(C)
+    c32, s32 = q32.quantize(C)
+    np.testing.assert_allclose(s32, s64, rtol=2 ** -22, atol=0)
+    diff = c32 != c64
+    assert np.abs(c32 - c64).max() <= 1
+    assert diff.mean() < 1e-3
+    for i, j in zip(*np.nonzero(diff)):
+        gi = 0 if j < 8 else (1 if j < 16 else 2)
+        u = abs(C[i, j] / s64[i, gi])
+        assert abs(u % 1.0 - 0.5) < 1e-5, (i, j, u)
+
+
+def test_latent_quant_fp32_pin_catches_float64_decisions(monkeypatch):
+    """A quantizer that divides in float64 instead of float32 is caught."""
+    real = O.LatentQuant.quantize
+
+    def f64_division(self, C):
+        keep = self.fp32
+        self.fp32 = False
+        try:
+            return real(self, np.asarray(C, dtype=np.float32).astype(np.float64))
+        finally:
+            self.fp32 = keep
+
+    monkeypatch.setattr(O.LatentQuant, "quantize", f64_division)
+    with pytest.raises(AssertionError):
+        test_latent_quant_fp32_is_the_nearest_float32_grid_point()
+
+
+def test_latent_quant_row_bytes_counts_codes_and_scales():
+    """A coded row keeps bits x channels of codes per group and one 4-byte
+    scale per group with codes (none for dropped groups)."""
+    q = O.LatentQuant([(8, 8), (8, 4), (16, 2)])
+    assert q.row_bytes() == 8 + 4 + 4 + 3 * 4
+    assert O.LatentQuant([(16, 8), (16, 0)]).row_bytes() == 16 + 4
+    codes, scales = q.quantize(np.ones((3, 32)))
+    per_row_bits = sum(n * b for n, b in q.groups)
+    assert per_row_bits // 8 + 4 * np.count_nonzero(scales[0]) == q.row_bytes()
+    assert O.persistent_kv_bytes(64, 10, 128, 32, 32, 2, 2, coef_row_bytes=100) == \
+        64 * 100 + 129 * 64 * 4 + 2 * 10 * 128 * 2
