@@ -24,11 +24,13 @@
 //   warp 1  TMEM allocation;
 //   warps 2-9 epilogue, two ping-pong groups of 4 warps (group = tile
 //           parity), one token row per thread:
-//           * rotate its row of K^ by R_t (t = row within the tile; the
-//             row's cos/sin(t w_i) sit in spare TMEM columns) and write it
-//             back to TMEM as fp16 pairs (dim i, dim 64 + i) per column; the
-//             query is pre-rotated per tile by R_{j0}^T (j0 = tile start), so
-//             q'.(R_t k) = q.(R_{j0+t} k);
+//           * read its row of K^ out of TMEM (then release the buffer to the
+//             issuer), rotate it by R_t (t = row within the tile; the row's
+//             cos/sin(t w_i) sit in spare TMEM columns) in packed fp32, and
+//             take the g scores as fp32 dot products with q' = R_{j0}^T q
+//             (pre-rotated per tile, j0 = tile start, so q'.(R_t k) =
+//             q.(R_{j0+t} k)), which every thread reads from shared memory
+//             as broadcasts;
 //           * online softmax per query head with a lazily updated maximum;
 //           * p as bf16 hi+lo parts for the value MMA;
 //           * at the end of a head the group publishes its own partial
@@ -38,17 +40,15 @@
 //             groups never wait for each other.
 //   warps 10-11 MMA issuer of group 0 / 1:
 //           * K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens, N=128 dims,
-//             fp32 accumulator in TMEM, rebuilt two tiles ahead;
-//           * scores S = K_rot q'^T, kind::f16 with A from TMEM and q' as
-//             fp16 hi+lo parts in the N dimension, issued in two halves of
-//             the head dimension as the epilogue finishes rotating them;
+//             fp32 accumulator in TMEM, rebuilt for the group's next tile as
+//             soon as the epilogue has read this one;
 //           * O = C_V^T P (kind::f16, C_V tile read MN-major in place; for
 //             exact rows O = V^T P with M = d).
-// Rotated keys are held in fp16 (finite for |k| < 65504; the same 11-bit
-// significand as tf32); the query as fp16 hi + lo parts keeps ~22 bits.
+// Keys, queries and scores stay fp32 after the rebuild (the tensor cores
+// rebuild keys and sum values; the scores, g per row, are CUDA-core work).
 // Every mbarrier wait is bounded; on timeout the CTA records
 // ISKV status bit 2, stops, drains its copies and frees its TMEM.  A score
-// that is not finite (a rotated key or query outside the fp16 range) sets
+// that is not finite (an inf or NaN key or query, or an fp32 overflow) sets
 // status bit 4.
 #include "iskv_internal.cuh"
 #include "tc_util.cuh"
@@ -66,17 +66,16 @@ constexpr int kTile = 128;
 // divides the ring and the protected-row capacity, so a tile never wraps
 constexpr int kThreads = 384;
 constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
-constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
 constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
-constexpr int kBufCols = 160;    // per TMEM buffer: K^ 128 | S 16 | O 16
+constexpr int kBufCols = 144;    // per TMEM buffer: K^ 128 | O 16
 constexpr int kCsCol = 2 * kBufCols;   // per-row RoPE table: cos 64 | sin 64 | -sin 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Bars {
     uint64_t full[6], empty[6];
     uint64_t bk_full[2], bk_empty[4];      // bk_empty[buffer * 2 + group]
-    uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
-    uint64_t krot_ready[2], krot_b[2], p_ready[2];   // epilogue -> group issuer: K_rot halves, P written
+    uint64_t kh_full[2], kfree[2], o_full[2];   // kfree: the group's epilogue has read K^
+    uint64_t p_ready[2];                         // epilogue -> group issuer: P written
     uint64_t drain[3];   // abort path: completion of each issuer's outstanding MMAs
 };
 
@@ -90,7 +89,7 @@ struct SmemPlan {
     uint32_t bk, stage, stage_k, stage_bytes, qb, pb, total;
 };
 
-constexpr int kQWords = kQN * 64;   // one q' buffer: kQN rows of 128 fp16 (64 words)
+constexpr int kQFloats = kMaxGroup * kHeadDim;   // one q' buffer: g <= 8 rows of 128 fp32
 
 __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, int nqb, int wt) {
     SmemPlan p;
@@ -101,7 +100,7 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, i
     if (sb < 2 * wt * kHeadDim * 2) sb = 2 * wt * kHeadDim * 2;   // exact K and V rows
     p.stage_bytes = sb + 1024;
     p.stage = off;             off += ns * p.stage_bytes;
-    p.qb = off;                off += 2 * nqb * (kQWords * 4);   // [group][nqb] q' buffers
+    p.qb = off;                off += 2 * nqb * (kQFloats * 4);   // [group][nqb] q' buffers
     p.pb = off;                off += 2 * (kPN * kTile * 2);
     p.total = off;
     return p;
@@ -129,13 +128,6 @@ __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
 // more than this (p <= e^8); otherwise the tile takes the exact rescale
 constexpr float kLazyMax = 8.f;
 
-// q' as the score MMA's B operand: fp16, K-major 8 x 8 core matrices over
-// K = 128 positions k, where k = 2u holds dim u and k = 2u + 1 dim 64 + u
-// (the order of the packed rotated keys in TMEM).  Word (32-bit) offset of
-// the pair (k = 2u, 2u + 1) of row n.
-__device__ __forceinline__ int qb_off(int n, int u) {
-    return ((n >> 3) * (kTile / 8) + (u >> 2)) * 32 + (n & 7) * 4 + (u & 3);
-}
 // p as the value MMA's B operand, MN-major: [token][16] in 8 x 8 blocks, so one
 // thread's (token's) 8 values of an n-block are one 16-byte row
 __device__ __forceinline__ int pb_off(int n, int k) {
@@ -182,7 +174,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     const SmemPlan P = plan_smem(rK, rV, ns, nbk, nqb, wt);
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
-    uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
+    float* qb = reinterpret_cast<float*>(smem + P.qb);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
     const uint32_t stage_bytes = P.stage_bytes;
     const int tiles_c = a.tiles_c, tiles_cw = a.tiles_c + a.tiles_w;
@@ -204,23 +196,15 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->bk_full[i], 1);
             mbar_init(&bars->kh_full[i], 1);
-            mbar_init(&bars->kfree[i], 1);
-            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->kfree[i], kEpi / 2);
             mbar_init(&bars->o_full[i], 1);
-            mbar_init(&bars->krot_ready[i], kEpi / 2);
-            mbar_init(&bars->krot_b[i], kEpi / 2);
             mbar_init(&bars->p_ready[i], 1);
         }
         for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // zero the padding rows (n >= 2g) of the q' and p operands once
-    for (int e = tid; e < 2 * nqb * kQN * 64; e += kThreads) {
-        const int buf = e / (kQN * 64), w = e % (kQN * 64);
-        const int n = w / 64, u = w % 64;
-        if (n >= 2 * g) qb[buf * kQWords + qb_off(n, u)] = 0u;
-    }
+    // zero the padding rows (n >= 2g) of the p operand once
     for (int e = tid; e < 2 * kPN * kTile; e += kThreads) {
         const int buf = e / (kPN * kTile), w = e % (kPN * kTile);
         const int n = w / kTile, k = w % kTile;
@@ -270,10 +254,12 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 }
                 uint8_t* sk = stage + st * stage_bytes;
                 if (tile < tiles_c) {
+                    // a joint-head factor's coefficients are shared by its heads
+                    const int64_t cidx = coef_inst(a.K, hidx);
                     const __nv_bfloat16* gk = reinterpret_cast<const __nv_bfloat16*>(a.K.coef) +
-                                              hidx * a.K.n_max * rK + (int64_t)tile * kTile * rK;
+                                              cidx * a.K.n_max * rK + (int64_t)tile * kTile * rK;
                     const __nv_bfloat16* gv = reinterpret_cast<const __nv_bfloat16*>(a.V.coef) +
-                                              hidx * a.V.n_max * rV + (int64_t)tile * kTile * rV;
+                                              cidx * a.V.n_max * rV + (int64_t)tile * kTile * rV;
                     mbar_arrive_expect_tx(&bars->full[st], P.stage_k + kTile * rV * 2);
                     bulk_g2s(sk, gk, P.stage_k, &bars->full[st]);
                     bulk_g2s(sk + P.stage_k, gv, kTile * rV * 2, &bars->full[st]);
@@ -356,18 +342,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
         float* gred = red + grp * 64;             // [max 4 x 8 | l 4 x 8] of this group
-        const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
-        uint32_t* qbb = qb + nqb * grp * kQWords;   // the group's first q' buffer (head-end exchange)
+        const uint32_t kh = tmem + grp * kBufCols;   // K^ / O buffer of this group
+        float* qbb = qb + nqb * grp * kQFloats;     // the group's first q' buffer (head-end exchange)
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
-        // q' operand offsets of this thread's items (hi of dims i, i + 64; lo likewise)
-        int qoff[kQItems][2];
-#pragma unroll
-        for (int k = 0; k < kQItems; ++k) {
-            const int item = gt + 128 * k;
-            const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
-            qoff[k][0] = qb_off(h, i);       // hi parts of dims i, 64 + i
-            qoff[k][1] = qb_off(G + h, i);   // lo parts
-        }
 
         float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
         // acc <- acc * alpha + (p^T C_V of a folded tile); accd likewise for exact tiles
@@ -420,9 +397,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                                     : lc < tiles_cw ? P32 + nc32 + (lc - tiles_c) * wt
                                                     : (lc - tiles_cw) * wt;
             };
-            // q' = R_{j0}^T q of tile nn as fp16 hi / lo parts (the score MMA's B
-            // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
-            // for i = gt & 63, the only frequency this thread rotates by
+            // q' = R_{j0}^T q of tile nn in fp32, [head][dim], in the group's q'
+            // buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i) for i = gt & 63, the
+            // only frequency this thread rotates by
             // this thread's items (head h, frequency i): item gt + 128 k; their
             // query pair (q_i, q_{i+64}) stays in registers for the whole head
             float qx1[kQItems], qx2[kQItems];
@@ -434,26 +411,26 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 qx2[k] = n_first < s1 ? __bfloat162float(sq[h * d + i + 64]) : 0.f;
             }
             auto build_q = [&](int nn, float2 rv) {
-                uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQWords;
+                float* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQFloats;
 #pragma unroll
                 for (int k = 0; k < kQItems; ++k) {
-                    if (gt + 128 * k >= G * 64) break;
-                    const float y1 = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
-                    const float y2 = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
-                    const __half2 hi = __floats2half2_rn(y1, y2);
-                    const float2 hf = __half22float2(hi);
-                    const __half2 lo = __floats2half2_rn(y1 - hf.x, y2 - hf.y);
-                    qd[qoff[k][0]] = *reinterpret_cast<const uint32_t*>(&hi);
-                    qd[qoff[k][1]] = *reinterpret_cast<const uint32_t*>(&lo);
+                    const int item = gt + 128 * k;
+                    if (item >= G * 64) break;
+                    const int h = item >> 6, i = item & 63;
+                    qd[h * d + i] = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
+                    qd[h * d + 64 + i] = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
                 }
-                fence_async_smem();
             };
             auto rope_of = [&](int nn) {
                 return a.rope ? a.rope[(int64_t)tile_j0(nn) * 64 + (gt & 63)] : make_float2(1.f, 0.f);
             };
-            // two q' buffers: tile n + 2's q' is built while tile n's scores run;
-            // one buffer: each tile builds its own before its RoPE
-            if (nqb == 2 && n_first < s1) build_q(n_first, rope_of(n_first));
+            // two q' buffers: tile n + 2's q' is built during tile n (the group's
+            // softmax barrier of tile n publishes it); one buffer: each tile
+            // builds its own, then a group barrier
+            if (nqb == 2 && n_first < s1) {
+                build_q(n_first, rope_of(n_first));
+                group_sync(grp);                  // the head's first q' is visible to the group
+            }
             for (int n = n_first; n < s1; n += 2) {
                 const int st = n % ns;
                 const int local = (int)(f0 + n - hbase);
@@ -464,8 +441,15 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 const int valid = (lim - j0) < span ? (lim - j0) : span;
                 // the next tile's query rotation, loaded now, used after this tile's RoPE
                 const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
-                if (nqb == 1) build_q(n, rope_of(n));
-                // rotate this row of K^ by R_t, store back as fp16 pairs
+                if (nqb == 1) {
+                    build_q(n, rope_of(n));
+                    group_sync(grp);
+                }
+                const float* qcur = qbb + (nqb == 2 ? ((n >> 1) & 1) : 0) * kQFloats;
+                float2 sacc[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) sacc[h] = make_float2(0.f, 0.f);
+                // rotate this row of K^ by R_t and take its scores against q'
                 if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 if (win && !mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) fail();
@@ -500,57 +484,58 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     tmem_ld16(tcs + lane_base + 64 + c0, ss);
                     tmem_ld16(tcs + lane_base + 128 + c0, nn);
                     tmem_wait_ld();
-                    // (k1, k2) -> (k1 c - k2 s, k1 s + k2 c), two columns per packed
-                    // fp32 op, rounded to fp16 pairs for the score MMA
-#pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        const float2 k1 = make_float2(__uint_as_float(x1[u]), __uint_as_float(x1[u + 1]));
-                        const float2 k2 = make_float2(__uint_as_float(x2[u]), __uint_as_float(x2[u + 1]));
-                        const float2 co = make_float2(__uint_as_float(cc[u]), __uint_as_float(cc[u + 1]));
-                        const float2 si = make_float2(__uint_as_float(ss[u]), __uint_as_float(ss[u + 1]));
-                        const float2 ns = make_float2(__uint_as_float(nn[u]), __uint_as_float(nn[u + 1]));
-                        const float2 y1 = __ffma2_rn(k1, co, __fmul2_rn(k2, ns));
-                        const float2 y2 = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
-                        // column c0 + u <- fp16 (dim c0 + u, dim 64 + c0 + u): over
-                        // the fp32 columns this chunk has just read
-                        const __half2 p0 = __floats2half2_rn(y1.x, y2.x);
-                        const __half2 p1 = __floats2half2_rn(y1.y, y2.y);
-                        x1[u] = *reinterpret_cast<const uint32_t*>(&p0);
-                        x1[u + 1] = *reinterpret_cast<const uint32_t*>(&p1);
-                    }
-                    tmem_st16(kh + lane_base + c0, x1);
-                    if (c0 == 16 || c0 == 48) {
-                        // dims 0..31 and 64..95 of this row are rotated (first barrier),
-                        // then the rest (second): the score MMA starts on the first half
-                        // while the second is rotated.  One barrier per half, so every
-                        // phase counts each thread exactly once.
-                        tmem_wait_st();
+                    if (c0 == 48) {
+                        // every K^ column of this row is in registers: the issuer may
+                        // rebuild the group's next tile into the buffer
                         tc_fence_before();
-                        mbar_arrive(c0 == 16 ? &bars->krot_ready[grp] : &bars->krot_b[grp]);
+                        mbar_arrive(&bars->kfree[grp]);
+                    }
+                    // (k1, k2) -> (k1 c - k2 s, k1 s + k2 c), two columns per packed
+                    // fp32 op; then the scores of the G query heads, q' (fp32, the same
+                    // for every row) read from shared memory as broadcasts
+#pragma unroll
+                    for (int u = 0; u < 16; u += 4) {
+                        float2 y1[2], y2[2];
+#pragma unroll
+                        for (int w = 0; w < 2; ++w) {
+                            const int uu = u + 2 * w;
+                            const float2 k1 = make_float2(__uint_as_float(x1[uu]), __uint_as_float(x1[uu + 1]));
+                            const float2 k2 = make_float2(__uint_as_float(x2[uu]), __uint_as_float(x2[uu + 1]));
+                            const float2 co = make_float2(__uint_as_float(cc[uu]), __uint_as_float(cc[uu + 1]));
+                            const float2 si = make_float2(__uint_as_float(ss[uu]), __uint_as_float(ss[uu + 1]));
+                            const float2 ns = make_float2(__uint_as_float(nn[uu]), __uint_as_float(nn[uu + 1]));
+                            y1[w] = __ffma2_rn(k1, co, __fmul2_rn(k2, ns));
+                            y2[w] = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
+                        }
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float4 qa = *reinterpret_cast<const float4*>(qcur + h * d + c0 + u);
+                            const float4 qc = *reinterpret_cast<const float4*>(qcur + h * d + 64 + c0 + u);
+                            sacc[h] = __ffma2_rn(y1[0], make_float2(qa.x, qa.y), sacc[h]);
+                            sacc[h] = __ffma2_rn(y1[1], make_float2(qa.z, qa.w), sacc[h]);
+                            sacc[h] = __ffma2_rn(y2[0], make_float2(qc.x, qc.y), sacc[h]);
+                            sacc[h] = __ffma2_rn(y2[1], make_float2(qc.z, qc.w), sacc[h]);
+                        }
                     }
                 }
-                // the next tile's q' goes to the other buffer while this tile's scores run
+                // the next tile's q' goes to the other buffer (published to the group
+                // by this tile's softmax barrier)
                 if (nqb == 2 && n + 2 < s1) build_q(n + 2, rq_next);
                 // this group's previous tile: p^T C_V accumulated (before O is reused)
                 if (have_prev) {
                     if (!mbar_wait(&bars->o_full[grp], ((n - 2) >> 1) & 1, deadline)) fail();
                     tc_fence_after();
                     uint32_t o[16];
-                    tmem_ld16(kh + 144 + lane_base, o);
+                    tmem_ld16(kh + 128 + lane_base, o);
                     tmem_wait_ld();
                     accumulate(o, prev_win);
                 }
                 // scores and the tile max of each head
-                if (!mbar_wait(&bars->s_full[grp], (n >> 1) & 1, deadline)) fail();
-                tc_fence_after();
-                uint32_t sv[16];
-                tmem_ld16(kh + 128 + lane_base, sv);
-                tmem_wait_ld();
                 float sc[G];
                 bool over = false;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    const float raw = __uint_as_float(sv[h]) + __uint_as_float(sv[G + h]);
+                    const float raw = sacc[h].x + sacc[h].y;
                     sc[h] = (row < valid) ? raw * a.scale : -INFINITY;
                     range_bad |= row < valid && !(fabsf(raw) <= 3.0e38f);   // inf or NaN
                     over |= sc[h] > m_run[h] + kLazyMax;   // always true while m_run = -inf
@@ -618,7 +603,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 if (!mbar_wait(&bars->o_full[grp], (last >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 uint32_t o[16];
-                tmem_ld16(kh + 144 + lane_base, o);
+                tmem_ld16(kh + 128 + lane_base, o);
                 tmem_wait_ld();
                 accumulate(o, prev_win);
             }
@@ -751,20 +736,17 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     } else if (warp >= 10) {
         // ---------------- MMA issuer of group warp - 10 ----------------
         // per tile n of the group: K^ = C_K (B_hi + B_lo)^T (issued as soon as the
-        // group's previous score MMA has released the K^ buffer), scores once the
-        // epilogue has rotated K^ and written q', values once P is written
+        // group's epilogue has read the previous tile's K^ out of the buffer),
+        // values once P is written
         const int grp = warp - 10;
         if (lane == 0) {
             const int MV = rV <= 64 ? 64 : 128;
             const uint32_t idesc_k = idesc_f32acc(1, kTile, d, 0, 0);
-            const uint32_t idesc_s = idesc_f32acc(0, kTile, kQN, 0, 0);   // fp16 x fp16
             const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 1);
             const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 1);   // exact rows: M = d
             const uint32_t sbo_k = (uint32_t)(rK / 8) * 128;
-            const uint32_t sbo_q = (kTile / 8) * 128;
             const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
             const uint32_t kh = tmem + grp * kBufCols;
-            const uint32_t qg = smem_u32(qb + nqb * grp * kQWords);
             const uint32_t p0 = smem_u32(pb + grp * kPN * kTile);
             // K^ of tile n into this group's buffer; exact-row tiles need none
             auto recon = [&](int n, int hb, bool win) -> bool {
@@ -799,37 +781,20 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     ok = mbar_wait(&bars->bk_full[hb], (hs / nbk) & 1, deadline) &&
                          (n_first < 2 || mbar_wait(&bars->kfree[grp], ((n_first >> 1) - 1) & 1, deadline)) &&
                          recon(n_first, hb, (int)(f0 + n_first - hbase) >= tiles_c);
+                } else {
+                    // no tile of this head for the group: its release of the basis
+                    // buffer below still waits until the producer has filled the
+                    // buffer for this head, so it can never run two releases ahead
+                    // of the producer's parity wait on the same barrier
+                    ok = mbar_wait(&bars->bk_full[hb], (hs / nbk) & 1, deadline);
                 }
                 for (int n = n_first; ok && n < s1; n += 2) {
                     const int st = n % ns;
                     const bool win = (int)(f0 + n - hbase) >= tiles_c;
-                    // scores in two halves of the head dimension, each once the epilogue
-                    // has rotated it: dims 0..31 and 64..95 (k-steps 0..3, 8..11), then
-                    // 32..63 and 96..127 (k-steps 4..7, 12..15)
-                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQWords * 4);
-                    bool got = true;
-                    for (int half = 0; half < 2; ++half) {
-                        if (!mbar_wait(half ? &bars->krot_b[grp] : &bars->krot_ready[grp], (n >> 1) & 1,
-                                       deadline)) {
-                            got = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        for (int j = 0; j < 4; ++j) {
-                            const int ks = 4 * half + j;   // K = 16: 8 TMEM columns per step
-                            mma_f16_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
-                                       idesc_s, (half | j) != 0);
-                        }
-                    }
-                    if (!got) {
-                        ok = false;
-                        break;
-                    }
-                    mma_commit(&bars->s_full[grp]);
-                    mma_commit(&bars->kfree[grp]);
-                    // K_rot of tile n consumed: rebuild tile n + 2 while the epilogue runs
-                    // this tile's softmax.  Its data sits in stage (n + 2) % ns, which with
-                    // two stages is tile n's own: then it has to wait for value(n) below.
+                    // K^ of tile n read by the epilogue: rebuild tile n + 2 while the
+                    // epilogue computes this tile's scores and softmax.  Its data sits in
+                    // stage (n + 2) % ns, which with two stages is tile n's own: then it
+                    // has to wait for value(n) below.
                     auto next_recon = [&]() {
                         return mbar_wait(&bars->kfree[grp], (n >> 1) & 1, deadline) &&
                                recon(n + 2, hb, (int)(f0 + n + 2 - hbase) >= tiles_c);
@@ -846,13 +811,13 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     if (!win) {
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
                         for (int ks = 0; ks < kTile / 16; ++ks)
-                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
+                            mma_f16_ss(kh + 128, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
                     } else {
                         // O = V^T P over wt exact rows: A = V tile, MN-major, M = d
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + win_bytes);
                         for (int ks = 0; ks < wt / 16; ++ks)
-                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
+                            mma_f16_ss(kh + 128, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_ow, ks != 0);
                     }
                     mma_commit(&bars->o_full[grp]);

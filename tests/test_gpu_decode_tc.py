@@ -113,3 +113,22 @@ def test_tc_decode_without_folded_rows():
     out_c = pc.cache.decode_attention(0, q.cuda()).cpu().numpy()
     assert max(errs.values()) < 1e-3, errs
     assert rel_err(out_t, out_c) < 5e-3
+
+
+def test_tc_decode_single_basis_buffer_heads_split_across_runs():
+    """r_K 64, r_V 96 leave room for one basis buffer; at this shape (16 heads
+    of 49 tiles on 148 SMs) eight CTA runs end with a head of which they hold
+    a single tile, so one epilogue group has no tile there.  That group's
+    release of the basis buffer must stay behind the producer's refill (an
+    early second release would look like no release to the producer's parity
+    wait): the decode completes with status OK and matches the oracle."""
+    cfg = _cfg(batch=2, kv_heads=8, q_heads=32, rank_k=64, rank_v=96, window=256,
+               max_tokens=6144)
+    p = _pair(True, cfg, seed=49)
+    p.prefill(5864, chunk=64, defer_every=16)
+    T, n_c = p.cache.counts(0)
+    assert (T, n_c) == (5864, 5568)
+    for _ in range(2):
+        errs, _ = p.decode(0, p.query())
+        assert max(errs.values()) < TOL_BF16, errs
+    assert p.cache.status() == 0

@@ -15,13 +15,16 @@ oracle, which emulates the bf16 rounding at every rewrite:
 
 Beside the kernel error the test reports the format drift: the same oracle
 run with float64 coefficient storage against the bf16-emulating one (what
-bf16 storage itself costs, separate from kernel error).  Tolerance 2e-2 on
-reconstructions C B^T and decode outputs, counters exact.
+bf16 storage itself costs, separate from kernel error).  Bars (derived in
+_report_and_check): reconstructions C B^T within 2e-2 of the bf16-emulating
+oracle, or twice the format drift once the drift is larger; no farther from
+the float64-storage result than 1.5 x the drift + 2e-3; decode outputs within
+2e-2; counters exact.
 """
 
 import pytest
 
-from iskv_testlib import SampledCache
+from iskv_testlib import SampledCache, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -44,12 +47,33 @@ def _cfg(**kw):
     return c
 
 
+def _recon_errors(s):
+    """Worst rel_err of the GPU reconstructions against the bf16-emulating
+    oracle and against the float64-storage oracle, and the format drift
+    (bf16-emulating against float64 storage), over the sampled heads."""
+    ik = s.ik
+    e_b = e_64 = drift = 0.0
+    T, n_c = s.cache.counts(0)
+    for which, of, sf in ((ik.WHICH_K, s.ok, s.sk), (ik.WHICH_V, s.ov, s.sv)):
+        got = s.cache.reconstruct(0, which)
+        for x in s.sample:
+            assert (T, n_c) == (of[x].T, of[x].n_c)
+            g = got[x[1], x[2]].cpu().numpy()
+            want_b, want_64 = of[x].reconstruct(), sf[x].reconstruct()
+            e_b = max(e_b, rel_err(g, want_b))
+            e_64 = max(e_64, rel_err(g, want_64))
+            drift = max(drift, rel_err(want_b, want_64))
+        del got
+    return e_b, e_64, drift
+
+
 def _chain(s, folds, check_every):
     """`folds` decode periods: 64 tokens appended in four steps (a decode
     check after the first every `check_every` periods), then one fold with
     the rewrite of every stored row.  Returns the table of worst errors."""
     rows = []
     for i in range(1, folds + 1):
+        dec = None
         for part in range(4):
             s.append(16)
             if part == 0 and i % check_every == 0:
@@ -57,17 +81,28 @@ def _chain(s, folds, check_every):
         assert s.ready() == 1
         s.fold_all(defer=False)
         if i % check_every == 0 or i == folds:
-            rec = s.check(tol=TOL)
-            dec = s.decode_check(tol=TOL)
-            rows.append((i, rec, dec, s.format_drift()))
+            e_b, e_64, drift = _recon_errors(s)
+            rows.append((i, e_b, e_64, drift, dec if dec is not None else s.decode_check(tol=TOL)))
     return rows
 
 
-def _report(name, rows):
+def _report_and_check(name, rows):
+    """Print the table, then check it.  Two bf16 chains fed values that differ
+    at fp32 level (the GPU folds in fp32, the oracle in fp64) round apart now
+    and then, and each such step persists through later rewrites, so the
+    distance between them grows with the number of rewrites the way the format
+    drift does.  The bars: within 2e-2 of the bf16-emulating oracle, or of
+    twice the measured format drift once that is larger; and no farther from
+    the float64-storage result than 1.5 x the format drift + 2e-3 (the GPU's
+    own chain drifts no more than the emulated one); decode within 2e-2."""
     print(f"\n{name}: per-fold rewrites against the oracle")
-    print(" folds  recon-err  decode-err  format-drift(bf16 vs fp64 storage)")
-    for i, rec, dec, drift in rows:
-        print(f" {i:5d}  {rec:9.2e}  {dec:10.2e}  {drift:9.2e}")
+    print(" folds  vs-bf16-oracle  vs-fp64-oracle  format-drift  decode")
+    for i, e_b, e_64, drift, dec in rows:
+        print(f" {i:5d}  {e_b:14.2e}  {e_64:14.2e}  {drift:12.2e}  {dec:8.2e}")
+    for i, e_b, e_64, drift, dec in rows:
+        assert e_b < max(TOL, 2 * drift), (i, e_b, drift)
+        assert e_64 < 1.5 * drift + 2e-3, (i, e_64, drift)
+        assert dec < TOL, (i, dec)
 
 
 def test_per_fold_rewrites_qwen3_geometry_256_folds():
@@ -77,7 +112,7 @@ def test_per_fold_rewrites_qwen3_geometry_256_folds():
     s.prefill(16384)
     s.check(tol=TOL)
     rows = _chain(s, 256, 32)
-    _report("qwen3 1 layer, batch 8, r_K 32, r_V 64", rows)
+    _report_and_check("qwen3 1 layer, batch 8, r_K 32, r_V 64", rows)
     T, n_c = s.cache.counts(0)
     assert n_c == 16384 - 1024 + 256 * 64
     assert s.cache.status() == 0
@@ -90,5 +125,5 @@ def test_per_fold_rewrites_cot_ranks_256_folds():
     s.prefill(8192)
     s.check(tol=TOL)
     rows = _chain(s, 256, 32)
-    _report("cot 1 layer, batch 1, r_K 64, r_V 96", rows)
+    _report_and_check("cot 1 layer, batch 1, r_K 64, r_V 96", rows)
     assert s.cache.status() == 0
