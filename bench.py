@@ -44,6 +44,16 @@ WORKLOADS = {
                             window=1024, prefill=32768, coef="bf16", gen="qwen3"),
     "qwen3-1L-b1-16k": dict(batch=1, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
                             window=1024, prefill=16384, coef="f32", gen="qwen3"),
+    # one factor per sequence over its 8 KV heads (D = 1024) at the explainer's
+    # worked-example ranks for Qwen3-8B (r_K 64, r_V 96)
+    "qwen3-1L-b8-32k-joint": dict(batch=8, layers=1, kv_heads=8, q_heads=32, rank_k=64,
+                                  rank_v=96, window=1024, prefill=32768, coef="bf16",
+                                  gen="qwen3", joint=1),
+    # low-bit latent-channel codes: K 16 ch x 8 b + 16 x 4 b, V 16 x 8 + 16 x 4 + 32 x 2
+    "qwen3-1L-b8-32k-codes": dict(batch=8, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
+                                  window=1024, prefill=32768, coef="codes", gen="qwen3",
+                                  quant_k=((16, 8), (16, 4)),
+                                  quant_v=((16, 8), (16, 4), (32, 2))),
 }
 # Long chain-of-thought growth: 36 layers, batch 1, grown from 8K to 128K
 # tokens; timed at each context bin, 30% of the decode steps carry queries
@@ -75,9 +85,9 @@ DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of on
 
 # What the path computes in: storage, tensor-core operand and accumulator types.
 PRECISION = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: bf16 MMA rebuilds keys "
-             "(basis as bf16 hi+lo) into fp32, rotated keys rounded to fp16, scores by fp16 "
-             "MMA with fp16 hi+lo queries, p as bf16 hi+lo, fp32 softmax and accumulators; "
-             "rewrite: bf16 MMA with an fp32-exact 3-part split of W_top; fold: fp32")
+             "(basis as bf16 hi+lo) into fp32, RoPE and scores in fp32 on CUDA cores, p as "
+             "bf16 hi+lo for the value MMA, fp32 softmax and accumulators; rewrite: bf16 MMA "
+             "with an fp32-exact 3-part split of W_top; fold: fp32")
 
 
 def _peaks():
@@ -267,6 +277,7 @@ def run_iskv(args, rank, world, local_rank):
     L, Bsz, H, Hq = wl["layers"], wl["batch"], wl["kv_heads"], wl["q_heads"]
     g = Hq // H
     coef = ik.BF16 if wl["coef"] == "bf16" else ik.F32
+    codes = wl["coef"] == "codes"
     e2e_periods = max(1, args.steps // 2)
     measure_periods = 1
     periods = args.warmup + args.steps + e2e_periods + measure_periods
@@ -275,7 +286,9 @@ def run_iskv(args, rank, world, local_rank):
     cfg = ik.Config(batch=Bsz, layers=L, kv_heads=H, q_heads=Hq, rank_k=wl["rank_k"],
                     rank_v=wl["rank_v"], window=wl["window"], max_tokens=max_tokens,
                     kv_dtype=ik.BF16, coef_dtype=coef, use_rope=1, rope_theta=1e6,
-                    max_deferred=64, protect=args.protect)
+                    max_deferred=64, protect=args.protect, joint=wl.get("joint", 0),
+                    coef_quant=1 if codes else 0, quant_k=wl.get("quant_k", ()),
+                    quant_v=wl.get("quant_v", ()))
     cache = ik.Cache(cfg)
     P = args.protect
     kdt = torch.bfloat16
@@ -390,12 +403,20 @@ def run_iskv(args, rank, world, local_rank):
     peak, peak_src = _peaks()
     dsum, bsum = 0.0, 0.0
     kvb, cb = 2, (2 if coef == ik.BF16 else 4)
+    rs = wl["rank_k"] + wl["rank_v"]
+    row_bytes = rs * cb   # one coefficient row of K and V
+    if codes:
+        # codes (bits x channels per group) and one fp32 scale per coded group
+        row_bytes = sum(n * b // 8 + (4 if b else 0) for n, b in wl["quant_k"] + wl["quant_v"])
     for e0, e1, T, n_c in dec_events:
         t = e0.elapsed_time(e1) / 1e3
         n_w = T - n_c
-        per_head = (n_c * (wl["rank_k"] + wl["rank_v"]) * cb + 2 * n_w * D * kvb
-                    + D * (wl["rank_k"] + wl["rank_v"]) * 4)
-        byts = Bsz * H * per_head + Bsz * Hq * D * (kvb + 4)
+        if wl.get("joint"):
+            # coefficients once per sequence, bases and exact rows per KV head
+            byts = Bsz * n_c * row_bytes + Bsz * H * (2 * n_w * D * kvb + D * rs * 4)
+        else:
+            byts = Bsz * H * (n_c * row_bytes + 2 * n_w * D * kvb + D * rs * 4)
+        byts += Bsz * Hq * D * (kvb + 4)
         dsum += t
         bsum += byts
     dec_avg_us = dsum / max(1, len(dec_events)) * 1e6
@@ -458,10 +479,13 @@ def run_iskv(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate" if coef == ik.BF16
+        "dtype": "mixed: bf16 MMA inputs, fp32 accumulate and scores" if coef == ik.BF16
+                 else "fp32 math on bf16 K/V and latent-channel codes" if codes
                  else "fp32 math on bf16 K/V, fp32 coefficients",
         "precision": PRECISION if coef == ik.BF16 else "bf16 K/V in HBM, fp32 coefficients "
-                     "and bases, fp32 CUDA-core math throughout",
+                     "and bases, fp32 CUDA-core math throughout" if not codes else
+                     "bf16 K/V in HBM, coefficients as 8/4/2-bit latent-channel codes with fp32 "
+                     "scales per row and group, fp32 CUDA-core decode",
         "data": "synthetic",
         "config": {
             "workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H, "q_heads": Hq,
@@ -483,7 +507,7 @@ def run_iskv(args, rank, world, local_rank):
         "prefill_s": prefill_s,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.workload)
-                     if coef == ik.BF16 and P == 0 else None,
+                     if coef == ik.BF16 and P == 0 and not codes else None,
                      "traffic_source": DECODE_TRAFFIC_SOURCE,
                      "kernel": "decode_tc_kernel (persistent split-K decode attention, "
                                "per-head combine fused), one launch per layer call",

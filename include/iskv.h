@@ -67,10 +67,9 @@ extern "C" {
                                       destroy the cache: its decode bookkeeping
                                       may be left inconsistent)             */
 #define ISKV_ERR_RANGE         -9  /* a score of the tensor-core decode was not
-                                      finite: a rotated key or a query went
-                                      beyond fp16's range (|x| >= 65504), the
-                                      type its score MMA takes (sticky; that
-                                      call's outputs are not finite)        */
+                                      finite: an inf or NaN key or query, or
+                                      a product beyond fp32's range (sticky;
+                                      that call's outputs are not finite)   */
 
 /* ---- element types ----------------------------------------------------- */
 #define ISKV_F32   0
@@ -87,6 +86,27 @@ extern "C" {
 #define ISKV_FOLD_DEFER_SYNC 1
 
 typedef struct iskv_cache* iskv_t;
+
+/* Low-bit coefficient codes in latent channels: the SVDq page ("SVDq:
+ * 1.25-bit and 410x Key Cache Compression for LLM Attention", Abstract) keeps
+ * a key cache in SVD latent channels and gives the more significant channels
+ * more bits; the iS-KV explainer (body paragraph on GQA and quantization)
+ * calls iS-KV combined with low-bit storage untried.  Here column c of a
+ * factor's coefficients C is latent channel c (columns are kept in
+ * descending singular-value order), and each coefficient row is stored per
+ * group of channels: group g covers `channels[g]` channels from the end of
+ * the previous group, with `bits[g]` bits per code (0: the channels are
+ * dropped and read as zero; 2, 4 or 8 otherwise).  Per row and group, in
+ * fp32: scale = max |x| / (2^(b-1) - 1) (0 for an all-zero group), code =
+ * x / scale rounded half to even into [-(2^(b-1) - 1), 2^(b-1) - 1], stored
+ * as code + 2^(b-1) - 1 in b bits, packed from the lowest bit of 32-bit words
+ * upward, each group starting a new word; the stored value is code * scale.
+ * Channels per group are multiples of 16, their sum is the factor's rank.   */
+typedef struct {
+    int32_t groups;         /* 1..4 groups, from latent channel 0 on        */
+    int32_t channels[4];    /* channels of each group (multiples of 16)     */
+    int32_t bits[4];        /* bits per code: 0, 2, 4 or 8                  */
+} iskv_quant_format;
 
 /* Shape and format of one cache (a batch of equal-length sequences, every
  * layer of a model).  head_dim must be 128 and block 64 in this build.      */
@@ -119,6 +139,20 @@ typedef struct {
                                the paint-shop section) leaves some prompt
                                positions uncompressed, besides the recent
                                window.                                      */
+    int32_t coef_quant;     /* 1: coefficients stored as low-bit latent-channel
+                               codes (quant_k, quant_v) instead of coef_dtype;
+                               every new row and every rewrite is coded again,
+                               and decode reads the codes (CUDA-core path)   */
+    iskv_quant_format quant_k;  /* code groups of the K factor (ranks sum to r_K) */
+    iskv_quant_format quant_v;  /* code groups of the V factor (ranks sum to r_V) */
+    int32_t joint;          /* 1: one K and one V factor per sequence and layer
+                               over all its KV heads, whose rows sit side by
+                               side (D = kv_heads * 128 <= 1024; the reading
+                               of the explainer's worked-example ranks 64, 96
+                               and 128 as layer-wide ranks); coefficients are
+                               then shared by the heads and each head decodes
+                               with its 128 rows of the basis.  0: one factor
+                               per KV head.                                 */
 } iskv_config;
 
 /* Fill `cfg` with the defaults of the one-layer Qwen3-8B-shaped cache
@@ -195,7 +229,8 @@ ISKV_API int iskv_reconstruct(iskv_t h, int layer, int which, float* out, void* 
 
 /* Copy out one factor: basis [batch, kv_heads, head_dim, r] fp32 (row i of a
  * head is basis row i), sigma [batch, kv_heads, r] fp32, coef
- * [batch, kv_heads, n_c, r] in coef_dtype.  Any pointer may be NULL.        */
+ * [batch, kv_heads, n_c, r] row-major in coef_dtype (fp32 values code * scale
+ * for a coef_quant cache).  Any pointer may be NULL.                       */
 ISKV_API int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
                      void* coef, void* stream);
 
@@ -212,6 +247,18 @@ ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
  * or temporary buffers.  Either pointer may be NULL.  Host only, no GPU work.
  * Errors: INVALID_ARG for a NULL cache.                                    */
 ISKV_API int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes);
+
+/* Code `n` fp32 rows of `rank` coefficients with the latent-channel format
+ * `fmt` (see iskv_quant_format): rows [n][rank] fp32, codes [n][words]
+ * uint32 (words = iskv_quant_words(fmt)), scales [n][4] fp32 (unused groups
+ * 0).  Device pointers; enqueued on `stream`.  The same device routine codes
+ * a cache's new rows and rewrites, so callers can prepare or check codes
+ * outside a cache.  Errors: INVALID_ARG (format, rank or pointers), CUDA.   */
+ISKV_API int iskv_quantize_rows(const iskv_quant_format* fmt, int rank, const float* rows,
+                                int64_t n, uint32_t* codes, float* scales, void* stream);
+
+/* 32-bit code words per row of a format (host only); -1 if invalid.        */
+ISKV_API int iskv_quant_words(const iskv_quant_format* fmt);
 
 /* Synchronize the device and return the cache's sticky device status, the
  * most severe first: ISKV_ERR_CUDA, ISKV_ERR_DEVICE_TIMEOUT, ISKV_ERR_RANGE,

@@ -16,8 +16,9 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["Config", "Cache", "IskvError", "DecodeOperands", "lib_path", "LIB", "F32", "BF16",
-           "WHICH_K", "WHICH_V", "ALL_LAYERS", "FOLD_DEFER_SYNC", "EXPORTED"]
+__all__ = ["Config", "Cache", "IskvError", "DecodeOperands", "QuantFormat", "quantize_rows",
+           "lib_path", "LIB", "F32", "BF16", "WHICH_K", "WHICH_V", "ALL_LAYERS", "FOLD_DEFER_SYNC",
+           "EXPORTED"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -51,12 +52,30 @@ class IskvError(RuntimeError):
         super().__init__(f"{where}: ISKV_ERR_{self.name} ({msg})")
 
 
+class QuantFormat(ctypes.Structure):
+    """Mirror of ``iskv_quant_format``: latent-channel code groups."""
+    _fields_ = [("groups", ctypes.c_int32), ("channels", ctypes.c_int32 * 4),
+                ("bits", ctypes.c_int32 * 4)]
+
+    @classmethod
+    def of(cls, groups):
+        """From a list of (channels, bits) pairs, first latent channel first."""
+        q = cls()
+        q.groups = len(groups)
+        for i, (n, b) in enumerate(groups):
+            q.channels[i] = int(n)
+            q.bits[i] = int(b)
+        return q
+
+
 class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "layers", "kv_heads", "q_heads", "head_dim", "rank_k", "rank_v", "window",
         "block", "max_tokens", "kv_dtype", "coef_dtype", "use_rope")] + [
         ("rope_theta", ctypes.c_double)] + [(n, ctypes.c_int32) for n in (
-            "sync", "max_deferred", "jacobi_max_sweeps", "ring_extra", "protect")]
+            "sync", "max_deferred", "jacobi_max_sweeps", "ring_extra", "protect",
+            "coef_quant")] + [("quant_k", QuantFormat), ("quant_v", QuantFormat)] + [
+        ("joint", ctypes.c_int32)]
 
 
 class DecodeOperands(ctypes.Structure):
@@ -85,6 +104,8 @@ _SIGS = {
     "iskv_status": ([_vp], _i),
     "iskv_strerror": ([_i], ctypes.c_char_p),
     "iskv_decode_attention_noalloc": ([ctypes.POINTER(DecodeOperands), _vp, _vp, _vp], _i),
+    "iskv_quantize_rows": ([ctypes.POINTER(QuantFormat), _i, _vp, ctypes.c_int64, _vp, _vp, _vp], _i),
+    "iskv_quant_words": ([ctypes.POINTER(QuantFormat)], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(LIB, _name)
@@ -135,10 +156,19 @@ class Config:
     jacobi_max_sweeps: int = 0
     ring_extra: int = 0
     protect: int = 0
+    coef_quant: int = 0
+    quant_k: tuple = ()        # ((channels, bits), ...) of the K factor's code groups
+    quant_v: tuple = ()
+    joint: int = 0             # 1: one factor per sequence over all KV heads (D = kv_heads*128)
 
     def _c(self) -> _Cfg:
         c = _Cfg()
         for f in _Cfg._fields_:
+            if f[0] in ("quant_k", "quant_v"):
+                groups = getattr(self, f[0])
+                if groups:
+                    setattr(c, f[0], QuantFormat.of(groups))
+                continue
             setattr(c, f[0], getattr(self, f[0]))
         return c
 
@@ -228,13 +258,20 @@ class Cache:
         return out
 
     def factors(self, layer: int, which: int, stream=None, device="cuda"):
-        """(basis [B,H,d,r] fp32, sigma [B,H,r] fp32, coef [B,H,n_c,r])."""
+        """(basis [B,H,d,r] fp32, sigma [B,H,r] fp32, coef [B,H,n_c,r]); for a
+        joint-head cache (basis [B,H*d,r], sigma [B,r], coef [B,n_c,r])."""
         c = self.cfg
         r = c.rank_k if which == WHICH_K else c.rank_v
         n_c = self.counts(layer)[1]
-        basis = torch.empty(c.batch, c.kv_heads, c.head_dim, r, dtype=torch.float32, device=device)
-        sigma = torch.empty(c.batch, c.kv_heads, r, dtype=torch.float32, device=device)
-        coef = torch.empty(c.batch, c.kv_heads, n_c, r, dtype=c.coef_torch_dtype, device=device)
+        cdt = torch.float32 if c.coef_quant else c.coef_torch_dtype   # coded: values code * scale
+        if c.joint:
+            basis = torch.empty(c.batch, c.kv_heads * c.head_dim, r, dtype=torch.float32, device=device)
+            sigma = torch.empty(c.batch, r, dtype=torch.float32, device=device)
+            coef = torch.empty(c.batch, n_c, r, dtype=cdt, device=device)
+        else:
+            basis = torch.empty(c.batch, c.kv_heads, c.head_dim, r, dtype=torch.float32, device=device)
+            sigma = torch.empty(c.batch, c.kv_heads, r, dtype=torch.float32, device=device)
+            coef = torch.empty(c.batch, c.kv_heads, n_c, r, dtype=cdt, device=device)
         _check(LIB.iskv_get_factors(self._h, layer, which, _ptr(basis), _ptr(sigma),
                                     _ptr(coef) if n_c else None, _stream(stream)),
                "iskv_get_factors")
@@ -255,3 +292,21 @@ class Cache:
 
     def status(self) -> int:
         return LIB.iskv_status(self._h)
+
+
+def quantize_rows(groups, rows: torch.Tensor, stream=None):
+    """Code fp32 rows [n, rank] (device) with the latent-channel format
+    ``groups`` = ((channels, bits), ...): returns (codes [n, words] int32
+    holding the uint32 words, scales [n, 4] fp32)."""
+    fmt = QuantFormat.of(groups)
+    words = LIB.iskv_quant_words(ctypes.byref(fmt))
+    if words < 0:
+        raise ValueError(f"invalid code format {groups}")
+    if rows.dtype != torch.float32 or rows.dim() != 2:
+        raise TypeError("rows must be a 2-d fp32 tensor")
+    n, rank = rows.shape
+    codes = torch.zeros(n, words, dtype=torch.int32, device=rows.device)
+    scales = torch.zeros(n, 4, dtype=torch.float32, device=rows.device)
+    _check(LIB.iskv_quantize_rows(ctypes.byref(fmt), rank, _ptr(rows), n, _ptr(codes), _ptr(scales),
+                                  _stream(stream)), "iskv_quantize_rows")
+    return codes, scales

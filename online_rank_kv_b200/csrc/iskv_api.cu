@@ -28,6 +28,7 @@ struct iskv_cache {
     int64_t cap = 0;      // ring rows per head
     int64_t n_max = 0;    // coefficient rows per head
     int BH = 0;
+    int FH = 0;           // factor instances per layer: BH, or batch for joint-head factors
     int D = 1;            // postponed-fold slots per head
     int kv_bytes = 4, coef_bytes = 4;
     // device memory
@@ -49,6 +50,14 @@ struct iskv_cache {
     float* qscr_k = nullptr;      // fold scratch: Q of every (layer, head)
     float* qscr_v = nullptr;
     int* seg_rows = nullptr;
+    // latent-channel codes (coef_quant): codes, scales and the fold's fp32 new rows
+    uint32_t* qcodes_k = nullptr;
+    uint32_t* qcodes_v = nullptr;
+    float* qscales_k = nullptr;
+    float* qscales_v = nullptr;
+    float* newrows_k = nullptr;
+    float* newrows_v = nullptr;
+    float* wide = nullptr;        // joint-head fold scratch
     float* partial = nullptr;
     int* done = nullptr;          // per-head arrival counters of the fused decode combine
     float2* rope = nullptr;
@@ -87,6 +96,34 @@ struct TraceRange {
 constexpr size_t kStageBytes = 16u << 20;
 constexpr bool kDecodeTcDefault = true;
 
+// Fill the code-format fields of a view from `q` for rank r; false if the
+// format is invalid (groups 1..4, channels multiples of 16 summing to r, bits
+// 0, 2, 4 or 8, at least one group with codes).
+bool quant_fill(const iskv_quant_format& q, int r, FactorView* f) {
+    if (q.groups < 1 || q.groups > 4) return false;
+    int lo = 0, word = 0, coded = 0;
+    for (int g = 0; g < 4; ++g) {
+        f->qbits[g] = 0;
+        f->qlo[g] = f->qhi[g] = r;
+        f->qword0[g] = 0;
+    }
+    for (int g = 0; g < q.groups; ++g) {
+        const int n = q.channels[g], b = q.bits[g];
+        if (n < 16 || n % 16 != 0 || !(b == 0 || b == 2 || b == 4 || b == 8)) return false;
+        f->qbits[g] = b;
+        f->qlo[g] = lo;
+        f->qhi[g] = lo + n;
+        f->qword0[g] = word;
+        lo += n;
+        word += n * b / 32;
+        coded += b > 0;
+    }
+    if (lo != r || coded == 0) return false;
+    f->qgroups = q.groups;
+    f->qwords = word;
+    return true;
+}
+
 bool is_device_ptr(const void* p) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
@@ -116,6 +153,14 @@ int validate(const iskv_config* c) {
     if (c->jacobi_max_sweeps < 0 || c->jacobi_max_sweeps > 1000) return ISKV_ERR_INVALID_ARG;
     if (c->ring_extra < 0 || c->ring_extra % kBlock != 0) return ISKV_ERR_INVALID_ARG;
     if (c->protect < 0 || c->protect > c->max_tokens) return ISKV_ERR_INVALID_ARG;
+    if (c->coef_quant != 0 && c->coef_quant != 1) return ISKV_ERR_INVALID_ARG;
+    if (c->joint != 0 && c->joint != 1) return ISKV_ERR_INVALID_ARG;
+    if (c->joint && (c->kv_heads * kHeadDim > 1024 || c->coef_quant)) return ISKV_ERR_UNSUPPORTED;
+    if (c->coef_quant) {
+        FactorView f{};
+        if (!quant_fill(c->quant_k, c->rank_k, &f) || !quant_fill(c->quant_v, c->rank_v, &f))
+            return ISKV_ERR_INVALID_ARG;
+    }
     return ISKV_OK;
 }
 
@@ -141,6 +186,27 @@ FactorView view(const iskv_cache* h, int which) {
     f.cap = h->cap;
     f.D = h->D;
     f.BH = h->BH;
+    f.coef_div = h->cfg.joint ? h->cfg.kv_heads : 1;
+    f.wide = h->wide;
+    if (h->cfg.coef_quant) {
+        f.quant = 1;
+        f.coef_bf16 = 0;
+        f.coef_blocked = 0;
+        quant_fill(K ? h->cfg.quant_k : h->cfg.quant_v, f.r, &f);
+        f.qcodes = K ? h->qcodes_k : h->qcodes_v;
+        f.qscales = K ? h->qscales_k : h->qscales_v;
+        f.newrows = K ? h->newrows_k : h->newrows_v;
+    }
+    return f;
+}
+
+// The view of the per-factor arrays (coefficients, sigma, postponed W_top) with
+// one instance per factor: kernels that never touch a head's basis rows or
+// exact rows (rewrite, composition, coefficient copies) take this one.
+FactorView view_factors(const iskv_cache* h, int which) {
+    FactorView f = view(h, which);
+    f.BH = h->FH;
+    f.coef_div = 1;
     return f;
 }
 
@@ -173,7 +239,9 @@ void free_all(iskv_cache* h) {
     free_events(h);
     void* ptrs[] = {h->ring_k, h->ring_v, h->prot_k, h->prot_v, h->coef_k, h->coef_v, h->basis_k, h->basis_v,
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
-                    h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out};
+                    h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out,
+                    h->qcodes_k, h->qcodes_v, h->qscales_k, h->qscales_v, h->newrows_k, h->newrows_v,
+                    h->wide};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -235,9 +303,11 @@ int run_resync(iskv_cache* h, const std::vector<int>& layers, const std::vector<
     bool chained = false;
     for (int i = 0; i < rl.n_tasks; ++i) chained = chained || rl.n_seg[i] > 1;
     for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) {
-        FactorView f = view(h, which);
+        FactorView f = view_factors(h, which);
         if (chained) CU(launch_compose(f, rl, s));
-        if (f.coef_blocked)
+        if (f.quant)
+            CU(launch_resync_quant(f, rl, s));
+        else if (f.coef_blocked)
             CU(launch_resync_tc(f, rl, h->status, s));
         else
             CU(launch_resync(f, rl, s));
@@ -291,6 +361,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     }
     const iskv_config& c = h->cfg;
     h->BH = c.batch * c.kv_heads;
+    h->FH = c.joint ? c.batch : h->BH;
     h->cap = (int64_t)c.window + kBlock + c.ring_extra;
     h->pcap = ((int64_t)c.protect + kBlock - 1) / kBlock * kBlock;
     int64_t nm = (int64_t)c.max_tokens - c.window;
@@ -298,7 +369,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     h->n_max = (nm / kBlock) * kBlock + 2 * kBlock;   // slack rows for whole tiles
     h->D = c.max_deferred > 0 ? c.max_deferred : 1;
     h->kv_bytes = c.kv_dtype == ISKV_BF16 ? 2 : 4;
-    h->coef_bytes = c.coef_dtype == ISKV_BF16 ? 2 : 4;
+    h->coef_bytes = c.coef_quant ? 4 : (c.coef_dtype == ISKV_BF16 ? 2 : 4);   // as copied out
     {
         // tensor-core decode over folded rows: on unless ISKV_TENSOR_CORES=0
         const char* env = std::getenv("ISKV_TENSOR_CORES");
@@ -314,6 +385,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     h->upd_evt.assign(c.layers, nullptr);
 
     const size_t heads = (size_t)c.layers * h->BH;
+    const size_t facs = (size_t)c.layers * h->FH;   // factor instances (coefficients, W_top)
     const size_t d = kHeadDim;
     size_t ring_bytes = heads * h->cap * d * h->kv_bytes;
     rc = ISKV_OK;
@@ -329,18 +401,38 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         rc = rc ? rc : dalloc(&h->prot_k, prot_bytes);
         rc = rc ? rc : dalloc(&h->prot_v, prot_bytes);
     }
-    rc = rc ? rc : dalloc(&h->coef_k, heads * h->n_max * c.rank_k * h->coef_bytes);
-    rc = rc ? rc : dalloc(&h->coef_v, heads * h->n_max * c.rank_v * h->coef_bytes);
+    const size_t coef_k_bytes = c.coef_quant ? 0 : facs * h->n_max * c.rank_k * h->coef_bytes;
+    const size_t coef_v_bytes = c.coef_quant ? 0 : facs * h->n_max * c.rank_v * h->coef_bytes;
+    rc = rc ? rc : dalloc(&h->coef_k, coef_k_bytes);
+    rc = rc ? rc : dalloc(&h->coef_v, coef_v_bytes);
+    size_t qk_bytes = 0, qv_bytes = 0, qs_bytes = 0;
+    if (c.coef_quant) {
+        FactorView fk{}, fv{};
+        quant_fill(c.quant_k, c.rank_k, &fk);
+        quant_fill(c.quant_v, c.rank_v, &fv);
+        qk_bytes = heads * h->n_max * fk.qwords * 4;
+        qv_bytes = heads * h->n_max * fv.qwords * 4;
+        qs_bytes = heads * h->n_max * 4 * sizeof(float);
+        rc = rc ? rc : dalloc(&h->qcodes_k, qk_bytes);
+        rc = rc ? rc : dalloc(&h->qcodes_v, qv_bytes);
+        rc = rc ? rc : dalloc(&h->qscales_k, qs_bytes);
+        rc = rc ? rc : dalloc(&h->qscales_v, qs_bytes);
+        rc = rc ? rc : dalloc(&h->newrows_k, heads * kBlock * c.rank_k * sizeof(float));
+        rc = rc ? rc : dalloc(&h->newrows_v, heads * kBlock * c.rank_v * sizeof(float));
+    }
     rc = rc ? rc : dalloc(&h->basis_k, heads * d * c.rank_k * 4);
     rc = rc ? rc : dalloc(&h->basis_v, heads * d * c.rank_v * 4);
     rc = rc ? rc : dalloc(&h->bsplit_k, heads * 2 * d * c.rank_k * 2);
     rc = rc ? rc : dalloc(&h->bsplit_v, heads * 2 * d * c.rank_v * 2);
     rc = rc ? rc : dalloc(&h->sigma_k, heads * c.rank_k * 4);
     rc = rc ? rc : dalloc(&h->sigma_v, heads * c.rank_v * 4);
-    rc = rc ? rc : dalloc(&h->pend_k, heads * h->D * (size_t)c.rank_k * c.rank_k * 4);
-    rc = rc ? rc : dalloc(&h->pend_v, heads * h->D * (size_t)c.rank_v * c.rank_v * 4);
-    rc = rc ? rc : dalloc(&h->qscr_k, heads * d * fold_q_cols(c.rank_k) * 4);
-    rc = rc ? rc : dalloc(&h->qscr_v, heads * d * fold_q_cols(c.rank_v) * 4);
+    rc = rc ? rc : dalloc(&h->pend_k, facs * h->D * (size_t)c.rank_k * c.rank_k * 4);
+    rc = rc ? rc : dalloc(&h->pend_v, facs * h->D * (size_t)c.rank_v * c.rank_v * 4);
+    rc = rc ? rc : dalloc(&h->qscr_k, c.joint ? 0 : heads * d * fold_q_cols(c.rank_k) * 4);
+    rc = rc ? rc : dalloc(&h->qscr_v, c.joint ? 0 : heads * d * fold_q_cols(c.rank_v) * 4);
+    if (c.joint)   // one scratch for K and V: their folds run one after the other
+        rc = rc ? rc : dalloc(&h->wide, facs * fold_wide_scratch_floats(c.kv_heads * kHeadDim,
+                                                                        std::max(c.rank_k, c.rank_v)) * 4);
     rc = rc ? rc : dalloc(&h->seg_rows, (size_t)c.layers * h->D * 4);
     rc = rc ? rc : dalloc(&h->partial, (size_t)c.batch * c.q_heads * h->max_splits *
                                            (2 + c.rank_v + d) * 4);
@@ -374,8 +466,12 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
             cudaMemsetAsync(h->ring_v, 0, ring_bytes, s) != cudaSuccess ||
             (prot_bytes > 0 && (cudaMemsetAsync(h->prot_k, 0, prot_bytes, s) != cudaSuccess ||
                                 cudaMemsetAsync(h->prot_v, 0, prot_bytes, s) != cudaSuccess)) ||
-            cudaMemsetAsync(h->coef_k, 0, heads * h->n_max * c.rank_k * h->coef_bytes, s) != cudaSuccess ||
-            cudaMemsetAsync(h->coef_v, 0, heads * h->n_max * c.rank_v * h->coef_bytes, s) != cudaSuccess ||
+            (coef_k_bytes > 0 && cudaMemsetAsync(h->coef_k, 0, coef_k_bytes, s) != cudaSuccess) ||
+            (coef_v_bytes > 0 && cudaMemsetAsync(h->coef_v, 0, coef_v_bytes, s) != cudaSuccess) ||
+            (qk_bytes > 0 && (cudaMemsetAsync(h->qcodes_k, 0, qk_bytes, s) != cudaSuccess ||
+                              cudaMemsetAsync(h->qcodes_v, 0, qv_bytes, s) != cudaSuccess ||
+                              cudaMemsetAsync(h->qscales_k, 0, qs_bytes, s) != cudaSuccess ||
+                              cudaMemsetAsync(h->qscales_v, 0, qs_bytes, s) != cudaSuccess)) ||
             cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess ||
             cudaMemsetAsync(h->done, 0, (size_t)h->BH * 4, s) != cudaSuccess ||
             cudaMemsetAsync(h->seg_rows, 0, (size_t)c.layers * h->D * 4, s) != cudaSuccess ||
@@ -493,7 +589,12 @@ int compress_on(iskv_cache* h, const std::vector<int>& ls, int flags, cudaStream
     }
     for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) {
         fl.qscratch = which == ISKV_WHICH_K ? h->qscr_k : h->qscr_v;
-        CU(launch_fold(view(h, which), fl, h->status, s));
+        const FactorView f = view(h, which);
+        if (h->cfg.joint)
+            CU(launch_fold_wide(f, fl, h->status, s));
+        else
+            CU(launch_fold(f, fl, h->status, s));
+        if (f.quant) CU(launch_quant_new_rows(f, fl, s));   // the block's rows, coded
     }
     std::vector<int> rl_layers, rl_seg, rl_rows;
     for (int l : fold_layers) {
@@ -610,7 +711,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.n_c = h->n_c[layer];
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
     const int sms = h->sms;
-    if (h->use_tc && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 &&
+    if (h->use_tc && !c.coef_quant && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 &&
         decode_tc_supports_group(a.g)) {
         // one persistent tensor-core kernel, one CTA per SM, over the flattened
         // (head, tile) space: 128-token tiles of folded rows, then 64-token
@@ -734,12 +835,13 @@ int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
         const int rc = order_after_update(h, layer, s);
         if (rc != ISKV_OK) return rc;
     }
-    const FactorView f = view(h, which);
-    const size_t heads = h->BH;
+    const FactorView f = view_factors(h, which);
+    const size_t heads = h->FH;   // factor instances: per head, or per sequence (joint)
     const int r = f.r;
+    const size_t rows_b = (size_t)h->BH * kHeadDim;   // basis rows of the layer, either way
     if (basis)
-        CU(cudaMemcpyAsync(basis, f.basis + (size_t)layer * heads * kHeadDim * r,
-                           heads * kHeadDim * r * sizeof(float), cudaMemcpyDefault, s));
+        CU(cudaMemcpyAsync(basis, f.basis + (size_t)layer * rows_b * r, rows_b * r * sizeof(float),
+                           cudaMemcpyDefault, s));
     if (sigma)
         CU(cudaMemcpyAsync(sigma, f.sigma + (size_t)layer * heads * r, heads * r * sizeof(float),
                            cudaMemcpyDefault, s));
@@ -771,7 +873,24 @@ int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes) {
         const int64_t T = h->T[l], n_c = h->n_c[l];
         const int64_t exact = T - n_c;   // protected rows and the window
         int64_t per_head = 2 * exact * d * h->kv_bytes;
-        if (n_c > 0) per_head += n_c * rs * h->coef_bytes + (d + 1) * rs * 4;   // C; B and S in fp32
+        int64_t row_bytes = rs * h->coef_bytes;   // one coefficient row of K and V
+        if (c.coef_quant) {
+            // codes, plus one fp32 scale per coded group
+            FactorView fk{}, fv{};
+            quant_fill(c.quant_k, c.rank_k, &fk);
+            quant_fill(c.quant_v, c.rank_v, &fv);
+            int64_t ng = 0;
+            for (int g = 0; g < 4; ++g) ng += (fk.qbits[g] > 0) + (fv.qbits[g] > 0);
+            row_bytes = (int64_t)(fk.qwords + fv.qwords) * 4 + ng * 4;
+        }
+        if (c.joint) {
+            // coefficients, basis (D rows) and sigma once per sequence
+            kept += per_head * h->BH;
+            if (n_c > 0) kept += (n_c * row_bytes + (d * c.kv_heads + 1) * rs * 4) * h->FH;
+            full += 2 * T * d * h->kv_bytes * h->BH;
+            continue;
+        }
+        if (n_c > 0) per_head += n_c * row_bytes + (d + 1) * rs * 4;   // C; B and S in fp32
         kept += per_head * h->BH;
         full += 2 * T * d * h->kv_bytes * h->BH;
     }
@@ -799,6 +918,29 @@ int iskv_status(iskv_t h) {
     return ISKV_OK;
 }
 
+int iskv_quant_words(const iskv_quant_format* fmt) {
+    if (!fmt) return -1;
+    int r = 0;
+    for (int g = 0; g < fmt->groups && g < 4; ++g) r += fmt->channels[g];
+    FactorView f{};
+    if (r < 16 || r > kHeadDim || !quant_fill(*fmt, r, &f)) return -1;
+    return f.qwords;
+}
+
+int iskv_quantize_rows(const iskv_quant_format* fmt, int rank, const float* rows, int64_t n,
+                       uint32_t* codes, float* scales, void* stream) {
+    if (!fmt || n < 0 || rank < 16 || rank > kHeadDim) return ISKV_ERR_INVALID_ARG;
+    FactorView f{};
+    if (!quant_fill(*fmt, rank, &f)) return ISKV_ERR_INVALID_ARG;
+    f.r = rank;
+    if (n == 0) return ISKV_OK;
+    if (!rows || !codes || !scales || !is_device_ptr(rows) || !is_device_ptr(codes) ||
+        !is_device_ptr(scales))
+        return ISKV_ERR_INVALID_ARG;
+    CU(launch_quant_rows(f, rows, n, codes, scales, reinterpret_cast<cudaStream_t>(stream)));
+    return ISKV_OK;
+}
+
 const char* iskv_strerror(int code) {
     switch (code) {
         case ISKV_OK: return "ok";
@@ -810,7 +952,7 @@ const char* iskv_strerror(int code) {
         case ISKV_ERR_NOMEM: return "device allocation failed";
         case ISKV_ERR_UNSUPPORTED: return "shape not supported by the compiled kernels";
         case ISKV_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up; that call's results are incomplete";
-        case ISKV_ERR_RANGE: return "a rotated key or query left the fp16 range of the tensor-core decode";
+        case ISKV_ERR_RANGE: return "a score of the tensor-core decode was not finite (inf or NaN input)";
         default: return "unknown status";
     }
 }

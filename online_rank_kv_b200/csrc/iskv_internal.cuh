@@ -21,7 +21,7 @@ constexpr int kMaxGroup = 8;      // query heads per KV head in the decode
 // Status bits of the sticky device word (bit 2, a bounded wait that gave up,
 // is defined with the waits in tc_util.cuh).
 constexpr int kStatusNoConverge = 1;
-constexpr int kStatusRange = 4;   // a non-finite score in the tensor-core decode
+constexpr int kStatusRange = 4;   // a score of the tensor-core decode was not finite
 
 // ---------------------------------------------------------------------------
 // Element conversions (explicit round-to-nearest-even for bf16 stores).
@@ -83,7 +83,93 @@ struct FactorView {
     int64_t cap;         // ring rows per head
     int D;               // postponed-fold slots per head
     int BH;              // batch * kv_heads
+    // low-bit latent-channel codes (iskv_quant_format) instead of coef
+    int quant;           // 1: coefficients live in qcodes / qscales
+    uint32_t* qcodes;    // [L][BH][n_max][qwords]
+    float* qscales;      // [L][BH][n_max][4]
+    float* newrows;      // [L][BH][64][r] fp32: a fold's new rows before they are coded
+    int qwords;          // code words per row
+    int qgroups;         // groups in use (1..4)
+    int qbits[4], qlo[4], qhi[4], qword0[4];   // bits, channel range and first word per group
+    // joint-head factors: one factor (coefficients, singular values, postponed
+    // W_top) per sequence over its `coef_div` KV heads, whose rows sit side by
+    // side (D = coef_div * 128); basis rows, their bf16 parts and the exact
+    // rows stay addressed per KV head (head h of a sequence holds basis rows
+    // h * 128 .. h * 128 + 127).  0 or 1: one factor per head.
+    int coef_div;
+    float* wide;         // joint fold scratch: per factor [D x (r+64)] + [D x 64] + [D x r]
 };
+
+// Factor instance (coefficients, sigma, postponed W_top) of head instance hidx.
+__host__ __device__ __forceinline__ int64_t coef_inst(const FactorView& f, int64_t hidx) {
+    return f.coef_div > 1 ? hidx / f.coef_div : hidx;
+}
+
+// ---------------------------------------------------------------------------
+// Latent-channel codes (iskv_quant_format): fp32 decisions throughout.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int quant_group_of(const FactorView& f, int c) {
+    int g = 0;
+#pragma unroll
+    for (int i = 1; i < 4; ++i) g += (i < f.qgroups && c >= f.qlo[i]) ? 1 : 0;
+    return g;
+}
+
+// The stored value of coefficient (row, c) of factor instance hidx.
+__device__ __forceinline__ float quant_value(const FactorView& f, int64_t hidx, int64_t row, int c) {
+    const int g = quant_group_of(f, c);
+    const int b = f.qbits[g];
+    if (b == 0) return 0.f;
+    const int idx = c - f.qlo[g];
+    const int64_t rbase = hidx * f.n_max + row;
+    const uint32_t w = f.qcodes[rbase * f.qwords + f.qword0[g] + ((idx * b) >> 5)];
+    const int qmax = (1 << (b - 1)) - 1;
+    const int code = (int)((w >> ((idx * b) & 31)) & ((1u << b) - 1u)) - qmax;
+    return (float)code * f.qscales[rbase * 4 + g];
+}
+
+// Code rows of r fp32 values: src[row * ld + c] for rows [0, nrows) of a
+// block, written to codes[row * qwords + w] and scales[row * 4 + g]; sScale
+// holds nrows * 4 floats of block scratch.  Called by every thread of the
+// block (blockDim.x threads); ends with the codes written.
+__device__ __forceinline__ void quant_rows_block(const FactorView& f, const float* src, int ld, int nrows,
+                                                 uint32_t* codes, float* scales, float* sScale) {
+    for (int e = threadIdx.x; e < nrows * 4; e += blockDim.x) {
+        const int row = e >> 2, g = e & 3;
+        float sc = 0.f;
+        if (g < f.qgroups && f.qbits[g] > 0) {
+            float amax = 0.f;
+            for (int c = f.qlo[g]; c < f.qhi[g]; ++c) amax = fmaxf(amax, fabsf(src[row * ld + c]));
+            sc = __fdiv_rn(amax, (float)((1 << (f.qbits[g] - 1)) - 1));
+        }
+        sScale[e] = sc;
+        scales[(int64_t)row * 4 + g] = sc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < nrows * f.qwords; e += blockDim.x) {
+        const int row = e / f.qwords, w = e % f.qwords;
+        int g = 0;
+#pragma unroll
+        for (int i = 1; i < 4; ++i) g += (i < f.qgroups && w >= f.qword0[i]) ? 1 : 0;
+        const int b = f.qbits[g];
+        uint32_t word = 0u;
+        if (b > 0) {
+            const int qmax = (1 << (b - 1)) - 1;
+            const float sc = sScale[row * 4 + g];
+            const int per = 32 / b;
+            const int c0 = f.qlo[g] + (w - f.qword0[g]) * per;
+            for (int e2 = 0; e2 < per; ++e2) {
+                int code = 0;
+                if (sc > 0.f) {
+                    code = __float2int_rn(__fdiv_rn(src[row * ld + c0 + e2], sc));
+                    code = code > qmax ? qmax : (code < -qmax ? -qmax : code);
+                }
+                word |= (uint32_t)(code + qmax) << (e2 * b);
+            }
+        }
+        codes[(int64_t)row * f.qwords + w] = word;
+    }
+}
 
 struct FoldLaunch {
     int n_tasks;                 // layers folded by this launch
@@ -156,6 +242,9 @@ cudaError_t launch_append(void* ring, const void* src, int BH, int t, int src_t,
                           int64_t T0, int64_t cap, int elem_bytes, int blocked, cudaStream_t s);
 cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status,
                         cudaStream_t s);
+cudaError_t launch_fold_wide(const FactorView& f, const FoldLaunch& fl, int* status,
+                             cudaStream_t s);
+size_t fold_wide_scratch_floats(int D, int r);
 cudaError_t launch_compose(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);
 cudaError_t launch_resync(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
@@ -166,6 +255,10 @@ cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64
                              cudaStream_t s);
 cudaError_t launch_resync_tc(const FactorView& f, const ResyncLaunch& rl, int* status,
                              cudaStream_t s);
+cudaError_t launch_resync_quant(const FactorView& f, const ResyncLaunch& rl, cudaStream_t s);
+cudaError_t launch_quant_new_rows(const FactorView& f, const FoldLaunch& fl, cudaStream_t s);
+cudaError_t launch_quant_rows(const FactorView& f, const float* rows, int64_t n, uint32_t* codes,
+                              float* scales, cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
 bool decode_tc_supports_group(int g);
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb, int wt);

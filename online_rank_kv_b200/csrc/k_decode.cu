@@ -87,8 +87,8 @@ decode_kernel(DecodeArgs a) {
 #pragma unroll
     for (int u = 0; u < kMaxAcc; ++u) acc[u] = 0.f;
 
-    const CoefT* Ck = reinterpret_cast<const CoefT*>(a.K.coef) + hidx * a.K.n_max * rK;
-    const CoefT* Cv = reinterpret_cast<const CoefT*>(a.V.coef) + hidx * a.V.n_max * rV;
+    const CoefT* Ck = reinterpret_cast<const CoefT*>(a.K.coef) + coef_inst(a.K, hidx) * a.K.n_max * rK;
+    const CoefT* Cv = reinterpret_cast<const CoefT*>(a.V.coef) + coef_inst(a.V, hidx) * a.V.n_max * rV;
     const KvT* Rk = reinterpret_cast<const KvT*>(a.K.ring) + hidx * a.K.cap * d;
     const KvT* Rv = reinterpret_cast<const KvT*>(a.V.ring) + hidx * a.V.cap * d;
     const KvT* Pk = reinterpret_cast<const KvT*>(a.K.prot) + hidx * a.K.pcap * d;
@@ -107,12 +107,20 @@ decode_kernel(DecodeArgs a) {
 
         if (comp) {
             const int64_t jc = j - P;   // coefficient row
-            for (int e = tid; e < kTile * rK; e += kThreads)
-                sCk[e] = (e / rK < nt) ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, jc + e / rK, e % rK)])
-                                       : 0.f;
-            for (int e = tid; e < kTile * rV; e += kThreads)
-                sCv[e] = (e / rV < nt) ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, jc + e / rV, e % rV)])
-                                       : 0.f;
+            if (a.K.quant) {
+                // latent-channel codes: decoded to fp32 while staged
+                for (int e = tid; e < kTile * rK; e += kThreads)
+                    sCk[e] = (e / rK < nt) ? quant_value(a.K, hidx, jc + e / rK, e % rK) : 0.f;
+                for (int e = tid; e < kTile * rV; e += kThreads)
+                    sCv[e] = (e / rV < nt) ? quant_value(a.V, hidx, jc + e / rV, e % rV) : 0.f;
+            } else {
+                for (int e = tid; e < kTile * rK; e += kThreads)
+                    sCk[e] = (e / rK < nt) ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, jc + e / rK, e % rK)])
+                                           : 0.f;
+                for (int e = tid; e < kTile * rV; e += kThreads)
+                    sCv[e] = (e / rV < nt) ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, jc + e / rV, e % rV)])
+                                           : 0.f;
+            }
             __syncthreads();
             for (int e = tid; e < kTile * d; e += kThreads) {
                 const int t = e / d, i = e % d;

@@ -890,7 +890,12 @@ fold_kernel(FactorView f, FoldLaunch fl, int* status) {
             }
         }
         const int64_t row = n_c + t;
-        if (f.coef_bf16) {
+        if (f.quant) {
+            // coded storage: the fp32 rows wait in newrows for the coding kernel
+            float* gN = f.newrows + hidx * kBlock * R;
+#pragma unroll
+            for (int v = 0; v < Q4; ++v) gN[t * R + h * Q4 + v] = acc[v];
+        } else if (f.coef_bf16) {
             __nv_bfloat16* gC = reinterpret_cast<__nv_bfloat16*>(f.coef) + hidx * f.n_max * R;
 #pragma unroll
             for (int v = 0; v < Q4; ++v)

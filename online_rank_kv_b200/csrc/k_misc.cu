@@ -15,7 +15,9 @@ __global__ void init_factor_kernel(FactorView f, int layers) {
          e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t h = e / per, w = e % per;
         const int i = (int)(w / r), j = (int)(w % r);
-        const float v = (i == j) ? 1.f : 0.f;
+        // joint-head factor: basis row i of head h is joint row (h mod heads) * 128 + i
+        const int hrow = f.coef_div > 1 ? (int)(h % f.coef_div) * kHeadDim + i : i;
+        const float v = (hrow == j) ? 1.f : 0.f;
         f.basis[e] = v;
         const int64_t bo = coef_index(1, r, i, j);
         f.bsplit[h * 2 * per + bo] = __float2bfloat16_rn(v);
@@ -59,12 +61,15 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(FactorView f, int laye
     float* sC = sm + kHeadDim * (r + 1);  // kRecRows x r
     const int64_t hidx = (int64_t)layer * f.BH + bh;
     const float* B = f.basis + hidx * kHeadDim * r;
-    const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + hidx * f.n_max * r;
+    const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + coef_inst(f, hidx) * f.n_max * r;
     const int nt = (int)((rows - t0) < kRecRows ? (rows - t0) : kRecRows);
     for (int e = threadIdx.x; e < kHeadDim * r; e += blockDim.x) sB[(e / r) * (r + 1) + e % r] = B[e];
     for (int e = threadIdx.x; e < kRecRows * r; e += blockDim.x) {
         const int t = e / r, c = e % r;
-        sC[e] = (t < nt) ? to_f32(C[coef_index(f.coef_blocked, r, row0 + t0 + t, c)]) : 0.f;
+        const int64_t row = row0 + t0 + t;
+        sC[e] = (t >= nt) ? 0.f
+              : f.quant ? quant_value(f, hidx, row, c)
+                        : to_f32(C[coef_index(f.coef_blocked, r, row, c)]);
     }
     __syncthreads();
     float* o = out + ((int64_t)bh * rows + t0) * kHeadDim;
@@ -87,8 +92,12 @@ __global__ void copy_coef_kernel(FactorView f, int layer, int64_t row0, int64_t 
         const int64_t row = (e / r) % rows;
         const int64_t bh = e / ((int64_t)r * rows);
         const int64_t hidx = (int64_t)layer * f.BH + bh;
-        const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + hidx * f.n_max * r;
-        dst[e] = C[coef_index(f.coef_blocked, r, row0 + row, c)];
+        if (f.quant) {
+            dst[e] = from_f32<CoefT>(quant_value(f, hidx, row0 + row, c));
+        } else {
+            const CoefT* C = reinterpret_cast<const CoefT*>(f.coef) + hidx * f.n_max * r;
+            dst[e] = C[coef_index(f.coef_blocked, r, row0 + row, c)];
+        }
     }
 }
 
@@ -100,7 +109,7 @@ cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64
     const int64_t total = (int64_t)f.BH * rows * f.r;
     int64_t blocks = (total + 255) / 256;
     if (blocks > 4736) blocks = 4736;
-    if (f.coef_bf16)
+    if (f.coef_bf16 && !f.quant)
         copy_coef_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
             f, layer, row0, rows, reinterpret_cast<__nv_bfloat16*>(dst));
     else
@@ -133,7 +142,7 @@ cudaError_t launch_reconstruct(const FactorView& f, int layer, int64_t row0, int
     if (rows <= 0) return cudaSuccess;
     const size_t bytes = ((size_t)kHeadDim * (f.r + 1) + (size_t)kRecRows * f.r) * sizeof(float);
     dim3 grid((unsigned)((rows + kRecRows - 1) / kRecRows), f.BH);
-    if (f.coef_bf16) {
+    if (f.coef_bf16 && !f.quant) {
         auto k = reconstruct_kernel<__nv_bfloat16>;
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return e;

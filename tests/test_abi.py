@@ -132,3 +132,21 @@ def test_binding_structs_match_the_header_layout(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_code_format_checks_on_the_host():
+    """Latent-channel code formats: words per row, and create refuses a format
+    whose groups do not cover the rank or use an unsupported width."""
+    ik = _lib()
+    q = ik.QuantFormat.of([(8 * 2, 8), (16, 2)])
+    assert ik.LIB.iskv_quant_words(ctypes.byref(q)) == 16 * 8 // 32 + 16 * 2 // 32
+    assert ik.LIB.iskv_quant_words(ctypes.byref(ik.QuantFormat.of([(16, 3)]))) == -1
+    assert ik.LIB.iskv_quant_words(ctypes.byref(ik.QuantFormat.of([(24, 8)]))) == -1
+    assert ik.LIB.iskv_quant_words(None) == -1
+    for qk, qv in (([(16, 8)], [(32, 8), (32, 4)]),          # K groups cover 16 of 32
+                   ([(32, 8)], [(32, 8), (32, 5)]),          # 5-bit codes
+                   ([(32, 0)], [(64, 8)])):                  # no coded group
+        cfg = ik.Config(rank_k=32, rank_v=64, coef_quant=1, quant_k=qk, quant_v=qv)
+        h = ctypes.c_void_p(1)
+        assert ik.LIB.iskv_create(ctypes.byref(cfg._c()), None, ctypes.byref(h)) == -1
+        assert h.value is None
