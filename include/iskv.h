@@ -67,9 +67,11 @@ extern "C" {
                                       destroy the cache: its decode bookkeeping
                                       may be left inconsistent)             */
 #define ISKV_ERR_RANGE         -9  /* a score of the tensor-core decode was not
-                                      finite: an inf or NaN key or query, or
-                                      a product beyond fp32's range (sticky;
-                                      that call's outputs are not finite)   */
+                                      finite: a rotated key or a query went
+                                      beyond fp16's range (|x| >= 65504), the
+                                      type its score MMA takes, or an input
+                                      was inf or NaN (sticky; that call's
+                                      outputs are not finite)               */
 
 /* ---- element types ----------------------------------------------------- */
 #define ISKV_F32   0

@@ -952,7 +952,7 @@ const char* iskv_strerror(int code) {
         case ISKV_ERR_NOMEM: return "device allocation failed";
         case ISKV_ERR_UNSUPPORTED: return "shape not supported by the compiled kernels";
         case ISKV_ERR_DEVICE_TIMEOUT: return "a device-side wait gave up; that call's results are incomplete";
-        case ISKV_ERR_RANGE: return "a score of the tensor-core decode was not finite (inf or NaN input)";
+        case ISKV_ERR_RANGE: return "a score of the tensor-core decode was not finite (fp16 range of its keys exceeded, or inf/NaN input)";
         default: return "unknown status";
     }
 }

@@ -16,39 +16,42 @@
 //
 // Persistent design, one CTA per SM; the flattened (head, tile) space is cut
 // into contiguous runs of equal cost (tiles, plus a fixed charge for every
-// head a run enters after its first), one run per CTA.  Per CTA 12 warps:
+// head a run enters after its first), one run per CTA.  Per CTA 20 warps:
 //   warp 0  producer: 1-D bulk copies (TMA engine) of the C_K and C_V tiles
 //           or of the exact K and V rows (all contiguous in the blocked
 //           layout) into an NS-stage ring, and of the bf16 hi/lo basis and
 //           the bf16 queries of each head it visits;
 //   warp 1  TMEM allocation;
-//   warps 2-9 epilogue, two ping-pong groups of 4 warps (group = tile
-//           parity), one token row per thread:
-//           * read its row of K^ out of TMEM (then release the buffer to the
-//             issuer), rotate it by R_t (t = row within the tile; the row's
-//             cos/sin(t w_i) sit in spare TMEM columns) in packed fp32, and
-//             take the g scores as fp32 dot products with q' = R_{j0}^T q
-//             (pre-rotated per tile, j0 = tile start, so q'.(R_t k) =
-//             q.(R_{j0+t} k)), which every thread reads from shared memory
-//             as broadcasts;
-//           * online softmax per query head with a lazily updated maximum;
+//   warps 2-3 MMA issuer of group 0 / 1:
+//           * K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens, N=128 dims,
+//             fp32 accumulator in TMEM, rebuilt two tiles ahead;
+//           * scores S = K_rot q'^T, kind::f16 with A from TMEM and q' as
+//             fp16 hi+lo parts in the N dimension, issued in two halves of
+//             the head dimension as the epilogue finishes rotating them;
+//           * O = C_V^T P (kind::f16, C_V tile read MN-major in place; for
+//             exact rows O = V^T P with M = d);
+//   warps 4-19 epilogue, two ping-pong groups of 8 warps (group = tile
+//           parity), two threads per token row: the row's two halves (subs)
+//           each take half of the RoPE frequencies and half of the query
+//           heads, so each SM sub-partition runs four epilogue warps:
+//           * rotate its half of the row of K^ by R_t (t = row within the
+//             tile; the row's cos/sin(t w_i) sit in spare TMEM columns) and
+//             write it back to TMEM as fp16 pairs (dim i, dim 64 + i) per
+//             column; the query is pre-rotated per tile by R_{j0}^T (j0 =
+//             tile start), so q'.(R_t k) = q.(R_{j0+t} k); each half starts
+//             its own score MMA half;
+//           * online softmax of its query heads with a lazily updated maximum;
 //           * p as bf16 hi+lo parts for the value MMA;
 //           * at the end of a head the group publishes its own partial
 //             (m, l, r_V-wide and d-wide sums); the last group to publish
 //             a head's partial merges them all by log-sum-exp, applies
 //             B_V^T once per query head and writes the output.  The two
 //             groups never wait for each other.
-//   warps 10-11 MMA issuer of group 0 / 1:
-//           * K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens, N=128 dims,
-//             fp32 accumulator in TMEM, rebuilt for the group's next tile as
-//             soon as the epilogue has read this one;
-//           * O = C_V^T P (kind::f16, C_V tile read MN-major in place; for
-//             exact rows O = V^T P with M = d).
-// Keys, queries and scores stay fp32 after the rebuild (the tensor cores
-// rebuild keys and sum values; the scores, g per row, are CUDA-core work).
+// Rotated keys are held in fp16 (finite for |k| < 65504; the same 11-bit
+// significand as tf32); the query as fp16 hi + lo parts keeps ~22 bits.
 // Every mbarrier wait is bounded; on timeout the CTA records
 // ISKV status bit 2, stops, drains its copies and frees its TMEM.  A score
-// that is not finite (an inf or NaN key or query, or an fp32 overflow) sets
+// that is not finite (a rotated key or query outside the fp16 range) sets
 // status bit 4.
 #include "iskv_internal.cuh"
 #include "tc_util.cuh"
@@ -64,18 +67,19 @@ using namespace tc;
 constexpr int kTile = 128;
 // exact-row tiles have 64 or 32 rows (the host's choice, win_rows): either
 // divides the ring and the protected-row capacity, so a tile never wraps
-constexpr int kThreads = 384;
-constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
+constexpr int kThreads = 640;
+constexpr int kEpi = 512;        // epilogue threads (warps 4-19, two groups of 8)
+constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
 constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
-constexpr int kBufCols = 144;    // per TMEM buffer: K^ 128 | O 16
+constexpr int kBufCols = 160;    // per TMEM buffer: K^ 128 | S 16 | O 16
 constexpr int kCsCol = 2 * kBufCols;   // per-row RoPE table: cos 64 | sin 64 | -sin 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Bars {
     uint64_t full[6], empty[6];
     uint64_t bk_full[2], bk_empty[4];      // bk_empty[buffer * 2 + group]
-    uint64_t kh_full[2], kfree[2], o_full[2];   // kfree: the group's epilogue has read K^
-    uint64_t p_ready[2];                         // epilogue -> group issuer: P written
+    uint64_t kh_full[2], kfree[2], s_full[2], o_full[2];
+    uint64_t krot_ready[2], krot_b[2], p_ready[2];   // epilogue -> group issuer: K_rot halves, P written
     uint64_t drain[3];   // abort path: completion of each issuer's outstanding MMAs
 };
 
@@ -89,7 +93,7 @@ struct SmemPlan {
     uint32_t bk, stage, stage_k, stage_bytes, qb, pb, total;
 };
 
-constexpr int kQFloats = kMaxGroup * kHeadDim;   // one q' buffer: g <= 8 rows of 128 fp32
+constexpr int kQWords = kQN * 64;   // one q' buffer: kQN rows of 128 fp16 (64 words)
 
 __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, int nqb, int wt) {
     SmemPlan p;
@@ -100,16 +104,16 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, i
     if (sb < 2 * wt * kHeadDim * 2) sb = 2 * wt * kHeadDim * 2;   // exact K and V rows
     p.stage_bytes = sb + 1024;
     p.stage = off;             off += ns * p.stage_bytes;
-    p.qb = off;                off += 2 * nqb * (kQFloats * 4);   // [group][nqb] q' buffers
+    p.qb = off;                off += 2 * nqb * (kQWords * 4);   // [group][nqb] q' buffers
     p.pb = off;                off += 2 * (kPN * kTile * 2);
     p.total = off;
     return p;
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// barrier of one ping-pong group (ids 2 and 3, 128 threads)
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+// barrier of one ping-pong group (ids 2 and 3, 256 threads)
 __device__ __forceinline__ void group_sync(int grp) {
-    asm volatile("bar.sync %0, 128;" ::"r"(2 + grp) : "memory");
+    asm volatile("bar.sync %0, 256;" ::"r"(2 + grp) : "memory");
 }
 // the same barrier, returning whether any of the group's threads passed true
 __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
@@ -117,7 +121,7 @@ __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
     asm volatile(
         "{\n\t.reg .pred q, p;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, %2, 128, q;\n\t"
+        "bar.red.or.pred p, %2, 256, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
         : "r"((uint32_t)pred), "r"(2 + grp)
@@ -128,6 +132,13 @@ __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
 // more than this (p <= e^8); otherwise the tile takes the exact rescale
 constexpr float kLazyMax = 8.f;
 
+// q' as the score MMA's B operand: fp16, K-major 8 x 8 core matrices over
+// K = 128 positions k, where k = 2u holds dim u and k = 2u + 1 dim 64 + u
+// (the order of the packed rotated keys in TMEM).  Word (32-bit) offset of
+// the pair (k = 2u, 2u + 1) of row n.
+__device__ __forceinline__ int qb_off(int n, int u) {
+    return ((n >> 3) * (kTile / 8) + (u >> 2)) * 32 + (n & 7) * 4 + (u & 3);
+}
 // p as the value MMA's B operand, MN-major: [token][16] in 8 x 8 blocks, so one
 // thread's (token's) 8 values of an n-block are one 16-byte row
 __device__ __forceinline__ int pb_off(int n, int k) {
@@ -157,7 +168,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs, nqb = a.q_bufs;
     const int wt = a.win_rows;      // rows of an exact-row tile (64 or 32)
     constexpr int g = G;
-    constexpr int kQItems = (G * 64 + 127) / 128;   // q' items per epilogue thread
+    constexpr int kQItems = (G * 64 + 255) / 256;   // q' items per epilogue thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int d = kHeadDim;
 
@@ -174,7 +185,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     const SmemPlan P = plan_smem(rK, rV, ns, nbk, nqb, wt);
     uint8_t* bk = smem + P.bk;
     uint8_t* stage = smem + P.stage;
-    float* qb = reinterpret_cast<float*>(smem + P.qb);
+    uint32_t* qb = reinterpret_cast<uint32_t*>(smem + P.qb);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
     const uint32_t stage_bytes = P.stage_bytes;
     const int tiles_c = a.tiles_c, tiles_cw = a.tiles_c + a.tiles_w;
@@ -196,15 +207,23 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->bk_full[i], 1);
             mbar_init(&bars->kh_full[i], 1);
-            mbar_init(&bars->kfree[i], kEpi / 2);
+            mbar_init(&bars->kfree[i], 1);
+            mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->o_full[i], 1);
+            mbar_init(&bars->krot_ready[i], kEpi / 4);   // one sub of the group each
+            mbar_init(&bars->krot_b[i], kEpi / 4);
             mbar_init(&bars->p_ready[i], 1);
         }
         for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // zero the padding rows (n >= 2g) of the p operand once
+    // zero the padding rows (n >= 2g) of the q' and p operands once
+    for (int e = tid; e < 2 * nqb * kQN * 64; e += kThreads) {
+        const int buf = e / (kQN * 64), w = e % (kQN * 64);
+        const int n = w / 64, u = w % 64;
+        if (n >= 2 * g) qb[buf * kQWords + qb_off(n, u)] = 0u;
+    }
     for (int e = tid; e < 2 * kPN * kTile; e += kThreads) {
         const int buf = e / (kPN * kTile), w = e % (kPN * kTile);
         const int n = w / kTile, k = w % kTile;
@@ -290,51 +309,53 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     mbar_wait(&bars->full[n % ns], (n / ns) & 1, deadline + kWaitCycles);
             }
         }
-    } else if (warp >= 2 && warp < 10) {
-        // ---------------- epilogue: two groups of 4 warps, alternate tiles ----------------
-        const int ept = tid - 64;                 // 0..255
+    } else if (warp >= 4) {
+        // ---------------- epilogue: two groups of 8 warps, alternate tiles ----------------
+        // A row (token) of a tile is shared by two threads of its group, one in
+        // each half (sub) of the group: sub s rotates frequencies 32 s .. 32 s + 31
+        // of the row and keeps the softmax of query heads s kH .. s kH + kH - 1.
+        const int ept = tid - 128;                // 0..511
         // positions: protected [0, P), folded [P, P + n_c), window [P + n_c, T)
         const int nc32 = (int)a.n_c, T32 = (int)a.T, P32 = (int)a.K.P;
         const int Pe32 = T32 < P32 ? T32 : P32;
-        const int grp = ept >> 7;                 // tiles n with n % 2 == grp
-        const int gt = ept & 127;                 // thread within the group
+        const int grp = ept >> 8;                 // tiles n with n % 2 == grp
+        const int gt = ept & 255;                 // thread within the group
+        const int sub = gt >> 7;                  // half of the frequencies and heads
         const int sp = warp & 3;                  // TMEM sub-partition of this warp
         const int row = sp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
         const uint32_t tcs = tmem + kCsCol;
+        constexpr int kH = (G + 1) / 2;           // query heads per sub
         // this row's in-tile RoPE table (cos, sin, -sin of row * w_i) into TMEM:
-        // group grp writes frequencies 32 grp .. 32 grp + 31, all loads issued first
+        // (group, sub) writes frequencies 16 (2 grp + sub) .. + 15
         {
-            float4 tv[16];
+            const int f0t = (2 * grp + sub) * 16;
+            float4 tv[8];
             if (a.rope) {
-                const float4* src = reinterpret_cast<const float4*>(a.rope + row * 64 + grp * 32);
+                const float4* src = reinterpret_cast<const float4*>(a.rope + row * 64 + f0t);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) tv[u] = src[u];
+                for (int u = 0; u < 8; ++u) tv[u] = src[u];
             } else {
 #pragma unroll
-                for (int u = 0; u < 16; ++u) tv[u] = make_float4(1.f, 0.f, 1.f, 0.f);
+                for (int u = 0; u < 8; ++u) tv[u] = make_float4(1.f, 0.f, 1.f, 0.f);
             }
+            uint32_t vc[16], vs[16], vn[16];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t vc[16], vs[16], vn[16];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float4 v = tv[hh * 8 + u];
-                    vc[2 * u] = __float_as_uint(v.x);
-                    vs[2 * u] = __float_as_uint(v.y);
-                    vn[2 * u] = __float_as_uint(-v.y);
-                    vc[2 * u + 1] = __float_as_uint(v.z);
-                    vs[2 * u + 1] = __float_as_uint(v.w);
-                    vn[2 * u + 1] = __float_as_uint(-v.w);
-                }
-                const int c0 = grp * 32 + hh * 16;
-                tmem_st16(tcs + lane_base + c0, vc);
-                tmem_st16(tcs + lane_base + 64 + c0, vs);
-                tmem_st16(tcs + lane_base + 128 + c0, vn);
+            for (int u = 0; u < 8; ++u) {
+                const float4 v = tv[u];
+                vc[2 * u] = __float_as_uint(v.x);
+                vs[2 * u] = __float_as_uint(v.y);
+                vn[2 * u] = __float_as_uint(-v.y);
+                vc[2 * u + 1] = __float_as_uint(v.z);
+                vs[2 * u + 1] = __float_as_uint(v.w);
+                vn[2 * u + 1] = __float_as_uint(-v.w);
             }
+            tmem_st16(tcs + lane_base + f0t, vc);
+            tmem_st16(tcs + lane_base + 64 + f0t, vs);
+            tmem_st16(tcs + lane_base + 128 + f0t, vn);
             tmem_wait_st();
         }
-        // both halves of the table written before either group's first RoPE
+        // the whole table written before any group's first RoPE
         tc_fence_before();
         epi_sync();
         tc_fence_after();
@@ -342,19 +363,29 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         const int c_acc = (MV == 64) ? (lane < 16 ? sp * 16 + lane : -1) : row;
         const bool acc_ok = c_acc >= 0 && c_acc < rV;
         float* gred = red + grp * 64;             // [max 4 x 8 | l 4 x 8] of this group
-        const uint32_t kh = tmem + grp * kBufCols;   // K^ / O buffer of this group
-        float* qbb = qb + nqb * grp * kQFloats;     // the group's first q' buffer (head-end exchange)
+        const uint32_t kh = tmem + grp * kBufCols;   // K^ / S / O buffer of this group
+        uint32_t* qbb = qb + nqb * grp * kQWords;   // the group's first q' buffer (head-end exchange)
         __nv_bfloat16* pbb = pb + grp * kPN * kTile;
+        // q' operand offsets of this thread's items (hi of dims i, i + 64; lo likewise)
+        int qoff[kQItems][2];
+#pragma unroll
+        for (int k = 0; k < kQItems; ++k) {
+            const int item = gt + 256 * k;
+            const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
+            qoff[k][0] = qb_off(h, i);       // hi parts of dims i, 64 + i
+            qoff[k][1] = qb_off(G + h, i);   // lo parts
+        }
 
-        float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
+        float m_run[kH], l_thr[kH], acc[kH], accd[kH], alpha[kH];
         // acc <- acc * alpha + (p^T C_V of a folded tile); accd likewise for exact tiles
         // (both rescaled every tile: they share the running max)
         auto accumulate = [&](const uint32_t (&o)[16], bool was_win) {
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
+            for (int hh = 0; hh < kH; ++hh) {
+                const int h = sub * kH + hh < G ? sub * kH + hh : 0;
                 const float add = __uint_as_float(o[h]) + __uint_as_float(o[G + h]);
-                acc[h] = (acc_ok && !was_win) ? fmaf(acc[h], alpha[h], add) : acc[h] * alpha[h];
-                accd[h] = was_win ? fmaf(accd[h], alpha[h], add) : accd[h] * alpha[h];
+                acc[hh] = (acc_ok && !was_win) ? fmaf(acc[hh], alpha[hh], add) : acc[hh] * alpha[hh];
+                accd[hh] = was_win ? fmaf(accd[hh], alpha[hh], add) : accd[hh] * alpha[hh];
             }
         };
         bool stop = false;
@@ -368,12 +399,12 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             if (s1 > ntiles) s1 = ntiles;
             ++hs;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                m_run[h] = -INFINITY;
-                l_thr[h] = 0.f;
-                acc[h] = 0.f;
-                accd[h] = 0.f;
-                alpha[h] = 0.f;
+            for (int hh = 0; hh < kH; ++hh) {
+                m_run[hh] = -INFINITY;
+                l_thr[hh] = 0.f;
+                acc[hh] = 0.f;
+                accd[hh] = 0.f;
+                alpha[hh] = 0.f;
             }
             // group-uniform abort check
             if (gt == 0) epi_abort[grp] = *abort_flag;
@@ -397,40 +428,39 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                                     : lc < tiles_cw ? P32 + nc32 + (lc - tiles_c) * wt
                                                     : (lc - tiles_cw) * wt;
             };
-            // q' = R_{j0}^T q of tile nn in fp32, [head][dim], in the group's q'
-            // buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i) for i = gt & 63, the
-            // only frequency this thread rotates by
-            // this thread's items (head h, frequency i): item gt + 128 k; their
-            // query pair (q_i, q_{i+64}) stays in registers for the whole head
+            // q' = R_{j0}^T q of tile nn as fp16 hi / lo parts (the score MMA's B
+            // operand), in the group's q' buffer (nn >> 1) & 1; this thread's items
+            // (head h, frequency i = gt & 63): item gt + 256 k; their query pair
+            // (q_i, q_{i+64}) stays in registers for the whole head
             float qx1[kQItems], qx2[kQItems];
 #pragma unroll
             for (int k = 0; k < kQItems; ++k) {
-                const int item = gt + 128 * k;
+                const int item = gt + 256 * k;
                 const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
                 qx1[k] = n_first < s1 ? __bfloat162float(sq[h * d + i]) : 0.f;
                 qx2[k] = n_first < s1 ? __bfloat162float(sq[h * d + i + 64]) : 0.f;
             }
             auto build_q = [&](int nn, float2 rv) {
-                float* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQFloats;
+                uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQWords;
 #pragma unroll
                 for (int k = 0; k < kQItems; ++k) {
-                    const int item = gt + 128 * k;
-                    if (item >= G * 64) break;
-                    const int h = item >> 6, i = item & 63;
-                    qd[h * d + i] = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
-                    qd[h * d + 64 + i] = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
+                    if (gt + 256 * k >= G * 64) break;
+                    const float y1 = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
+                    const float y2 = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
+                    const __half2 hi = __floats2half2_rn(y1, y2);
+                    const float2 hf = __half22float2(hi);
+                    const __half2 lo = __floats2half2_rn(y1 - hf.x, y2 - hf.y);
+                    qd[qoff[k][0]] = *reinterpret_cast<const uint32_t*>(&hi);
+                    qd[qoff[k][1]] = *reinterpret_cast<const uint32_t*>(&lo);
                 }
+                fence_async_smem();
             };
             auto rope_of = [&](int nn) {
                 return a.rope ? a.rope[(int64_t)tile_j0(nn) * 64 + (gt & 63)] : make_float2(1.f, 0.f);
             };
-            // two q' buffers: tile n + 2's q' is built during tile n (the group's
-            // softmax barrier of tile n publishes it); one buffer: each tile
-            // builds its own, then a group barrier
-            if (nqb == 2 && n_first < s1) {
-                build_q(n_first, rope_of(n_first));
-                group_sync(grp);                  // the head's first q' is visible to the group
-            }
+            // two q' buffers: tile n + 2's q' is built while tile n's scores run;
+            // one buffer: each tile builds its own before its RoPE
+            if (nqb == 2 && n_first < s1) build_q(n_first, rope_of(n_first));
             for (int n = n_first; n < s1; n += 2) {
                 const int st = n % ns;
                 const int local = (int)(f0 + n - hbase);
@@ -441,146 +471,127 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 const int valid = (lim - j0) < span ? (lim - j0) : span;
                 // the next tile's query rotation, loaded now, used after this tile's RoPE
                 const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
-                if (nqb == 1) {
-                    build_q(n, rope_of(n));
-                    group_sync(grp);
-                }
-                const float* qcur = qbb + (nqb == 2 ? ((n >> 1) & 1) : 0) * kQFloats;
-                float2 sacc[G];
-#pragma unroll
-                for (int h = 0; h < G; ++h) sacc[h] = make_float2(0.f, 0.f);
-                // rotate this row of K^ by R_t and take its scores against q'
+                if (nqb == 1) build_q(n, rope_of(n));
+                // rotate this thread's half of the row of K^ by R_t, store back as fp16 pairs
                 if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 if (win && !mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) fail();
                 const uint4* krow = reinterpret_cast<const uint4*>(stage + st * stage_bytes);
 #pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 16) {
-                    uint32_t x1[16], x2[16], cc[16], ss[16];
+                for (int cc0 = 0; cc0 < 32; cc0 += 8) {
+                    const int c0 = sub * 32 + cc0;
+                    uint32_t x1[8], x2[8], cc[8], ss[8], nn[8];
                     if (!win) {
-                        tmem_ld16(kh + lane_base + c0, x1);
-                        tmem_ld16(kh + lane_base + 64 + c0, x2);
+                        tmem_ld8(kh + lane_base + c0, x1);
+                        tmem_ld8(kh + lane_base + 64 + c0, x2);
                     } else {
                         // this row's exact key, dims c0.. and 64 + c0.. (blocked 8 x 8 layout)
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
+                            uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
+                            if (row < valid) q4 = krow[((row >> 3) * 16 + ((half * 64 + c0) >> 3)) * 8 + (row & 7)];
+                            uint32_t* dst = half ? x2 : x1;
+                            const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                            for (int v = 0; v < 2; ++v) {
-                                uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
-                                if (row < valid)
-                                    q4 = krow[((row >> 3) * 16 + ((half * 64 + c0) >> 3) + v) * 8 + (row & 7)];
-                                uint32_t* dst = half ? x2 : x1;
-                                const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    dst[v * 8 + 2 * e] = w4[e] << 16;            // low bf16 -> fp32
-                                    dst[v * 8 + 2 * e + 1] = w4[e] & 0xFFFF0000u; // high bf16 -> fp32
-                                }
+                            for (int e = 0; e < 4; ++e) {
+                                dst[2 * e] = w4[e] << 16;             // low bf16 -> fp32
+                                dst[2 * e + 1] = w4[e] & 0xFFFF0000u;  // high bf16 -> fp32
                             }
                         }
                     }
-                    uint32_t nn[16];
-                    tmem_ld16(tcs + lane_base + c0, cc);
-                    tmem_ld16(tcs + lane_base + 64 + c0, ss);
-                    tmem_ld16(tcs + lane_base + 128 + c0, nn);
+                    tmem_ld8(tcs + lane_base + c0, cc);
+                    tmem_ld8(tcs + lane_base + 64 + c0, ss);
+                    tmem_ld8(tcs + lane_base + 128 + c0, nn);
                     tmem_wait_ld();
-                    if (c0 == 48) {
-                        // every K^ column of this row is in registers: the issuer may
-                        // rebuild the group's next tile into the buffer
-                        tc_fence_before();
-                        mbar_arrive(&bars->kfree[grp]);
-                    }
                     // (k1, k2) -> (k1 c - k2 s, k1 s + k2 c), two columns per packed
-                    // fp32 op; then the scores of the G query heads, q' (fp32, the same
-                    // for every row) read from shared memory as broadcasts
+                    // fp32 op, rounded to fp16 pairs for the score MMA
 #pragma unroll
-                    for (int u = 0; u < 16; u += 4) {
-                        float2 y1[2], y2[2];
-#pragma unroll
-                        for (int w = 0; w < 2; ++w) {
-                            const int uu = u + 2 * w;
-                            const float2 k1 = make_float2(__uint_as_float(x1[uu]), __uint_as_float(x1[uu + 1]));
-                            const float2 k2 = make_float2(__uint_as_float(x2[uu]), __uint_as_float(x2[uu + 1]));
-                            const float2 co = make_float2(__uint_as_float(cc[uu]), __uint_as_float(cc[uu + 1]));
-                            const float2 si = make_float2(__uint_as_float(ss[uu]), __uint_as_float(ss[uu + 1]));
-                            const float2 ns = make_float2(__uint_as_float(nn[uu]), __uint_as_float(nn[uu + 1]));
-                            y1[w] = __ffma2_rn(k1, co, __fmul2_rn(k2, ns));
-                            y2[w] = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
-                        }
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float4 qa = *reinterpret_cast<const float4*>(qcur + h * d + c0 + u);
-                            const float4 qc = *reinterpret_cast<const float4*>(qcur + h * d + 64 + c0 + u);
-                            sacc[h] = __ffma2_rn(y1[0], make_float2(qa.x, qa.y), sacc[h]);
-                            sacc[h] = __ffma2_rn(y1[1], make_float2(qa.z, qa.w), sacc[h]);
-                            sacc[h] = __ffma2_rn(y2[0], make_float2(qc.x, qc.y), sacc[h]);
-                            sacc[h] = __ffma2_rn(y2[1], make_float2(qc.z, qc.w), sacc[h]);
-                        }
+                    for (int u = 0; u < 8; u += 2) {
+                        const float2 k1 = make_float2(__uint_as_float(x1[u]), __uint_as_float(x1[u + 1]));
+                        const float2 k2 = make_float2(__uint_as_float(x2[u]), __uint_as_float(x2[u + 1]));
+                        const float2 co = make_float2(__uint_as_float(cc[u]), __uint_as_float(cc[u + 1]));
+                        const float2 si = make_float2(__uint_as_float(ss[u]), __uint_as_float(ss[u + 1]));
+                        const float2 ns2 = make_float2(__uint_as_float(nn[u]), __uint_as_float(nn[u + 1]));
+                        const float2 y1 = __ffma2_rn(k1, co, __fmul2_rn(k2, ns2));
+                        const float2 y2 = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
+                        // column c0 + u <- fp16 (dim c0 + u, dim 64 + c0 + u)
+                        const __half2 p0 = __floats2half2_rn(y1.x, y2.x);
+                        const __half2 p1 = __floats2half2_rn(y1.y, y2.y);
+                        x1[u] = *reinterpret_cast<const uint32_t*>(&p0);
+                        x1[u + 1] = *reinterpret_cast<const uint32_t*>(&p1);
                     }
+                    tmem_st8(kh + lane_base + c0, x1);
                 }
-                // the next tile's q' goes to the other buffer (published to the group
-                // by this tile's softmax barrier)
+                // this half of the row is rotated: sub 0 holds dims 0..31 and
+                // 64..95 (the first score MMA half), sub 1 the rest
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(sub == 0 ? &bars->krot_ready[grp] : &bars->krot_b[grp]);
+                // the next tile's q' goes to the other buffer while this tile's scores run
                 if (nqb == 2 && n + 2 < s1) build_q(n + 2, rq_next);
                 // this group's previous tile: p^T C_V accumulated (before O is reused)
                 if (have_prev) {
                     if (!mbar_wait(&bars->o_full[grp], ((n - 2) >> 1) & 1, deadline)) fail();
                     tc_fence_after();
                     uint32_t o[16];
-                    tmem_ld16(kh + 128 + lane_base, o);
+                    tmem_ld16(kh + 144 + lane_base, o);
                     tmem_wait_ld();
                     accumulate(o, prev_win);
                 }
-                // scores and the tile max of each head
-                float sc[G];
+                // scores and the tile max of this thread's heads
+                if (!mbar_wait(&bars->s_full[grp], (n >> 1) & 1, deadline)) fail();
+                tc_fence_after();
+                uint32_t sv[16];
+                tmem_ld16(kh + 128 + lane_base, sv);
+                tmem_wait_ld();
+                float sc[kH];
                 bool over = false;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float raw = sacc[h].x + sacc[h].y;
-                    sc[h] = (row < valid) ? raw * a.scale : -INFINITY;
-                    range_bad |= row < valid && !(fabsf(raw) <= 3.0e38f);   // inf or NaN
-                    over |= sc[h] > m_run[h] + kLazyMax;   // always true while m_run = -inf
+                for (int hh = 0; hh < kH; ++hh) {
+                    const int h = sub * kH + hh;
+                    const bool mine = h < G;
+                    const int hc = mine ? h : 0;
+                    const float raw = __uint_as_float(sv[hc]) + __uint_as_float(sv[G + hc]);
+                    sc[hh] = (row < valid && mine) ? raw * a.scale : -INFINITY;
+                    range_bad |= row < valid && mine && !(fabsf(raw) <= 3.0e38f);   // inf or NaN
+                    over |= sc[hh] > m_run[hh] + kLazyMax;   // always true while m_run = -inf
                 }
-                // p of this row, bf16 hi parts then lo parts, one or two 16-byte rows
-                auto store_p = [&](const float (&pv)[G]) {
-                    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                    __nv_bfloat16 hv[2 * G];
+                // p of this row and heads, bf16 hi parts and lo parts
+                auto store_p = [&](const float (&pv)[kH]) {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        hv[h] = __float2bfloat16_rn(pv[h]);
-                        hv[G + h] = __float2bfloat16_rn(pv[h] - __bfloat162float(hv[h]));
+                    for (int hh = 0; hh < kH; ++hh) {
+                        const int h = sub * kH + hh;
+                        if (h >= G) continue;
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(pv[hh]);
+                        pbb[pb_off(h, row)] = hi;
+                        pbb[pb_off(G + h, row)] = __float2bfloat16_rn(pv[hh] - __bfloat162float(hi));
                     }
-#pragma unroll
-                    for (int e = 0; e < 2 * G; ++e) {
-                        const uint32_t bits = (uint32_t)__bfloat16_as_ushort(hv[e]);
-                        w[e >> 1] |= (e & 1) ? (bits << 16) : bits;
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(pbb + pb_off(0, row));
-                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    if (2 * G > 8) reinterpret_cast<uint4*>(pbb + pb_off(8, row))[0] = make_uint4(w[4], w[5], w[6], w[7]);
                 };
-                float pv[G];
+                float pv[kH];
 #pragma unroll
-                for (int h = 0; h < G; ++h)
-                    pv[h] = (sc[h] == -INFINITY || m_run[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_run[h]);
+                for (int hh = 0; hh < kH; ++hh)
+                    pv[hh] = (sc[hh] == -INFINITY || m_run[hh] == -INFINITY) ? 0.f : __expf(sc[hh] - m_run[hh]);
                 store_p(pv);
                 fence_async_smem();
                 tc_fence_before();
                 if (group_sync_or(grp, over)) {          // P complete; rare: exact rescale
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float wm = warp_max(sc[h]);
-                        if (lane == 0) gred[sp * 8 + h] = wm;
+                    for (int hh = 0; hh < kH; ++hh) {
+                        const int h = sub * kH + hh;
+                        const float wm = warp_max(sc[hh]);
+                        if (lane == 0 && h < G) gred[sp * 8 + h] = wm;
                     }
                     group_sync(grp);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
+                    for (int hh = 0; hh < kH; ++hh) {
+                        const int h = sub * kH + hh < G ? sub * kH + hh : 0;
                         const float tmax = fmaxf(fmaxf(gred[h], gred[8 + h]), fmaxf(gred[16 + h], gred[24 + h]));
-                        const float m_new = fmaxf(m_run[h], tmax);
-                        const float al = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
-                        pv[h] = (sc[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_new);
-                        l_thr[h] = fmaf(l_thr[h], al, pv[h]);
-                        m_run[h] = m_new;
-                        alpha[h] = al;
+                        const float m_new = fmaxf(m_run[hh], tmax);
+                        const float al = (m_run[hh] == -INFINITY) ? 0.f : __expf(m_run[hh] - m_new);
+                        pv[hh] = (sc[hh] == -INFINITY) ? 0.f : __expf(sc[hh] - m_new);
+                        l_thr[hh] = fmaf(l_thr[hh], al, pv[hh]);
+                        m_run[hh] = m_new;
+                        alpha[hh] = al;
                     }
                     store_p(pv);
                     fence_async_smem();
@@ -588,9 +599,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     group_sync(grp);                  // rescaled P complete, maxima read
                 } else {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        l_thr[h] += pv[h];
-                        alpha[h] = 1.f;
+                    for (int hh = 0; hh < kH; ++hh) {
+                        l_thr[hh] += pv[hh];
+                        alpha[hh] = 1.f;
                     }
                 }
                 if (gt == 0) mbar_arrive(&bars->p_ready[grp]);   // P of tile n complete
@@ -603,14 +614,15 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 if (!mbar_wait(&bars->o_full[grp], (last >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 uint32_t o[16];
-                tmem_ld16(kh + 128 + lane_base, o);
+                tmem_ld16(kh + 144 + lane_base, o);
                 tmem_wait_ld();
                 accumulate(o, prev_win);
             }
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float ws = warp_sum(l_thr[h]);
-                if (lane == 0) gred[32 + sp * 8 + h] = ws;
+            for (int hh = 0; hh < kH; ++hh) {
+                const int h = sub * kH + hh;
+                const float ws = warp_sum(l_thr[hh]);
+                if (lane == 0 && h < G) gred[32 + sp * 8 + h] = ws;
             }
             tc_fence_before();
             group_sync(grp);
@@ -622,12 +634,14 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             {
                 const int slot = 2 * (cta - c_first) + grp;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
+                for (int hh = 0; hh < kH; ++hh) {
+                    const int h = sub * kH + hh;
+                    if (h >= G) continue;
                     float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
-                    if (acc_ok) Pp[2 + c_acc] = acc[h];
-                    Pp[2 + rV + row] = accd[h];   // d = 128 = group size: row owns dim row
-                    if (gt == 0) {
-                        Pp[0] = m_run[h];
+                    if (acc_ok) Pp[2 + c_acc] = acc[hh];
+                    Pp[2 + rV + row] = accd[hh];   // d = 128 rows: row owns dim row
+                    if (row == 0) {
+                        Pp[0] = m_run[hh];
                         Pp[1] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
                     }
                 }
@@ -649,9 +663,12 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             }
             group_sync(grp);
             if (last_flag[grp]) {
+                // thread (sub, j = gt & 127): column j of the r_V-wide sums and dim j
+                // of the d-wide sums, for the sub's query heads
+                const int j = gt & 127;
                 const int nsl = 2 * (c_last - c_first + 1);
                 const float* Pbase = a.partial + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * a.splits_total * stride;
-                const float* br = a.V.basis + (((int64_t)a.layer * BH + head) * d + gt) * rV;
+                const float* br = a.V.basis + (((int64_t)a.layer * BH + head) * d + j) * rV;
                 for (int c = 0; c < rV; c += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(br + c));
                 // scratch: m, l of every (slot, head) in the group's q' buffers
                 // (nqb x 4 KB; the host keeps slots x g <= nqb x 512), the [g][r_V]
@@ -661,92 +678,105 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 float* sacc = reinterpret_cast<float*>(pbb);
                 float* sml = reinterpret_cast<float*>(qbb);   // [slot][G] m, then [slot][G] l
                 const int nml = nsl * G;
-                for (int e = gt; e < nml; e += 128) {
+                for (int e = gt; e < nml; e += 256) {
                     const float* q = Pbase + ((int64_t)(e % G) * a.splits_total + e / G) * stride;
                     sml[e] = __ldcg(q);
                     sml[nml + e] = __ldcg(q + 1);
                 }
-                // this thread's columns (acc column gt, exact-row dim gt) of kC slots
-                // per batch; the first batch is in flight across the barrier
-                constexpr int kC = 32 / G;
-                float xa[kC][G], xd[kC][G];
+                // this thread's columns of kC slots per batch; the first batch is in
+                // flight across the barrier
+                constexpr int kC = G >= 16 ? 1 : 16 / G;
+                float xa[kC][kH], xd[kC][kH];
                 auto load_batch = [&](int s0) {
 #pragma unroll
-                    for (int j = 0; j < kC; ++j)
+                    for (int jj = 0; jj < kC; ++jj)
 #pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float* q = Pbase + ((int64_t)h * a.splits_total + s0 + j) * stride;
-                            const bool in = s0 + j < nsl;
-                            xa[j][h] = (in && gt < rV) ? __ldcg(q + 2 + gt) : 0.f;
-                            xd[j][h] = in ? __ldcg(q + 2 + rV + gt) : 0.f;
+                        for (int hh = 0; hh < kH; ++hh) {
+                            const int h = sub * kH + hh < G ? sub * kH + hh : 0;
+                            const float* q = Pbase + ((int64_t)h * a.splits_total + s0 + jj) * stride;
+                            const bool in = s0 + jj < nsl && sub * kH + hh < G;
+                            xa[jj][hh] = (in && j < rV) ? __ldcg(q + 2 + j) : 0.f;
+                            xd[jj][hh] = in ? __ldcg(q + 2 + rV + j) : 0.f;
                         }
                 };
                 load_batch(0);
                 group_sync(grp);
-                float M[G], L[G], va[G], vd[G];
+                float M[kH], L[kH], va[kH], vd[kH];
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    M[h] = -INFINITY;
-                    L[h] = 0.f;
-                    va[h] = 0.f;
-                    vd[h] = 0.f;
+                for (int hh = 0; hh < kH; ++hh) {
+                    M[hh] = -INFINITY;
+                    L[hh] = 0.f;
+                    va[hh] = 0.f;
+                    vd[hh] = 0.f;
                 }
                 for (int sl = 0; sl < nsl; ++sl)
 #pragma unroll
-                    for (int h = 0; h < G; ++h) M[h] = fmaxf(M[h], sml[sl * G + h]);
+                    for (int hh = 0; hh < kH; ++hh) {
+                        const int h = sub * kH + hh < G ? sub * kH + hh : 0;
+                        M[hh] = fmaxf(M[hh], sml[sl * G + h]);
+                    }
                 for (int s0 = 0; s0 < nsl; s0 += kC) {
                     if (s0 > 0) load_batch(s0);
 #pragma unroll
-                    for (int j = 0; j < kC; ++j)
+                    for (int jj = 0; jj < kC; ++jj)
 #pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            if (s0 + j >= nsl) continue;
-                            const float m = sml[(s0 + j) * G + h];
-                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M[h]);
-                            L[h] = fmaf(w, sml[nml + (s0 + j) * G + h], L[h]);
-                            va[h] = fmaf(w, xa[j][h], va[h]);
-                            vd[h] = fmaf(w, xd[j][h], vd[h]);   // exact-row sum, dim gt
+                        for (int hh = 0; hh < kH; ++hh) {
+                            if (s0 + jj >= nsl) continue;
+                            const int h = sub * kH + hh < G ? sub * kH + hh : 0;
+                            const float m = sml[(s0 + jj) * G + h];
+                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M[hh]);
+                            L[hh] = fmaf(w, sml[nml + (s0 + jj) * G + h], L[hh]);
+                            va[hh] = fmaf(w, xa[jj][hh], va[hh]);
+                            vd[hh] = fmaf(w, xd[jj][hh], vd[hh]);   // exact-row sum, dim j
                         }
                 }
 #pragma unroll
-                for (int h = 0; h < G; ++h)
-                    if (gt < rV) sacc[h * rV + gt] = va[h];
+                for (int hh = 0; hh < kH; ++hh) {
+                    const int h = sub * kH + hh;
+                    if (h < G && j < rV) sacc[h * rV + j] = va[hh];
+                }
                 group_sync(grp);
-                // out[h][i] = (sum_c acc[h][c] B_V[i][c] + accd[h][i]) / L_h, i = gt
+                // out[h][i] = (sum_c acc[h][c] B_V[i][c] + accd[h][i]) / L_h, i = j
 #pragma unroll 4
                 for (int c = 0; c < rV; c += 4) {
                     const float4 b4 = *reinterpret_cast<const float4*>(br + c);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
+                    for (int hh = 0; hh < kH; ++hh) {
+                        const int h = sub * kH + hh < G ? sub * kH + hh : 0;
                         const float4 s4 = *reinterpret_cast<const float4*>(sacc + h * rV + c);
-                        vd[h] = fmaf(s4.x, b4.x, vd[h]);
-                        vd[h] = fmaf(s4.y, b4.y, vd[h]);
-                        vd[h] = fmaf(s4.z, b4.z, vd[h]);
-                        vd[h] = fmaf(s4.w, b4.w, vd[h]);
+                        vd[hh] = fmaf(s4.x, b4.x, vd[hh]);
+                        vd[hh] = fmaf(s4.y, b4.y, vd[hh]);
+                        vd[hh] = fmaf(s4.z, b4.z, vd[hh]);
+                        vd[hh] = fmaf(s4.w, b4.w, vd[hh]);
                     }
                 }
 #pragma unroll
-                for (int h = 0; h < G; ++h)
-                    a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + gt] = vd[h] / L[h];
+                for (int hh = 0; hh < kH; ++hh) {
+                    const int h = sub * kH + hh;
+                    if (h < G) a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + j] = vd[hh] / L[hh];
+                }
                 group_sync(grp);                      // P buffer free again
             }
             n0 = s1;
         }
         if (__any_sync(0xffffffffu, range_bad) && lane == 0) atomicOr(a.status, kStatusRange);
-    } else if (warp >= 10) {
-        // ---------------- MMA issuer of group warp - 10 ----------------
+    } else if (warp == 2 || warp == 3) {
+        // ---------------- MMA issuer of group warp - 2 ----------------
         // per tile n of the group: K^ = C_K (B_hi + B_lo)^T (issued as soon as the
-        // group's epilogue has read the previous tile's K^ out of the buffer),
-        // values once P is written
-        const int grp = warp - 10;
+        // group's previous score MMA has released the K^ buffer), scores once the
+        // epilogue has rotated K^ and written q', values once P is written
+        const int grp = warp - 2;
         if (lane == 0) {
             const int MV = rV <= 64 ? 64 : 128;
             const uint32_t idesc_k = idesc_f32acc(1, kTile, d, 0, 0);
+            const uint32_t idesc_s = idesc_f32acc(0, kTile, kQN, 0, 0);   // fp16 x fp16
             const uint32_t idesc_o = idesc_f32acc(1, MV, kPN, 1, 1);
             const uint32_t idesc_ow = idesc_f32acc(1, kTile, kPN, 1, 1);   // exact rows: M = d
             const uint32_t sbo_k = (uint32_t)(rK / 8) * 128;
+            const uint32_t sbo_q = (kTile / 8) * 128;
             const uint32_t lbo_v = (uint32_t)(rV / 8) * 128;
             const uint32_t kh = tmem + grp * kBufCols;
+            const uint32_t qg = smem_u32(qb + nqb * grp * kQWords);
             const uint32_t p0 = smem_u32(pb + grp * kPN * kTile);
             // K^ of tile n into this group's buffer; exact-row tiles need none
             auto recon = [&](int n, int hb, bool win) -> bool {
@@ -791,10 +821,33 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 for (int n = n_first; ok && n < s1; n += 2) {
                     const int st = n % ns;
                     const bool win = (int)(f0 + n - hbase) >= tiles_c;
-                    // K^ of tile n read by the epilogue: rebuild tile n + 2 while the
-                    // epilogue computes this tile's scores and softmax.  Its data sits in
-                    // stage (n + 2) % ns, which with two stages is tile n's own: then it
-                    // has to wait for value(n) below.
+                    // scores in two halves of the head dimension, each once the epilogue
+                    // has rotated it: dims 0..31 and 64..95 (k-steps 0..3, 8..11), then
+                    // 32..63 and 96..127 (k-steps 4..7, 12..15)
+                    const uint32_t q0 = qg + (nqb == 2 ? ((n >> 1) & 1) : 0) * (kQWords * 4);
+                    bool got = true;
+                    for (int half = 0; half < 2; ++half) {
+                        if (!mbar_wait(half ? &bars->krot_b[grp] : &bars->krot_ready[grp], (n >> 1) & 1,
+                                       deadline)) {
+                            got = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        for (int j = 0; j < 4; ++j) {
+                            const int ks = 4 * half + j;   // K = 16: 8 TMEM columns per step
+                            mma_f16_ts(kh + 128, kh + ks * 8, desc_noswizzle(q0 + ks * 256, 128, sbo_q),
+                                       idesc_s, (half | j) != 0);
+                        }
+                    }
+                    if (!got) {
+                        ok = false;
+                        break;
+                    }
+                    mma_commit(&bars->s_full[grp]);
+                    mma_commit(&bars->kfree[grp]);
+                    // K_rot of tile n consumed: rebuild tile n + 2 while the epilogue runs
+                    // this tile's softmax.  Its data sits in stage (n + 2) % ns, which with
+                    // two stages is tile n's own: then it has to wait for value(n) below.
                     auto next_recon = [&]() {
                         return mbar_wait(&bars->kfree[grp], (n >> 1) & 1, deadline) &&
                                recon(n + 2, hb, (int)(f0 + n + 2 - hbase) >= tiles_c);
@@ -811,13 +864,13 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     if (!win) {
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + P.stage_k);
                         for (int ks = 0; ks < kTile / 16; ++ks)
-                            mma_f16_ss(kh + 128, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
+                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * lbo_v, lbo_v, 128),
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_o, ks != 0);
                     } else {
                         // O = V^T P over wt exact rows: A = V tile, MN-major, M = d
                         const uint32_t v0 = smem_u32(stage + st * stage_bytes + win_bytes);
                         for (int ks = 0; ks < wt / 16; ++ks)
-                            mma_f16_ss(kh + 128, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
+                            mma_f16_ss(kh + 144, desc_noswizzle(v0 + ks * 2 * 2048, 2048, 128),
                                        desc_noswizzle(p0 + ks * 512, 256, 128), idesc_ow, ks != 0);
                     }
                     mma_commit(&bars->o_full[grp]);

@@ -64,6 +64,11 @@ def _run(rk, rv, coef, H=8, batch=2, tokens=1280, window=256, tol=1e-4, defer=Fa
                 ok[b].fold(defer=defer)
                 ov[b].fold(defer=defer)
             folds += 1
+            if defer and folds % 8 == 0:       # max_deferred postponed folds, then the rewrite
+                cache.sync(0)
+                for b in range(batch):
+                    ok[b].sync()
+                    ov[b].sync()
     if defer:
         cache.sync(0)
         for b in range(batch):
@@ -120,10 +125,11 @@ def test_joint_persistent_bytes():
     cfg = ik.Config(batch=batch, layers=1, kv_heads=H, q_heads=32, rank_k=64, rank_v=96, window=256,
                     max_tokens=1024, kv_dtype=ik.BF16, coef_dtype=ik.BF16, joint=1)
     cache = ik.Cache(cfg)
-    k = torch.randn(batch, H, 512, 128, dtype=torch.bfloat16, device="cuda")
-    ready = cache.append(0, k, k.clone())
-    for _ in range(ready):
-        cache.compress_block(0)
+    for _ in range(8):
+        k = torch.randn(batch, H, 64, 128, dtype=torch.bfloat16, device="cuda")
+        ready = cache.append(0, k, k.clone())
+        for _ in range(ready):
+            cache.compress_block(0)
     T, n_c = cache.counts(0)
     kept, full = cache.kv_bytes()
     want = batch * (n_c * (64 + 96) * 2 + (D + 1) * (64 + 96) * 4) + batch * H * 2 * (T - n_c) * 128 * 2
