@@ -58,6 +58,8 @@ struct iskv_cache {
     float* newrows_k = nullptr;
     float* newrows_v = nullptr;
     float* wide = nullptr;        // joint-head fold scratch
+    __nv_bfloat16* qws_k = nullptr;   // coded caches: one layer's coefficients as bf16
+    __nv_bfloat16* qws_v = nullptr;   // (the tensor-core decode's workspace)
     float* partial = nullptr;
     int* done = nullptr;          // per-head arrival counters of the fused decode combine
     float2* rope = nullptr;
@@ -241,7 +243,7 @@ void free_all(iskv_cache* h) {
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
                     h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out,
                     h->qcodes_k, h->qcodes_v, h->qscales_k, h->qscales_v, h->newrows_k, h->newrows_v,
-                    h->wide};
+                    h->wide, h->qws_k, h->qws_v};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -419,6 +421,14 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         rc = rc ? rc : dalloc(&h->qscales_v, qs_bytes);
         rc = rc ? rc : dalloc(&h->newrows_k, heads * kBlock * c.rank_k * sizeof(float));
         rc = rc ? rc : dalloc(&h->newrows_v, heads * kBlock * c.rank_v * sizeof(float));
+        if (c.kv_dtype == ISKV_BF16) {   // the tensor-core decode reads codes expanded per call
+            rc = rc ? rc : dalloc(&h->qws_k, (size_t)h->BH * h->n_max * c.rank_k * 2);
+            rc = rc ? rc : dalloc(&h->qws_v, (size_t)h->BH * h->n_max * c.rank_v * 2);
+            if (rc == ISKV_OK &&
+                (cudaMemsetAsync(h->qws_k, 0, (size_t)h->BH * h->n_max * c.rank_k * 2, s) != cudaSuccess ||
+                 cudaMemsetAsync(h->qws_v, 0, (size_t)h->BH * h->n_max * c.rank_v * 2, s) != cudaSuccess))
+                rc = ISKV_ERR_CUDA;
+        }
     }
     rc = rc ? rc : dalloc(&h->basis_k, heads * d * c.rank_k * 4);
     rc = rc ? rc : dalloc(&h->basis_v, heads * d * c.rank_v * 4);
@@ -711,14 +721,28 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.n_c = h->n_c[layer];
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
     const int sms = h->sms;
-    if (h->use_tc && !c.coef_quant && c.coef_dtype == ISKV_BF16 && c.kv_dtype == ISKV_BF16 &&
-        decode_tc_supports_group(a.g)) {
+    const bool coded_tc = c.coef_quant && h->qws_k != nullptr;
+    if (h->use_tc && (coded_tc || (!c.coef_quant && c.coef_dtype == ISKV_BF16)) &&
+        c.kv_dtype == ISKV_BF16 && decode_tc_supports_group(a.g)) {
         // one persistent tensor-core kernel, one CTA per SM, over the flattened
         // (head, tile) space: 128-token tiles of folded rows, then 64-token
         // tiles of exact rows, all under one online softmax per head
         DecodeTcArgs t{};
         t.K = a.K;
         t.V = a.V;
+        if (coded_tc) {
+            // coded coefficients: this layer's rows expanded to bf16 tiles in the
+            // workspace, then the same tensor-core decode
+            CU(launch_expand_codes(a.K, layer, a.n_c, h->qws_k, s));
+            CU(launch_expand_codes(a.V, layer, a.n_c, h->qws_v, s));
+            for (FactorView* f : {&t.K, &t.V}) {
+                f->coef = f == &t.K ? (void*)h->qws_k : (void*)h->qws_v;
+                f->quant = 0;
+                f->coef_bf16 = 1;
+                f->coef_blocked = 1;
+                f->coef_ws = 1;
+            }
+        }
         t.q = qd;
         t.partial = h->partial;
         t.rope = a.rope;

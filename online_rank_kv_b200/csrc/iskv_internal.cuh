@@ -98,6 +98,7 @@ struct FactorView {
     // h * 128 .. h * 128 + 127).  0 or 1: one factor per head.
     int coef_div;
     float* wide;         // joint fold scratch: per factor [D x (r+64)] + [D x 64] + [D x r]
+    int coef_ws;         // 1: coef holds one layer only (a decode workspace): instance = head
 };
 
 // Factor instance (coefficients, sigma, postponed W_top) of head instance hidx.
@@ -259,6 +260,8 @@ cudaError_t launch_resync_quant(const FactorView& f, const ResyncLaunch& rl, cud
 cudaError_t launch_quant_new_rows(const FactorView& f, const FoldLaunch& fl, cudaStream_t s);
 cudaError_t launch_quant_rows(const FactorView& f, const float* rows, int64_t n, uint32_t* codes,
                               float* scales, cudaStream_t s);
+cudaError_t launch_expand_codes(const FactorView& f, int layer, int64_t rows, __nv_bfloat16* dst,
+                                cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
 bool decode_tc_supports_group(int g);
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb, int wt);

@@ -16,37 +16,34 @@
 //
 // Persistent design, one CTA per SM; the flattened (head, tile) space is cut
 // into contiguous runs of equal cost (tiles, plus a fixed charge for every
-// head a run enters after its first), one run per CTA.  Per CTA 20 warps:
+// head a run enters after its first), one run per CTA.  Per CTA 12 warps:
 //   warp 0  producer: 1-D bulk copies (TMA engine) of the C_K and C_V tiles
 //           or of the exact K and V rows (all contiguous in the blocked
 //           layout) into an NS-stage ring, and of the bf16 hi/lo basis and
 //           the bf16 queries of each head it visits;
 //   warp 1  TMEM allocation;
-//   warps 2-3 MMA issuer of group 0 / 1:
-//           * K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens, N=128 dims,
-//             fp32 accumulator in TMEM, rebuilt two tiles ahead;
-//           * scores S = K_rot q'^T, kind::f16 with A from TMEM and q' as
-//             fp16 hi+lo parts in the N dimension, issued in two halves of
-//             the head dimension as the epilogue finishes rotating them;
-//           * O = C_V^T P (kind::f16, C_V tile read MN-major in place; for
-//             exact rows O = V^T P with M = d);
-//   warps 4-19 epilogue, two ping-pong groups of 8 warps (group = tile
-//           parity), two threads per token row: the row's two halves (subs)
-//           each take half of the RoPE frequencies and half of the query
-//           heads, so each SM sub-partition runs four epilogue warps:
-//           * rotate its half of the row of K^ by R_t (t = row within the
-//             tile; the row's cos/sin(t w_i) sit in spare TMEM columns) and
-//             write it back to TMEM as fp16 pairs (dim i, dim 64 + i) per
-//             column; the query is pre-rotated per tile by R_{j0}^T (j0 =
-//             tile start), so q'.(R_t k) = q.(R_{j0+t} k); each half starts
-//             its own score MMA half;
-//           * online softmax of its query heads with a lazily updated maximum;
+//   warps 2-9 epilogue, two ping-pong groups of 4 warps (group = tile
+//           parity), one token row per thread:
+//           * rotate its row of K^ by R_t (t = row within the tile; the
+//             row's cos/sin(t w_i) sit in spare TMEM columns) and write it
+//             back to TMEM as fp16 pairs (dim i, dim 64 + i) per column; the
+//             query is pre-rotated per tile by R_{j0}^T (j0 = tile start), so
+//             q'.(R_t k) = q.(R_{j0+t} k);
+//           * online softmax per query head with a lazily updated maximum;
 //           * p as bf16 hi+lo parts for the value MMA;
 //           * at the end of a head the group publishes its own partial
 //             (m, l, r_V-wide and d-wide sums); the last group to publish
 //             a head's partial merges them all by log-sum-exp, applies
 //             B_V^T once per query head and writes the output.  The two
 //             groups never wait for each other.
+//   warps 10-11 MMA issuer of group 0 / 1:
+//           * K^ = C_K (B_hi + B_lo)^T, kind::f16, M=128 tokens, N=128 dims,
+//             fp32 accumulator in TMEM, rebuilt two tiles ahead;
+//           * scores S = K_rot q'^T, kind::f16 with A from TMEM and q' as
+//             fp16 hi+lo parts in the N dimension, issued in two halves of
+//             the head dimension as the epilogue finishes rotating them;
+//           * O = C_V^T P (kind::f16, C_V tile read MN-major in place; for
+//             exact rows O = V^T P with M = d).
 // Rotated keys are held in fp16 (finite for |k| < 65504; the same 11-bit
 // significand as tf32); the query as fp16 hi + lo parts keeps ~22 bits.
 // Every mbarrier wait is bounded; on timeout the CTA records
@@ -67,8 +64,8 @@ using namespace tc;
 constexpr int kTile = 128;
 // exact-row tiles have 64 or 32 rows (the host's choice, win_rows): either
 // divides the ring and the protected-row capacity, so a tile never wraps
-constexpr int kThreads = 640;
-constexpr int kEpi = 512;        // epilogue threads (warps 4-19, two groups of 8)
+constexpr int kThreads = 384;
+constexpr int kEpi = 256;        // epilogue threads (warps 2-9, two groups of 4)
 constexpr int kQN = 16;          // N of the score MMA (q' hi and lo of g <= 8 heads)
 constexpr int kPN = 16;          // N of the value MMA (p hi and lo of g <= 8 heads)
 constexpr int kBufCols = 160;    // per TMEM buffer: K^ 128 | S 16 | O 16
@@ -110,10 +107,10 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int nbk, i
     return p;
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
-// barrier of one ping-pong group (ids 2 and 3, 256 threads)
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// barrier of one ping-pong group (ids 2 and 3, 128 threads)
 __device__ __forceinline__ void group_sync(int grp) {
-    asm volatile("bar.sync %0, 256;" ::"r"(2 + grp) : "memory");
+    asm volatile("bar.sync %0, 128;" ::"r"(2 + grp) : "memory");
 }
 // the same barrier, returning whether any of the group's threads passed true
 __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
@@ -121,7 +118,7 @@ __device__ __forceinline__ bool group_sync_or(int grp, bool pred) {
     asm volatile(
         "{\n\t.reg .pred q, p;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, %2, 256, q;\n\t"
+        "bar.red.or.pred p, %2, 128, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
         : "r"((uint32_t)pred), "r"(2 + grp)
@@ -168,7 +165,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
     const int rK = a.K.r, rV = a.V.r, ns = a.stages, nbk = a.basis_bufs, nqb = a.q_bufs;
     const int wt = a.win_rows;      // rows of an exact-row tile (64 or 32)
     constexpr int g = G;
-    constexpr int kQItems = (G * 64 + 255) / 256;   // q' items per epilogue thread
+    constexpr int kQItems = (G * 64 + 127) / 128;   // q' items per epilogue thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int d = kHeadDim;
 
@@ -210,8 +207,8 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             mbar_init(&bars->kfree[i], 1);
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->o_full[i], 1);
-            mbar_init(&bars->krot_ready[i], kEpi / 4);   // one sub of the group each
-            mbar_init(&bars->krot_b[i], kEpi / 4);
+            mbar_init(&bars->krot_ready[i], kEpi / 2);
+            mbar_init(&bars->krot_b[i], kEpi / 2);
             mbar_init(&bars->p_ready[i], 1);
         }
         for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
@@ -274,7 +271,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 uint8_t* sk = stage + st * stage_bytes;
                 if (tile < tiles_c) {
                     // a joint-head factor's coefficients are shared by its heads
-                    const int64_t cidx = coef_inst(a.K, hidx);
+                    const int64_t cidx = a.K.coef_ws ? head : coef_inst(a.K, hidx);
                     const __nv_bfloat16* gk = reinterpret_cast<const __nv_bfloat16*>(a.K.coef) +
                                               cidx * a.K.n_max * rK + (int64_t)tile * kTile * rK;
                     const __nv_bfloat16* gv = reinterpret_cast<const __nv_bfloat16*>(a.V.coef) +
@@ -309,53 +306,51 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     mbar_wait(&bars->full[n % ns], (n / ns) & 1, deadline + kWaitCycles);
             }
         }
-    } else if (warp >= 4) {
-        // ---------------- epilogue: two groups of 8 warps, alternate tiles ----------------
-        // A row (token) of a tile is shared by two threads of its group, one in
-        // each half (sub) of the group: sub s rotates frequencies 32 s .. 32 s + 31
-        // of the row and keeps the softmax of query heads s kH .. s kH + kH - 1.
-        const int ept = tid - 128;                // 0..511
+    } else if (warp >= 2 && warp < 10) {
+        // ---------------- epilogue: two groups of 4 warps, alternate tiles ----------------
+        const int ept = tid - 64;                 // 0..255
         // positions: protected [0, P), folded [P, P + n_c), window [P + n_c, T)
         const int nc32 = (int)a.n_c, T32 = (int)a.T, P32 = (int)a.K.P;
         const int Pe32 = T32 < P32 ? T32 : P32;
-        const int grp = ept >> 8;                 // tiles n with n % 2 == grp
-        const int gt = ept & 255;                 // thread within the group
-        const int sub = gt >> 7;                  // half of the frequencies and heads
+        const int grp = ept >> 7;                 // tiles n with n % 2 == grp
+        const int gt = ept & 127;                 // thread within the group
         const int sp = warp & 3;                  // TMEM sub-partition of this warp
         const int row = sp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
         const uint32_t tcs = tmem + kCsCol;
-        constexpr int kH = (G + 1) / 2;           // query heads per sub
         // this row's in-tile RoPE table (cos, sin, -sin of row * w_i) into TMEM:
-        // (group, sub) writes frequencies 16 (2 grp + sub) .. + 15
+        // group grp writes frequencies 32 grp .. 32 grp + 31, all loads issued first
         {
-            const int f0t = (2 * grp + sub) * 16;
-            float4 tv[8];
+            float4 tv[16];
             if (a.rope) {
-                const float4* src = reinterpret_cast<const float4*>(a.rope + row * 64 + f0t);
+                const float4* src = reinterpret_cast<const float4*>(a.rope + row * 64 + grp * 32);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) tv[u] = src[u];
+                for (int u = 0; u < 16; ++u) tv[u] = src[u];
             } else {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) tv[u] = make_float4(1.f, 0.f, 1.f, 0.f);
+                for (int u = 0; u < 16; ++u) tv[u] = make_float4(1.f, 0.f, 1.f, 0.f);
             }
-            uint32_t vc[16], vs[16], vn[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float4 v = tv[u];
-                vc[2 * u] = __float_as_uint(v.x);
-                vs[2 * u] = __float_as_uint(v.y);
-                vn[2 * u] = __float_as_uint(-v.y);
-                vc[2 * u + 1] = __float_as_uint(v.z);
-                vs[2 * u + 1] = __float_as_uint(v.w);
-                vn[2 * u + 1] = __float_as_uint(-v.w);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t vc[16], vs[16], vn[16];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float4 v = tv[hh * 8 + u];
+                    vc[2 * u] = __float_as_uint(v.x);
+                    vs[2 * u] = __float_as_uint(v.y);
+                    vn[2 * u] = __float_as_uint(-v.y);
+                    vc[2 * u + 1] = __float_as_uint(v.z);
+                    vs[2 * u + 1] = __float_as_uint(v.w);
+                    vn[2 * u + 1] = __float_as_uint(-v.w);
+                }
+                const int c0 = grp * 32 + hh * 16;
+                tmem_st16(tcs + lane_base + c0, vc);
+                tmem_st16(tcs + lane_base + 64 + c0, vs);
+                tmem_st16(tcs + lane_base + 128 + c0, vn);
             }
-            tmem_st16(tcs + lane_base + f0t, vc);
-            tmem_st16(tcs + lane_base + 64 + f0t, vs);
-            tmem_st16(tcs + lane_base + 128 + f0t, vn);
             tmem_wait_st();
         }
-        // the whole table written before any group's first RoPE
+        // both halves of the table written before either group's first RoPE
         tc_fence_before();
         epi_sync();
         tc_fence_after();
@@ -370,22 +365,21 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
         int qoff[kQItems][2];
 #pragma unroll
         for (int k = 0; k < kQItems; ++k) {
-            const int item = gt + 256 * k;
+            const int item = gt + 128 * k;
             const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
             qoff[k][0] = qb_off(h, i);       // hi parts of dims i, 64 + i
             qoff[k][1] = qb_off(G + h, i);   // lo parts
         }
 
-        float m_run[kH], l_thr[kH], acc[kH], accd[kH], alpha[kH];
+        float m_run[G], l_thr[G], acc[G], accd[G], alpha[G];
         // acc <- acc * alpha + (p^T C_V of a folded tile); accd likewise for exact tiles
         // (both rescaled every tile: they share the running max)
         auto accumulate = [&](const uint32_t (&o)[16], bool was_win) {
 #pragma unroll
-            for (int hh = 0; hh < kH; ++hh) {
-                const int h = sub * kH + hh < G ? sub * kH + hh : 0;
+            for (int h = 0; h < G; ++h) {
                 const float add = __uint_as_float(o[h]) + __uint_as_float(o[G + h]);
-                acc[hh] = (acc_ok && !was_win) ? fmaf(acc[hh], alpha[hh], add) : acc[hh] * alpha[hh];
-                accd[hh] = was_win ? fmaf(accd[hh], alpha[hh], add) : accd[hh] * alpha[hh];
+                acc[h] = (acc_ok && !was_win) ? fmaf(acc[h], alpha[h], add) : acc[h] * alpha[h];
+                accd[h] = was_win ? fmaf(accd[h], alpha[h], add) : accd[h] * alpha[h];
             }
         };
         bool stop = false;
@@ -399,12 +393,12 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             if (s1 > ntiles) s1 = ntiles;
             ++hs;
 #pragma unroll
-            for (int hh = 0; hh < kH; ++hh) {
-                m_run[hh] = -INFINITY;
-                l_thr[hh] = 0.f;
-                acc[hh] = 0.f;
-                accd[hh] = 0.f;
-                alpha[hh] = 0.f;
+            for (int h = 0; h < G; ++h) {
+                m_run[h] = -INFINITY;
+                l_thr[h] = 0.f;
+                acc[h] = 0.f;
+                accd[h] = 0.f;
+                alpha[h] = 0.f;
             }
             // group-uniform abort check
             if (gt == 0) epi_abort[grp] = *abort_flag;
@@ -429,13 +423,14 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                                                     : (lc - tiles_cw) * wt;
             };
             // q' = R_{j0}^T q of tile nn as fp16 hi / lo parts (the score MMA's B
-            // operand), in the group's q' buffer (nn >> 1) & 1; this thread's items
-            // (head h, frequency i = gt & 63): item gt + 256 k; their query pair
-            // (q_i, q_{i+64}) stays in registers for the whole head
+            // operand), in the group's q' buffer (nn >> 1) & 1; rv = cos / sin(j0 w_i)
+            // for i = gt & 63, the only frequency this thread rotates by
+            // this thread's items (head h, frequency i): item gt + 128 k; their
+            // query pair (q_i, q_{i+64}) stays in registers for the whole head
             float qx1[kQItems], qx2[kQItems];
 #pragma unroll
             for (int k = 0; k < kQItems; ++k) {
-                const int item = gt + 256 * k;
+                const int item = gt + 128 * k;
                 const int h = (item >> 6) < G ? (item >> 6) : 0, i = item & 63;
                 qx1[k] = n_first < s1 ? __bfloat162float(sq[h * d + i]) : 0.f;
                 qx2[k] = n_first < s1 ? __bfloat162float(sq[h * d + i + 64]) : 0.f;
@@ -444,7 +439,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 uint32_t* qd = qbb + (nqb == 2 ? ((nn >> 1) & 1) : 0) * kQWords;
 #pragma unroll
                 for (int k = 0; k < kQItems; ++k) {
-                    if (gt + 256 * k >= G * 64) break;
+                    if (gt + 128 * k >= G * 64) break;
                     const float y1 = fmaf(rv.x, qx1[k], rv.y * qx2[k]);
                     const float y2 = fmaf(rv.x, qx2[k], -rv.y * qx1[k]);
                     const __half2 hi = __floats2half2_rn(y1, y2);
@@ -472,61 +467,70 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 // the next tile's query rotation, loaded now, used after this tile's RoPE
                 const float2 rq_next = (nqb == 2 && n + 2 < s1) ? rope_of(n + 2) : make_float2(1.f, 0.f);
                 if (nqb == 1) build_q(n, rope_of(n));
-                // rotate this thread's half of the row of K^ by R_t, store back as fp16 pairs
+                // rotate this row of K^ by R_t, store back as fp16 pairs
                 if (!mbar_wait(&bars->kh_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 if (win && !mbar_wait(&bars->full[st], (n / ns) & 1, deadline)) fail();
                 const uint4* krow = reinterpret_cast<const uint4*>(stage + st * stage_bytes);
 #pragma unroll
-                for (int cc0 = 0; cc0 < 32; cc0 += 8) {
-                    const int c0 = sub * 32 + cc0;
-                    uint32_t x1[8], x2[8], cc[8], ss[8], nn[8];
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    uint32_t x1[16], x2[16], cc[16], ss[16];
                     if (!win) {
-                        tmem_ld8(kh + lane_base + c0, x1);
-                        tmem_ld8(kh + lane_base + 64 + c0, x2);
+                        tmem_ld16(kh + lane_base + c0, x1);
+                        tmem_ld16(kh + lane_base + 64 + c0, x2);
                     } else {
                         // this row's exact key, dims c0.. and 64 + c0.. (blocked 8 x 8 layout)
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
-                            uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
-                            if (row < valid) q4 = krow[((row >> 3) * 16 + ((half * 64 + c0) >> 3)) * 8 + (row & 7)];
-                            uint32_t* dst = half ? x2 : x1;
-                            const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                dst[2 * e] = w4[e] << 16;             // low bf16 -> fp32
-                                dst[2 * e + 1] = w4[e] & 0xFFFF0000u;  // high bf16 -> fp32
+                            for (int v = 0; v < 2; ++v) {
+                                uint4 q4 = make_uint4(0u, 0u, 0u, 0u);
+                                if (row < valid)
+                                    q4 = krow[((row >> 3) * 16 + ((half * 64 + c0) >> 3) + v) * 8 + (row & 7)];
+                                uint32_t* dst = half ? x2 : x1;
+                                const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    dst[v * 8 + 2 * e] = w4[e] << 16;            // low bf16 -> fp32
+                                    dst[v * 8 + 2 * e + 1] = w4[e] & 0xFFFF0000u; // high bf16 -> fp32
+                                }
                             }
                         }
                     }
-                    tmem_ld8(tcs + lane_base + c0, cc);
-                    tmem_ld8(tcs + lane_base + 64 + c0, ss);
-                    tmem_ld8(tcs + lane_base + 128 + c0, nn);
+                    uint32_t nn[16];
+                    tmem_ld16(tcs + lane_base + c0, cc);
+                    tmem_ld16(tcs + lane_base + 64 + c0, ss);
+                    tmem_ld16(tcs + lane_base + 128 + c0, nn);
                     tmem_wait_ld();
                     // (k1, k2) -> (k1 c - k2 s, k1 s + k2 c), two columns per packed
                     // fp32 op, rounded to fp16 pairs for the score MMA
 #pragma unroll
-                    for (int u = 0; u < 8; u += 2) {
+                    for (int u = 0; u < 16; u += 2) {
                         const float2 k1 = make_float2(__uint_as_float(x1[u]), __uint_as_float(x1[u + 1]));
                         const float2 k2 = make_float2(__uint_as_float(x2[u]), __uint_as_float(x2[u + 1]));
                         const float2 co = make_float2(__uint_as_float(cc[u]), __uint_as_float(cc[u + 1]));
                         const float2 si = make_float2(__uint_as_float(ss[u]), __uint_as_float(ss[u + 1]));
-                        const float2 ns2 = make_float2(__uint_as_float(nn[u]), __uint_as_float(nn[u + 1]));
-                        const float2 y1 = __ffma2_rn(k1, co, __fmul2_rn(k2, ns2));
+                        const float2 ns = make_float2(__uint_as_float(nn[u]), __uint_as_float(nn[u + 1]));
+                        const float2 y1 = __ffma2_rn(k1, co, __fmul2_rn(k2, ns));
                         const float2 y2 = __ffma2_rn(k1, si, __fmul2_rn(k2, co));
-                        // column c0 + u <- fp16 (dim c0 + u, dim 64 + c0 + u)
+                        // column c0 + u <- fp16 (dim c0 + u, dim 64 + c0 + u): over
+                        // the fp32 columns this chunk has just read
                         const __half2 p0 = __floats2half2_rn(y1.x, y2.x);
                         const __half2 p1 = __floats2half2_rn(y1.y, y2.y);
                         x1[u] = *reinterpret_cast<const uint32_t*>(&p0);
                         x1[u + 1] = *reinterpret_cast<const uint32_t*>(&p1);
                     }
-                    tmem_st8(kh + lane_base + c0, x1);
+                    tmem_st16(kh + lane_base + c0, x1);
+                    if (c0 == 16 || c0 == 48) {
+                        // dims 0..31 and 64..95 of this row are rotated (first barrier),
+                        // then the rest (second): the score MMA starts on the first half
+                        // while the second is rotated.  One barrier per half, so every
+                        // phase counts each thread exactly once.
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(c0 == 16 ? &bars->krot_ready[grp] : &bars->krot_b[grp]);
+                    }
                 }
-                // this half of the row is rotated: sub 0 holds dims 0..31 and
-                // 64..95 (the first score MMA half), sub 1 the rest
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(sub == 0 ? &bars->krot_ready[grp] : &bars->krot_b[grp]);
                 // the next tile's q' goes to the other buffer while this tile's scores run
                 if (nqb == 2 && n + 2 < s1) build_q(n + 2, rq_next);
                 // this group's previous tile: p^T C_V accumulated (before O is reused)
@@ -538,60 +542,62 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     tmem_wait_ld();
                     accumulate(o, prev_win);
                 }
-                // scores and the tile max of this thread's heads
+                // scores and the tile max of each head
                 if (!mbar_wait(&bars->s_full[grp], (n >> 1) & 1, deadline)) fail();
                 tc_fence_after();
                 uint32_t sv[16];
                 tmem_ld16(kh + 128 + lane_base, sv);
                 tmem_wait_ld();
-                float sc[kH];
+                float sc[G];
                 bool over = false;
 #pragma unroll
-                for (int hh = 0; hh < kH; ++hh) {
-                    const int h = sub * kH + hh;
-                    const bool mine = h < G;
-                    const int hc = mine ? h : 0;
-                    const float raw = __uint_as_float(sv[hc]) + __uint_as_float(sv[G + hc]);
-                    sc[hh] = (row < valid && mine) ? raw * a.scale : -INFINITY;
-                    range_bad |= row < valid && mine && !(fabsf(raw) <= 3.0e38f);   // inf or NaN
-                    over |= sc[hh] > m_run[hh] + kLazyMax;   // always true while m_run = -inf
+                for (int h = 0; h < G; ++h) {
+                    const float raw = __uint_as_float(sv[h]) + __uint_as_float(sv[G + h]);
+                    sc[h] = (row < valid) ? raw * a.scale : -INFINITY;
+                    range_bad |= row < valid && !(fabsf(raw) <= 3.0e38f);   // inf or NaN
+                    over |= sc[h] > m_run[h] + kLazyMax;   // always true while m_run = -inf
                 }
-                // p of this row and heads, bf16 hi parts and lo parts
-                auto store_p = [&](const float (&pv)[kH]) {
+                // p of this row, bf16 hi parts then lo parts, one or two 16-byte rows
+                auto store_p = [&](const float (&pv)[G]) {
+                    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                    __nv_bfloat16 hv[2 * G];
 #pragma unroll
-                    for (int hh = 0; hh < kH; ++hh) {
-                        const int h = sub * kH + hh;
-                        if (h >= G) continue;
-                        const __nv_bfloat16 hi = __float2bfloat16_rn(pv[hh]);
-                        pbb[pb_off(h, row)] = hi;
-                        pbb[pb_off(G + h, row)] = __float2bfloat16_rn(pv[hh] - __bfloat162float(hi));
+                    for (int h = 0; h < G; ++h) {
+                        hv[h] = __float2bfloat16_rn(pv[h]);
+                        hv[G + h] = __float2bfloat16_rn(pv[h] - __bfloat162float(hv[h]));
                     }
-                };
-                float pv[kH];
 #pragma unroll
-                for (int hh = 0; hh < kH; ++hh)
-                    pv[hh] = (sc[hh] == -INFINITY || m_run[hh] == -INFINITY) ? 0.f : __expf(sc[hh] - m_run[hh]);
+                    for (int e = 0; e < 2 * G; ++e) {
+                        const uint32_t bits = (uint32_t)__bfloat16_as_ushort(hv[e]);
+                        w[e >> 1] |= (e & 1) ? (bits << 16) : bits;
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(pbb + pb_off(0, row));
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (2 * G > 8) reinterpret_cast<uint4*>(pbb + pb_off(8, row))[0] = make_uint4(w[4], w[5], w[6], w[7]);
+                };
+                float pv[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    pv[h] = (sc[h] == -INFINITY || m_run[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_run[h]);
                 store_p(pv);
                 fence_async_smem();
                 tc_fence_before();
                 if (group_sync_or(grp, over)) {          // P complete; rare: exact rescale
 #pragma unroll
-                    for (int hh = 0; hh < kH; ++hh) {
-                        const int h = sub * kH + hh;
-                        const float wm = warp_max(sc[hh]);
-                        if (lane == 0 && h < G) gred[sp * 8 + h] = wm;
+                    for (int h = 0; h < G; ++h) {
+                        const float wm = warp_max(sc[h]);
+                        if (lane == 0) gred[sp * 8 + h] = wm;
                     }
                     group_sync(grp);
 #pragma unroll
-                    for (int hh = 0; hh < kH; ++hh) {
-                        const int h = sub * kH + hh < G ? sub * kH + hh : 0;
+                    for (int h = 0; h < G; ++h) {
                         const float tmax = fmaxf(fmaxf(gred[h], gred[8 + h]), fmaxf(gred[16 + h], gred[24 + h]));
-                        const float m_new = fmaxf(m_run[hh], tmax);
-                        const float al = (m_run[hh] == -INFINITY) ? 0.f : __expf(m_run[hh] - m_new);
-                        pv[hh] = (sc[hh] == -INFINITY) ? 0.f : __expf(sc[hh] - m_new);
-                        l_thr[hh] = fmaf(l_thr[hh], al, pv[hh]);
-                        m_run[hh] = m_new;
-                        alpha[hh] = al;
+                        const float m_new = fmaxf(m_run[h], tmax);
+                        const float al = (m_run[h] == -INFINITY) ? 0.f : __expf(m_run[h] - m_new);
+                        pv[h] = (sc[h] == -INFINITY) ? 0.f : __expf(sc[h] - m_new);
+                        l_thr[h] = fmaf(l_thr[h], al, pv[h]);
+                        m_run[h] = m_new;
+                        alpha[h] = al;
                     }
                     store_p(pv);
                     fence_async_smem();
@@ -599,9 +605,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     group_sync(grp);                  // rescaled P complete, maxima read
                 } else {
 #pragma unroll
-                    for (int hh = 0; hh < kH; ++hh) {
-                        l_thr[hh] += pv[hh];
-                        alpha[hh] = 1.f;
+                    for (int h = 0; h < G; ++h) {
+                        l_thr[h] += pv[h];
+                        alpha[h] = 1.f;
                     }
                 }
                 if (gt == 0) mbar_arrive(&bars->p_ready[grp]);   // P of tile n complete
@@ -619,10 +625,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 accumulate(o, prev_win);
             }
 #pragma unroll
-            for (int hh = 0; hh < kH; ++hh) {
-                const int h = sub * kH + hh;
-                const float ws = warp_sum(l_thr[hh]);
-                if (lane == 0 && h < G) gred[32 + sp * 8 + h] = ws;
+            for (int h = 0; h < G; ++h) {
+                const float ws = warp_sum(l_thr[h]);
+                if (lane == 0) gred[32 + sp * 8 + h] = ws;
             }
             tc_fence_before();
             group_sync(grp);
@@ -634,14 +639,12 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             {
                 const int slot = 2 * (cta - c_first) + grp;
 #pragma unroll
-                for (int hh = 0; hh < kH; ++hh) {
-                    const int h = sub * kH + hh;
-                    if (h >= G) continue;
+                for (int h = 0; h < G; ++h) {
                     float* Pp = a.partial + (((int64_t)bq * a.Hq + kvh * g + h) * a.splits_total + slot) * stride;
-                    if (acc_ok) Pp[2 + c_acc] = acc[hh];
-                    Pp[2 + rV + row] = accd[hh];   // d = 128 rows: row owns dim row
-                    if (row == 0) {
-                        Pp[0] = m_run[hh];
+                    if (acc_ok) Pp[2 + c_acc] = acc[h];
+                    Pp[2 + rV + row] = accd[h];   // d = 128 = group size: row owns dim row
+                    if (gt == 0) {
+                        Pp[0] = m_run[h];
                         Pp[1] = gred[32 + h] + gred[40 + h] + gred[48 + h] + gred[56 + h];
                     }
                 }
@@ -663,12 +666,9 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             }
             group_sync(grp);
             if (last_flag[grp]) {
-                // thread (sub, j = gt & 127): column j of the r_V-wide sums and dim j
-                // of the d-wide sums, for the sub's query heads
-                const int j = gt & 127;
                 const int nsl = 2 * (c_last - c_first + 1);
                 const float* Pbase = a.partial + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * a.splits_total * stride;
-                const float* br = a.V.basis + (((int64_t)a.layer * BH + head) * d + j) * rV;
+                const float* br = a.V.basis + (((int64_t)a.layer * BH + head) * d + gt) * rV;
                 for (int c = 0; c < rV; c += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(br + c));
                 // scratch: m, l of every (slot, head) in the group's q' buffers
                 // (nqb x 4 KB; the host keeps slots x g <= nqb x 512), the [g][r_V]
@@ -678,94 +678,84 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 float* sacc = reinterpret_cast<float*>(pbb);
                 float* sml = reinterpret_cast<float*>(qbb);   // [slot][G] m, then [slot][G] l
                 const int nml = nsl * G;
-                for (int e = gt; e < nml; e += 256) {
+                for (int e = gt; e < nml; e += 128) {
                     const float* q = Pbase + ((int64_t)(e % G) * a.splits_total + e / G) * stride;
                     sml[e] = __ldcg(q);
                     sml[nml + e] = __ldcg(q + 1);
                 }
-                // this thread's columns of kC slots per batch; the first batch is in
-                // flight across the barrier
-                constexpr int kC = G >= 16 ? 1 : 16 / G;
-                float xa[kC][kH], xd[kC][kH];
+                // this thread's columns (acc column gt, exact-row dim gt) of kC slots
+                // per batch; the first batch is in flight across the barrier
+                constexpr int kC = 32 / G;
+                float xa[kC][G], xd[kC][G];
                 auto load_batch = [&](int s0) {
 #pragma unroll
-                    for (int jj = 0; jj < kC; ++jj)
+                    for (int j = 0; j < kC; ++j)
 #pragma unroll
-                        for (int hh = 0; hh < kH; ++hh) {
-                            const int h = sub * kH + hh < G ? sub * kH + hh : 0;
-                            const float* q = Pbase + ((int64_t)h * a.splits_total + s0 + jj) * stride;
-                            const bool in = s0 + jj < nsl && sub * kH + hh < G;
-                            xa[jj][hh] = (in && j < rV) ? __ldcg(q + 2 + j) : 0.f;
-                            xd[jj][hh] = in ? __ldcg(q + 2 + rV + j) : 0.f;
+                        for (int h = 0; h < G; ++h) {
+                            const float* q = Pbase + ((int64_t)h * a.splits_total + s0 + j) * stride;
+                            const bool in = s0 + j < nsl;
+                            xa[j][h] = (in && gt < rV) ? __ldcg(q + 2 + gt) : 0.f;
+                            xd[j][h] = in ? __ldcg(q + 2 + rV + gt) : 0.f;
                         }
                 };
                 load_batch(0);
                 group_sync(grp);
-                float M[kH], L[kH], va[kH], vd[kH];
+                float M[G], L[G], va[G], vd[G];
 #pragma unroll
-                for (int hh = 0; hh < kH; ++hh) {
-                    M[hh] = -INFINITY;
-                    L[hh] = 0.f;
-                    va[hh] = 0.f;
-                    vd[hh] = 0.f;
+                for (int h = 0; h < G; ++h) {
+                    M[h] = -INFINITY;
+                    L[h] = 0.f;
+                    va[h] = 0.f;
+                    vd[h] = 0.f;
                 }
                 for (int sl = 0; sl < nsl; ++sl)
 #pragma unroll
-                    for (int hh = 0; hh < kH; ++hh) {
-                        const int h = sub * kH + hh < G ? sub * kH + hh : 0;
-                        M[hh] = fmaxf(M[hh], sml[sl * G + h]);
-                    }
+                    for (int h = 0; h < G; ++h) M[h] = fmaxf(M[h], sml[sl * G + h]);
                 for (int s0 = 0; s0 < nsl; s0 += kC) {
                     if (s0 > 0) load_batch(s0);
 #pragma unroll
-                    for (int jj = 0; jj < kC; ++jj)
+                    for (int j = 0; j < kC; ++j)
 #pragma unroll
-                        for (int hh = 0; hh < kH; ++hh) {
-                            if (s0 + jj >= nsl) continue;
-                            const int h = sub * kH + hh < G ? sub * kH + hh : 0;
-                            const float m = sml[(s0 + jj) * G + h];
-                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M[hh]);
-                            L[hh] = fmaf(w, sml[nml + (s0 + jj) * G + h], L[hh]);
-                            va[hh] = fmaf(w, xa[jj][hh], va[hh]);
-                            vd[hh] = fmaf(w, xd[jj][hh], vd[hh]);   // exact-row sum, dim j
+                        for (int h = 0; h < G; ++h) {
+                            if (s0 + j >= nsl) continue;
+                            const float m = sml[(s0 + j) * G + h];
+                            const float w = (m == -INFINITY) ? 0.f : __expf(m - M[h]);
+                            L[h] = fmaf(w, sml[nml + (s0 + j) * G + h], L[h]);
+                            va[h] = fmaf(w, xa[j][h], va[h]);
+                            vd[h] = fmaf(w, xd[j][h], vd[h]);   // exact-row sum, dim gt
                         }
                 }
 #pragma unroll
-                for (int hh = 0; hh < kH; ++hh) {
-                    const int h = sub * kH + hh;
-                    if (h < G && j < rV) sacc[h * rV + j] = va[hh];
-                }
+                for (int h = 0; h < G; ++h)
+                    if (gt < rV) sacc[h * rV + gt] = va[h];
                 group_sync(grp);
-                // out[h][i] = (sum_c acc[h][c] B_V[i][c] + accd[h][i]) / L_h, i = j
+                // out[h][i] = (sum_c acc[h][c] B_V[i][c] + accd[h][i]) / L_h, i = gt
 #pragma unroll 4
                 for (int c = 0; c < rV; c += 4) {
                     const float4 b4 = *reinterpret_cast<const float4*>(br + c);
 #pragma unroll
-                    for (int hh = 0; hh < kH; ++hh) {
-                        const int h = sub * kH + hh < G ? sub * kH + hh : 0;
+                    for (int h = 0; h < G; ++h) {
                         const float4 s4 = *reinterpret_cast<const float4*>(sacc + h * rV + c);
-                        vd[hh] = fmaf(s4.x, b4.x, vd[hh]);
-                        vd[hh] = fmaf(s4.y, b4.y, vd[hh]);
-                        vd[hh] = fmaf(s4.z, b4.z, vd[hh]);
-                        vd[hh] = fmaf(s4.w, b4.w, vd[hh]);
+                        vd[h] = fmaf(s4.x, b4.x, vd[h]);
+                        vd[h] = fmaf(s4.y, b4.y, vd[h]);
+                        vd[h] = fmaf(s4.z, b4.z, vd[h]);
+                        vd[h] = fmaf(s4.w, b4.w, vd[h]);
                     }
                 }
 #pragma unroll
-                for (int hh = 0; hh < kH; ++hh) {
-                    const int h = sub * kH + hh;
-                    if (h < G) a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + j] = vd[hh] / L[hh];
-                }
+                for (int h = 0; h < G; ++h)
+                    a.out[((int64_t)bq * a.Hq + (int64_t)kvh * g + h) * d + gt] = vd[h] / L[h];
                 group_sync(grp);                      // P buffer free again
             }
             n0 = s1;
         }
         if (__any_sync(0xffffffffu, range_bad) && lane == 0) atomicOr(a.status, kStatusRange);
-    } else if (warp == 2 || warp == 3) {
-        // ---------------- MMA issuer of group warp - 2 ----------------
+    } else if (warp >= 10) {
+        // ---------------- MMA issuer of group warp - 10 ----------------
         // per tile n of the group: K^ = C_K (B_hi + B_lo)^T (issued as soon as the
         // group's previous score MMA has released the K^ buffer), scores once the
         // epilogue has rotated K^ and written q', values once P is written
-        const int grp = warp - 2;
+        const int grp = warp - 10;
         if (lane == 0) {
             const int MV = rV <= 64 ? 64 : 128;
             const uint32_t idesc_k = idesc_f32acc(1, kTile, d, 0, 0);

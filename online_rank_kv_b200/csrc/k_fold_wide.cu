@@ -53,20 +53,29 @@ __host__ __device__ inline WideGeo wide_geo(int D, int r) {
     return g;
 }
 
-// shared memory (floats): K^T (m x ldn), P (64 x r), then small arrays
 // global scratch floats per factor: [B | X^T] (D x (r+64)), Q (D x 64), B'' (D x r)
 __host__ __device__ inline size_t wide_scratch(int D, int r) {
     const WideGeo g = wide_geo(D, r);
     return (size_t)D * g.nA + (size_t)D * kBlock + (size_t)D * r;
 }
 
-__host__ __device__ inline size_t wide_smem_floats(int D, int r) {
+// shared memory (floats): K^T (m x ldn), the P region, then small arrays
+__host__ __device__ inline size_t wide_kt_floats(int D, int r) {
     const WideGeo g = wide_geo(D, r);
     size_t kt = (size_t)g.m * g.ldn;
     const size_t tile = (size_t)64 * 64 + (size_t)64 * r;   // (a) and new-row tiles alias K^T
     if (kt < tile) kt = tile;
     if (kt < (size_t)r * r) kt = (size_t)r * r;             // Bjorck Gram matrix
-    return kt + (size_t)64 * r + 6 * kMaxCols + 64;
+    return kt;
+}
+// the P region: P (64 x r), later 32-row tiles of [B | Q] (32 x n) and of B''
+__host__ __device__ inline size_t wide_p_floats(int D, int r) {
+    const WideGeo g = wide_geo(D, r);
+    const size_t p = (size_t)64 * r, t = (size_t)32 * g.n;
+    return p > t ? p : t;
+}
+__host__ __device__ inline size_t wide_smem_floats(int D, int r) {
+    return wide_kt_floats(D, r) + wide_p_floats(D, r) + 6 * kMaxCols + 64;
 }
 
 __device__ __forceinline__ float block_sum(float v, float* red) {
@@ -114,8 +123,8 @@ fold_wide_kernel(FactorView f, FoldLaunch fl, int* status) {
 
     extern __shared__ __align__(16) float smem[];
     float* KT = smem;                                  // K^T, column c at KT + c * ldn
-    float* Pm = smem + (wide_smem_floats(D, r) - (size_t)64 * r - 6 * kMaxCols - 64);
-    float* tau = Pm + 64 * r;
+    float* Pm = smem + wide_kt_floats(D, r);
+    float* tau = Pm + wide_p_floats(D, r);
     float* vd = tau + kMaxCols;
     float* al = vd + kMaxCols;
     float* sig2 = al + kMaxCols;
@@ -374,13 +383,24 @@ fold_wide_kernel(FactorView f, FoldLaunch fl, int* status) {
         gW[e] = KT[order[j] * ldn + c];
     }
     if (tid == 0 && seq == 0) f.seg_rows[layer * f.D + slot] = (int)n_c;
-    for (int e = tid; e < D * r; e += kThreads) {
-        const int i = e / r, j = e % r;
-        const float* w = KT + order[j] * ldn;
-        float acc = 0.f;
-        for (int c = 0; c < r; ++c) acc = fmaf(Bold[(size_t)i * r + c], w[c], acc);
-        for (int a = 0; a < k; ++a) acc = fmaf(Y[(size_t)a * D + i], w[r + a], acc);
-        Bn[e] = acc;
+    {
+        // 32-row tiles of [B | Q] through shared memory (the P region, free now)
+        float* At = Pm;              // [32 rows][n]
+        const int jj = tid % r, i_off = tid / r, i_step = kThreads / r;
+        const float* w = KT + order[jj] * ldn;
+        for (int i0 = 0; i0 < D; i0 += 32) {
+            __syncthreads();
+            for (int e = tid; e < 32 * n; e += kThreads) {
+                const int ii = e / n, c = e % n;
+                At[e] = c < r ? Bold[(size_t)(i0 + ii) * r + c] : Y[(size_t)(c - r) * D + i0 + ii];
+            }
+            __syncthreads();
+            for (int ii = i_off; ii < 32; ii += i_step) {
+                float acc = 0.f;
+                for (int c = 0; c < n; ++c) acc = fmaf(At[ii * n + c], w[c], acc);
+                Bn[(size_t)(i0 + ii) * r + jj] = acc;
+            }
+        }
     }
     __syncthreads();
 
@@ -424,11 +444,34 @@ fold_wide_kernel(FactorView f, FoldLaunch fl, int* status) {
 
     // ---- one Bjorck step on B'' and the stores of B' (fp32; bf16 hi/lo per KV head)
     float* Gm = KT;   // r x r
-    for (int e = tid; e < r * r; e += kThreads) {
-        const int a = e / r, b = e % r;
-        float acc = 0.f;
-        for (int i = 0; i < D; ++i) acc = fmaf(Bn[(size_t)i * r + a], Bn[(size_t)i * r + b], acc);
-        Gm[e] = acc;
+    {
+        // Gram matrix over 32-row tiles of B'' in shared memory (the P region)
+        float* Bt = Pm;              // [32 rows][r]
+        float gacc[32];
+        const int ne = (r * r + kThreads - 1) / kThreads;   // entries per thread, <= 32
+#pragma unroll
+        for (int u = 0; u < 32; ++u) gacc[u] = 0.f;
+        for (int i0 = 0; i0 < D; i0 += 32) {
+            __syncthreads();
+            for (int e = tid; e < 32 * r; e += kThreads) Bt[e] = Bn[(size_t)i0 * r + e];
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int e = tid + u * kThreads;
+                if (u >= ne || e >= r * r) break;
+                const int a = e / r, b = e % r;
+                float acc = gacc[u];
+                for (int ii = 0; ii < 32; ++ii) acc = fmaf(Bt[ii * r + a], Bt[ii * r + b], acc);
+                gacc[u] = acc;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const int e = tid + u * kThreads;
+            if (u >= ne || e >= r * r) break;
+            Gm[e] = gacc[u];
+        }
     }
     __syncthreads();
     float* gB = f.basis + fidx * (int64_t)D * r;

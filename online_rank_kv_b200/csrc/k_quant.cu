@@ -78,7 +78,43 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(FactorView f, cons
     quant_rows_block(f, rows + row0 * f.r, f.r, nr, codes + row0 * f.qwords, scales + row0 * 4, sScale);
 }
 
+// The decode workspace of a coded layer: rows [0, rows) of every head as bf16
+// values code * scale, in the 8 x 8 blocked layout the tensor-core decode
+// bulk-copies.  One thread per (head, row, 8 columns): one 16-byte store.
+__global__ void __launch_bounds__(kThreads) expand_codes_kernel(FactorView f, int layer, int64_t rows,
+                                                                 __nv_bfloat16* dst) {
+    const int r = f.r;
+    const int cg = r / 8;
+    const int64_t total = (int64_t)f.BH * rows * cg;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int c0 = (int)(e % cg) * 8;
+        const int64_t row = (e / cg) % rows;
+        const int64_t bh = e / ((int64_t)cg * rows);
+        const int64_t hidx = (int64_t)layer * f.BH + bh;
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat16 lo = __float2bfloat16_rn(quant_value(f, hidx, row, c0 + 2 * u));
+            const __nv_bfloat16 hi = __float2bfloat16_rn(quant_value(f, hidx, row, c0 + 2 * u + 1));
+            w[u] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+        }
+        *reinterpret_cast<uint4*>(dst + bh * f.n_max * r + coef_index(1, r, row, c0)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_expand_codes(const FactorView& f, int layer, int64_t rows, __nv_bfloat16* dst,
+                                cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    const int64_t total = (int64_t)f.BH * rows * (f.r / 8);
+    int64_t blocks = (total + kThreads - 1) / kThreads;
+    if (blocks > 8 * 148) blocks = 8 * 148;
+    expand_codes_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(f, layer, rows, dst);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quant_new_rows(const FactorView& f, const FoldLaunch& fl, cudaStream_t s) {
     if (fl.n_tasks <= 0) return cudaSuccess;

@@ -78,8 +78,13 @@ def _cfg(**kw):
     return c
 
 
-def test_coded_cache_tracks_the_coded_oracle_through_many_rewrites():
+@pytest.mark.parametrize("tensor_cores", ["1", "0"])
+def test_coded_cache_tracks_the_coded_oracle_through_many_rewrites(tensor_cores, monkeypatch):
+    """Decode through the tensor-core kernel (the layer's codes expanded to
+    bf16 tiles per call) and through the CUDA-core kernel (codes read in
+    place)."""
     import online_rank_kv_b200 as ik
+    monkeypatch.setenv("ISKV_TENSOR_CORES", tensor_cores)
     cfg = _cfg()
     cache = ik.Cache(cfg)
     H = cfg.batch * cfg.kv_heads
