@@ -85,9 +85,9 @@ DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of on
 
 # What the path computes in: storage, tensor-core operand and accumulator types.
 PRECISION = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: bf16 MMA rebuilds keys "
-             "(basis as bf16 hi+lo) into fp32, RoPE and scores in fp32 on CUDA cores, p as "
-             "bf16 hi+lo for the value MMA, fp32 softmax and accumulators; rewrite: bf16 MMA "
-             "with an fp32-exact 3-part split of W_top; fold: fp32")
+             "(basis as bf16 hi+lo) into fp32, RoPE in fp32, rotated keys rounded to fp16, "
+             "scores by fp16 MMA with fp16 hi+lo queries, p as bf16 hi+lo, fp32 softmax and "
+             "accumulators; rewrite: bf16 MMA with an fp32-exact 3-part split of W_top; fold: fp32")
 
 
 def _peaks():
@@ -479,7 +479,7 @@ def run_iskv(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "mixed: bf16 MMA inputs, fp32 accumulate and scores" if coef == ik.BF16
+        "dtype": "mixed: bf16/fp16 MMA inputs, fp32 accumulate" if coef == ik.BF16
                  else "fp32 math on bf16 K/V and latent-channel codes" if codes
                  else "fp32 math on bf16 K/V, fp32 coefficients",
         "precision": PRECISION if coef == ik.BF16 else "bf16 K/V in HBM, fp32 coefficients "
