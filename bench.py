@@ -74,14 +74,14 @@ BLOCK = 64
 
 # DRAM bytes (read + write) of one decode-attention launch at the per-layer
 # shape of the 32K-context, batch-8 workloads (8 KV / 32 query heads, r_K 32,
-# r_V 64), taken from an ncu launch list of the one-layer workload (the
+# r_V 64), taken from an ncu capture of the one-layer workload (the
 # 36-layer run issues the same launch once per layer).  Not measured by this
 # run: reported as copied, with its source, and only while the decode kernel
 # is the one that was captured (None otherwise, and for other workloads).
-DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.3e6, "qwen3-1L-b8-32k": 433.3e6}
+DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.4e6, "qwen3-1L-b8-32k": 433.4e6}
 DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode launch "
-                         "at this per-layer shape (one-layer 32K workload, launch list of the "
-                         "timed steps); copied, not measured in this run")
+                         "at this per-layer shape (one-layer 32K workload, full ncu capture of the "
+                         "decode kernel); copied, not measured in this run")
 
 # What the path computes in: storage, tensor-core operand and accumulator types.
 PRECISION = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: bf16 MMA rebuilds keys "
