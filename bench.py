@@ -78,16 +78,43 @@ BLOCK = 64
 # 36-layer run issues the same launch once per layer).  Not measured by this
 # run: reported as copied, with its source, and only while the decode kernel
 # is the one that was captured (None otherwise, and for other workloads).
-DECODE_TRAFFIC = {"qwen3-36L-b8-32k": 433.4e6, "qwen3-1L-b8-32k": 433.4e6}
+DECODE_TRAFFIC = {("qwen3-36L-b8-32k", "decode_tc_kernel"): 433.4e6,
+                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 433.4e6}
 DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode launch "
                          "at this per-layer shape (one-layer 32K workload, full ncu capture of the "
                          "decode kernel); copied, not measured in this run")
 
+
+
+# the library's names of its decode kernels (Cache.decode_kernel) -> kernel symbols
+KERNEL_OF = {"cuda_core": "decode_kernel", "rotate": "decode_tc_kernel", "query_rope": "decode_u_kernel"}
+
+
+KERNEL_TEXT = {
+    "decode_u_kernel": "decode_u_kernel (persistent split-K decode attention, RoPE folded into the "
+                       "queries: U = position table x (query, basis) products on the tensor cores, "
+                       "per-head combine fused), one launch per layer call",
+    "decode_tc_kernel": "decode_tc_kernel (persistent split-K decode attention, keys rebuilt and "
+                        "rotated per tile, per-head combine fused), one launch per layer call",
+    "decode_kernel": "decode_kernel (split-K fp32 CUDA-core decode) + combine_kernel, timed "
+                     "together per layer call",
+}
+
 # What the path computes in: storage, tensor-core operand and accumulator types.
-PRECISION = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: bf16 MMA rebuilds keys "
-             "(basis as bf16 hi+lo) into fp32, RoPE in fp32, rotated keys rounded to fp16, "
-             "scores by fp16 MMA with fp16 hi+lo queries, p as bf16 hi+lo, fp32 softmax and "
-             "accumulators; rewrite: bf16 MMA with an fp32-exact 3-part split of W_top; fold: fp32")
+PRECISION_ROT = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: bf16 MMA rebuilds keys "
+                 "(basis as bf16 hi+lo) into fp32, RoPE in fp32, rotated keys rounded to fp16, "
+                 "scores by fp16 MMA with fp16 hi+lo queries, p as bf16 hi+lo, fp32 softmax and "
+                 "accumulators; rewrite: bf16 MMA with an fp32-exact 3-part split of W_top; "
+                 "fold: fp32")
+PRECISION_U = ("bf16 K/V and coefficients in HBM, fp32 bases; decode: per tile an fp16 MMA of the "
+               "rows' position table (cos, sin rounded to fp16) with the head's query-basis "
+               "products (fp32, rounded to fp16), fp32 accumulate; scores as fp32 FMAs of the bf16 "
+               "coefficients with those products; exact rows rotated and scored in fp32; p as "
+               "bf16 hi+lo for the bf16 value MMA, fp32 softmax and accumulators; rewrite: bf16 MMA "
+               "with an fp32-exact 3-part split of W_top; fold: fp32")
+PRECISION = {"decode_u_kernel": PRECISION_U, "decode_tc_kernel": PRECISION_ROT,
+             "decode_kernel": "stored K/V and coefficients widened to fp32; decode, softmax and "
+                              "accumulators in fp32 on the CUDA cores; fold: fp32"}
 
 
 def _peaks():
@@ -290,6 +317,7 @@ def run_iskv(args, rank, world, local_rank):
                     coef_quant=1 if codes else 0, quant_k=wl.get("quant_k", ()),
                     quant_v=wl.get("quant_v", ()))
     cache = ik.Cache(cfg)
+    dec_kernel = KERNEL_OF[cache.decode_kernel()]
     P = args.protect
     kdt = torch.bfloat16
     nh = L * Bsz * H
@@ -472,20 +500,23 @@ def run_iskv(args, rank, world, local_rank):
     status = cache.status()
     kept_bytes, full_bytes = cache.kv_bytes()
 
-    # per decode step and layer: append (K, V) + decode attention; per period:
-    # fold (K, V) + coefficient rewrite (K, V)
-    launches_per_period = BLOCK * L * 3 + 4
+    # per decode step and layer: append (K, V) + decode attention (one launch on
+    # the tensor-core path; split kernel + combine on the CUDA-core path; coded
+    # caches first expand their K and V codes); per period and layer: fold (K, V)
+    # + coefficient rewrite (K, V), coded caches also code the new rows (K, V)
+    per_step = 2 + (1 if coef == ik.BF16 else 3 if codes else 2)
+    launches_per_period = L * (BLOCK * per_step + (6 if codes else 4))
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "mixed: bf16/fp16 MMA inputs, fp32 accumulate" if coef == ik.BF16
-                 else "fp32 math on bf16 K/V and latent-channel codes" if codes
+        "dtype": "mixed: bf16/fp16 MMA inputs, fp32 accumulate" if coef == ik.BF16 or codes
                  else "fp32 math on bf16 K/V, fp32 coefficients",
-        "precision": PRECISION if coef == ik.BF16 else "bf16 K/V in HBM, fp32 coefficients "
+        "precision": PRECISION[dec_kernel] if coef == ik.BF16 else "bf16 K/V in HBM, fp32 coefficients "
                      "and bases, fp32 CUDA-core math throughout" if not codes else
                      "bf16 K/V in HBM, coefficients as 8/4/2-bit latent-channel codes with fp32 "
-                     "scales per row and group, fp32 CUDA-core decode",
+                     "scales per row and group, expanded per call to bf16 tiles (code x scale in "
+                     "fp32, rounded to bf16) for the tensor-core decode; " + PRECISION[dec_kernel],
         "data": "synthetic",
         "config": {
             "workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H, "q_heads": Hq,
@@ -506,11 +537,13 @@ def run_iskv(args, rank, world, local_rank):
         "decode_attention_us_avg": dec_avg_us,
         "prefill_s": prefill_s,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.workload)
+                     "frac": achieved / peak,
+                     "traffic": DECODE_TRAFFIC.get((args.workload, dec_kernel))
                      if coef == ik.BF16 and P == 0 and not codes else None,
                      "traffic_source": DECODE_TRAFFIC_SOURCE,
-                     "kernel": "decode_tc_kernel (persistent split-K decode attention, "
-                               "per-head combine fused), one launch per layer call",
+                     "kernel": KERNEL_TEXT[dec_kernel]
+                               + ("; the codes are expanded first (expand_codes_kernel, timed "
+                                  "inside the call)" if codes else ""),
                      "algorithmic_bytes_per_launch": bsum / max(1, len(dec_events)),
                      "peak_source": peak_src},
         # bytes kept between decode steps at the end of the run against the
@@ -645,6 +678,7 @@ def run_growth(args, rank, world, local_rank):
                     max_tokens=max_tokens, kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1,
                     rope_theta=1e6, max_deferred=64, ring_extra=512)
     cache = ik.Cache(cfg)
+    dec_kernel = KERNEL_OF[cache.decode_kernel()]
     nh = L * Bsz * H
     seed_k, seed_v, seed_q = replica_seeds(rank)
     ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=seed_k, device=dev, dtype=torch.bfloat16)
@@ -719,7 +753,8 @@ def run_growth(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": BLOCK, "ms_per_step": tot_ms / (args.steps * len(bins)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate", "precision": PRECISION,
+        "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate",
+        "precision": PRECISION[dec_kernel],
         "data": "synthetic",
         "config": {"workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H,
                    "q_heads": Hq, "head_dim": D, "rank_k": rK, "rank_v": rV, "window": W,

@@ -67,11 +67,14 @@ extern "C" {
                                       destroy the cache: its decode bookkeeping
                                       may be left inconsistent)             */
 #define ISKV_ERR_RANGE         -9  /* a score of the tensor-core decode was not
-                                      finite: a rotated key or a query went
-                                      beyond fp16's range (|x| >= 65504), the
-                                      type its score MMA takes, or an input
-                                      was inf or NaN (sticky; that call's
-                                      outputs are not finite)               */
+                                      finite: a value its MMAs take as fp16
+                                      went beyond fp16's range (|x| >=
+                                      65504) -- a rotated key or a query in
+                                      the rotation kernel (r_K g > 128), a
+                                      query-basis product in the query-side
+                                      RoPE kernel -- or an input was inf or
+                                      NaN (sticky; that call's outputs are
+                                      not finite)                           */
 
 /* ---- element types ----------------------------------------------------- */
 #define ISKV_F32   0
@@ -249,6 +252,20 @@ ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
  * or temporary buffers.  Either pointer may be NULL.  Host only, no GPU work.
  * Errors: INVALID_ARG for a NULL cache.                                    */
 ISKV_API int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes);
+
+/* The kernel iskv_decode_attention runs for this cache (fixed at creation
+ * by the configuration and the environment): ISKV_DECODE_CUDA_CORE (split
+ * fp32 CUDA-core kernel plus combine: fp32 coefficients or K/V, or the
+ * tensor-core paths switched off with ISKV_TENSOR_CORES=0),
+ * ISKV_DECODE_ROTATE (tensor cores; folded keys rebuilt, rotated and scored
+ * per tile), ISKV_DECODE_QUERY_ROPE (tensor cores; RoPE folded into the
+ * queries, scores from a position table times per-head query-basis products
+ * -- where r_K * g <= 128; ISKV_DECODE_KERNEL=rot or =u overrides the
+ * default between the two).  Host only.  Errors: INVALID_ARG.             */
+#define ISKV_DECODE_CUDA_CORE  0
+#define ISKV_DECODE_ROTATE     1
+#define ISKV_DECODE_QUERY_ROPE 2
+ISKV_API int iskv_decode_kernel(iskv_t h, int* kernel);
 
 /* Code `n` fp32 rows of `rank` coefficients with the latent-channel format
  * `fmt` (see iskv_quant_format): rows [n][rank] fp32, codes [n][words]

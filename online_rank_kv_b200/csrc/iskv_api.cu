@@ -63,6 +63,9 @@ struct iskv_cache {
     float* partial = nullptr;
     int* done = nullptr;          // per-head arrival counters of the fused decode combine
     float2* rope = nullptr;
+    __half* ptab = nullptr;       // fp16 position table (decode_u): factor rows j at
+                                  // P + j, then the protected positions 0 .. P - 1
+    int64_t ptab_rows = 0;        // rows of the factor-row part
     int* status = nullptr;
     void* stage_in = nullptr;     // host-input staging
     size_t stage_in_bytes = 0;
@@ -70,6 +73,7 @@ struct iskv_cache {
     size_t stage_out_bytes = 0;
     int max_splits = 256;
     bool use_tc = true;           // tensor-core paths for bf16 coefficients
+    bool use_u = true;            // RoPE-in-the-queries decode where it applies
     int sms = 148;
     // clock cycles a tensor-core pipeline wait may take before the call gives
     // up with DEVICE_TIMEOUT; tests shorten it through the environment to make
@@ -97,6 +101,8 @@ struct TraceRange {
 
 constexpr size_t kStageBytes = 16u << 20;
 constexpr bool kDecodeTcDefault = true;
+// query-side RoPE decode by default where it applies (else the rotation kernel)
+constexpr bool kDecodeUDefault = false;
 
 // Fill the code-format fields of a view from `q` for rank r; false if the
 // format is invalid (groups 1..4, channels multiples of 16 summing to r, bits
@@ -243,7 +249,7 @@ void free_all(iskv_cache* h) {
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
                     h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out,
                     h->qcodes_k, h->qcodes_v, h->qscales_k, h->qscales_v, h->newrows_k, h->newrows_v,
-                    h->wide, h->qws_k, h->qws_v};
+                    h->wide, h->qws_k, h->qws_v, h->ptab};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -260,7 +266,21 @@ int dalloc(T** p, size_t bytes) {
     return ISKV_OK;
 }
 
-// Layers named by a call: one, or all of them.
+// The decode kernel of a cache (iskv_decode_kernel): tensor cores for bf16
+// K/V with bf16 (or coded, expanded per call) coefficients and g in {1, 2, 4,
+// 8}; among those the query-side RoPE kernel where r_K g <= 128 and it is
+// selected, else the rotation kernel.
+int decode_path(const iskv_cache* h) {
+    const iskv_config& c = h->cfg;
+    const int g = c.q_heads / c.kv_heads;
+    const bool coded_tc = c.coef_quant && h->qws_k != nullptr;
+    if (!(h->use_tc && (coded_tc || (!c.coef_quant && c.coef_dtype == ISKV_BF16)) &&
+          c.kv_dtype == ISKV_BF16 && decode_tc_supports_group(g)))
+        return ISKV_DECODE_CUDA_CORE;
+    if (h->use_u && h->ptab != nullptr && decode_u_supports(g, c.rank_k)) return ISKV_DECODE_QUERY_ROPE;
+    return ISKV_DECODE_ROTATE;
+}
+
 // A call on stream s that touches the listed layers runs after their last
 // asynchronous update (the swap to the updated factors happens here, at the
 // next call, not at the update's launch).  Callers keep every other call on
@@ -278,6 +298,7 @@ int order_after_update(iskv_cache* h, int layer, cudaStream_t s) {
     return order_after_updates(h, std::vector<int>{layer}, s);
 }
 
+// Layers named by a call: one, or all of them.
 bool layers_of(const iskv_cache* h, int layer, std::vector<int>* out) {
     out->clear();
     if (layer == ISKV_ALL_LAYERS) {
@@ -377,6 +398,12 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         const char* env = std::getenv("ISKV_TENSOR_CORES");
         h->use_tc = kDecodeTcDefault ? !(env && env[0] == '0') : (env && env[0] == '1');
         cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+        // decode kernel for bf16 coefficient tiles: "rot" keeps the kernel that
+        // rebuilds and rotates the keys, otherwise the query-side RoPE kernel
+        // wherever r_K g <= 128
+        const char* dk = std::getenv("ISKV_DECODE_KERNEL");
+        h->use_u = dk && std::strcmp(dk, "u") == 0 ? true
+                 : dk && std::strcmp(dk, "rot") == 0 ? false : kDecodeUDefault;
         const char* w = std::getenv("ISKV_TEST_PIPELINE_WAIT_CYCLES");
         if (w && std::atoll(w) > 0) h->pipe_wait = std::atoll(w);
     }
@@ -467,6 +494,35 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
                     tab[p * (d / 2) + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
                 }
             if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) !=
+                cudaSuccess)
+                rc = ISKV_ERR_CUDA;
+        }
+    }
+    if (rc == ISKV_OK && c.kv_dtype == ISKV_BF16 && (c.coef_quant || c.coef_dtype == ISKV_BF16)) {
+        // the query-side RoPE decode's table: coefficient row j sits at position
+        // P + j; 128 fp16 per row (cos, sin of each frequency, interleaved) in
+        // 8 x 8 blocks, 8-row groups outermost, so a 128-row tile is contiguous
+        // rows: every factor position a folded or window row can take; a second
+        // table holds the protected positions 0 .. P - 1 (rounded up to 64)
+        const int64_t rows = std::max<int64_t>(h->n_max, (c.max_tokens + 63) / 64 * 64 + 128);
+        const int64_t prows = (c.protect + 63) / 64 * 64;
+        h->ptab_rows = rows;
+        rc = dalloc(&h->ptab, (size_t)(rows + prows) * 128 * sizeof(__half));
+        if (rc == ISKV_OK) {
+            std::vector<__half> tab((size_t)(rows + prows) * 128);
+            std::vector<double> inv(d / 2);
+            for (size_t i = 0; i < d / 2; ++i) inv[i] = std::pow(c.rope_theta, -2.0 * (double)i / (double)d);
+            for (int64_t j = 0; j < rows + prows; ++j) {
+                const int64_t pos = j < rows ? c.protect + j : j - rows;
+                for (int i = 0; i < d / 2; ++i) {
+                    const double ang = (double)pos * inv[i];
+                    const float cs = c.use_rope ? (float)std::cos(ang) : 1.f;
+                    const float sn = c.use_rope ? (float)std::sin(ang) : 0.f;
+                    tab[tc::blocked8(j, 2 * i, 128)] = __float2half_rn(cs);
+                    tab[tc::blocked8(j, 2 * i + 1, 128)] = __float2half_rn(sn);
+                }
+            }
+            if (cudaMemcpy(h->ptab, tab.data(), tab.size() * sizeof(__half), cudaMemcpyHostToDevice) !=
                 cudaSuccess)
                 rc = ISKV_ERR_CUDA;
         }
@@ -722,8 +778,8 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
     const int sms = h->sms;
     const bool coded_tc = c.coef_quant && h->qws_k != nullptr;
-    if (h->use_tc && (coded_tc || (!c.coef_quant && c.coef_dtype == ISKV_BF16)) &&
-        c.kv_dtype == ISKV_BF16 && decode_tc_supports_group(a.g)) {
+    const int path = decode_path(h);
+    if (path != ISKV_DECODE_CUDA_CORE) {
         // one persistent tensor-core kernel, one CTA per SM, over the flattened
         // (head, tile) space: 128-token tiles of folded rows, then 64-token
         // tiles of exact rows, all under one online softmax per head
@@ -758,13 +814,25 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.T = a.T;
         t.scale = a.scale;
         t.pipe_wait = h->pipe_wait;
+        t.ptab = h->ptab;
+        t.ptab_rows = h->ptab_rows;
         // exact-row tiles of 64 rows, or of 32 when 64 rows of K and V would make
         // a stage larger than a folded tile's C_K and C_V
         const int64_t coef_tile = (int64_t)128 * (c.rank_k + c.rank_v) * 2;
         t.win_rows = 2 * 64 * kHeadDim * 2 > coef_tile ? 32 : 64;
+        // query-side RoPE kernel where U (r_K g columns) fits one TMEM buffer
+        const bool use_u = path == ISKV_DECODE_QUERY_ROPE;
         // deepest pipeline that fits: stages first, then two basis buffers, then
         // double-buffered q'
         t.stages = 0;
+        if (use_u) {
+            // exact tiles also stage their rows' fp16 RoPE table: 3 x wt rows of 256 bytes
+            t.win_rows = 3 * 64 * kHeadDim * 2 > coef_tile ? 32 : 64;
+            for (int ns = 6; ns >= 2 && t.stages == 0; --ns)
+                if (decode_u_smem_bytes(c.rank_k, c.rank_v, ns, t.win_rows) <= 227 * 1024) t.stages = ns;
+            t.basis_bufs = 1;
+            t.q_bufs = 1;
+        }
         for (int ns = 6; ns >= 2 && t.stages == 0; --ns)
             for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
                 for (int nqb = 2; nqb >= 1; --nqb)
@@ -786,7 +854,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         // partial buffer holds (few heads, long context)
         const int ncta = (int)std::min<int64_t>(std::min(sms, kDecodeMaxCtas), t.total_tiles);
         // partial slots per query head: the buffer's, and the merge scratch's
-        // (slots x g <= 512 per q' buffer of a group)
+        // (slots x g <= 512 per q' buffer of a group; 512 for the query-side kernel)
         const int cap_slots = std::min(h->max_splits, 512 * t.q_bufs / a.g);
         if (!plan_decode_grid(t.total_tiles, t.tiles_per_head, h->BH, ncta, cap_slots, 2, &h->grid_plan))
             return ISKV_ERR_UNSUPPORTED;
@@ -796,7 +864,8 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.slots_c = slots_c;
         t.splits_total = 2 * slots_c;
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
-        CU(launch_decode_tc(t, s));   // merges the partials of each head itself
+        if (use_u) CU(launch_decode_u(t, s));   // both merge the partials of each head
+        else CU(launch_decode_tc(t, s));
         if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
         return ISKV_OK;
     }
@@ -885,6 +954,12 @@ int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
             }
         }
     }
+    return ISKV_OK;
+}
+
+int iskv_decode_kernel(iskv_t h, int* kernel) {
+    if (!h || !kernel) return ISKV_ERR_INVALID_ARG;
+    *kernel = decode_path(h);
     return ISKV_OK;
 }
 

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <vector>
@@ -129,6 +130,32 @@ __device__ __forceinline__ float quant_value(const FactorView& f, int64_t hidx, 
     return (float)code * f.qscales[rbase * 4 + g];
 }
 
+// The stored values of coefficients (row, c0 .. c0 + 7) of one row, given
+// that row's code words and group scales; c0 a multiple of 8.  Channel groups
+// start at multiples of 16, so the 8 channels share one group and their codes
+// are 8 b consecutive bits starting at a multiple of 8 b: two whole words for
+// b = 8, one for b = 4, one half word for b = 2.  Same values as quant_value.
+__device__ __forceinline__ void quant_decode8(const FactorView& f, const uint32_t* row_codes,
+                                              const float* row_scales, int c0, float (&v)[8]) {
+    const int g = quant_group_of(f, c0);
+    const int b = f.qbits[g];
+    if (b == 0) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = 0.f;
+        return;
+    }
+    const int bit0 = (c0 - f.qlo[g]) * b;
+    const uint32_t* wp = row_codes + f.qword0[g] + (bit0 >> 5);
+    uint64_t bits = wp[0];
+    if (b == 8) bits |= (uint64_t)wp[1] << 32;
+    bits >>= (bit0 & 31);
+    const uint32_t mask = (1u << b) - 1u;
+    const int qmax = (1 << (b - 1)) - 1;
+    const float sc = row_scales[g];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = (float)((int)((uint32_t)(bits >> (k * b)) & mask) - qmax) * sc;
+}
+
 // Code rows of r fp32 values: src[row * ld + c] for rows [0, nrows) of a
 // block, written to codes[row * qwords + w] and scales[row * 4 + g]; sScale
 // holds nrows * 4 floats of block scratch.  Called by every thread of the
@@ -233,6 +260,10 @@ struct DecodeTcArgs {
     float scale;
     long long pipe_wait;         // clock cycles a pipeline wait may take before the
                                  // call gives up (drain waits keep their own limit)
+    const void* ptab;            // fp16 [ptab_rows + P rounded to 64][128], 8 x 8 blocked:
+                                 // cos, sin of pos w_i interleaved; row j < ptab_rows is
+                                 // factor row j (pos = P + j), row ptab_rows + p is pos p
+    int64_t ptab_rows;
 };
 
 // ---------------------------------------------------------------------------
@@ -264,6 +295,9 @@ cudaError_t launch_expand_codes(const FactorView& f, int layer, int64_t rows, __
                                 cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeTcArgs& a, cudaStream_t s);
 bool decode_tc_supports_group(int g);
+cudaError_t launch_decode_u(const DecodeTcArgs& a, cudaStream_t s);
+bool decode_u_supports(int g, int rK);
+size_t decode_u_smem_bytes(int rK, int rV, int ns, int wt);
 size_t decode_tc_smem_bytes(int rK, int rV, int ns, int nbk, int nqb, int wt);
 
 size_t fold_smem_bytes(int r);

@@ -20,30 +20,45 @@ namespace iskv {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr int kTile = 64;
 constexpr int kMaxAcc = kMaxGroup * (kHeadDim + kHeadDim) / kThreads;  // 8
 
+// Shared memory (floats).  Row strides are padded by 4 so that 16-byte
+// vector reads stay aligned and the rows a warp touches fall in different banks.
 struct Smem {
-    size_t bk, q, kt, ck, cv, s, misc;
+    int ldc, ldv;                       // row strides of the C_K and C_V / V tiles
+    size_t b, q, c, v, s, misc;
 };
 
 __host__ __device__ inline Smem smem_layout(int rK, int rV, int g) {
     Smem L;
-    L.bk = (size_t)kHeadDim * (rK + 1);
-    L.q = (size_t)g * kHeadDim;
-    L.kt = (size_t)kTile * kHeadDim;
-    L.ck = (size_t)kTile * rK;
-    L.cv = (size_t)kTile * (rV > kHeadDim ? rV : kHeadDim);
-    L.s = (size_t)g * kTile;
+    L.ldc = (rK > kHeadDim ? rK : kHeadDim) + 4;   // C_K tile, or exact K rows (d wide)
+    L.ldv = (rV > kHeadDim ? rV : kHeadDim) + 4;   // C_V tile, or exact V rows
+    L.b = (size_t)rK * kHeadDim;                   // B_K^T: row c = basis column c over the dims
+    L.q = (size_t)kMaxGroup * kHeadDim;
+    L.c = (size_t)kTile * L.ldc;
+    L.v = (size_t)kTile * L.ldv;
+    L.s = (size_t)kMaxGroup * kTile;
     L.misc = 4 * (size_t)kMaxGroup;
     return L;
 }
 
 __host__ __device__ inline size_t smem_floats(const Smem& L) {
-    return L.bk + L.q + L.kt + L.ck + L.cv + L.s + L.misc;
+    return L.b + L.q + L.c + L.v + L.s + L.misc;
 }
 
+__device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+
+// One CTA per (split, KV head, sequence), 64-token tiles.  Per folded tile the
+// key rows are rebuilt on the CUDA cores in fp32, register-tiled: thread
+// (ti, tj) = (tid / 16, tid % 16) owns rows 4 ti .. 4 ti + 3 and dims
+// 4 tj .. 4 tj + 3 with their RoPE partners 64 + 4 tj .. 64 + 4 tj + 3, so the
+// rotation needs no data exchange; each k-step of the rebuild reads one
+// 16-byte C_K word per row and two B words for 32 FMAs.  The 16 threads of a
+// row group (one half-warp) then reduce their partial dot products with the
+// queries by shuffles.
 template <typename KvT, typename CoefT>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(DecodeArgs a) {
@@ -61,21 +76,23 @@ decode_kernel(DecodeArgs a) {
     const int slot = a.split_base + split;
 
     const Smem L = smem_layout(rK, rV, g);
-    extern __shared__ float sm[];
-    float* sBk = sm;
-    float* sQ = sBk + L.bk;
-    float* sK = sQ + L.q;
-    float* sCk = sK + L.kt;
-    float* sCv = sCk + L.ck;
-    float* sS = sCv + L.cv;
+    extern __shared__ __align__(16) float sm[];
+    float* sB = sm;
+    float* sQ = sB + L.b;
+    float* sC = sQ + L.q;
+    float* sV = sC + L.c;
+    float* sS = sV + L.v;
     float* sMax = sS + L.s;
     float* sSum = sMax + kMaxGroup;
     float* sScale = sSum + kMaxGroup;
 
-    const float* Bk = a.K.basis + hidx * d * rK;
-    for (int e = tid; e < d * rK; e += kThreads) sBk[(e / rK) * (rK + 1) + e % rK] = Bk[e];
+    const float* Bk = a.K.basis + hidx * d * rK;   // [d][rK]
+    for (int e = tid; e < d * rK; e += kThreads) {
+        const int i = e / rK, c = e - i * rK;
+        sB[c * d + i] = Bk[e];
+    }
     const KvT* q = reinterpret_cast<const KvT*>(a.q) + ((int64_t)b * a.Hq + (int64_t)kvh * g) * d;
-    for (int e = tid; e < g * d; e += kThreads) sQ[e] = to_f32(q[e]);
+    for (int e = tid; e < kMaxGroup * d; e += kThreads) sQ[e] = e < g * d ? to_f32(q[e]) : 0.f;
     if (tid < kMaxGroup) {
         sMax[tid] = -INFINITY;
         sSum[tid] = 0.f;
@@ -94,6 +111,8 @@ decode_kernel(DecodeArgs a) {
     const KvT* Pk = reinterpret_cast<const KvT*>(a.K.prot) + hidx * a.K.pcap * d;
     const KvT* Pv = reinterpret_cast<const KvT*>(a.V.prot) + hidx * a.V.pcap * d;
     const int64_t P = a.K.P, c_end = P + a.n_c;   // folded positions: [P, P + n_c)
+    const int ti = tid >> 4, tj = tid & 15;
+    const int dlo = 4 * tj;                       // dims dlo..dlo+3 and 64+dlo..64+dlo+3
     __syncthreads();
 
     for (int64_t j = j0; j < j1;) {
@@ -105,28 +124,63 @@ decode_kernel(DecodeArgs a) {
         if (comp && jend > c_end) jend = c_end;
         const int nt = (int)(jend - j);
 
+        // ---- stage the tile: C_K and C_V rows, or exact K and V rows ----
         if (comp) {
             const int64_t jc = j - P;   // coefficient row
             if (a.K.quant) {
-                // latent-channel codes: decoded to fp32 while staged
-                for (int e = tid; e < kTile * rK; e += kThreads)
-                    sCk[e] = (e / rK < nt) ? quant_value(a.K, hidx, jc + e / rK, e % rK) : 0.f;
-                for (int e = tid; e < kTile * rV; e += kThreads)
-                    sCv[e] = (e / rV < nt) ? quant_value(a.V, hidx, jc + e / rV, e % rV) : 0.f;
+                // latent-channel codes, decoded 8 channels at a time
+                for (int e = tid; e < kTile * (rK / 8); e += kThreads) {
+                    const int t = e / (rK / 8), c0 = (e - t * (rK / 8)) * 8;
+                    float v[8];
+                    if (t < nt) {
+                        const int64_t rb = hidx * a.K.n_max + jc + t;
+                        quant_decode8(a.K, a.K.qcodes + rb * a.K.qwords, a.K.qscales + rb * 4, c0, v);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) v[k] = 0.f;
+                    }
+                    store4(sC + t * L.ldc + c0, v[0], v[1], v[2], v[3]);
+                    store4(sC + t * L.ldc + c0 + 4, v[4], v[5], v[6], v[7]);
+                }
+                for (int e = tid; e < kTile * (rV / 8); e += kThreads) {
+                    const int t = e / (rV / 8), c0 = (e - t * (rV / 8)) * 8;
+                    float v[8];
+                    if (t < nt) {
+                        const int64_t rb = hidx * a.V.n_max + jc + t;
+                        quant_decode8(a.V, a.V.qcodes + rb * a.V.qwords, a.V.qscales + rb * 4, c0, v);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) v[k] = 0.f;
+                    }
+                    store4(sV + t * L.ldv + c0, v[0], v[1], v[2], v[3]);
+                    store4(sV + t * L.ldv + c0 + 4, v[4], v[5], v[6], v[7]);
+                }
+            } else if (!a.K.coef_blocked && sizeof(CoefT) == 4 &&
+                       ((reinterpret_cast<uintptr_t>(Ck) | reinterpret_cast<uintptr_t>(Cv)) & 15) == 0) {
+                // fp32 row-major rows: the tile is one contiguous run, read as 16-byte words
+                const float4* gk = reinterpret_cast<const float4*>(Ck + jc * rK);
+                for (int e = tid; e < kTile * rK / 4; e += kThreads) {
+                    const int t = (4 * e) / rK, c = 4 * e - t * rK;
+                    const float4 v = t < nt ? gk[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4*>(sC + t * L.ldc + c) = v;
+                }
+                const float4* gv = reinterpret_cast<const float4*>(Cv + jc * rV);
+                for (int e = tid; e < kTile * rV / 4; e += kThreads) {
+                    const int t = (4 * e) / rV, c = 4 * e - t * rV;
+                    const float4 v = t < nt ? gv[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4*>(sV + t * L.ldv + c) = v;
+                }
             } else {
-                for (int e = tid; e < kTile * rK; e += kThreads)
-                    sCk[e] = (e / rK < nt) ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, jc + e / rK, e % rK)])
-                                           : 0.f;
-                for (int e = tid; e < kTile * rV; e += kThreads)
-                    sCv[e] = (e / rV < nt) ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, jc + e / rV, e % rV)])
-                                           : 0.f;
-            }
-            __syncthreads();
-            for (int e = tid; e < kTile * d; e += kThreads) {
-                const int t = e / d, i = e % d;
-                float s = 0.f;
-                for (int c = 0; c < rK; ++c) s = fmaf(sCk[t * rK + c], sBk[i * (rK + 1) + c], s);
-                sK[e] = s;
+                for (int e = tid; e < kTile * rK; e += kThreads) {
+                    const int t = e / rK, c = e - t * rK;
+                    sC[t * L.ldc + c] =
+                        t < nt ? to_f32(Ck[coef_index(a.K.coef_blocked, rK, jc + t, c)]) : 0.f;
+                }
+                for (int e = tid; e < kTile * rV; e += kThreads) {
+                    const int t = e / rV, c = e - t * rV;
+                    sV[t * L.ldv + c] =
+                        t < nt ? to_f32(Cv[coef_index(a.V.coef_blocked, rV, jc + t, c)]) : 0.f;
+                }
             }
         } else {
             for (int e = tid; e < kTile * d; e += kThreads) {
@@ -140,32 +194,104 @@ decode_kernel(DecodeArgs a) {
                     kv = to_f32(Rk[coef_index(a.K.ring_blocked, d, slot, i)]);
                     vv = to_f32(Rv[coef_index(a.V.ring_blocked, d, slot, i)]);
                 }
-                sK[e] = kv;
-                sCv[e] = vv;
+                sC[t * L.ldc + i] = kv;
+                sV[t * L.ldv + i] = vv;
             }
         }
         __syncthreads();
 
-        if (a.rope) {
-            for (int e = tid; e < kTile * (d / 2); e += kThreads) {
-                const int t = e / (d / 2), i = e % (d / 2);
-                if (t < nt) {
-                    const float2 cs = a.rope[(j + t) * (d / 2) + i];
-                    const float x1 = sK[t * d + i], x2 = sK[t * d + i + d / 2];
-                    sK[t * d + i] = x1 * cs.x - x2 * cs.y;
-                    sK[t * d + i + d / 2] = x1 * cs.y + x2 * cs.x;
+        // ---- this thread's 4 rows x 8 dims of the key tile ----
+        float k[4][8];
+        if (comp) {
+            // packed fp32 FMAs: dims (2e, 2e + 1) of the thread's 8 per instruction
+            float2 k2[4][4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) k2[u][e] = make_float2(0.f, 0.f);
+            const float* crow = sC + (4 * ti) * L.ldc;
+            for (int c0 = 0; c0 < rK; c0 += 4) {
+                float4 cv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) cv[u] = *reinterpret_cast<const float4*>(crow + u * L.ldc + c0);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const float4 b0 = *reinterpret_cast<const float4*>(sB + (c0 + cc) * d + dlo);
+                    const float4 b1 = *reinterpret_cast<const float4*>(sB + (c0 + cc) * d + 64 + dlo);
+                    const float2 bp[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w),
+                                          make_float2(b1.x, b1.y), make_float2(b1.z, b1.w)};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float cu = cc == 0 ? cv[u].x : cc == 1 ? cv[u].y : cc == 2 ? cv[u].z : cv[u].w;
+                        const float2 c2 = make_float2(cu, cu);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) k2[u][e] = __ffma2_rn(c2, bp[e], k2[u][e]);
+                    }
                 }
             }
-            __syncthreads();
-        }
-
-        for (int pidx = warp; pidx < g * kTile; pidx += kWarps) {
-            const int h = pidx / kTile, t = pidx % kTile;
-            float s = 0.f;
 #pragma unroll
-            for (int u = 0; u < d / 32; ++u) s = fmaf(sQ[h * d + lane + 32 * u], sK[t * d + lane + 32 * u], s);
-            s = warp_sum(s);
-            if (lane == 0) sS[h * kTile + t] = (t < nt) ? s * a.scale : -INFINITY;
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    k[u][2 * e] = k2[u][e].x;
+                    k[u][2 * e + 1] = k2[u][e].y;
+                }
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 x0 = *reinterpret_cast<const float4*>(sC + (4 * ti + u) * L.ldc + dlo);
+                const float4 x1 = *reinterpret_cast<const float4*>(sC + (4 * ti + u) * L.ldc + 64 + dlo);
+                k[u][0] = x0.x; k[u][1] = x0.y; k[u][2] = x0.z; k[u][3] = x0.w;
+                k[u][4] = x1.x; k[u][5] = x1.y; k[u][6] = x1.z; k[u][7] = x1.w;
+            }
+        }
+        // ---- RoPE at the row's position: (k_i, k_{i+64}) by angle pos * w_i ----
+        if (a.rope) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = 4 * ti + u;
+                if (t < nt) {
+                    const float2* cs = a.rope + (j + t) * (d / 2) + dlo;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 r = cs[m];
+                        const float x1 = k[u][m], x2 = k[u][m + 4];
+                        k[u][m] = x1 * r.x - x2 * r.y;
+                        k[u][m + 4] = x1 * r.y + x2 * r.x;
+                    }
+                }
+            }
+        }
+        // ---- scores: partial dot products over this thread's 8 dims, then
+        // a butterfly over the 16 threads of the row group ----
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            if (h < g) {
+                const float4 q0 = *reinterpret_cast<const float4*>(sQ + h * d + dlo);
+                const float4 q1 = *reinterpret_cast<const float4*>(sQ + h * d + 64 + dlo);
+                float s4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float s = k[u][0] * q0.x;
+                    s = fmaf(k[u][1], q0.y, s);
+                    s = fmaf(k[u][2], q0.z, s);
+                    s = fmaf(k[u][3], q0.w, s);
+                    s = fmaf(k[u][4], q1.x, s);
+                    s = fmaf(k[u][5], q1.y, s);
+                    s = fmaf(k[u][6], q1.z, s);
+                    s = fmaf(k[u][7], q1.w, s);
+                    s4[u] = s;
+                }
+#pragma unroll
+                for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) s4[u] += __shfl_xor_sync(0xffffffffu, s4[u], off);
+                if (tj < 4) {
+                    const int t = 4 * ti + tj;
+                    const float sv = tj == 0 ? s4[0] : tj == 1 ? s4[1] : tj == 2 ? s4[2] : s4[3];
+                    sS[h * kTile + t] = (t < nt) ? sv * a.scale : -INFINITY;
+                }
+            }
         }
         __syncthreads();
 
@@ -195,11 +321,12 @@ decode_kernel(DecodeArgs a) {
             if (e < n_acc) {
                 const int h = e / width, col = e % width;
                 float v = acc[u] * sScale[h];
+                const float* ph = sS + h * kTile;
                 if (comp && col < rV) {
-                    for (int t = 0; t < nt; ++t) v = fmaf(sS[h * kTile + t], sCv[t * rV + col], v);
+                    for (int t = 0; t < nt; ++t) v = fmaf(ph[t], sV[t * L.ldv + col], v);
                 } else if (!comp && col >= rV) {
                     const int i = col - rV;
-                    for (int t = 0; t < nt; ++t) v = fmaf(sS[h * kTile + t], sCv[t * d + i], v);
+                    for (int t = 0; t < nt; ++t) v = fmaf(ph[t], sV[t * L.ldv + i], v);
                 }
                 acc[u] = v;
             }
@@ -213,63 +340,79 @@ decode_kernel(DecodeArgs a) {
         const int e = tid + u * kThreads;
         if (e < n_acc) {
             const int h = e / width, col = e % width;
-            float* P = a.partial + (((int64_t)b * a.Hq + kvh * g + h) * slots + slot) * stride;
-            P[2 + col] = acc[u];
+            float* Pp = a.partial + (((int64_t)b * a.Hq + kvh * g + h) * slots + slot) * stride;
+            Pp[2 + col] = acc[u];
         }
     }
     if (tid < g) {
-        float* P = a.partial + (((int64_t)b * a.Hq + kvh * g + tid) * slots + slot) * stride;
-        P[0] = sMax[tid];
-        P[1] = sSum[tid];
+        float* Pp = a.partial + (((int64_t)b * a.Hq + kvh * g + tid) * slots + slot) * stride;
+        Pp[0] = sMax[tid];
+        Pp[1] = sSum[tid];
     }
 }
 
-// One CTA per (sequence, KV head): B_V is staged once (coalesced) for the
-// query group; thread i owns output dim i.
+// One CTA per (query head, sequence), thread i owns output dim i: the split
+// maxima and sums are reduced by the whole block, the weighted sums of the
+// partials read with independent (unrolled, predicated) loads, then B_V^T.
 __global__ void __launch_bounds__(kHeadDim)
 combine_kernel(DecodeArgs a, float* out) {
-    const int kvh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int qh = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
     const int rV = a.V.r, d = kHeadDim, g = a.g;
+    const int kvh = qh / g;
     const int64_t hidx = (int64_t)a.layer * a.V.BH + b * a.Hkv + kvh;
     const int stride = 2 + rV + d;
     const int slots = a.splits_total > 0 ? a.splits_total : a.splits;
     extern __shared__ float cs[];
-    float* sBv = cs;                               // d x (rV + 1)
-    float* sAcc = sBv + d * (rV + 1);              // rV
+    float* sAcc = cs;                              // rV
     float* sW = sAcc + kHeadDim;                   // slots (<= 256)
-    const float* Bv = a.V.basis + hidx * d * rV;
-    for (int e = tid; e < d * rV; e += blockDim.x) sBv[(e / rV) * (rV + 1) + e % rV] = Bv[e];
-    for (int hq = 0; hq < g; ++hq) {
-        const int qh = kvh * g + hq;
-        const float* P = a.partial + ((int64_t)b * a.Hq + qh) * slots * stride;
-        float M = -INFINITY;
-        for (int s = 0; s < slots; ++s) M = fmaxf(M, P[s * stride]);
-        __syncthreads();                           // sW / sAcc of the previous head consumed
-        for (int s = tid; s < slots; s += blockDim.x) {
-            const float ms = P[s * stride];
-            sW[s] = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-        }
-        __syncthreads();
+    float* sRed = sW + 256;                        // 4 warps
+    const float* P = a.partial + ((int64_t)b * a.Hq + qh) * slots * stride;
+    float m = -INFINITY;
+    for (int s = tid; s < slots; s += kHeadDim) m = fmaxf(m, P[s * stride]);
+    m = warp_max(m);
+    if (lane == 0) sRed[warp] = m;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(sRed[0], sRed[1]), fmaxf(sRed[2], sRed[3]));
+    float ls = 0.f;
+    for (int s = tid; s < slots; s += kHeadDim) {
+        const float ms = P[s * stride];
+        const float w = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+        sW[s] = w;
         // empty slots (weight 0) are skipped: their other entries are not written
-        float Ls = 0.f, vd = 0.f;
-        for (int s = 0; s < slots; ++s) {
-            const float w = sW[s];
-            if (w != 0.f) {
-                Ls = fmaf(w, P[s * stride + 1], Ls);
-                vd = fmaf(w, P[s * stride + 2 + rV + tid], vd);
-            }
-        }
-        if (tid < rV) {
-            float v = 0.f;
-            for (int s = 0; s < slots; ++s)
-                if (sW[s] != 0.f) v = fmaf(sW[s], P[s * stride + 2 + tid], v);
-            sAcc[tid] = v;
-        }
-        __syncthreads();
-        float o = vd;
-        for (int c = 0; c < rV; ++c) o = fmaf(sAcc[c], sBv[tid * (rV + 1) + c], o);
-        out[((int64_t)b * a.Hq + qh) * d + tid] = o / Ls;
+        if (w != 0.f) ls = fmaf(w, P[s * stride + 1], ls);
     }
+    ls = warp_sum(ls);
+    __syncthreads();                               // sRed (maxima) read by every thread
+    if (lane == 0) sRed[warp] = ls;
+    __syncthreads();
+    const float Ls = sRed[0] + sRed[1] + sRed[2] + sRed[3];
+    float vd = 0.f, va = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < slots; ++s) {
+        const float w = sW[s];
+        const float* ps = P + s * stride;
+        const float xd = w != 0.f ? ps[2 + rV + tid] : 0.f;
+        const float xa = (w != 0.f && tid < rV) ? ps[2 + tid] : 0.f;
+        vd = fmaf(w, xd, vd);
+        va = fmaf(w, xa, va);
+    }
+    if (tid < rV) sAcc[tid] = va;
+    __syncthreads();
+    const float* bv = a.V.basis + (hidx * d + tid) * rV;
+    float o = vd;
+    if ((reinterpret_cast<uintptr_t>(a.V.basis) & 15) == 0) {
+        for (int c = 0; c < rV; c += 4) {
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(bv + c));
+            o = fmaf(sAcc[c], b4.x, o);
+            o = fmaf(sAcc[c + 1], b4.y, o);
+            o = fmaf(sAcc[c + 2], b4.z, o);
+            o = fmaf(sAcc[c + 3], b4.w, o);
+        }
+    } else {
+        for (int c = 0; c < rV; ++c) o = fmaf(sAcc[c], __ldg(bv + c), o);
+    }
+    out[((int64_t)b * a.Hq + qh) * d + tid] = o / Ls;
 }
 
 }  // namespace
@@ -307,11 +450,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, float* out, cudaStream_t s) {
-    const size_t bytes = ((size_t)kHeadDim * (a.V.r + 1) + kHeadDim + 256) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)bytes);
-    if (e != cudaSuccess) return e;
-    combine_kernel<<<dim3(a.Hkv, a.B), kHeadDim, bytes, s>>>(a, out);
+    const size_t bytes = ((size_t)kHeadDim + 256 + 4) * sizeof(float);
+    combine_kernel<<<dim3(a.Hq, a.B), kHeadDim, bytes, s>>>(a, out);
     return cudaGetLastError();
 }
 

@@ -35,7 +35,11 @@ __global__ void __launch_bounds__(kThreads) quant_new_rows_kernel(FactorView f, 
 
 // The rewrite of coded rows, one block of 64 rows per CTA: decode, multiply by
 // the block's segment matrix (W_top of one fold, or the product of the
-// postponed ones from compose_kernel), code again in place.
+// postponed ones from compose_kernel), code again in place.  The product is
+// register-tiled: each thread owns 4 rows x r/16 columns (columns tx, tx + 16,
+// ...), so a k-step reads 4 + r/16 shared values for 4 r/16 FMAs; rows are
+// padded to r + 1 floats so the 4-row reads of a warp's two row groups fall in
+// different banks.
 __global__ void __launch_bounds__(kThreads) resync_quant_kernel(FactorView f, ResyncLaunch rl) {
     const int task = blockIdx.z, bh = blockIdx.y;
     const int layer = rl.layer[task];
@@ -46,26 +50,54 @@ __global__ void __launch_bounds__(kThreads) resync_quant_kernel(FactorView f, Re
     int seg = 0;
     while (seg < nseg && row0 >= bounds[seg]) ++seg;
     if (seg >= nseg) return;
-    const int r = f.r;
+    const int r = f.r, ld = r + 1, cg = r >> 3;
     extern __shared__ float sm[];
     float* sW = sm;                    // r x r
-    float* sC = sW + r * r;            // kRows x r, decoded rows
-    float* sO = sC + kRows * r;        // kRows x r, rewritten rows
-    float* sScale = sO + kRows * r;    // kRows x 4
+    float* sC = sW + r * r;            // kRows x ld, decoded rows
+    float* sO = sC + kRows * ld;       // kRows x ld, rewritten rows
+    float* sScale = sO + kRows * ld;   // kRows x 4
     const int64_t hidx = (int64_t)layer * f.BH + bh;
     const float* W = f.pend + (hidx * f.D + seg) * (int64_t)r * r;
     for (int e = threadIdx.x; e < r * r; e += kThreads) sW[e] = W[e];
-    for (int e = threadIdx.x; e < kRows * r; e += kThreads)
-        sC[e] = quant_value(f, hidx, row0 + e / r, e % r);
-    __syncthreads();
-    for (int e = threadIdx.x; e < kRows * r; e += kThreads) {
-        const int t = e / r, cc = e % r;
-        float acc = 0.f;
-        for (int j = 0; j < r; ++j) acc = fmaf(sC[t * r + j], sW[j * r + cc], acc);
-        sO[e] = acc;
+    const uint32_t* codes = f.qcodes + (hidx * f.n_max + row0) * f.qwords;
+    const float* scales = f.qscales + (hidx * f.n_max + row0) * 4;
+    for (int e = threadIdx.x; e < kRows * cg; e += kThreads) {
+        const int t = e / cg, c0 = (e - t * cg) * 8;
+        float v[8];
+        quant_decode8(f, codes + (int64_t)t * f.qwords, scales + t * 4, c0, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sC[t * ld + c0 + k] = v[k];
     }
     __syncthreads();
-    quant_rows_block(f, sO, r, kRows, f.qcodes + (hidx * f.n_max + row0) * f.qwords,
+    {
+        const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;   // rows 4 ty.., columns tx + 16 k
+        const int nk = r >> 4;                                    // 1..8
+        float acc[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+        const float* cr = sC + (4 * ty) * ld;
+        for (int j = 0; j < r; ++j) {
+            float a[4], w[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = cr[i * ld + j];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[k] = k < nk ? sW[j * r + tx + 16 * k] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < nk) acc[i][k] = fmaf(a[i], w[k], acc[i][k]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < nk) sO[(4 * ty + i) * ld + tx + 16 * k] = acc[i][k];
+    }
+    __syncthreads();
+    quant_rows_block(f, sO, ld, kRows, f.qcodes + (hidx * f.n_max + row0) * f.qwords,
                      f.qscales + (hidx * f.n_max + row0) * 4, sScale);
 }
 
@@ -80,27 +112,35 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(FactorView f, cons
 
 // The decode workspace of a coded layer: rows [0, rows) of every head as bf16
 // values code * scale, in the 8 x 8 blocked layout the tensor-core decode
-// bulk-copies.  One thread per (head, row, 8 columns): one 16-byte store.
-__global__ void __launch_bounds__(kThreads) expand_codes_kernel(FactorView f, int layer, int64_t rows,
+// bulk-copies.  Thread e of a head writes the 16 bytes at element 8 e of the
+// head's blocked rows: row (e >> 3) / cg * 8 + (e & 7), columns 8 ((e >> 3) %
+// cg) .. + 7, so a warp's stores are one contiguous 512-byte run.  Rows of the
+// last 8-row group past `rows` are written as zeros.
+__global__ void __launch_bounds__(kThreads) expand_codes_kernel(FactorView f, int layer, int rows,
                                                                  __nv_bfloat16* dst) {
-    const int r = f.r;
-    const int cg = r / 8;
-    const int64_t total = (int64_t)f.BH * rows * cg;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int c0 = (int)(e % cg) * 8;
-        const int64_t row = (e / cg) % rows;
-        const int64_t bh = e / ((int64_t)cg * rows);
-        const int64_t hidx = (int64_t)layer * f.BH + bh;
-        uint32_t w[4];
+    const int r = f.r, cg = r >> 3;
+    const int bh = blockIdx.y;
+    const int64_t hidx = (int64_t)layer * f.BH + bh;
+    const uint32_t* codes = f.qcodes + hidx * f.n_max * f.qwords;
+    const float* scales = f.qscales + hidx * f.n_max * 4;
+    uint4* out = reinterpret_cast<uint4*>(dst + (int64_t)bh * f.n_max * r);
+    const int total = ((rows + 7) >> 3) * cg * 8;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+        const int q = e >> 3;
+        const int rb = q / cg;
+        const int row = rb * 8 + (e & 7), c0 = (q - rb * cg) * 8;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (row < rows) {
+            float v[8];
+            quant_decode8(f, codes + (int64_t)row * f.qwords, scales + (int64_t)row * 4, c0, v);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const __nv_bfloat16 lo = __float2bfloat16_rn(quant_value(f, hidx, row, c0 + 2 * u));
-            const __nv_bfloat16 hi = __float2bfloat16_rn(quant_value(f, hidx, row, c0 + 2 * u + 1));
-            w[u] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            for (int u = 0; u < 4; ++u) {
+                const __nv_bfloat16 lo = __float2bfloat16_rn(v[2 * u]);
+                const __nv_bfloat16 hi = __float2bfloat16_rn(v[2 * u + 1]);
+                w[u] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            }
         }
-        *reinterpret_cast<uint4*>(dst + bh * f.n_max * r + coef_index(1, r, row, c0)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        out[e] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -109,10 +149,13 @@ __global__ void __launch_bounds__(kThreads) expand_codes_kernel(FactorView f, in
 cudaError_t launch_expand_codes(const FactorView& f, int layer, int64_t rows, __nv_bfloat16* dst,
                                 cudaStream_t s) {
     if (rows <= 0) return cudaSuccess;
-    const int64_t total = (int64_t)f.BH * rows * (f.r / 8);
-    int64_t blocks = (total + kThreads - 1) / kThreads;
-    if (blocks > 8 * 148) blocks = 8 * 148;
-    expand_codes_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(f, layer, rows, dst);
+    if (rows > f.n_max || f.BH > 65535) return cudaErrorInvalidValue;
+    const int64_t per_head = ((rows + 7) / 8) * (f.r / 8) * 8;
+    int64_t bx = (per_head + kThreads - 1) / kThreads;
+    // about 8 resident CTAs per SM over all heads; each thread loops over the rest
+    const int64_t want = (8 * 148 + f.BH - 1) / f.BH;
+    if (bx > want) bx = want;
+    expand_codes_kernel<<<dim3((unsigned)bx, (unsigned)f.BH), kThreads, 0, s>>>(f, layer, (int)rows, dst);
     return cudaGetLastError();
 }
 
@@ -127,7 +170,7 @@ cudaError_t launch_resync_quant(const FactorView& f, const ResyncLaunch& rl, cud
     int max_rows = 0;
     for (int i = 0; i < rl.n_tasks; ++i) max_rows = rl.n_rows[i] > max_rows ? rl.n_rows[i] : max_rows;
     if (max_rows <= 0) return cudaSuccess;
-    const size_t bytes = ((size_t)f.r * f.r + 2 * (size_t)kRows * f.r + kRows * 4) * sizeof(float);
+    const size_t bytes = ((size_t)f.r * f.r + 2 * (size_t)kRows * (f.r + 1) + kRows * 4) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(resync_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;

