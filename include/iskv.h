@@ -166,15 +166,18 @@ typedef struct {
 ISKV_API int iskv_config_default(iskv_config* cfg);
 
 /* Create a cache: validates `cfg`, allocates every device buffer for
- * max_tokens on `stream`, sets B = I_d[:, :r], S = 0, T = n_c = 0.  On
- * success *out owns the cache; on failure *out is NULL and nothing leaks.   */
+ * max_tokens on `stream`, sets B = I_d[:, :r], S = 0, T = n_c = 0 (the
+ * explainer's empty factorization before the first block, Jargon:
+ * Block-incremental SVD).  On success *out owns the cache; on failure *out
+ * is NULL and nothing leaks.                                               */
 ISKV_API int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out);
 
 /* Synchronize the cache's streams, free everything.  NULL is a no-op.      */
 ISKV_API int iskv_destroy(iskv_t h);
 
 /* Append t tokens to every sequence of `layer`: k, v are
- * [batch, kv_heads, t, head_dim] in kv_dtype, PRE-RoPE.  T += t.  Never folds.
+ * [batch, kv_heads, t, head_dim] in kv_dtype, PRE-RoPE (explainer, Jargon:
+ * Pre-RoPE keys; the newest W tokens stay exact).  T += t.  Never folds.
  * *ready_blocks (may be NULL) receives floor((T - P - n_c - W) / 64), at
  * least 0 (P = protected positions): the whole blocks that have left the
  * exact window and may be folded.  Positions below P go to the protected
@@ -184,8 +187,9 @@ ISKV_API int iskv_append(iskv_t h, int layer, const void* k, const void* v, int 
                 void* stream, int* ready_blocks);
 
 /* Fold the oldest ready block of `layer` (or of every layer that has one,
- * for ISKV_ALL_LAYERS), K and V factors of every (sequence, KV head), in one
- * launch: (a) P = X B; (b) residual and Householder QR of the complement;
+ * for ISKV_ALL_LAYERS), K and V factors of every (sequence, KV head) -- the
+ * explainer's block update (Jargon: Block-incremental SVD; steps as in
+ * Brand's update): (a) P = X B; (b) residual and Householder QR of the complement;
  * (c) one-sided Jacobi SVD of the (r+64) x (r+k) core, truncated to r;
  * (d) B' = [B, Q] W_r, S' and the block's coefficient rows; (e) unless
  * ISKV_FOLD_DEFER_SYNC is set, every old row is rewritten, C <- C W_r[0:r,:].
@@ -212,13 +216,17 @@ ISKV_API int iskv_compress_block_async(iskv_t h, int layer, int flags, void* str
 
 /* Apply the postponed rewrites of `layer` (or ISKV_ALL_LAYERS) in fold order:
  * one pass over the stored rows, each row multiplied by the product of the
- * W_r[0:r,:] of the folds that came after it was written.  No-op if nothing
- * is pending.                                                              */
+ * W_r[0:r,:] of the folds that came after it was written -- the explainer's
+ * basis synchronization (body paragraph on drift: old coefficients follow
+ * every basis update), applied late but in the same order.  No-op if
+ * nothing is pending.                                                      */
 ISKV_API int iskv_sync(iskv_t h, int layer, void* stream);
 
-/* Decode attention of `layer`: q is [batch, q_heads, head_dim] in kv_dtype,
- * already rotated for position T - 1; out is [batch, q_heads, head_dim]
- * fp32.  Query head j reads KV head j / (q_heads / kv_heads).  Scores over
+/* Decode attention of `layer` over the mixed cache (explainer, Jargon:
+ * Pre-RoPE keys -- folded keys rotated at their positions when read; ASKV
+ * design report, Design requirements -- values never rebuilt): q is
+ * [batch, q_heads, head_dim] in kv_dtype, already rotated for position T - 1;
+ * out is [batch, q_heads, head_dim] fp32.  Query head j reads KV head j / (q_heads / kv_heads).  Scores over
  * all T tokens (folded rows rebuilt as C_K B_K^T and rotated at their absolute
  * positions, exact rows rotated likewise), scale 1/sqrt(d), one softmax; the
  * value side is (p^T C_V) B_V^T + p_win^T V_win.  Errors: STATE if T = 0 or
@@ -226,7 +234,8 @@ ISKV_API int iskv_sync(iskv_t h, int layer, void* stream);
 ISKV_API int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out,
                           void* stream);
 
-/* Rebuild the folded rows of one factor before RoPE: out is
+/* Rebuild the folded rows of one factor before RoPE (explainer, Jargon:
+ * Block-incremental SVD: the stored form is C B^T): out is
  * [batch, kv_heads, n_c, head_dim] fp32 = C B^T.  `which` is ISKV_WHICH_K or
  * ISKV_WHICH_V.  With n_c = 0 nothing is written and `out` may be NULL.
  * Errors: STATE if rewrites are pending.                                   */

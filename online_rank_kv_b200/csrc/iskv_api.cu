@@ -57,7 +57,8 @@ struct iskv_cache {
     float* qscales_v = nullptr;
     float* newrows_k = nullptr;
     float* newrows_v = nullptr;
-    float* wide = nullptr;        // joint-head fold scratch
+    float* wide = nullptr;        // joint-head fold scratch: K's, then V's
+    size_t wide_floats = 0;       // floats of one of the two
     __nv_bfloat16* qws_k = nullptr;   // coded caches: one layer's coefficients as bf16
     __nv_bfloat16* qws_v = nullptr;   // (the tensor-core decode's workspace)
     float* partial = nullptr;
@@ -88,6 +89,9 @@ struct iskv_cache {
     std::vector<cudaEvent_t> upd_evt;
     std::vector<char> upd_wait;
     cudaEvent_t enq_evt = nullptr;   // orders an update's stream after the caller's
+    // the V fold of a compress call runs on this stream beside the K fold
+    cudaStream_t fold_side = nullptr;
+    cudaEvent_t fork_evt = nullptr, join_evt = nullptr;
     DecodeGridPlan grid_plan;        // the last decode grid, reused while its shape holds
 };
 
@@ -195,7 +199,7 @@ FactorView view(const iskv_cache* h, int which) {
     f.D = h->D;
     f.BH = h->BH;
     f.coef_div = h->cfg.joint ? h->cfg.kv_heads : 1;
-    f.wide = h->wide;
+    f.wide = h->wide ? h->wide + (which == ISKV_WHICH_V ? h->wide_floats : 0) : nullptr;
     if (h->cfg.coef_quant) {
         f.quant = 1;
         f.coef_bf16 = 0;
@@ -241,6 +245,11 @@ void free_events(iskv_cache* h) {
     h->upd_evt.clear();
     if (h->enq_evt) cudaEventDestroy(h->enq_evt);
     h->enq_evt = nullptr;
+    if (h->fork_evt) cudaEventDestroy(h->fork_evt);
+    if (h->join_evt) cudaEventDestroy(h->join_evt);
+    if (h->fold_side) cudaStreamDestroy(h->fold_side);
+    h->fork_evt = h->join_evt = nullptr;
+    h->fold_side = nullptr;
 }
 
 void free_all(iskv_cache* h) {
@@ -423,6 +432,10 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
             rc = ISKV_ERR_CUDA;
     if (rc == ISKV_OK && cudaEventCreateWithFlags(&h->enq_evt, cudaEventDisableTiming) != cudaSuccess)
         rc = ISKV_ERR_CUDA;
+    if (rc == ISKV_OK && (cudaEventCreateWithFlags(&h->fork_evt, cudaEventDisableTiming) != cudaSuccess ||
+                          cudaEventCreateWithFlags(&h->join_evt, cudaEventDisableTiming) != cudaSuccess ||
+                          cudaStreamCreateWithFlags(&h->fold_side, cudaStreamNonBlocking) != cudaSuccess))
+        rc = ISKV_ERR_CUDA;
     rc = rc ? rc : dalloc(&h->ring_k, ring_bytes);
     rc = rc ? rc : dalloc(&h->ring_v, ring_bytes);
     const size_t prot_bytes = heads * h->pcap * d * h->kv_bytes;
@@ -467,9 +480,10 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
     rc = rc ? rc : dalloc(&h->pend_v, facs * h->D * (size_t)c.rank_v * c.rank_v * 4);
     rc = rc ? rc : dalloc(&h->qscr_k, c.joint ? 0 : heads * d * fold_q_cols(c.rank_k) * 4);
     rc = rc ? rc : dalloc(&h->qscr_v, c.joint ? 0 : heads * d * fold_q_cols(c.rank_v) * 4);
-    if (c.joint)   // one scratch for K and V: their folds run one after the other
-        rc = rc ? rc : dalloc(&h->wide, facs * fold_wide_scratch_floats(c.kv_heads * kHeadDim,
-                                                                        std::max(c.rank_k, c.rank_v)) * 4);
+    if (c.joint) {   // K's and V's scratch: their folds run side by side
+        h->wide_floats = facs * fold_wide_scratch_floats(c.kv_heads * kHeadDim, std::max(c.rank_k, c.rank_v));
+        rc = rc ? rc : dalloc(&h->wide, 2 * h->wide_floats * 4);
+    }
     rc = rc ? rc : dalloc(&h->seg_rows, (size_t)c.layers * h->D * 4);
     rc = rc ? rc : dalloc(&h->partial, (size_t)c.batch * c.q_heads * h->max_splits *
                                            (2 + c.rank_v + d) * 4);
@@ -653,15 +667,22 @@ int compress_on(iskv_cache* h, const std::vector<int>& ls, int flags, cudaStream
         fl.slot[fl.n_tasks] = defer ? h->n_pend[l] : 0;
         ++fl.n_tasks;
     }
+    // the K and V folds share nothing: V's runs on the side stream, forked from
+    // and joined back into s, so small launches (few heads) fill the GPU together
+    CU(cudaEventRecord(h->fork_evt, s));
+    CU(cudaStreamWaitEvent(h->fold_side, h->fork_evt, 0));
     for (int which : {ISKV_WHICH_K, ISKV_WHICH_V}) {
+        cudaStream_t fs = which == ISKV_WHICH_K ? s : h->fold_side;
         fl.qscratch = which == ISKV_WHICH_K ? h->qscr_k : h->qscr_v;
         const FactorView f = view(h, which);
         if (h->cfg.joint)
-            CU(launch_fold_wide(f, fl, h->status, s));
+            CU(launch_fold_wide(f, fl, h->status, fs));
         else
-            CU(launch_fold(f, fl, h->status, s));
-        if (f.quant) CU(launch_quant_new_rows(f, fl, s));   // the block's rows, coded
+            CU(launch_fold(f, fl, h->status, fs));
+        if (f.quant) CU(launch_quant_new_rows(f, fl, fs));   // the block's rows, coded
     }
+    CU(cudaEventRecord(h->join_evt, h->fold_side));
+    CU(cudaStreamWaitEvent(s, h->join_evt, 0));
     std::vector<int> rl_layers, rl_seg, rl_rows;
     for (int l : fold_layers) {
         const bool defer = h->cfg.sync && (want_defer || h->n_pend[l] > 0);
@@ -814,6 +835,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.T = a.T;
         t.scale = a.scale;
         t.pipe_wait = h->pipe_wait;
+        t.idle_hint_ns = h->pipe_wait < tc::kWaitCycles ? 0u : 20000u;
         t.ptab = h->ptab;
         t.ptab_rows = h->ptab_rows;
         // exact-row tiles of 64 rows, or of 32 when 64 rows of K and V would make

@@ -260,6 +260,7 @@ struct DecodeTcArgs {
     float scale;
     long long pipe_wait;         // clock cycles a pipeline wait may take before the
                                  // call gives up (drain waits keep their own limit)
+    uint32_t idle_hint_ns;       // suspend hint of the single-lane warps' waits
     const void* ptab;            // fp16 [ptab_rows + P rounded to 64][128], 8 x 8 blocked:
                                  // cos, sin of pos w_i interleaved; row j < ptab_rows is
                                  // factor row j (pos = P + j), row ptab_rows + p is pos p

@@ -250,8 +250,8 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 if (head != prev) {
                     ++hs;
                     const int hb = hs % nbk;
-                    if (hs >= nbk && (!mbar_wait_idle(&bars->bk_empty[2 * hb], ((hs / nbk) - 1) & 1, deadline) ||
-                                      !mbar_wait_idle(&bars->bk_empty[2 * hb + 1], ((hs / nbk) - 1) & 1, deadline))) {
+                    if (hs >= nbk && (!mbar_wait_idle(&bars->bk_empty[2 * hb], ((hs / nbk) - 1) & 1, deadline, a.idle_hint_ns) ||
+                                      !mbar_wait_idle(&bars->bk_empty[2 * hb + 1], ((hs / nbk) - 1) & 1, deadline, a.idle_hint_ns))) {
                         fail();
                         break;
                     }
@@ -264,7 +264,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     prev = head;
                 }
                 const int st = n % ns;
-                if (n >= ns && !mbar_wait_idle(&bars->empty[st], ((n / ns) - 1) & 1, deadline)) {
+                if (n >= ns && !mbar_wait_idle(&bars->empty[st], ((n / ns) - 1) & 1, deadline, a.idle_hint_ns)) {
                     fail();
                     break;
                 }
@@ -771,7 +771,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
             // K^ of tile n into this group's buffer; exact-row tiles need none
             auto recon = [&](int n, int hb, bool win) -> bool {
                 const int st = n % ns;
-                if (!mbar_wait_idle(&bars->full[st], (n / ns) & 1, deadline)) return false;
+                if (!mbar_wait_idle(&bars->full[st], (n / ns) & 1, deadline, a.idle_hint_ns)) return false;
                 if (win) {
                     mbar_arrive(&bars->kh_full[grp]);
                     return true;
@@ -798,15 +798,15 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                 const int hb = hs % nbk;
                 const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
                 if (n_first < s1) {
-                    ok = mbar_wait_idle(&bars->bk_full[hb], (hs / nbk) & 1, deadline) &&
-                         (n_first < 2 || mbar_wait_idle(&bars->kfree[grp], ((n_first >> 1) - 1) & 1, deadline)) &&
+                    ok = mbar_wait_idle(&bars->bk_full[hb], (hs / nbk) & 1, deadline, a.idle_hint_ns) &&
+                         (n_first < 2 || mbar_wait_idle(&bars->kfree[grp], ((n_first >> 1) - 1) & 1, deadline, a.idle_hint_ns)) &&
                          recon(n_first, hb, (int)(f0 + n_first - hbase) >= tiles_c);
                 } else {
                     // no tile of this head for the group: its release of the basis
                     // buffer below still waits until the producer has filled the
                     // buffer for this head, so it can never run two releases ahead
                     // of the producer's parity wait on the same barrier
-                    ok = mbar_wait_idle(&bars->bk_full[hb], (hs / nbk) & 1, deadline);
+                    ok = mbar_wait_idle(&bars->bk_full[hb], (hs / nbk) & 1, deadline, a.idle_hint_ns);
                 }
                 for (int n = n_first; ok && n < s1; n += 2) {
                     const int st = n % ns;
@@ -818,7 +818,7 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     bool got = true;
                     for (int half = 0; half < 2; ++half) {
                         if (!mbar_wait_idle(half ? &bars->krot_b[grp] : &bars->krot_ready[grp], (n >> 1) & 1,
-                                       deadline)) {
+                                            deadline, a.idle_hint_ns)) {
                             got = false;
                             break;
                         }
@@ -839,14 +839,14 @@ decode_tc_kernel(const __grid_constant__ DecodeTcArgs a) {
                     // this tile's softmax.  Its data sits in stage (n + 2) % ns, which with
                     // two stages is tile n's own: then it has to wait for value(n) below.
                     auto next_recon = [&]() {
-                        return mbar_wait_idle(&bars->kfree[grp], (n >> 1) & 1, deadline) &&
+                        return mbar_wait_idle(&bars->kfree[grp], (n >> 1) & 1, deadline, a.idle_hint_ns) &&
                                recon(n + 2, hb, (int)(f0 + n + 2 - hbase) >= tiles_c);
                     };
                     if (ns >= 3 && n + 2 < s1 && !next_recon()) {
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait_idle(&bars->p_ready[grp], (n >> 1) & 1, deadline)) {
+                    if (!mbar_wait_idle(&bars->p_ready[grp], (n >> 1) & 1, deadline, a.idle_hint_ns)) {
                         ok = false;
                         break;
                     }

@@ -265,7 +265,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
             int issued = 0;
             for (int n = 0; n < ntiles && !*abort_flag; ++n) {
                 const int st = n % ns;
-                if (n >= ns && !mbar_wait_idle(&bars->empty[st], ((n / ns) - 1) & 1, deadline)) {
+                if (n >= ns && !mbar_wait_idle(&bars->empty[st], ((n / ns) - 1) & 1, deadline, a.idle_hint_ns)) {
                     fail();
                     break;
                 }
@@ -292,7 +292,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                 if (head != prev) {
                     ++hs;
                     const int b = hs & 1;
-                    if (hs >= 2 && !mbar_wait_idle(&bars->qempty[b], ((hs >> 1) - 1) & 1, deadline)) {
+                    if (hs >= 2 && !mbar_wait_idle(&bars->qempty[b], ((hs >> 1) - 1) & 1, deadline, a.idle_hint_ns)) {
                         fail();
                         break;
                     }
@@ -305,7 +305,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                     prev = head;
                 }
                 const int s = n & 1;
-                if (n >= 2 && !mbar_wait_idle(&bars->tempty[s], ((n >> 1) - 1) & 1, deadline)) {
+                if (n >= 2 && !mbar_wait_idle(&bars->tempty[s], ((n >> 1) - 1) & 1, deadline, a.idle_hint_ns)) {
                     fail();
                     break;
                 }
@@ -738,8 +738,8 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
             const uint32_t p0 = smem_u32(pb + grp * kPN * kTile);
             // U of tile n (this group's): after the epilogue has read U of tile n - 2
             auto issue_u = [&](int n, bool win) -> bool {
-                if (n >= 2 && !mbar_wait_idle(&bars->ufree[grp], ((n - 2) >> 1) & 1, deadline)) return false;
-                if (!mbar_wait_idle(&bars->tfull[grp], (n >> 1) & 1, deadline)) return false;
+                if (n >= 2 && !mbar_wait_idle(&bars->ufree[grp], ((n - 2) >> 1) & 1, deadline, a.idle_hint_ns)) return false;
+                if (!mbar_wait_idle(&bars->tfull[grp], (n >> 1) & 1, deadline, a.idle_hint_ns)) return false;
                 if (win) {
                     mbar_arrive(&bars->tempty[grp]);
                     mbar_arrive(&bars->u_full[grp]);
@@ -763,7 +763,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                 ++hs;
                 const int n_first = n0 + ((n0 & 1) != grp ? 1 : 0);
                 if (n_first < s1)
-                    ok = mbar_wait_idle(&bars->bq_full, hs & 1, deadline) &&
+                    ok = mbar_wait_idle(&bars->bq_full, hs & 1, deadline, a.idle_hint_ns) &&
                          issue_u(n_first, (int)(f0 + n_first - hbase) >= tiles_c);
                 for (int n = n_first; ok && n < s1; n += 2) {
                     const int st = n % ns;
@@ -772,8 +772,8 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait_idle(&bars->p_ready[grp], (n >> 1) & 1, deadline) ||
-                        !mbar_wait_idle(&bars->full[st], (n / ns) & 1, deadline)) {
+                    if (!mbar_wait_idle(&bars->p_ready[grp], (n >> 1) & 1, deadline, a.idle_hint_ns) ||
+                        !mbar_wait_idle(&bars->full[st], (n / ns) & 1, deadline, a.idle_hint_ns)) {
                         ok = false;
                         break;
                     }

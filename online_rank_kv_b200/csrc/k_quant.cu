@@ -19,6 +19,7 @@ namespace {
 
 constexpr int kRows = 64;
 constexpr int kThreads = 256;
+constexpr int kChunks = 4;   // 64-row chunks per rewrite block (W loaded once per segment)
 
 // Rows n_c .. n_c + 63 of every listed layer's factors from the fold's fp32
 // new rows.
@@ -33,9 +34,10 @@ __global__ void __launch_bounds__(kThreads) quant_new_rows_kernel(FactorView f, 
                      f.qscales + (hidx * f.n_max + n_c) * 4, sScale);
 }
 
-// The rewrite of coded rows, one block of 64 rows per CTA: decode, multiply by
-// the block's segment matrix (W_top of one fold, or the product of the
-// postponed ones from compose_kernel), code again in place.  The product is
+// The rewrite of coded rows, four chunks of 64 rows per CTA: decode, multiply
+// by the chunk's segment matrix (W_top of one fold, or the product of the
+// postponed ones from compose_kernel; loaded once while the segment lasts),
+// code again in place.  The product is
 // register-tiled: each thread owns 4 rows x r/16 columns (columns tx, tx + 16,
 // ...), so a k-step reads 4 + r/16 shared values for 4 r/16 FMAs; rows are
 // padded to r + 1 floats so the 4-row reads of a warp's two row groups fall in
@@ -43,13 +45,10 @@ __global__ void __launch_bounds__(kThreads) quant_new_rows_kernel(FactorView f, 
 __global__ void __launch_bounds__(kThreads) resync_quant_kernel(FactorView f, ResyncLaunch rl) {
     const int task = blockIdx.z, bh = blockIdx.y;
     const int layer = rl.layer[task];
-    const int64_t row0 = (int64_t)blockIdx.x * kRows;
-    if (row0 >= rl.n_rows[task]) return;
+    const int64_t base = (int64_t)blockIdx.x * kRows * kChunks;
+    if (base >= rl.n_rows[task]) return;
     const int nseg = rl.n_seg[task];
     const int* bounds = f.seg_rows + layer * f.D;
-    int seg = 0;
-    while (seg < nseg && row0 >= bounds[seg]) ++seg;
-    if (seg >= nseg) return;
     const int r = f.r, ld = r + 1, cg = r >> 3;
     extern __shared__ float sm[];
     float* sW = sm;                    // r x r
@@ -57,48 +56,61 @@ __global__ void __launch_bounds__(kThreads) resync_quant_kernel(FactorView f, Re
     float* sO = sC + kRows * ld;       // kRows x ld, rewritten rows
     float* sScale = sO + kRows * ld;   // kRows x 4
     const int64_t hidx = (int64_t)layer * f.BH + bh;
-    const float* W = f.pend + (hidx * f.D + seg) * (int64_t)r * r;
-    for (int e = threadIdx.x; e < r * r; e += kThreads) sW[e] = W[e];
-    const uint32_t* codes = f.qcodes + (hidx * f.n_max + row0) * f.qwords;
-    const float* scales = f.qscales + (hidx * f.n_max + row0) * 4;
-    for (int e = threadIdx.x; e < kRows * cg; e += kThreads) {
-        const int t = e / cg, c0 = (e - t * cg) * 8;
-        float v[8];
-        quant_decode8(f, codes + (int64_t)t * f.qwords, scales + t * 4, c0, v);
+    int loaded = -1;                   // segment whose matrix sits in sW
+    for (int ch = 0; ch < kChunks; ++ch) {
+        const int64_t row0 = base + ch * kRows;
+        if (row0 >= rl.n_rows[task]) break;
+        int seg = 0;
+        while (seg < nseg && row0 >= bounds[seg]) ++seg;
+        if (seg >= nseg) break;
+        if (seg != loaded) {
+            __syncthreads();           // the previous chunk's product has read sW
+            const float* W = f.pend + (hidx * f.D + seg) * (int64_t)r * r;
+            for (int e = threadIdx.x; e < r * r; e += kThreads) sW[e] = W[e];
+            loaded = seg;
+        }
+        const uint32_t* codes = f.qcodes + (hidx * f.n_max + row0) * f.qwords;
+        const float* scales = f.qscales + (hidx * f.n_max + row0) * 4;
+        for (int e = threadIdx.x; e < kRows * cg; e += kThreads) {
+            const int t = e / cg, c0 = (e - t * cg) * 8;
+            float v[8];
+            quant_decode8(f, codes + (int64_t)t * f.qwords, scales + t * 4, c0, v);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) sC[t * ld + c0 + k] = v[k];
-    }
-    __syncthreads();
-    {
-        const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;   // rows 4 ty.., columns tx + 16 k
-        const int nk = r >> 4;                                    // 1..8
-        float acc[4][8];
+            for (int k = 0; k < 8; ++k) sC[t * ld + c0 + k] = v[k];
+        }
+        __syncthreads();
+        {
+            const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;   // rows 4 ty.., columns tx + 16 k
+            const int nk = r >> 4;                                    // 1..8
+            float acc[4][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
-        const float* cr = sC + (4 * ty) * ld;
-        for (int j = 0; j < r; ++j) {
-            float a[4], w[8];
+                for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+            const float* cr = sC + (4 * ty) * ld;
+            for (int j = 0; j < r; ++j) {
+                float a[4], w[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = cr[i * ld + j];
+                for (int i = 0; i < 4; ++i) a[i] = cr[i * ld + j];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) w[k] = k < nk ? sW[j * r + tx + 16 * k] : 0.f;
+                for (int k = 0; k < 8; ++k) w[k] = k < nk ? sW[j * r + tx + 16 * k] : 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        if (k < nk) acc[i][k] = fmaf(a[i], w[k], acc[i][k]);
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    if (k < nk) acc[i][k] = fmaf(a[i], w[k], acc[i][k]);
+                    if (k < nk) sO[(4 * ty + i) * ld + tx + 16 * k] = acc[i][k];
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                if (k < nk) sO[(4 * ty + i) * ld + tx + 16 * k] = acc[i][k];
+        __syncthreads();
+        // (its last reads of sO come before the next chunk's barrier after decoding)
+        quant_rows_block(f, sO, ld, kRows, f.qcodes + (hidx * f.n_max + row0) * f.qwords,
+                         f.qscales + (hidx * f.n_max + row0) * 4, sScale);
     }
-    __syncthreads();
-    quant_rows_block(f, sO, ld, kRows, f.qcodes + (hidx * f.n_max + row0) * f.qwords,
-                     f.qscales + (hidx * f.n_max + row0) * 4, sScale);
 }
 
 // Caller rows (iskv_quantize_rows): rows [n][r] fp32 -> codes, scales.
@@ -174,7 +186,7 @@ cudaError_t launch_resync_quant(const FactorView& f, const ResyncLaunch& rl, cud
     cudaError_t e = cudaFuncSetAttribute(resync_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)bytes);
     if (e != cudaSuccess) return e;
-    dim3 grid((max_rows + kRows - 1) / kRows, f.BH, rl.n_tasks);
+    dim3 grid((max_rows + kRows * kChunks - 1) / (kRows * kChunks), f.BH, rl.n_tasks);
     resync_quant_kernel<<<grid, kThreads, bytes, s>>>(f, rl);
     return cudaGetLastError();
 }

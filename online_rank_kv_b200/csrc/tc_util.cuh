@@ -68,10 +68,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     return true;
 }
 // The same for a single-lane warp (producer, MMA issuer) that shares its
-// scheduler with compute warps: each try_wait may sleep up to 20 us, so a
-// long wait costs fewer issue slots (about 1 % of the decode time measured).
-__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, long long deadline) {
-    while (!mbar_try_wait_hint(bar, parity, 20000u)) {
+// scheduler with compute warps: each try_wait may sleep up to `hint_ns`
+// (20 us in normal calls), so a long wait costs fewer issue slots (about 1 %
+// of the decode time measured); 0 when a test shortens the pipeline waits, so
+// that a wait which must run out does.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, long long deadline,
+                                               uint32_t hint_ns) {
+    while (!mbar_try_wait_hint(bar, parity, hint_ns)) {
         if (clock64() > deadline) return false;
     }
     return true;

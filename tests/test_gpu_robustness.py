@@ -95,8 +95,10 @@ def test_query_side_kernel_range(monkeypatch):
     loud.close()
 
 
-def test_pipeline_wait_limit_reports_timeout_and_context_survives(monkeypatch):
+@pytest.mark.parametrize("kernel", ["rot", "u"])
+def test_pipeline_wait_limit_reports_timeout_and_context_survives(kernel, monkeypatch):
     import online_rank_kv_b200 as ik
+    monkeypatch.setenv("ISKV_DECODE_KERNEL", kernel)
     monkeypatch.setenv("ISKV_TEST_PIPELINE_WAIT_CYCLES", "1")
     short = ik.Cache(_cfg())
     monkeypatch.delenv("ISKV_TEST_PIPELINE_WAIT_CYCLES")
