@@ -317,7 +317,6 @@ def run_iskv(args, rank, world, local_rank):
                     coef_quant=1 if codes else 0, quant_k=wl.get("quant_k", ()),
                     quant_v=wl.get("quant_v", ()))
     cache = ik.Cache(cfg)
-    dec_kernel = KERNEL_OF[cache.decode_kernel()]
     P = args.protect
     kdt = torch.bfloat16
     nh = L * Bsz * H
@@ -504,6 +503,8 @@ def run_iskv(args, rank, world, local_rank):
     # the tensor-core path; split kernel + combine on the CUDA-core path; coded
     # caches first expand their K and V codes); per period and layer: fold (K, V)
     # + coefficient rewrite (K, V), coded caches also code the new rows (K, V)
+    # the decode kernel of the timed calls (the library's choice at the final n_c)
+    dec_kernel = KERNEL_OF[cache.decode_kernel(0)]
     per_step = 2 + (1 if coef == ik.BF16 else 3 if codes else 2)
     launches_per_period = L * (BLOCK * per_step + (6 if codes else 4))
     result = {
@@ -678,7 +679,6 @@ def run_growth(args, rank, world, local_rank):
                     max_tokens=max_tokens, kv_dtype=ik.BF16, coef_dtype=ik.BF16, use_rope=1,
                     rope_theta=1e6, max_deferred=64, ring_extra=512)
     cache = ik.Cache(cfg)
-    dec_kernel = KERNEL_OF[cache.decode_kernel()]
     nh = L * Bsz * H
     seed_k, seed_v, seed_q = replica_seeds(rank)
     ks = synth.KVStream(synth.spec_for(wl["gen"], "K"), nh, seed=seed_k, device=dev, dtype=torch.bfloat16)
@@ -734,7 +734,8 @@ def run_growth(args, rank, world, local_rank):
         fold_us, rw_us = _fold_and_rewrite_us(cache, ik, stream)
         rw_bytes = 2 * n_c1 * (rK + rV) * 2 * L * Bsz * H
         steps = args.steps * BLOCK
-        bins_out.append({"context": T0, "steps_per_s": steps / (ms / 1e3) * world,
+        bins_out.append({"context": T0, "decode_kernel": KERNEL_OF[cache.decode_kernel(0)],
+                         "steps_per_s": steps / (ms / 1e3) * world,
                          "ms_per_period": ms / args.steps,
                          "decode_us": dsum / max(1, len(dec_events)) * 1e6,
                          "decode_hbm_frac": (bsum / dsum / 1e9) / peak if dsum > 0 else None,
@@ -754,7 +755,7 @@ def run_growth(args, rank, world, local_rank):
         "warmup": BLOCK, "ms_per_step": tot_ms / (args.steps * len(bins)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "mixed bf16/fp16 MMA inputs, fp32 accumulate",
-        "precision": PRECISION[dec_kernel],
+        "precision": "; ".join(PRECISION[k] for k in sorted({b["decode_kernel"] for b in bins_out})),
         "data": "synthetic",
         "config": {"workload": args.workload, "batch": Bsz, "layers": L, "kv_heads": H,
                    "q_heads": Hq, "head_dim": D, "rank_k": rK, "rank_v": rV, "window": W,
@@ -823,6 +824,7 @@ def run_sweep(args, rank, world, local_rank):
                 ms = max_over_ranks(ms, world, dev)
                 dsum = sum(a.elapsed_time(b) for a, b, _, _ in dec_events) / 1e3
                 bsum = sum(_decode_bytes(Bsz, H, Hq, r, r, Tn, n_c, 2) for _, _, Tn, n_c in dec_events)
+                dk = KERNEL_OF[cache.decode_kernel(0)]   # the kernel the timed calls ran
                 _bring_to_ready(cache, ik, ks, vs, L, Bsz, H, W)
                 _, n_c1 = cache.counts(0)
                 fold_us, rw_us = _fold_and_rewrite_us(cache, ik, stream)
@@ -842,6 +844,7 @@ def run_sweep(args, rank, world, local_rank):
                                "context_start": T,
                                "step": "fold period: 64 decode steps + 1 fold with its rewrite"},
                     "decode_us": dsum / max(1, len(dec_events)) * 1e6,
+                    "decode_kernel": dk,
                     "decode_hbm_frac": (bsum / dsum / 1e9) / peak if dsum > 0 else None,
                     "peak": {"hbm_gbs": peak, "source": peak_src},
                     "fold_us": fold_us, "rewrite_us": rw_us,

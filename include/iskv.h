@@ -262,19 +262,22 @@ ISKV_API int iskv_get_counts(iskv_t h, int layer, int64_t* T, int64_t* n_c);
  * Errors: INVALID_ARG for a NULL cache.                                    */
 ISKV_API int iskv_kv_bytes(iskv_t h, int64_t* persistent_bytes, int64_t* full_bytes);
 
-/* The kernel iskv_decode_attention runs for this cache (fixed at creation
- * by the configuration and the environment): ISKV_DECODE_CUDA_CORE (split
- * fp32 CUDA-core kernel plus combine: fp32 coefficients or K/V, or the
- * tensor-core paths switched off with ISKV_TENSOR_CORES=0),
- * ISKV_DECODE_ROTATE (tensor cores; folded keys rebuilt, rotated and scored
- * per tile), ISKV_DECODE_QUERY_ROPE (tensor cores; RoPE folded into the
- * queries, scores from a position table times per-head query-basis products
- * -- where r_K * g <= 128; ISKV_DECODE_KERNEL=rot or =u overrides the
- * default between the two).  Host only.  Errors: INVALID_ARG.             */
+/* The kernel the next iskv_decode_attention of `layer` runs, given the
+ * configuration, the environment read at creation and the layer's current
+ * n_c: ISKV_DECODE_CUDA_CORE (split fp32 CUDA-core kernel plus combine: fp32
+ * coefficients or K/V, or tensor cores switched off with
+ * ISKV_TENSOR_CORES=0), ISKV_DECODE_ROTATE (tensor cores; folded keys
+ * rebuilt, rotated and scored per tile), ISKV_DECODE_QUERY_ROPE (tensor
+ * cores; RoPE folded into the queries, scores from a position table times
+ * per-head query-basis products; only where r_K * g <= 128).  Between the
+ * two tensor-core kernels the default takes the query-side one when the
+ * call's folded 128-row tiles number at least 200 per SM;
+ * ISKV_DECODE_KERNEL=u or =rot fixes the choice.  Host only.
+ * Errors: INVALID_ARG (NULL pointers, layer out of range).                */
 #define ISKV_DECODE_CUDA_CORE  0
 #define ISKV_DECODE_ROTATE     1
 #define ISKV_DECODE_QUERY_ROPE 2
-ISKV_API int iskv_decode_kernel(iskv_t h, int* kernel);
+ISKV_API int iskv_decode_kernel(iskv_t h, int layer, int* kernel);
 
 /* Code `n` fp32 rows of `rank` coefficients with the latent-channel format
  * `fmt` (see iskv_quant_format): rows [n][rank] fp32, codes [n][words]

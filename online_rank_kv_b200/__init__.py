@@ -100,7 +100,7 @@ _SIGS = {
     "iskv_get_factors": ([_vp, _i, _i, _vp, _vp, _vp, _vp], _i),
     "iskv_get_counts": ([_vp, _i, _i64p, _i64p], _i),
     "iskv_kv_bytes": ([_vp, _i64p, _i64p], _i),
-    "iskv_decode_kernel": ([_vp, ctypes.POINTER(_i)], _i),
+    "iskv_decode_kernel": ([_vp, _i, ctypes.POINTER(_i)], _i),
     "iskv_compress_block_async": ([_vp, _i, _i, _vp, _vp], _i),
     "iskv_status": ([_vp], _i),
     "iskv_strerror": ([_i], ctypes.c_char_p),
@@ -291,12 +291,12 @@ class Cache:
         _check(LIB.iskv_kv_bytes(self._h, ctypes.byref(p), ctypes.byref(f)), "iskv_kv_bytes")
         return p.value, f.value
 
-    def decode_kernel(self) -> str:
-        """The kernel decode_attention runs for this cache: "cuda_core",
+    def decode_kernel(self, layer: int = 0) -> str:
+        """The kernel the next decode_attention of `layer` runs: "cuda_core",
         "rotate" (tensor cores, keys rebuilt and rotated per tile) or
         "query_rope" (tensor cores, RoPE folded into the queries)."""
         k = _i()
-        _check(LIB.iskv_decode_kernel(self._h, ctypes.byref(k)), "iskv_decode_kernel")
+        _check(LIB.iskv_decode_kernel(self._h, layer, ctypes.byref(k)), "iskv_decode_kernel")
         return {0: "cuda_core", 1: "rotate", 2: "query_rope"}[k.value]
 
     def status(self) -> int:

@@ -74,7 +74,8 @@ struct iskv_cache {
     size_t stage_out_bytes = 0;
     int max_splits = 256;
     bool use_tc = true;           // tensor-core paths for bf16 coefficients
-    bool use_u = true;            // RoPE-in-the-queries decode where it applies
+    int use_u = 2;                // query-side RoPE decode: 0 never, 1 wherever it applies,
+                                  // 2 where a call gives each SM enough folded tiles
     int sms = 148;
     // clock cycles a tensor-core pipeline wait may take before the call gives
     // up with DEVICE_TIMEOUT; tests shorten it through the environment to make
@@ -105,8 +106,12 @@ struct TraceRange {
 
 constexpr size_t kStageBytes = 16u << 20;
 constexpr bool kDecodeTcDefault = true;
-// query-side RoPE decode by default where it applies (else the rotation kernel)
-constexpr bool kDecodeUDefault = false;
+// The query-side RoPE decode pays a fixed cost per CTA and head (building the
+// head's query-basis products) and keeps four stages instead of six; same-box
+// A/B (one layer, 8 KV / 32 query heads) put it ahead from about 200 folded
+// tiles per SM (batch 8 at 64K: -4 %; batch 32 at 64K: -17 %) and behind
+// below (batch 8 at 32K: +7 %; batch 1 at 128K: +28 %).
+constexpr int64_t kDecodeUMinTilesPerSm = 200;
 
 // Fill the code-format fields of a view from `q` for rank r; false if the
 // format is invalid (groups 1..4, channels multiples of 16 summing to r, bits
@@ -275,19 +280,23 @@ int dalloc(T** p, size_t bytes) {
     return ISKV_OK;
 }
 
-// The decode kernel of a cache (iskv_decode_kernel): tensor cores for bf16
-// K/V with bf16 (or coded, expanded per call) coefficients and g in {1, 2, 4,
-// 8}; among those the query-side RoPE kernel where r_K g <= 128 and it is
-// selected, else the rotation kernel.
-int decode_path(const iskv_cache* h) {
+// The decode kernel of a layer's next decode call (iskv_decode_kernel): tensor
+// cores for bf16 K/V with bf16 (or coded, expanded per call) coefficients and
+// g in {1, 2, 4, 8}; among those the query-side RoPE kernel where r_K g <= 128
+// and it is selected -- by ISKV_DECODE_KERNEL=u, or by default when the folded
+// tiles of the call give every SM at least kDecodeUMinTilesPerSm -- else the
+// rotation kernel.
+int decode_path(const iskv_cache* h, int layer) {
     const iskv_config& c = h->cfg;
     const int g = c.q_heads / c.kv_heads;
     const bool coded_tc = c.coef_quant && h->qws_k != nullptr;
     if (!(h->use_tc && (coded_tc || (!c.coef_quant && c.coef_dtype == ISKV_BF16)) &&
           c.kv_dtype == ISKV_BF16 && decode_tc_supports_group(g)))
         return ISKV_DECODE_CUDA_CORE;
-    if (h->use_u && h->ptab != nullptr && decode_u_supports(g, c.rank_k)) return ISKV_DECODE_QUERY_ROPE;
-    return ISKV_DECODE_ROTATE;
+    if (h->use_u == 0 || h->ptab == nullptr || !decode_u_supports(g, c.rank_k)) return ISKV_DECODE_ROTATE;
+    if (h->use_u == 1) return ISKV_DECODE_QUERY_ROPE;
+    const int64_t tiles = (int64_t)h->BH * ((h->n_c[layer] + 127) / 128);
+    return tiles >= kDecodeUMinTilesPerSm * h->sms ? ISKV_DECODE_QUERY_ROPE : ISKV_DECODE_ROTATE;
 }
 
 // A call on stream s that touches the listed layers runs after their last
@@ -411,8 +420,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         // rebuilds and rotates the keys, otherwise the query-side RoPE kernel
         // wherever r_K g <= 128
         const char* dk = std::getenv("ISKV_DECODE_KERNEL");
-        h->use_u = dk && std::strcmp(dk, "u") == 0 ? true
-                 : dk && std::strcmp(dk, "rot") == 0 ? false : kDecodeUDefault;
+        h->use_u = dk && std::strcmp(dk, "u") == 0 ? 1 : dk && std::strcmp(dk, "rot") == 0 ? 0 : 2;
         const char* w = std::getenv("ISKV_TEST_PIPELINE_WAIT_CYCLES");
         if (w && std::atoll(w) > 0) h->pipe_wait = std::atoll(w);
     }
@@ -799,7 +807,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.scale = 1.0f / std::sqrt((float)kHeadDim);
     const int sms = h->sms;
     const bool coded_tc = c.coef_quant && h->qws_k != nullptr;
-    const int path = decode_path(h);
+    const int path = decode_path(h, layer);
     if (path != ISKV_DECODE_CUDA_CORE) {
         // one persistent tensor-core kernel, one CTA per SM, over the flattened
         // (head, tile) space: 128-token tiles of folded rows, then 64-token
@@ -979,9 +987,9 @@ int iskv_get_factors(iskv_t h, int layer, int which, float* basis, float* sigma,
     return ISKV_OK;
 }
 
-int iskv_decode_kernel(iskv_t h, int* kernel) {
-    if (!h || !kernel) return ISKV_ERR_INVALID_ARG;
-    *kernel = decode_path(h);
+int iskv_decode_kernel(iskv_t h, int layer, int* kernel) {
+    if (!h || !kernel || layer < 0 || layer >= h->cfg.layers) return ISKV_ERR_INVALID_ARG;
+    *kernel = decode_path(h, layer);
     return ISKV_OK;
 }
 
