@@ -67,6 +67,7 @@ struct iskv_cache {
     __half* ptab = nullptr;       // fp16 position table (decode_u): factor rows j at
                                   // P + j, then the protected positions 0 .. P - 1
     int64_t ptab_rows = 0;        // rows of the factor-row part
+    uint32_t* aq = nullptr;       // per-call query-basis products of every head (decode_u)
     int* status = nullptr;
     void* stage_in = nullptr;     // host-input staging
     size_t stage_in_bytes = 0;
@@ -263,7 +264,7 @@ void free_all(iskv_cache* h) {
                     h->bsplit_k, h->bsplit_v, h->sigma_k, h->sigma_v, h->pend_k, h->pend_v,
                     h->qscr_k, h->qscr_v, h->seg_rows, h->partial, h->done, h->rope, h->status, h->stage_in, h->stage_out,
                     h->qcodes_k, h->qcodes_v, h->qscales_k, h->qscales_v, h->newrows_k, h->newrows_v,
-                    h->wide, h->qws_k, h->qws_v, h->ptab};
+                    h->wide, h->qws_k, h->qws_v, h->ptab, h->aq};
     for (void* p : ptrs)
         if (p) cudaFree(p);
 }
@@ -530,6 +531,7 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         const int64_t prows = (c.protect + 63) / 64 * 64;
         h->ptab_rows = rows;
         rc = dalloc(&h->ptab, (size_t)(rows + prows) * 128 * sizeof(__half));
+        rc = rc ? rc : dalloc(&h->aq, (size_t)h->BH * 128 * 64 * sizeof(uint32_t));
         if (rc == ISKV_OK) {
             std::vector<__half> tab((size_t)(rows + prows) * 128);
             std::vector<double> inv(d / 2);
@@ -846,6 +848,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.idle_hint_ns = h->pipe_wait < tc::kWaitCycles ? 0u : 20000u;
         t.ptab = h->ptab;
         t.ptab_rows = h->ptab_rows;
+        t.aq = h->aq;
         // exact-row tiles of 64 rows, or of 32 when 64 rows of K and V would make
         // a stage larger than a folded tile's C_K and C_V
         const int64_t coef_tile = (int64_t)128 * (c.rank_k + c.rank_v) * 2;

@@ -265,6 +265,7 @@ struct DecodeTcArgs {
                                  // cos, sin of pos w_i interleaved; row j < ptab_rows is
                                  // factor row j (pos = P + j), row ptab_rows + p is pos p
     int64_t ptab_rows;
+    uint32_t* aq;                // [BH][128 * 64] words: each head's query-basis products
 };
 
 // ---------------------------------------------------------------------------

@@ -322,11 +322,19 @@ decode_kernel(DecodeArgs a) {
                 const int h = e / width, col = e % width;
                 float v = acc[u] * sScale[h];
                 const float* ph = sS + h * kTile;
-                if (comp && col < rV) {
-                    for (int t = 0; t < nt; ++t) v = fmaf(ph[t], sV[t * L.ldv + col], v);
-                } else if (!comp && col >= rV) {
-                    const int i = col - rV;
-                    for (int t = 0; t < nt; ++t) v = fmaf(ph[t], sV[t * L.ldv + i], v);
+                // rows with t >= nt have p = 0 (their scores were -inf) and zeroed
+                // coefficients; whole tiles read four p values per shared load
+                const int c = comp ? col : col - rV;
+                if ((comp && col < rV) || (!comp && col >= rV)) {
+                    float v2 = 0.f;
+                    for (int t = 0; t < kTile; t += 4) {
+                        const float4 p4 = *reinterpret_cast<const float4*>(ph + t);
+                        v = fmaf(p4.x, sV[t * L.ldv + c], v);
+                        v2 = fmaf(p4.y, sV[(t + 1) * L.ldv + c], v2);
+                        v = fmaf(p4.z, sV[(t + 2) * L.ldv + c], v);
+                        v2 = fmaf(p4.w, sV[(t + 3) * L.ldv + c], v2);
+                    }
+                    v += v2;
                 }
                 acc[u] = v;
             }

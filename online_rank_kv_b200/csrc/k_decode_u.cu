@@ -19,21 +19,22 @@
 // epilogue thread then needs its row's r_K coefficients and r_K g products.
 // No key is rebuilt, rotated or rounded: the only roundings are the fp16
 // table and the fp16 A_h, both ~2^-12 relative.  Exact rows (the window and
-// the protected rows) are rotated and scored on the CUDA cores in fp32 with
-// the full-position RoPE table.  Values as in the rebuild kernel:
+// the protected rows) are rotated and scored on the CUDA cores in fp32, four
+// threads per row, with their rows of the fp16 position table.  Values as in the rebuild kernel:
 // acc_h = sum_j p_j C_V[j] by the value MMA, B_V^T once per query head.
 //
 // Persistent, one CTA per SM over cost-balanced runs of the flattened (head,
 // tile) space.  Per CTA 12 warps:
-//   warp 0  lane 0: C_K, C_V tiles or exact K, V rows into an ns-stage ring;
+//   warp 0  lane 0: C_K, C_V tiles or exact K, V rows (and their fp16 RoPE
+//           table rows) into an ns-stage ring;
 //   warp 1  TMEM allocation; lane 0: the position-table slice of each tile
-//           (one slot per epilogue group) and each head's queries;
+//           (one slot per epilogue group), each head's queries, and each
+//           head's A_h (prepared for all heads by aq_kernel before the decode
+//           kernel) once both groups are done with the previous head's;
 //   warps 2-9 epilogue, two groups of 4 warps (group = tile parity), one
 //           row per thread: scores, online softmax with a lazy maximum, p as
-//           bf16 hi + lo; at each head change all 256 threads build A_h (fp16,
-//           the MMA's B operand) and the fp32 queries for exact rows;
-//           per head each group publishes its partial, the last to publish
-//           merges them all by log-sum-exp and applies B_V^T;
+//           bf16 hi + lo; per head each group publishes its partial, the
+//           last to publish merges them all by log-sum-exp and applies B_V^T;
 //   warps 10-11 MMA issuer of group 0 / 1: U = T_p A_h for the group's next
 //           tile as soon as the previous U has been read, O = C_V^T P.
 // Every mbarrier wait is bounded (status bit 2 on timeout, copies drained,
@@ -61,13 +62,14 @@ struct __align__(8) Bars {
     uint64_t full[kMaxStages], empty[kMaxStages];   // coefficient / exact-row stage ring
     uint64_t tfull[2], tempty[2];                   // position-table slot of each group
     uint64_t qfull[2], qempty[2];                   // a head's bf16 queries (two buffers)
-    uint64_t bq_full;                               // A_h of the current head built
+    uint64_t bq_full;                               // A_h of the current head copied in
+    uint64_t bq_free;                               // both groups done with the current A_h
     uint64_t u_full[2], ufree[2], o_full[2], p_ready[2];
     uint64_t drain[3];
 };
 
 struct SmemPlan {
-    uint32_t tab, bq, qraw, qf, stage, stage_k, stage_bytes, pb, ms, total;
+    uint32_t tab, bq, qraw, stage, stage_k, stage_bytes, pb, ms, total;
 };
 
 __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int wt) {
@@ -76,7 +78,6 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int wt) {
     p.tab = off;    off += 2 * kTabBytes;                    // [group] table slice
     p.bq = off;     off += kBqBytes;                         // A_h
     p.qraw = off;   off += 2 * kMaxGroup * kHeadDim * 2;     // [2] bf16 queries
-    p.qf = off;     off += kMaxGroup * kHeadDim * 4;         // fp32 queries
     p.stage_k = (uint32_t)kTile * rK * 2;
     uint32_t sb = p.stage_k + kTile * rV * 2;
     if (sb < 3 * wt * kHeadDim * 2) sb = 3 * wt * kHeadDim * 2;   // exact: K, V, RoPE rows
@@ -88,7 +89,6 @@ __host__ __device__ inline SmemPlan plan_smem(int rK, int rV, int ns, int wt) {
     return p;
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ void group_sync(int grp) {
     asm volatile("bar.sync %0, 128;" ::"r"(2 + grp) : "memory");
 }
@@ -156,7 +156,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
     Bars* bars = reinterpret_cast<Bars*>(smem);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + sizeof(Bars));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 4);
-    volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);
+    volatile int* epi_abort = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 8);    // [2]
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + sizeof(Bars) + 16);   // [2]
     static_assert(sizeof(Bars) + 24 <= 512, "scratch words fit below the reduction area");
     float* red = reinterpret_cast<float*>(smem + 512);          // [2 groups][max 4x8 | l 4x8]
@@ -164,7 +164,6 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
     uint8_t* tab = smem + P.tab;
     uint32_t* bqw = reinterpret_cast<uint32_t*>(smem + P.bq);
     __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(smem + P.qraw);
-    float* qf = reinterpret_cast<float*>(smem + P.qf);
     uint8_t* stage = smem + P.stage;
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem + P.pb);
     float* mscr = reinterpret_cast<float*>(smem + P.ms);
@@ -189,13 +188,14 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
             mbar_init(&bars->tfull[i], 1);
             mbar_init(&bars->tempty[i], 1);
             mbar_init(&bars->qfull[i], 1);
-            mbar_init(&bars->qempty[i], 1);
+            mbar_init(&bars->qempty[i], 2);   // both groups, after their tiles of the head
             mbar_init(&bars->u_full[i], 1);
             mbar_init(&bars->ufree[i], 128);
             mbar_init(&bars->o_full[i], 1);
             mbar_init(&bars->p_ready[i], 1);
         }
         mbar_init(&bars->bq_full, 1);
+        mbar_init(&bars->bq_free, 2);
         for (int i = 0; i < 3; ++i) mbar_init(&bars->drain[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -285,7 +285,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
     } else if (warp == 1) {
         // ---------------- producer: position-table slices and queries ----------------
         if (lane == 0) {
-            int hs = -1, prev = -1, tissued = 0, qissued = 0;
+            int hs = -1, prev = -1, tissued = 0, qissued = 0, bqissued = 0;
             for (int n = 0; n < ntiles && !*abort_flag; ++n) {
                 const int64_t fi = f0 + n;
                 const int head = (int)(fi / tph), tile = (int)(fi % tph);
@@ -301,6 +301,15 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                                               ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
                     mbar_arrive_expect_tx(&bars->qfull[b], q_bytes);
                     bulk_g2s(qraw + b * kMaxGroup * d, qg, q_bytes, &bars->qfull[b]);
+                    // the head's query-basis products (prepared for every head by
+                    // aq_kernel) once both groups are done with the previous head's
+                    if (hs >= 1 && !mbar_wait_idle(&bars->bq_free, (hs - 1) & 1, deadline, a.idle_hint_ns)) {
+                        fail();
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars->bq_full, (uint32_t)NU * 256);
+                    bulk_g2s(bqw, a.aq + (int64_t)head * kUN * 64, (uint32_t)NU * 256, &bars->bq_full);
+                    bqissued = hs + 1;
                     qissued = hs + 1;
                     prev = head;
                 }
@@ -322,6 +331,7 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                     mbar_wait(&bars->tfull[n & 1], (n >> 1) & 1, deadline + kWaitCycles);
                 for (int h = qissued - 2 > 0 ? qissued - 2 : 0; h < qissued; ++h)
                     mbar_wait(&bars->qfull[h & 1], (h >> 1) & 1, deadline + kWaitCycles);
+                if (bqissued > 0) mbar_wait(&bars->bq_full, (bqissued - 1) & 1, deadline + kWaitCycles);
             }
         }
     } else if (warp >= 2 && warp < 10) {
@@ -356,46 +366,14 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
             int s1 = (int)(((int64_t)head + 1) * tph - f0);
             if (s1 > ntiles) s1 = ntiles;
             ++hs;
-            // epilogue-uniform abort check (both groups build A_h together)
-            if (ept == 0) *epi_abort = *abort_flag;
-            epi_sync();
-            if (*epi_abort) break;
-            // ---- A_h and the fp32 queries of this head (all 256 threads) ----
-            {
-                const int b = hs & 1;
-                if (!mbar_wait(&bars->qfull[b], (hs >> 1) & 1, deadline)) fail();
-                const __nv_bfloat16* sq = qraw + b * kMaxGroup * d;
-                const float* Bk = a.K.basis + ((int64_t)a.layer * BH + head) * d * rK;
-                // items e = (i, n): 8 per thread in flight (the basis comes from L2/HBM)
-                for (int e0 = ept; e0 < NU * 64; e0 += 256 * 8) {
-                    float b1[8], b2[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int e = e0 + 256 * u;
-                        const int i = e / NU, m = (e - i * NU) % rK;
-                        b1[u] = e < NU * 64 ? __ldg(Bk + i * rK + m) : 0.f;
-                        b2[u] = e < NU * 64 ? __ldg(Bk + (i + 64) * rK + m) : 0.f;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int e = e0 + 256 * u;
-                        if (e >= NU * 64) break;
-                        const int i = e / NU, n = e - i * NU;
-                        const int h = n / rK;
-                        const float q1 = __bfloat162float(sq[h * d + i]), q2 = __bfloat162float(sq[h * d + i + 64]);
-                        const __half2 w = __floats2half2_rn(fmaf(q1, b1[u], q2 * b2[u]), fmaf(q2, b1[u], -q1 * b2[u]));
-                        bqw[bq_off(n, i)] = *reinterpret_cast<const uint32_t*>(&w);
-                    }
-                }
-                for (int e = ept; e < g * d; e += 256) qf[e] = __bfloat162float(sq[e]);
-                fence_async_smem();
-                epi_sync();
-                if (ept == 0) {
-                    mbar_arrive(&bars->bq_full);
-                    mbar_arrive(&bars->qempty[b]);
-                }
-            }
-            const float* qfh = qf;
+            // group-uniform abort check
+            if (gt == 0) epi_abort[grp] = *abort_flag;
+            group_sync(grp);
+            if (epi_abort[grp]) break;
+            // the head's bf16 queries (exact rows read them)
+            const int qbuf = hs & 1;
+            if (!mbar_wait(&bars->qfull[qbuf], (hs >> 1) & 1, deadline)) fail();
+            const __nv_bfloat16* sq = qraw + qbuf * kMaxGroup * d;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 m_run[h] = -INFINITY;
@@ -489,20 +467,20 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                             }
 #pragma unroll
                             for (int h = 0; h < G; ++h) {
-                                const float4* q1 = reinterpret_cast<const float4*>(qfh + h * d + 16 * part);
-                                const float4* q2 = reinterpret_cast<const float4*>(qfh + h * d + 64 + 16 * part);
+                                // the query's dims 16 p .. 16 p + 15 and 64 + 16 p .. (bf16)
+                                const uint4* q1 = reinterpret_cast<const uint4*>(sq + h * d + 16 * part);
+                                const uint4* q2 = reinterpret_cast<const uint4*>(sq + h * d + 64 + 16 * part);
                                 float sa = 0.f, sb = 0.f;
 #pragma unroll
-                                for (int k4 = 0; k4 < 4; ++k4) {
-                                    const float4 a4 = q1[k4], b4 = q2[k4];
-                                    sa = fmaf(a4.x, x1[4 * k4], sa);
-                                    sa = fmaf(a4.y, x1[4 * k4 + 1], sa);
-                                    sa = fmaf(a4.z, x1[4 * k4 + 2], sa);
-                                    sa = fmaf(a4.w, x1[4 * k4 + 3], sa);
-                                    sb = fmaf(b4.x, x2[4 * k4], sb);
-                                    sb = fmaf(b4.y, x2[4 * k4 + 1], sb);
-                                    sb = fmaf(b4.z, x2[4 * k4 + 2], sb);
-                                    sb = fmaf(b4.w, x2[4 * k4 + 3], sb);
+                                for (int k8 = 0; k8 < 2; ++k8) {
+                                    float qa[8], qb8[8];
+                                    unpack_bf16x8(q1[k8], qa);
+                                    unpack_bf16x8(q2[k8], qb8);
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) {
+                                        sa = fmaf(qa[e], x1[8 * k8 + e], sa);
+                                        sb = fmaf(qb8[e], x2[8 * k8 + e], sb);
+                                    }
                                 }
                                 s4[h] = sa + sb;
                             }
@@ -596,6 +574,11 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
                 have_prev = true;
                 prev_win = win;
                 last = n;
+            }
+            // this group has read every U of the head and its queries: release both
+            if (gt == 0) {
+                mbar_arrive(&bars->bq_free);
+                mbar_arrive(&bars->qempty[qbuf]);
             }
             // close this group's share of the head
             if (have_prev) {
@@ -808,6 +791,32 @@ decode_u_kernel(const __grid_constant__ DecodeTcArgs a) {
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// A_h of every (sequence, KV head) of the call, in the word order of the U
+// product's B operand (bq_off): alpha, beta of frequency i for row n = h r_K + m
+// as an fp16 pair, computed in fp32 from the bf16 queries and the fp32 basis.
+// One CTA per head; the decode kernel bulk-copies a head's 32 KB when it
+// reaches the head.
+__global__ void __launch_bounds__(256) aq_kernel(const __grid_constant__ DecodeTcArgs a) {
+    const int head = blockIdx.x;
+    const int rK = a.K.r, g = a.g, NU = rK * g;
+    constexpr int d = kHeadDim;
+    const int bq = head / a.Hkv, kvh = head % a.Hkv;
+    __shared__ float sq[kMaxGroup * kHeadDim];
+    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(a.q) + ((int64_t)bq * a.Hq + (int64_t)kvh * g) * d;
+    for (int e = threadIdx.x; e < g * d; e += 256) sq[e] = __bfloat162float(q[e]);
+    __syncthreads();
+    const float* Bk = a.K.basis + ((int64_t)a.layer * a.K.BH + head) * d * rK;
+    uint32_t* out = a.aq + (int64_t)head * kUN * 64;
+    for (int e = threadIdx.x; e < NU * 64; e += 256) {
+        const int i = e / NU, n = e - i * NU;
+        const int h = n / rK, m = n - h * rK;
+        const float b1 = __ldg(Bk + i * rK + m), b2 = __ldg(Bk + (i + 64) * rK + m);
+        const float q1 = sq[h * d + i], q2 = sq[h * d + i + 64];
+        const __half2 w = __floats2half2_rn(fmaf(q1, b1, q2 * b2), fmaf(q2, b1, -q1 * b2));
+        out[bq_off(n, i)] = *reinterpret_cast<const uint32_t*>(&w);
+    }
+}
+
 }  // namespace
 
 size_t decode_u_smem_bytes(int rK, int rV, int ns, int wt) { return plan_smem(rK, rV, ns, wt).total; }
@@ -827,8 +836,11 @@ static cudaError_t launch_u(const DecodeTcArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_decode_u(const DecodeTcArgs& a, cudaStream_t s) {
-    if (!decode_u_supports(a.g, a.K.r) || a.stages < 2 || a.stages > kMaxStages || a.ptab == nullptr)
+    if (!decode_u_supports(a.g, a.K.r) || a.stages < 2 || a.stages > kMaxStages || a.ptab == nullptr ||
+        a.aq == nullptr)
         return cudaErrorNotSupported;
+    aq_kernel<<<a.K.BH, 256, 0, s>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
     switch (a.g) {
         case 1: return launch_u<1>(a, s);
         case 2: return launch_u<2>(a, s);
