@@ -145,3 +145,36 @@ def test_tc_decode_single_basis_buffer_heads_split_across_runs():
         errs, _ = p.decode(0, p.query())
         assert max(errs.values()) < TOL_BF16, errs
     assert p.cache.status() == 0
+
+
+def test_decode_kernel_choice(monkeypatch):
+    """iskv_decode_kernel names the kernel the next decode call runs: the
+    CUDA-core kernel for fp32 coefficients or with tensor cores off; between
+    the tensor-core kernels the query-side one only where r_K g <= 128, by
+    request, or by default once a call has >= 200 folded tiles per SM (none
+    at n_c = 0)."""
+    import online_rank_kv_b200 as ik
+
+    def kernel(env=None, **kw):
+        for k in ("ISKV_DECODE_KERNEL", "ISKV_TENSOR_CORES"):
+            monkeypatch.delenv(k, raising=False)
+        for k, v in (env or {}).items():
+            monkeypatch.setenv(k, v)
+        c = ik.Cache(_cfg(**kw))
+        try:
+            return c.decode_kernel(0)
+        finally:
+            c.close()
+
+    assert kernel(coef_dtype=ik.F32) == "cuda_core"
+    assert kernel({"ISKV_TENSOR_CORES": "0"}) == "cuda_core"
+    assert kernel() == "rotate"                                  # n_c = 0: no folded tiles yet
+    assert kernel({"ISKV_DECODE_KERNEL": "u"}) == "query_rope"   # r_K g = 32 * 4 = 128
+    assert kernel({"ISKV_DECODE_KERNEL": "rot"}) == "rotate"
+    assert kernel({"ISKV_DECODE_KERNEL": "u"}, rank_k=64) == "rotate"   # r_K g = 256
+    with pytest.raises(ik.IskvError):
+        c = ik.Cache(_cfg())
+        try:
+            c.decode_kernel(5)                                   # layer out of range
+        finally:
+            c.close()
