@@ -49,6 +49,10 @@ WORKLOADS = {
     "qwen3-1L-b8-32k-joint": dict(batch=8, layers=1, kv_heads=8, q_heads=32, rank_k=64,
                                   rank_v=96, window=1024, prefill=32768, coef="bf16",
                                   gen="qwen3", joint=1),
+    # one point of the sweep (r 32, 64K, batch 32) as its own workload: the decode
+    # runs the query-side RoPE kernel there (>= 200 folded tiles per SM)
+    "qwen3-1L-b32-64k-r32": dict(batch=32, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=32,
+                                 window=1024, prefill=65536, coef="bf16", gen="qwen3"),
     # low-bit latent-channel codes: K 16 ch x 8 b + 16 x 4 b, V 16 x 8 + 16 x 4 + 32 x 2
     "qwen3-1L-b8-32k-codes": dict(batch=8, layers=1, kv_heads=8, q_heads=32, rank_k=32, rank_v=64,
                                   window=1024, prefill=32768, coef="codes", gen="qwen3",
@@ -68,6 +72,7 @@ SWEEP = {"sweep": dict(layers=1, kv_heads=8, q_heads=32, window=1024, coef="bf16
                        ranks=[16, 32, 64, 128], contexts=[4096, 16384, 65536, 262144],
                        batches=[1, 8, 32])}
 DEFAULT_WORKLOAD = "qwen3-36L-b8-32k"
+L2_BYTES = 126e6   # B200 L2
 D = 128
 BLOCK = 64
 
@@ -78,8 +83,8 @@ BLOCK = 64
 # 36-layer run issues the same launch once per layer).  Not measured by this
 # run: reported as copied, with its source, and only while the decode kernel
 # is the one that was captured (None otherwise, and for other workloads).
-DECODE_TRAFFIC = {("qwen3-36L-b8-32k", "decode_tc_kernel"): 433.4e6,
-                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 433.4e6}
+DECODE_TRAFFIC = {("qwen3-36L-b8-32k", "decode_tc_kernel"): 434.6e6,
+                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 434.6e6}
 DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode launch "
                          "at this per-layer shape (one-layer 32K workload, full ncu capture of the "
                          "decode kernel); copied, not measured in this run")
@@ -448,6 +453,7 @@ def run_iskv(args, rank, world, local_rank):
         bsum += byts
     dec_avg_us = dsum / max(1, len(dec_events)) * 1e6
     achieved = bsum / dsum / 1e9 if dsum > 0 else 0.0
+    step_bytes = bsum / max(1, len(dec_events)) * L   # one decode step over every layer
 
     # ---- block update timing (fold and rewrite separately), untimed pass
     fold_us = resync_us = None
@@ -526,7 +532,10 @@ def run_iskv(args, rank, world, local_rank):
             "storage": f"K/V bf16, coefficients {wl['coef']}, bases fp32",
             "step": "64 decode steps (append + decode attention, every layer) + 1 block fold "
                     "of every layer (fold + coefficient rewrite)",
-            "l2": "inputs larger than L2 (each decode step streams ~15 GB)",
+            "l2": (f"inputs larger than L2 (each decode step streams {step_bytes / 1e9:.2f} GB "
+                   f"over {L} layer(s), L2 126 MB)" if step_bytes > L2_BYTES else
+                   f"inputs smaller than L2 ({step_bytes / 1e6:.0f} MB per decode step, L2 126 MB): "
+                   f"steps reuse L2, no flush"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
         "tokens_per_s": value * Bsz,
