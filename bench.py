@@ -77,17 +77,17 @@ D = 128
 BLOCK = 64
 
 
-# DRAM bytes (read + write) of one decode-attention launch at the per-layer
-# shape of the 32K-context, batch-8 workloads (8 KV / 32 query heads, r_K 32,
-# r_V 64), taken from an ncu capture of the one-layer workload (the
-# 36-layer run issues the same launch once per layer).  Not measured by this
+# DRAM bytes (read + write) of one decode-attention launch of the named kernel
+# at a workload's per-layer shape, taken from an ncu capture of the one-layer
+# workload (the 36-layer run issues the same launch once per layer).  Not measured by this
 # run: reported as copied, with its source, and only while the decode kernel
 # is the one that was captured (None otherwise, and for other workloads).
 DECODE_TRAFFIC = {("qwen3-36L-b8-32k", "decode_tc_kernel"): 434.6e6,
-                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 434.6e6}
+                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 434.6e6,
+                  ("qwen3-1L-b32-64k-r32", "decode_u_kernel"): 2338.4e6}
 DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode launch "
-                         "at this per-layer shape (one-layer 32K workload, full ncu capture of the "
-                         "decode kernel); copied, not measured in this run")
+                         "at this per-layer shape (full ncu capture of the decode kernel on the "
+                         "one-layer workload of this shape); copied, not measured in this run")
 
 
 
