@@ -27,7 +27,7 @@ constexpr int kMaxAcc = kMaxGroup * (kHeadDim + kHeadDim) / kThreads;  // 8
 // vector reads stay aligned and the rows a warp touches fall in different banks.
 struct Smem {
     int ldc, ldv;                       // row strides of the C_K and C_V / V tiles
-    size_t b, q, c, v, s, misc;
+    size_t b, q, c, v, s, rt, misc;
 };
 
 __host__ __device__ inline Smem smem_layout(int rK, int rV, int g) {
@@ -39,12 +39,13 @@ __host__ __device__ inline Smem smem_layout(int rK, int rV, int g) {
     L.c = (size_t)kTile * L.ldc;
     L.v = (size_t)kTile * L.ldv;
     L.s = (size_t)kMaxGroup * kTile;
+    L.rt = (size_t)17 * 64 * 2;                    // RoPE steps: R(4 t_i) for t_i < 16, R(1)
     L.misc = 4 * (size_t)kMaxGroup;
     return L;
 }
 
 __host__ __device__ inline size_t smem_floats(const Smem& L) {
-    return L.b + L.q + L.c + L.v + L.s + L.misc;
+    return L.b + L.q + L.c + L.v + L.s + L.rt + L.misc;
 }
 
 __device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
@@ -85,6 +86,7 @@ decode_kernel(DecodeArgs a) {
     float* sMax = sS + L.s;
     float* sSum = sMax + kMaxGroup;
     float* sScale = sSum + kMaxGroup;
+    float2* sR = reinterpret_cast<float2*>(sScale + kMaxGroup);   // [17][64]
 
     const float* Bk = a.K.basis + hidx * d * rK;   // [d][rK]
     for (int e = tid; e < d * rK; e += kThreads) {
@@ -98,6 +100,13 @@ decode_kernel(DecodeArgs a) {
         sSum[tid] = 0.f;
         sScale[tid] = 1.f;
     }
+    // RoPE steps from the table's exact rows: R(4 t_i) (positions 0, 4, .., 60)
+    // and R(1); a row at j + 4 t_i + u turns by R(j) R(4 t_i) R(1)^u
+    if (a.rope)
+        for (int e = tid; e < 17 * 64; e += kThreads) {
+            const int rr = e >> 6, fq = e & 63;
+            sR[e] = a.rope[(rr < 16 ? 4 * rr : 1) * (d / 2) + fq];
+        }
     const int width = rV + d;
     const int n_acc = g * width;
     float acc[kMaxAcc];
@@ -116,6 +125,10 @@ decode_kernel(DecodeArgs a) {
     __syncthreads();
 
     for (int64_t j = j0; j < j1;) {
+        // R(j) of this thread's four frequencies: loaded now, used after the rebuild
+        float2 rj[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) rj[m] = a.rope ? a.rope[j * (d / 2) + dlo + m] : make_float2(1.f, 0.f);
         const bool prot = j < P;
         const bool comp = !prot && j < c_end;
         int64_t jend = j + kTile;
@@ -247,18 +260,22 @@ decode_kernel(DecodeArgs a) {
         }
         // ---- RoPE at the row's position: (k_i, k_{i+64}) by angle pos * w_i ----
         if (a.rope) {
+            float2 rb[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float2 r4 = sR[ti * 64 + dlo + m];
+                rb[m] = make_float2(rj[m].x * r4.x - rj[m].y * r4.y, rj[m].x * r4.y + rj[m].y * r4.x);
+            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int t = 4 * ti + u;
-                if (t < nt) {
-                    const float2* cs = a.rope + (j + t) * (d / 2) + dlo;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const float2 r = cs[m];
-                        const float x1 = k[u][m], x2 = k[u][m + 4];
-                        k[u][m] = x1 * r.x - x2 * r.y;
-                        k[u][m + 4] = x1 * r.y + x2 * r.x;
-                    }
+                for (int m = 0; m < 4; ++m) {
+                    const float2 r = rb[m];
+                    const float x1 = k[u][m], x2 = k[u][m + 4];
+                    k[u][m] = x1 * r.x - x2 * r.y;
+                    k[u][m + 4] = x1 * r.y + x2 * r.x;
+                    const float2 r1 = sR[16 * 64 + dlo + m];
+                    rb[m] = make_float2(r.x * r1.x - r.y * r1.y, r.x * r1.y + r.y * r1.x);
                 }
             }
         }

@@ -124,10 +124,10 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(FactorView f, cons
 
 // The decode workspace of a coded layer: rows [0, rows) of every head as bf16
 // values code * scale, in the 8 x 8 blocked layout the tensor-core decode
-// bulk-copies.  Thread e of a head writes the 16 bytes at element 8 e of the
-// head's blocked rows: row (e >> 3) / cg * 8 + (e & 7), columns 8 ((e >> 3) %
-// cg) .. + 7, so a warp's stores are one contiguous 512-byte run.  Rows of the
-// last 8-row group past `rows` are written as zeros.
+// bulk-copies.  One thread per row: a warp reads 32 consecutive rows' code
+// words and scales (contiguous runs), and writes each 8-column block of its
+// rows as 16-byte words (8 rows of a block are one contiguous 128 bytes).
+// Rows of the last 8-row group past `rows` are written as zeros.
 __global__ void __launch_bounds__(kThreads) expand_codes_kernel(FactorView f, int layer, int rows,
                                                                  __nv_bfloat16* dst) {
     const int r = f.r, cg = r >> 3;
@@ -136,23 +136,24 @@ __global__ void __launch_bounds__(kThreads) expand_codes_kernel(FactorView f, in
     const uint32_t* codes = f.qcodes + hidx * f.n_max * f.qwords;
     const float* scales = f.qscales + hidx * f.n_max * 4;
     uint4* out = reinterpret_cast<uint4*>(dst + (int64_t)bh * f.n_max * r);
-    const int total = ((rows + 7) >> 3) * cg * 8;
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-        const int q = e >> 3;
-        const int rb = q / cg;
-        const int row = rb * 8 + (e & 7), c0 = (q - rb * cg) * 8;
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        if (row < rows) {
-            float v[8];
-            quant_decode8(f, codes + (int64_t)row * f.qwords, scales + (int64_t)row * 4, c0, v);
+    const int total = (rows + 7) & ~7;
+    for (int row = blockIdx.x * blockDim.x + threadIdx.x; row < total; row += gridDim.x * blockDim.x) {
+        const uint32_t* rc = codes + (int64_t)row * f.qwords;
+        const float* rs = scales + (int64_t)row * 4;
+        for (int cb = 0; cb < cg; ++cb) {
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            if (row < rows) {
+                float v[8];
+                quant_decode8(f, rc, rs, cb * 8, v);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const __nv_bfloat16 lo = __float2bfloat16_rn(v[2 * u]);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(v[2 * u + 1]);
-                w[u] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+                for (int u = 0; u < 4; ++u) {
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(v[2 * u]);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(v[2 * u + 1]);
+                    w[u] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+                }
             }
+            out[((row >> 3) * cg + cb) * 8 + (row & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        out[e] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -162,7 +163,7 @@ cudaError_t launch_expand_codes(const FactorView& f, int layer, int64_t rows, __
                                 cudaStream_t s) {
     if (rows <= 0) return cudaSuccess;
     if (rows > f.n_max || f.BH > 65535) return cudaErrorInvalidValue;
-    const int64_t per_head = ((rows + 7) / 8) * (f.r / 8) * 8;
+    const int64_t per_head = (rows + 7) / 8 * 8;   // one thread per row
     int64_t bx = (per_head + kThreads - 1) / kThreads;
     // about 8 resident CTAs per SM over all heads; each thread loops over the rest
     const int64_t want = (8 * 148 + f.BH - 1) / f.BH;
