@@ -113,6 +113,15 @@ def test_joint_factor_bf16_rank_128_tensor_core_decode():
     _run(128, 128, ik.BF16, tol=2e-2)
 
 
+def test_joint_factor_query_side_decode(monkeypatch):
+    """The query-side RoPE kernel on joint-head factors (r_K 32, g 4: N = 128):
+    each head's A_h from its 128 rows of the layer-wide basis, coefficient
+    tiles shared by the sequence's heads."""
+    import online_rank_kv_b200 as ik
+    monkeypatch.setenv("ISKV_DECODE_KERNEL", "u")
+    _run(32, 64, ik.BF16, tol=2e-2)
+
+
 def test_joint_factor_postponed_rewrites_four_heads():
     import online_rank_kv_b200 as ik
     _run(64, 64, ik.BF16, H=4, batch=3, tol=2e-2, defer=True)

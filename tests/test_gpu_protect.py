@@ -32,10 +32,14 @@ def _cfg(**kw):
     return c
 
 
-@pytest.mark.parametrize("coef", ["f32", "bf16"])
+@pytest.mark.parametrize("coef", ["f32", "bf16", "bf16-u"])
 @pytest.mark.parametrize("P", [1, 37, 64, 100, 300])
-def test_protected_rows_parity(P, coef):
+def test_protected_rows_parity(P, coef, monkeypatch):
+    """bf16-u: the query-side RoPE kernel, whose position table has a second
+    part for the protected positions and whose folded rows sit at P + j."""
     import online_rank_kv_b200 as ik
+    if coef == "bf16-u":
+        monkeypatch.setenv("ISKV_DECODE_KERNEL", "u")
     cdt = ik.F32 if coef == "f32" else ik.BF16
     tol = TOL_F32 if coef == "f32" else TOL_BF16
     p = Pair(_cfg(protect=P, coef_dtype=cdt), "qwen3", seed=200 + P)
@@ -53,11 +57,13 @@ def test_protected_rows_parity(P, coef):
     assert p.cache.status() == 0
 
 
-@pytest.mark.parametrize("coef", ["f32", "bf16"])
-def test_decode_while_only_protected_rows(coef):
+@pytest.mark.parametrize("coef", ["f32", "bf16", "bf16-u"])
+def test_decode_while_only_protected_rows(coef, monkeypatch):
     """T below P: every row is a protected row (no window, nothing folded),
     then the stream crosses P and the first blocks fold."""
     import online_rank_kv_b200 as ik
+    if coef == "bf16-u":
+        monkeypatch.setenv("ISKV_DECODE_KERNEL", "u")
     cdt = ik.F32 if coef == "f32" else ik.BF16
     tol = TOL_F32 if coef == "f32" else TOL_BF16
     P = 300

@@ -78,13 +78,15 @@ def _cfg(**kw):
     return c
 
 
-@pytest.mark.parametrize("tensor_cores", ["1", "0"])
+@pytest.mark.parametrize("tensor_cores", ["1", "0", "u"])
 def test_coded_cache_tracks_the_coded_oracle_through_many_rewrites(tensor_cores, monkeypatch):
-    """Decode through the tensor-core kernel (the layer's codes expanded to
-    bf16 tiles per call) and through the CUDA-core kernel (codes read in
-    place)."""
+    """Decode through the tensor-core kernels (the layer's codes expanded to
+    bf16 tiles per call; "u" forces the query-side RoPE kernel) and through the
+    CUDA-core kernel (codes read in place)."""
     import online_rank_kv_b200 as ik
-    monkeypatch.setenv("ISKV_TENSOR_CORES", tensor_cores)
+    monkeypatch.setenv("ISKV_TENSOR_CORES", "0" if tensor_cores == "0" else "1")
+    if tensor_cores == "u":
+        monkeypatch.setenv("ISKV_DECODE_KERNEL", "u")
     cfg = _cfg()
     cache = ik.Cache(cfg)
     H = cfg.batch * cfg.kv_heads
