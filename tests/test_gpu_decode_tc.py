@@ -79,11 +79,12 @@ def test_tc_decode_matches_oracle_and_cuda_core(rk, rv, g, W, T, kernel):
     assert pt.cache.status() == 0
 
 
-def test_tc_decode_ctas_span_heads():
+@pytest.mark.parametrize("kernel", ["rot", "u"])
+def test_tc_decode_ctas_span_heads(kernel):
     """64 (sequence, KV head) pairs with 3 tiles each: 192 tiles on 148 SMs,
     so most CTAs cover parts of two heads."""
     cfg = _cfg(batch=8, kv_heads=8, q_heads=32, window=128, max_tokens=1024)
-    p = _pair(True, cfg, seed=41)
+    p = _pair(True, cfg, seed=41, kernel=kernel)
     p.prefill(128 + 3 * 128 - 64 + 17, chunk=64)
     T, n_c = p.cache.counts(0)
     assert n_c == 320                       # 2.5 tiles: last tile half full
@@ -92,11 +93,12 @@ def test_tc_decode_ctas_span_heads():
     assert p.cache.status() == 0
 
 
-def test_tc_decode_recall_query():
+@pytest.mark.parametrize("kernel", ["rot", "u"])
+def test_tc_decode_recall_query(kernel):
     """A query aimed at one folded token (its score ~25 above the rest):
     the sharpest attention the decode has to reproduce."""
     cfg = _cfg(kv_heads=2, q_heads=8, window=256)
-    p = _pair(True, cfg, seed=43)
+    p = _pair(True, cfg, seed=43, kernel=kernel)
     p.prefill(2048)
     q = p.query().double()
     pos = 333
@@ -112,11 +114,12 @@ def test_tc_decode_recall_query():
     assert max(errs.values()) < TOL_BF16, errs
 
 
-def test_tc_decode_without_folded_rows():
+@pytest.mark.parametrize("kernel", ["rot", "u"])
+def test_tc_decode_without_folded_rows(kernel):
     """Nothing folded yet (T < W + 64): only exact-row tiles, including a
     ragged last tile, go through the tensor-core kernel."""
     cfg = _cfg(window=512, max_tokens=1024)
-    pt = _pair(True, cfg, seed=47)
+    pt = _pair(True, cfg, seed=47, kernel=kernel)
     pc = _pair(False, cfg, seed=47)
     pt.prefill(300, chunk=100)
     pc.prefill(300, chunk=100)
