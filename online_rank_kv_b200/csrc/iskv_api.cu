@@ -849,10 +849,12 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.ptab = h->ptab;
         t.ptab_rows = h->ptab_rows;
         t.aq = h->aq;
-        // exact-row tiles of 64 rows, or of 32 when 64 rows of K and V would make
-        // a stage larger than a folded tile's C_K and C_V
+        // exact-row tiles of 64 rows while the pipeline keeps >= 4 stages, else of
+        // 32 (a same-box A/B at r_K 32, r_V 64: 64-row tiles and five stages
+        // 142 us against 32-row tiles and six stages 151 us: half as many exact
+        // tiles, each a full pass of the epilogue's per-tile chain)
         const int64_t coef_tile = (int64_t)128 * (c.rank_k + c.rank_v) * 2;
-        t.win_rows = 2 * 64 * kHeadDim * 2 > coef_tile ? 32 : 64;
+        t.win_rows = decode_tc_smem_bytes(c.rank_k, c.rank_v, 4, 1, 1, 64) <= 227 * 1024 ? 64 : 32;
         // query-side RoPE kernel where U (r_K g columns) fits one TMEM buffer
         const bool use_u = path == ISKV_DECODE_QUERY_ROPE;
         // deepest pipeline that fits: stages first, then two basis buffers, then
