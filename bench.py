@@ -82,8 +82,8 @@ BLOCK = 64
 # workload (the 36-layer run issues the same launch once per layer).  Not measured by this
 # run: reported as copied, with its source, and only while the decode kernel
 # is the one that was captured (None otherwise, and for other workloads).
-DECODE_TRAFFIC = {("qwen3-36L-b8-32k", "decode_tc_kernel"): 434.6e6,
-                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 434.6e6,
+DECODE_TRAFFIC = {("qwen3-36L-b8-32k", "decode_tc_kernel"): 434.3e6,
+                  ("qwen3-1L-b8-32k", "decode_tc_kernel"): 434.3e6,
                   ("qwen3-1L-b32-64k-r32", "decode_u_kernel"): 2338.4e6}
 DECODE_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one decode launch "
                          "at this per-layer shape (full ncu capture of the decode kernel on the "
