@@ -849,16 +849,9 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         t.ptab = h->ptab;
         t.ptab_rows = h->ptab_rows;
         t.aq = h->aq;
-        // exact-row tiles of 64 rows while the pipeline keeps >= 4 stages, else of
-        // 32 (a same-box A/B at r_K 32, r_V 64: 64-row tiles and five stages
-        // 142 us against 32-row tiles and six stages 151 us: half as many exact
-        // tiles, each a full pass of the epilogue's per-tile chain)
         const int64_t coef_tile = (int64_t)128 * (c.rank_k + c.rank_v) * 2;
-        t.win_rows = decode_tc_smem_bytes(c.rank_k, c.rank_v, 4, 1, 1, 64) <= 227 * 1024 ? 64 : 32;
         // query-side RoPE kernel where U (r_K g columns) fits one TMEM buffer
         const bool use_u = path == ISKV_DECODE_QUERY_ROPE;
-        // deepest pipeline that fits: stages first, then two basis buffers, then
-        // double-buffered q'
         t.stages = 0;
         if (use_u) {
             // exact tiles also stage their rows' fp16 RoPE table: 3 x wt rows of 256 bytes
@@ -867,16 +860,35 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
                 if (decode_u_smem_bytes(c.rank_k, c.rank_v, ns, t.win_rows) <= 227 * 1024) t.stages = ns;
             t.basis_bufs = 1;
             t.q_bufs = 1;
+        } else {
+            // deepest pipeline that fits for exact-row tiles of wt rows: stages
+            // first, then two basis buffers, then double-buffered q'
+            struct Fit { int ns = 0, nbk = 0, nqb = 0; };
+            auto fit = [&](int wt) {
+                Fit f;
+                for (int ns = 6; ns >= 2 && f.ns == 0; --ns)
+                    for (int nbk = 2; nbk >= 1 && f.ns == 0; --nbk)
+                        for (int nqb = 2; nqb >= 1; --nqb)
+                            if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk, nqb, wt) <= 227 * 1024) {
+                                f = Fit{ns, nbk, nqb};
+                                break;
+                            }
+                return f;
+            };
+            // exact-row tiles of 64 rows unless that costs a basis or q' buffer, or
+            // more than the stages down to four, against 32-row tiles (a same-box
+            // A/B at r_K 32, r_V 64: 64-row tiles and five stages 142 us against
+            // 32-row tiles and six stages 151 us: half as many exact tiles, each a
+            // full pass of the epilogue's per-tile chain)
+            const Fit f64 = fit(64), f32 = fit(32);
+            const bool wide = f64.ns > 0 && f64.nbk == f32.nbk && f64.nqb == f32.nqb &&
+                              f64.ns >= std::min(f32.ns, 4);
+            const Fit f = wide ? f64 : f32;
+            t.win_rows = wide ? 64 : 32;
+            t.stages = f.ns;
+            t.basis_bufs = f.nbk;
+            t.q_bufs = f.nqb;
         }
-        for (int ns = 6; ns >= 2 && t.stages == 0; --ns)
-            for (int nbk = 2; nbk >= 1 && t.stages == 0; --nbk)
-                for (int nqb = 2; nqb >= 1; --nqb)
-                    if (decode_tc_smem_bytes(c.rank_k, c.rank_v, ns, nbk, nqb, t.win_rows) <= 227 * 1024) {
-                        t.stages = ns;
-                        t.basis_bufs = nbk;
-                        t.q_bufs = nqb;
-                        break;
-                    }
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
         const int wt = t.win_rows;
         const int64_t P = c.protect, Pe = std::min<int64_t>(a.T, P);
