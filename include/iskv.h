@@ -25,9 +25,16 @@
  *    one cache must be ordered on one stream (or ordered by the caller).
  *  - Caller buffers (k, v, q, out, ...): contiguous, row-major, owned by the
  *    caller and borrowed only for the stream-ordered duration of the call.
- *    They may be device memory or host memory (pinned or pageable); host
- *    buffers are detected with cudaPointerGetAttributes and staged through the
- *    cache's own device buffers with cudaMemcpyAsync on `stream`.
+ *    They may be memory of the current device, host memory (pinned or
+ *    pageable) or another GPU's memory; the kind is detected with
+ *    cudaPointerGetAttributes.  In iskv_append and iskv_decode_attention,
+ *    page-locked host buffers on a 16-byte boundary are read and written in
+ *    place over PCIe by the library's kernels (k, v by the append kernel; q
+ *    and out through the cache's staging buffers by a copy kernel); every
+ *    other non-device buffer, and a device k, v or q off the 16-byte boundary,
+ *    is staged through the cache's own device buffers with cudaMemcpyAsync on
+ *    `stream`.  Either way the call does not wait: a host buffer must stay
+ *    valid, and an output unread, until `stream` has passed the call.
  *  - Counters: T (tokens appended) and n_c (tokens folded, a multiple of 64)
  *    are kept per layer on the host and are shared by the whole batch; they
  *    advance when a call is enqueued, so they are exact integers at all times.

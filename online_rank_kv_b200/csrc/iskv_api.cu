@@ -142,14 +142,38 @@ bool quant_fill(const iskv_quant_format& q, int r, FactorView* f) {
     return true;
 }
 
-bool is_device_ptr(const void* p) {
+// The address at which this device's kernels may dereference caller buffer
+// p: p itself for memory of the current device or managed memory, the mapped
+// address for page-locked host memory (*mapped = true), nullptr for pageable
+// host memory and for another GPU's memory (both staged with cudaMemcpyAsync,
+// which also copies between peers).
+const void* kernel_addr(const void* p, bool* mapped = nullptr) {
+    if (mapped) *mapped = false;
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
         cudaGetLastError();
-        return false;
+        return nullptr;
     }
-    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+    if (at.type == cudaMemoryTypeManaged) return p;
+    if (at.type == cudaMemoryTypeDevice) {
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess || at.device != dev) return nullptr;
+        return p;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
+        if (mapped) *mapped = true;
+        return at.devicePointer;
+    }
+    return nullptr;
 }
+
+// memory of the current device (or managed): read and written by kernels as is
+bool is_device_ptr(const void* p) {
+    bool mapped;
+    return kernel_addr(p, &mapped) != nullptr && !mapped;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 int validate(const iskv_config* c) {
     if (!c) return ISKV_ERR_INVALID_ARG;
@@ -625,8 +649,11 @@ int iskv_append(iskv_t h, int layer, const void* k, const void* v, int t, void* 
             return ISKV_OK;
         };
         for (int w = 0; w < 2; ++w) {
-            if (is_device_ptr(srcs[w])) {
-                const int rc = place(w, srcs[w], t, t, 0, h->T[layer]);
+            // device memory and mapped page-locked host memory are read in place
+            // by the append kernel (16-byte vectors); everything else is staged
+            const void* src = kernel_addr(srcs[w]);
+            if (src != nullptr && aligned16(src)) {
+                const int rc = place(w, src, t, t, 0, h->T[layer]);
                 if (rc != ISKV_OK) return rc;
             } else {
                 // stage token chunks of every (sequence, head) through device memory
@@ -783,15 +810,26 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     const size_t o_bytes = (size_t)c.batch * c.q_heads * kHeadDim * sizeof(float);
     const void* qd = q;
     // host queries, or device queries off the 16-byte alignment of the bulk
-    // copies that fetch them, go through the staging buffer
-    if (!is_device_ptr(q) || (reinterpret_cast<uintptr_t>(q) & 15) != 0) {
+    // copies that fetch them, go through the staging buffer: by a copy kernel
+    // from mapped page-locked memory, else by cudaMemcpyAsync
+    bool q_mapped = false;
+    const void* qk = kernel_addr(q, &q_mapped);
+    if (qk == nullptr || q_mapped || !aligned16(qk)) {
         if (q_bytes > h->stage_in_bytes) return ISKV_ERR_UNSUPPORTED;
-        CU(cudaMemcpyAsync(h->stage_in, q, q_bytes, cudaMemcpyDefault, s));
+        if (q_mapped && aligned16(qk)) CU(launch_copy_vec(h->stage_in, qk, q_bytes, s));
+        else CU(cudaMemcpyAsync(h->stage_in, q, q_bytes, cudaMemcpyDefault, s));
         qd = h->stage_in;
     }
-    const bool host_out = !is_device_ptr(out);
+    bool out_mapped = false;
+    void* ok = const_cast<void*>(kernel_addr(out, &out_mapped));
+    const bool host_out = ok == nullptr || out_mapped;
     if (host_out && o_bytes > h->stage_out_bytes) return ISKV_ERR_UNSUPPORTED;
     float* od = host_out ? h->stage_out : out;
+    // the result leaves the staging buffer the same two ways
+    auto copy_out = [&]() -> cudaError_t {
+        if (out_mapped && aligned16(ok)) return launch_copy_vec(ok, od, o_bytes, s);
+        return cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s);
+    };
 
     DecodeArgs a{};
     a.K = view(h, ISKV_WHICH_K);
@@ -913,7 +951,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         if (t.stages == 0) return ISKV_ERR_UNSUPPORTED;
         if (use_u) CU(launch_decode_u(t, s));   // both merge the partials of each head
         else CU(launch_decode_tc(t, s));
-        if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
+        if (host_out) CU(copy_out());
         return ISKV_OK;
     }
     // split the token axis so that the grid covers the GPU several times
@@ -930,7 +968,7 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
     a.splits = (int)splits;
     CU(launch_decode(a, s));
     CU(launch_combine(a, od, s));
-    if (host_out) CU(cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s));
+    if (host_out) CU(copy_out());
     return ISKV_OK;
 }
 

@@ -1,5 +1,6 @@
 // Small kernels of the cache: factor initialization, appending exact rows to
-// the window ring, and rebuilding folded rows (C B^T, before RoPE).
+// the window ring, rebuilding folded rows (C B^T, before RoPE), and moving a
+// call's operands to and from page-locked host memory.
 #include "iskv_internal.cuh"
 
 namespace iskv {
@@ -101,7 +102,29 @@ __global__ void copy_coef_kernel(FactorView f, int layer, int64_t row0, int64_t 
     }
 }
 
+// dst[i] = src[i] over n 16-byte vectors.  Either side may be page-locked
+// host memory mapped into the device's address space: its loads or stores
+// then cross PCIe in place, with no copy-engine hand-off between the kernels
+// of a call on the same stream.
+__global__ void copy_vec_kernel(uint4* dst, const uint4* src, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = src[i];
+}
+
 }  // namespace
+
+cudaError_t launch_copy_vec(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+    if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | bytes) & 15) != 0)
+        return cudaErrorInvalidValue;
+    const int64_t n = (int64_t)(bytes / 16);
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 592) blocks = 592;
+    copy_vec_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(dst),
+                                                     reinterpret_cast<const uint4*>(src), n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_copy_coef(const FactorView& f, int layer, int64_t row0, int64_t rows, void* dst,
                              cudaStream_t s) {

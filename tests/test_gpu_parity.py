@@ -268,6 +268,66 @@ def test_decode_before_any_fold_and_host_buffers():
     assert max(errs.values()) < TOL_F32
 
 
+def _offset_view(x: torch.Tensor, elems: int, device=None, pinned=False) -> torch.Tensor:
+    """A contiguous copy of x that starts `elems` elements into a fresh buffer
+    (an odd offset puts it off the 16-byte alignment)."""
+    buf = torch.zeros(x.numel() + 16, dtype=x.dtype, device=device)
+    if pinned:
+        buf = buf.pin_memory()
+    view = buf[elems:elems + x.numel()].view(x.shape)
+    view.copy_(x)
+    return view
+
+
+BUFFER_KINDS = {
+    "pageable": lambda x: x.clone(),
+    "pinned": lambda x: x.pin_memory(),
+    "pinned, unaligned": lambda x: _offset_view(x, 1, pinned=True),
+    "device, unaligned": lambda x: _offset_view(x, 1, device="cuda"),
+}
+
+
+@pytest.mark.parametrize("coef", ["f32", "bf16"])
+def test_caller_buffers_of_every_kind(coef):
+    """Page-locked host buffers are read and written in place by the library's
+    kernels; pageable ones, another alignment than 16 bytes (host or device)
+    and device buffers the bulk copies cannot take are staged.  Rows appended
+    from every kind reach the oracle's factors, and the decode writes the same
+    output bits into every kind of buffer from every kind of query buffer."""
+    ik = _ik()
+    cfg = qwen_cfg(kv_heads=2, q_heads=8, window=256, max_tokens=2048,
+                   coef_dtype=ik.F32 if coef == "f32" else ik.BF16)
+    tol = TOL_F32 if coef == "f32" else TOL_BF16
+    p = Pair(cfg, "qwen3", seed=11)
+    p.prefill(600, chunk=100)
+    g = torch.Generator().manual_seed(3)
+    for kind, make in BUFFER_KINDS.items():
+        for t in (1, 37):
+            k = torch.randn(cfg.batch, cfg.kv_heads, t, cfg.head_dim, generator=g).to(torch.bfloat16)
+            v = torch.randn(cfg.batch, cfg.kv_heads, t, cfg.head_dim, generator=g).to(torch.bfloat16)
+            kx, vx = make(k), make(v)
+            p.cache.append(0, kx, vx)
+            torch.cuda.synchronize()        # the sources outlive the enqueued reads
+            for (l, b, h) in p.heads:
+                p.ok[(l, b, h)].append(k[b, h].double().numpy())
+                p.ov[(l, b, h)].append(v[b, h].double().numpy())
+            p.fold_ready()
+    p.check_counts()
+    assert p.cache.counts(0)[1] > 0
+    q = p.query()
+    errs, out_dev = p.decode(0, q)
+    assert max(errs.values()) < tol, errs
+    out_kinds = dict(BUFFER_KINDS, device=lambda x: x.cuda())
+    for qkind, make_q in BUFFER_KINDS.items():
+        for okind, make_o in out_kinds.items():
+            qx = make_q(q)
+            ox = make_o(torch.full(tuple(q.shape), float("nan"), dtype=torch.float32))
+            p.cache.decode_attention(0, qx, out=ox)
+            torch.cuda.synchronize()
+            assert np.array_equal(ox.cpu().numpy(), out_dev), (qkind, okind)
+    assert p.cache.status() == 0
+
+
 def test_error_codes():
     ik = _ik()
     cfg = qwen_cfg(kv_heads=1, q_heads=4, window=128, max_tokens=1024)   # ring: 128 + 128 rows
