@@ -28,13 +28,14 @@
  *    They may be memory of the current device, host memory (pinned or
  *    pageable) or another GPU's memory; the kind is detected with
  *    cudaPointerGetAttributes.  In iskv_append and iskv_decode_attention,
- *    page-locked host buffers on a 16-byte boundary are read and written in
- *    place over PCIe by the library's kernels (k, v by the append kernel; q
- *    and out through the cache's staging buffers by a copy kernel); every
- *    other non-device buffer, and a device k, v or q off the 16-byte boundary,
- *    is staged through the cache's own device buffers with cudaMemcpyAsync on
- *    `stream`.  Either way the call does not wait: a host buffer must stay
- *    valid, and an output unread, until `stream` has passed the call.
+ *    page-locked host buffers are read and written in place over PCIe by the
+ *    library's kernels: k, v (16-byte aligned) by the append kernel, q
+ *    (16-byte aligned) by a copy kernel into the cache's staging buffer, out
+ *    (4-byte aligned) by the decode's own stores.  Every other non-device
+ *    buffer, and device buffers off those boundaries, are staged through the
+ *    cache's own device buffers with cudaMemcpyAsync on `stream`.  Either way
+ *    the call does not wait: a host buffer must stay valid, and an output
+ *    unread, until `stream` has passed the call.
  *  - Counters: T (tokens appended) and n_c (tokens folded, a multiple of 64)
  *    are kept per layer on the host and are shared by the whole batch; they
  *    advance when a call is enqueued, so they are exact integers at all times.

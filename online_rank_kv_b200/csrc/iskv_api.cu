@@ -820,16 +820,14 @@ int iskv_decode_attention(iskv_t h, int layer, const void* q, float* out, void* 
         else CU(cudaMemcpyAsync(h->stage_in, q, q_bytes, cudaMemcpyDefault, s));
         qd = h->stage_in;
     }
-    bool out_mapped = false;
-    void* ok = const_cast<void*>(kernel_addr(out, &out_mapped));
-    const bool host_out = ok == nullptr || out_mapped;
+    // device memory and mapped page-locked memory take the kernels' 4-byte
+    // stores of the result in place; anything else gets it through the
+    // staging buffer and cudaMemcpyAsync
+    void* ok = const_cast<void*>(kernel_addr(out));
+    const bool host_out = ok == nullptr || (reinterpret_cast<uintptr_t>(ok) & 3) != 0;
     if (host_out && o_bytes > h->stage_out_bytes) return ISKV_ERR_UNSUPPORTED;
-    float* od = host_out ? h->stage_out : out;
-    // the result leaves the staging buffer the same two ways
-    auto copy_out = [&]() -> cudaError_t {
-        if (out_mapped && aligned16(ok)) return launch_copy_vec(ok, od, o_bytes, s);
-        return cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s);
-    };
+    float* od = host_out ? h->stage_out : static_cast<float*>(ok);
+    auto copy_out = [&]() { return cudaMemcpyAsync(out, od, o_bytes, cudaMemcpyDefault, s); };
 
     DecodeArgs a{};
     a.K = view(h, ISKV_WHICH_K);

@@ -275,7 +275,8 @@ cudaError_t launch_init_factor(const FactorView& f, int layers, cudaStream_t s);
 cudaError_t launch_append(void* ring, const void* src, int BH, int t, int src_t, int src_row0,
                           int64_t T0, int64_t cap, int elem_bytes, int blocked, cudaStream_t s);
 // bytes from src to dst by a kernel (both 16-byte aligned, bytes a multiple
-// of 16, else cudaErrorInvalidValue); either may be mapped page-locked host memory
+// of 16, else cudaErrorInvalidValue); either may be mapped page-locked host
+// memory (the decode call's host queries)
 cudaError_t launch_copy_vec(void* dst, const void* src, size_t bytes, cudaStream_t s);
 cudaError_t launch_fold(const FactorView& f, const FoldLaunch& fl, int* status,
                         cudaStream_t s);
