@@ -104,6 +104,30 @@ def test_null_handles():
     assert ik.LIB.iskv_compress_block(None, 0, 0, None) == -1
 
 
+def test_every_handle_call_refuses_a_null_handle_on_the_host():
+    """Each entry point that takes a cache returns INVALID_ARG for a NULL
+    handle (or NULL operands) before any CUDA call, so these run without a GPU."""
+    ik = _lib()
+    L = ik.LIB
+    n = ctypes.c_int(7)
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    calls = {
+        "iskv_append": lambda: L.iskv_append(None, 0, None, None, 1, None, ctypes.byref(n)),
+        "iskv_compress_block_async": lambda: L.iskv_compress_block_async(None, 0, 0, None, None),
+        "iskv_sync": lambda: L.iskv_sync(None, 0, None),
+        "iskv_decode_attention": lambda: L.iskv_decode_attention(None, 0, None, None, None),
+        "iskv_decode_kernel": lambda: L.iskv_decode_kernel(None, 0, ctypes.byref(n)),
+        "iskv_reconstruct": lambda: L.iskv_reconstruct(None, 0, 0, None, None),
+        "iskv_get_factors": lambda: L.iskv_get_factors(None, 0, 0, None, None, None, None),
+        "iskv_kv_bytes": lambda: L.iskv_kv_bytes(None, ctypes.byref(a), ctypes.byref(b)),
+        "iskv_decode_attention_noalloc": lambda: L.iskv_decode_attention_noalloc(None, None, None, None),
+        "iskv_quantize_rows": lambda: L.iskv_quantize_rows(None, 32, None, 0, None, None, None),
+    }
+    for name, call in calls.items():
+        assert call() == -1, name
+    assert n.value == 7                       # outputs untouched on refusal
+
+
 def test_binding_structs_match_the_header_layout(tmp_path):
     """The ctypes mirrors of iskv_config and iskv_decode_operands have the C
     structs' size and field offsets (compiled here with the host compiler)."""
