@@ -8,7 +8,8 @@ shows up here as well as there:
 * the per-tile query pre-rotation: q . R_j k = (R_t^T q) . R_(j-t) k;
 * split-K softmax with a lazily kept running maximum, merged by log-sum-exp;
 * the three-part bf16 split of an fp32 matrix (exact) and the hi + lo
-  splits of the basis (bf16) and the queries (fp16).
+  splits of the basis (bf16) and the queries (fp16);
+* the CUDA-core decode's RoPE by stepped fp32 rotations, R(j) R(4t) R(1)^u.
 """
 
 import numpy as np
@@ -136,3 +137,38 @@ def test_hi_lo_splits_of_basis_and_queries():
     err = np.abs(qh + ql - q)
     assert np.all(err <= np.maximum(2.0 ** -22 * np.abs(q), 2.0 ** -25))
     assert np.max(np.abs(qh - q) / np.abs(q)) > 2.0 ** -13       # one fp16 part alone is coarse
+
+
+def _cmul32(a, b):
+    """(a.x + i a.y)(b.x + i b.y) with every product and sum rounded to fp32."""
+    f = np.float32
+    ax, ay, bx, by = (np.asarray(v, dtype=f) for v in (a[0], a[1], b[0], b[1]))
+    return (f(ax * bx) - f(ay * by)).astype(f), (f(ax * by) + f(ay * bx)).astype(f)
+
+
+def test_stepped_fp32_rope_stays_within_a_few_ulps():
+    """The CUDA-core decode turns row j + 4t + u of a 64-row tile starting at
+    j by R(j) R(4t) R(1)^u: the tile's base rotation and the steps R(4t),
+    R(1) are fp32 roundings of float64 tables, the products fp32.  Four
+    complex products keep cos and sin within 1.5e-6 of the float64 values at
+    any position up to 2^18, far inside the 1e-4 parity bar of fp32
+    coefficients (fp32 angles at such positions would be off by ~1e-2 rad)."""
+    rng = np.random.default_rng(5)
+    w = O.rope_inv_freq(D, THETA)
+    tab = lambda pos: (np.cos(pos * w).astype(np.float32), np.sin(pos * w).astype(np.float32))
+    worst = 0.0
+    for j in list(rng.integers(0, 2 ** 18 // 64, 40) * 64) + [2 ** 18 - 64]:
+        rj = tab(j)
+        r1 = tab(1)
+        for t in range(16):
+            rb = _cmul32(rj, tab(4 * t))
+            for u in range(4):
+                pos = j + 4 * t + u
+                worst = max(worst, np.max(np.abs(rb[0] - np.cos(pos * w))),
+                            np.max(np.abs(rb[1] - np.sin(pos * w))))
+                rb = _cmul32(rb, r1)
+    assert worst < 1.5e-6, worst
+    # the shortcut the table avoids: the angle formed in fp32
+    pos = np.float32(2 ** 18 - 1)
+    ang32 = (pos * w.astype(np.float32)).astype(np.float32)
+    assert np.max(np.abs(np.cos(ang32.astype(np.float64)) - np.cos(float(pos) * w))) > 1e-3
