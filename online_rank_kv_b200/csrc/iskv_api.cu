@@ -441,9 +441,9 @@ int iskv_create(const iskv_config* cfg, void* stream, iskv_t* out) {
         const char* env = std::getenv("ISKV_TENSOR_CORES");
         h->use_tc = kDecodeTcDefault ? !(env && env[0] == '0') : (env && env[0] == '1');
         cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
-        // decode kernel for bf16 coefficient tiles: "rot" keeps the kernel that
-        // rebuilds and rotates the keys, otherwise the query-side RoPE kernel
-        // wherever r_K g <= 128
+        // decode kernel for bf16 coefficient tiles: "rot" always the kernel that
+        // rebuilds and rotates the keys, "u" the query-side RoPE kernel wherever
+        // r_K g <= 128, unset a choice per call (decode_path)
         const char* dk = std::getenv("ISKV_DECODE_KERNEL");
         h->use_u = dk && std::strcmp(dk, "u") == 0 ? 1 : dk && std::strcmp(dk, "rot") == 0 ? 0 : 2;
         const char* w = std::getenv("ISKV_TEST_PIPELINE_WAIT_CYCLES");
